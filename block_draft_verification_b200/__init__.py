@@ -1,0 +1,225 @@
+"""Python binding of libdflash2.so, the C ABI of the DFlash 2 draft -> select
+-> verify step on B200 (declared in include/dflash2.h).
+
+Argument marshalling only: every function takes CUDA torch tensors, allocates
+the outputs with torch, and passes raw device pointers and the current CUDA
+stream to the library, where all of the work runs.  There is no other code
+path: if the library is not built, or a call fails, an exception is raised.
+"""
+import ctypes as C
+import os
+
+import torch
+
+__all__ = ["F32", "BF16", "Q_SOFTMAX", "Q_ONEHOT", "K", "DFlash2Error", "lib", "workspace_bytes",
+           "Workspace", "topk_softmax", "pair_select", "verify_greedy", "verify_sample",
+           "dynconv2", "status_string", "version"]
+
+F32, BF16 = 0, 1
+Q_SOFTMAX, Q_ONEHOT = 0, 1
+K = 16
+MAX_BLOCK = 32
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdflash2.so")
+_lib = None
+
+
+class DFlash2Error(RuntimeError):
+    def __init__(self, where, status):
+        super().__init__("%s: %s" % (where, status_string(status) if _lib else status))
+        self.status = status
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libdflash2.so is not built (python -m block_draft_verification_b200.build)")
+        L = C.CDLL(LIB_PATH)
+        vp, i32, i64, u32, u64, f32, sz = (C.c_void_p, C.c_int, C.c_int64, C.c_uint32, C.c_uint64,
+                                           C.c_float, C.c_size_t)
+        L.dflash2_status_string.argtypes = [i32]
+        L.dflash2_status_string.restype = C.c_char_p
+        L.dflash2_version.restype = i32
+        L.dflash2_workspace_bytes.argtypes = [i32, i32, i64]
+        L.dflash2_workspace_bytes.restype = sz
+        L.dflash2_topk_softmax.argtypes = [vp, i32, i64, i64, i64, f32, vp, vp, vp, vp, vp, sz, vp]
+        L.dflash2_pair_select.argtypes = [vp, vp, vp, vp, i32, i64, i32, vp, i32, i32, vp, vp, vp,
+                                          vp, sz, vp]
+        L.dflash2_verify_greedy.argtypes = [vp, i32, i32, i32, i64, vp, vp, vp, vp, sz, vp]
+        L.dflash2_verify_sample.argtypes = [vp, vp, i32, i32, i32, i64, vp, f32, u64, u32, vp, i32,
+                                            vp, vp, vp, vp, vp, sz, vp]
+        L.dflash2_dynconv2.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp]
+        for f in ("dflash2_topk_softmax", "dflash2_pair_select", "dflash2_verify_greedy",
+                  "dflash2_verify_sample", "dflash2_dynconv2"):
+            getattr(L, f).restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().dflash2_status_string(int(status)).decode()
+
+
+def version():
+    v = lib().dflash2_version()
+    return (v >> 16, v & 0xFFFF)
+
+
+def workspace_bytes(B, G, V):
+    return int(lib().dflash2_workspace_bytes(int(B), int(G), int(V)))
+
+
+def _check(where, rc):
+    if rc != 0:
+        raise DFlash2Error(where, rc)
+
+
+def _dtype(t):
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError("expected float32 or bfloat16, got %s" % t.dtype)
+
+
+def _p(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(dev):
+    return C.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("dflash2 calls take CUDA tensors")
+
+
+class Workspace:
+    """A device scratch buffer for the calls that take one.  Calls on one
+    stream run in order, so one Workspace serves every call on that stream."""
+
+    def __init__(self, device=None, nbytes=0):
+        self.device = torch.device(device if device is not None else "cuda")
+        self.buf = torch.empty(0, dtype=torch.uint8, device=self.device)
+        self.reserve(nbytes)
+
+    def reserve(self, nbytes):
+        if nbytes > self.buf.numel():
+            self.buf = torch.empty(int(nbytes), dtype=torch.uint8, device=self.device)
+        return self
+
+    def args(self, B, G, V):
+        self.reserve(workspace_bytes(B, G, V))
+        return C.c_void_p(self.buf.data_ptr()), C.c_size_t(self.buf.numel())
+
+
+_ws_cache = {}
+
+
+def _ws(ws, dev, B, G, V):
+    if ws is None:
+        ws = _ws_cache.setdefault((dev.index, torch.cuda.current_stream(dev).cuda_stream),
+                                  Workspace(dev))
+    return ws.args(B, G, V)
+
+
+def topk_softmax(logits, inv_temperature=1.0, out=None, ws=None):
+    """logits [..., V] (rows may be strided) -> idx [..., 16] int32, prob, logp
+    [..., 16] float32, logz [...] float32."""
+    _cuda(logits)
+    V = logits.shape[-1]
+    x = logits.reshape(-1, V) if logits.dim() != 2 else logits
+    if x.stride(-1) != 1:
+        x = x.contiguous()
+    rows = x.shape[0]
+    lead = logits.shape[:-1]
+    dev = logits.device
+    if out is None:
+        out = (torch.empty(lead + (K,), dtype=torch.int32, device=dev),
+               torch.empty(lead + (K,), dtype=torch.float32, device=dev),
+               torch.empty(lead + (K,), dtype=torch.float32, device=dev),
+               torch.empty(lead, dtype=torch.float32, device=dev))
+    idx, prob, logp, logz = out
+    wp, wb = _ws(ws, dev, rows, 1, V)
+    _check("dflash2_topk_softmax", lib().dflash2_topk_softmax(
+        _p(x), _dtype(x), rows, V, x.stride(0) if rows > 1 else V, float(inv_temperature),
+        _p(idx), _p(prob), _p(logp), _p(logz), wp, wb, _stream(dev)))
+    return idx, prob, logp, logz
+
+
+def pair_select(idx, logp, anchor, emb, W, out=None, ws=None):
+    """idx, logp [B, G, 16], anchor [B] int32 or None, emb [V, d], W [d, d] float32
+    -> path_tok [B, G] int32, path_rank [B, G] int32, path_score [B] float32."""
+    _cuda(idx, logp, anchor, emb, W)
+    B, G, _ = idx.shape
+    V, d = emb.shape
+    dev = idx.device
+    if out is None:
+        out = (torch.empty((B, G), dtype=torch.int32, device=dev),
+               torch.empty((B, G), dtype=torch.int32, device=dev),
+               torch.empty((B,), dtype=torch.float32, device=dev))
+    tok, rank, score = out
+    wp, wb = _ws(ws, dev, B, G, V)
+    _check("dflash2_pair_select", lib().dflash2_pair_select(
+        _p(idx.contiguous()), _p(logp.contiguous()), _p(anchor), _p(emb.contiguous()), _dtype(emb),
+        V, d, _p(W.contiguous()), B, G, _p(tok), _p(rank), _p(score), wp, wb, _stream(dev)))
+    return tok, rank, score
+
+
+def verify_greedy(target, draft_tok, out=None, ws=None):
+    """target [B, G+1, V], draft_tok [B, G] int32 -> n_accept [B], out_tok [B, G+1] int32."""
+    _cuda(target, draft_tok)
+    B, G1, V = target.shape
+    dev = target.device
+    if out is None:
+        out = (torch.empty((B,), dtype=torch.int32, device=dev),
+               torch.empty((B, G1), dtype=torch.int32, device=dev))
+    n, toks = out
+    wp, wb = _ws(ws, dev, B, G1 - 1, V)
+    _check("dflash2_verify_greedy", lib().dflash2_verify_greedy(
+        _p(target.contiguous()), _dtype(target), B, G1 - 1, V, _p(draft_tok.contiguous()), _p(n),
+        _p(toks), wp, wb, _stream(dev)))
+    return n, toks
+
+
+def verify_sample(target, draft, draft_tok, seed, step, seq_id=None, inv_temperature=1.0,
+                  q_mode=Q_SOFTMAX, debug=False, out=None, ws=None):
+    """target [B, G+1, V], draft [B, G, V] (None in one-hot mode), draft_tok [B, G]
+    -> n_accept [B], out_tok [B, G+1] (+ ratio [B, G], u [B, G] if debug)."""
+    _cuda(target, draft, draft_tok, seq_id)
+    B, G1, V = target.shape
+    G = G1 - 1
+    dev = target.device
+    if out is None:
+        out = (torch.empty((B,), dtype=torch.int32, device=dev),
+               torch.empty((B, G1), dtype=torch.int32, device=dev))
+        if debug:
+            out = out + (torch.empty((B, G), dtype=torch.float32, device=dev),
+                         torch.empty((B, G), dtype=torch.float32, device=dev))
+    n, toks = out[0], out[1]
+    ratio = out[2] if len(out) > 2 else None
+    u = out[3] if len(out) > 3 else None
+    wp, wb = _ws(ws, dev, B, G, V)
+    q = None if draft is None else draft.contiguous()
+    sid = None if seq_id is None else seq_id.to(torch.int32).contiguous()
+    _check("dflash2_verify_sample", lib().dflash2_verify_sample(
+        _p(target.contiguous()), _p(q), _dtype(target), B, G, V, _p(draft_tok.contiguous()),
+        float(inv_temperature), int(seed) & (2 ** 64 - 1), int(step) & 0xFFFFFFFF, _p(sid),
+        int(q_mode), _p(n), _p(toks), _p(ratio), _p(u), wp, wb, _stream(dev)))
+    return out
+
+
+def dynconv2(x, x_prev, w_tap, out=None):
+    """x [B, T, H], x_prev [B, H], w_tap [2H, H] (one dtype) -> out [B, T, H]."""
+    _cuda(x, x_prev, w_tap)
+    B, T, H = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check("dflash2_dynconv2", lib().dflash2_dynconv2(
+        _p(x.contiguous()), _p(x_prev.contiguous()), _p(w_tap.contiguous()), _dtype(x), B, T, H,
+        _p(out), _stream(x.device)))
+    return out

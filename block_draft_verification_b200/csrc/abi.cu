@@ -1,0 +1,31 @@
+// abi.cu -- the entry points of the C ABI that launch nothing: status names,
+// the version, and the workspace size every call can use.
+#include "common.cuh"
+#include "workspace.cuh"
+
+using namespace dfl;
+
+extern "C" const char* dflash2_status_string(int status) {
+    switch (status) {
+        case DFLASH2_OK: return "DFLASH2_OK";
+        case DFLASH2_EINVAL: return "DFLASH2_EINVAL: null pointer or invalid scalar argument";
+        case DFLASH2_EDTYPE: return "DFLASH2_EDTYPE: unsupported dtype";
+        case DFLASH2_ESHAPE: return "DFLASH2_ESHAPE: size outside the supported range";
+        case DFLASH2_EWORKSPACE: return "DFLASH2_EWORKSPACE: workspace missing, misaligned or too small";
+        case DFLASH2_ECUDA: return "DFLASH2_ECUDA: a CUDA launch or memset failed";
+        case DFLASH2_EALIGN: return "DFLASH2_EALIGN: pointer or stride misaligned";
+        default: return "DFLASH2_UNKNOWN_STATUS";
+    }
+}
+
+extern "C" int dflash2_version(void) { return (1 << 16) | 0; }
+
+extern "C" size_t dflash2_workspace_bytes(int B, int G, int64_t V) {
+    if (B < 0 || G < 1 || G >= DFLASH2_MAX_BLOCK || V < 1) return 0;
+    const int64_t rows = (int64_t)B * G;
+    size_t need = topk_layout(rows, V).total;
+    need = need > greedy_layout(B, G, V).total ? need : greedy_layout(B, G, V).total;
+    need = need > sample_layout(B, G, V).total ? need : sample_layout(B, G, V).total;
+    need = need > select_layout(B, G).total ? need : select_layout(B, G).total;
+    return need;
+}

@@ -1,0 +1,75 @@
+// workspace.cuh -- layout of the caller-provided workspace of each call.
+//
+// Every layout puts the arrival counters first (cleared by the call with one
+// cudaMemsetAsync) and the per-unit partial results after them; both regions
+// start on 256-byte boundaries.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace dfl {
+
+// Partial result of one (row, chunk) unit of dflash2_topk_softmax.
+struct TopkPartial {
+    float m;
+    float s;
+    uint32_t pad[2];
+    uint64_t key[K];
+};
+
+// Per-sequence state handed from the verify_sample scan to its draw:
+// p_v = exp2((x_v - mt) * c - l2t) on the target row used, likewise q.
+struct SampleInfo {
+    float mt, l2t;    // target row max and log2 of its sum-exp
+    float mq, l2q;    // draft row (mode 0 only)
+    float u_res;      // u' of the draw
+    int32_t n;        // accepted count = row the draw uses
+    int32_t mode;     // 0 = residual max(0, p - q), 1 = p without d_n, 2 = p
+    int32_t d;        // the rejected drafted token (mode 1)
+};
+
+struct Layout {
+    size_t counters_off, counters_bytes;
+    size_t part_off, part_bytes;
+    size_t part2_off, part2_bytes;
+    size_t info_off, info_bytes;
+    size_t total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+inline Layout make_layout(size_t counters, size_t part, size_t part2 = 0, size_t info = 0) {
+    Layout L;
+    L.counters_off = 0;
+    L.counters_bytes = align256(counters);
+    L.part_off = L.counters_bytes;
+    L.part_bytes = align256(part);
+    L.part2_off = L.part_off + L.part_bytes;
+    L.part2_bytes = align256(part2);
+    L.info_off = L.part2_off + L.part2_bytes;
+    L.info_bytes = align256(info);
+    L.total = L.info_off + L.info_bytes;
+    return L;
+}
+
+inline Layout topk_layout(int64_t rows, int64_t V) {
+    int64_t S = n_chunks(V);
+    return make_layout((size_t)rows * 4, (size_t)(rows * S) * sizeof(TopkPartial));
+}
+inline Layout greedy_layout(int B, int G, int64_t V) {
+    int64_t S = n_chunks(V);
+    return make_layout((size_t)B * 4, (size_t)((int64_t)B * (G + 1) * S) * sizeof(uint64_t));
+}
+inline Layout sample_layout(int B, int G, int64_t V) {
+    int64_t S = n_chunks(V);
+    return make_layout((size_t)B * 2 * 4, (size_t)((int64_t)B * (2 * G + 1) * S) * sizeof(LseD),
+                       (size_t)((int64_t)B * S) * 2 * sizeof(double), (size_t)B * sizeof(SampleInfo));
+}
+inline Layout select_layout(int B, int G) {
+    return make_layout((size_t)B * 4, (size_t)B * (K + (size_t)K * K * (G - 1)) * sizeof(float));
+}
+
+}  // namespace dfl

@@ -1,0 +1,213 @@
+/*
+ * dflash2.h -- C ABI of the DFlash 2 draft -> select -> verify step on B200.
+ *
+ * The library (libdflash2.so) runs the step that follows the drafter and
+ * target forwards of one-pass block-parallel speculative decoding:
+ *
+ *   dflash2_topk_softmax   softmax over the vocabulary and the 16 best
+ *                          candidates of every drafted position
+ *   dflash2_pair_select    bilinear adjacent-pair scores and the exact best
+ *                          path through the 16 candidates per position
+ *   dflash2_verify_greedy  greedy lossless verify (longest prefix match)
+ *   dflash2_verify_sample  sampling lossless verify (rejection sampling with
+ *                          residual resample and bonus draw)
+ *   dflash2_dynconv2       two-tap dynamic depthwise conv fused with its tap
+ *                          projection and the residual add
+ *
+ * Source pages (cited by title and section):
+ *   [tamsi]    "DFlash 2 — 3× plus de tokens sur Qwen3.8-27B, même sortie",
+ *              sections "L’idée, sans le papier" and "Les chiffres qui
+ *              comptent sur Qwen3.8-27B".
+ *   [myaiexp]  "DFlash 2" (myaiexp.com), section "主な機能" (features).
+ *   [latenode] "DFlash 2: un drafter de 3.43× que cae a 1.45× bajo carga",
+ *              sections "Un drafter que adivina el bloque entero de una vez",
+ *              "El desacuerdo empieza en las propias tablas del proveedor".
+ *   [psi]      "Qwen 3.8 27B + DFlash2: 140 Token/Sec?", section "Résumé".
+ *   [philox]   Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3",
+ *              SC'11, section 5.
+ *
+ * Conventions for every call:
+ *   - Tensor arguments are DEVICE pointers owned by the caller; the library
+ *     never frees or keeps them.  Layouts are dense row-major unless a stride
+ *     is given.  bf16 data is passed as its 16-bit storage.
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default
+ *     stream) and never synchronises the host.
+ *   - The return value is a dflash2_status.  Host-side validation happens
+ *     before anything is enqueued: on any status other than DFLASH2_OK no
+ *     work was enqueued, except DFLASH2_ECUDA, which reports a failed launch
+ *     or memset (read with cudaGetLastError, which also clears it).
+ *   - Preconditions the library does not check on the device: logits,
+ *     embeddings and weights are finite; token ids are in [0, V); output
+ *     buffers do not overlap inputs.
+ *   - Calls that take a workspace (`ws`, `ws_bytes`): a device buffer of at
+ *     least dflash2_workspace_bytes(B, G, V) bytes, 256-byte aligned, used
+ *     for per-chunk partial results and arrival counters.  The call clears
+ *     the part it needs at its start, so its contents between calls do not
+ *     matter; two calls that may run concurrently need separate workspaces.
+ *   - Results are deterministic: a sequence's outputs depend only on its own
+ *     inputs (and seq_id), not on the batch it runs in or on B.
+ */
+#ifndef DFLASH2_H
+#define DFLASH2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Every entry point is exported from the shared library; nothing else is. */
+#if defined(__GNUC__)
+#define DFLASH2_API __attribute__((visibility("default")))
+#else
+#define DFLASH2_API
+#endif
+
+/* The driver stream handle; identical to cudaStream_t / CUstream. */
+typedef struct CUstream_st* dflash2_stream_t;
+
+typedef enum {
+    DFLASH2_OK = 0,
+    DFLASH2_EINVAL = 1,     /* null pointer, non-finite or non-positive scalar */
+    DFLASH2_EDTYPE = 2,     /* dtype not DFLASH2_F32 / DFLASH2_BF16 */
+    DFLASH2_ESHAPE = 3,     /* size out of the supported range */
+    DFLASH2_EWORKSPACE = 4, /* ws NULL, misaligned or smaller than required */
+    DFLASH2_ECUDA = 5,      /* a CUDA launch or memset failed */
+    DFLASH2_EALIGN = 6      /* a pointer or stride violates the stated alignment */
+} dflash2_status;
+
+typedef enum { DFLASH2_F32 = 0, DFLASH2_BF16 = 1 } dflash2_dtype;
+typedef enum { DFLASH2_Q_SOFTMAX = 0, DFLASH2_Q_ONEHOT = 1 } dflash2_qmode;
+
+/* Candidates kept per drafted position ([tamsi] "L’idée, sans le papier":
+ * the right token is in the drafter's top 16 far more often than at top 1). */
+#define DFLASH2_K 16
+/* Largest block size (drafted positions + 1) the verify and select calls take. */
+#define DFLASH2_MAX_BLOCK 32
+
+/* Human-readable name of a status code (static storage, never NULL). */
+DFLASH2_API const char* dflash2_status_string(int status);
+
+/* Library ABI version, (major << 16) | minor. */
+DFLASH2_API int dflash2_version(void);
+
+/* Workspace bytes that any call with at most B sequences, G drafted positions
+ * per sequence (B*G rows for dflash2_topk_softmax) and vocabulary V needs.
+ * Returns 0 for B < 0, G < 1, G >= DFLASH2_MAX_BLOCK or V < 1. */
+DFLASH2_API size_t dflash2_workspace_bytes(int B, int G, int64_t V);
+
+/*
+ * Softmax and top-16 per drafted position.  [tamsi] "L’idée, sans le papier";
+ * [myaiexp] "主な機能" (the selector keeps the 16 best candidates per position).
+ *
+ * For each of `rows` rows (row r starts at logits + r * row_stride elements):
+ *   z_v = x_v * inv_temperature,  logz = log(sum_v exp(z_v)),
+ *   idx[r][k]  = the k-th best v by (x_v descending, v ascending), -0 == +0,
+ *   prob[r][k] = exp(z_idx - logz),  logp[r][k] = z_idx - logz.
+ *
+ * logits      [rows, row_stride] of `dtype`; rows V..row_stride-1 unused.
+ * rows        >= 0 (0 is a no-op); V in [16, 2^31 - 1]; row_stride >= V.
+ * inv_temperature  finite, > 0.
+ * idx         [rows, 16] int32;  prob, logp [rows, 16] float;  logz [rows] float.
+ * ws          workspace for B*G >= rows sequences-positions at this V.
+ * Rows whose start is 16-byte aligned are read with 128-bit loads; others are
+ * read element by element (correct, slower).
+ */
+DFLASH2_API int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows, int64_t V,
+                         int64_t row_stride, float inv_temperature, int32_t* idx, float* prob,
+                         float* logp, float* logz, void* ws, size_t ws_bytes,
+                         dflash2_stream_t stream);
+
+/*
+ * Bilinear adjacent-pair selector and the exact best path.  [tamsi] "L’idée,
+ * sans le papier" (choose a coherent path through the top-16 lists);
+ * [myaiexp] "主な機能" (adjacent candidate pairs are scored); [psi] "Résumé"
+ * (candidates chosen by a bilinear attention).  The pages give the selector
+ * in outline only; this call fixes it as
+ *   score(path) = sum_i logp[i][k_i] + pair(anchor, c[0][k_0])
+ *               + sum_{i>0} pair(c[i-1][k_{i-1}], c[i][k_i]),
+ *   pair(a, b)  = e(a)^T W e(b),
+ * maximised exactly over all 16^G paths (max-sum recursion over positions);
+ * on equal scores the smaller rank wins at every back-pointer and at the end.
+ *
+ * idx, logp   [B, G, 16] as written by dflash2_topk_softmax (c = idx).
+ * anchor      [B] int32 last accepted token per sequence, or NULL (no term).
+ * emb         [V, d] of `emb_dtype`; d in {64, 128}.
+ * W           [d, d] float, row-major (W[j][l] at j * d + l).
+ * B >= 0, 1 <= G < DFLASH2_MAX_BLOCK.
+ * path_tok    [B, G] int32 chosen tokens; path_rank [B, G] int32 their ranks;
+ * path_score  [B] float score of the chosen path.
+ */
+DFLASH2_API int dflash2_pair_select(const int32_t* idx, const float* logp, const int32_t* anchor,
+                        const void* emb, int emb_dtype, int64_t V, int d, const float* W, int B,
+                        int G, int32_t* path_tok, int32_t* path_rank, float* path_score,
+                        void* ws, size_t ws_bytes, dflash2_stream_t stream);
+
+/*
+ * Greedy lossless verify.  [tamsi] "Les chiffres qui comptent sur
+ * Qwen3.8-27B" (greedy output is exactly the target's); [latenode] "El
+ * desacuerdo..." (acceptance length = tokens completed per verify step).
+ *
+ * target      [B, G+1, V] of `dtype`: row j scores drafted position j, row G
+ *             the position after the block.
+ * draft_tok   [B, G] int32 drafted tokens (the selected path).
+ * t_j = argmax_v target[j][v] (lowest v on ties, -0 == +0);
+ * n = first j with draft_tok[j] != t_j, else G.
+ * n_accept    [B] int32 = n;  out_tok [B, G+1] int32 = draft_tok[0..n-1],
+ *             then t_n (correction, or bonus when n = G), then -1.
+ */
+DFLASH2_API int dflash2_verify_greedy(const void* target, int dtype, int B, int G, int64_t V,
+                          const int32_t* draft_tok, int32_t* n_accept, int32_t* out_tok,
+                          void* ws, size_t ws_bytes, dflash2_stream_t stream);
+
+/*
+ * Sampling lossless verify by rejection sampling.  [tamsi] "Les chiffres qui
+ * comptent sur Qwen3.8-27B" (rejection sampling keeps the target
+ * distribution); uniforms from Philox4x32-10 ([philox]).
+ *
+ * p_j = softmax(target[j] * inv_temperature), q_j = softmax(draft[j] * inv_temperature).
+ * For j = 0, 1, ...: r_j = p_j(d_j) / q_j(d_j); accept iff u_j < r_j; stop at
+ * the first rejection; n = accepted count.  If n < G the last token is drawn
+ * from max(0, p_n - q_n) (normalised; p_n if that is empty by rounding),
+ * else the bonus token is drawn from p_G.  A draw takes t = u' * R (R the
+ * total mass) and returns the smallest v whose inclusive prefix sum exceeds t
+ * (the last v with mass if rounding leaves none).
+ * q_mode DFLASH2_Q_ONEHOT: q_j is a point mass on d_j (the reading for a
+ * deterministic selector): r_j = p_j(d_j), residual = p_n without d_n, and
+ * `draft` is not read (may be NULL).
+ * Uniforms: Philox4x32-10 with key (seed low 32, seed high 32) and counter
+ * (step, seq_id[b], position, purpose); u = (word0 >> 8) * 2^-24; purpose 0
+ * for u_j, 1 for u' (position = n).
+ *
+ * target [B, G+1, V], draft [B, G, V] of `dtype`, rows 16-byte aligned for
+ * the fast path; draft_tok [B, G] int32; seq_id [B] uint32 or NULL (= b).
+ * n_accept [B], out_tok [B, G+1] as in dflash2_verify_greedy.
+ * ratio_dbg [B, G] float r_j for every j, u_dbg [B, G] float u_j; both
+ * optional (NULL).
+ */
+DFLASH2_API int dflash2_verify_sample(const void* target, const void* draft, int dtype, int B, int G,
+                          int64_t V, const int32_t* draft_tok, float inv_temperature,
+                          uint64_t seed, uint32_t step, const uint32_t* seq_id, int q_mode,
+                          int32_t* n_accept, int32_t* out_tok, float* ratio_dbg, float* u_dbg,
+                          void* ws, size_t ws_bytes, dflash2_stream_t stream);
+
+/*
+ * Two-tap dynamic depthwise conv fused with its tap projection and the
+ * residual add.  [tamsi] "L’idée, sans le papier" (two-tap conv before and
+ * after each attention and MLP); [myaiexp] "主な機能" (2-tap dynamic conv).
+ *
+ *   [a_t; b_t] = W_tap x_t  (W_tap [2H, H]: rows 0..H-1 give a, H..2H-1 give b)
+ *   out_t = x_t + a_t * x_t + b_t * x_{t-1},   x_{-1} = x_prev
+ * x [B, T, H], x_prev [B, H], w_tap [2H, H], out [B, T, H], all of `dtype`,
+ * 16-byte aligned; H a multiple of 64; B, T >= 0.  fp32 accumulation, one
+ * rounding at the output.
+ */
+DFLASH2_API int dflash2_dynconv2(const void* x, const void* x_prev, const void* w_tap, int dtype, int B,
+                     int T, int H, void* out, dflash2_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DFLASH2_H */

@@ -1,0 +1,151 @@
+"""The C ABI library loads on a machine without a GPU, exports every entry
+point include/dflash2.h declares, and rejects bad arguments on the host with
+the documented status codes before any CUDA call (none of these tests needs a
+device: validation returns before anything is enqueued)."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+OK, EINVAL, EDTYPE, ESHAPE, EWORKSPACE, ECUDA, EALIGN = range(7)
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_draft_verification_b200 import build
+    build.build()
+    import block_draft_verification_b200 as d
+    return d.lib()
+
+
+def declared_symbols():
+    names = set()
+    for f in os.listdir(HEADER_DIR):
+        if f.endswith(".h"):
+            text = open(os.path.join(HEADER_DIR, f)).read()
+            names |= set(re.findall(r"DFLASH2_API\s+[\w\s\*]+?\b(dflash2_\w+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_symbols()
+    assert {"dflash2_topk_softmax", "dflash2_pair_select", "dflash2_verify_greedy",
+            "dflash2_verify_sample", "dflash2_dynconv2"} <= names
+    from block_draft_verification_b200 import LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (dflash2_\w+)", out))
+    assert names <= exported, names - exported
+    # nothing but the declared ABI is exported under the dflash2_ prefix
+    assert exported == names
+    for n in names:
+        assert getattr(L, n) is not None
+
+
+def test_status_strings_and_version(L):
+    import block_draft_verification_b200 as d
+    for code in range(7):
+        assert d.status_string(code).startswith("DFLASH2_")
+    assert d.status_string(99) == "DFLASH2_UNKNOWN_STATUS"
+    assert d.version() == (1, 0)
+
+
+def test_workspace_bytes(L):
+    import block_draft_verification_b200 as d
+    assert d.workspace_bytes(1, 7, 151936) > 0
+    assert d.workspace_bytes(32, 7, 151936) > d.workspace_bytes(8, 7, 151936)
+    assert d.workspace_bytes(8, 15, 151936) > d.workspace_bytes(8, 7, 151936)
+    assert d.workspace_bytes(1, 0, 100) == 0
+    assert d.workspace_bytes(1, 32, 100) == 0
+    assert d.workspace_bytes(-1, 7, 100) == 0
+    assert d.workspace_bytes(0, 7, 100) >= 0
+    assert d.workspace_bytes(4, 7, 100) % 256 == 0
+
+
+# fake, aligned, never dereferenced device addresses: validation fails first
+P = C.c_void_p(0x10000)
+P2 = C.c_void_p(0x20000)
+ODD = C.c_void_p(0x10001)
+S0 = C.c_void_p(0)
+
+
+def topk(L, logits=P, dtype=1, rows=7, V=151936, stride=151936, invT=1.0, idx=P, prob=P,
+         logp=P, logz=P, ws=P2, wsb=1 << 30):
+    return L.dflash2_topk_softmax(logits, dtype, rows, V, stride, invT, idx, prob, logp, logz, ws,
+                                  wsb, S0)
+
+
+def test_topk_validation(L):
+    assert topk(L, dtype=5) == EDTYPE
+    assert topk(L, V=15) == ESHAPE
+    assert topk(L, stride=100) == ESHAPE
+    assert topk(L, rows=-1) == ESHAPE
+    assert topk(L, invT=0.0) == EINVAL
+    assert topk(L, invT=float("inf")) == EINVAL
+    assert topk(L, invT=float("nan")) == EINVAL
+    assert topk(L, rows=0) == OK          # nothing to do, nothing launched
+    assert topk(L, logits=None) == EINVAL
+    assert topk(L, logz=None) == EINVAL
+    assert topk(L, logits=ODD) == EALIGN
+    assert topk(L, ws=None) == EWORKSPACE
+    assert topk(L, ws=C.c_void_p(0x20010)) == EWORKSPACE   # not 256-aligned
+    assert topk(L, wsb=1000) == EWORKSPACE
+
+
+def test_select_validation(L):
+    def sel(idx=P, logp=P, anchor=None, emb=P, edt=1, V=151936, d=128, W=P, B=2, G=7, tok=P,
+            rank=P, score=P, ws=P2, wsb=1 << 30):
+        return L.dflash2_pair_select(idx, logp, anchor, emb, edt, V, d, W, B, G, tok, rank, score,
+                                     ws, wsb, S0)
+    assert sel(edt=3) == EDTYPE
+    assert sel(d=96) == ESHAPE
+    assert sel(G=0) == ESHAPE
+    assert sel(G=32) == ESHAPE
+    assert sel(B=-2) == ESHAPE
+    assert sel(B=0) == OK
+    assert sel(W=None) == EINVAL
+    assert sel(idx=ODD) == EALIGN
+    assert sel(wsb=16) == EWORKSPACE
+
+
+def test_verify_validation(L):
+    def greedy(t=P, dt=1, B=2, G=7, V=151936, d=P, n=P, o=P, ws=P2, wsb=1 << 30):
+        return L.dflash2_verify_greedy(t, dt, B, G, V, d, n, o, ws, wsb, S0)
+    assert greedy(dt=2) == EDTYPE
+    assert greedy(G=0) == ESHAPE
+    assert greedy(G=32) == ESHAPE
+    assert greedy(V=0) == ESHAPE
+    assert greedy(B=0) == OK
+    assert greedy(n=None) == EINVAL
+    assert greedy(o=ODD) == EALIGN
+    assert greedy(ws=None) == EWORKSPACE
+
+    def sample(t=P, q=P, dt=1, B=2, G=7, V=151936, d=P, invT=1.0, qm=0, n=P, o=P, ws=P2,
+               wsb=1 << 30):
+        return L.dflash2_verify_sample(t, q, dt, B, G, V, d, invT, 0, 0, None, qm, n, o, None,
+                                       None, ws, wsb, S0)
+    assert sample(dt=9) == EDTYPE
+    assert sample(G=40) == ESHAPE
+    assert sample(invT=-1.0) == EINVAL
+    assert sample(qm=2) == EINVAL
+    assert sample(q=None) == EINVAL            # softmax mode needs the draft logits
+    assert sample(B=0) == OK
+    assert sample(t=ODD) == EALIGN
+    assert sample(wsb=0) == EWORKSPACE
+
+
+def test_dynconv_validation(L):
+    def conv(x=P, xp=P, w=P, dt=1, B=2, T=8, H=5120, out=P2):
+        return L.dflash2_dynconv2(x, xp, w, dt, B, T, H, out, S0)
+    assert conv(dt=4) == EDTYPE
+    assert conv(H=100) == ESHAPE
+    assert conv(H=0) == ESHAPE
+    assert conv(B=-1) == ESHAPE
+    assert conv(T=0) == OK
+    assert conv(w=None) == EINVAL
+    assert conv(x=C.c_void_p(0x10008)) == EALIGN
