@@ -192,7 +192,11 @@ __global__ void __launch_bounds__(NT) verify_sample_scan_kernel(
         I.mt = ltm;
         I.l2t = (float)log2(lts);
         I.mq = lqm;
-        I.l2q = (n < G && q_mode == DFLASH2_Q_SOFTMAX) ? (float)log2(lqs) : 0.0f;
+        const bool resid = n < G && q_mode == DFLASH2_Q_SOFTMAX;
+        I.l2q = resid ? (float)log2(lqs) : 0.0f;
+        I.dl = resid ? (float)(((double)ltm - (double)lqm) * (double)inv_t + log(lts) - log(lqs))
+                     : 0.0f;
+        I.pad = 0;
         I.u_res = philox_uniform(seed, step, sid, (uint32_t)n, 1u);
         I.n = n;
         I.mode = (n == G) ? 2 : (q_mode == DFLASH2_Q_SOFTMAX ? 0 : 1);
@@ -205,16 +209,23 @@ __global__ void __launch_bounds__(NT) verify_sample_scan_kernel(
 // ------------------------------------------------------------------ sampling, pass 2
 // The draw weights of element v of the row the sequence draws from:
 //   p_v = exp2((x_v - mt) * c - l2t),  q_v likewise,
-//   mode 0: w = max(0, p - q);  mode 1: w = p, 0 at d;  mode 2: w = p.
+//   mode 0: w = max(0, p - q), evaluated as q * expm1(ln p - ln q) with
+//           ln p - ln q = (xt - xq) * invT - (logZ_t - logZ_q): the same
+//           value, without the cancellation of p - q when p and q agree;
+//   mode 1: w = p, 0 at d;  mode 2: w = p.
 // The fallback weight (R = 0) is p.
 template <bool BF16>
 __device__ __forceinline__ void draw_weight(const uint4& rt, const uint4& rq, int e, int64_t v,
-                                            const SampleInfo& I, float c, float& w, float& p) {
+                                            const SampleInfo& I, float c, float inv_t, float& w,
+                                            float& p) {
     using R = Row<BF16>;
-    p = ex2((R::elem(rt, e) - I.mt) * c - I.l2t);
+    const float xt = R::elem(rt, e);
+    p = ex2((xt - I.mt) * c - I.l2t);
     if (I.mode == 0) {
-        const float q = ex2((R::elem(rq, e) - I.mq) * c - I.l2q);
-        w = fmaxf(0.0f, p - q);
+        const float xq = R::elem(rq, e);
+        const float q = ex2((xq - I.mq) * c - I.l2q);
+        const float dlog = (xt - xq) * inv_t - I.dl;
+        w = dlog > 0.0f ? q * expm1f(dlog) : 0.0f;
     } else if (I.mode == 1) {
         w = (v == I.d) ? 0.0f : p;
     } else {
@@ -257,7 +268,7 @@ __device__ __forceinline__ void load_contig(const void* row, int64_t v0, int64_t
 template <bool BF16, bool VEC>
 __global__ void __launch_bounds__(NT) verify_sample_draw_kernel(
     const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int S,
-    float c2, const SampleInfo* __restrict__ info, double* __restrict__ part2,
+    float c2, float inv_t, const SampleInfo* __restrict__ info, double* __restrict__ part2,
     unsigned* __restrict__ counters2, int32_t* __restrict__ out_tok) {
     using R = Row<BF16>;
     constexpr int ES = BF16 ? 2 : 4;
@@ -287,8 +298,8 @@ __global__ void __launch_bounds__(NT) verify_sample_draw_kernel(
 #pragma unroll
             for (int e = 0; e < R::VW; ++e) {
                 float w, p;
-                draw_weight<BF16>(rt[i], rq[i], e, v0 + (int64_t)t * EPT + i * R::VW + e, I, c2, w,
-                                  p);
+                draw_weight<BF16>(rt[i], rq[i], e, v0 + (int64_t)t * EPT + i * R::VW + e, I, c2, inv_t,
+                                  w, p);
                 sw += (double)w;
                 sp += (double)p;
             }
@@ -364,7 +375,8 @@ __global__ void __launch_bounds__(NT) verify_sample_draw_kernel(
 #pragma unroll
         for (int e = 0; e < R::VW; ++e) {
             float w, p;
-            draw_weight<BF16>(rt[i], rq[i], e, v0 + (int64_t)t * EPT + i * R::VW + e, I, c2, w, p);
+            draw_weight<BF16>(rt[i], rq[i], e, v0 + (int64_t)t * EPT + i * R::VW + e, I, c2, inv_t, w,
+                              p);
             wreg[i * R::VW + e] = fb ? p : w;
             mysum += (double)wreg[i * R::VW + e];
         }
@@ -490,7 +502,8 @@ extern "C" int dflash2_verify_sample(const void* target, const void* draft, int 
         verify_sample_scan_kernel<BF, VE><<<grid1, block, 0, s>>>(                                  \
             target, q, G, V, (int)S, rows_per_seq, inv_temperature, c2, draft_tok, seed, step,       \
             seq_id, q_mode, n_accept, out_tok, ratio_dbg, u_dbg, part, info, counters);             \
-        verify_sample_draw_kernel<BF, VE><<<grid2, block, 0, s>>>(target, q, G, V, (int)S, c2, info, \
+        verify_sample_draw_kernel<BF, VE><<<grid2, block, 0, s>>>(target, q, G, V, (int)S, c2,     \
+                                                                  inv_temperature, info,        \
                                                                   part2, counters + B, out_tok);    \
     } while (0)
     if (dtype == DFLASH2_BF16) {

@@ -21,14 +21,17 @@ struct TopkPartial {
 };
 
 // Per-sequence state handed from the verify_sample scan to its draw:
-// p_v = exp2((x_v - mt) * c - l2t) on the target row used, likewise q.
+// p_v = exp2((x_v - mt) * c - l2t) on the target row used, likewise q, and
+// dl = logZ_t - logZ_q (natural log) for the residual.
 struct SampleInfo {
     float mt, l2t;    // target row max and log2 of its sum-exp
     float mq, l2q;    // draft row (mode 0 only)
+    float dl;         // logZ_t - logZ_q (mode 0 only)
     float u_res;      // u' of the draw
     int32_t n;        // accepted count = row the draw uses
     int32_t mode;     // 0 = residual max(0, p - q), 1 = p without d_n, 2 = p
     int32_t d;        // the rejected drafted token (mode 1)
+    int32_t pad;
 };
 
 struct Layout {
