@@ -13,7 +13,7 @@ import torch
 
 __all__ = ["F32", "BF16", "Q_SOFTMAX", "Q_ONEHOT", "K", "DFlash2Error", "lib", "workspace_bytes",
            "Workspace", "topk_softmax", "pair_select", "verify_greedy", "verify_sample",
-           "dynconv2", "status_string", "version"]
+           "dynconv2", "status_string", "version", "device_errors"]
 
 F32, BF16 = 0, 1
 Q_SOFTMAX, Q_ONEHOT = 0, 1
@@ -51,6 +51,8 @@ def lib():
         L.dflash2_verify_sample.argtypes = [vp, vp, i32, i32, i32, i64, vp, f32, u64, u32, vp, i32,
                                             vp, vp, vp, vp, vp, sz, vp]
         L.dflash2_dynconv2.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp]
+        L.dflash2_device_errors.argtypes = [i32]
+        L.dflash2_device_errors.restype = C.c_uint32
         for f in ("dflash2_topk_softmax", "dflash2_pair_select", "dflash2_verify_greedy",
                   "dflash2_verify_sample", "dflash2_dynconv2"):
             getattr(L, f).restype = i32
@@ -65,6 +67,11 @@ def status_string(status):
 def version():
     v = lib().dflash2_version()
     return (v >> 16, v & 0xFFFF)
+
+
+def device_errors(clear=True):
+    """Flags set by a tensor-core kernel whose bounded wait ran out (0 = none)."""
+    return int(lib().dflash2_device_errors(1 if clear else 0))
 
 
 def workspace_bytes(B, G, V):

@@ -9,10 +9,11 @@
 //   [a_t; b_t] = W_tap x_t           (W_tap [2H, H], nn.Linear layout)
 //   out_t = x_t + a_t * x_t + b_t * x_{t-1},   x_{-1} = x_prev
 //
-// SIMT path: one warp per (output channel h, block of 8 tokens) streams the
-// two weight rows h and H + h with 128-bit loads and dots them with the 8
-// token vectors, fp32 accumulation, then applies the conv and residual in the
-// epilogue and rounds once.
+// fp32 operands take the SIMT path here: one warp per (output channel h,
+// block of 8 tokens) streams the two weight rows h and H + h with 128-bit
+// loads and dots them with the 8 token vectors, fp32 accumulation, then
+// applies the conv and residual in the epilogue.  bf16 operands take the
+// tensor-core path of dynconv2_tc.cu.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -98,6 +99,9 @@ __global__ void __launch_bounds__(NT) dynconv2_simt_kernel(const void* __restric
 using namespace dfl;
 using namespace dfl_host;
 
+int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_tap, int B, int T,
+                               int H, void* out, cudaStream_t s);
+
 extern "C" int dflash2_dynconv2(const void* x, const void* x_prev, const void* w_tap, int dtype,
                                 int B, int T, int H, void* out, dflash2_stream_t stream) {
     if (!dtype_ok(dtype)) return DFLASH2_EDTYPE;
@@ -112,11 +116,9 @@ extern "C" int dflash2_dynconv2(const void* x, const void* x_prev, const void* w
     const int64_t blocks = (warps + NT / 32 - 1) / (NT / 32);
     if (blocks > (int64_t)INT32_MAX) return DFLASH2_ESHAPE;
     cudaStream_t s = (cudaStream_t)stream;
-    if (dtype == DFLASH2_BF16)
-        dynconv2_simt_kernel<true><<<(unsigned)blocks, NT, 0, s>>>(x, x_prev, w_tap, T, H,
-                                                                   (int)ntok, out);
-    else
-        dynconv2_simt_kernel<false><<<(unsigned)blocks, NT, 0, s>>>(x, x_prev, w_tap, T, H,
-                                                                    (int)ntok, out);
+    if (dtype == DFLASH2_BF16)  // tensor cores (tcgen05 + TMA), dynconv2_tc.cu
+        return dflash2_dynconv2_tc_launch(x, x_prev, w_tap, B, T, H, out, s);
+    dynconv2_simt_kernel<false><<<(unsigned)blocks, NT, 0, s>>>(x, x_prev, w_tap, T, H, (int)ntok,
+                                                                out);
     return launch_status();
 }

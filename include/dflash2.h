@@ -206,6 +206,16 @@ DFLASH2_API int dflash2_verify_sample(const void* target, const void* draft, int
 DFLASH2_API int dflash2_dynconv2(const void* x, const void* x_prev, const void* w_tap, int dtype, int B,
                      int T, int H, void* out, dflash2_stream_t stream);
 
+/*
+ * Device-side error flags of the tensor-core kernels on the current device
+ * (0 = none).  Every wait inside those kernels is bounded; a wait that runs
+ * out sets a flag bit (1 producer, 2 MMA issuer, 4 epilogue, 8 drain), the
+ * kernel releases its tensor memory and returns, and the call's outputs are
+ * not valid.  Synchronous (reads device memory); clear != 0 resets the flags.
+ * Returns 0xFFFFFFFF if the flags cannot be read.
+ */
+DFLASH2_API unsigned dflash2_device_errors(int clear);
+
 #ifdef __cplusplus
 }
 #endif
