@@ -29,3 +29,14 @@ extern "C" size_t dflash2_workspace_bytes(int B, int G, int64_t V) {
     need = need > select_layout(B, G).total ? need : select_layout(B, G).total;
     return need;
 }
+
+unsigned dfl_errors_topk(int clear);
+unsigned dfl_errors_verify(int clear);
+unsigned dfl_errors_dynconv(int clear);
+
+extern "C" unsigned dflash2_device_errors(int clear) {
+    const unsigned a = dfl_errors_topk(clear), b = dfl_errors_verify(clear),
+                   c = dfl_errors_dynconv(clear);
+    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu) return 0xFFFFFFFFu;
+    return a | b | c;
+}

@@ -21,19 +21,16 @@
 //   warps 4-7 epilogue: tcgen05.ld of their 32 TMEM lanes; the b rows go
 //            through shared memory to the a rows' threads, which load x and
 //            x_prev, apply the conv and the residual and store bf16
-// Every mbarrier wait is bounded (about one second); on a timeout the kernel
-// records a flag (dflash2_device_errors), stops issuing work, releases TMEM
-// and returns.  No TMA load here uses cluster multicast.
+// Every mbarrier wait is bounded (one second, stream.cuh); on a timeout the
+// kernel records a flag (dflash2_device_errors), stops issuing work, releases
+// TMEM and returns.  No TMA load here uses cluster multicast.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "stream.cuh"
 
 namespace dfl {
-
-__device__ unsigned int g_device_errors;
-
-enum : unsigned { ERR_PRODUCER = 1u, ERR_MMA = 2u, ERR_EPILOGUE = 4u, ERR_DRAIN = 8u };
 
 constexpr int TC_BM = 128;          // accumulator rows: 64 a-channels + 64 b-channels
 constexpr int TC_CH = 64;           // channels per CTA
@@ -41,40 +38,7 @@ constexpr int TC_BK = 64;           // K elements per stage (128 bytes of bf16)
 constexpr int TC_MAXN = 256;        // tokens per accumulator
 constexpr int TC_THREADS = 256;
 constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;  // 16 KB
-constexpr uint64_t WAIT_NS = 1000000000ull;    // bound on any single wait
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-// Wait for the completion of the phase with the given parity; false after
-// WAIT_NS nanoseconds without it.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    const uint64_t t0 = global_ns();
-    while (true) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (done) return true;
-        if (global_ns() - t0 > WAIT_NS) return false;
-    }
-}
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             uint32_t bar) {
     asm volatile(
@@ -162,7 +126,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
             mbar_init(empty0 + 8 * s, 1);
         }
         mbar_init(accf, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_fence_init();
     }
     if (warp == 2) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -182,7 +146,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
         for (; kb < sh.nkb; ++kb) {
             const int s = kb % sh.stages, r = kb / sh.stages;
             if (r > 0 && !mbar_wait(empty0 + 8 * s, (r - 1) & 1)) {
-                atomicOr(&g_device_errors, ERR_PRODUCER);
+                atomicOr(&g_dev_err, ERR_PRODUCER);
                 break;
             }
             const uint32_t a = smem_u32(base + s * stage_bytes);
@@ -197,7 +161,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
         for (int k = (kb > sh.stages ? kb - sh.stages : 0); k < kb; ++k) {
             const int s = k % sh.stages, r = k / sh.stages;
             if (!mbar_wait(empty0 + 8 * s, r & 1)) {
-                atomicOr(&g_device_errors, ERR_DRAIN);
+                atomicOr(&g_dev_err, ERR_DRAIN);
                 break;
             }
         }
@@ -207,7 +171,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
         for (int kb = 0; kb < sh.nkb; ++kb) {
             const int s = kb % sh.stages, r = kb / sh.stages;
             if (!mbar_wait(full0 + 8 * s, r & 1)) {
-                atomicOr(&g_device_errors, ERR_MMA);
+                atomicOr(&g_dev_err, ERR_MMA);
                 break;
             }
             tc_fence_after();
@@ -224,7 +188,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
         // ---------------- epilogue
         const int q = warp - 4;  // TMEM lanes 32q .. 32q + 31
         bool ok = mbar_wait(accf, 0);
-        if (!ok) atomicOr(&g_device_errors, ERR_EPILOGUE);
+        if (!ok) atomicOr(&g_dev_err, ERR_EPILOGUE);
         ok = __all_sync(FULL, ok);  // tcgen05.ld is warp-collective
         tc_fence_after();
         for (int c0 = 0; c0 < sh.BN; c0 += 32) {
@@ -336,14 +300,12 @@ int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_
     return cudaGetLastError() == cudaSuccess ? DFLASH2_OK : DFLASH2_ECUDA;
 }
 
-// Reads (and with clear != 0 resets) the device-side error flags of the
-// tensor-core kernels on the current device.  Synchronous.
-extern "C" DFLASH2_API unsigned dflash2_device_errors(int clear) {
+unsigned dfl_errors_dynconv(int clear) {
     unsigned v = 0;
-    if (cudaMemcpyFromSymbol(&v, dfl::g_device_errors, sizeof v) != cudaSuccess) return 0xFFFFFFFFu;
-    if (clear) {
+    if (cudaMemcpyFromSymbol(&v, dfl::g_dev_err, sizeof v) != cudaSuccess) return 0xFFFFFFFFu;
+    if (clear && v) {
         unsigned z = 0;
-        cudaMemcpyToSymbol(dfl::g_device_errors, &z, sizeof z);
+        cudaMemcpyToSymbol(dfl::g_dev_err, &z, sizeof z);
     }
     return v;
 }

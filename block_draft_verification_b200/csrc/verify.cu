@@ -10,15 +10,17 @@
 // tablas del proveedor": acceptance length = tokens completed per verify step.
 // Uniforms: Philox4x32-10 (Salmon et al., SC'11, section 5).
 //
-// Both verifies stream every logit row once in 16384-element chunks, one CTA
-// per (sequence, row, chunk).  The last CTA of a sequence (arrival ticket, no
-// waiting) reduces the per-chunk partials in chunk order and decides.  The
-// sampling draw needs the normalisers first, so it is a second kernel: one
-// CTA per chunk of the one row each sequence draws from (L2-resident after
-// the first pass), then the last of them finds the chunk where the inverse
-// CDF crosses t = u' * R and scans only that chunk.  No probability vector is
-// ever written to memory.
+// Both verifies stream every logit row once in 16384-element chunks: work
+// unit = (sequence, row, chunk), persistent CTAs, TMA bulk copies into a
+// two-slot shared-memory ring.  The last unit of a sequence to finish
+// (arrival ticket, no waiting) reduces the partials in chunk order and
+// decides.  The sampling draw needs the normalisers first, so it is a second
+// kernel over the one row each sequence draws from (L2-resident after the
+// first pass): one CTA per chunk sums the draw weights, and the last of them
+// finds the chunk where the inverse CDF crosses t = u' * R and scans only that
+// chunk.  No probability vector is ever written to memory.
 #include "common.cuh"
+#include "stream.cuh"
 #include "workspace.cuh"
 
 namespace dfl {
@@ -26,149 +28,152 @@ namespace dfl {
 constexpr double LOG2E = 1.4426950408889634;
 
 // ------------------------------------------------------------------ greedy
-template <bool BF16, bool VEC>
-__global__ void __launch_bounds__(NT) verify_greedy_kernel(
-    const void* __restrict__ target, int G, int64_t V, int S, const int32_t* __restrict__ draft_tok,
-    int32_t* __restrict__ n_accept, int32_t* __restrict__ out_tok, uint64_t* __restrict__ part,
-    unsigned* __restrict__ counters) {
-    using R = Row<BF16>;
-    __shared__ float s_max[NT / 32];
-    __shared__ unsigned s_first;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int units = (G + 1) * S;
-    const int b = blockIdx.x / units;
-    const int rem = blockIdx.x - b * units;
-    const int j = rem / S, chunk = rem - j * S;
-    const int64_t row = (int64_t)b * (G + 1) + j;
-    const int64_t v0 = (int64_t)chunk * CHUNK, vend = min(V, v0 + (int64_t)CHUNK);
+struct GreedySmem {
+    float wmax[NT / 32];
+    unsigned first;
+};
 
-    uint4 r[R::NV];
-    R::template load<VEC>((const char*)target + row * V * (BF16 ? 2 : 4), v0, vend, r);
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < R::NV; ++i)
-#pragma unroll
-        for (int e = 0; e < R::VW; ++e) m = fmaxf(m, R::elem(r[i], e));
+template <bool BF16, class C>
+__device__ __forceinline__ void greedy_unit(const C& ch, GreedySmem& sm, uint64_t* slot) {
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const float m = view_max<BF16>(ch);
     float wm = m;
 #pragma unroll
     for (int k = 16; k > 0; k >>= 1) wm = fmaxf(wm, __shfl_xor_sync(FULL, wm, k));
-    if (lane == 0) s_max[warp] = wm;
-    if (t == 0) s_first = 0xFFFFFFFFu;
+    if (lane == 0) sm.wmax[warp] = wm;
+    if (t == 0) sm.first = 0xFFFFFFFFu;
     __syncthreads();
-    float M = s_max[0];
+    float M = sm.wmax[0];
 #pragma unroll
-    for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, s_max[w]);
-    // the lowest index holding the chunk max (-0 == +0 in the compare)
-    if (m == M) {
-        uint32_t first = 0xFFFFFFFFu;
-#pragma unroll
-        for (int i = R::NV - 1; i >= 0; --i)
-#pragma unroll
-            for (int e = R::VW - 1; e >= 0; --e)
-                if (R::elem(r[i], e) == M) first = (uint32_t)R::index_of(v0, i, e);
-        atomicMin(&s_first, first);
-    }
+    for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, sm.wmax[w]);
+    if (m == M) atomicMin(&sm.first, view_first<BF16>(ch, M));  // -0 == +0
     __syncthreads();
     if (t == 0) {
-        part[row * S + chunk] = make_key(M, s_first);
+        *slot = make_key(M, sm.first);
         __threadfence();
     }
-    if (!arrive_last(&counters[b], (unsigned)units)) return;
-    if (warp != 0) return;
+}
 
-    // lane j reduces target row j over its chunks (G + 1 <= 32 rows)
-    uint64_t best = 0;
-    if (lane <= G) {
-        const uint64_t* P = part + ((int64_t)b * (G + 1) + lane) * S;
+__device__ __forceinline__ void greedy_finish(const uint64_t* P, int S, int G, int b,
+                                              const int32_t* __restrict__ draft_tok,
+                                              int32_t* __restrict__ n_accept,
+                                              int32_t* __restrict__ out_tok) {
+    const int lane = threadIdx.x & 31;
+    uint64_t best = 0;  // lane j reduces target row j over its chunks (G + 1 <= 32)
+    if (lane <= G)
         for (int c = 0; c < S; ++c) {
-            uint64_t k = (uint64_t)__ldcg((const unsigned long long*)&P[c]);
+            const uint64_t k = (uint64_t)__ldcg((const unsigned long long*)&P[(int64_t)lane * S + c]);
             best = k > best ? k : best;
         }
-    }
     const int32_t tj = (int32_t)key_index(best);
     const int32_t dj = (lane < G) ? draft_tok[(int64_t)b * G + lane] : -1;
     const unsigned miss = __ballot_sync(FULL, lane < G && dj != tj);
     const int n = miss ? (__ffs(miss) - 1) : G;
-    if (lane <= G) {
-        int32_t o = -1;
-        if (lane < n) o = dj;
-        else if (lane == n) o = tj;
-        out_tok[(int64_t)b * (G + 1) + lane] = o;
-    }
+    if (lane <= G) out_tok[(int64_t)b * (G + 1) + lane] = (lane < n) ? dj : (lane == n ? tj : -1);
     if (lane == 0) n_accept[b] = n;
+}
+
+template <bool BF16, bool TMA>
+__global__ void __launch_bounds__(NT, 3) verify_greedy_kernel(
+    const void* __restrict__ target, int G, int64_t V, int S, int64_t units,
+    const int32_t* __restrict__ draft_tok, int32_t* __restrict__ n_accept,
+    int32_t* __restrict__ out_tok, uint64_t* __restrict__ part, unsigned* __restrict__ counters) {
+    constexpr int ES = BF16 ? 2 : 4;
+    constexpr int SLOT = CHUNK * ES;
+    extern __shared__ __align__(128) uint8_t ring[];
+    __shared__ GreedySmem sm;
+    __shared__ __align__(8) uint64_t s_bar[2];
+    const int t = threadIdx.x, warp = t >> 5;
+    const uint32_t bar0 = smem_u32(&s_bar[0]);
+    const int per_seq = (G + 1) * S;
+    auto geom = [&](int64_t u, int& b, int64_t& row, int64_t& v0, int64_t& vend) {
+        b = (int)(u / per_seq);
+        const int rem = (int)(u - (int64_t)b * per_seq);
+        const int j = rem / S;
+        row = (int64_t)b * (G + 1) + j;
+        v0 = (int64_t)(rem - j * S) * CHUNK;
+        vend = min(V, v0 + (int64_t)CHUNK);
+    };
+    auto issue = [&](int64_t u, int slot) {
+        int b;
+        int64_t row, v0, vend;
+        geom(u, b, row, v0, vend);
+        bulk_g2s(smem_u32(ring + slot * SLOT), (const char*)target + (row * V + v0) * ES,
+                 (uint32_t)((vend - v0) * ES), bar0 + 8 * slot);
+    };
+    if (TMA) {
+        if (t == 0) {
+            mbar_init(bar0, 1);
+            mbar_init(bar0 + 8, 1);
+            mbar_fence_init();
+            if ((int64_t)blockIdx.x < units) issue(blockIdx.x, 0);
+        }
+        __syncthreads();
+    }
+    int k = 0;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++k) {
+        int b;
+        int64_t row, v0, vend;
+        geom(u, b, row, v0, vend);
+        uint64_t* slot = part + row * S + (v0 / CHUNK);
+        if (TMA) {
+            const int64_t un = u + gridDim.x;
+            if (t == 0 && un < units) issue(un, (k + 1) & 1);
+            if (!__syncthreads_and(mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1))) {
+                if (t == 0) {
+                    atomicOr(&g_dev_err, ERR_STREAM);
+                    if (un < units) mbar_wait(bar0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
+                }
+                return;
+            }
+            greedy_unit<BF16>(SmemChunk<BF16>{ring + (k & 1) * SLOT, v0, vend}, sm, slot);
+        } else {
+            RegChunk<BF16> ch;
+            ch.load((const char*)target + row * V * ES, v0, vend);
+            greedy_unit<BF16>(ch, sm, slot);
+        }
+        const bool last = arrive_last(&counters[b], (unsigned)per_seq);
+        if (last && warp == 0)
+            greedy_finish(part + (int64_t)b * (G + 1) * S, S, G, b, draft_tok, n_accept, out_tok);
+        __syncthreads();  // ring slot k & 1 is free for the prefetch of iteration k + 1
+    }
 }
 
 // ------------------------------------------------------------------ sampling, pass 1
 // Units: for sequence b, rows 0..G are target rows, G+1..2G draft rows (softmax
-// mode only).  Each unit writes its (max, fp64 sum-exp) partial.
-template <bool BF16, bool VEC>
-__global__ void __launch_bounds__(NT) verify_sample_scan_kernel(
-    const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int S,
-    int rows_per_seq, float inv_t, float c2, const int32_t* __restrict__ draft_tok, uint64_t seed,
-    uint32_t step, const uint32_t* __restrict__ seq_id, int q_mode, int32_t* __restrict__ n_accept,
+// mode only).  Each unit writes its (max, fp64 sum-exp) partial; the last
+// unit of the sequence runs the accept tests.
+__device__ __forceinline__ void sample_finish(
+    const void* __restrict__ target, const void* __restrict__ draft, const LseD* P, int G,
+    int64_t V, int S, int es, float inv_t, float c2, const int32_t* __restrict__ draft_tok,
+    uint64_t seed, uint32_t step, uint32_t sid, int q_mode, int b, int32_t* __restrict__ n_accept,
     int32_t* __restrict__ out_tok, float* __restrict__ ratio_dbg, float* __restrict__ u_dbg,
-    LseD* __restrict__ part, SampleInfo* __restrict__ info, unsigned* __restrict__ counters) {
-    using R = Row<BF16>;
-    constexpr int ES = BF16 ? 2 : 4;
-    __shared__ LseD s_lse[NT / 32];
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int units = rows_per_seq * S;
-    const int b = blockIdx.x / units;
-    const int rem = blockIdx.x - b * units;
-    const int rr = rem / S, chunk = rem - rr * S;
-    const int64_t v0 = (int64_t)chunk * CHUNK, vend = min(V, v0 + (int64_t)CHUNK);
-    const char* rowp = (rr <= G)
-                           ? (const char*)target + ((int64_t)b * (G + 1) + rr) * V * ES
-                           : (const char*)draft + ((int64_t)b * G + (rr - G - 1)) * V * ES;
-
-    uint4 r[R::NV];
-    R::template load<VEC>(rowp, v0, vend, r);
-    LseD mine = thread_lse_d<BF16>(r, c2);
-    LseD wl = warp_lse(mine, c2);
-    if (lane == 0) s_lse[warp] = wl;
-    __syncthreads();
-    if (t == 0) {
-        LseD tot = s_lse[0];
-        for (int w = 1; w < NT / 32; ++w) tot = lse_merge(tot, s_lse[w], c2);
-        part[((int64_t)b * rows_per_seq + rr) * S + chunk] = tot;
-        __threadfence();
-    }
-    if (!arrive_last(&counters[b], (unsigned)units)) return;
-    if (warp != 0) return;
-
-    // Lane j: logZ of target row j (j <= G) and of draft row j (j < G), in
-    // chunk order; then the ratio and the accept test of position j.
-    auto row_lse = [&](int rrow) {
-        const LseD* P = part + ((int64_t)b * rows_per_seq + rrow) * S;
+    SampleInfo* __restrict__ info) {
+    const int lane = threadIdx.x & 31;
+    auto row_lse = [&](int rrow) {  // chunk order
         LseD acc{-INFINITY, 0.0f, 0.0};
         for (int c = 0; c < S; ++c) {
-            LseD p;
-            p.m = __ldcg(&P[c].m);
-            p.pad = 0.0f;
-            p.s = __ldcg(&P[c].s);
+            LseD p{__ldcg(&P[(int64_t)rrow * S + c].m), 0.0f, __ldcg(&P[(int64_t)rrow * S + c].s)};
             acc = lse_merge(acc, p, c2);
         }
         return acc;
     };
-    const uint32_t sid = seq_id ? seq_id[b] : (uint32_t)b;
+    auto elem = [&](const void* base, int64_t row, int32_t v) -> double {
+        if (es == 2)
+            return (double)__uint_as_float((uint32_t)((const uint16_t*)base)[row * V + v] << 16);
+        return (double)((const float*)base)[row * V + v];
+    };
     LseD lt{-INFINITY, 0.0f, 0.0}, lq{-INFINITY, 0.0f, 0.0};
     if (lane <= G) lt = row_lse(lane);
     if (q_mode == DFLASH2_Q_SOFTMAX && lane < G) lq = row_lse(G + 1 + lane);
     bool reject = false;
     if (lane < G) {
         const int32_t d = draft_tok[(int64_t)b * G + lane];
-        const char* trow = (const char*)target + ((int64_t)b * (G + 1) + lane) * V * ES;
-        const double xt = BF16 ? (double)__uint_as_float((uint32_t)((const uint16_t*)trow)[d] << 16)
-                               : (double)((const float*)trow)[d];
-        // lp = z_t[d] - logZ_t = ((x - m) * invT) - ln(s)
-        double lr = (xt - (double)lt.m) * (double)inv_t - log(lt.s);
-        if (q_mode == DFLASH2_Q_SOFTMAX) {
-            const char* qrow = (const char*)draft + ((int64_t)b * G + lane) * V * ES;
-            const double xq = BF16
-                ? (double)__uint_as_float((uint32_t)((const uint16_t*)qrow)[d] << 16)
-                : (double)((const float*)qrow)[d];
-            lr -= (xq - (double)lq.m) * (double)inv_t - log(lq.s);
-        }
+        // lp = z_t[d] - logZ_t = (x - m) * invT - ln(s); likewise lq
+        double lr = (elem(target, (int64_t)b * (G + 1) + lane, d) - (double)lt.m) * (double)inv_t -
+                    log(lt.s);
+        if (q_mode == DFLASH2_Q_SOFTMAX)
+            lr -= (elem(draft, (int64_t)b * G + lane, d) - (double)lq.m) * (double)inv_t - log(lq.s);
         const double ratio = exp(lr);
         const float u = philox_uniform(seed, step, sid, (uint32_t)lane, 0u);
         reject = !((double)u < ratio);
@@ -178,10 +183,7 @@ __global__ void __launch_bounds__(NT) verify_sample_scan_kernel(
     const unsigned rej = __ballot_sync(FULL, reject);
     const int n = rej ? (__ffs(rej) - 1) : G;
     const int32_t dn = (lane < G) ? draft_tok[(int64_t)b * G + lane] : -1;
-    if (lane <= G) {
-        // the drawn token at position n is written by the draw kernel
-        out_tok[(int64_t)b * (G + 1) + lane] = (lane < n) ? dn : -1;
-    }
+    if (lane <= G) out_tok[(int64_t)b * (G + 1) + lane] = (lane < n) ? dn : -1;  // draw fills n
     const float ltm = __shfl_sync(FULL, lt.m, n);
     const double lts = __shfl_sync(FULL, lt.s, n);
     const float lqm = __shfl_sync(FULL, lq.m, n);
@@ -189,53 +191,132 @@ __global__ void __launch_bounds__(NT) verify_sample_scan_kernel(
     const int32_t d_n = __shfl_sync(FULL, dn, n);
     if (lane == 0) {
         SampleInfo I;
+        const bool resid = n < G && q_mode == DFLASH2_Q_SOFTMAX;
         I.mt = ltm;
         I.l2t = (float)log2(lts);
         I.mq = lqm;
-        const bool resid = n < G && q_mode == DFLASH2_Q_SOFTMAX;
         I.l2q = resid ? (float)log2(lqs) : 0.0f;
         I.dl = resid ? (float)(((double)ltm - (double)lqm) * (double)inv_t + log(lts) - log(lqs))
                      : 0.0f;
-        I.pad = 0;
         I.u_res = philox_uniform(seed, step, sid, (uint32_t)n, 1u);
         I.n = n;
         I.mode = (n == G) ? 2 : (q_mode == DFLASH2_Q_SOFTMAX ? 0 : 1);
         I.d = d_n;
+        I.pad = 0;
         info[b] = I;
         n_accept[b] = n;
     }
 }
 
+template <bool BF16, bool TMA>
+__global__ void __launch_bounds__(NT, 3) verify_sample_scan_kernel(
+    const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int S,
+    int rows_per_seq, int64_t units, float inv_t, float c2, const int32_t* __restrict__ draft_tok,
+    uint64_t seed, uint32_t step, const uint32_t* __restrict__ seq_id, int q_mode,
+    int32_t* __restrict__ n_accept, int32_t* __restrict__ out_tok, float* __restrict__ ratio_dbg,
+    float* __restrict__ u_dbg, LseD* __restrict__ part, SampleInfo* __restrict__ info,
+    unsigned* __restrict__ counters) {
+    constexpr int ES = BF16 ? 2 : 4;
+    constexpr int SLOT = CHUNK * ES;
+    extern __shared__ __align__(128) uint8_t ring[];
+    __shared__ LseD s_lse[NT / 32];
+    __shared__ __align__(8) uint64_t s_bar[2];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const uint32_t bar0 = smem_u32(&s_bar[0]);
+    const int per_seq = rows_per_seq * S;
+    auto geom = [&](int64_t u, int& b, int& rr, const char*& rowp, int64_t& v0, int64_t& vend) {
+        b = (int)(u / per_seq);
+        const int rem = (int)(u - (int64_t)b * per_seq);
+        rr = rem / S;
+        rowp = (rr <= G) ? (const char*)target + ((int64_t)b * (G + 1) + rr) * V * ES
+                         : (const char*)draft + ((int64_t)b * G + (rr - G - 1)) * V * ES;
+        v0 = (int64_t)(rem - rr * S) * CHUNK;
+        vend = min(V, v0 + (int64_t)CHUNK);
+    };
+    auto issue = [&](int64_t u, int slot) {
+        int b, rr;
+        const char* rowp;
+        int64_t v0, vend;
+        geom(u, b, rr, rowp, v0, vend);
+        bulk_g2s(smem_u32(ring + slot * SLOT), rowp + v0 * ES, (uint32_t)((vend - v0) * ES),
+                 bar0 + 8 * slot);
+    };
+    if (TMA) {
+        if (t == 0) {
+            mbar_init(bar0, 1);
+            mbar_init(bar0 + 8, 1);
+            mbar_fence_init();
+            if ((int64_t)blockIdx.x < units) issue(blockIdx.x, 0);
+        }
+        __syncthreads();
+    }
+    int k = 0;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++k) {
+        int b, rr;
+        const char* rowp;
+        int64_t v0, vend;
+        geom(u, b, rr, rowp, v0, vend);
+        LseD mine;
+        if (TMA) {
+            const int64_t un = u + gridDim.x;
+            if (t == 0 && un < units) issue(un, (k + 1) & 1);
+            if (!__syncthreads_and(mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1))) {
+                if (t == 0) {
+                    atomicOr(&g_dev_err, ERR_STREAM);
+                    if (un < units) mbar_wait(bar0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
+                }
+                return;
+            }
+            mine = view_lse_d<BF16>(SmemChunk<BF16>{ring + (k & 1) * SLOT, v0, vend}, c2);
+        } else {
+            RegChunk<BF16> ch;
+            ch.load(rowp, v0, vend);
+            mine = view_lse_d<BF16>(ch, c2);
+        }
+        const LseD wl = warp_lse(mine, c2);
+        if (lane == 0) s_lse[warp] = wl;
+        __syncthreads();
+        if (t == 0) {
+            LseD tot = s_lse[0];
+            for (int w = 1; w < NT / 32; ++w) tot = lse_merge(tot, s_lse[w], c2);
+            part[((int64_t)b * rows_per_seq + rr) * S + v0 / CHUNK] = tot;
+            __threadfence();
+        }
+        const bool last = arrive_last(&counters[b], (unsigned)per_seq);
+        if (last && warp == 0)
+            sample_finish(target, draft, part + (int64_t)b * rows_per_seq * S, G, V, S, ES, inv_t, c2,
+                          draft_tok, seed, step, seq_id ? seq_id[b] : (uint32_t)b, q_mode, b,
+                          n_accept, out_tok, ratio_dbg, u_dbg, info);
+        __syncthreads();
+    }
+}
+
 // ------------------------------------------------------------------ sampling, pass 2
-// The draw weights of element v of the row the sequence draws from:
+// Draw weight of one element of the row the sequence draws from:
 //   p_v = exp2((x_v - mt) * c - l2t),  q_v likewise,
 //   mode 0: w = max(0, p - q), evaluated as q * expm1(ln p - ln q) with
 //           ln p - ln q = (xt - xq) * invT - (logZ_t - logZ_q): the same
 //           value, without the cancellation of p - q when p and q agree;
 //   mode 1: w = p, 0 at d;  mode 2: w = p.
-// The fallback weight (R = 0) is p.
+// With use_p (the residual was empty by rounding) the weight is p.
 template <bool BF16>
-__device__ __forceinline__ void draw_weight(const uint4& rt, const uint4& rq, int e, int64_t v,
-                                            const SampleInfo& I, float c, float inv_t, float& w,
-                                            float& p) {
+__device__ __forceinline__ float draw_weight(const uint4& rt, const uint4& rq, int e, int64_t v,
+                                             const SampleInfo& I, float c, float inv_t,
+                                             bool use_p) {
     using R = Row<BF16>;
     const float xt = R::elem(rt, e);
-    p = ex2((xt - I.mt) * c - I.l2t);
-    if (I.mode == 0) {
+    if (I.mode == 0 && !use_p) {
         const float xq = R::elem(rq, e);
-        const float q = ex2((xq - I.mq) * c - I.l2q);
         const float dlog = (xt - xq) * inv_t - I.dl;
-        w = dlog > 0.0f ? q * expm1f(dlog) : 0.0f;
-    } else if (I.mode == 1) {
-        w = (v == I.d) ? 0.0f : p;
-    } else {
-        w = p;
+        if (!(dlog > 0.0f)) return 0.0f;
+        return ex2((xq - I.mq) * c - I.l2q) * expm1f(dlog);
     }
+    if (I.mode == 1 && !use_p && v == I.d) return 0.0f;
+    return ex2((xt - I.mt) * c - I.l2t);
 }
 
-// Per-thread contiguous block of the chunk: thread t owns elements
-// [v0 + t * 64, v0 + t * 64 + 64) as NV vectors, so a thread's running sum
-// follows index order (needed by the inverse-CDF scan).
+// Thread t's contiguous 64 elements [v0 + 64 t, v0 + 64 t + 64) of a chunk:
+// a thread's running sum follows index order (the inverse-CDF scan needs it).
 template <bool BF16, bool VEC>
 __device__ __forceinline__ void load_contig(const void* row, int64_t v0, int64_t vend,
                                             uint4 (&r)[Row<BF16>::NV]) {
@@ -251,7 +332,7 @@ __device__ __forceinline__ void load_contig(const void* row, int64_t v0, int64_t
 #pragma unroll
             for (int e = 0; e < R::VW; ++e)
                 if (vb + e < vend) {
-                    uint32_t bits = R::scalar_bits(row, vb + e);
+                    const uint32_t bits = R::scalar_bits(row, vb + e);
                     if (BF16) {
                         uint32_t& word = w[e >> 1];
                         word = (e & 1) ? ((word & 0x0000FFFFu) | (bits << 16))
@@ -265,159 +346,171 @@ __device__ __forceinline__ void load_contig(const void* row, int64_t v0, int64_t
     }
 }
 
+// Sum of the draw weights of this thread's 64 elements (fp32 per vector,
+// fp64 across vectors).
 template <bool BF16, bool VEC>
-__global__ void __launch_bounds__(NT) verify_sample_draw_kernel(
+__device__ __forceinline__ double thread_weight_sum(const char* trow, const char* qrow, int64_t v0,
+                                                    int64_t vend, const SampleInfo& I, float c2,
+                                                    float inv_t, bool use_p) {
+    using R = Row<BF16>;
+    uint4 rt[R::NV], rq[R::NV];
+    load_contig<BF16, VEC>(trow, v0, vend, rt);
+    if (I.mode == 0 && !use_p) load_contig<BF16, VEC>(qrow, v0, vend, rq);
+    double s = 0.0;
+    const int64_t vb = v0 + (int64_t)threadIdx.x * EPT;
+#pragma unroll
+    for (int i = 0; i < R::NV; ++i) {
+        float sv = 0.0f;
+#pragma unroll
+        for (int e = 0; e < R::VW; ++e)
+            sv += draw_weight<BF16>(rt[i], rq[i], e, vb + i * R::VW + e, I, c2, inv_t, use_p);
+        s += (double)sv;
+    }
+    return s;
+}
+
+// Block sum in a fixed order (warp butterflies, then the warps in order).
+__device__ __forceinline__ double block_sum(double v, double* s_warp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int k = 16; k > 0; k >>= 1) v += __shfl_xor_sync(FULL, v, k);
+    __syncthreads();
+    if (lane == 0) s_warp[warp] = v;
+    __syncthreads();
+    double tot = 0.0;
+    for (int w = 0; w < NT / 32; ++w) tot += s_warp[w];
+    return tot;
+}
+
+template <bool BF16, bool VEC>
+__global__ void __launch_bounds__(NT, 2) verify_sample_draw_kernel(
     const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int S,
     float c2, float inv_t, const SampleInfo* __restrict__ info, double* __restrict__ part2,
     unsigned* __restrict__ counters2, int32_t* __restrict__ out_tok) {
-    using R = Row<BF16>;
     constexpr int ES = BF16 ? 2 : 4;
-    __shared__ double s_w[NT / 32], s_p[NT / 32];
+    using R = Row<BF16>;
+    __shared__ double s_warp[NT / 32];
     __shared__ double s_scan[NT];
-    __shared__ int s_pick_thread;
-    __shared__ int s_cstar;
     __shared__ double s_base, s_t;
-    __shared__ int s_fallback, s_done, s_last;
+    __shared__ int s_cstar, s_fallback, s_pick_thread, s_done, s_last;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int b = blockIdx.x / S, chunk = blockIdx.x - b * S;
     const SampleInfo I = info[b];
     const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
     const char* qrow = (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
+    double* P2 = part2 + (int64_t)b * S;
 
-    // chunk sums of w (and of p, for the fallback), fp64, thread order
-    uint4 rt[R::NV], rq[R::NV];
-#pragma unroll
-    for (int i = 0; i < R::NV; ++i) rq[i] = make_uint4(0, 0, 0, 0);
-    double sw = 0.0, sp = 0.0;
     {
         const int64_t v0 = (int64_t)chunk * CHUNK, vend = min(V, v0 + (int64_t)CHUNK);
-        load_contig<BF16, VEC>(trow, v0, vend, rt);
-        if (I.mode == 0) load_contig<BF16, VEC>(qrow, v0, vend, rq);
-#pragma unroll
-        for (int i = 0; i < R::NV; ++i)
-#pragma unroll
-            for (int e = 0; e < R::VW; ++e) {
-                float w, p;
-                draw_weight<BF16>(rt[i], rq[i], e, v0 + (int64_t)t * EPT + i * R::VW + e, I, c2, inv_t,
-                                  w, p);
-                sw += (double)w;
-                sp += (double)p;
-            }
-    }
-    double a = sw, bsum = sp;
-#pragma unroll
-    for (int k = 16; k > 0; k >>= 1) {
-        a += __shfl_xor_sync(FULL, a, k);
-        bsum += __shfl_xor_sync(FULL, bsum, k);
-    }
-    if (lane == 0) {
-        s_w[warp] = a;
-        s_p[warp] = bsum;
-    }
-    __syncthreads();
-    if (t == 0) {
-        double W = 0.0, Pp = 0.0;
-        for (int w = 0; w < NT / 32; ++w) {
-            W += s_w[w];
-            Pp += s_p[w];
+        const double W = block_sum(
+            thread_weight_sum<BF16, VEC>(trow, qrow, v0, vend, I, c2, inv_t, false), s_warp);
+        if (t == 0) {
+            P2[chunk] = W;
+            __threadfence();
         }
-        part2[((int64_t)b * S + chunk) * 2 + 0] = W;
-        part2[((int64_t)b * S + chunk) * 2 + 1] = Pp;
-        __threadfence();
     }
     if (!arrive_last(&counters2[b], (unsigned)S)) return;
 
-    // Last chunk of this sequence: total mass, the chunk where the prefix
-    // crosses t, then an in-chunk scan.
+    // ---- last chunk of this sequence: total mass, crossing chunk, in-chunk scan
     if (t == 0) {
-        const double* P2 = part2 + (int64_t)b * S * 2;
-        double R_ = 0.0;
-        for (int c = 0; c < S; ++c) R_ += __ldcg(&P2[c * 2]);
-        int fb = 0;
-        if (!(R_ > 0.0)) {  // residual empty by rounding: draw from p instead
-            fb = 1;
-            R_ = 0.0;
-            for (int c = 0; c < S; ++c) R_ += __ldcg(&P2[c * 2 + 1]);
+        double Rm = 0.0;
+        for (int c = 0; c < S; ++c) Rm += __ldcg(&P2[c]);
+        s_fallback = !(Rm > 0.0);
+    }
+    __syncthreads();
+    const bool use_p = s_fallback != 0;
+    if (use_p) {  // residual empty by rounding: draw from p_n instead (rare)
+        for (int c = 0; c < S; ++c) {
+            const int64_t v0 = (int64_t)c * CHUNK, vend = min(V, v0 + (int64_t)CHUNK);
+            const double W = block_sum(
+                thread_weight_sum<BF16, VEC>(trow, qrow, v0, vend, I, c2, inv_t, true), s_warp);
+            if (t == 0) P2[c] = W;
         }
-        const double tt = (double)I.u_res * R_;
+        __syncthreads();
+    }
+    if (t == 0) {
+        double Rm = 0.0;
+        for (int c = 0; c < S; ++c) Rm += __ldcg(&P2[c]);
+        const double tt = (double)I.u_res * Rm;
         double pre = 0.0;
         int cstar = -1, clast = 0;
         for (int c = 0; c < S; ++c) {
-            const double wc = __ldcg(&P2[c * 2 + fb]);
+            const double wc = __ldcg(&P2[c]);
             if (wc > 0.0) clast = c;
             if (cstar < 0 && pre + wc > tt) cstar = c;
             if (cstar < 0) pre += wc;
         }
-        if (cstar < 0) {  // rounding left t at the top: last chunk with mass
+        if (cstar < 0) {  // rounding left t at the top: the last chunk with mass
             cstar = clast;
             pre = 0.0;
-            for (int c = 0; c < clast; ++c) pre += __ldcg(&P2[c * 2 + fb]);
+            for (int c = 0; c < clast; ++c) pre += __ldcg(&P2[c]);
         }
         s_cstar = cstar;
         s_base = pre;
         s_t = tt;
-        s_fallback = fb;
         s_pick_thread = NT;
         s_done = 0;
         s_last = -1;
     }
     __syncthreads();
-    const int cstar = s_cstar;
-    const int fb = s_fallback;
+    const int64_t v0 = (int64_t)s_cstar * CHUNK, vend = min(V, v0 + (int64_t)CHUNK);
     const double tt = s_t;
-    const int64_t v0 = (int64_t)cstar * CHUNK, vend = min(V, v0 + (int64_t)CHUNK);
-    load_contig<BF16, VEC>(trow, v0, vend, rt);
-    if (I.mode == 0) load_contig<BF16, VEC>(qrow, v0, vend, rq);
-    float wreg[EPT];
-    double mysum = 0.0;
-#pragma unroll
-    for (int i = 0; i < R::NV; ++i)
-#pragma unroll
-        for (int e = 0; e < R::VW; ++e) {
-            float w, p;
-            draw_weight<BF16>(rt[i], rq[i], e, v0 + (int64_t)t * EPT + i * R::VW + e, I, c2, inv_t, w,
-                              p);
-            wreg[i * R::VW + e] = fb ? p : w;
-            mysum += (double)wreg[i * R::VW + e];
-        }
+    const double mysum = thread_weight_sum<BF16, VEC>(trow, qrow, v0, vend, I, c2, inv_t, use_p);
     // inclusive scan of the thread sums in thread (= index) order
-    s_scan[t] = mysum;
-    __syncthreads();
-    for (int off = 1; off < NT; off <<= 1) {
-        double v = (t >= off) ? s_scan[t - off] : 0.0;
-        __syncthreads();
-        s_scan[t] += v;
-        __syncthreads();
+    double incl = mysum;
+#pragma unroll
+    for (int k = 1; k < 32; k <<= 1) {
+        const double o = __shfl_up_sync(FULL, incl, k);
+        if (lane >= k) incl += o;
     }
-    const double incl = s_base + s_scan[t];
-    if (incl > tt) atomicMin(&s_pick_thread, t);
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    double wbase = 0.0;
+    for (int w = 0; w < warp; ++w) wbase += s_warp[w];
+    incl += wbase;
+    s_scan[t] = incl;
+    if (s_base + incl > tt) atomicMin(&s_pick_thread, t);
     __syncthreads();
     const int pt = s_pick_thread;
     if (pt < NT && t == pt) {
+        uint4 rt[R::NV], rq[R::NV];
+        load_contig<BF16, VEC>(trow, v0, vend, rt);
+        if (I.mode == 0 && !use_p) load_contig<BF16, VEC>(qrow, v0, vend, rq);
         double acc = s_base + (t > 0 ? s_scan[t - 1] : 0.0);
         int pick = -1, lastpos = -1;
-        for (int k = 0; k < EPT; ++k) {
-            const float w = wreg[k];
-            if (w > 0.0f) lastpos = k;
-            acc += (double)w;
-            if (acc > tt) {
-                pick = k;
-                break;
+        const int64_t vb = v0 + (int64_t)t * EPT;
+        for (int i = 0; i < R::NV && pick < 0; ++i)
+            for (int e = 0; e < R::VW; ++e) {
+                const float w =
+                    draw_weight<BF16>(rt[i], rq[i], e, vb + i * R::VW + e, I, c2, inv_t, use_p);
+                if (w > 0.0f) lastpos = i * R::VW + e;
+                acc += (double)w;
+                if (acc > tt) {
+                    pick = i * R::VW + e;
+                    break;
+                }
             }
-        }
         if (pick < 0) pick = lastpos;  // rounding: the last element with mass
         if (pick >= 0) {
-            out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(v0 + (int64_t)t * EPT + pick);
+            out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(vb + pick);
             s_done = 1;
         }
     }
     __syncthreads();
     if (!s_done) {  // block-uniform: rounding left t above the chunk's scan
-        for (int k = EPT - 1; k >= 0; --k)
-            if (wreg[k] > 0.0f) {
-                atomicMax(&s_last, t * EPT + k);
-                break;
-            }
+        if (mysum > 0.0) {
+            uint4 rt[R::NV], rq[R::NV];
+            load_contig<BF16, VEC>(trow, v0, vend, rt);
+            if (I.mode == 0 && !use_p) load_contig<BF16, VEC>(qrow, v0, vend, rq);
+            int lastpos = -1;
+            const int64_t vb = v0 + (int64_t)t * EPT;
+            for (int i = 0; i < R::NV; ++i)
+                for (int e = 0; e < R::VW; ++e)
+                    if (draw_weight<BF16>(rt[i], rq[i], e, vb + i * R::VW + e, I, c2, inv_t, use_p) >
+                        0.0f)
+                        lastpos = i * R::VW + e;
+            if (lastpos >= 0) atomicMax(&s_last, t * EPT + lastpos);
+        }
         __syncthreads();
         if (t == 0 && s_last >= 0) out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(v0 + s_last);
     }
@@ -427,6 +520,24 @@ __global__ void __launch_bounds__(NT) verify_sample_draw_kernel(
 
 using namespace dfl;
 using namespace dfl_host;
+
+unsigned dfl_errors_verify(int clear) {
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_dev_err, sizeof v) != cudaSuccess) return 0xFFFFFFFFu;
+    if (clear && v) {
+        unsigned z = 0;
+        cudaMemcpyToSymbol(g_dev_err, &z, sizeof z);
+    }
+    return v;
+}
+
+template <class Kern>
+static int prep_stream_kernel(Kern kern, size_t dyn) {
+    if (dyn > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess)
+        return DFLASH2_ECUDA;
+    return DFLASH2_OK;
+}
 
 extern "C" int dflash2_verify_greedy(const void* target, int dtype, int B, int G, int64_t V,
                                      const int32_t* draft_tok, int32_t* n_accept, int32_t* out_tok,
@@ -440,23 +551,30 @@ extern "C" int dflash2_verify_greedy(const void* target, int dtype, int B, int G
         !aligned(out_tok, 4))
         return DFLASH2_EALIGN;
     const int64_t S = n_chunks(V);
-    if ((int64_t)B * (G + 1) * S > (int64_t)INT32_MAX) return DFLASH2_ESHAPE;
+    const int64_t units = (int64_t)B * (G + 1) * S;
+    if (units > (int64_t)INT32_MAX) return DFLASH2_ESHAPE;
     const Layout L = greedy_layout(B, G, V);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return DFLASH2_EWORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     unsigned* counters = (unsigned*)((char*)ws + L.counters_off);
     uint64_t* part = (uint64_t*)((char*)ws + L.part_off);
     if (cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
-    const bool vec = aligned(target, 16) && (V * es) % 16 == 0;
-    const dim3 grid((unsigned)((int64_t)B * (G + 1) * S)), block(NT);
-#define DFL_GREEDY(BF, VE)                                                                      \
-    verify_greedy_kernel<BF, VE><<<grid, block, 0, s>>>(target, G, V, (int)S, draft_tok, n_accept, \
-                                                        out_tok, part, counters)
+    // TMA bulk copies need 16-byte aligned chunk starts and 16-byte multiples
+    const bool tma = aligned(target, 16) && (V * es) % 16 == 0;
+#define DFL_GREEDY(BF, TM)                                                                      \
+    do {                                                                                        \
+        auto kern = verify_greedy_kernel<BF, TM>;                                               \
+        const size_t dyn = TM ? 2 * (size_t)CHUNK * (BF ? 2 : 4) : 0;                           \
+        if (prep_stream_kernel(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;                  \
+        kern<<<persistent_grid(kern, NT, dyn, units), NT, dyn, s>>>(target, G, V, (int)S, units, \
+                                                                  draft_tok, n_accept, out_tok, \
+                                                                  part, counters);              \
+    } while (0)
     if (dtype == DFLASH2_BF16) {
-        if (vec) DFL_GREEDY(true, true);
+        if (tma) DFL_GREEDY(true, true);
         else DFL_GREEDY(true, false);
     } else {
-        if (vec) DFL_GREEDY(false, true);
+        if (tma) DFL_GREEDY(false, true);
         else DFL_GREEDY(false, false);
     }
 #undef DFL_GREEDY
@@ -483,7 +601,8 @@ extern "C" int dflash2_verify_sample(const void* target, const void* draft, int 
         return DFLASH2_EALIGN;
     const int64_t S = n_chunks(V);
     const int rows_per_seq = (q_mode == DFLASH2_Q_SOFTMAX) ? 2 * G + 1 : G + 1;
-    if ((int64_t)B * rows_per_seq * S > (int64_t)INT32_MAX) return DFLASH2_ESHAPE;
+    const int64_t units = (int64_t)B * rows_per_seq * S;
+    if (units > (int64_t)INT32_MAX) return DFLASH2_ESHAPE;
     const Layout L = sample_layout(B, G, V);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return DFLASH2_EWORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
@@ -492,25 +611,27 @@ extern "C" int dflash2_verify_sample(const void* target, const void* draft, int 
     double* part2 = (double*)((char*)ws + L.part2_off);
     SampleInfo* info = (SampleInfo*)((char*)ws + L.info_off);
     if (cudaMemsetAsync(counters, 0, (size_t)B * 2 * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
-    const bool vec = aligned(target, 16) && (!draft || aligned(draft, 16)) && (V * es) % 16 == 0;
-    const float c2 = (float)((double)inv_temperature * LOG2E);
     const void* q = (q_mode == DFLASH2_Q_SOFTMAX) ? draft : nullptr;
-    const dim3 grid1((unsigned)((int64_t)B * rows_per_seq * S)), grid2((unsigned)((int64_t)B * S));
-    const dim3 block(NT);
-#define DFL_SAMPLE(BF, VE)                                                                          \
-    do {                                                                                            \
-        verify_sample_scan_kernel<BF, VE><<<grid1, block, 0, s>>>(                                  \
-            target, q, G, V, (int)S, rows_per_seq, inv_temperature, c2, draft_tok, seed, step,       \
-            seq_id, q_mode, n_accept, out_tok, ratio_dbg, u_dbg, part, info, counters);             \
-        verify_sample_draw_kernel<BF, VE><<<grid2, block, 0, s>>>(target, q, G, V, (int)S, c2,     \
-                                                                  inv_temperature, info,        \
-                                                                  part2, counters + B, out_tok);    \
+    const bool tma = aligned(target, 16) && (!q || aligned(q, 16)) && (V * es) % 16 == 0;
+    const float c2 = (float)((double)inv_temperature * LOG2E);
+    const dim3 grid2((unsigned)((int64_t)B * S));
+#define DFL_SAMPLE(BF, TM)                                                                        \
+    do {                                                                                          \
+        auto kern = verify_sample_scan_kernel<BF, TM>;                                            \
+        const size_t dyn = TM ? 2 * (size_t)CHUNK * (BF ? 2 : 4) : 0;                             \
+        if (prep_stream_kernel(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;                    \
+        kern<<<persistent_grid(kern, NT, dyn, units), NT, dyn, s>>>(                              \
+            target, q, G, V, (int)S, rows_per_seq, units, inv_temperature, c2, draft_tok, seed,   \
+            step, seq_id, q_mode, n_accept, out_tok, ratio_dbg, u_dbg, part, info, counters);     \
+        verify_sample_draw_kernel<BF, TM><<<grid2, NT, 0, s>>>(target, q, G, V, (int)S, c2,        \
+                                                               inv_temperature, info, part2,      \
+                                                               counters + B, out_tok);            \
     } while (0)
     if (dtype == DFLASH2_BF16) {
-        if (vec) DFL_SAMPLE(true, true);
+        if (tma) DFL_SAMPLE(true, true);
         else DFL_SAMPLE(true, false);
     } else {
-        if (vec) DFL_SAMPLE(false, true);
+        if (tma) DFL_SAMPLE(false, true);
         else DFL_SAMPLE(false, false);
     }
 #undef DFL_SAMPLE
