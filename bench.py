@@ -14,8 +14,9 @@ One step = the whole path over one batch, each call through the C ABI:
   dflash2_dynconv2.
 value = steps per second over all ranks (each rank runs its own batch:
 weak scaling, no collective on the data path).  L2 (126 MB) is flushed by a
-256 MB write before every call; each call is timed with CUDA events on the
-launching stream and the flushes are outside the timed intervals.
+256 MB write followed by a read of the same buffer (no dirty lines left)
+before every call; each call is timed with CUDA events on the launching
+stream and the flushes are outside the timed intervals.
 
 --impl reference times the CPU oracle (the plain fp64 restatement the tests
 check against) on the same workload, metric and unit, one sequence of the
@@ -236,6 +237,7 @@ def run_ours(args, rank, world, local_rank):
         conv=torch.empty((B, w.T, w.H), dtype=torch.bfloat16, device=dev),
     )
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_sink = torch.zeros((), dtype=torch.int64, device=dev)
     names = ["topk_softmax", "pair_select", "verify_sample", "verify_greedy", "dynconv2"]
     kernels_per_step = {"topk_softmax": 1, "pair_select": 1, "verify_sample": 2,
                         "verify_greedy": 1, "dynconv2": 1}
@@ -260,7 +262,11 @@ def run_ours(args, rank, world, local_rank):
             inp = inputs[(step0 + s) % 2]
             row = []
             for fn in calls(inp, step0 + s):
+                # L2 flush: write a buffer twice the size of L2, then read it,
+                # so the timed call starts with no data of its own in L2 and
+                # no dirty lines left to write back
                 flush.fill_(s & 0xFF)
+                flush_sink.add_(flush.view(torch.int64).sum())
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
@@ -382,7 +388,7 @@ def run_ours(args, rank, world, local_rank):
                                "sampling at T=1.0 and greedy verify, dynconv H=5120 over 32x8 "
                                "tokens; one step = all five calls",
                    "global_batch": B * world, "parallelism": "dp%d (independent batches)" % world,
-                   "l2": "256 MB flush before every call, outside the timed intervals",
+                   "l2": "256 MB write + read flush before every call, outside the timed intervals",
                    "step_hbm_GBps": round(step_gbs, 1),
                    "step_frac_of_hbm_peak": round(step_gbs / peak, 4),
                    "sampling_cycle_per_s": round(1e6 / sample_cycle_us, 1),

@@ -33,10 +33,15 @@ extern "C" size_t dflash2_workspace_bytes(int B, int G, int64_t V) {
 unsigned dfl_errors_topk(int clear);
 unsigned dfl_errors_verify(int clear);
 unsigned dfl_errors_dynconv(int clear);
+unsigned dfl_errors_select(int clear);
 
 extern "C" unsigned dflash2_device_errors(int clear) {
-    const unsigned a = dfl_errors_topk(clear), b = dfl_errors_verify(clear),
-                   c = dfl_errors_dynconv(clear);
-    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu) return 0xFFFFFFFFu;
-    return a | b | c;
+    const unsigned f[4] = {dfl_errors_topk(clear), dfl_errors_verify(clear),
+                           dfl_errors_dynconv(clear), dfl_errors_select(clear)};
+    unsigned v = 0;
+    for (unsigned x : f) {
+        if (x == 0xFFFFFFFFu) return 0xFFFFFFFFu;
+        v |= x;
+    }
+    return v;
 }

@@ -152,9 +152,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
             const uint32_t a = smem_u32(base + s * stage_bytes);
             const uint32_t b = a + TC_A_BYTES;
             mbar_expect_tx(full0 + 8 * s, tx);
-            tma_load_2d(a, &map_w, kb * TC_BK, h0, full0 + 8 * s);
-            tma_load_2d(a + TC_A_BYTES / 2, &map_w, kb * TC_BK, sh.H + h0, full0 + 8 * s);
-            tma_load_2d(b, &map_x, kb * TC_BK, tok0, full0 + 8 * s);
+            // each CTA starts its K walk at its own offset, so the CTAs do
+            // not all request the same token tile from L2 at the same time
+            const int kp = (kb + blockIdx.x * 7) % sh.nkb;
+            tma_load_2d(a, &map_w, kp * TC_BK, h0, full0 + 8 * s);
+            tma_load_2d(a + TC_A_BYTES / 2, &map_w, kp * TC_BK, sh.H + h0, full0 + 8 * s);
+            tma_load_2d(b, &map_x, kp * TC_BK, tok0, full0 + 8 * s);
         }
         // drain: the last loads in flight have landed once their stages are
         // consumed (bounded; only a failed MMA thread leaves them pending)

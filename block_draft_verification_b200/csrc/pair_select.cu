@@ -14,27 +14,31 @@
 // maximised exactly by the max-sum recursion over positions (ties: the smaller
 // rank, at every back-pointer and at the end).
 //
-// One CTA per (sequence, position i): it gathers the left embeddings (the
-// anchor for i = 0, else the 16 candidates of position i-1) and the 16 right
-// ones, forms F = E_left W (fp32, W read once per CTA from L2) and
-// S_i = F E_right^T, and stores S_i in the workspace.  The last CTA of the
+// One CTA per (sequence, position i): one TMA bulk copy brings W (fp32,
+// 64 KB at d = 128) into shared memory while the threads gather the left
+// embeddings (the anchor for i = 0, else the 16 candidates of position i-1)
+// and the 16 right ones; then F = E_left W and S_i = F E_right^T from shared
+// memory, and S_i goes to the workspace.  The last CTA of the
 // sequence (arrival ticket) runs the recursion in one warp, lane k = state k,
 // in fp64, and backtracks.
 #include "common.cuh"
+#include "stream.cuh"
 #include "workspace.cuh"
 
 namespace dfl {
 
 template <bool EMB_BF16, int D>
-__global__ void __launch_bounds__(NT) pair_select_kernel(
+__global__ void __launch_bounds__(NT, 2) pair_select_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ logp,
     const int32_t* __restrict__ anchor, const void* __restrict__ emb, const float* __restrict__ W,
     int G, int32_t* __restrict__ path_tok, int32_t* __restrict__ path_rank,
     float* __restrict__ path_score, float* __restrict__ scores, unsigned* __restrict__ counters) {
     constexpr int LD = D + 1;  // padded rows: conflict-free column walks
+    extern __shared__ __align__(128) float s_w[];  // W [D][D]
     __shared__ float s_left[K][LD], s_right[K][LD], s_f[K][LD];
     __shared__ int32_t s_ltok[K], s_rtok[K];
     __shared__ uint8_t s_back[DFLASH2_MAX_BLOCK][K];
+    __shared__ __align__(8) uint64_t s_bar;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int b = blockIdx.x / G, i = blockIdx.x - b * G;
     const int32_t* cand = idx + (int64_t)b * G * K;
@@ -44,6 +48,12 @@ __global__ void __launch_bounds__(NT) pair_select_kernel(
                  (i == 0 ? 0 : K + (int64_t)K * K * (i - 1));
 
     if (has_left) {
+        const uint32_t bar = smem_u32(&s_bar);
+        if (t == 0) {
+            mbar_init(bar, 1);
+            mbar_fence_init();
+            bulk_g2s(smem_u32(s_w), W, (uint32_t)(D * D * 4), bar);
+        }
         if (t < K) {
             s_rtok[t] = cand[i * K + t];
             if (t < nl) s_ltok[t] = (i == 0) ? anchor[b] : cand[(i - 1) * K + t];
@@ -60,30 +70,37 @@ __global__ void __launch_bounds__(NT) pair_select_kernel(
             s_right[k][j] = ld_emb(s_rtok[k], j);
             if (k < nl) s_left[k][j] = ld_emb(s_ltok[k], j);
         }
-        __syncthreads();
-        // F = E_left W: thread -> column l, a group of left rows
-        constexpr int GROUPS = NT / D;          // 2 for d = 128, 4 for d = 64
-        constexpr int RPG = K / GROUPS;         // rows per group
-        const int l = t % D, g = t / D;
-        float acc[RPG];
+        const bool ok = __syncthreads_and(mbar_wait(bar, 0));
+        if (!ok) {  // W never arrived: flag it, leave this position's scores unset
+            if (t == 0) atomicOr(&g_dev_err, ERR_STREAM);
+        } else {
+            // F = E_left W: thread -> column l, a group of left rows
+            constexpr int GROUPS = NT / D;  // 2 for d = 128, 4 for d = 64
+            constexpr int RPG = K / GROUPS;  // rows per group
+            const int l = t % D, g = t / D;
+            float acc[RPG];
 #pragma unroll
-        for (int q = 0; q < RPG; ++q) acc[q] = 0.0f;
-        for (int j = 0; j < D; ++j) {
-            const float w = __ldg(&W[j * D + l]);
-#pragma unroll
-            for (int q = 0; q < RPG; ++q) acc[q] = fmaf(s_left[g * RPG + q][j], w, acc[q]);
-        }
-#pragma unroll
-        for (int q = 0; q < RPG; ++q)
-            if (g * RPG + q < nl) s_f[g * RPG + q][l] = acc[q];
-        __syncthreads();
-        // S[k][k'] = F[k] . E_right[k']
-        const int k = t / K, k2 = t % K;
-        if (k < nl) {
-            float s = 0.0f;
+            for (int q = 0; q < RPG; ++q) acc[q] = 0.0f;
+            if (g * RPG < nl) {
 #pragma unroll 8
-            for (int l2 = 0; l2 < D; ++l2) s = fmaf(s_f[k][l2], s_right[k2][l2], s);
-            out[k * K + k2] = s;
+                for (int j = 0; j < D; ++j) {
+                    const float w = s_w[j * D + l];
+#pragma unroll
+                    for (int q = 0; q < RPG; ++q) acc[q] = fmaf(s_left[g * RPG + q][j], w, acc[q]);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < RPG; ++q)
+                if (g * RPG + q < nl) s_f[g * RPG + q][l] = acc[q];
+            __syncthreads();
+            // S[k][k'] = F[k] . E_right[k']
+            const int k = t / K, k2 = t % K;
+            if (k < nl) {
+                float sc = 0.0f;
+#pragma unroll 8
+                for (int l2 = 0; l2 < D; ++l2) sc = fmaf(s_f[k][l2], s_right[k2][l2], sc);
+                out[k * K + k2] = sc;
+            }
         }
     } else if (t < K) {
         out[t] = 0.0f;  // no anchor: no term before position 0
@@ -143,6 +160,16 @@ __global__ void __launch_bounds__(NT) pair_select_kernel(
 using namespace dfl;
 using namespace dfl_host;
 
+unsigned dfl_errors_select(int clear) {
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_dev_err, sizeof v) != cudaSuccess) return 0xFFFFFFFFu;
+    if (clear && v) {
+        unsigned z = 0;
+        cudaMemcpyToSymbol(g_dev_err, &z, sizeof z);
+    }
+    return v;
+}
+
 extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const int32_t* anchor,
                                    const void* emb, int emb_dtype, int64_t V, int d,
                                    const float* W, int B, int G, int32_t* path_tok,
@@ -155,7 +182,7 @@ extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const 
     if (!idx || !logp || !emb || !W || !path_tok || !path_rank || !path_score)
         return DFLASH2_EINVAL;
     if (!aligned(idx, 4) || !aligned(logp, 4) || (anchor && !aligned(anchor, 4)) ||
-        !aligned(emb, elem_size(emb_dtype)) || !aligned(W, 4) || !aligned(path_tok, 4) ||
+        !aligned(emb, elem_size(emb_dtype)) || !aligned(W, 16) || !aligned(path_tok, 4) ||
         !aligned(path_rank, 4) || !aligned(path_score, 4))
         return DFLASH2_EALIGN;
     if ((int64_t)B * G > (int64_t)INT32_MAX) return DFLASH2_ESHAPE;
@@ -166,9 +193,17 @@ extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const 
     float* scores = (float*)((char*)ws + L.part_off);
     if (cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
     const dim3 grid((unsigned)((int64_t)B * G)), block(NT);
-#define DFL_SEL(BF, DD)                                                                      \
-    pair_select_kernel<BF, DD><<<grid, block, 0, s>>>(idx, logp, anchor, emb, W, G, path_tok, \
-                                                      path_rank, path_score, scores, counters)
+#define DFL_SEL(BF, DD)                                                                          \
+    do {                                                                                         \
+        auto kern = pair_select_kernel<BF, DD>;                                                  \
+        const int dyn = DD * DD * 4;                                                             \
+        if (dyn > 48 * 1024 &&                                                                   \
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) !=      \
+                cudaSuccess)                                                                     \
+            return DFLASH2_ECUDA;                                                                \
+        kern<<<grid, block, dyn, s>>>(idx, logp, anchor, emb, W, G, path_tok, path_rank,         \
+                                      path_score, scores, counters);                             \
+    } while (0)
     if (emb_dtype == DFLASH2_BF16) {
         if (d == 128) DFL_SEL(true, 128);
         else DFL_SEL(true, 64);

@@ -187,6 +187,27 @@ __device__ __forceinline__ uint32_t view_first(const C& ch, float x) {
     return first;
 }
 
+// Contiguous share [lo, hi) of `units` for this CTA (consecutive units of a
+// row / sequence mostly stay on one CTA, so it publishes them together).
+__device__ __forceinline__ void cta_range(int64_t units, int64_t& lo, int64_t& hi) {
+    lo = units * (int64_t)blockIdx.x / gridDim.x;
+    hi = units * (int64_t)(blockIdx.x + 1) / gridDim.x;
+}
+
+// Publish `count` units of group g whose partials this thread (thread 0) has
+// already stored, with one acquire-release add: the release orders those
+// stores before the count, the acquire lets the last publisher read every
+// other CTA's partials.  Returns true on the publisher that completes the
+// group (expected units in all).
+__device__ __forceinline__ bool publish(unsigned* counter, unsigned count, unsigned expected) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(counter), "r"(count)
+                 : "memory");
+    return old + count == expected;
+}
+
 // Persistent grid size for a kernel: resident CTAs per SM x SMs, at most
 // units.  The occupancy query runs once per (kernel, device, smem) and is
 // cached.

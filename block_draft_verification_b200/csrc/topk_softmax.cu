@@ -7,9 +7,11 @@
 // those 16 per position; "DFlash 2" (myaiexp.com), section "主な機能": the
 // path selector keeps the top-16 candidates of each position.
 //
-// Work unit: (row, 16384-element chunk).  Persistent CTAs stream their units
-// through a two-slot shared-memory ring filled by TMA bulk copies (rows whose
-// start is 16-byte aligned; others are read element by element).  Per unit,
+// Work unit: (row, 16384-element chunk).  Persistent CTAs each stream a
+// contiguous range of units through a two-slot shared-memory ring filled by
+// TMA bulk copies (rows whose start is 16-byte aligned; others are read
+// element by element), publishing a row's finished chunks with one
+// acquire-release add when they leave that row.  Per unit,
 // each thread takes the max and sum-exp of its 64 elements and the block
 // merges them in a fixed order.  The chunk's top-16 is exact without sorting
 // the chunk: the 16th largest per-thread maximum T bounds it, only the (at
@@ -23,7 +25,8 @@
 
 namespace dfl {
 
-struct TopkSmem {
+struct __align__(16) TopkSmem {
+    uint64_t keys[K];
     uint32_t top[NT / 32][K];
     uint64_t cand[K * EPT];
     Lse lse[NT / 32];
@@ -107,12 +110,15 @@ __device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm,
             if (lane >= K) v = (base + lane - K < n) ? sm.cand[base + lane - K] : 0ull;
             acc = warp_sort_desc(v);
         }
-        if (lane < K) part[unit].key[lane] = acc;
-        if (lane == 0) {
-            part[unit].m = sm.chunk.m;
-            part[unit].s = sm.chunk.s;
+        if (lane < K) sm.keys[lane] = acc;
+        __syncwarp();
+        if (lane == 0) {  // thread 0 alone stores the partial (published by its release add)
+            uint4* dst = (uint4*)&part[unit];
+            dst[0] = make_uint4(__float_as_uint(sm.chunk.m), __float_as_uint(sm.chunk.s), 0u, 0u);
+            const uint4* kv = (const uint4*)sm.keys;
+#pragma unroll
+            for (int j = 0; j < K / 2; ++j) dst[1 + j] = kv[j];
         }
-        __threadfence();
     }
 }
 
@@ -172,27 +178,29 @@ __global__ void __launch_bounds__(NT, 3) topk_softmax_kernel(
         const char* src = (const char*)logits + (row * row_stride + v0) * ES;
         bulk_g2s(smem_u32(ring + slot * SLOT), src, (uint32_t)((vend - v0) * ES), bar0 + 8 * slot);
     };
+    int64_t lo, hi;
+    cta_range(units, lo, hi);
     if (TMA) {
         if (t == 0) {
             mbar_init(bar0, 1);
             mbar_init(bar0 + 8, 1);
             mbar_fence_init();
-            if ((int64_t)blockIdx.x < units) issue(blockIdx.x, 0);
+            if (lo < hi) issue(lo, 0);
         }
         __syncthreads();
     }
+    __shared__ bool s_last;
+    unsigned pending = 0;
     int k = 0;
-    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++k) {
+    for (int64_t u = lo; u < hi; ++u, ++k) {
         int64_t row, v0, vend;
         unit_geom(u, row, v0, vend);
         if (TMA) {
-            const int64_t un = u + gridDim.x;
-            if (t == 0 && un < units) issue(un, (k + 1) & 1);
-            const bool ok = __syncthreads_and(mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1));
-            if (!ok) {
+            if (t == 0 && u + 1 < hi) issue(u + 1, (k + 1) & 1);
+            if (!__syncthreads_and(mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1))) {
                 if (t == 0) {
                     atomicOr(&g_dev_err, ERR_STREAM);
-                    if (un < units) mbar_wait(bar0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
+                    if (u + 1 < hi) mbar_wait(bar0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
                 }
                 return;
             }
@@ -203,8 +211,15 @@ __global__ void __launch_bounds__(NT, 3) topk_softmax_kernel(
             ch.load((const char*)logits + row * row_stride * ES, v0, vend);
             topk_unit<BF16>(ch, c2, sm, part, u);
         }
-        const bool last = arrive_last(&counters[row], (unsigned)S);
-        if (last && warp == 0) topk_row_merge(part + row * S, S, row, inv_t, c2, idx, prob, logp, logz);
+        ++pending;
+        if (u + 1 == hi || (u + 1) / S != row) {  // this CTA is done with the row: publish
+            __syncthreads();
+            if (t == 0) s_last = publish(&counters[row], pending, (unsigned)S);
+            __syncthreads();
+            if (s_last && warp == 0)
+                topk_row_merge(part + row * S, S, row, inv_t, c2, idx, prob, logp, logz);
+            pending = 0;
+        }
         __syncthreads();  // ring slot k & 1 is free for the prefetch of iteration k + 1
     }
 }

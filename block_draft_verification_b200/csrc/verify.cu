@@ -11,10 +11,11 @@
 // Uniforms: Philox4x32-10 (Salmon et al., SC'11, section 5).
 //
 // Both verifies stream every logit row once in 16384-element chunks: work
-// unit = (sequence, row, chunk), persistent CTAs, TMA bulk copies into a
-// two-slot shared-memory ring.  The last unit of a sequence to finish
-// (arrival ticket, no waiting) reduces the partials in chunk order and
-// decides.  The sampling draw needs the normalisers first, so it is a second
+// unit = (sequence, row, chunk); persistent CTAs each take a contiguous range
+// of units through a two-slot shared-memory ring filled by TMA bulk copies,
+// and publish a sequence's finished units with one acquire-release add.  The
+// publisher that completes a sequence (no CTA waits) reduces the partials in
+// chunk order and decides.  The sampling draw needs the normalisers first, so it is a second
 // kernel over the one row each sequence draws from (L2-resident after the
 // first pass): one CTA per chunk sums the draw weights, and the last of them
 // finds the chunk where the inverse CDF crosses t = u' * R and scans only that
@@ -48,10 +49,7 @@ __device__ __forceinline__ void greedy_unit(const C& ch, GreedySmem& sm, uint64_
     for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, sm.wmax[w]);
     if (m == M) atomicMin(&sm.first, view_first<BF16>(ch, M));  // -0 == +0
     __syncthreads();
-    if (t == 0) {
-        *slot = make_key(M, sm.first);
-        __threadfence();
-    }
+    if (t == 0) *slot = make_key(M, sm.first);  // published by thread 0's release add
 }
 
 __device__ __forceinline__ void greedy_finish(const uint64_t* P, int S, int G, int b,
@@ -101,28 +99,31 @@ __global__ void __launch_bounds__(NT, 3) verify_greedy_kernel(
         bulk_g2s(smem_u32(ring + slot * SLOT), (const char*)target + (row * V + v0) * ES,
                  (uint32_t)((vend - v0) * ES), bar0 + 8 * slot);
     };
+    int64_t lo, hi;
+    cta_range(units, lo, hi);
     if (TMA) {
         if (t == 0) {
             mbar_init(bar0, 1);
             mbar_init(bar0 + 8, 1);
             mbar_fence_init();
-            if ((int64_t)blockIdx.x < units) issue(blockIdx.x, 0);
+            if (lo < hi) issue(lo, 0);
         }
         __syncthreads();
     }
+    __shared__ bool s_last;
+    unsigned pending = 0;
     int k = 0;
-    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++k) {
+    for (int64_t u = lo; u < hi; ++u, ++k) {
         int b;
         int64_t row, v0, vend;
         geom(u, b, row, v0, vend);
         uint64_t* slot = part + row * S + (v0 / CHUNK);
         if (TMA) {
-            const int64_t un = u + gridDim.x;
-            if (t == 0 && un < units) issue(un, (k + 1) & 1);
+            if (t == 0 && u + 1 < hi) issue(u + 1, (k + 1) & 1);
             if (!__syncthreads_and(mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1))) {
                 if (t == 0) {
                     atomicOr(&g_dev_err, ERR_STREAM);
-                    if (un < units) mbar_wait(bar0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
+                    if (u + 1 < hi) mbar_wait(bar0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
                 }
                 return;
             }
@@ -132,9 +133,15 @@ __global__ void __launch_bounds__(NT, 3) verify_greedy_kernel(
             ch.load((const char*)target + row * V * ES, v0, vend);
             greedy_unit<BF16>(ch, sm, slot);
         }
-        const bool last = arrive_last(&counters[b], (unsigned)per_seq);
-        if (last && warp == 0)
-            greedy_finish(part + (int64_t)b * (G + 1) * S, S, G, b, draft_tok, n_accept, out_tok);
+        ++pending;
+        if (u + 1 == hi || (u + 1) / per_seq != b) {  // done with this sequence: publish
+            __syncthreads();
+            if (t == 0) s_last = publish(&counters[b], pending, (unsigned)per_seq);
+            __syncthreads();
+            if (s_last && warp == 0)
+                greedy_finish(part + (int64_t)b * (G + 1) * S, S, G, b, draft_tok, n_accept, out_tok);
+            pending = 0;
+        }
         __syncthreads();  // ring slot k & 1 is free for the prefetch of iteration k + 1
     }
 }
@@ -241,29 +248,32 @@ __global__ void __launch_bounds__(NT, 3) verify_sample_scan_kernel(
         bulk_g2s(smem_u32(ring + slot * SLOT), rowp + v0 * ES, (uint32_t)((vend - v0) * ES),
                  bar0 + 8 * slot);
     };
+    int64_t lo, hi;
+    cta_range(units, lo, hi);
     if (TMA) {
         if (t == 0) {
             mbar_init(bar0, 1);
             mbar_init(bar0 + 8, 1);
             mbar_fence_init();
-            if ((int64_t)blockIdx.x < units) issue(blockIdx.x, 0);
+            if (lo < hi) issue(lo, 0);
         }
         __syncthreads();
     }
+    __shared__ bool s_last;
+    unsigned pending = 0;
     int k = 0;
-    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++k) {
+    for (int64_t u = lo; u < hi; ++u, ++k) {
         int b, rr;
         const char* rowp;
         int64_t v0, vend;
         geom(u, b, rr, rowp, v0, vend);
         LseD mine;
         if (TMA) {
-            const int64_t un = u + gridDim.x;
-            if (t == 0 && un < units) issue(un, (k + 1) & 1);
+            if (t == 0 && u + 1 < hi) issue(u + 1, (k + 1) & 1);
             if (!__syncthreads_and(mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1))) {
                 if (t == 0) {
                     atomicOr(&g_dev_err, ERR_STREAM);
-                    if (un < units) mbar_wait(bar0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
+                    if (u + 1 < hi) mbar_wait(bar0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
                 }
                 return;
             }
@@ -276,18 +286,22 @@ __global__ void __launch_bounds__(NT, 3) verify_sample_scan_kernel(
         const LseD wl = warp_lse(mine, c2);
         if (lane == 0) s_lse[warp] = wl;
         __syncthreads();
-        if (t == 0) {
+        if (t == 0) {  // thread 0 alone stores the partial (published by its release add)
             LseD tot = s_lse[0];
             for (int w = 1; w < NT / 32; ++w) tot = lse_merge(tot, s_lse[w], c2);
             part[((int64_t)b * rows_per_seq + rr) * S + v0 / CHUNK] = tot;
-            __threadfence();
         }
-        const bool last = arrive_last(&counters[b], (unsigned)per_seq);
-        if (last && warp == 0)
-            sample_finish(target, draft, part + (int64_t)b * rows_per_seq * S, G, V, S, ES, inv_t, c2,
-                          draft_tok, seed, step, seq_id ? seq_id[b] : (uint32_t)b, q_mode, b,
-                          n_accept, out_tok, ratio_dbg, u_dbg, info);
-        __syncthreads();
+        ++pending;
+        if (u + 1 == hi || (u + 1) / per_seq != b) {  // done with this sequence: publish
+            if (t == 0) s_last = publish(&counters[b], pending, (unsigned)per_seq);
+            __syncthreads();
+            if (s_last && warp == 0)
+                sample_finish(target, draft, part + (int64_t)b * rows_per_seq * S, G, V, S, ES, inv_t,
+                              c2, draft_tok, seed, step, seq_id ? seq_id[b] : (uint32_t)b, q_mode, b,
+                              n_accept, out_tok, ratio_dbg, u_dbg, info);
+            pending = 0;
+        }
+        __syncthreads();  // ring slot k & 1 is free; s_lse may be rewritten
     }
 }
 
@@ -472,27 +486,63 @@ __global__ void __launch_bounds__(NT, 2) verify_sample_draw_kernel(
     if (s_base + incl > tt) atomicMin(&s_pick_thread, t);
     __syncthreads();
     const int pt = s_pick_thread;
-    if (pt < NT && t == pt) {
-        uint4 rt[R::NV], rq[R::NV];
-        load_contig<BF16, VEC>(trow, v0, vend, rt);
-        if (I.mode == 0 && !use_p) load_contig<BF16, VEC>(qrow, v0, vend, rq);
-        double acc = s_base + (t > 0 ? s_scan[t - 1] : 0.0);
-        int pick = -1, lastpos = -1;
-        const int64_t vb = v0 + (int64_t)t * EPT;
-        for (int i = 0; i < R::NV && pick < 0; ++i)
-            for (int e = 0; e < R::VW; ++e) {
-                const float w =
-                    draw_weight<BF16>(rt[i], rq[i], e, vb + i * R::VW + e, I, c2, inv_t, use_p);
-                if (w > 0.0f) lastpos = i * R::VW + e;
-                acc += (double)w;
-                if (acc > tt) {
-                    pick = i * R::VW + e;
-                    break;
-                }
+    if (pt < NT && warp == 0) {
+        // warp 0 walks thread pt's 64 elements, two per lane, in index order
+        const int64_t vb = v0 + (int64_t)pt * EPT + 2 * lane;
+        const int i = (2 * lane) / R::VW, e = (2 * lane) % R::VW;
+        uint4 xt = make_uint4(0, 0, 0, 0), xq = make_uint4(0, 0, 0, 0);
+        if (vb < vend) {  // the 16-byte vector holding this lane's pair
+            const int64_t v8 = v0 + (int64_t)pt * EPT + i * R::VW;
+            if (VEC && v8 + R::VW <= vend) {
+                xt = *(const uint4*)(trow + v8 * ES);
+                if (I.mode == 0 && !use_p) xq = *(const uint4*)(qrow + v8 * ES);
+            } else {
+                uint32_t wt[4] = {R::NEG_INF_WORD, R::NEG_INF_WORD, R::NEG_INF_WORD, R::NEG_INF_WORD};
+                uint32_t wq[4] = {R::NEG_INF_WORD, R::NEG_INF_WORD, R::NEG_INF_WORD, R::NEG_INF_WORD};
+                for (int ee = 0; ee < R::VW; ++ee)
+                    if (v8 + ee < vend) {
+                        const uint32_t bt = R::scalar_bits(trow, v8 + ee);
+                        const uint32_t bq = (I.mode == 0 && !use_p) ? R::scalar_bits(qrow, v8 + ee) : 0u;
+                        if (BF16) {
+                            const int sh = (ee & 1) ? 16 : 0;
+                            const uint32_t msk = (ee & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+                            wt[ee >> 1] = (wt[ee >> 1] & msk) | (bt << sh);
+                            wq[ee >> 1] = (wq[ee >> 1] & msk) | (bq << sh);
+                        } else {
+                            wt[ee] = bt;
+                            wq[ee] = bq;
+                        }
+                    }
+                xt = make_uint4(wt[0], wt[1], wt[2], wt[3]);
+                xq = make_uint4(wq[0], wq[1], wq[2], wq[3]);
             }
-        if (pick < 0) pick = lastpos;  // rounding: the last element with mass
-        if (pick >= 0) {
-            out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(vb + pick);
+        }
+        const float w0 = (vb < vend) ? draw_weight<BF16>(xt, xq, e, vb, I, c2, inv_t, use_p) : 0.0f;
+        const float w1 =
+            (vb + 1 < vend) ? draw_weight<BF16>(xt, xq, e + 1, vb + 1, I, c2, inv_t, use_p) : 0.0f;
+        double incl2 = (double)w0 + (double)w1;
+#pragma unroll
+        for (int kk = 1; kk < 32; kk <<= 1) {
+            const double o = __shfl_up_sync(FULL, incl2, kk);
+            if (lane >= kk) incl2 += o;
+        }
+        const double base = s_base + (pt > 0 ? s_scan[pt - 1] : 0.0);
+        const double before = base + incl2 - ((double)w0 + (double)w1);
+        const bool c0 = before + (double)w0 > tt;
+        const bool c1 = before + (double)w0 + (double)w1 > tt;
+        const unsigned m0 = __ballot_sync(FULL, c0), m1 = __ballot_sync(FULL, c1);
+        const unsigned has = __ballot_sync(FULL, w0 > 0.0f || w1 > 0.0f);
+        int pick = -1;
+        if (m0 | m1) {  // the first element whose inclusive prefix exceeds t
+            const int l0 = m0 ? __ffs(m0) - 1 : 32, l1 = m1 ? __ffs(m1) - 1 : 32;
+            pick = (l0 <= l1) ? 2 * l0 : 2 * l1 + 1;
+        } else if (has) {  // rounding: the last element with mass
+            const int ll = 31 - __clz(has);
+            const float lw1 = __shfl_sync(FULL, w1, ll);
+            pick = 2 * ll + (lw1 > 0.0f ? 1 : 0);
+        }
+        if (lane == 0 && pick >= 0) {
+            out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(v0 + (int64_t)pt * EPT + pick);
             s_done = 1;
         }
     }

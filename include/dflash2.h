@@ -134,7 +134,7 @@ DFLASH2_API int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows
  * idx, logp   [B, G, 16] as written by dflash2_topk_softmax (c = idx).
  * anchor      [B] int32 last accepted token per sequence, or NULL (no term).
  * emb         [V, d] of `emb_dtype`; d in {64, 128}.
- * W           [d, d] float, row-major (W[j][l] at j * d + l).
+ * W           [d, d] float, row-major (W[j][l] at j * d + l), 16-byte aligned.
  * B >= 0, 1 <= G < DFLASH2_MAX_BLOCK.
  * path_tok    [B, G] int32 chosen tokens; path_rank [B, G] int32 their ranks;
  * path_score  [B] float score of the chosen path.
@@ -207,12 +207,14 @@ DFLASH2_API int dflash2_dynconv2(const void* x, const void* x_prev, const void* 
                      int T, int H, void* out, dflash2_stream_t stream);
 
 /*
- * Device-side error flags of the tensor-core kernels on the current device
- * (0 = none).  Every wait inside those kernels is bounded; a wait that runs
- * out sets a flag bit (1 producer, 2 MMA issuer, 4 epilogue, 8 drain), the
- * kernel releases its tensor memory and returns, and the call's outputs are
- * not valid.  Synchronous (reads device memory); clear != 0 resets the flags.
- * Returns 0xFFFFFFFF if the flags cannot be read.
+ * Device-side error flags of the kernels on the current device (0 = none).
+ * Every wait inside the kernels (on a TMA copy or a tensor-core MMA) is
+ * bounded to one second; a wait that runs out sets a flag bit (1 producer,
+ * 2 MMA issuer, 4 epilogue, 8 drain, 16 streamed copy), the kernel waits
+ * (bounded) for its own copies in flight, releases its tensor memory and
+ * returns, and the call's outputs are not valid.  Synchronous (reads device
+ * memory); clear != 0 resets the flags.  Returns 0xFFFFFFFF if the flags
+ * cannot be read.
  */
 DFLASH2_API unsigned dflash2_device_errors(int clear);
 
