@@ -56,6 +56,16 @@ __device__ __forceinline__ uint64_t shfl_xor(uint64_t v, int m) {
 __device__ __forceinline__ uint32_t shfl_xor(uint32_t v, int m) {
     return __shfl_xor_sync(FULL, v, m);
 }
+__device__ __forceinline__ uint64_t shfl_up64(uint64_t v) {
+    uint32_t lo = __shfl_up_sync(FULL, (uint32_t)v, 1);
+    uint32_t hi = __shfl_up_sync(FULL, (uint32_t)(v >> 32), 1);
+    return ((uint64_t)hi << 32) | lo;
+}
+__device__ __forceinline__ uint64_t shfl64(uint64_t v, int src) {
+    uint32_t lo = __shfl_sync(FULL, (uint32_t)v, src);
+    uint32_t hi = __shfl_sync(FULL, (uint32_t)(v >> 32), src);
+    return ((uint64_t)hi << 32) | lo;
+}
 
 // Bitonic sort of one key per lane, descending in lane order (KeyT is
 // uint32_t or uint64_t).

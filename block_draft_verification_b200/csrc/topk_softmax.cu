@@ -10,15 +10,18 @@
 // Work unit: (row, 16384-element chunk).  Persistent CTAs each stream a
 // contiguous range of units through a two-slot shared-memory ring filled by
 // TMA bulk copies (rows whose start is 16-byte aligned; others are read
-// element by element), publishing a row's finished chunks with one
-// acquire-release add when they leave that row.  Per unit,
-// each thread takes the max and sum-exp of its 64 elements and the block
-// merges them in a fixed order.  The chunk's top-16 is exact without sorting
-// the chunk: the 16th largest per-thread maximum T bounds it, only the (at
-// most 16) threads holding keys at or above it contribute candidates, and one
-// warp sorts those.  The last unit of a row to finish (arrival ticket, no
-// waiting) merges the row's chunk partials in chunk order and writes
-// idx / prob / logp / logz.
+// element by element).  Softmax: per chunk, the block max, then the sum of
+// exp2((x - M) c) against it, both in a fixed order, so a chunk's partial
+// does not depend on the batch or the grid.  Top-16: every warp keeps a
+// running top-16 of the row segment it streams (the CTA's consecutive chunks
+// of one row); an element is looked at only if its 8-element vector reaches
+// the warp's current 16th value, which after the first few thousand
+// elements almost never happens, and qualifying elements are inserted with a
+// shuffle.  At the end of the segment the 8 warp lists are merged and the
+// segment is published with one acquire-release add.  The publisher that
+// completes a row (no CTA waits) merges the chunk partials in chunk order and
+// the segment lists, and writes idx / prob / logp / logz.  Keys compare
+// (value, -index) exactly, so the top-16 set does not depend on who merged.
 #include "common.cuh"
 #include "stream.cuh"
 #include "workspace.cuh"
@@ -27,99 +30,105 @@ namespace dfl {
 
 struct __align__(16) TopkSmem {
     uint64_t keys[K];
-    uint32_t top[NT / 32][K];
-    uint64_t cand[K * EPT];
-    Lse lse[NT / 32];
-    uint32_t tie[NT];
-    unsigned ncand, ntie;
-    uint32_t thr, vk;
-    Lse chunk;
+    uint64_t wlist[NT / 32][K];
+    float wmax[NT / 32];
+    float wsum[NT / 32];
 };
 
-// One unit: chunk partial (max, sum-exp, top-16 keys) into part[unit].
+// A warp's running top-16 of the current row segment: lanes 0..15 hold keys
+// in descending order (0 = empty), lanes 16..31 hold 0.
+struct WarpTop {
+    uint64_t key;
+    float thr;  // value of the 16th key (-inf while fewer than 16)
+};
+__device__ __forceinline__ void warp_insert(WarpTop& w, uint64_t k) {
+    const int lane = threadIdx.x & 31;
+    const uint64_t up = shfl_up64(w.key);
+    if (lane < K) w.key = (lane > 0 && k > up) ? up : (k > w.key ? k : w.key);
+    const uint64_t last = shfl64(w.key, K - 1);
+    w.thr = last ? key_value(last) : -INFINITY;
+}
+
+// One unit: the chunk's softmax partial (block max, then the sum of
+// exp2((x - M) c) in a fixed order) and the warps' running top-16 updated
+// with the chunk's elements whose value reaches the warp's threshold.
 template <bool BF16, class C>
-__device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm,
-                                          TopkPartial* __restrict__ part, int64_t unit) {
+__device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm, WarpTop& wt,
+                                          float& chunk_m, float& chunk_s) {
     using R = Row<BF16>;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const Lse mine = view_lse<BF16>(ch, c2);
-    if (t == 0) {
-        sm.ncand = 0;
-        sm.ntie = 0;
-    }
-    // (1) chunk softmax partial and (2) the 16th largest thread maximum, T.
-    const Lse wl = warp_lse(mine, c2);
-    if (lane == 0) sm.lse[warp] = wl;
-    const uint32_t my_ord = (mine.m == -INFINITY) ? 0u : ord32(mine.m);
-    const uint32_t srt = warp_sort_desc(my_ord);
-    if (lane < K) sm.top[warp][lane] = srt;
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t acc = (lane < K) ? sm.top[0][lane] : 0u;
-        for (int w = 1; w < NT / 32; ++w) acc = warp_merge_desc(lane < K ? acc : sm.top[w][31 - lane]);
-        if (lane == K - 1) sm.thr = acc;  // 0: fewer than 16 threads hold elements
-        if (lane == 0) {
-            Lse tot = sm.lse[0];
-            for (int w = 1; w < NT / 32; ++w) tot = lse_merge(tot, sm.lse[w], c2);
-            sm.chunk = tot;
-        }
-    }
-    __syncthreads();
-    // (3) Threads that can hold a top-16 element: maximum above T, or equal to
-    // T with a first index among the lowest (16 - #above) of those.
-    const uint32_t thr = sm.thr;
-    const bool above = my_ord > thr;
-    const bool tie = thr != 0u && my_ord == thr;
-    const int n_above = __syncthreads_count(above);
-    uint32_t my_first = 0xFFFFFFFFu;
-    if (tie) {
-        my_first = view_first<BF16>(ch, mine.m);
-        sm.tie[atomicAdd(&sm.ntie, 1u)] = my_first;
-    }
-    __syncthreads();
-    if (tie) {
-        const unsigned n = sm.ntie;
-        unsigned rank = 0;
-        for (unsigned j = 0; j < n; ++j) rank += sm.tie[j] < my_first;
-        if (rank == (unsigned)(K - n_above - 1)) sm.vk = my_first;
-    }
-    __syncthreads();
-    // (4) Candidates: keys at or above (T, vk); at most 16 threads x 64.
-    const float tv = (thr == 0u) ? -INFINITY : unord32(thr);
-    const uint32_t vk = (thr == 0u) ? 0u : sm.vk;
-    if (above || (tie && my_first <= vk)) {
+    // pass 1: thread max and the top-16 filter, vector by vector
+    float m = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < R::NV; ++i) {
-            const uint4 v4 = ch.vec(i);
+    for (int i = 0; i < R::NV; ++i) {
+        const uint4 v4 = ch.vec(i);
+        float vm = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < R::VW; ++e) vm = fmaxf(vm, R::elem(v4, e));
+        m = fmaxf(m, vm);
+        unsigned cand = __ballot_sync(FULL, vm >= wt.thr && vm != -INFINITY);
+        while (cand) {  // rare after the first chunks: insert this vector's qualifying elements
+            const int src = __ffs(cand) - 1;
+            cand &= cand - 1;
+            const uint4 sv = make_uint4(__shfl_sync(FULL, v4.x, src), __shfl_sync(FULL, v4.y, src),
+                                        __shfl_sync(FULL, v4.z, src), __shfl_sync(FULL, v4.w, src));
 #pragma unroll
             for (int e = 0; e < R::VW; ++e) {
-                const float x = R::elem(v4, e);
-                const uint32_t v = (uint32_t)R::index_of(ch.v0, i, e);
-                if (x > tv || (thr != 0u && x == tv && v <= vk))
-                    sm.cand[atomicAdd(&sm.ncand, 1u)] = make_key(x, v);
+                const float x = R::elem(sv, e);
+                if (x >= wt.thr && x != -INFINITY) {  // warp-uniform
+                    const int64_t v = ch.v0 + (int64_t)(i * NT + (warp * 32 + src)) * R::VW + e;
+                    warp_insert(wt, make_key(x, (uint32_t)v));
+                }
             }
         }
     }
-    __syncthreads();
-    // (5) Sort the candidates 16 at a time into a running top-16 (warp 0).
-    if (warp == 0) {
-        const unsigned n = sm.ncand;
-        uint64_t acc = 0;
-        for (unsigned base = 0; base < n; base += K) {
-            uint64_t v = acc;
-            if (lane >= K) v = (base + lane - K < n) ? sm.cand[base + lane - K] : 0ull;
-            acc = warp_sort_desc(v);
-        }
-        if (lane < K) sm.keys[lane] = acc;
-        __syncwarp();
-        if (lane == 0) {  // thread 0 alone stores the partial (published by its release add)
-            uint4* dst = (uint4*)&part[unit];
-            dst[0] = make_uint4(__float_as_uint(sm.chunk.m), __float_as_uint(sm.chunk.s), 0u, 0u);
-            const uint4* kv = (const uint4*)sm.keys;
+    // block max, then the sum against it (no rescaling), both in a fixed order
 #pragma unroll
-            for (int j = 0; j < K / 2; ++j) dst[1 + j] = kv[j];
+    for (int j = 16; j > 0; j >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, j));
+    if (lane == 0) sm.wmax[warp] = m;
+    __syncthreads();
+    float M = sm.wmax[0];
+#pragma unroll
+    for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, sm.wmax[w]);
+    float s = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+        for (int i = 0; i < R::NV; ++i) {
+            const uint4 v4 = ch.vec(i);
+            float tt[R::VW];
+#pragma unroll
+            for (int e = 0; e < R::VW; ++e) tt[e] = ex2((R::elem(v4, e) - M) * c2);
+#pragma unroll
+            for (int w = R::VW / 2; w > 0; w >>= 1)
+#pragma unroll
+                for (int e = 0; e < w; ++e) tt[e] += tt[e + w];
+            s += tt[0];
         }
     }
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) s += __shfl_xor_sync(FULL, s, j);
+    if (lane == 0) sm.wsum[warp] = s;
+    __syncthreads();
+    float S = 0.0f;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) S += sm.wsum[w];
+    chunk_m = M;
+    chunk_s = S;
+}
+
+// End of a row segment: merge the 8 warp lists (warp 0) into sm.keys.
+__device__ __forceinline__ void topk_segment_merge(TopkSmem& sm, WarpTop& wt) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane < K) sm.wlist[warp][lane] = wt.key;
+    __syncthreads();
+    if (warp == 0) {
+        uint64_t acc = (lane < K) ? sm.wlist[0][lane] : 0ull;
+        for (int w = 1; w < NT / 32; ++w) acc = warp_merge_desc(lane < K ? acc : sm.wlist[w][31 - lane]);
+        if (lane < K) sm.keys[lane] = acc;
+    }
+    __syncthreads();
+    wt.key = 0ull;
+    wt.thr = -INFINITY;
 }
 
 // The row's final merge (warp 0 of the last unit of the row).
@@ -191,10 +200,12 @@ __global__ void __launch_bounds__(NT, 3) topk_softmax_kernel(
     }
     __shared__ bool s_last;
     unsigned pending = 0;
+    WarpTop wt{0ull, -INFINITY};
     int k = 0;
     for (int64_t u = lo; u < hi; ++u, ++k) {
         int64_t row, v0, vend;
         unit_geom(u, row, v0, vend);
+        float cm, cs;
         if (TMA) {
             if (t == 0 && u + 1 < hi) issue(u + 1, (k + 1) & 1);
             if (!__syncthreads_and(mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1))) {
@@ -204,16 +215,24 @@ __global__ void __launch_bounds__(NT, 3) topk_softmax_kernel(
                 }
                 return;
             }
-            SmemChunk<BF16> ch{ring + (k & 1) * SLOT, v0, vend};
-            topk_unit<BF16>(ch, c2, sm, part, u);
+            topk_unit<BF16>(SmemChunk<BF16>{ring + (k & 1) * SLOT, v0, vend}, c2, sm, wt, cm, cs);
         } else {
             RegChunk<BF16> ch;
             ch.load((const char*)logits + row * row_stride * ES, v0, vend);
-            topk_unit<BF16>(ch, c2, sm, part, u);
+            topk_unit<BF16>(ch, c2, sm, wt, cm, cs);
         }
         ++pending;
-        if (u + 1 == hi || (u + 1) / S != row) {  // this CTA is done with the row: publish
-            __syncthreads();
+        const bool seg_end = (u + 1 == hi) || ((u + 1) / S != row);
+        if (seg_end) topk_segment_merge(sm, wt);
+        if (t == 0) {  // thread 0 alone stores the partial (published by its release add);
+                       // only the last unit of a segment carries the segment's top-16
+            uint4* dst = (uint4*)&part[u];
+            dst[0] = make_uint4(__float_as_uint(cm), __float_as_uint(cs), 0u, 0u);
+            const uint4* kv = (const uint4*)sm.keys;
+#pragma unroll
+            for (int j = 0; j < K / 2; ++j) dst[1 + j] = seg_end ? kv[j] : make_uint4(0, 0, 0, 0);
+        }
+        if (seg_end) {  // this CTA is done with the row: publish
             if (t == 0) s_last = publish(&counters[row], pending, (unsigned)S);
             __syncthreads();
             if (s_last && warp == 0)

@@ -215,6 +215,46 @@ __device__ __forceinline__ void sample_finish(
     }
 }
 
+// A chunk's (max, sum-exp): the block max first, then each thread's sum of
+// exp2((x - M) c) (fp32 per vector, fp64 across vectors), then the block
+// sum in a fixed order -- no rescaling, no exp in the merge.
+template <bool BF16, class C>
+__device__ __forceinline__ LseD block_lse(const C& ch, float c2, float* s_max, double* s_sum) {
+    using R = Row<BF16>;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float m = view_max<BF16>(ch);
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, j));
+    if (lane == 0) s_max[warp] = m;
+    __syncthreads();
+    float M = s_max[0];
+#pragma unroll
+    for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, s_max[w]);
+    double s = 0.0;
+    if (M != -INFINITY) {
+#pragma unroll
+        for (int i = 0; i < R::NV; ++i) {
+            const uint4 v4 = ch.vec(i);
+            float tt[R::VW];
+#pragma unroll
+            for (int e = 0; e < R::VW; ++e) tt[e] = ex2((R::elem(v4, e) - M) * c2);
+#pragma unroll
+            for (int w = R::VW / 2; w > 0; w >>= 1)
+#pragma unroll
+                for (int e = 0; e < w; ++e) tt[e] += tt[e + w];
+            s += (double)tt[0];
+        }
+    }
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) s += __shfl_xor_sync(FULL, s, j);
+    if (lane == 0) s_sum[warp] = s;
+    __syncthreads();
+    double S = 0.0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) S += s_sum[w];
+    return {M, 0.0f, S};
+}
+
 template <bool BF16, bool TMA>
 __global__ void __launch_bounds__(NT, 3) verify_sample_scan_kernel(
     const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int S,
@@ -226,9 +266,10 @@ __global__ void __launch_bounds__(NT, 3) verify_sample_scan_kernel(
     constexpr int ES = BF16 ? 2 : 4;
     constexpr int SLOT = CHUNK * ES;
     extern __shared__ __align__(128) uint8_t ring[];
-    __shared__ LseD s_lse[NT / 32];
+    __shared__ float s_max[NT / 32];
+    __shared__ double s_sum[NT / 32];
     __shared__ __align__(8) uint64_t s_bar[2];
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int t = threadIdx.x, warp = t >> 5;
     const uint32_t bar0 = smem_u32(&s_bar[0]);
     const int per_seq = rows_per_seq * S;
     auto geom = [&](int64_t u, int& b, int& rr, const char*& rowp, int64_t& v0, int64_t& vend) {
@@ -267,7 +308,7 @@ __global__ void __launch_bounds__(NT, 3) verify_sample_scan_kernel(
         const char* rowp;
         int64_t v0, vend;
         geom(u, b, rr, rowp, v0, vend);
-        LseD mine;
+        LseD tot;
         if (TMA) {
             if (t == 0 && u + 1 < hi) issue(u + 1, (k + 1) & 1);
             if (!__syncthreads_and(mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1))) {
@@ -277,20 +318,14 @@ __global__ void __launch_bounds__(NT, 3) verify_sample_scan_kernel(
                 }
                 return;
             }
-            mine = view_lse_d<BF16>(SmemChunk<BF16>{ring + (k & 1) * SLOT, v0, vend}, c2);
+            tot = block_lse<BF16>(SmemChunk<BF16>{ring + (k & 1) * SLOT, v0, vend}, c2, s_max, s_sum);
         } else {
             RegChunk<BF16> ch;
             ch.load(rowp, v0, vend);
-            mine = view_lse_d<BF16>(ch, c2);
+            tot = block_lse<BF16>(ch, c2, s_max, s_sum);
         }
-        const LseD wl = warp_lse(mine, c2);
-        if (lane == 0) s_lse[warp] = wl;
-        __syncthreads();
-        if (t == 0) {  // thread 0 alone stores the partial (published by its release add)
-            LseD tot = s_lse[0];
-            for (int w = 1; w < NT / 32; ++w) tot = lse_merge(tot, s_lse[w], c2);
+        if (t == 0)  // thread 0 alone stores the partial (published by its release add)
             part[((int64_t)b * rows_per_seq + rr) * S + v0 / CHUNK] = tot;
-        }
         ++pending;
         if (u + 1 == hi || (u + 1) / per_seq != b) {  // done with this sequence: publish
             if (t == 0) s_last = publish(&counters[b], pending, (unsigned)per_seq);
@@ -301,7 +336,7 @@ __global__ void __launch_bounds__(NT, 3) verify_sample_scan_kernel(
                               n_accept, out_tok, ratio_dbg, u_dbg, info);
             pending = 0;
         }
-        __syncthreads();  // ring slot k & 1 is free; s_lse may be rewritten
+        __syncthreads();  // ring slot k & 1 is free
     }
 }
 
@@ -397,7 +432,7 @@ __device__ __forceinline__ double block_sum(double v, double* s_warp) {
 }
 
 template <bool BF16, bool VEC>
-__global__ void __launch_bounds__(NT, 2) verify_sample_draw_kernel(
+__global__ void __launch_bounds__(NT, 3) verify_sample_draw_kernel(
     const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int S,
     float c2, float inv_t, const SampleInfo* __restrict__ info, double* __restrict__ part2,
     unsigned* __restrict__ counters2, int32_t* __restrict__ out_tok) {
