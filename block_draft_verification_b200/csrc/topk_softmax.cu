@@ -307,3 +307,52 @@ extern "C" int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows,
 #undef DFL_TOPK
     return launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant.  Some callers cannot hand us device memory: an
+// inference engine that reserved nearly all of the GPU for its own memory
+// pools (KV cache, activations) at start-up and does not let a plugin call
+// cudaMalloc, or a latency-critical path where cudaMalloc could synchronise
+// the device.  For them the scratch (arrival counters and per-chunk partials)
+// lives in one fixed array of device memory inside this library, loaded with
+// the library on every GPU that uses it and kept until the process exits.
+namespace {
+
+constexpr size_t NOALLOC_SCRATCH_BYTES = DFLASH2_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+// Device address of the array on each device.  The host-side name of the
+// array is only a stand-in; the address a kernel can use is looked up once per
+// device, with that device current.
+constexpr int NOALLOC_MAX_DEVICES = 64;
+void* g_noalloc_addr[NOALLOC_MAX_DEVICES];
+std::mutex g_noalloc_mu;
+
+void* noalloc_scratch_on_current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_addr[dev] = p;
+    }
+    return g_noalloc_addr[dev];
+}
+
+}  // namespace
+
+extern "C" int dflash2_topk_softmax_noalloc(const void* logits, int dtype, int64_t rows, int64_t V,
+                                            int64_t row_stride, float inv_temperature, int32_t* idx,
+                                            float* prob, float* logp, float* logz,
+                                            dflash2_stream_t stream) {
+    if (!dtype_ok(dtype)) return DFLASH2_EDTYPE;
+    if (rows < 0 || V < K || V > INT32_MAX || row_stride < V) return DFLASH2_ESHAPE;
+    if (rows > 0 && topk_layout(rows, V).total > NOALLOC_SCRATCH_BYTES)
+        return DFLASH2_EWORKSPACE;  // more rows than the built-in scratch holds
+    if (rows == 0) return DFLASH2_OK;
+    void* scratch = noalloc_scratch_on_current_device();
+    if (!scratch) return DFLASH2_ECUDA;
+    return dflash2_topk_softmax(logits, dtype, rows, V, row_stride, inv_temperature, idx, prob, logp,
+                                logz, scratch, NOALLOC_SCRATCH_BYTES, stream);
+}

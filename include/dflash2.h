@@ -120,6 +120,35 @@ DFLASH2_API int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows
                          dflash2_stream_t stream);
 
 /*
+ * Allocation-free dflash2_topk_softmax.  The paper has no counterpart: this
+ * entry exists for callers that cannot give the library device memory -- an
+ * inference engine that reserved nearly all of the GPU for its own pools at
+ * start-up and does not let plugins call cudaMalloc, or a latency-critical
+ * path where cudaMalloc could synchronise the device.
+ *
+ * Same arguments, results and errors as dflash2_topk_softmax, minus the
+ * workspace: the scratch is a fixed array of DFLASH2_NOALLOC_SCRATCH_BYTES in
+ * the library's own device memory, present on every GPU that loads the
+ * library until the process exits.  The call allocates nothing (no
+ * cudaMalloc, no cudaFree, no allocating library routine); it clears the part
+ * of the array it uses with cudaMemsetAsync on `stream`.
+ *   - Limit: rows * ceil(V / 16384) * 144 + rows * 4 bytes (each rounded up
+ *     to 256) must fit in the array; larger shapes return DFLASH2_EWORKSPACE
+ *     and enqueue nothing.  At V = 151,936 that is up to 2,900 rows.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind: two calls that can overlap on the GPU (different streams without
+ *     an ordering between them) race and give wrong results.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ *     first call before any stream capture.
+ */
+#define DFLASH2_NOALLOC_SCRATCH_BYTES (4u << 20)
+DFLASH2_API int dflash2_topk_softmax_noalloc(const void* logits, int dtype, int64_t rows, int64_t V,
+                                             int64_t row_stride, float inv_temperature,
+                                             int32_t* idx, float* prob, float* logp, float* logz,
+                                             dflash2_stream_t stream);
+
+/*
  * Bilinear adjacent-pair selector and the exact best path.  [tamsi] "L’idée,
  * sans le papier" (choose a coherent path through the top-16 lists);
  * [myaiexp] "主な機能" (adjacent candidate pairs are scored); [psi] "Résumé"
