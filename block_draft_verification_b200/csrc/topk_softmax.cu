@@ -12,16 +12,17 @@
 // TMA bulk copies (rows whose start is 16-byte aligned; others are read
 // element by element).  Softmax: per chunk, the block max, then the sum of
 // exp2((x - M) c) against it, both in a fixed order, so a chunk's partial
-// does not depend on the batch or the grid.  Top-16: every warp keeps a
-// running top-16 of the row segment it streams (the CTA's consecutive chunks
-// of one row); an element is looked at only if its 8-element vector reaches
-// the warp's current 16th value, which after the first few thousand
-// elements almost never happens, and qualifying elements are inserted with a
-// shuffle.  At the end of the segment the 8 warp lists are merged and the
-// segment is published with one acquire-release add.  The publisher that
-// completes a row (no CTA waits) merges the chunk partials in chunk order and
-// the segment lists, and writes idx / prob / logp / logz.  Keys compare
-// (value, -index) exactly, so the top-16 set does not depend on who merged.
+// does not depend on the batch or the grid.  Top-16: the block keeps a
+// running top-16 of the row segment it streams (its consecutive chunks of one
+// row).  The first chunk of a segment takes the exact bounded path (the 16th
+// largest per-thread maximum bounds the answer, at most 16 threads contribute
+// candidates, one warp sorts them); later chunks only look at elements whose
+// key beats the running 16th key, about 16/c of them in the c-th chunk.  The
+// segment's list is published with one acquire-release add; the publisher
+// that completes a row (no CTA waits) merges the chunk softmax partials in
+// chunk order and the segment lists, and writes idx / prob / logp / logz.
+// Keys compare (value, -index) exactly, so the top-16 set does not depend on
+// how the row was split.
 #include "common.cuh"
 #include "stream.cuh"
 #include "workspace.cuh"
@@ -29,67 +30,143 @@
 namespace dfl {
 
 struct __align__(16) TopkSmem {
-    uint64_t keys[K];
-    uint64_t wlist[NT / 32][K];
+    uint64_t run[K];          // running top-16 of the row segment (descending; 0 = empty)
+    uint32_t top[NT / 32][K];
+    uint64_t cand[K * EPT];   // candidate keys (capacity 1024)
+    uint32_t tie[NT];
     float wmax[NT / 32];
     float wsum[NT / 32];
+    unsigned ncand, ntie;
+    uint32_t thr, vk;
 };
+constexpr unsigned CAND_CAP = K * EPT;
 
-// A warp's running top-16 of the current row segment: lanes 0..15 hold keys
-// in descending order (0 = empty), lanes 16..31 hold 0.
-struct WarpTop {
-    uint64_t key;
-    float thr;  // value of the 16th key (-inf while fewer than 16)
-};
-__device__ __forceinline__ void warp_insert(WarpTop& w, uint64_t k) {
+// Warp 0: merge sm.cand[0..n) into the running list (16 candidates a round).
+__device__ __forceinline__ void merge_candidates(TopkSmem& sm, unsigned n) {
     const int lane = threadIdx.x & 31;
-    const uint64_t up = shfl_up64(w.key);
-    if (lane < K) w.key = (lane > 0 && k > up) ? up : (k > w.key ? k : w.key);
-    const uint64_t last = shfl64(w.key, K - 1);
-    w.thr = last ? key_value(last) : -INFINITY;
+    uint64_t acc = (lane < K) ? sm.run[lane] : 0ull;
+    for (unsigned base = 0; base < n; base += K) {
+        uint64_t v = acc;
+        if (lane >= K) v = (base + lane - K < n) ? sm.cand[base + lane - K] : 0ull;
+        acc = warp_sort_desc(v);
+    }
+    if (lane < K) sm.run[lane] = acc;
 }
 
-// One unit: the chunk's softmax partial (block max, then the sum of
-// exp2((x - M) c) in a fixed order) and the warps' running top-16 updated
-// with the chunk's elements whose value reaches the warp's threshold.
+// The chunk's exact top-16 without sorting the chunk: T = the 16th largest
+// per-thread maximum bounds it; only threads whose maximum is above T, or
+// equal to T with a first index among the lowest (16 - #above) of those, can
+// hold a top-16 element (at most 16 threads x 64 candidates); they are merged
+// into the running list.  m = this thread's maximum.
 template <bool BF16, class C>
-__device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm, WarpTop& wt,
-                                          float& chunk_m, float& chunk_s) {
+__device__ __forceinline__ void chunk_top16_exact(const C& ch, float m, TopkSmem& sm) {
     using R = Row<BF16>;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    // pass 1: thread max and the top-16 filter, vector by vector
-    float m = -INFINITY;
+    const uint32_t my_ord = (m == -INFINITY) ? 0u : ord32(m);
+    const uint32_t srt = warp_sort_desc(my_ord);
+    if (lane < K) sm.top[warp][lane] = srt;
+    if (t == 0) {
+        sm.ncand = 0;
+        sm.ntie = 0;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t acc = (lane < K) ? sm.top[0][lane] : 0u;
+        for (int w = 1; w < NT / 32; ++w) acc = warp_merge_desc(lane < K ? acc : sm.top[w][31 - lane]);
+        if (lane == K - 1) sm.thr = acc;  // 0: fewer than 16 threads hold elements
+    }
+    __syncthreads();
+    const uint32_t thr = sm.thr;
+    const bool above = my_ord > thr;
+    const bool tie = thr != 0u && my_ord == thr;
+    const int n_above = __syncthreads_count(above);
+    uint32_t my_first = 0xFFFFFFFFu;
+    if (tie) {
+        my_first = view_first<BF16>(ch, m);
+        sm.tie[atomicAdd(&sm.ntie, 1u)] = my_first;
+    }
+    __syncthreads();
+    if (tie) {
+        const unsigned n = sm.ntie;
+        unsigned rank = 0;
+        for (unsigned j = 0; j < n; ++j) rank += sm.tie[j] < my_first;
+        if (rank == (unsigned)(K - n_above - 1)) sm.vk = my_first;
+    }
+    __syncthreads();
+    const float tv = (thr == 0u) ? -INFINITY : unord32(thr);
+    const uint32_t vk = (thr == 0u) ? 0u : sm.vk;
+    if (above || (tie && my_first <= vk)) {
 #pragma unroll
-    for (int i = 0; i < R::NV; ++i) {
-        const uint4 v4 = ch.vec(i);
-        float vm = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < R::VW; ++e) vm = fmaxf(vm, R::elem(v4, e));
-        m = fmaxf(m, vm);
-        unsigned cand = __ballot_sync(FULL, vm >= wt.thr && vm != -INFINITY);
-        while (cand) {  // rare after the first chunks: insert this vector's qualifying elements
-            const int src = __ffs(cand) - 1;
-            cand &= cand - 1;
-            const uint4 sv = make_uint4(__shfl_sync(FULL, v4.x, src), __shfl_sync(FULL, v4.y, src),
-                                        __shfl_sync(FULL, v4.z, src), __shfl_sync(FULL, v4.w, src));
+        for (int i = 0; i < R::NV; ++i) {
+            const uint4 v4 = ch.vec(i);
 #pragma unroll
             for (int e = 0; e < R::VW; ++e) {
-                const float x = R::elem(sv, e);
-                if (x >= wt.thr && x != -INFINITY) {  // warp-uniform
-                    const int64_t v = ch.v0 + (int64_t)(i * NT + (warp * 32 + src)) * R::VW + e;
-                    warp_insert(wt, make_key(x, (uint32_t)v));
-                }
+                const float x = R::elem(v4, e);
+                const uint32_t v = (uint32_t)R::index_of(ch.v0, i, e);
+                if (x > tv || (thr != 0u && x == tv && v <= vk))
+                    sm.cand[atomicAdd(&sm.ncand, 1u)] = make_key(x, v);
             }
         }
     }
-    // block max, then the sum against it (no rescaling), both in a fixed order
+    __syncthreads();
+    if (warp == 0) merge_candidates(sm, sm.ncand);
+    __syncthreads();
+}
+
+// One unit: the chunk's softmax partial (block max, then the sum of
+// exp2((x - M) c) against it, in a fixed order) and the running top-16.
+// Once the running list is full, only elements whose key beats its 16th key
+// are candidates: about 16/c of them in the c-th chunk of a segment, usually
+// none; if they would not fit (adversarial orders), the chunk takes the exact
+// bounded path instead.
+template <bool BF16, class C>
+__device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm, float& chunk_m,
+                                          float& chunk_s) {
+    using R = Row<BF16>;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const float m = view_max<BF16>(ch);
+    float wm = m;
 #pragma unroll
-    for (int j = 16; j > 0; j >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, j));
-    if (lane == 0) sm.wmax[warp] = m;
+    for (int j = 16; j > 0; j >>= 1) wm = fmaxf(wm, __shfl_xor_sync(FULL, wm, j));
+    if (lane == 0) sm.wmax[warp] = wm;
+    if (t == 0) sm.ncand = 0;
     __syncthreads();
     float M = sm.wmax[0];
 #pragma unroll
     for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, sm.wmax[w]);
+
+    const uint64_t r16 = sm.run[K - 1];
+    bool exact = (r16 == 0ull);
+    if (!exact) {
+        const float rv = key_value(r16);
+        if (m >= rv) {
+#pragma unroll
+            for (int i = 0; i < R::NV; ++i) {
+                const uint4 v4 = ch.vec(i);
+#pragma unroll
+                for (int e = 0; e < R::VW; ++e) {
+                    const float x = R::elem(v4, e);
+                    if (x >= rv) {
+                        const uint64_t key = make_key(x, (uint32_t)R::index_of(ch.v0, i, e));
+                        if (key > r16) {
+                            const unsigned slot = atomicAdd(&sm.ncand, 1u);
+                            if (slot < CAND_CAP) sm.cand[slot] = key;
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        const unsigned n = sm.ncand;
+        if (n > CAND_CAP) {
+            exact = true;  // block-uniform
+        } else if (n > 0) {
+            if (warp == 0) merge_candidates(sm, n);
+        }
+        __syncthreads();
+    }
+    if (exact) chunk_top16_exact<BF16>(ch, m, sm);
+
     float s = 0.0f;
     if (M != -INFINITY) {
 #pragma unroll
@@ -114,21 +191,6 @@ __device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm, W
     for (int w = 0; w < NT / 32; ++w) S += sm.wsum[w];
     chunk_m = M;
     chunk_s = S;
-}
-
-// End of a row segment: merge the 8 warp lists (warp 0) into sm.keys.
-__device__ __forceinline__ void topk_segment_merge(TopkSmem& sm, WarpTop& wt) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (lane < K) sm.wlist[warp][lane] = wt.key;
-    __syncthreads();
-    if (warp == 0) {
-        uint64_t acc = (lane < K) ? sm.wlist[0][lane] : 0ull;
-        for (int w = 1; w < NT / 32; ++w) acc = warp_merge_desc(lane < K ? acc : sm.wlist[w][31 - lane]);
-        if (lane < K) sm.keys[lane] = acc;
-    }
-    __syncthreads();
-    wt.key = 0ull;
-    wt.thr = -INFINITY;
 }
 
 // The row's final merge (warp 0 of the last unit of the row).
@@ -200,7 +262,7 @@ __global__ void __launch_bounds__(NT, 3) topk_softmax_kernel(
     }
     __shared__ bool s_last;
     unsigned pending = 0;
-    WarpTop wt{0ull, -INFINITY};
+    if (t < K) sm.run[t] = 0ull;
     int k = 0;
     for (int64_t u = lo; u < hi; ++u, ++k) {
         int64_t row, v0, vend;
@@ -215,20 +277,19 @@ __global__ void __launch_bounds__(NT, 3) topk_softmax_kernel(
                 }
                 return;
             }
-            topk_unit<BF16>(SmemChunk<BF16>{ring + (k & 1) * SLOT, v0, vend}, c2, sm, wt, cm, cs);
+            topk_unit<BF16>(SmemChunk<BF16>{ring + (k & 1) * SLOT, v0, vend}, c2, sm, cm, cs);
         } else {
             RegChunk<BF16> ch;
             ch.load((const char*)logits + row * row_stride * ES, v0, vend);
-            topk_unit<BF16>(ch, c2, sm, wt, cm, cs);
+            topk_unit<BF16>(ch, c2, sm, cm, cs);
         }
         ++pending;
         const bool seg_end = (u + 1 == hi) || ((u + 1) / S != row);
-        if (seg_end) topk_segment_merge(sm, wt);
         if (t == 0) {  // thread 0 alone stores the partial (published by its release add);
                        // only the last unit of a segment carries the segment's top-16
             uint4* dst = (uint4*)&part[u];
             dst[0] = make_uint4(__float_as_uint(cm), __float_as_uint(cs), 0u, 0u);
-            const uint4* kv = (const uint4*)sm.keys;
+            const uint4* kv = (const uint4*)sm.run;
 #pragma unroll
             for (int j = 0; j < K / 2; ++j) dst[1 + j] = seg_end ? kv[j] : make_uint4(0, 0, 0, 0);
         }
@@ -238,6 +299,8 @@ __global__ void __launch_bounds__(NT, 3) topk_softmax_kernel(
             if (s_last && warp == 0)
                 topk_row_merge(part + row * S, S, row, inv_t, c2, idx, prob, logp, logz);
             pending = 0;
+            __syncthreads();
+            if (t < K) sm.run[t] = 0ull;  // the next segment starts empty
         }
         __syncthreads();  // ring slot k & 1 is free for the prefetch of iteration k + 1
     }
