@@ -18,9 +18,9 @@
 //   warp 1   MMA issuer: one thread issues tcgen05.mma (M=128, N, K=16) x 4
 //            per K block, accumulating in TMEM; tcgen05.commit frees stages
 //   warp 2   TMEM allocation / release
-//   warps 4-7 epilogue: tcgen05.ld of their 32 TMEM lanes; the b rows go
-//            through shared memory to the a rows' threads, which load x and
-//            x_prev, apply the conv and the residual and store bf16
+//   warps 4-7 epilogue: tcgen05.ld of their 32 TMEM lanes into shared
+//            memory, then (token, 8-channel) items: 16-byte loads of x_t and
+//            x_{t-1}, conv + residual, one 16-byte bf16 store
 // Every mbarrier wait is bounded (one second, stream.cuh); on a timeout the
 // kernel records a flag (dflash2_device_errors), stops issuing work, releases
 // TMEM and returns.  No TMA load here uses cluster multicast.
@@ -109,8 +109,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int stage_bytes = TC_A_BYTES + sh.BN * TC_BK * 2;
     uint8_t* tail = base + sh.stages * stage_bytes;
-    float* s_b = (float*)tail;                                  // [64][33] b values
-    uint64_t* bars = (uint64_t*)(tail + TC_CH * 33 * 4);        // full[S], empty[S], accf
+    float* s_acc = (float*)tail;                                // [128][33] a, b values
+    uint64_t* bars = (uint64_t*)(tail + TC_BM * 33 * 4);        // full[S], empty[S], accf
     uint32_t* s_tmem = (uint32_t*)(bars + 2 * sh.stages + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -188,34 +188,56 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
         }
         mma_commit(accf);
     } else if (warp >= 4) {
-        // ---------------- epilogue
+        // ---------------- epilogue: 32 token columns at a time, TMEM -> shared
+        // (a in rows 0..63, b in rows 64..127), then each thread takes
+        // (token, 8-channel group) items with 16-byte loads of x_t and x_{t-1}
+        // and one 16-byte store of the 8 outputs.
         const int q = warp - 4;  // TMEM lanes 32q .. 32q + 31
+        const int e = threadIdx.x - 128;
         bool ok = mbar_wait(accf, 0);
         if (!ok) atomicOr(&g_dev_err, ERR_EPILOGUE);
         ok = __all_sync(FULL, ok);  // tcgen05.ld is warp-collective
         tc_fence_after();
         for (int c0 = 0; c0 < sh.BN; c0 += 32) {
-            float v[32];
-            if (ok) tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
-            if (q >= 2 && ok) {
+            if (ok) {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) s_b[((q - 2) * 32 + lane) * 33 + j] = v[j];
+                for (int j = 0; j < 32; ++j) s_acc[(32 * q + lane) * 33 + j] = v[j];
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (q < 2 && ok) {
-                const int ch = q * 32 + lane;
-                const int h = h0 + ch;
+            if (ok) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
+                for (int rep = 0; rep < 2; ++rep) {
+                    const int it = e + 128 * rep;
+                    const int j = it >> 3, g = it & 7;
                     const int tok = tok0 + c0 + j;
                     if (tok < sh.ntok) {
-                        const float xc = __bfloat162float(x[(int64_t)tok * sh.H + h]);
+                        const int h = h0 + 8 * g;
                         const int bi = tok / sh.T;
-                        const float xp = (tok - bi * sh.T == 0)
-                                             ? __bfloat162float(x_prev[(int64_t)bi * sh.H + h])
-                                             : __bfloat162float(x[(int64_t)(tok - 1) * sh.H + h]);
-                        const float y = fmaf(s_b[ch * 33 + j], xp, fmaf(v[j], xc, xc));
-                        out[(int64_t)tok * sh.H + h] = __float2bfloat16_rn(y);
+                        const uint4 xv = *(const uint4*)(x + (int64_t)tok * sh.H + h);
+                        const uint4 pv = (tok == bi * sh.T)
+                                             ? *(const uint4*)(x_prev + (int64_t)bi * sh.H + h)
+                                             : *(const uint4*)(x + (int64_t)(tok - 1) * sh.H + h);
+                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                        const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
+                        uint32_t ow[4];
+#pragma unroll
+                        for (int c = 0; c < 8; c += 2) {
+                            float y2[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const uint32_t xb = (u ? (xw[c >> 1] & 0xFFFF0000u) : (xw[c >> 1] << 16));
+                                const uint32_t pb = (u ? (pw[c >> 1] & 0xFFFF0000u) : (pw[c >> 1] << 16));
+                                const float xc = __uint_as_float(xb), xp = __uint_as_float(pb);
+                                const float a = s_acc[(8 * g + c + u) * 33 + j];
+                                const float b = s_acc[(64 + 8 * g + c + u) * 33 + j];
+                                y2[u] = fmaf(b, xp, fmaf(a, xc, xc));
+                            }
+                            const __nv_bfloat162 pr = __floats2bfloat162_rn(y2[0], y2[1]);
+                            ow[c >> 1] = *(const uint32_t*)&pr;
+                        }
+                        *(uint4*)(out + (int64_t)tok * sh.H + h) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                     }
                 }
             }
@@ -283,7 +305,7 @@ int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_
     if (!make_map(&mw, w_tap, (uint64_t)H, (uint64_t)2 * H, TC_BK, TC_CH)) return DFLASH2_ECUDA;
     if (!make_map(&mx, x, (uint64_t)H, (uint64_t)ntok, TC_BK, (uint32_t)BN)) return DFLASH2_ECUDA;
     const int stage_bytes = TC_A_BYTES + BN * TC_BK * 2;
-    const int fixed = 1024 + TC_CH * 33 * 4 + 64 * 8 + 16;
+    const int fixed = 1024 + TC_BM * 33 * 4 + 64 * 8 + 16;
     int stages = (227 * 1024 - fixed) / stage_bytes;
     stages = stages > 8 ? 8 : stages;
     if (stages < 2) return DFLASH2_ESHAPE;

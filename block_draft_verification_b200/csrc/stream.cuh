@@ -82,14 +82,21 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 // element v0 + (i * NT + t) * VW (see Row in common.cuh).  Elements at or past
 // vend read as -inf.
 template <bool BF16>
-struct SmemChunk {  // the chunk sits in shared memory (TMA ring slot)
+struct SmemChunk {  // the chunk sits in shared memory (TMA ring slot); its
+                    // length is a whole number of 16-byte vectors
     using R = Row<BF16>;
     const uint8_t* buf;
-    int64_t v0, vend;
+    int64_t v0;
+    int nvec;  // valid vectors in the chunk
+    __device__ __forceinline__ SmemChunk(const uint8_t* b, int64_t v0_, int64_t vend_)
+        : buf(b), v0(v0_), nvec((int)((vend_ - v0_) / R::VW)) {}
     __device__ __forceinline__ uint4 vec(int i) const {
-        const int64_t vb = v0 + (int64_t)(i * NT + (int)threadIdx.x) * R::VW;
-        if (vb < vend) return *(const uint4*)(buf + (vb - v0) * (BF16 ? 2 : 4));
+        const int idx = i * NT + (int)threadIdx.x;
+        if (idx < nvec) return *(const uint4*)(buf + idx * 16);
         return make_uint4(R::NEG_INF_WORD, R::NEG_INF_WORD, R::NEG_INF_WORD, R::NEG_INF_WORD);
+    }
+    __device__ __forceinline__ int64_t index_of(int i, int e) const {
+        return v0 + (int64_t)(i * NT + (int)threadIdx.x) * R::VW + e;
     }
 };
 template <bool BF16>
@@ -103,6 +110,9 @@ struct RegChunk {  // the chunk is read element by element into registers
         R::template load<false>(row, v0, vend, r);
     }
     __device__ __forceinline__ uint4 vec(int i) const { return r[i]; }
+    __device__ __forceinline__ int64_t index_of(int i, int e) const {
+        return v0 + (int64_t)(i * NT + (int)threadIdx.x) * R::VW + e;
+    }
 };
 
 // Thread max and sum-exp over a chunk view (two passes; pairwise per vector).
@@ -182,7 +192,7 @@ __device__ __forceinline__ uint32_t view_first(const C& ch, float x) {
         const uint4 v = ch.vec(i);
 #pragma unroll
         for (int e = R::VW - 1; e >= 0; --e)
-            if (R::elem(v, e) == x) first = (uint32_t)R::index_of(ch.v0, i, e);
+            if (R::elem(v, e) == x) first = (uint32_t)ch.index_of(i, e);
     }
     return first;
 }

@@ -35,6 +35,7 @@ struct __align__(16) TopkSmem {
     uint64_t cand[K * EPT];   // candidate keys (capacity 1024)
     uint32_t tie[NT];
     float wmax[NT / 32];
+    float wmax2[NT / 32];
     float wsum[NT / 32];
     unsigned ncand, ntie;
     uint32_t thr, vk;
@@ -62,6 +63,7 @@ template <bool BF16, class C>
 __device__ __forceinline__ void chunk_top16_exact(const C& ch, float m, TopkSmem& sm) {
     using R = Row<BF16>;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    __syncthreads();  // everyone has read the count that sent the block here
     const uint32_t my_ord = (m == -INFINITY) ? 0u : ord32(m);
     const uint32_t srt = warp_sort_desc(my_ord);
     if (lane < K) sm.top[warp][lane] = srt;
@@ -102,7 +104,7 @@ __device__ __forceinline__ void chunk_top16_exact(const C& ch, float m, TopkSmem
 #pragma unroll
             for (int e = 0; e < R::VW; ++e) {
                 const float x = R::elem(v4, e);
-                const uint32_t v = (uint32_t)R::index_of(ch.v0, i, e);
+                const uint32_t v = (uint32_t)ch.index_of(i, e);
                 if (x > tv || (thr != 0u && x == tv && v <= vk))
                     sm.cand[atomicAdd(&sm.ncand, 1u)] = make_key(x, v);
             }
@@ -114,67 +116,101 @@ __device__ __forceinline__ void chunk_top16_exact(const C& ch, float m, TopkSmem
 }
 
 // One unit: the chunk's softmax partial (block max, then the sum of
-// exp2((x - M) c) against it, in a fixed order) and the running top-16.
-// Once the running list is full, only elements whose key beats its 16th key
-// are candidates: about 16/c of them in the c-th chunk of a segment, usually
-// none; if they would not fit (adversarial orders), the chunk takes the exact
-// bounded path instead.
+// exp2(x c - M c) against it, in a fixed order) and the running top-16.
+//  - Running list full: elements whose key beats its 16th key are pushed as
+//    candidates during the max pass (about 16/c of them in the c-th chunk of
+//    a segment); warp 0 merges them while the other warps sum exps.
+//  - Running list empty (first chunk of a segment): T' = the smallest of the
+//    warps' second-largest thread maxima has at least 16 elements at or above
+//    it (two per warp), so the elements >= T' hold the chunk's top-16; they are
+//    pushed and merged.
+//  - More candidates than the buffer holds (adversarial orders, mass ties):
+//    the chunk takes the exact bounded path.
 template <bool BF16, class C>
 __device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm, float& chunk_m,
                                           float& chunk_s) {
     using R = Row<BF16>;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const float m = view_max<BF16>(ch);
+    const uint64_t r16 = sm.run[K - 1];
+    const float rv = r16 ? key_value(r16) : INFINITY;
+    // pass 1: thread max, and candidates against the running list
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < R::NV; ++i) {
+        const uint4 v4 = ch.vec(i);
+        float vm = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < R::VW; ++e) vm = fmaxf(vm, R::elem(v4, e));
+        m = fmaxf(m, vm);
+        if (vm >= rv) {
+#pragma unroll
+            for (int e = 0; e < R::VW; ++e) {
+                const float x = R::elem(v4, e);
+                if (x >= rv) {
+                    const uint64_t key = make_key(x, (uint32_t)ch.index_of(i, e));
+                    if (key > r16) {
+                        const unsigned slot = atomicAdd(&sm.ncand, 1u);
+                        if (slot < CAND_CAP) sm.cand[slot] = key;
+                    }
+                }
+            }
+        }
+    }
+    // warp max and (for seeding) the warp's second-largest thread maximum
     float wm = m;
 #pragma unroll
     for (int j = 16; j > 0; j >>= 1) wm = fmaxf(wm, __shfl_xor_sync(FULL, wm, j));
-    if (lane == 0) sm.wmax[warp] = wm;
-    if (t == 0) sm.ncand = 0;
-    __syncthreads();
+    const unsigned at_max = __ballot_sync(FULL, m == wm);
+    float m2 = (lane == __ffs(at_max) - 1) ? -INFINITY : m;
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) m2 = fmaxf(m2, __shfl_xor_sync(FULL, m2, j));
+    if (lane == 0) {
+        sm.wmax[warp] = wm;
+        sm.wmax2[warp] = m2;
+    }
+    __syncthreads();  // A
     float M = sm.wmax[0];
 #pragma unroll
     for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, sm.wmax[w]);
-
-    const uint64_t r16 = sm.run[K - 1];
-    bool exact = (r16 == 0ull);
-    if (!exact) {
-        const float rv = key_value(r16);
-        if (m >= rv) {
+    bool exact = false;
+    if (r16 == 0ull) {  // seed the segment's list from this chunk
+        float Tp = sm.wmax2[0];
+#pragma unroll
+        for (int w = 1; w < NT / 32; ++w) Tp = fminf(Tp, sm.wmax2[w]);
+        if (m >= Tp && m != -INFINITY) {
 #pragma unroll
             for (int i = 0; i < R::NV; ++i) {
                 const uint4 v4 = ch.vec(i);
 #pragma unroll
                 for (int e = 0; e < R::VW; ++e) {
                     const float x = R::elem(v4, e);
-                    if (x >= rv) {
-                        const uint64_t key = make_key(x, (uint32_t)R::index_of(ch.v0, i, e));
-                        if (key > r16) {
-                            const unsigned slot = atomicAdd(&sm.ncand, 1u);
-                            if (slot < CAND_CAP) sm.cand[slot] = key;
-                        }
+                    if (x >= Tp && x != -INFINITY) {
+                        const unsigned slot = atomicAdd(&sm.ncand, 1u);
+                        if (slot < CAND_CAP) sm.cand[slot] = make_key(x, (uint32_t)ch.index_of(i, e));
                     }
                 }
             }
         }
-        __syncthreads();
-        const unsigned n = sm.ncand;
-        if (n > CAND_CAP) {
-            exact = true;  // block-uniform
-        } else if (n > 0) {
-            if (warp == 0) merge_candidates(sm, n);
-        }
-        __syncthreads();
+        __syncthreads();  // B (seeding chunks only)
+    }
+    const unsigned n = sm.ncand;
+    if (n > CAND_CAP) {
+        exact = true;  // block-uniform
+    } else if (n > 0 && warp == 0) {
+        merge_candidates(sm, n);  // overlaps the other warps' exp pass
     }
     if (exact) chunk_top16_exact<BF16>(ch, m, sm);
 
+    // pass 2: sum of exp2(x c - M c) (fixed order)
     float s = 0.0f;
     if (M != -INFINITY) {
+        const float mc = M * c2;
 #pragma unroll
         for (int i = 0; i < R::NV; ++i) {
             const uint4 v4 = ch.vec(i);
             float tt[R::VW];
 #pragma unroll
-            for (int e = 0; e < R::VW; ++e) tt[e] = ex2((R::elem(v4, e) - M) * c2);
+            for (int e = 0; e < R::VW; ++e) tt[e] = ex2(fmaf(R::elem(v4, e), c2, -mc));
 #pragma unroll
             for (int w = R::VW / 2; w > 0; w >>= 1)
 #pragma unroll
@@ -185,12 +221,13 @@ __device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm, f
 #pragma unroll
     for (int j = 16; j > 0; j >>= 1) s += __shfl_xor_sync(FULL, s, j);
     if (lane == 0) sm.wsum[warp] = s;
-    __syncthreads();
+    __syncthreads();  // D: sums ready, candidates merged
     float S = 0.0f;
 #pragma unroll
     for (int w = 0; w < NT / 32; ++w) S += sm.wsum[w];
     chunk_m = M;
     chunk_s = S;
+    if (t == 0) sm.ncand = 0;  // read by everyone before D; next pushes come after
 }
 
 // The row's final merge (warp 0 of the last unit of the row).
@@ -263,6 +300,7 @@ __global__ void __launch_bounds__(NT, 3) topk_softmax_kernel(
     __shared__ bool s_last;
     unsigned pending = 0;
     if (t < K) sm.run[t] = 0ull;
+    if (t == 0) sm.ncand = 0;
     int k = 0;
     for (int64_t u = lo; u < hi; ++u, ++k) {
         int64_t row, v0, vend;
