@@ -5,6 +5,7 @@
 // streaming vocabulary-row loads, Philox4x32-10, and the host-side checks.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -219,6 +220,21 @@ struct Row {
         return v0 + (int64_t)(i * NT + (int)threadIdx.x) * VW + e;
     }
 };
+
+// Max of the 8 bf16 (or 4 fp32) elements of a 16-byte vector, widened to fp32.
+// bf16 uses packed two-lane max instructions (values are finite; -0 and +0
+// may come back either way, and every later compare treats them as equal).
+template <bool BF16>
+__device__ __forceinline__ float vec_max(const uint4& v) {
+    if (BF16) {
+        auto b2 = [](uint32_t w) { return *reinterpret_cast<const __nv_bfloat162*>(&w); };
+        const __nv_bfloat162 m = __hmax2(__hmax2(b2(v.x), b2(v.y)), __hmax2(b2(v.z), b2(v.w)));
+        const uint32_t mw = *reinterpret_cast<const uint32_t*>(&m);
+        return fmaxf(__uint_as_float(mw << 16), __uint_as_float(mw & 0xFFFF0000u));
+    }
+    return fmaxf(fmaxf(__uint_as_float(v.x), __uint_as_float(v.y)),
+                 fmaxf(__uint_as_float(v.z), __uint_as_float(v.w)));
+}
 
 // Thread max and sum-exp over the loaded vectors (pairwise within a vector).
 template <bool BF16>

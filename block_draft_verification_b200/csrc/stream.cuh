@@ -175,11 +175,7 @@ __device__ __forceinline__ float view_max(const C& ch) {
     using R = Row<BF16>;
     float m = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < R::NV; ++i) {
-        const uint4 v = ch.vec(i);
-#pragma unroll
-        for (int e = 0; e < R::VW; ++e) m = fmaxf(m, R::elem(v, e));
-    }
+    for (int i = 0; i < R::NV; ++i) m = fmaxf(m, vec_max<BF16>(ch.vec(i)));
     return m;
 }
 // Lowest index of this thread's elements equal to x (0xFFFFFFFF if none).

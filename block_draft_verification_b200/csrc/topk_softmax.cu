@@ -138,9 +138,7 @@ __device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm, f
 #pragma unroll
     for (int i = 0; i < R::NV; ++i) {
         const uint4 v4 = ch.vec(i);
-        float vm = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < R::VW; ++e) vm = fmaxf(vm, R::elem(v4, e));
+        const float vm = vec_max<BF16>(v4);
         m = fmaxf(m, vm);
         if (vm >= rv) {
 #pragma unroll

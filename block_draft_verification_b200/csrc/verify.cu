@@ -348,6 +348,22 @@ __global__ void __launch_bounds__(NT, 3) verify_sample_scan_kernel(
 //           value, without the cancellation of p - q when p and q agree;
 //   mode 1: w = p, 0 at d;  mode 2: w = p.
 // With use_p (the residual was empty by rounding) the weight is p.
+// e^d - 1 for d > 0: the Taylor series to d^8 for d <= 1/2 (truncation below
+// 6e-9 relative there), e^d - 1 from exp2 above, where the subtraction costs
+// at most two bits.
+__device__ __forceinline__ float expm1_pos(float d) {
+    if (d > 0.5f) return ex2(d * 1.4426950408889634f) - 1.0f;
+    float p = 1.0f / 40320.0f;
+    p = fmaf(p, d, 1.0f / 5040.0f);
+    p = fmaf(p, d, 1.0f / 720.0f);
+    p = fmaf(p, d, 1.0f / 120.0f);
+    p = fmaf(p, d, 1.0f / 24.0f);
+    p = fmaf(p, d, 1.0f / 6.0f);
+    p = fmaf(p, d, 0.5f);
+    p = fmaf(p, d, 1.0f);
+    return p * d;
+}
+
 template <bool BF16>
 __device__ __forceinline__ float draw_weight(const uint4& rt, const uint4& rq, int e, int64_t v,
                                              const SampleInfo& I, float c, float inv_t,
@@ -358,7 +374,7 @@ __device__ __forceinline__ float draw_weight(const uint4& rt, const uint4& rq, i
         const float xq = R::elem(rq, e);
         const float dlog = (xt - xq) * inv_t - I.dl;
         if (!(dlog > 0.0f)) return 0.0f;
-        return ex2((xq - I.mq) * c - I.l2q) * expm1f(dlog);
+        return ex2((xq - I.mq) * c - I.l2q) * expm1_pos(dlog);
     }
     if (I.mode == 1 && !use_p && v == I.d) return 0.0f;
     return ex2((xt - I.mt) * c - I.l2t);
@@ -395,24 +411,44 @@ __device__ __forceinline__ void load_contig(const void* row, int64_t v0, int64_t
     }
 }
 
-// Sum of the draw weights of this thread's 64 elements (fp32 per vector,
-// fp64 across vectors).
+// One 16-byte vector (element vb .. vb + VW - 1) of a row; -inf past vend.
 template <bool BF16, bool VEC>
-__device__ __forceinline__ double thread_weight_sum(const char* trow, const char* qrow, int64_t v0,
-                                                    int64_t vend, const SampleInfo& I, float c2,
-                                                    float inv_t, bool use_p) {
+__device__ __forceinline__ uint4 load_vec(const char* row, int64_t vb, int64_t vend) {
     using R = Row<BF16>;
-    uint4 rt[R::NV], rq[R::NV];
-    load_contig<BF16, VEC>(trow, v0, vend, rt);
-    if (I.mode == 0 && !use_p) load_contig<BF16, VEC>(qrow, v0, vend, rq);
+    if (VEC && vb + R::VW <= vend) return *(const uint4*)(row + vb * (BF16 ? 2 : 4));
+    uint32_t w[4] = {R::NEG_INF_WORD, R::NEG_INF_WORD, R::NEG_INF_WORD, R::NEG_INF_WORD};
+    for (int e = 0; e < R::VW; ++e)
+        if (vb + e < vend) {
+            const uint32_t bits = R::scalar_bits(row, vb + e);
+            if (BF16) {
+                uint32_t& word = w[e >> 1];
+                word = (e & 1) ? ((word & 0x0000FFFFu) | (bits << 16)) : ((word & 0xFFFF0000u) | bits);
+            } else {
+                w[e] = bits;
+            }
+        }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Sum of the draw weights of this thread's 64 elements (fp32 per vector,
+// fp64 across vectors).  The vector loop is not unrolled: the kernel's code
+// stays small enough for the instruction cache.
+template <bool BF16, bool VEC>
+__device__ __noinline__ double thread_weight_sum(const char* trow, const char* qrow, int64_t v0,
+                                                 int64_t vend, const SampleInfo& I, float c2,
+                                                 float inv_t, bool use_p) {
+    using R = Row<BF16>;
+    const bool with_q = I.mode == 0 && !use_p;
     double s = 0.0;
     const int64_t vb = v0 + (int64_t)threadIdx.x * EPT;
-#pragma unroll
+#pragma unroll 1
     for (int i = 0; i < R::NV; ++i) {
+        const uint4 rt = load_vec<BF16, VEC>(trow, vb + i * R::VW, vend);
+        const uint4 rq = with_q ? load_vec<BF16, VEC>(qrow, vb + i * R::VW, vend) : make_uint4(0, 0, 0, 0);
         float sv = 0.0f;
 #pragma unroll
         for (int e = 0; e < R::VW; ++e)
-            sv += draw_weight<BF16>(rt[i], rq[i], e, vb + i * R::VW + e, I, c2, inv_t, use_p);
+            sv += draw_weight<BF16>(rt, rq, e, vb + i * R::VW + e, I, c2, inv_t, use_p);
         s += (double)sv;
     }
     return s;
@@ -584,16 +620,19 @@ __global__ void __launch_bounds__(NT, 3) verify_sample_draw_kernel(
     __syncthreads();
     if (!s_done) {  // block-uniform: rounding left t above the chunk's scan
         if (mysum > 0.0) {
-            uint4 rt[R::NV], rq[R::NV];
-            load_contig<BF16, VEC>(trow, v0, vend, rt);
-            if (I.mode == 0 && !use_p) load_contig<BF16, VEC>(qrow, v0, vend, rq);
+            const bool with_q = I.mode == 0 && !use_p;
             int lastpos = -1;
             const int64_t vb = v0 + (int64_t)t * EPT;
-            for (int i = 0; i < R::NV; ++i)
+#pragma unroll 1
+            for (int i = 0; i < R::NV; ++i) {
+                const uint4 rt = load_vec<BF16, VEC>(trow, vb + i * R::VW, vend);
+                const uint4 rq =
+                    with_q ? load_vec<BF16, VEC>(qrow, vb + i * R::VW, vend) : make_uint4(0, 0, 0, 0);
+#pragma unroll 1
                 for (int e = 0; e < R::VW; ++e)
-                    if (draw_weight<BF16>(rt[i], rq[i], e, vb + i * R::VW + e, I, c2, inv_t, use_p) >
-                        0.0f)
+                    if (draw_weight<BF16>(rt, rq, e, vb + i * R::VW + e, I, c2, inv_t, use_p) > 0.0f)
                         lastpos = i * R::VW + e;
+            }
             if (lastpos >= 0) atomicMax(&s_last, t * EPT + lastpos);
         }
         __syncthreads();
