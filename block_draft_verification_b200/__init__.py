@@ -50,7 +50,9 @@ def lib():
         L.dflash2_verify_greedy.argtypes = [vp, i32, i32, i32, i64, vp, vp, vp, vp, sz, vp]
         L.dflash2_verify_sample.argtypes = [vp, vp, i32, i32, i32, i64, vp, f32, u64, u32, vp, i32,
                                             vp, vp, vp, vp, vp, sz, vp]
-        L.dflash2_dynconv2.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp]
+        L.dflash2_dynconv2.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]
+        L.dflash2_dynconv2_workspace_bytes.argtypes = [i32, i32, i32, i32]
+        L.dflash2_dynconv2_workspace_bytes.restype = sz
         L.dflash2_device_errors.argtypes = [i32]
         L.dflash2_device_errors.restype = C.c_uint32
         for f in ("dflash2_topk_softmax", "dflash2_pair_select", "dflash2_verify_greedy",
@@ -121,6 +123,10 @@ class Workspace:
 
     def args(self, B, G, V):
         self.reserve(workspace_bytes(B, G, V))
+        return C.c_void_p(self.buf.data_ptr()), C.c_size_t(self.buf.numel())
+
+    def args_bytes(self, nbytes):
+        self.reserve(nbytes)
         return C.c_void_p(self.buf.data_ptr()), C.c_size_t(self.buf.numel())
 
 
@@ -220,13 +226,18 @@ def verify_sample(target, draft, draft_tok, seed, step, seq_id=None, inv_tempera
     return out
 
 
-def dynconv2(x, x_prev, w_tap, out=None):
+def dynconv2(x, x_prev, w_tap, out=None, ws=None):
     """x [B, T, H], x_prev [B, H], w_tap [2H, H] (one dtype) -> out [B, T, H]."""
     _cuda(x, x_prev, w_tap)
     B, T, H = x.shape
     if out is None:
         out = torch.empty_like(x)
+    need = lib().dflash2_dynconv2_workspace_bytes(_dtype(x), B, T, H)
+    if ws is None:
+        ws = _ws_cache.setdefault((x.device.index, torch.cuda.current_stream(x.device).cuda_stream),
+                                  Workspace(x.device))
+    wp, wb = ws.args_bytes(need)
     _check("dflash2_dynconv2", lib().dflash2_dynconv2(
         _p(x.contiguous()), _p(x_prev.contiguous()), _p(w_tap.contiguous()), _dtype(x), B, T, H,
-        _p(out), _stream(x.device)))
+        _p(out), wp, wb, _stream(x.device)))
     return out

@@ -100,24 +100,37 @@ using namespace dfl;
 using namespace dfl_host;
 
 int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_tap, int B, int T,
-                               int H, void* out, cudaStream_t s);
+                               int H, void* out, void* ws, cudaStream_t s);
+size_t dflash2_dynconv2_tc_workspace(int64_t ntok, int H);
+
+static bool dynconv_shape_ok(int B, int T, int H) {
+    return B >= 0 && T >= 0 && H >= 64 && H % 64 == 0 && (int64_t)B * T <= (int64_t)INT32_MAX / 2;
+}
+
+extern "C" size_t dflash2_dynconv2_workspace_bytes(int dtype, int B, int T, int H) {
+    if (!dtype_ok(dtype) || !dynconv_shape_ok(B, T, H)) return 0;
+    if (dtype != DFLASH2_BF16 || (int64_t)B * T == 0) return 0;
+    return dflash2_dynconv2_tc_workspace((int64_t)B * T, H);
+}
 
 extern "C" int dflash2_dynconv2(const void* x, const void* x_prev, const void* w_tap, int dtype,
-                                int B, int T, int H, void* out, dflash2_stream_t stream) {
+                                int B, int T, int H, void* out, void* ws, size_t ws_bytes,
+                                dflash2_stream_t stream) {
     if (!dtype_ok(dtype)) return DFLASH2_EDTYPE;
-    if (B < 0 || T < 0 || H < 64 || H % 64 != 0) return DFLASH2_ESHAPE;
+    if (!dynconv_shape_ok(B, T, H)) return DFLASH2_ESHAPE;
     if ((int64_t)B * T == 0) return DFLASH2_OK;
     if (!x || !x_prev || !w_tap || !out) return DFLASH2_EINVAL;
     if (!aligned(x, 16) || !aligned(x_prev, 16) || !aligned(w_tap, 16) || !aligned(out, 16))
         return DFLASH2_EALIGN;
     const int64_t ntok = (int64_t)B * T;
-    if (ntok > (int64_t)INT32_MAX / 2) return DFLASH2_ESHAPE;
     const int64_t warps = (int64_t)H * ((ntok + DC_TOK - 1) / DC_TOK);
     const int64_t blocks = (warps + NT / 32 - 1) / (NT / 32);
     if (blocks > (int64_t)INT32_MAX) return DFLASH2_ESHAPE;
+    const size_t need = dflash2_dynconv2_workspace_bytes(dtype, B, T, H);
+    if (need > 0 && (!ws || !aligned(ws, 256) || ws_bytes < need)) return DFLASH2_EWORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     if (dtype == DFLASH2_BF16)  // tensor cores (tcgen05 + TMA), dynconv2_tc.cu
-        return dflash2_dynconv2_tc_launch(x, x_prev, w_tap, B, T, H, out, s);
+        return dflash2_dynconv2_tc_launch(x, x_prev, w_tap, B, T, H, out, ws, s);
     dynconv2_simt_kernel<false><<<(unsigned)blocks, NT, 0, s>>>(x, x_prev, w_tap, T, H, (int)ntok,
                                                                 out);
     return launch_status();

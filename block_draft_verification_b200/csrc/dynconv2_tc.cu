@@ -8,24 +8,41 @@
 // [a_t; b_t] = W_tap x_t and x_{-1} = x_prev.
 //
 // The tap projection is the GEMM D[2H x N] = W_tap[2H x H] . X^T[H x N] over
-// the N = B*T tokens.  A CTA owns 64 output channels h0..h0+63: its M = 128
-// tile stacks the 64 W_a rows and the 64 matching W_b rows, so a and b of a
-// channel meet in one accumulator and the conv, the residual and the rounding
-// run in the epilogue straight out of tensor memory.
+// the N = B*T tokens.  A tile is 64 output channels h0..h0+63 of one chunk of
+// up to 256 tokens: its M = 128 accumulator stacks the 64 W_a rows and the 64
+// matching W_b rows, so a and b of a channel meet in one accumulator and the
+// conv, the residual and the rounding run in the epilogue.
+//
+// Work is split stream-K: the (tile, 64-wide K block) steps, tile-major, are
+// cut into one contiguous run per CTA (one CTA per SM, launched
+// cooperatively so all are resident), so every SM streams the same share of
+// W_tap whatever the tile count.  A run is a sequence of segments (the part
+// of the run inside one tile).  The CTA holding a tile's K block 0 owns the
+// tile; a CTA whose run starts inside a tile (at most its first segment)
+// writes that segment's fp32 accumulator to the workspace and raises its
+// flag.  The owner adds those partials in K order (CTA order) to its own
+// accumulator before the epilogue: a fixed summation order for given shapes.
+// An owner only ever waits for the FIRST segment of later CTAs, which waits
+// for nothing, so no wait chain forms.
 //   warp 0   TMA producer: W tile (2 boxes of 64 x 64) + X tile (N x 64) per
-//            64-wide K block into a ring of shared-memory stages (128-byte
-//            swizzle), one mbarrier pair per stage
-//   warp 1   MMA issuer: one thread issues tcgen05.mma (M=128, N, K=16) x 4
-//            per K block, accumulating in TMEM; tcgen05.commit frees stages
+//            step into a ring of shared-memory stages (128-byte swizzle)
+//   warp 1   MMA issuer: tcgen05.mma (M=128, N, K=16) x 4 per step into one of
+//            two TMEM accumulators (segments alternate, so a segment's
+//            epilogue overlaps the next segment's MMAs)
 //   warp 2   TMEM allocation / release
-//   warps 4-7 epilogue: tcgen05.ld of their 32 TMEM lanes into shared
-//            memory, then (token, 8-channel) items: 16-byte loads of x_t and
-//            x_{t-1}, conv + residual, one 16-byte bf16 store
-// Every mbarrier wait is bounded (one second, stream.cuh); on a timeout the
-// kernel records a flag (dflash2_device_errors), stops issuing work, releases
-// TMEM and returns.  No TMA load here uses cluster multicast.
+//   warps 4-7 epilogue: tcgen05.ld of their 32 TMEM lanes; a partial goes to
+//            the workspace, an owned tile adds the partials, stages the
+//            values in shared memory, then (token, 8-channel) items with
+//            16-byte loads of x_t and x_{t-1} and one 16-byte store
+// Every wait is bounded (one second, stream.cuh); on a timeout the kernel
+// records a flag (dflash2_device_errors), stops issuing work, waits (bounded)
+// for its tensor-core work in flight, releases TMEM and returns.  No TMA load
+// here uses cluster multicast.
 #include <cuda.h>
 #include <cuda_bf16.h>
+
+#include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "stream.cuh"
@@ -96,37 +113,66 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+constexpr int TC_MAXCTA = 256;  // stream-K CTAs at most (one per SM)
+
 struct TcShape {
-    int H, T, ntok, tok0, BN, stages, nkb;
+    int H, T, ntok, BN, stages, nkb, nh;  // nh: channel tiles per token chunk
+    int bufcols;                           // TMEM columns per accumulator (power of 2, >= BN)
+    int ngroups;                           // 32-column groups per accumulator
+    int nctas;                             // stream-K CTAs
+    int64_t steps;                         // tiles * nkb
 };
+
+__device__ __forceinline__ int64_t run_start(const TcShape& sh, int p) {
+    return sh.steps * p / sh.nctas;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ x_prev,
-    __nv_bfloat16* __restrict__ out, TcShape sh) {
+    __nv_bfloat16* __restrict__ out, TcShape sh, float4* __restrict__ partial,
+    unsigned* __restrict__ flags) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // stage ring, 1024-byte aligned for the 128-byte swizzle
     uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int stage_bytes = TC_A_BYTES + sh.BN * TC_BK * 2;
     uint8_t* tail = base + sh.stages * stage_bytes;
-    float* s_acc = (float*)tail;                                // [128][33] a, b values
-    uint64_t* bars = (uint64_t*)(tail + TC_BM * 33 * 4);        // full[S], empty[S], accf
-    uint32_t* s_tmem = (uint32_t*)(bars + 2 * sh.stages + 1);
+    float* s_acc = (float*)tail;  // [128][33] a, b values of 32 token columns
+    // full[S], empty[S], tmem_full[2], tmem_empty[2], mma_done
+    uint64_t* bars = (uint64_t*)(tail + TC_BM * 33 * 4);
+    uint32_t* s_tmem = (uint32_t*)(bars + 2 * sh.stages + 5);
+    int* s_fail = (int*)(s_tmem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h0 = blockIdx.x * TC_CH;
-    const int tok0 = sh.tok0 + blockIdx.y * TC_MAXN;
+    const int p = blockIdx.x;
+    const int64_t s0 = run_start(sh, p), s1 = run_start(sh, p + 1);
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + sh.stages);
-    const uint32_t accf = smem_u32(bars + 2 * sh.stages);
-    const uint32_t ncols = sh.BN <= 32 ? 32 : (sh.BN <= 64 ? 64 : (sh.BN <= 128 ? 128 : 256));
+    const uint32_t tfull0 = smem_u32(bars + 2 * sh.stages);
+    const uint32_t tempty0 = tfull0 + 16;
+    const uint32_t mdone = tfull0 + 32;
+    const uint32_t ncols = 2 * (uint32_t)sh.bufcols;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < sh.stages; ++s) {
-            mbar_init(full0 + 8 * s, 1);
-            mbar_init(empty0 + 8 * s, 1);
+        for (int i = 0; i < sh.stages; ++i) {
+            mbar_init(full0 + 8 * i, 1);
+            mbar_init(empty0 + 8 * i, 1);
         }
-        mbar_init(accf, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(tfull0 + 8 * i, 1);
+            mbar_init(tempty0 + 8 * i, 1);
+        }
+        mbar_init(mdone, 1);
         mbar_fence_init();
+        *s_fail = 0;
     }
     if (warp == 2) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -140,80 +186,159 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     const uint32_t tmem = *s_tmem;
 
     if (warp == 0 && lane == 0) {
-        // ---------------- TMA producer
+        // ---------------- TMA producer: the run's steps in order
         const uint32_t tx = TC_A_BYTES + sh.BN * TC_BK * 2;
-        int kb = 0;
-        for (; kb < sh.nkb; ++kb) {
-            const int s = kb % sh.stages, r = kb / sh.stages;
-            if (r > 0 && !mbar_wait(empty0 + 8 * s, (r - 1) & 1)) {
+        int i = 0;
+        const int n = (int)(s1 - s0);
+        for (; i < n; ++i) {
+            const int st = i % sh.stages, r = i / sh.stages;
+            if (r > 0 && !mbar_wait(empty0 + 8 * st, (r - 1) & 1)) {
                 atomicOr(&g_dev_err, ERR_PRODUCER);
                 break;
             }
-            const uint32_t a = smem_u32(base + s * stage_bytes);
+            const int64_t step = s0 + i;
+            const int tile = (int)(step / sh.nkb), kb = (int)(step - (int64_t)tile * sh.nkb);
+            const int ct = tile / sh.nh, hb = tile - ct * sh.nh;
+            const int h0 = hb * TC_CH, tok0 = ct * TC_MAXN;
+            const uint32_t a = smem_u32(base + st * stage_bytes);
             const uint32_t b = a + TC_A_BYTES;
-            mbar_expect_tx(full0 + 8 * s, tx);
-            // each CTA starts its K walk at its own offset, so the CTAs do
-            // not all request the same token tile from L2 at the same time
-            const int kp = (kb + blockIdx.x * 7) % sh.nkb;
-            tma_load_2d(a, &map_w, kp * TC_BK, h0, full0 + 8 * s);
-            tma_load_2d(a + TC_A_BYTES / 2, &map_w, kp * TC_BK, sh.H + h0, full0 + 8 * s);
-            tma_load_2d(b, &map_x, kp * TC_BK, tok0, full0 + 8 * s);
+            mbar_expect_tx(full0 + 8 * st, tx);
+            tma_load_2d(a, &map_w, kb * TC_BK, h0, full0 + 8 * st);
+            tma_load_2d(a + TC_A_BYTES / 2, &map_w, kb * TC_BK, sh.H + h0, full0 + 8 * st);
+            tma_load_2d(b, &map_x, kb * TC_BK, tok0, full0 + 8 * st);
         }
         // drain: the last loads in flight have landed once their stages are
         // consumed (bounded; only a failed MMA thread leaves them pending)
-        for (int k = (kb > sh.stages ? kb - sh.stages : 0); k < kb; ++k) {
-            const int s = k % sh.stages, r = k / sh.stages;
-            if (!mbar_wait(empty0 + 8 * s, r & 1)) {
+        for (int k = (i > sh.stages ? i - sh.stages : 0); k < i; ++k) {
+            const int st = k % sh.stages, r = k / sh.stages;
+            if (!mbar_wait(empty0 + 8 * st, r & 1)) {
                 atomicOr(&g_dev_err, ERR_DRAIN);
                 break;
             }
         }
     } else if (warp == 1 && lane == 0) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer: segment j accumulates in buffer j & 1
         const uint32_t idesc = instr_desc(TC_BM, sh.BN);
-        for (int kb = 0; kb < sh.nkb; ++kb) {
-            const int s = kb % sh.stages, r = kb / sh.stages;
-            if (!mbar_wait(full0 + 8 * s, r & 1)) {
+        int i = 0, j = 0;
+        bool ok = true;
+        for (int64_t sg = s0; sg < s1 && ok; ++j) {
+            const int tile = (int)(sg / sh.nkb);
+            const int klo = (int)(sg - (int64_t)tile * sh.nkb);
+            const int khi = (int)min((int64_t)sh.nkb, s1 - (int64_t)tile * sh.nkb);
+            const int buf = j & 1;
+            if (j >= 2 && !mbar_wait(tempty0 + 8 * buf, ((j - 2) >> 1) & 1)) {
                 atomicOr(&g_dev_err, ERR_MMA);
                 break;
             }
             tc_fence_after();
-            const uint32_t a = smem_u32(base + s * stage_bytes);
-            const uint32_t b = a + TC_A_BYTES;
+            const uint32_t d = tmem + (uint32_t)(buf * sh.bufcols);
+            for (int kb = klo; kb < khi; ++kb, ++i) {
+                const int st = i % sh.stages, r = i / sh.stages;
+                if (!mbar_wait(full0 + 8 * st, r & 1)) {
+                    atomicOr(&g_dev_err, ERR_MMA);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a = smem_u32(base + st * stage_bytes);
+                const uint32_t b = a + TC_A_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < TC_BK / 16; ++kk)
-                mma_bf16(tmem, smem_desc(a + kk * 32), smem_desc(b + kk * 32), idesc,
-                         (kb > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(empty0 + 8 * s);
+                for (int kk = 0; kk < TC_BK / 16; ++kk)
+                    mma_bf16(d, smem_desc(a + kk * 32), smem_desc(b + kk * 32), idesc,
+                             (kb > klo || kk > 0) ? 1u : 0u);
+                mma_commit(empty0 + 8 * st);
+            }
+            if (ok) mma_commit(tfull0 + 8 * buf);
+            sg = (int64_t)tile * sh.nkb + khi;
         }
-        mma_commit(accf);
+        mma_commit(mdone);  // every MMA this thread issued has completed once this fires
     } else if (warp >= 4) {
-        // ---------------- epilogue: 32 token columns at a time, TMEM -> shared
-        // (a in rows 0..63, b in rows 64..127), then each thread takes
-        // (token, 8-channel group) items with 16-byte loads of x_t and x_{t-1}
-        // and one 16-byte store of the 8 outputs.
+        // ---------------- epilogue
         const int q = warp - 4;  // TMEM lanes 32q .. 32q + 31
         const int e = threadIdx.x - 128;
-        bool ok = mbar_wait(accf, 0);
-        if (!ok) atomicOr(&g_dev_err, ERR_EPILOGUE);
-        ok = __all_sync(FULL, ok);  // tcgen05.ld is warp-collective
-        tc_fence_after();
-        for (int c0 = 0; c0 < sh.BN; c0 += 32) {
-            if (ok) {
-                float v[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) s_acc[(32 * q + lane) * 33 + j] = v[j];
+        const int row = 32 * q + lane;
+        int j = 0;
+        for (int64_t sg = s0; sg < s1; ++j) {
+            const int tile = (int)(sg / sh.nkb);
+            const int klo = (int)(sg - (int64_t)tile * sh.nkb);
+            const int khi = (int)min((int64_t)sh.nkb, s1 - (int64_t)tile * sh.nkb);
+            sg = (int64_t)tile * sh.nkb + khi;
+            const int buf = j & 1;
+            if (!mbar_wait(tfull0 + 8 * buf, (j >> 1) & 1)) {
+                atomicOr(&g_dev_err, ERR_EPILOGUE);
+                *s_fail = 1;
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (ok) {
+            epi_sync();
+            if (*s_fail) break;  // uniform over the four warps
+            tc_fence_after();
+            const uint32_t tacc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * sh.bufcols);
+            if (klo > 0) {
+                // a run that starts inside the tile: hand the partial to its owner
+                float4* dst = partial + (int64_t)p * sh.ngroups * 8 * TC_BM;
+                for (int g = 0; g < sh.ngroups; ++g) {
+                    float v[32];
+                    tmem_ld32(tacc + 32 * g, v);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        dst[((int64_t)g * 8 + c) * TC_BM + row] =
+                            make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                }
+                tc_fence_before();
+                epi_sync();
+                if (e == 0) {
+                    __threadfence();
+                    st_release(&flags[p], 1u);
+                    mbar_arrive(tempty0 + 8 * buf);
+                }
+                continue;
+            }
+            // owned tile: wait for the runs that start inside it (CTA order = K order)
+            int q_end = p + 1;
+            while (q_end < sh.nctas && run_start(sh, q_end) < (int64_t)(tile + 1) * sh.nkb) ++q_end;
+            if (e == 0) {
+                for (int q2 = p + 1; q2 < q_end; ++q2) {
+                    const uint64_t t0 = global_ns();
+                    while (ld_acquire(&flags[q2]) == 0u) {
+                        if (global_ns() - t0 > WAIT_NS) {
+                            atomicOr(&g_dev_err, ERR_EPILOGUE);
+                            *s_fail = 1;
+                            break;
+                        }
+                    }
+                    if (*s_fail) break;
+                }
+                __threadfence();
+            }
+            epi_sync();
+            const bool have_parts = *s_fail == 0;
+            const int ct = tile / sh.nh, hb = tile - ct * sh.nh;
+            const int h0 = hb * TC_CH, tok0 = ct * TC_MAXN;
+            for (int g = 0; g < sh.ngroups; ++g) {
+                float v[32];
+                tmem_ld32(tacc + 32 * g, v);
+                if (have_parts)
+                    for (int q2 = p + 1; q2 < q_end; ++q2) {
+                        const float4* src = partial + (int64_t)q2 * sh.ngroups * 8 * TC_BM;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const float4 w = __ldcg(&src[((int64_t)g * 8 + c) * TC_BM + row]);
+                            v[4 * c] += w.x;
+                            v[4 * c + 1] += w.y;
+                            v[4 * c + 2] += w.z;
+                            v[4 * c + 3] += w.w;
+                        }
+                    }
+#pragma unroll
+                for (int c = 0; c < 32; ++c) s_acc[row * 33 + c] = v[c];
+                epi_sync();
+                // (token, 8-channel group) items: a in rows 0..63, b in rows 64..127
 #pragma unroll
                 for (int rep = 0; rep < 2; ++rep) {
                     const int it = e + 128 * rep;
-                    const int j = it >> 3, g = it & 7;
-                    const int tok = tok0 + c0 + j;
-                    if (tok < sh.ntok) {
-                        const int h = h0 + 8 * g;
+                    const int jj = it >> 3, gg = it & 7;
+                    const int tok = tok0 + 32 * g + jj;
+                    if (32 * g + jj < sh.BN && tok < sh.ntok) {
+                        const int h = h0 + 8 * gg;
                         const int bi = tok / sh.T;
                         const uint4 xv = *(const uint4*)(x + (int64_t)tok * sh.H + h);
                         const uint4 pv = (tok == bi * sh.T)
@@ -230,9 +355,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
                                 const uint32_t xb = (u ? (xw[c >> 1] & 0xFFFF0000u) : (xw[c >> 1] << 16));
                                 const uint32_t pb = (u ? (pw[c >> 1] & 0xFFFF0000u) : (pw[c >> 1] << 16));
                                 const float xc = __uint_as_float(xb), xp = __uint_as_float(pb);
-                                const float a = s_acc[(8 * g + c + u) * 33 + j];
-                                const float b = s_acc[(64 + 8 * g + c + u) * 33 + j];
-                                y2[u] = fmaf(b, xp, fmaf(a, xc, xc));
+                                const float a = s_acc[(8 * gg + c + u) * 33 + jj];
+                                const float bb = s_acc[(64 + 8 * gg + c + u) * 33 + jj];
+                                y2[u] = fmaf(bb, xp, fmaf(a, xc, xc));
                             }
                             const __nv_bfloat162 pr = __floats2bfloat162_rn(y2[0], y2[1]);
                             ow[c >> 1] = *(const uint32_t*)&pr;
@@ -240,13 +365,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
                         *(uint4*)(out + (int64_t)tok * sh.H + h) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                     }
                 }
+                epi_sync();
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            tc_fence_before();
+            epi_sync();
+            if (e == 0) mbar_arrive(tempty0 + 8 * buf);
         }
-        tc_fence_before();
     }
     __syncthreads();
     if (warp == 2) {
+        // every MMA has completed before TMEM goes back (bounded)
+        if (!mbar_wait(mdone, 0)) atomicOr(&g_dev_err, ERR_DRAIN);
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols));
     }
@@ -292,37 +421,92 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, ui
 
 }  // namespace
 
+// Stream-K plan of one call: token chunks of up to 256 (the accumulator
+// width), 64-channel tiles, 64-wide K blocks; one CTA per SM (at most
+// TC_MAXCTA) and never more CTAs than steps.
+struct TcPlan {
+    int BN, ngroups, bufcols, nh, nkb, nctas;
+    int64_t steps;
+    size_t flags_bytes, part_bytes;
+};
+static TcPlan tc_plan(int64_t ntok, int H, int sms) {
+    using namespace dfl;
+    TcPlan P;
+    const int64_t nt = (ntok + TC_MAXN - 1) / TC_MAXN;
+    const int64_t chunk_tok = nt > 1 ? TC_MAXN : ntok;
+    P.BN = (int)(((chunk_tok + 15) / 16) * 16);
+    P.ngroups = (P.BN + 31) / 32;
+    P.bufcols = 32;
+    while (P.bufcols < P.BN) P.bufcols *= 2;
+    P.nh = H / TC_CH;
+    P.nkb = H / TC_BK;
+    P.steps = nt * P.nh * P.nkb;
+    P.nctas = (int)std::min<int64_t>(std::min(sms, TC_MAXCTA), P.steps);
+    P.flags_bytes = (size_t)TC_MAXCTA * 4;
+    P.part_bytes = (size_t)P.nctas * P.ngroups * 8 * TC_BM * sizeof(float4);
+    return P;
+}
+
+// Workspace of the bf16 path, sized for TC_MAXCTA CTAs so that it does not
+// depend on the device.
+size_t dflash2_dynconv2_tc_workspace(int64_t ntok, int H) {
+    const TcPlan P = tc_plan(ntok, H, dfl::TC_MAXCTA);
+    return P.flags_bytes + P.part_bytes;
+}
+
 // Launches the tensor-core path for bf16 operands (H a multiple of 64,
-// 16-byte aligned pointers, checked by the caller).  Returns a dflash2 status.
+// 16-byte aligned pointers and a large enough 256-byte aligned workspace,
+// checked by the caller).  Returns a dflash2 status.
 int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_tap, int B, int T,
-                               int H, void* out, cudaStream_t s) {
+                               int H, void* out, void* ws, cudaStream_t s) {
     using namespace dfl;
     const int ntok = B * T;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DFLASH2_ECUDA;
+    const TcPlan P = tc_plan(ntok, H, sms);
     CUtensorMap mw, mx;
-    const int n_chunks_tok = (ntok + TC_MAXN - 1) / TC_MAXN;
-    const int chunk_tok = n_chunks_tok > 1 ? TC_MAXN : ntok;
-    const int BN = ((chunk_tok + 15) / 16) * 16;
     if (!make_map(&mw, w_tap, (uint64_t)H, (uint64_t)2 * H, TC_BK, TC_CH)) return DFLASH2_ECUDA;
-    if (!make_map(&mx, x, (uint64_t)H, (uint64_t)ntok, TC_BK, (uint32_t)BN)) return DFLASH2_ECUDA;
-    const int stage_bytes = TC_A_BYTES + BN * TC_BK * 2;
+    if (!make_map(&mx, x, (uint64_t)H, (uint64_t)ntok, TC_BK, (uint32_t)P.BN)) return DFLASH2_ECUDA;
+    const int stage_bytes = TC_A_BYTES + P.BN * TC_BK * 2;
     const int fixed = 1024 + TC_BM * 33 * 4 + 64 * 8 + 16;
     int stages = (227 * 1024 - fixed) / stage_bytes;
     stages = stages > 8 ? 8 : stages;
     if (stages < 2) return DFLASH2_ESHAPE;
     const int smem = fixed + stages * stage_bytes;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(dynconv2_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 227 * 1024) != cudaSuccess)
-            return DFLASH2_ECUDA;
-        attr_set = true;
+    {
+        static std::mutex mu;
+        static bool attr_set[64] = {};
+        std::lock_guard<std::mutex> g(mu);
+        if (dev < 64 && !attr_set[dev]) {
+            if (cudaFuncSetAttribute(dynconv2_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     227 * 1024) != cudaSuccess)
+                return DFLASH2_ECUDA;
+            attr_set[dev] = true;
+        }
     }
-    TcShape sh{H, T, ntok, 0, BN, stages, H / TC_BK};
-    dim3 grid((unsigned)(H / TC_CH), (unsigned)n_chunks_tok);
-    dynconv2_tc_kernel<<<grid, TC_THREADS, smem, s>>>(mw, mx, (const __nv_bfloat16*)x,
-                                                      (const __nv_bfloat16*)x_prev,
-                                                      (__nv_bfloat16*)out, sh);
-    return cudaGetLastError() == cudaSuccess ? DFLASH2_OK : DFLASH2_ECUDA;
+    unsigned* flags = (unsigned*)ws;
+    float4* part = (float4*)((char*)ws + P.flags_bytes);
+    if (cudaMemsetAsync(flags, 0, (size_t)P.nctas * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
+    TcShape sh{H, T, ntok, P.BN, stages, P.nkb, P.nh, P.bufcols, P.ngroups, P.nctas, P.steps};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)P.nctas);
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    // cooperative: every CTA is resident, so an owner's bounded wait for a
+    // later CTA's partial always has a running producer
+    cudaLaunchAttribute a[1];
+    a[0].id = cudaLaunchAttributeCooperative;
+    a[0].val.cooperative = 1;
+    cfg.attrs = a;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, dynconv2_tc_kernel, mw, mx, (const __nv_bfloat16*)x,
+                           (const __nv_bfloat16*)x_prev, (__nv_bfloat16*)out, sh, part,
+                           flags) != cudaSuccess)
+        return DFLASH2_ECUDA;
+    return DFLASH2_OK;
 }
 
 unsigned dfl_errors_dynconv(int clear) {

@@ -199,10 +199,12 @@ __device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm, f
     }
     if (exact) chunk_top16_exact<BF16>(ch, m, sm);
 
-    // pass 2: sum of exp2(x c - M c) (fixed order)
+    // pass 2: sum of exp2(x c - M c) (fixed order), each exponent one FMA
+    // against mc = fl(M c); the product's rounding error M c - mc (exact in
+    // fp32) is taken out of the sum once per chunk below.
     float s = 0.0f;
+    const float mc = M * c2;
     if (M != -INFINITY) {
-        const float mc = M * c2;
 #pragma unroll
         for (int i = 0; i < R::NV; ++i) {
             const uint4 v4 = ch.vec(i);
@@ -224,7 +226,7 @@ __device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm, f
 #pragma unroll
     for (int w = 0; w < NT / 32; ++w) S += sm.wsum[w];
     chunk_m = M;
-    chunk_s = S;
+    chunk_s = (M != -INFINITY) ? S * ex2(-fmaf(M, c2, -mc)) : S;
     if (t == 0) sm.ncand = 0;  // read by everyone before D; next pushes come after
 }
 

@@ -68,8 +68,8 @@ inline Layout greedy_layout(int B, int G, int64_t V) {
 }
 inline Layout sample_layout(int B, int G, int64_t V) {
     int64_t S = n_chunks(V);
-    return make_layout((size_t)B * 2 * 4, (size_t)((int64_t)B * (2 * G + 1) * S) * sizeof(LseD),
-                       (size_t)((int64_t)B * S) * 2 * sizeof(double), (size_t)B * sizeof(SampleInfo));
+    return make_layout((size_t)B * 4, (size_t)((int64_t)B * (2 * G + 1) * S) * sizeof(LseD), 0,
+                       (size_t)B * sizeof(SampleInfo));
 }
 inline Layout select_layout(int B, int G) {
     return make_layout((size_t)B * 4, (size_t)B * (K + (size_t)K * K * (G - 1)) * sizeof(float));

@@ -162,7 +162,7 @@ DFLASH2_API int dflash2_topk_softmax_noalloc(const void* logits, int dtype, int6
  *
  * idx, logp   [B, G, 16] as written by dflash2_topk_softmax (c = idx).
  * anchor      [B] int32 last accepted token per sequence, or NULL (no term).
- * emb         [V, d] of `emb_dtype`; d in {64, 128}.
+ * emb         [V, d] of `emb_dtype`, 16-byte aligned; d in {64, 128}.
  * W           [d, d] float, row-major (W[j][l] at j * d + l), 16-byte aligned.
  * B >= 0, 1 <= G < DFLASH2_MAX_BLOCK.
  * path_tok    [B, G] int32 chosen tokens; path_rank [B, G] int32 their ranks;
@@ -210,7 +210,8 @@ DFLASH2_API int dflash2_verify_greedy(const void* target, int dtype, int B, int 
  * for u_j, 1 for u' (position = n).
  *
  * target [B, G+1, V], draft [B, G, V] of `dtype`, rows 16-byte aligned for
- * the fast path; draft_tok [B, G] int32; seq_id [B] uint32 or NULL (= b).
+ * the fast path; V <= 67,108,864 (4096 chunks of 16384; DFLASH2_ESHAPE
+ * above); draft_tok [B, G] int32; seq_id [B] uint32 or NULL (= b).
  * n_accept [B], out_tok [B, G+1] as in dflash2_verify_greedy.
  * ratio_dbg [B, G] float r_j for every j, u_dbg [B, G] float u_j; both
  * optional (NULL).
@@ -229,11 +230,22 @@ DFLASH2_API int dflash2_verify_sample(const void* target, const void* draft, int
  *   [a_t; b_t] = W_tap x_t  (W_tap [2H, H]: rows 0..H-1 give a, H..2H-1 give b)
  *   out_t = x_t + a_t * x_t + b_t * x_{t-1},   x_{-1} = x_prev
  * x [B, T, H], x_prev [B, H], w_tap [2H, H], out [B, T, H], all of `dtype`,
- * 16-byte aligned; H a multiple of 64; B, T >= 0.  fp32 accumulation, one
- * rounding at the output.
+ * 16-byte aligned; H a multiple of 64; B, T >= 0, B * T <= 2^30 - 1.  fp32
+ * accumulation, one rounding at the output.
+ * bf16 runs on the tensor cores with the K dimension of a 64-channel tile
+ * possibly split between SMs; the split depends on B * T, H and the SM
+ * count only, and the parts are added in K order, so a given shape on a
+ * given device always rounds the same way.  It needs a workspace of
+ * dflash2_dynconv2_workspace_bytes bytes (256-byte aligned; contents need
+ * not be initialised; one call at a time per workspace); fp32 needs none
+ * (ws may be NULL).
  */
 DFLASH2_API int dflash2_dynconv2(const void* x, const void* x_prev, const void* w_tap, int dtype, int B,
-                     int T, int H, void* out, dflash2_stream_t stream);
+                     int T, int H, void* out, void* ws, size_t ws_bytes, dflash2_stream_t stream);
+
+/* Workspace bytes dflash2_dynconv2 needs for these arguments (0 when it
+ * needs none or the arguments are invalid). */
+DFLASH2_API size_t dflash2_dynconv2_workspace_bytes(int dtype, int B, int T, int H);
 
 /*
  * Device-side error flags of the kernels on the current device (0 = none).

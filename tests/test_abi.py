@@ -140,8 +140,8 @@ def test_verify_validation(L):
 
 
 def test_dynconv_validation(L):
-    def conv(x=P, xp=P, w=P, dt=1, B=2, T=8, H=5120, out=P2):
-        return L.dflash2_dynconv2(x, xp, w, dt, B, T, H, out, S0)
+    def conv(x=P, xp=P, w=P, dt=1, B=2, T=8, H=5120, out=P2, ws=P2, wsb=1 << 30):
+        return L.dflash2_dynconv2(x, xp, w, dt, B, T, H, out, ws, wsb, S0)
     assert conv(dt=4) == EDTYPE
     assert conv(H=100) == ESHAPE
     assert conv(H=0) == ESHAPE
@@ -149,3 +149,11 @@ def test_dynconv_validation(L):
     assert conv(T=0) == OK
     assert conv(w=None) == EINVAL
     assert conv(x=C.c_void_p(0x10008)) == EALIGN
+    assert conv(ws=None) == EWORKSPACE
+    assert conv(ws=C.c_void_p(0x20010)) == EWORKSPACE   # not 256-aligned
+    assert conv(wsb=1000) == EWORKSPACE
+    # fp32 runs without a workspace
+    assert L.dflash2_dynconv2_workspace_bytes(0, 2, 8, 5120) == 0
+    need = L.dflash2_dynconv2_workspace_bytes(1, 32, 8, 5120)
+    assert need > 0 and need == L.dflash2_dynconv2_workspace_bytes(1, 8, 32, 5120)
+    assert L.dflash2_dynconv2_workspace_bytes(1, 2, 8, 100) == 0

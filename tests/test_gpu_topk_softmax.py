@@ -146,3 +146,21 @@ def test_output_guard_bands(orc):
         assert np.all(h[:pad] == fill) and np.all(h[pad + 48:] == fill)
     hz = to_host(canary_z)
     assert np.all(hz[:pad] == 777.0) and np.all(hz[pad + 3:] == 777.0)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("invT", [1.0, 1.7])
+def test_large_magnitude_logits(orc, dt, invT):
+    """Logits near +-1000 and a one-hot row: the exponent of the row maximum
+    must come out as exactly 0, not as the rounding error of max * c (up to
+    6e-5 at this size, which would scale every probability by 2^6e-5)."""
+    rng = np.random.default_rng(77)
+    V = 2 * 16384 + 7
+    rows = [rng.standard_normal(V) * 2.0 + off for off in (-900.0, 300.0, 1000.0)]
+    hot = np.zeros(V)
+    hot[12345] = 1000.0
+    rows.append(hot)
+    x = np.stack(rows).astype(np.float32)
+    if dt == "bf16":
+        x = synth.to_bf16_bits(x)
+    check_rows(orc, x, invT)

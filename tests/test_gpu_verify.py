@@ -184,6 +184,21 @@ def test_sample_special_cases(orc):
     assert np.all(on == G)
 
 
+def test_sample_large_magnitude_logits(orc):
+    """Logits offset by +-700: ratios and draws must not pick up the rounding
+    error of max * c in the exponent reference."""
+    rng = np.random.default_rng(41)
+    B, G, V = 16, 5, 20000
+    off = np.where(np.arange(B) % 2 == 0, 700.0, -700.0)[:, None, None]
+    t = (rng.standard_normal((B, G + 1, V)) * 1.5 + off).astype(np.float32)
+    q = (t[:, :G] + rng.standard_normal((B, G, V)) * 0.3).astype(np.float32)
+    d = np.argmax(q, axis=2).astype(np.int32)
+    ties = NearTies()
+    check_sample(orc, t, q, d, 3, 1, None, 1.0, 0, ties)
+    check_sample(orc, t, None, d, 3, 2, None, 1.0, 1, ties)
+    print("near-ties:", ties.report())
+
+
 def test_sample_batch_invariance(orc):
     need_cuda()
     w = synth.WORKLOADS["b8"]
