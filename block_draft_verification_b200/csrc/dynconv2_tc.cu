@@ -64,6 +64,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         "l"(map), "r"(c0), "r"(c1), "r"(bar)
         : "memory");
 }
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+        "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+        : "memory");
+}
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), version 1.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
@@ -120,6 +128,7 @@ struct TcShape {
     int bufcols;                           // TMEM columns per accumulator (power of 2, >= BN)
     int ngroups;                           // 32-column groups per accumulator
     int nctas;                             // stream-K CTAs
+    int R;                                 // x_prev rows staged per tile (batches it touches)
     int64_t steps;                         // tiles * nkb
 };
 
@@ -134,10 +143,29 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+// One bf16 from shared memory, widened to fp32 (exact).
+__device__ __forceinline__ float lds_bf16(uint32_t addr) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return __uint_as_float((uint32_t)v << 16);
+}
+__device__ __forceinline__ void sts_bf16(uint32_t addr, float v) {
+    const unsigned short b = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(b) : "memory");
+}
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+    const __grid_constant__ CUtensorMap map_xe, const __grid_constant__ CUtensorMap map_pe,
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ x_prev,
     __nv_bfloat16* __restrict__ out, TcShape sh, float4* __restrict__ partial,
     unsigned* __restrict__ flags) {
@@ -146,10 +174,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int stage_bytes = TC_A_BYTES + sh.BN * TC_BK * 2;
     uint8_t* tail = base + sh.stages * stage_bytes;
-    float* s_acc = (float*)tail;  // [128][33] a, b values of 32 token columns
-    // full[S], empty[S], tmem_full[2], tmem_empty[2], mma_done
-    uint64_t* bars = (uint64_t*)(tail + TC_BM * 33 * 4);
-    uint32_t* s_tmem = (uint32_t*)(bars + 2 * sh.stages + 5);
+    // an owned tile's inputs, row-major 128-byte rows (64 channels):
+    // x of its BN tokens, x_prev of the R batches it touches, x of token tok0-1
+    uint8_t* s_x = tail;
+    uint8_t* s_xp = s_x + sh.BN * 128;
+    uint8_t* s_x0 = s_xp + sh.R * 128;
+    uint8_t* s_out = s_x0 + 128;  // [2][32 tokens][64 channels] bf16 outputs
+    // full[S], empty[S], tmem_full[2], tmem_empty[2], mma_done, x tile
+    uint64_t* bars = (uint64_t*)(s_out + 8192);
+    uint32_t* s_tmem = (uint32_t*)(bars + 2 * sh.stages + 6);
     int* s_fail = (int*)(s_tmem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -159,6 +192,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     const uint32_t tfull0 = smem_u32(bars + 2 * sh.stages);
     const uint32_t tempty0 = tfull0 + 16;
     const uint32_t mdone = tfull0 + 32;
+    const uint32_t xbar = tfull0 + 40;
     const uint32_t ncols = 2 * (uint32_t)sh.bufcols;
 
     if (threadIdx.x == 0) {
@@ -171,6 +205,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
             mbar_init(tempty0 + 8 * i, 1);
         }
         mbar_init(mdone, 1);
+        mbar_init(xbar, 1);
         mbar_fence_init();
         *s_fail = 0;
     }
@@ -203,8 +238,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
             const uint32_t a = smem_u32(base + st * stage_bytes);
             const uint32_t b = a + TC_A_BYTES;
             mbar_expect_tx(full0 + 8 * st, tx);
-            tma_load_2d(a, &map_w, kb * TC_BK, h0, full0 + 8 * st);
-            tma_load_2d(a + TC_A_BYTES / 2, &map_w, kb * TC_BK, sh.H + h0, full0 + 8 * st);
+            // one box of the 4-D view (k, 16 channels, a|b, 16-channel block):
+            // accumulator rows 32q .. 32q+15 are a of channels h0+16q ..
+            // h0+16q+15, rows 32q+16 .. 32q+31 are b of the same channels
+            tma_load_4d(a, &map_w, kb * TC_BK, 0, 0, h0 / 16, full0 + 8 * st);
             tma_load_2d(b, &map_x, kb * TC_BK, tok0, full0 + 8 * st);
         }
         // drain: the last loads in flight have landed once their stages are
@@ -257,13 +294,56 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
         const int q = warp - 4;  // TMEM lanes 32q .. 32q + 31
         const int e = threadIdx.x - 128;
         const int row = 32 * q + lane;
-        int j = 0;
+        int j = 0, nown = 0;  // segments, owned segments (x tile barrier phases)
+        float4 pp0[8], pp1[8];  // the first partial, two groups ahead of its use
         for (int64_t sg = s0; sg < s1; ++j) {
             const int tile = (int)(sg / sh.nkb);
             const int klo = (int)(sg - (int64_t)tile * sh.nkb);
             const int khi = (int)min((int64_t)sh.nkb, s1 - (int64_t)tile * sh.nkb);
             sg = (int64_t)tile * sh.nkb + khi;
             const int buf = j & 1;
+            const int ct = tile / sh.nh, hb = tile - ct * sh.nh;
+            const int h0 = hb * TC_CH, tok0 = ct * TC_MAXN, bi0 = tok0 / sh.T;
+            // runs that start inside an owned tile hand it partials (CTA order = K order)
+            int q_end = p + 1;
+            const float4* part1 = partial + (int64_t)(p + 1) * sh.ngroups * 8 * TC_BM;
+            auto load_part = [&](int g, float4 (&po)[8]) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) po[c] = __ldcg(&part1[((int64_t)g * 8 + c) * TC_BM + row]);
+            };
+            if (klo == 0) {
+                // owned tile, while its MMAs run: stage its x rows, the x_prev
+                // rows of the batches it touches and x of token tok0 - 1 in
+                // shared memory (the previous owned tile's epilogue is done with
+                // them), wait for the partials of later runs and request the
+                // first two groups of the first one
+                if (e == 0 && !*s_fail) {
+                    mbar_expect_tx(xbar, (uint32_t)(sh.BN + sh.R) * 128u);
+                    tma_load_2d(smem_u32(s_x), &map_xe, h0, tok0, xbar);
+                    tma_load_2d(smem_u32(s_xp), &map_pe, h0, tok0 / sh.T, xbar);
+                }
+                if (e < 8 && tok0 > 0)
+                    ((uint4*)s_x0)[e] = *(const uint4*)(x + (int64_t)(tok0 - 1) * sh.H + h0 + 8 * e);
+                while (q_end < sh.nctas && run_start(sh, q_end) < (int64_t)(tile + 1) * sh.nkb) ++q_end;
+                if (e == 0) {
+                    for (int q2 = p + 1; q2 < q_end && !*s_fail; ++q2) {
+                        const uint64_t t0 = global_ns();
+                        while (ld_acquire(&flags[q2]) == 0u) {
+                            if (global_ns() - t0 > WAIT_NS) {
+                                atomicOr(&g_dev_err, ERR_EPILOGUE);
+                                *s_fail = 1;
+                                break;
+                            }
+                        }
+                    }
+                    __threadfence();
+                }
+                epi_sync();
+                if (!*s_fail && q_end > p + 1) {
+                    load_part(0, pp0);
+                    if (sh.ngroups > 1) load_part(1, pp1);
+                }
+            }
             if (!mbar_wait(tfull0 + 8 * buf, (j >> 1) & 1)) {
                 atomicOr(&g_dev_err, ERR_EPILOGUE);
                 *s_fail = 1;
@@ -292,32 +372,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
                 }
                 continue;
             }
-            // owned tile: wait for the runs that start inside it (CTA order = K order)
-            int q_end = p + 1;
-            while (q_end < sh.nctas && run_start(sh, q_end) < (int64_t)(tile + 1) * sh.nkb) ++q_end;
-            if (e == 0) {
-                for (int q2 = p + 1; q2 < q_end; ++q2) {
-                    const uint64_t t0 = global_ns();
-                    while (ld_acquire(&flags[q2]) == 0u) {
-                        if (global_ns() - t0 > WAIT_NS) {
-                            atomicOr(&g_dev_err, ERR_EPILOGUE);
-                            *s_fail = 1;
-                            break;
-                        }
-                    }
-                    if (*s_fail) break;
-                }
-                __threadfence();
+            if (!mbar_wait(xbar, (uint32_t)(nown & 1))) {  // the staged x, x_prev rows
+                atomicOr(&g_dev_err, ERR_EPILOGUE);
+                *s_fail = 1;
             }
+            ++nown;
             epi_sync();
-            const bool have_parts = *s_fail == 0;
-            const int ct = tile / sh.nh, hb = tile - ct * sh.nh;
-            const int h0 = hb * TC_CH, tok0 = ct * TC_MAXN;
+            const bool first_part = *s_fail == 0 && q_end > p + 1;
+            // lane l of epilogue warp q: channel cl = 16q + (l & 15) of the tile,
+            // tokens 16 (l >> 4) .. +15 of each 32-token group; a and b of the
+            // channel meet by one exchange between lanes l and l ^ 16
+            const int cl = 16 * q + (lane & 15), half = lane >> 4;
             for (int g = 0; g < sh.ngroups; ++g) {
                 float v[32];
                 tmem_ld32(tacc + 32 * g, v);
-                if (have_parts)
-                    for (int q2 = p + 1; q2 < q_end; ++q2) {
+                if (first_part) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        v[4 * c] += pp0[c].x;
+                        v[4 * c + 1] += pp0[c].y;
+                        v[4 * c + 2] += pp0[c].z;
+                        v[4 * c + 3] += pp0[c].w;
+                        pp0[c] = pp1[c];
+                    }
+                    if (g + 2 < sh.ngroups) load_part(g + 2, pp1);
+                    for (int q2 = p + 2; q2 < q_end; ++q2) {  // further partials, in K order
                         const float4* src = partial + (int64_t)q2 * sh.ngroups * 8 * TC_BM;
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
@@ -328,44 +407,54 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
                             v[4 * c + 3] += w.w;
                         }
                     }
+                }
+                float av[16], bv[16];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) s_acc[row * 33 + c] = v[c];
-                epi_sync();
-                // (token, 8-channel group) items: a in rows 0..63, b in rows 64..127
+                for (int t = 0; t < 16; ++t) {
+                    const float recv = __shfl_xor_sync(FULL, half ? v[t] : v[16 + t], 16);
+                    av[t] = half ? recv : v[t];
+                    bv[t] = half ? v[16 + t] : recv;
+                }
+                const int jt0 = 32 * g + 16 * half;
+                const int tokf = tok0 + jt0, bif = tokf / sh.T;
+                // every shared-memory read first (branch-free, so they overlap):
+                // x of tokens jt0-1 .. jt0+15, and x_prev of each token's batch
+                float xv[17], pv[16];
+                xv[0] = jt0 == 0 ? lds_bf16(smem_u32(s_x0) + 2 * cl)
+                                 : lds_bf16(smem_u32(s_x) + (min(jt0, sh.BN) - 1) * 128 + 2 * cl);
+                bool bstart[16];
+                {
+                    int ti = tokf - bif * sh.T, bl = bif - bi0;
 #pragma unroll
-                for (int rep = 0; rep < 2; ++rep) {
-                    const int it = e + 128 * rep;
-                    const int jj = it >> 3, gg = it & 7;
-                    const int tok = tok0 + 32 * g + jj;
-                    if (32 * g + jj < sh.BN && tok < sh.ntok) {
-                        const int h = h0 + 8 * gg;
-                        const int bi = tok / sh.T;
-                        const uint4 xv = *(const uint4*)(x + (int64_t)tok * sh.H + h);
-                        const uint4 pv = (tok == bi * sh.T)
-                                             ? *(const uint4*)(x_prev + (int64_t)bi * sh.H + h)
-                                             : *(const uint4*)(x + (int64_t)(tok - 1) * sh.H + h);
-                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                        const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
-                        uint32_t ow[4];
-#pragma unroll
-                        for (int c = 0; c < 8; c += 2) {
-                            float y2[2];
-#pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const uint32_t xb = (u ? (xw[c >> 1] & 0xFFFF0000u) : (xw[c >> 1] << 16));
-                                const uint32_t pb = (u ? (pw[c >> 1] & 0xFFFF0000u) : (pw[c >> 1] << 16));
-                                const float xc = __uint_as_float(xb), xp = __uint_as_float(pb);
-                                const float a = s_acc[(8 * gg + c + u) * 33 + jj];
-                                const float bb = s_acc[(64 + 8 * gg + c + u) * 33 + jj];
-                                y2[u] = fmaf(bb, xp, fmaf(a, xc, xc));
-                            }
-                            const __nv_bfloat162 pr = __floats2bfloat162_rn(y2[0], y2[1]);
-                            ow[c >> 1] = *(const uint32_t*)&pr;
+                    for (int t = 0; t < 16; ++t) {
+                        const int jt = min(jt0 + t, sh.BN - 1);
+                        xv[t + 1] = lds_bf16(smem_u32(s_x) + jt * 128 + 2 * cl);
+                        bstart[t] = ti == 0;
+                        pv[t] = lds_bf16(smem_u32(s_xp) + min(bl, sh.R - 1) * 128 + 2 * cl);
+                        if (++ti == sh.T) {
+                            ti = 0;
+                            ++bl;
                         }
-                        *(uint4*)(out + (int64_t)tok * sh.H + h) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                     }
                 }
+                // the 16 outputs of this lane into the group's output tile
+                // [32 tokens][64 channels] bf16 (double-buffered by group)
+                const uint32_t ob = smem_u32(s_out) + (g & 1) * 4096 + (16 * half) * 128 + 2 * cl;
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const float xc = xv[t + 1], xm = bstart[t] ? pv[t] : xv[t];
+                    sts_bf16(ob + t * 128, fmaf(bv[t], xm, fmaf(av[t], xc, xc)));
+                }
                 epi_sync();
+                // 16-byte rows out: item = (token, 8-channel group)
+#pragma unroll
+                for (int rep = 0; rep < 2; ++rep) {
+                    const int it = e + 128 * rep, tl = it >> 3, gg = it & 7;
+                    const int jt = 32 * g + tl, tok = tok0 + jt;
+                    if (jt < sh.BN && tok < sh.ntok)
+                        *(uint4*)(out + (int64_t)tok * sh.H + h0 + 8 * gg) =
+                            lds_v4(smem_u32(s_out) + (g & 1) * 4096 + tl * 128 + 16 * gg);
+                }
             }
             tc_fence_before();
             epi_sync();
@@ -407,7 +496,7 @@ EncodeTiledFn encode_fn() {
 }
 
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_inner,
-              uint32_t box_rows) {
+              uint32_t box_rows, bool swizzle = true) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {inner, rows};
@@ -415,7 +504,24 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, ui
     cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// W_tap [2H, H] seen as (k, r, ab, blk): row = ab * H + 16 * blk + r; one box
+// (64, 16, 2, 4) is a 64-channel tile with a and b rows interleaved in
+// 16-row runs, 128-byte swizzle.
+bool make_wmap(CUtensorMap* m, const void* w, int H) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const uint64_t rb = (uint64_t)H * 2;  // bytes per W row
+    cuuint64_t dims[4] = {(cuuint64_t)H, 16, 2, (cuuint64_t)H / 16};
+    cuuint64_t strides[3] = {rb, rb * H, rb * 16};
+    cuuint32_t box[4] = {64, 16, 2, 4};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(w), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -467,10 +573,17 @@ int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_
         return DFLASH2_ECUDA;
     const TcPlan P = tc_plan(ntok, H, sms);
     CUtensorMap mw, mx;
-    if (!make_map(&mw, w_tap, (uint64_t)H, (uint64_t)2 * H, TC_BK, TC_CH)) return DFLASH2_ECUDA;
+    if (!make_wmap(&mw, w_tap, H)) return DFLASH2_ECUDA;
     if (!make_map(&mx, x, (uint64_t)H, (uint64_t)ntok, TC_BK, (uint32_t)P.BN)) return DFLASH2_ECUDA;
+    // epilogue staging: an owned tile's x rows and the x_prev rows of the
+    // (at most R) batches its tokens belong to, 128 bytes per row, unswizzled
+    const int R = std::min(B, (P.BN - 1 + T - 1) / T + 1);
+    CUtensorMap mxe, mpe;
+    if (!make_map(&mxe, x, (uint64_t)H, (uint64_t)ntok, TC_CH, (uint32_t)P.BN, false) ||
+        !make_map(&mpe, x_prev, (uint64_t)H, (uint64_t)B, TC_CH, (uint32_t)R, false))
+        return DFLASH2_ECUDA;
     const int stage_bytes = TC_A_BYTES + P.BN * TC_BK * 2;
-    const int fixed = 1024 + TC_BM * 33 * 4 + 64 * 8 + 16;
+    const int fixed = 1024 + (P.BN + R + 1) * 128 + 8192 + 64 * 8 + 16;
     int stages = (227 * 1024 - fixed) / stage_bytes;
     stages = stages > 8 ? 8 : stages;
     if (stages < 2) return DFLASH2_ESHAPE;
@@ -489,7 +602,7 @@ int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_
     unsigned* flags = (unsigned*)ws;
     float4* part = (float4*)((char*)ws + P.flags_bytes);
     if (cudaMemsetAsync(flags, 0, (size_t)P.nctas * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
-    TcShape sh{H, T, ntok, P.BN, stages, P.nkb, P.nh, P.bufcols, P.ngroups, P.nctas, P.steps};
+    TcShape sh{H, T, ntok, P.BN, stages, P.nkb, P.nh, P.bufcols, P.ngroups, P.nctas, R, P.steps};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)P.nctas);
     cfg.blockDim = dim3(TC_THREADS);
@@ -502,7 +615,7 @@ int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_
     a[0].val.cooperative = 1;
     cfg.attrs = a;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, dynconv2_tc_kernel, mw, mx, (const __nv_bfloat16*)x,
+    if (cudaLaunchKernelEx(&cfg, dynconv2_tc_kernel, mw, mx, mxe, mpe, (const __nv_bfloat16*)x,
                            (const __nv_bfloat16*)x_prev, (__nv_bfloat16*)out, sh, part,
                            flags) != cudaSuccess)
         return DFLASH2_ECUDA;

@@ -17,10 +17,13 @@
 // One CTA per (sequence, position i): one TMA bulk copy brings W (fp32,
 // 64 KB at d = 128) into shared memory while the threads gather the left
 // embeddings (the anchor for i = 0, else the 16 candidates of position i-1)
-// and the 16 right ones; then F = E_left W and S_i = F E_right^T from shared
-// memory, and S_i goes to the workspace.  The last CTA of the
-// sequence (arrival ticket) runs the recursion in one warp, lane k = state k,
-// in fp64, and backtracks.
+// and the 16 right ones with 16-byte loads issued together; then
+// F = E_left W and S_i = F E_right^T from shared memory, and S_i goes to the
+// workspace.  The last CTA of the sequence (arrival ticket) fetches every S_i,
+// logp and the candidate ids of the sequence into shared memory in one
+// parallel pass, runs the recursion in one warp from there (lane k = state k,
+// fp64), backtracks in shared memory and writes the path with one store per
+// position.
 #include "common.cuh"
 #include "stream.cuh"
 #include "workspace.cuh"
@@ -33,102 +36,163 @@ __global__ void __launch_bounds__(NT, 2) pair_select_kernel(
     const int32_t* __restrict__ anchor, const void* __restrict__ emb, const float* __restrict__ W,
     int G, int32_t* __restrict__ path_tok, int32_t* __restrict__ path_rank,
     float* __restrict__ path_score, float* __restrict__ scores, unsigned* __restrict__ counters) {
-    constexpr int LD = D + 1;  // padded rows: conflict-free column walks
-    extern __shared__ __align__(128) float s_w[];  // W [D][D]
-    __shared__ float s_left[K][LD], s_right[K][LD], s_f[K][LD];
-    __shared__ int32_t s_ltok[K], s_rtok[K];
+    constexpr int LD = D + 4;                  // padded rows, still 16-byte aligned
+    constexpr int ES = EMB_BF16 ? 2 : 4;
+    constexpr int VE = 16 / ES;                // elements per 16-byte vector
+    constexpr int RV = D / VE;                 // vectors per embedding row
+    constexpr int IPT = (2 * K * RV + NT - 1) / NT;
+    // W [D][D] in phase 1; the sequence's pair scores in phase 2
+    extern __shared__ __align__(128) float s_dyn[];
+    __shared__ __align__(16) float s_left[K][LD];
+    __shared__ __align__(16) float s_right[K][LD];
+    __shared__ __align__(16) float s_f[K][LD];
+    __shared__ int32_t s_tok[2 * K];           // right rows 0..15, left rows 16..
+    __shared__ float s_lp[DFLASH2_MAX_BLOCK * K];
+    __shared__ int32_t s_cand[DFLASH2_MAX_BLOCK * K];
+    __shared__ double s_delta[2][K];
     __shared__ uint8_t s_back[DFLASH2_MAX_BLOCK][K];
+    __shared__ int s_path[DFLASH2_MAX_BLOCK];
     __shared__ __align__(8) uint64_t s_bar;
+    __shared__ int s_bad;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int b = blockIdx.x / G, i = blockIdx.x - b * G;
     const int32_t* cand = idx + (int64_t)b * G * K;
     const int nl = (i == 0) ? 1 : K;
     const bool has_left = (i > 0) || (anchor != nullptr);
-    float* out = scores + (int64_t)b * (K + (int64_t)K * K * (G - 1)) +
-                 (i == 0 ? 0 : K + (int64_t)K * K * (i - 1));
+    const int64_t seq_scores = K + (int64_t)K * K * (G - 1);
+    float* out = scores + (int64_t)b * seq_scores + (i == 0 ? 0 : K + (int64_t)K * K * (i - 1));
 
+    bool ok = true;
     if (has_left) {
         const uint32_t bar = smem_u32(&s_bar);
         if (t == 0) {
             mbar_init(bar, 1);
             mbar_fence_init();
-            bulk_g2s(smem_u32(s_w), W, (uint32_t)(D * D * 4), bar);
+            bulk_g2s(smem_u32(s_dyn), W, (uint32_t)(D * D * 4), bar);
         }
-        if (t < K) {
-            s_rtok[t] = cand[i * K + t];
-            if (t < nl) s_ltok[t] = (i == 0) ? anchor[b] : cand[(i - 1) * K + t];
-        }
+        if (t < K) s_tok[t] = cand[i * K + t];
+        else if (t < K + nl) s_tok[t] = (i == 0) ? anchor[b] : cand[(i - 1) * K + (t - K)];
         __syncthreads();
-        auto ld_emb = [&](int32_t tok, int j) -> float {
-            const int64_t o = (int64_t)tok * D + j;
-            if (EMB_BF16)
-                return __uint_as_float((uint32_t)__ldg((const unsigned short*)emb + o) << 16);
-            return __ldg((const float*)emb + o);
-        };
-        for (int e = t; e < K * D; e += NT) {
-            const int k = e / D, j = e - k * D;
-            s_right[k][j] = ld_emb(s_rtok[k], j);
-            if (k < nl) s_left[k][j] = ld_emb(s_ltok[k], j);
+        uint4 v[IPT];
+#pragma unroll
+        for (int q = 0; q < IPT; ++q) {  // all loads first: one memory round trip
+            const int e = t + q * NT, r = e / RV, c = e - r * RV;
+            if (r < K + nl)
+                v[q] = __ldg((const uint4*)((const char*)emb + (int64_t)s_tok[r] * (D * ES)) + c);
         }
-        const bool ok = __syncthreads_and(mbar_wait(bar, 0));
+#pragma unroll
+        for (int q = 0; q < IPT; ++q) {
+            const int e = t + q * NT, r = e / RV, c = e - r * RV;
+            if (r < K + nl) {
+                float4* dst = reinterpret_cast<float4*>((r < K) ? &s_right[r][c * VE]
+                                                                : &s_left[r - K][c * VE]);
+                const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+                if (EMB_BF16) {
+                    dst[0] = make_float4(__uint_as_float(w[0] << 16), __uint_as_float(w[0] & 0xFFFF0000u),
+                                         __uint_as_float(w[1] << 16), __uint_as_float(w[1] & 0xFFFF0000u));
+                    dst[1] = make_float4(__uint_as_float(w[2] << 16), __uint_as_float(w[2] & 0xFFFF0000u),
+                                         __uint_as_float(w[3] << 16), __uint_as_float(w[3] & 0xFFFF0000u));
+                } else {
+                    dst[0] = make_float4(__uint_as_float(w[0]), __uint_as_float(w[1]),
+                                         __uint_as_float(w[2]), __uint_as_float(w[3]));
+                }
+            }
+        }
+        ok = __syncthreads_and(mbar_wait(bar, 0));
         if (!ok) {  // W never arrived: flag it, leave this position's scores unset
             if (t == 0) atomicOr(&g_dev_err, ERR_STREAM);
         } else {
-            // F = E_left W: thread -> column l, a group of left rows
-            constexpr int GROUPS = NT / D;  // 2 for d = 128, 4 for d = 64
-            constexpr int RPG = K / GROUPS;  // rows per group
-            const int l = t % D, g = t / D;
-            float acc[RPG];
+            // F = E_left W: thread -> 4 columns (a quad) of 16 / (NT / (D / 4)) left
+            // rows; each step of 4 along j reads 4 W rows and the rows' 4
+            // embedding values as 16-byte words (j ascending, one FMA chain
+            // per output)
+            constexpr int QUADS = D / 4;               // 32 for d = 128, 16 for d = 64
+            constexpr int RPT = K / (NT / QUADS);      // rows per thread: 2 or 1
+            const int cq = t % QUADS, r0 = (t / QUADS) * RPT;
+            const float4* w4 = reinterpret_cast<const float4*>(s_dyn);
+            if (r0 < nl) {
+                float4 acc[RPT];
 #pragma unroll
-            for (int q = 0; q < RPG; ++q) acc[q] = 0.0f;
-            if (g * RPG < nl) {
-#pragma unroll 8
-                for (int j = 0; j < D; ++j) {
-                    const float w = s_w[j * D + l];
+                for (int q = 0; q < RPT; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+                for (int j = 0; j < D; j += 4) {
+                    const float4 wj[4] = {w4[(j + 0) * QUADS + cq], w4[(j + 1) * QUADS + cq],
+                                          w4[(j + 2) * QUADS + cq], w4[(j + 3) * QUADS + cq]};
 #pragma unroll
-                    for (int q = 0; q < RPG; ++q) acc[q] = fmaf(s_left[g * RPG + q][j], w, acc[q]);
+                    for (int q = 0; q < RPT; ++q) {
+                        const float4 el = *reinterpret_cast<const float4*>(&s_left[r0 + q][j]);
+                        const float ev[4] = {el.x, el.y, el.z, el.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            acc[q].x = fmaf(ev[u], wj[u].x, acc[q].x);
+                            acc[q].y = fmaf(ev[u], wj[u].y, acc[q].y);
+                            acc[q].z = fmaf(ev[u], wj[u].z, acc[q].z);
+                            acc[q].w = fmaf(ev[u], wj[u].w, acc[q].w);
+                        }
+                    }
                 }
-            }
 #pragma unroll
-            for (int q = 0; q < RPG; ++q)
-                if (g * RPG + q < nl) s_f[g * RPG + q][l] = acc[q];
+                for (int q = 0; q < RPT; ++q)
+                    if (r0 + q < nl) *reinterpret_cast<float4*>(&s_f[r0 + q][4 * cq]) = acc[q];
+            }
             __syncthreads();
-            // S[k][k'] = F[k] . E_right[k']
+            // S[k][k'] = F[k] . E_right[k'] (l ascending)
             const int k = t / K, k2 = t % K;
             if (k < nl) {
                 float sc = 0.0f;
 #pragma unroll 8
-                for (int l2 = 0; l2 < D; ++l2) sc = fmaf(s_f[k][l2], s_right[k2][l2], sc);
+                for (int l2 = 0; l2 < D; l2 += 4) {
+                    const float4 f = *reinterpret_cast<const float4*>(&s_f[k][l2]);
+                    const float4 r = *reinterpret_cast<const float4*>(&s_right[k2][l2]);
+                    sc = fmaf(f.x, r.x, sc);
+                    sc = fmaf(f.y, r.y, sc);
+                    sc = fmaf(f.z, r.z, sc);
+                    sc = fmaf(f.w, r.w, sc);
+                }
                 out[k * K + k2] = sc;
             }
         }
     } else if (t < K) {
         out[t] = 0.0f;  // no anchor: no term before position 0
     }
+    if (t == 0) s_bad = ok ? 0 : 1;
     __syncthreads();
     if (t == 0) __threadfence();
 
     if (!arrive_last(&counters[b], (unsigned)G)) return;
+    if (s_bad) return;  // this CTA's W copy may still be in flight: leave its smem alone
+
+    // ---- last CTA of the sequence: everything the recursion reads, in one pass
+    const float* sc = scores + (int64_t)b * seq_scores;
+    float* s_sc = s_dyn;
+#pragma unroll 4
+    for (int e = t; e < seq_scores; e += NT) s_sc[e] = __ldcg(&sc[e]);
+    for (int e = t; e < G * K; e += NT) {
+        s_lp[e] = logp[(int64_t)b * G * K + e];
+        s_cand[e] = cand[e];
+    }
+    __syncthreads();
     if (warp != 0) return;
 
     // Max-sum recursion, lane k = candidate rank k (lanes 16..31 mirror 0..15).
-    const float* sc = scores + (int64_t)b * (K + (int64_t)K * K * (G - 1));
-    const float* lp = logp + (int64_t)b * G * K;
     const int k = lane & (K - 1);
-    double delta = (double)lp[k] + (double)__ldcg(&sc[k]);
+    double delta = (double)s_lp[k] + (double)s_sc[k];
     for (int p = 1; p < G; ++p) {
-        const float* Sp = sc + K + (int64_t)K * K * (p - 1);
+        if (lane < K) s_delta[(p - 1) & 1][k] = delta;
+        __syncwarp();
+        const double* dprev = s_delta[(p - 1) & 1];
+        const float* Sp = s_sc + K + K * K * (p - 1);
         double best = 0.0;
         int arg = -1;
+#pragma unroll
         for (int kk = 0; kk < K; ++kk) {
-            const double dk = __shfl_sync(FULL, delta, kk);
-            const double cand_s = dk + (double)__ldcg(&Sp[kk * K + k]);
-            if (arg < 0 || cand_s > best) {
-                best = cand_s;
+            const double c_s = dprev[kk] + (double)Sp[kk * K + k];
+            if (arg < 0 || c_s > best) {
+                best = c_s;
                 arg = kk;
             }
         }
-        delta = (double)lp[p * K + k] + best;
+        delta = (double)s_lp[p * K + k] + best;
         if (lane < K) s_back[p][k] = (uint8_t)arg;
     }
     // smallest rank with the maximal final score
@@ -137,10 +201,10 @@ __global__ void __launch_bounds__(NT, 2) pair_select_kernel(
 #pragma unroll
     for (int j = 16; j > 0; j >>= 1) {
         const double ov = __shfl_xor_sync(FULL, bv, j);
-        const int ok = __shfl_xor_sync(FULL, bk, j);
-        if (ov > bv || (ov == bv && ok < bk)) {
+        const int ok2 = __shfl_xor_sync(FULL, bk, j);
+        if (ov > bv || (ov == bv && ok2 < bk)) {
             bv = ov;
-            bk = ok;
+            bk = ok2;
         }
     }
     __syncwarp();
@@ -148,10 +212,15 @@ __global__ void __launch_bounds__(NT, 2) pair_select_kernel(
         path_score[b] = (float)bv;
         int kk = bk;
         for (int p = G - 1; p >= 0; --p) {
-            path_rank[(int64_t)b * G + p] = kk;
-            path_tok[(int64_t)b * G + p] = cand[p * K + kk];
+            s_path[p] = kk;
             if (p > 0) kk = s_back[p][kk];
         }
+    }
+    __syncwarp();
+    if (lane < G) {
+        const int r = s_path[lane];
+        path_rank[(int64_t)b * G + lane] = r;
+        path_tok[(int64_t)b * G + lane] = s_cand[lane * K + r];
     }
 }
 
@@ -182,7 +251,7 @@ extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const 
     if (!idx || !logp || !emb || !W || !path_tok || !path_rank || !path_score)
         return DFLASH2_EINVAL;
     if (!aligned(idx, 4) || !aligned(logp, 4) || (anchor && !aligned(anchor, 4)) ||
-        !aligned(emb, elem_size(emb_dtype)) || !aligned(W, 16) || !aligned(path_tok, 4) ||
+        !aligned(emb, 16) || !aligned(W, 16) || !aligned(path_tok, 4) ||
         !aligned(path_rank, 4) || !aligned(path_score, 4))
         return DFLASH2_EALIGN;
     if ((int64_t)B * G > (int64_t)INT32_MAX) return DFLASH2_ESHAPE;
@@ -196,7 +265,7 @@ extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const 
 #define DFL_SEL(BF, DD)                                                                          \
     do {                                                                                         \
         auto kern = pair_select_kernel<BF, DD>;                                                  \
-        const int dyn = DD * DD * 4;                                                             \
+        const int dyn = (int)(4 * std::max<int64_t>((int64_t)DD * DD, K + (int64_t)K * K * (G - 1))); \
         if (dyn > 48 * 1024 &&                                                                   \
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) !=      \
                 cudaSuccess)                                                                     \
