@@ -49,6 +49,10 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["topk_softmax", "pair_select", "verify_sample",
+                                       "verify_greedy", "dynconv2"], default=None,
+                    help="run and time one call of the step only (for profiling); prints a "
+                         "per-call line, not a bench line")
     return ap.parse_args()
 
 
@@ -261,7 +265,9 @@ def run_ours(args, rank, world, local_rank):
         for s in range(n):
             inp = inputs[(step0 + s) % 2]
             row = []
-            for fn in calls(inp, step0 + s):
+            for name, fn in zip(names, calls(inp, step0 + s)):
+                if record and args.only and name != args.only:
+                    continue
                 # L2 flush: write a buffer twice the size of L2, then read it,
                 # so the timed call starts with no data of its own in L2 and
                 # no dirty lines left to write back
@@ -291,6 +297,14 @@ def run_ours(args, rank, world, local_rank):
         t_wall = time.perf_counter() - t_wall0
     barrier()
     per_call = np.array([[e0.elapsed_time(e1) for (e0, e1) in row] for row in evs])  # ms
+    if args.only:  # one call alone: a per-call line for profiling, not a bench line
+        if rank == 0:
+            us = float(per_call.mean()) * 1e3
+            nbytes = algorithmic_bytes(w, B)[args.only]
+            print(json.dumps({"only": args.only, "us": round(us, 2), "algorithmic_bytes": nbytes,
+                              "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1),
+                              "steps": args.steps}), flush=True)
+        return
     step_ms = per_call.sum(axis=1)
     local = torch.tensor([float(step_ms.sum())] + per_call.mean(axis=0).tolist(),
                          dtype=torch.float64, device=dev)
