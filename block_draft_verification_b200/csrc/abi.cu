@@ -23,9 +23,10 @@ extern "C" int dflash2_version(void) { return (1 << 16) | 0; }
 extern "C" size_t dflash2_workspace_bytes(int B, int G, int64_t V) {
     if (B < 0 || G < 1 || G >= DFLASH2_MAX_BLOCK || V < 1) return 0;
     const int64_t rows = (int64_t)B * G;
-    size_t need = topk_layout(rows, V).total;
-    need = need > greedy_layout(B, G, V).total ? need : greedy_layout(B, G, V).total;
-    need = need > sample_layout(B, G, V).total ? need : sample_layout(B, G, V).total;
+    // sized for fp32 (es = 4), whose chunks are the shorter: serves bf16 too
+    size_t need = topk_layout(rows, V, 4).total;
+    need = need > greedy_layout(B, G, V, 4).total ? need : greedy_layout(B, G, V, 4).total;
+    need = need > sample_layout(B, G, V, 4).total ? need : sample_layout(B, G, V, 4).total;
     need = need > select_layout(B, G).total ? need : select_layout(B, G).total;
     return need;
 }

@@ -236,56 +236,6 @@ __device__ __forceinline__ float vec_max(const uint4& v) {
                  fmaxf(__uint_as_float(v.z), __uint_as_float(v.w)));
 }
 
-// Thread max and sum-exp over the loaded vectors (pairwise within a vector).
-template <bool BF16>
-__device__ __forceinline__ Lse thread_lse(const uint4 (&r)[Row<BF16>::NV], float c) {
-    using R = Row<BF16>;
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < R::NV; ++i)
-#pragma unroll
-        for (int e = 0; e < R::VW; ++e) m = fmaxf(m, R::elem(r[i], e));
-    if (m == -INFINITY) return {m, 0.0f};
-    float s = 0.0f;
-#pragma unroll
-    for (int i = 0; i < R::NV; ++i) {
-        float t[R::VW];
-#pragma unroll
-        for (int e = 0; e < R::VW; ++e) t[e] = ex2((R::elem(r[i], e) - m) * c);
-#pragma unroll
-        for (int w = R::VW / 2; w > 0; w >>= 1)
-#pragma unroll
-            for (int e = 0; e < w; ++e) t[e] += t[e + w];
-        s += t[0];
-    }
-    return {m, s};
-}
-
-// Thread max and sum-exp with an fp64 running sum of the per-vector sums.
-template <bool BF16>
-__device__ __forceinline__ LseD thread_lse_d(const uint4 (&r)[Row<BF16>::NV], float c) {
-    using R = Row<BF16>;
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < R::NV; ++i)
-#pragma unroll
-        for (int e = 0; e < R::VW; ++e) m = fmaxf(m, R::elem(r[i], e));
-    if (m == -INFINITY) return {m, 0.0f, 0.0};
-    double s = 0.0;
-#pragma unroll
-    for (int i = 0; i < R::NV; ++i) {
-        float t[R::VW];
-#pragma unroll
-        for (int e = 0; e < R::VW; ++e) t[e] = ex2((R::elem(r[i], e) - m) * c);
-#pragma unroll
-        for (int w = R::VW / 2; w > 0; w >>= 1)
-#pragma unroll
-            for (int e = 0; e < w; ++e) t[e] += t[e + w];
-        s += (double)t[0];
-    }
-    return {m, 0.0f, s};
-}
-
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon et al., SC'11, section 5): ten rounds of
 //   (c0,c1,c2,c3) -> (hi(M1*c2)^c1^k0, lo(M1*c2), hi(M0*c0)^c3^k1, lo(M0*c0))

@@ -7,249 +7,160 @@
 // those 16 per position; "DFlash 2" (myaiexp.com), section "主な機能": the
 // path selector keeps the top-16 candidates of each position.
 //
-// Work unit: (row, 16384-element chunk).  Persistent CTAs each stream a
-// contiguous range of units through a two-slot shared-memory ring filled by
-// TMA bulk copies (rows whose start is 16-byte aligned; others are read
-// element by element).  Softmax: per chunk, the block max, then the sum of
-// exp2((x - M) c) against it, both in a fixed order, so a chunk's partial
-// does not depend on the batch or the grid.  Top-16: the block keeps a
-// running top-16 of the row segment it streams (its consecutive chunks of one
-// row).  The first chunk of a segment takes the exact bounded path (the 16th
-// largest per-thread maximum bounds the answer, at most 16 threads contribute
-// candidates, one warp sorts them); later chunks only look at elements whose
-// key beats the running 16th key, about 16/c of them in the c-th chunk.  The
-// segment's list is published with one acquire-release add; the publisher
-// that completes a row (no CTA waits) merges the chunk softmax partials in
-// chunk order and the segment lists, and writes idx / prob / logp / logz.
-// Keys compare (value, -index) exactly, so the top-16 set does not depend on
-// how the row was split.
+// Work unit: (row, chunk of 16 KB of logits).  One CTA per SM streams a
+// contiguous range of units through a ring of TMA bulk copies kept in flight
+// by a producer warp (rows whose start is 16-byte aligned; others are read
+// element by element); each consumer warp reduces whole chunks on its own:
+// the chunk maximum, the sum of exp2((x - M) c) against it and the chunk's
+// exact top-16, all in a fixed order, so a chunk's partial does not depend
+// on the batch or the grid.  A unit's partial is published with one
+// acquire-release add; the warp that completes a row (no warp waits) merges
+// the chunk lists and softmax partials in chunk order and writes
+// idx / prob / logp / logz.  Keys compare (value, -index) exactly, so the
+// top-16 set does not depend on how the row was split.
 #include "common.cuh"
-#include "stream.cuh"
+#include "ring.cuh"
 #include "workspace.cuh"
 
 namespace dfl {
 
-struct __align__(16) TopkSmem {
-    uint64_t run[K];          // running top-16 of the row segment (descending; 0 = empty)
-    uint32_t top[NT / 32][K];
-    uint64_t cand[K * EPT];   // candidate keys (capacity 1024)
-    uint32_t tie[NT];
-    float wmax[NT / 32];
-    float wmax2[NT / 32];
-    float wsum[NT / 32];
-    unsigned ncand, ntie;
-    uint32_t thr, vk;
+// Candidate buffer of one consumer warp: keys pushed during the exp pass,
+// merged into the running list whenever more than CAND_FLUSH are waiting (at
+// most 32 lanes x 8 elements arrive between two checks).
+constexpr unsigned CAND_FLUSH = 64;
+constexpr unsigned CAND_CAP = CAND_FLUSH + 32 * 8;
+struct CandBuf {
+    uint64_t key[CAND_CAP];
+    unsigned n;
 };
-constexpr unsigned CAND_CAP = K * EPT;
 
-// Warp 0: merge sm.cand[0..n) into the running list (16 candidates a round).
-__device__ __forceinline__ void merge_candidates(TopkSmem& sm, unsigned n) {
+// Merge the buffered candidates into the running list (lanes 0..15 hold it,
+// descending; 0 = empty) sixteen at a time, and raise the threshold to the
+// list's 16th key once the list is full.  Warp-uniform.
+__device__ __forceinline__ void flush_candidates(CandBuf& cb, uint64_t& run, uint64_t& tkey,
+                                                 float& tv) {
     const int lane = threadIdx.x & 31;
-    uint64_t acc = (lane < K) ? sm.run[lane] : 0ull;
+    __syncwarp();
+    const unsigned n = *(volatile unsigned*)&cb.n;
     for (unsigned base = 0; base < n; base += K) {
-        uint64_t v = acc;
-        if (lane >= K) v = (base + lane - K < n) ? sm.cand[base + lane - K] : 0ull;
-        acc = warp_sort_desc(v);
+        uint64_t v = run;
+        if (lane >= K) {
+            const unsigned j = base + (unsigned)(lane - K);
+            v = (j < n) ? cb.key[j] : 0ull;
+        }
+        v = warp_sort_desc(v);
+        run = (lane < K) ? v : 0ull;
     }
-    if (lane < K) sm.run[lane] = acc;
+    __syncwarp();
+    if (lane == 0) cb.n = 0;
+    __syncwarp();
+    const uint64_t k16 = shfl64(run, K - 1);
+    if (k16 > tkey) {
+        tkey = k16;
+        tv = key_value(k16);
+    }
 }
 
-// The chunk's exact top-16 without sorting the chunk: T = the 16th largest
-// per-thread maximum bounds it; only threads whose maximum is above T, or
-// equal to T with a first index among the lowest (16 - #above) of those, can
-// hold a top-16 element (at most 16 threads x 64 candidates); they are merged
-// into the running list.  m = this thread's maximum.
-template <bool BF16, class C>
-__device__ __forceinline__ void chunk_top16_exact(const C& ch, float m, TopkSmem& sm) {
-    using R = Row<BF16>;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    __syncthreads();  // everyone has read the count that sent the block here
-    const uint32_t my_ord = (m == -INFINITY) ? 0u : ord32(m);
-    const uint32_t srt = warp_sort_desc(my_ord);
-    if (lane < K) sm.top[warp][lane] = srt;
-    if (t == 0) {
-        sm.ncand = 0;
-        sm.ntie = 0;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t acc = (lane < K) ? sm.top[0][lane] : 0u;
-        for (int w = 1; w < NT / 32; ++w) acc = warp_merge_desc(lane < K ? acc : sm.top[w][31 - lane]);
-        if (lane == K - 1) sm.thr = acc;  // 0: fewer than 16 threads hold elements
-    }
-    __syncthreads();
-    const uint32_t thr = sm.thr;
-    const bool above = my_ord > thr;
-    const bool tie = thr != 0u && my_ord == thr;
-    const int n_above = __syncthreads_count(above);
-    uint32_t my_first = 0xFFFFFFFFu;
-    if (tie) {
-        my_first = view_first<BF16>(ch, m);
-        sm.tie[atomicAdd(&sm.ntie, 1u)] = my_first;
-    }
-    __syncthreads();
-    if (tie) {
-        const unsigned n = sm.ntie;
-        unsigned rank = 0;
-        for (unsigned j = 0; j < n; ++j) rank += sm.tie[j] < my_first;
-        if (rank == (unsigned)(K - n_above - 1)) sm.vk = my_first;
-    }
-    __syncthreads();
-    const float tv = (thr == 0u) ? -INFINITY : unord32(thr);
-    const uint32_t vk = (thr == 0u) ? 0u : sm.vk;
-    if (above || (tie && my_first <= vk)) {
-#pragma unroll
-        for (int i = 0; i < R::NV; ++i) {
-            const uint4 v4 = ch.vec(i);
-#pragma unroll
-            for (int e = 0; e < R::VW; ++e) {
-                const float x = R::elem(v4, e);
-                const uint32_t v = (uint32_t)ch.index_of(i, e);
-                if (x > tv || (thr != 0u && x == tv && v <= vk))
-                    sm.cand[atomicAdd(&sm.ncand, 1u)] = make_key(x, v);
-            }
+// One chunk, one warp: the chunk maximum M, the sum of exp2((x - M) c) and
+// the running top-16 `run` of the row segment (lanes 0..15, descending by
+// (value, -index); 0 = empty) updated with the chunk's elements.
+//   Pass 1: the packed maximum of every vector of the lane, kept in
+//   registers, and the lane maxima.  While the list is not full, T = the 16th
+//   largest lane maximum bounds the chunk's own top 16 (at least 16 elements
+//   are >= T); once it is full its 16th key is the bound.
+//   Candidates: only the vectors whose maximum reaches the bound's value are
+//   looked at element by element (one per lane per round); keys beating the
+//   bound are pushed and merged whenever more than CAND_FLUSH wait, and the
+//   bound rises to the list's 16th key at every merge.
+//   Pass 2: the exponentials (chunk_expsum).
+template <bool BF16, class View>
+__device__ __forceinline__ void topk_chunk(const View& v, float c2, CandBuf& cb, float& M_out,
+                                           double& S_out, uint64_t& run) {
+    using C = ChunkT<BF16>;
+    const int lane = threadIdx.x & 31, nv = v.nvec();
+    uint32_t vm[NVL];
+    const float m = chunk_pass1<BF16>(v, vm);
+    const float M = warp_max(m);
+    float tv = -INFINITY;
+    uint64_t tkey = shfl64(run, K - 1);  // the full list's 16th key, or 0
+    if (tkey != 0ull) {
+        tv = key_value(tkey);
+    } else {
+        const uint32_t t16 =
+            __shfl_sync(FULL, warp_sort_desc(m == -INFINITY ? 0u : ord32(m)), K - 1);
+        if (t16 != 0u) {  // else fewer than 16 lanes hold elements: every element qualifies
+            tv = unord32(t16);
+            tkey = ((uint64_t)t16 << 32) - 1ull;  // below every key of value tv
         }
     }
-    __syncthreads();
-    if (warp == 0) merge_candidates(sm, sm.ncand);
-    __syncthreads();
-}
-
-// One unit: the chunk's softmax partial (block max, then the sum of
-// exp2(x c - M c) against it, in a fixed order) and the running top-16.
-//  - Running list full: elements whose key beats its 16th key are pushed as
-//    candidates during the max pass (about 16/c of them in the c-th chunk of
-//    a segment); warp 0 merges them while the other warps sum exps.
-//  - Running list empty (first chunk of a segment): T' = the smallest of the
-//    warps' second-largest thread maxima has at least 16 elements at or above
-//    it (two per warp), so the elements >= T' hold the chunk's top-16; they are
-//    pushed and merged.
-//  - More candidates than the buffer holds (adversarial orders, mass ties):
-//    the chunk takes the exact bounded path.
-template <bool BF16, class C>
-__device__ __forceinline__ void topk_unit(const C& ch, float c2, TopkSmem& sm, float& chunk_m,
-                                          float& chunk_s) {
-    using R = Row<BF16>;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const uint64_t r16 = sm.run[K - 1];
-    const float rv = r16 ? key_value(r16) : INFINITY;
-    // pass 1: thread max, and candidates against the running list
-    float m = -INFINITY;
+    const uint32_t t2 = (tv == -INFINITY) ? C::NEG_INF_WORD : pack_value<BF16>(tv);
+    uint32_t hits = 0;
 #pragma unroll
-    for (int i = 0; i < R::NV; ++i) {
-        const uint4 v4 = ch.vec(i);
-        const float vm = vec_max<BF16>(v4);
-        m = fmaxf(m, vm);
-        if (vm >= rv) {
+    for (int i = 0; i < NVL; ++i)
+        if (32 * i + lane < nv && any_ge<BF16>(vm[i], t2)) hits |= 1u << i;
+    if (__any_sync(FULL, hits != 0u)) {
+        while (__any_sync(FULL, hits != 0u)) {  // one vector per lane per round
+            if (hits) {
+                const int i = __ffs(hits) - 1;
+                hits &= hits - 1u;
+                const int q = 32 * i + lane;
+                const uint4 w = v.vec(q);
 #pragma unroll
-            for (int e = 0; e < R::VW; ++e) {
-                const float x = R::elem(v4, e);
-                if (x >= rv) {
-                    const uint64_t key = make_key(x, (uint32_t)ch.index_of(i, e));
-                    if (key > r16) {
-                        const unsigned slot = atomicAdd(&sm.ncand, 1u);
-                        if (slot < CAND_CAP) sm.cand[slot] = key;
+                for (int e = 0; e < C::VW; ++e) {
+                    const float x = C::elem(w, e);
+                    if (x >= tv && q * C::VW + e < v.n) {
+                        const uint64_t key = make_key(x, (uint32_t)v.index(q, e));
+                        if (key > tkey) cb.key[atomicAdd(&cb.n, 1u)] = key;
                     }
                 }
             }
+            __syncwarp();
+            if (*(volatile unsigned*)&cb.n > CAND_FLUSH) flush_candidates(cb, run, tkey, tv);
         }
+        __syncwarp();
+        if (*(volatile unsigned*)&cb.n > 0u) flush_candidates(cb, run, tkey, tv);
     }
-    // warp max and (for seeding) the warp's second-largest thread maximum
-    float wm = m;
-#pragma unroll
-    for (int j = 16; j > 0; j >>= 1) wm = fmaxf(wm, __shfl_xor_sync(FULL, wm, j));
-    const unsigned at_max = __ballot_sync(FULL, m == wm);
-    float m2 = (lane == __ffs(at_max) - 1) ? -INFINITY : m;
-#pragma unroll
-    for (int j = 16; j > 0; j >>= 1) m2 = fmaxf(m2, __shfl_xor_sync(FULL, m2, j));
-    if (lane == 0) {
-        sm.wmax[warp] = wm;
-        sm.wmax2[warp] = m2;
-    }
-    __syncthreads();  // A
-    float M = sm.wmax[0];
-#pragma unroll
-    for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, sm.wmax[w]);
-    bool exact = false;
-    if (r16 == 0ull) {  // seed the segment's list from this chunk
-        float Tp = sm.wmax2[0];
-#pragma unroll
-        for (int w = 1; w < NT / 32; ++w) Tp = fminf(Tp, sm.wmax2[w]);
-        if (m >= Tp && m != -INFINITY) {
-#pragma unroll
-            for (int i = 0; i < R::NV; ++i) {
-                const uint4 v4 = ch.vec(i);
-#pragma unroll
-                for (int e = 0; e < R::VW; ++e) {
-                    const float x = R::elem(v4, e);
-                    if (x >= Tp && x != -INFINITY) {
-                        const unsigned slot = atomicAdd(&sm.ncand, 1u);
-                        if (slot < CAND_CAP) sm.cand[slot] = make_key(x, (uint32_t)ch.index_of(i, e));
-                    }
-                }
-            }
-        }
-        __syncthreads();  // B (seeding chunks only)
-    }
-    const unsigned n = sm.ncand;
-    if (n > CAND_CAP) {
-        exact = true;  // block-uniform
-    } else if (n > 0 && warp == 0) {
-        merge_candidates(sm, n);  // overlaps the other warps' exp pass
-    }
-    if (exact) chunk_top16_exact<BF16>(ch, m, sm);
-
-    // pass 2: sum of exp2(x c - M c) (fixed order), each exponent one FMA
-    // against mc = fl(M c); the product's rounding error M c - mc (exact in
-    // fp32) is taken out of the sum once per chunk below.
-    float s = 0.0f;
-    const float mc = M * c2;
-    if (M != -INFINITY) {
-#pragma unroll
-        for (int i = 0; i < R::NV; ++i) {
-            const uint4 v4 = ch.vec(i);
-            float tt[R::VW];
-#pragma unroll
-            for (int e = 0; e < R::VW; ++e) tt[e] = ex2(fmaf(R::elem(v4, e), c2, -mc));
-#pragma unroll
-            for (int w = R::VW / 2; w > 0; w >>= 1)
-#pragma unroll
-                for (int e = 0; e < w; ++e) tt[e] += tt[e + w];
-            s += tt[0];
-        }
-    }
-#pragma unroll
-    for (int j = 16; j > 0; j >>= 1) s += __shfl_xor_sync(FULL, s, j);
-    if (lane == 0) sm.wsum[warp] = s;
-    __syncthreads();  // D: sums ready, candidates merged
-    float S = 0.0f;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w) S += sm.wsum[w];
-    chunk_m = M;
-    chunk_s = (M != -INFINITY) ? S * ex2(-fmaf(M, c2, -mc)) : S;
-    if (t == 0) sm.ncand = 0;  // read by everyone before D; next pushes come after
+    M_out = M;
+    S_out = chunk_expsum<BF16>(v, M, c2);
 }
 
-// The row's final merge (warp 0 of the last unit of the row).
-__device__ __forceinline__ void topk_row_merge(const TopkPartial* P, int S, int64_t row, float inv_t,
+// The row's final merge by one warp, after its last chunk was published:
+// the segment lists (bitonic merges in chunk order), the maximum, and the
+// fp64 sum of the chunk sums rescaled to it (lane c takes chunks c, c + 32,
+// ...; then a fixed butterfly).
+__device__ __forceinline__ void topk_row_merge(const TopkPart* P, int S, int64_t row, float inv_t,
                                                float c2, int32_t* __restrict__ idx,
                                                float* __restrict__ prob, float* __restrict__ logp,
                                                float* __restrict__ logz) {
     const int lane = threadIdx.x & 31;
     auto ldkey = [](const uint64_t* p) { return (uint64_t)__ldcg((const unsigned long long*)p); };
-    uint64_t acc = (lane < K) ? ldkey(&P[0].key[lane]) : 0ull;
-    for (int c = 1; c < S; ++c) acc = warp_merge_desc(lane < K ? acc : ldkey(&P[c].key[31 - lane]));
+    // only a row segment's last chunk carries a list (key[0] != 0)
+    uint64_t acc = 0ull;
+    bool first = true;
+    for (int c0 = 0; c0 < S; c0 += 32) {
+        const int c = c0 + lane;
+        unsigned has = __ballot_sync(FULL, c < S && ldkey(&P[c].key[0]) != 0ull);
+        while (has) {
+            const int cc = c0 + __ffs(has) - 1;
+            has &= has - 1;
+            if (first) {
+                acc = (lane < K) ? ldkey(&P[cc].key[lane]) : 0ull;
+                first = false;
+            } else {
+                acc = warp_merge_desc(lane < K ? acc : ldkey(&P[cc].key[31 - lane]));
+            }
+        }
+    }
     float M = -INFINITY;
     for (int c = lane; c < S; c += 32) M = fmaxf(M, __ldcg(&P[c].m));
-#pragma unroll
-    for (int j = 16; j > 0; j >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, j));
+    M = warp_max(M);
     double ssum = 0.0;
-    if (lane == 0)  // sum in chunk order, fp64
-        for (int c = 0; c < S; ++c) {
-            const float mc = __ldcg(&P[c].m), sc = __ldcg(&P[c].s);
-            if (mc != -INFINITY) ssum += (double)sc * exp2(((double)mc - (double)M) * (double)c2);
-        }
-    ssum = __shfl_sync(FULL, ssum, 0);
+    for (int c = lane; c < S; c += 32) {
+        const float mc = __ldcg(&P[c].m);
+        const double sc = __ldcg(&P[c].s);
+        if (mc != -INFINITY) ssum += sc * exp2(((double)mc - (double)M) * (double)c2);
+    }
+    ssum = warp_sum(ssum);
     const double lns = log(ssum);
     if (lane < K) {
         const double x = (double)key_value(acc);
@@ -261,86 +172,83 @@ __device__ __forceinline__ void topk_row_merge(const TopkPartial* P, int S, int6
     }
 }
 
+// Units (row, chunk): one CTA per SM over a contiguous range, each warp a
+// contiguous part of it streamed through its own two ring slots.  Every
+// chunk leaves its softmax partial in the workspace; a warp's consecutive
+// chunks of one row (a segment) share one running top-16, left with the
+// segment's last chunk, and are published together with one acquire-release
+// add on the row's counter.  The warp whose add completes the row merges it.
+// No warp waits for another.
 template <bool BF16, bool TMA>
-__global__ void __launch_bounds__(NT, 3) topk_softmax_kernel(
+__global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
     const void* __restrict__ logits, int64_t V, int64_t row_stride, int S, int64_t units,
     float inv_t, float c2, int32_t* __restrict__ idx, float* __restrict__ prob,
-    float* __restrict__ logp, float* __restrict__ logz, TopkPartial* __restrict__ part,
+    float* __restrict__ logp, float* __restrict__ logz, TopkPart* __restrict__ part,
     unsigned* __restrict__ counters) {
     constexpr int ES = BF16 ? 2 : 4;
-    constexpr int SLOT = CHUNK * ES;
+    constexpr int LEN = chunk_len(ES);
     extern __shared__ __align__(128) uint8_t ring[];
-    __shared__ TopkSmem sm;
-    __shared__ __align__(8) uint64_t s_bar[2];
-    const int t = threadIdx.x, warp = t >> 5;
-    const uint32_t bar0 = smem_u32(&s_bar[0]);
-
-    auto unit_geom = [&](int64_t u, int64_t& row, int64_t& v0, int64_t& vend) {
-        row = u / S;
-        v0 = (u - row * S) * (int64_t)CHUNK;
-        vend = min(V, v0 + (int64_t)CHUNK);
-    };
-    auto issue = [&](int64_t u, int slot) {
-        int64_t row, v0, vend;
-        unit_geom(u, row, v0, vend);
-        const char* src = (const char*)logits + (row * row_stride + v0) * ES;
-        bulk_g2s(smem_u32(ring + slot * SLOT), src, (uint32_t)((vend - v0) * ES), bar0 + 8 * slot);
-    };
+    __shared__ __align__(8) uint64_t bars[2 * NCW];
+    __shared__ CandBuf cbuf[NCW];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    CandBuf& cb = cbuf[warp];
+    if (lane == 0) cb.n = 0;
     int64_t lo, hi;
-    cta_range(units, lo, hi);
-    if (TMA) {
-        if (t == 0) {
-            mbar_init(bar0, 1);
-            mbar_init(bar0 + 8, 1);
-            mbar_fence_init();
-            if (lo < hi) issue(lo, 0);
-        }
-        __syncthreads();
-    }
-    __shared__ bool s_last;
-    unsigned pending = 0;
-    if (t < K) sm.run[t] = 0ull;
-    if (t == 0) sm.ncand = 0;
-    int k = 0;
-    for (int64_t u = lo; u < hi; ++u, ++k) {
-        int64_t row, v0, vend;
-        unit_geom(u, row, v0, vend);
-        float cm, cs;
+    warp_range(units, lo, hi);
+    const int n = (int)(hi - lo);
+    UnitCursor uc, ic;  // the unit being reduced, the next unit to bring in
+    uc.init(lo, S, 1);
+    ic = uc;
+    auto src = [&](const UnitCursor& cu, const char*& p, uint32_t& bytes) {
+        const int64_t v0 = (int64_t)cu.c * LEN;
+        p = (const char*)logits + (cu.g * row_stride + v0) * ES;
+        bytes = (uint32_t)(min((int64_t)LEN, V - v0) * ES);
+    };
+    WarpRing r{nullptr, 0u};
+    if (TMA) r = warp_ring_start(ring, bars, n, ic, ChunkT<BF16>::NEG_INF_WORD, src);
+    __syncwarp();
+    uint64_t run = 0ull;  // the segment's running top-16
+    unsigned seg = 0;     // chunks in the segment so far
+    for (int k = 0; k < n; ++k, uc.next()) {
+        const int64_t row = uc.g, v0 = (int64_t)uc.c * LEN;
+        const int len = (int)min((int64_t)LEN, V - v0);
+        float M;
+        double Ssum;
         if (TMA) {
-            if (t == 0 && u + 1 < hi) issue(u + 1, (k + 1) & 1);
-            if (!__syncthreads_and(mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1))) {
-                if (t == 0) {
-                    atomicOr(&g_dev_err, ERR_STREAM);
-                    if (u + 1 < hi) mbar_wait(bar0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
-                }
+            if (!r.wait(k)) {
+                warp_ring_abort(r, k, n);
                 return;
             }
-            topk_unit<BF16>(SmemChunk<BF16>{ring + (k & 1) * SLOT, v0, vend}, c2, sm, cm, cs);
+            topk_chunk<BF16>(SmemView<BF16>{r.slot(k), v0, len}, c2, cb, M, Ssum, run);
+            warp_ring_next(r, k, n, ic, ChunkT<BF16>::NEG_INF_WORD, src);
         } else {
-            RegChunk<BF16> ch;
-            ch.load((const char*)logits + row * row_stride * ES, v0, vend);
-            topk_unit<BF16>(ch, c2, sm, cm, cs);
+            topk_chunk<BF16>(
+                GlobalView<BF16>{(const uint8_t*)logits + row * row_stride * ES, v0, len}, c2, cb,
+                M, Ssum, run);
         }
-        ++pending;
-        const bool seg_end = (u + 1 == hi) || ((u + 1) / S != row);
-        if (t == 0) {  // thread 0 alone stores the partial (published by its release add);
-                       // only the last unit of a segment carries the segment's top-16
-            uint4* dst = (uint4*)&part[u];
-            dst[0] = make_uint4(__float_as_uint(cm), __float_as_uint(cs), 0u, 0u);
-            const uint4* kv = (const uint4*)sm.run;
-#pragma unroll
-            for (int j = 0; j < K / 2; ++j) dst[1 + j] = seg_end ? kv[j] : make_uint4(0, 0, 0, 0);
+        ++seg;
+        const bool seg_end = (k + 1 == n) || uc.last_of_row();
+        TopkPart* P = part + row * S + uc.c;
+        if (seg_end) {
+            if (lane < K) P->key[lane] = run;
+        } else if (lane == 0) {
+            P->key[0] = 0ull;  // no list here
         }
-        if (seg_end) {  // this CTA is done with the row: publish
-            if (t == 0) s_last = publish(&counters[row], pending, (unsigned)S);
-            __syncthreads();
-            if (s_last && warp == 0)
+        if (lane == 0) {
+            P->m = M;
+            P->s = Ssum;
+        }
+        if (seg_end) {
+            __syncwarp();
+            bool last = false;
+            if (lane == 0) last = publish(&counters[row], seg, (unsigned)S);
+            if (__shfl_sync(FULL, last, 0)) {
+                __syncwarp();  // lane 0's acquire covers the whole warp's reads
                 topk_row_merge(part + row * S, S, row, inv_t, c2, idx, prob, logp, logz);
-            pending = 0;
-            __syncthreads();
-            if (t < K) sm.run[t] = 0ull;  // the next segment starts empty
+            }
+            run = 0ull;
+            seg = 0;
         }
-        __syncthreads();  // ring slot k & 1 is free for the prefetch of iteration k + 1
     }
 }
 
@@ -372,15 +280,15 @@ extern "C" int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows,
     if (!aligned(logits, es) || !aligned(idx, 4) || !aligned(prob, 4) || !aligned(logp, 4) ||
         !aligned(logz, 4))
         return DFLASH2_EALIGN;
-    const int64_t S = n_chunks(V);
+    const int64_t S = row_chunks(V, es);
     const int64_t units = rows * S;
     if (units > (int64_t)INT32_MAX) return DFLASH2_ESHAPE;
-    const Layout L = topk_layout(rows, V);
+    const Layout L = topk_layout(rows, V, es);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return DFLASH2_EWORKSPACE;
 
     cudaStream_t s = (cudaStream_t)stream;
     unsigned* counters = (unsigned*)((char*)ws + L.counters_off);
-    TopkPartial* part = (TopkPartial*)((char*)ws + L.part_off);
+    TopkPart* part = (TopkPart*)((char*)ws + L.part_off);
     if (cudaMemsetAsync(counters, 0, (size_t)rows * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
 
     // TMA bulk copies need 16-byte aligned chunk starts and 16-byte multiples
@@ -389,14 +297,11 @@ extern "C" int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows,
 #define DFL_TOPK(BF, TM)                                                                          \
     do {                                                                                          \
         auto kern = topk_softmax_kernel<BF, TM>;                                                  \
-        const size_t dyn = TM ? 2 * (size_t)CHUNK * (BF ? 2 : 4) : 0;                             \
-        if (dyn > 48 * 1024 &&                                                                    \
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) !=  \
-                cudaSuccess)                                                                      \
-            return DFLASH2_ECUDA;                                                                 \
-        const int grid = persistent_grid(kern, NT, dyn, units);                                   \
-        kern<<<grid, NT, dyn, s>>>(logits, V, row_stride, (int)S, units, inv_temperature, c2, idx, \
-                                   prob, logp, logz, part, counters);                             \
+        const size_t dyn = TM ? (size_t)RING_BYTES : 0;                                           \
+        if (ring_prepare(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;                          \
+        kern<<<ring_grid(units), RING_THREADS, dyn, s>>>(logits, V, row_stride, (int)S, units,    \
+                                                         inv_temperature, c2, idx, prob, logp,    \
+                                                         logz, part, counters);                   \
     } while (0)
     if (dtype == DFLASH2_BF16) {
         if (tma) DFL_TOPK(true, true);
@@ -449,7 +354,7 @@ extern "C" int dflash2_topk_softmax_noalloc(const void* logits, int dtype, int64
                                             dflash2_stream_t stream) {
     if (!dtype_ok(dtype)) return DFLASH2_EDTYPE;
     if (rows < 0 || V < K || V > INT32_MAX || row_stride < V) return DFLASH2_ESHAPE;
-    if (rows > 0 && topk_layout(rows, V).total > NOALLOC_SCRATCH_BYTES)
+    if (rows > 0 && topk_layout(rows, V, elem_size(dtype)).total > NOALLOC_SCRATCH_BYTES)
         return DFLASH2_EWORKSPACE;  // more rows than the built-in scratch holds
     if (rows == 0) return DFLASH2_OK;
     void* scratch = noalloc_scratch_on_current_device();

@@ -10,59 +10,92 @@
 // tablas del proveedor": acceptance length = tokens completed per verify step.
 // Uniforms: Philox4x32-10 (Salmon et al., SC'11, section 5).
 //
-// Both verifies stream every logit row once in 16384-element chunks: work
-// unit = (sequence, row, chunk); persistent CTAs each take a contiguous range
-// of units through a two-slot shared-memory ring filled by TMA bulk copies,
-// and publish a sequence's finished units with one acquire-release add.  The
-// publisher that completes a sequence (no CTA waits) reduces the partials in
-// chunk order and decides.  The sampling draw needs the normalisers first, so
-// it is a second kernel over the one row each sequence draws from
-// (L2-resident after the first pass): one thread-block cluster per sequence,
-// each CTA holding its chunks in shared memory; the chunk sums of the draw
-// weights are exchanged through distributed shared memory, and the CTA that
-// holds the chunk where the inverse CDF crosses t = u' * R scans it there.
+// Both verifies stream every logit row once, in chunks of 16 KB: work unit =
+// (sequence, row, chunk), one CTA per SM over a contiguous range of units, a
+// producer warp keeping TMA bulk copies in flight and consumer warps each
+// reducing whole chunks (ring.cuh).  A unit's partial is published with one
+// acquire-release add on its sequence's counter; the warp whose add completes
+// the sequence (no warp waits) reduces the partials in chunk order and
+// decides.  The sampling draw needs the normalisers first, so it is a second
+// kernel over the one row each sequence draws from (launched as a dependent
+// of the scan, so its launch overlaps the scan's tail): one CTA per 4096
+// elements of that row sums its draw weights; the last CTA of the sequence
+// finds the chunk where the inverse CDF crosses t = u' * R and scans it.
 // No probability vector is ever written to memory.
 #include "common.cuh"
-#include "stream.cuh"
+#include "ring.cuh"
 #include "workspace.cuh"
 
 #include <algorithm>
-#include <map>
 #include <mutex>
-#include <tuple>
 
 namespace dfl {
 
 constexpr double LOG2E = 1.4426950408889634;
-// Chunks per row the sampling draw handles (its per-chunk sums sit in shared
-// memory): V <= 4096 * 16384.
-constexpr int64_t DRAW_MAX_CHUNKS = 4096;
-// Dynamic shared memory of the draw: the target and draft chunks, then two
-// rounds of per-chunk sums.
-inline size_t draw_smem(int es, int64_t S) { return 2 * (size_t)CHUNK * es + (size_t)S * 2 * sizeof(double); }
+
+// Programmatic dependent launch (PTX griddepcontrol): the scan lets its
+// dependent grid launch early; the draw waits for the scan's results.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ------------------------------------------------------------------ greedy
-struct GreedySmem {
-    float wmax[NT / 32];
-    unsigned first;
-};
+// One chunk, one warp: the chunk maximum M and the lowest index holding it,
+// as one key.  Pass 1 keeps every vector's packed maximum; a lane holding M
+// finds it in its first vector whose maximum is M (vectors of a lane are in
+// index order), and the warp takes the lowest index.
+template <bool BF16, class View>
+__device__ __forceinline__ uint64_t greedy_chunk(const View& v) {
+    using C = ChunkT<BF16>;
+    const int lane = threadIdx.x & 31;
+    uint32_t vm[NVL];
+    const float m = chunk_pass1<BF16>(v, vm);
+    const float M = warp_max(m);
+    uint32_t first = 0xFFFFFFFFu;
+    if (m == M) {
+        const uint32_t m2 = pack_value<BF16>(M);
+        int i0 = NVL;
+#pragma unroll
+        for (int i = NVL - 1; i >= 0; --i)
+            if (any_ge<BF16>(vm[i], m2)) i0 = i;
+        if (i0 < NVL) {
+            const int q = 32 * i0 + lane;
+            const uint4 w = v.vec(q);
+#pragma unroll
+            for (int e = C::VW - 1; e >= 0; --e)  // -0 == +0
+                if (C::elem(w, e) == M && q * C::VW + e < v.n) first = (uint32_t)v.index(q, e);
+        }
+    }
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) first = min(first, __shfl_xor_sync(FULL, first, j));
+    return make_key(M, first);
+}
 
-template <bool BF16, class C>
-__device__ __forceinline__ void greedy_unit(const C& ch, GreedySmem& sm, uint64_t* slot) {
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const float m = view_max<BF16>(ch);
-    float wm = m;
+// Largest key of rows r0 .. r0+NB-1 (of S chunk keys each), warp-collective:
+// lane c takes chunks c, c + 32, ...; the loads of all NB rows are issued
+// together.  Every lane returns the same keys.
+template <int NB>
+__device__ __forceinline__ void rows_max_key(const uint64_t* P, int S, int r0, int nrows,
+                                             uint64_t (&out)[NB]) {
+    const int lane = threadIdx.x & 31;
+    const unsigned long long* Q = (const unsigned long long*)P;
 #pragma unroll
-    for (int k = 16; k > 0; k >>= 1) wm = fmaxf(wm, __shfl_xor_sync(FULL, wm, k));
-    if (lane == 0) sm.wmax[warp] = wm;
-    if (t == 0) sm.first = 0xFFFFFFFFu;
-    __syncthreads();
-    float M = sm.wmax[0];
+    for (int j = 0; j < NB; ++j) out[j] = 0ull;
+    for (int c = lane; c < S; c += 32) {
+        uint64_t k[NB];
 #pragma unroll
-    for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, sm.wmax[w]);
-    if (m == M) atomicMin(&sm.first, view_first<BF16>(ch, M));  // -0 == +0
-    __syncthreads();
-    if (t == 0) *slot = make_key(M, sm.first);  // published by thread 0's release add
+        for (int j = 0; j < NB; ++j) k[j] = (j < nrows) ? (uint64_t)__ldcg(Q + (int64_t)(r0 + j) * S + c) : 0ull;
+#pragma unroll
+        for (int j = 0; j < NB; ++j) out[j] = k[j] > out[j] ? k[j] : out[j];
+    }
+#pragma unroll
+    for (int j = 0; j < NB; ++j)
+#pragma unroll
+        for (int h = 16; h > 0; h >>= 1) {
+            const uint64_t o = shfl_xor(out[j], h);
+            out[j] = o > out[j] ? o : out[j];
+        }
 }
 
 __device__ __forceinline__ void greedy_finish(const uint64_t* P, int S, int G, int b,
@@ -70,13 +103,14 @@ __device__ __forceinline__ void greedy_finish(const uint64_t* P, int S, int G, i
                                               int32_t* __restrict__ n_accept,
                                               int32_t* __restrict__ out_tok) {
     const int lane = threadIdx.x & 31;
-    uint64_t best = 0;  // lane j reduces target row j over its chunks (G + 1 <= 32)
-    if (lane <= G)
-        for (int c = 0; c < S; ++c) {
-            const uint64_t k = (uint64_t)__ldcg((const unsigned long long*)&P[(int64_t)lane * S + c]);
-            best = k > best ? k : best;
-        }
-    const int32_t tj = (int32_t)key_index(best);
+    int32_t tj = -1;  // lane j: argmax of target row j (G + 1 <= 32)
+    for (int r0 = 0; r0 <= G; r0 += 4) {
+        uint64_t best[4];
+        rows_max_key<4>(P, S, r0, min(4, G + 1 - r0), best);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (lane == r0 + j) tj = (int32_t)key_index(best[j]);
+    }
     const int32_t dj = (lane < G) ? draft_tok[(int64_t)b * G + lane] : -1;
     const unsigned miss = __ballot_sync(FULL, lane < G && dj != tj);
     const int n = miss ? (__ffs(miss) - 1) : G;
@@ -84,85 +118,100 @@ __device__ __forceinline__ void greedy_finish(const uint64_t* P, int S, int G, i
     if (lane == 0) n_accept[b] = n;
 }
 
+// Units (sequence b, row j, chunk): one CTA per SM over a contiguous range,
+// each warp a contiguous part of it streamed through its own ring slots; a
+// warp publishes its consecutive units of one sequence together, and the
+// warp whose add completes the sequence decides it.
 template <bool BF16, bool TMA>
-__global__ void __launch_bounds__(NT, 3) verify_greedy_kernel(
+__global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_kernel(
     const void* __restrict__ target, int G, int64_t V, int S, int64_t units,
     const int32_t* __restrict__ draft_tok, int32_t* __restrict__ n_accept,
     int32_t* __restrict__ out_tok, uint64_t* __restrict__ part, unsigned* __restrict__ counters) {
     constexpr int ES = BF16 ? 2 : 4;
-    constexpr int SLOT = CHUNK * ES;
+    constexpr int LEN = chunk_len(ES);
     extern __shared__ __align__(128) uint8_t ring[];
-    __shared__ GreedySmem sm;
-    __shared__ __align__(8) uint64_t s_bar[2];
-    const int t = threadIdx.x, warp = t >> 5;
-    const uint32_t bar0 = smem_u32(&s_bar[0]);
-    const int per_seq = (G + 1) * S;
-    auto geom = [&](int64_t u, int& b, int64_t& row, int64_t& v0, int64_t& vend) {
-        b = (int)(u / per_seq);
-        const int rem = (int)(u - (int64_t)b * per_seq);
-        const int j = rem / S;
-        row = (int64_t)b * (G + 1) + j;
-        v0 = (int64_t)(rem - j * S) * CHUNK;
-        vend = min(V, v0 + (int64_t)CHUNK);
-    };
-    auto issue = [&](int64_t u, int slot) {
-        int b;
-        int64_t row, v0, vend;
-        geom(u, b, row, v0, vend);
-        bulk_g2s(smem_u32(ring + slot * SLOT), (const char*)target + (row * V + v0) * ES,
-                 (uint32_t)((vend - v0) * ES), bar0 + 8 * slot);
-    };
+    __shared__ __align__(8) uint64_t bars[2 * NCW];
+    const int lane = threadIdx.x & 31;
     int64_t lo, hi;
-    cta_range(units, lo, hi);
-    if (TMA) {
-        if (t == 0) {
-            mbar_init(bar0, 1);
-            mbar_init(bar0 + 8, 1);
-            mbar_fence_init();
-            if (lo < hi) issue(lo, 0);
-        }
-        __syncthreads();
-    }
-    __shared__ bool s_last;
-    unsigned pending = 0;
-    int k = 0;
-    for (int64_t u = lo; u < hi; ++u, ++k) {
-        int b;
-        int64_t row, v0, vend;
-        geom(u, b, row, v0, vend);
-        uint64_t* slot = part + row * S + (v0 / CHUNK);
+    warp_range(units, lo, hi);
+    const int n = (int)(hi - lo);
+    UnitCursor uc, ic;  // (sequence, target row, chunk) being reduced / to bring in
+    uc.init(lo, S, G + 1);
+    ic = uc;
+    auto src = [&](const UnitCursor& cu, const char*& p, uint32_t& bytes) {
+        const int64_t v0 = (int64_t)cu.c * LEN;
+        p = (const char*)target + ((cu.g * (G + 1) + cu.r) * V + v0) * ES;
+        bytes = (uint32_t)(min((int64_t)LEN, V - v0) * ES);
+    };
+    WarpRing r{nullptr, 0u};
+    if (TMA) r = warp_ring_start(ring, bars, n, ic, ChunkT<BF16>::NEG_INF_WORD, src);
+    unsigned seg = 0;
+    for (int k = 0; k < n; ++k, uc.next()) {
+        const int64_t b = uc.g, v0 = (int64_t)uc.c * LEN;
+        const int64_t row = b * (G + 1) + uc.r;
+        const int len = (int)min((int64_t)LEN, V - v0);
+        uint64_t key;
         if (TMA) {
-            if (t == 0 && u + 1 < hi) issue(u + 1, (k + 1) & 1);
-            if (!__syncthreads_and(mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1))) {
-                if (t == 0) {
-                    atomicOr(&g_dev_err, ERR_STREAM);
-                    if (u + 1 < hi) mbar_wait(bar0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
-                }
+            if (!r.wait(k)) {
+                warp_ring_abort(r, k, n);
                 return;
             }
-            greedy_unit<BF16>(SmemChunk<BF16>{ring + (k & 1) * SLOT, v0, vend}, sm, slot);
+            key = greedy_chunk<BF16>(SmemView<BF16>{r.slot(k), v0, len});
+            warp_ring_next(r, k, n, ic, ChunkT<BF16>::NEG_INF_WORD, src);
         } else {
-            RegChunk<BF16> ch;
-            ch.load((const char*)target + row * V * ES, v0, vend);
-            greedy_unit<BF16>(ch, sm, slot);
+            key = greedy_chunk<BF16>(GlobalView<BF16>{(const uint8_t*)target + row * V * ES, v0, len});
         }
-        ++pending;
-        if (u + 1 == hi || (u + 1) / per_seq != b) {  // done with this sequence: publish
-            __syncthreads();
-            if (t == 0) s_last = publish(&counters[b], pending, (unsigned)per_seq);
-            __syncthreads();
-            if (s_last && warp == 0)
-                greedy_finish(part + (int64_t)b * (G + 1) * S, S, G, b, draft_tok, n_accept, out_tok);
-            pending = 0;
+        ++seg;
+        if (lane == 0) part[row * S + uc.c] = key;
+        if (k + 1 == n || uc.last_of_group()) {  // done with this sequence: publish
+            bool last = false;
+            if (lane == 0) last = publish(&counters[b], seg, (unsigned)((G + 1) * S));
+            if (__shfl_sync(FULL, last, 0)) {
+                __syncwarp();  // lane 0's acquire covers the whole warp's reads
+                greedy_finish(part + b * (G + 1) * S, S, G, (int)b, draft_tok, n_accept, out_tok);
+            }
+            seg = 0;
         }
-        __syncthreads();  // ring slot k & 1 is free for the prefetch of iteration k + 1
     }
 }
 
 // ------------------------------------------------------------------ sampling, pass 1
-// Units: for sequence b, rows 0..G are target rows, G+1..2G draft rows (softmax
-// mode only).  Each unit writes its (max, fp64 sum-exp) partial; the last
-// unit of the sequence runs the accept tests.
+// (maximum, fp64 sum of exp2((x - maximum) c)) of rows r0 .. r0+NB-1 from
+// their S chunk partials, warp-collective: lane c takes chunks c, c + 32, ...
+// (the loads of all NB rows issued together), then fixed butterflies.  Every
+// lane returns the same values.
+template <int NB>
+__device__ __forceinline__ void rows_lse(const LseD* P, int S, int r0, int nrows, float c2,
+                                         float (&Mo)[NB], double (&So)[NB]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+        Mo[j] = -INFINITY;
+        So[j] = 0.0;
+    }
+    for (int c = lane; c < S; c += 32) {
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+            if (j < nrows) Mo[j] = fmaxf(Mo[j], __ldcg(&P[(int64_t)(r0 + j) * S + c].m));
+    }
+#pragma unroll
+    for (int j = 0; j < NB; ++j) Mo[j] = warp_max(Mo[j]);
+    for (int c = lane; c < S; c += 32) {
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+            if (j < nrows) {
+                const LseD* p = &P[(int64_t)(r0 + j) * S + c];
+                const float pm = __ldcg(&p->m);
+                const double ps = __ldcg(&p->s);
+                if (pm != -INFINITY) So[j] += ps * exp2(((double)pm - (double)Mo[j]) * (double)c2);
+            }
+    }
+#pragma unroll
+    for (int j = 0; j < NB; ++j) So[j] = warp_sum(So[j]);
+}
+
+// The accept tests of one sequence, by the warp whose unit completed it:
+// lane j takes target row j (and draft row j) from the chunk partials.
 __device__ __forceinline__ void sample_finish(
     const void* __restrict__ target, const void* __restrict__ draft, const LseD* P, int G,
     int64_t V, int S, int es, float inv_t, float c2, const int32_t* __restrict__ draft_tok,
@@ -170,22 +219,25 @@ __device__ __forceinline__ void sample_finish(
     int32_t* __restrict__ out_tok, float* __restrict__ ratio_dbg, float* __restrict__ u_dbg,
     SampleInfo* __restrict__ info) {
     const int lane = threadIdx.x & 31;
-    auto row_lse = [&](int rrow) {  // chunk order
-        LseD acc{-INFINITY, 0.0f, 0.0};
-        for (int c = 0; c < S; ++c) {
-            LseD p{__ldcg(&P[(int64_t)rrow * S + c].m), 0.0f, __ldcg(&P[(int64_t)rrow * S + c].s)};
-            acc = lse_merge(acc, p, c2);
-        }
-        return acc;
-    };
     auto elem = [&](const void* base, int64_t row, int32_t v) -> double {
         if (es == 2)
             return (double)__uint_as_float((uint32_t)((const uint16_t*)base)[row * V + v] << 16);
         return (double)((const float*)base)[row * V + v];
     };
+    // lane j: (max, sum-exp) of target row j and draft row j
     LseD lt{-INFINITY, 0.0f, 0.0}, lq{-INFINITY, 0.0f, 0.0};
-    if (lane <= G) lt = row_lse(lane);
-    if (q_mode == DFLASH2_Q_SOFTMAX && lane < G) lq = row_lse(G + 1 + lane);
+    const int nrows = (q_mode == DFLASH2_Q_SOFTMAX) ? 2 * G + 1 : G + 1;
+    for (int r0 = 0; r0 < nrows; r0 += 4) {
+        float Mr[4];
+        double Sr[4];
+        rows_lse<4>(P, S, r0, min(4, nrows - r0), c2, Mr, Sr);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int rr = r0 + j;
+            if (rr <= G && lane == rr) lt = LseD{Mr[j], 0.0f, Sr[j]};
+            if (rr > G && rr < nrows && lane == rr - G - 1) lq = LseD{Mr[j], 0.0f, Sr[j]};
+        }
+    }
     bool reject = false;
     if (lane < G) {
         const int32_t d = draft_tok[(int64_t)b * G + lane];
@@ -228,70 +280,12 @@ __device__ __forceinline__ void sample_finish(
     }
 }
 
-// A chunk's (max, sum-exp) in two levels.  Each thread holds its 64
-// elements in registers, takes its own max m and s = sum exp2(x c - m c)
-// (fp32 within a 16-byte vector, fp64 across vectors), each exponent one FMA
-// against mc = fl(m c); its warp rescales the thread sums to the warp max,
-// taking out the product's rounding error e = m c - mc (exact in fp32, and as
-// large as 6e-5 at |m c| ~ 1e3) in the same factor, adds them (butterfly),
-// and lane 0 leaves (M_w, S_w) in shared memory.  The CTA's eight warp pairs are merged later by
-// thread 0 in warp order (warp_pairs_merge).
-template <bool BF16, class C>
-__device__ __forceinline__ void warp_lse_pair(const C& ch, float c2, float* s_m, double* s_s) {
-    using R = Row<BF16>;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint4 v[R::NV];
-#pragma unroll
-    for (int i = 0; i < R::NV; ++i) v[i] = ch.vec(i);
-    float m = vec_max<BF16>(v[0]);
-#pragma unroll
-    for (int i = 1; i < R::NV; ++i) m = fmaxf(m, vec_max<BF16>(v[i]));
-    double s = 0.0;
-    const float mc = -m * c2;
-    if (m != -INFINITY) {
-#pragma unroll
-        for (int i = 0; i < R::NV; ++i) {
-            float tt[R::VW];
-#pragma unroll
-            for (int e = 0; e < R::VW; ++e) tt[e] = ex2(fmaf(R::elem(v[i], e), c2, mc));
-#pragma unroll
-            for (int w = R::VW / 2; w > 0; w >>= 1)
-#pragma unroll
-                for (int e = 0; e < w; ++e) tt[e] += tt[e + w];
-            s += (double)tt[0];
-        }
-    }
-    float M = m;
-#pragma unroll
-    for (int j = 16; j > 0; j >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, j));
-    if (s > 0.0) s *= (double)ex2((m - M) * c2 - fmaf(m, c2, mc));
-#pragma unroll
-    for (int j = 16; j > 0; j >>= 1) s += __shfl_xor_sync(FULL, s, j);
-    if (lane == 0) {
-        s_m[warp] = M;
-        s_s[warp] = s;
-    }
-}
-__device__ __forceinline__ LseD warp_pairs_merge(const float* s_m, const double* s_s, float c2) {
-    float M = s_m[0];
-#pragma unroll
-    for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, s_m[w]);
-    double S = 0.0;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w)
-        if (s_s[w] > 0.0) S += s_s[w] * (double)ex2((s_m[w] - M) * c2);
-    return {M, 0.0f, S};
-}
-
 // Units are (sequence b, row rr, chunk): rows 0..G of a sequence are its
-// target rows, G+1..2G its draft rows (softmax mode only).  Per unit the
-// block meets once: after the unit's copy has landed.  At that barrier every
-// warp has also left its pair for the previous unit and finished reading the
-// previous slot, so warp 0 then refills that slot with the unit after next,
-// merges the previous unit's pairs and stores its partial; the publisher that
-// completes a sequence runs its accept tests in warp 0.
+// target rows, G+1..2G its draft rows (softmax mode only).  A unit's partial
+// is the chunk maximum and the fp64 sum of exp2((x - m) c) against it; a
+// warp publishes its consecutive units of one sequence together.
 template <bool BF16, bool TMA>
-__global__ void __launch_bounds__(NT, 3) verify_sample_scan_kernel(
+__global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_scan_kernel(
     const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int S,
     int rows_per_seq, int64_t units, float inv_t, float c2, const int32_t* __restrict__ draft_tok,
     uint64_t seed, uint32_t step, const uint32_t* __restrict__ seq_id, int q_mode,
@@ -299,109 +293,74 @@ __global__ void __launch_bounds__(NT, 3) verify_sample_scan_kernel(
     float* __restrict__ u_dbg, LseD* __restrict__ part, SampleInfo* __restrict__ info,
     unsigned* __restrict__ counters) {
     constexpr int ES = BF16 ? 2 : 4;
-    constexpr int SLOT = CHUNK * ES;
+    constexpr int LEN = chunk_len(ES);
     extern __shared__ __align__(128) uint8_t ring[];
-    __shared__ float s_m[2][NT / 32];
-    __shared__ double s_s[2][NT / 32];
-    __shared__ __align__(8) uint64_t s_bar[2];
-    const int t = threadIdx.x, warp = t >> 5;
-    const uint32_t bar0 = smem_u32(&s_bar[0]);
-    const int per_seq = rows_per_seq * S;  // units of one sequence (fits int: checked on the host)
-    struct Geo {
-        int b, rr, c;
-        const char* rowp;
-        int64_t v0, vend;
+    __shared__ __align__(8) uint64_t bars[2 * NCW];
+    const int lane = threadIdx.x & 31;
+    auto rowp = [&](int64_t b, int rr) {
+        return (rr <= G) ? (const char*)target + (b * (G + 1) + rr) * V * ES
+                         : (const char*)draft + (b * G + (rr - G - 1)) * V * ES;
     };
-    auto geom = [&](int u) {
-        Geo g;
-        g.b = u / per_seq;
-        const int rem = u - g.b * per_seq;
-        g.rr = rem / S;
-        g.c = rem - g.rr * S;
-        g.rowp = (g.rr <= G) ? (const char*)target + ((int64_t)g.b * (G + 1) + g.rr) * V * ES
-                             : (const char*)draft + ((int64_t)g.b * G + (g.rr - G - 1)) * V * ES;
-        g.v0 = (int64_t)g.c * CHUNK;
-        g.vend = min(V, g.v0 + (int64_t)CHUNK);
-        return g;
+    pdl_launch_dependents();
+    int64_t lo, hi;
+    warp_range(units, lo, hi);
+    const int n = (int)(hi - lo);
+    UnitCursor uc, ic;  // (sequence, row, chunk) being reduced / to bring in
+    uc.init(lo, S, rows_per_seq);
+    ic = uc;
+    auto src = [&](const UnitCursor& cu, const char*& p, uint32_t& bytes) {
+        const int64_t v0 = (int64_t)cu.c * LEN;
+        p = rowp(cu.g, cu.r) + v0 * ES;
+        bytes = (uint32_t)(min((int64_t)LEN, V - v0) * ES);
     };
-    auto issue = [&](int u, int slot) {
-        const Geo g = geom(u);
-        bulk_g2s(smem_u32(ring + slot * SLOT), g.rowp + g.v0 * ES, (uint32_t)((g.vend - g.v0) * ES),
-                 bar0 + 8 * slot);
-    };
-    int64_t lo64, hi64;
-    cta_range(units, lo64, hi64);
-    const int lo = (int)lo64, hi = (int)hi64;
-    if (TMA) {
-        if (t == 0) {
-            mbar_init(bar0, 1);
-            mbar_init(bar0 + 8, 1);
-            mbar_fence_init();
-            if (lo < hi) issue(lo, 0);
-            if (lo + 1 < hi) issue(lo + 1, 1);
-        }
-        __syncthreads();
-    }
-    // warp 0's record of the previous unit, finished at the next barrier
-    int pb = 0, ppart = 0;
-    bool plast = false;
-    unsigned pending = 0;
-    auto finish_prev = [&](int kk) {  // warp 0
-        if (t == 0) part[ppart] = warp_pairs_merge(s_m[kk & 1], s_s[kk & 1], c2);
-        ++pending;
-        if (plast) {  // done with this sequence: publish its units
-            bool last = false;
-            if (t == 0) last = publish(&counters[pb], pending, (unsigned)per_seq);
-            last = __shfl_sync(FULL, last, 0);
-            if (last)
-                sample_finish(target, draft, part + (int64_t)pb * rows_per_seq * S, G, V, S, ES, inv_t,
-                              c2, draft_tok, seed, step, seq_id ? seq_id[pb] : (uint32_t)pb, q_mode,
-                              pb, n_accept, out_tok, ratio_dbg, u_dbg, info);
-            pending = 0;
-        }
-    };
-    int k = 0;
-    for (int u = lo; u < hi; ++u, ++k) {
-        const Geo g = geom(u);
+    WarpRing r{nullptr, 0u};
+    if (TMA) r = warp_ring_start(ring, bars, n, ic, ChunkT<BF16>::NEG_INF_WORD, src);
+    unsigned seg = 0;
+    for (int k = 0; k < n; ++k, uc.next()) {
+        const int64_t b = uc.g, v0 = (int64_t)uc.c * LEN;
+        const int len = (int)min((int64_t)LEN, V - v0);
+        float M;
+        double Ssum;
         if (TMA) {
-            if (!__syncthreads_and(mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1))) {
-                if (t == 0) {
-                    atomicOr(&g_dev_err, ERR_STREAM);
-                    if (u + 1 < hi) mbar_wait(bar0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
-                }
+            if (!r.wait(k)) {
+                warp_ring_abort(r, k, n);
                 return;
             }
+            const SmemView<BF16> view{r.slot(k), v0, len};
+            uint32_t vm[NVL];
+            M = warp_max(chunk_pass1<BF16>(view, vm));
+            Ssum = chunk_expsum<BF16>(view, M, c2);
+            warp_ring_next(r, k, n, ic, ChunkT<BF16>::NEG_INF_WORD, src);
         } else {
-            __syncthreads();
+            const GlobalView<BF16> view{(const uint8_t*)rowp(b, uc.r), v0, len};
+            uint32_t vm[NVL];
+            M = warp_max(chunk_pass1<BF16>(view, vm));
+            Ssum = chunk_expsum<BF16>(view, M, c2);
         }
-        if (warp == 0) {
-            if (TMA && t == 0 && k >= 1 && u + 1 < hi) issue(u + 1, (k + 1) & 1);
-            if (k >= 1) finish_prev(k - 1);
-            pb = g.b;
-            ppart = (g.b * rows_per_seq + g.rr) * S + g.c;
-            plast = (u + 1 == hi) || ((u + 1) / per_seq != g.b);
-        }
-        if (TMA) {
-            warp_lse_pair<BF16>(SmemChunk<BF16>{ring + (k & 1) * SLOT, g.v0, g.vend}, c2, s_m[k & 1],
-                                s_s[k & 1]);
-        } else {
-            RegChunk<BF16> ch;
-            ch.load(g.rowp, g.v0, g.vend);
-            warp_lse_pair<BF16>(ch, c2, s_m[k & 1], s_s[k & 1]);
+        ++seg;
+        if (lane == 0) part[(b * rows_per_seq + uc.r) * S + uc.c] = LseD{M, 0.0f, Ssum};
+        if (k + 1 == n || uc.last_of_group()) {  // done with this sequence: publish
+            bool last = false;
+            if (lane == 0) last = publish(&counters[b], seg, (unsigned)(rows_per_seq * S));
+            if (__shfl_sync(FULL, last, 0)) {
+                __syncwarp();  // lane 0's acquire covers the whole warp's reads
+                sample_finish(target, draft, part + b * rows_per_seq * S, G, V, S, ES, inv_t, c2,
+                              draft_tok, seed, step, seq_id ? seq_id[b] : (uint32_t)b, q_mode,
+                              (int)b, n_accept, out_tok, ratio_dbg, u_dbg, info);
+            }
+            seg = 0;
         }
     }
-    __syncthreads();
-    if (warp == 0 && k >= 1) finish_prev(k - 1);
 }
 
 // ------------------------------------------------------------------ sampling, pass 2
-// Draw weight of one element of the row the sequence draws from:
+// Draw weight of one element of the row the sequence draws from (draw_w):
 //   p_v = exp2((x_v - mt) * c - l2t),  q_v likewise,
 //   mode 0: w = max(0, p - q), evaluated as q * expm1(ln p - ln q) with
 //           ln p - ln q = (xt - xq) * invT - (logZ_t - logZ_q): the same
 //           value, without the cancellation of p - q when p and q agree;
-//   mode 1: w = p, 0 at d;  mode 2: w = p.
-// With use_p (the residual was empty by rounding) the weight is p.
+//   mode 1: w = p, 0 at d;  mode 2: w = p (also the fallback when the
+//   residual is empty by rounding).
 // e^d - 1 for d > 0: the Taylor series to d^8 for d <= 1/2 (truncation below
 // 6e-9 relative there), e^d - 1 from exp2 above, where the subtraction costs
 // at most two bits.
@@ -418,237 +377,104 @@ __device__ __forceinline__ float expm1_pos(float d) {
     return p * d;
 }
 
-__device__ __forceinline__ float draw_weight(float xt, float xq, int64_t v, const SampleInfo& I,
-                                             float c, float inv_t, bool use_p) {
-    if (I.mode == 0 && !use_p) {
+// The draw of one sequence covers DLEN elements per CTA of the row it draws
+// from; thread t holds DEPT consecutive elements.  A thread's sum: fp32 over a
+// 16-byte vector (index order, pairwise), fp64 across vectors.
+constexpr int DLEN = 8192;
+constexpr int DT = 256;
+constexpr int DEPT = DLEN / DT;
+// CTAs per row the draw handles (their sums sit in shared memory): V <= 4096 * 8192.
+constexpr int64_t DRAW_MAX_CHUNKS = 4096;
+
+// The draw weight for a mode known at compile time (MODE 0: residual,
+// 1: p without d, 2: p; the residual-empty fallback draws with MODE 2).
+template <int MODE>
+__device__ __forceinline__ float draw_w(float xt, float xq, int64_t v, const SampleInfo& I, float c2,
+                                        float inv_t) {
+    if (MODE == 0) {
         const float dlog = (xt - xq) * inv_t - I.dl;
         if (!(dlog > 0.0f)) return 0.0f;
-        return ex2((xq - I.mq) * c - I.l2q) * expm1_pos(dlog);
+        return ex2((xq - I.mq) * c2 - I.l2q) * expm1_pos(dlog);
     }
-    if (I.mode == 1 && !use_p && v == I.d) return 0.0f;
-    return ex2((xt - I.mt) * c - I.l2t);
+    if (MODE == 1 && v == I.d) return 0.0f;
+    return ex2((xt - I.mt) * c2 - I.l2t);
 }
 
-// Element `off` of a chunk held in shared memory, widened to fp32 (exact).
-template <bool BF16>
-__device__ __forceinline__ float smem_elem(const uint8_t* buf, int off) {
-    if (BF16) return __uint_as_float((uint32_t)((const uint16_t*)buf)[off] << 16);
-    return ((const float*)buf)[off];
-}
-
-// Sum of the draw weights of thread t's 64 contiguous elements
-// [v0 + 64 t, v0 + 64 t + 64) of the chunk in shared memory: fp32 within a
-// 16-byte vector (index order), fp64 across the vectors.  Thread t starts at
-// its vector t mod NV, so the eight threads of a quarter warp read eight
-// different bank groups.
-template <bool BF16>
-__device__ __forceinline__ double chunk_thread_sum(const uint8_t* tb, const uint8_t* qb, int64_t v0,
-                                                   int64_t vend, const SampleInfo& I, float c2,
-                                                   float inv_t, bool use_p) {
-    using R = Row<BF16>;
-    constexpr int ES = BF16 ? 2 : 4;
-    const int t = threadIdx.x;
-    const bool with_q = I.mode == 0 && !use_p;
-    double s = 0.0;
-#pragma unroll 2
-    for (int j = 0; j < R::NV; ++j) {
-        const int off = t * EPT + ((j + t) & (R::NV - 1)) * R::VW;
-        if (v0 + off >= vend) continue;
-        const uint4 rt = *(const uint4*)(tb + off * ES);
-        const uint4 rq = with_q ? *(const uint4*)(qb + off * ES) : make_uint4(0, 0, 0, 0);
-        float sv = 0.0f;
+// The DEPT elements [vb, vb + DEPT) of a row as 16-byte vectors (-inf past V).
+template <bool BF16, bool VEC>
+__device__ __forceinline__ void draw_load(const char* row, int64_t vb, int64_t V,
+                                          uint4 (&x)[DEPT / ChunkT<BF16>::VW]) {
+    using C = ChunkT<BF16>;
+    constexpr int NV = DEPT / C::VW;
+    if (VEC && vb + DEPT <= V) {
+        const uint4* p = (const uint4*)(row + vb * C::ES);
 #pragma unroll
-        for (int e = 0; e < R::VW; ++e) {
-            const int64_t v = v0 + off + e;
-            if (v < vend)
-                sv += draw_weight(R::elem(rt, e), R::elem(rq, e), v, I, c2, inv_t, use_p);
-        }
-        s += (double)sv;
+        for (int g = 0; g < NV; ++g) x[g] = __ldg(p + g);
+    } else {
+        const GlobalView<BF16> view{(const uint8_t*)row, vb, (int)max((int64_t)0, min((int64_t)DEPT, V - vb))};
+#pragma unroll
+        for (int g = 0; g < NV; ++g) x[g] = view.vec(g);
+    }
+}
+
+// A thread's weight sum over its DEPT elements.
+template <bool BF16, bool VEC, int MODE>
+__device__ __forceinline__ double draw_thread_sum(const char* trow, const char* qrow, int64_t vb,
+                                                  int64_t V, const SampleInfo& I, float c2,
+                                                  float inv_t) {
+    using C = ChunkT<BF16>;
+    constexpr int NV = DEPT / C::VW;
+    uint4 xt[NV], xq[NV];
+    draw_load<BF16, VEC>(trow, vb, V, xt);
+    if (MODE == 0) draw_load<BF16, VEC>(qrow, vb, V, xq);
+    double s = 0.0;
+#pragma unroll
+    for (int g = 0; g < NV; ++g) {
+        float sv[C::VW];
+#pragma unroll
+        for (int e = 0; e < C::VW; ++e)
+            sv[e] = draw_w<MODE>(C::elem(xt[g], e), MODE == 0 ? C::elem(xq[g], e) : 0.0f,
+                                 vb + g * C::VW + e, I, c2, inv_t);
+#pragma unroll
+        for (int h = C::VW / 2; h > 0; h >>= 1)
+#pragma unroll
+            for (int e = 0; e < h; ++e) sv[e] += sv[e + h];
+        s += (double)sv[0];
     }
     return s;
 }
 
-// Block sum in a fixed order (warp butterflies, then the warps in order).
-__device__ __forceinline__ double block_sum(double v, double* s_warp) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// The first element of [vb, vb + DEPT) whose running prefix (from `run`)
+// exceeds t, else the last element with mass, else -1.
+template <bool BF16, bool VEC, int MODE>
+__device__ __forceinline__ int draw_walk(const char* trow, const char* qrow, int64_t vb, int64_t V,
+                                         const SampleInfo& I, float c2, float inv_t, double run,
+                                         double tt) {
+    using C = ChunkT<BF16>;
+    constexpr int NV = DEPT / C::VW;
+    uint4 xt[NV], xq[NV];
+    draw_load<BF16, VEC>(trow, vb, V, xt);
+    if (MODE == 0) draw_load<BF16, VEC>(qrow, vb, V, xq);
+    int pick = -1, lastm = -1;
 #pragma unroll
-    for (int k = 16; k > 0; k >>= 1) v += __shfl_xor_sync(FULL, v, k);
-    __syncthreads();
-    if (lane == 0) s_warp[warp] = v;
-    __syncthreads();
-    double tot = 0.0;
-    for (int w = 0; w < NT / 32; ++w) tot += s_warp[w];
-    return tot;
+    for (int g = 0; g < NV; ++g)
+#pragma unroll
+        for (int e = 0; e < C::VW; ++e) {
+            const float w = draw_w<MODE>(C::elem(xt[g], e), MODE == 0 ? C::elem(xq[g], e) : 0.0f,
+                                         vb + g * C::VW + e, I, c2, inv_t);
+            if (w > 0.0f) lastm = g * C::VW + e;
+            run += (double)w;
+            if (pick < 0 && run > tt) pick = g * C::VW + e;
+        }
+    return pick >= 0 ? pick : lastm;
 }
 
-// Thread-block cluster plumbing (PTX ISA: barrier.cluster, mapa).
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ uint32_t cluster_size() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Store v at `local` (a shared-memory address of this kernel) in CTA `rank`
-// of the cluster.
-__device__ __forceinline__ void st_cluster(double* local, double v, uint32_t rank) {
-    uint32_t ra;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
-    asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(ra), "d"(v) : "memory");
-}
-
-// One cluster of CL CTAs per sequence; CTA r holds the chunks
-// [r S / CL, (r + 1) S / CL) of the row the sequence draws from (and of the
-// draft row in mode 0), brought into shared memory by one bulk copy each.
-// Every CTA sums its chunks' draw weights and stores each chunk sum into
-// every CTA of the cluster; after one cluster barrier all CTAs hold the same
-// S sums, take R and the crossing chunk c* (the first c whose inclusive
-// prefix exceeds t = u' R) in the same order, and the CTA holding c* finds the
-// thread, then the element, from the data it already has.  Control flow up to
-// the last cluster barrier is the same in every CTA of the cluster (the
-// fallback to p is decided from the same sums everywhere).
-template <bool BF16, bool TMA>
-__global__ void __launch_bounds__(NT, 3) verify_sample_draw_kernel(
-    const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int S,
-    float c2, float inv_t, const SampleInfo* __restrict__ info, int32_t* __restrict__ out_tok) {
-    constexpr int ES = BF16 ? 2 : 4;
-    using R = Row<BF16>;
-    extern __shared__ __align__(128) uint8_t s_dyn[];  // target chunk | draft chunk | sums[2][S]
-    uint8_t* tbuf = s_dyn;
-    uint8_t* qbuf = s_dyn + CHUNK * ES;
-    double* s_all = (double*)(s_dyn + 2 * CHUNK * ES);
-    __shared__ double s_warp[NT / 32];
-    __shared__ double s_scan[NT];
-    __shared__ double s_base, s_t;
-    __shared__ int s_cstar, s_fallback, s_pick_thread, s_done, s_last;
-    __shared__ __align__(8) uint64_t s_bar;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int CL = (int)cluster_size(), rank = (int)cluster_rank();
-    const int b = blockIdx.x / CL;
-    const SampleInfo I = info[b];
-    const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
-    const char* qrow = (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
-    const int c0 = (int)((int64_t)rank * S / CL), c1 = (int)((int64_t)(rank + 1) * S / CL);
-    const uint32_t bar = smem_u32(&s_bar);
-    if (TMA && t == 0) {
-        mbar_init(bar, 1);
-        mbar_fence_init();
-    }
-    __syncthreads();
-    cluster_arrive_relaxed();  // this CTA has started: its shared memory may be written
-
-    int loaded = -1, nload = 0;
-    bool copies_ok = true;
-    // Bring chunk c of the target row (and of the draft row if need_q) into
-    // shared memory; block-uniform.
-    auto load_chunk = [&](int c, bool need_q) {
-        const int64_t v0 = (int64_t)c * CHUNK, vend = min(V, v0 + (int64_t)CHUNK);
-        const int n = (int)(vend - v0);
-        __syncthreads();  // every thread is done with the previous chunk
-        if (TMA) {
-            if (!copies_ok) return;
-            if (t == 0) {
-                const uint32_t bytes = (uint32_t)n * ES;
-                mbar_expect_tx(bar, need_q ? 2 * bytes : bytes);
-                bulk_g2s_nx(smem_u32(tbuf), trow + v0 * ES, bytes, bar);
-                if (need_q) bulk_g2s_nx(smem_u32(qbuf), qrow + v0 * ES, bytes, bar);
-            }
-            const bool ok = __syncthreads_and(mbar_wait(bar, (uint32_t)(nload & 1)));
-            ++nload;
-            if (!ok) {  // the copy never landed: flag it and issue no more
-                if (t == 0) atomicOr(&g_dev_err, ERR_STREAM);
-                copies_ok = false;
-            }
-        } else {
-            for (int e = t; e < n; e += NT) {
-                if (BF16) {
-                    ((uint16_t*)tbuf)[e] = ((const uint16_t*)trow)[v0 + e];
-                    if (need_q) ((uint16_t*)qbuf)[e] = ((const uint16_t*)qrow)[v0 + e];
-                } else {
-                    ((float*)tbuf)[e] = ((const float*)trow)[v0 + e];
-                    if (need_q) ((float*)qbuf)[e] = ((const float*)qrow)[v0 + e];
-                }
-            }
-            __syncthreads();
-        }
-        loaded = c;
-    };
-    // One round: every owned chunk's sum into sums[round][c] of every CTA,
-    // then the cluster barrier.  Returns this thread's sum of the last chunk.
-    auto round_sums = [&](int round, bool use_p) -> double {
-        const bool need_q = I.mode == 0 && !use_p;
-        double my = 0.0;
-        for (int c = c0; c < c1; ++c) {
-            if (loaded != c) load_chunk(c, need_q);
-            const int64_t v0 = (int64_t)c * CHUNK, vend = min(V, v0 + (int64_t)CHUNK);
-            my = chunk_thread_sum<BF16>(tbuf, qbuf, v0, vend, I, c2, inv_t, use_p);
-            const double cs = block_sum(my, s_warp);
-            if (round == 0 && c == c0) cluster_wait();  // every CTA of the cluster has started
-            if (t < CL) st_cluster(&s_all[round * S + c], cs, (uint32_t)t);
-        }
-        cluster_arrive();
-        cluster_wait();
-        return my;
-    };
-
-    double mysum = round_sums(0, false);
-    if (t == 0) {
-        double Rm = 0.0;
-        for (int c = 0; c < S; ++c) Rm += s_all[c];
-        s_fallback = !(Rm > 0.0);
-    }
-    __syncthreads();
-    const bool use_p = s_fallback != 0;  // the same in every CTA of the cluster
-    if (use_p) mysum = round_sums(1, true);  // residual empty by rounding: draw from p_n (rare)
-    const double* sums = s_all + (use_p ? S : 0);
-    if (t == 0) {
-        double Rm = 0.0;
-        for (int c = 0; c < S; ++c) Rm += sums[c];
-        const double tt = (double)I.u_res * Rm;
-        double pre = 0.0;
-        int cstar = -1, clast = 0;
-        for (int c = 0; c < S; ++c) {
-            const double wc = sums[c];
-            if (wc > 0.0) clast = c;
-            if (cstar < 0 && pre + wc > tt) cstar = c;
-            if (cstar < 0) pre += wc;
-        }
-        if (cstar < 0) {  // rounding left t at the top: the last chunk with mass
-            cstar = clast;
-            pre = 0.0;
-            for (int c = 0; c < clast; ++c) pre += sums[c];
-        }
-        s_cstar = cstar;
-        s_base = pre;
-        s_t = tt;
-        s_pick_thread = NT;
-        s_done = 0;
-        s_last = -1;
-    }
-    __syncthreads();
-    const int cstar = s_cstar;
-    if (cstar < c0 || cstar >= c1) return;  // another CTA of the cluster draws
-    if (loaded != cstar) {  // this CTA holds several chunks: fetch c* again
-        load_chunk(cstar, I.mode == 0 && !use_p);
-        const int64_t v0 = (int64_t)cstar * CHUNK, vend = min(V, v0 + (int64_t)CHUNK);
-        mysum = chunk_thread_sum<BF16>(tbuf, qbuf, v0, vend, I, c2, inv_t, use_p);
-    }
-    const int64_t v0 = (int64_t)cstar * CHUNK, vend = min(V, v0 + (int64_t)CHUNK);
-    const double tt = s_t;
-    // inclusive scan of the thread sums in thread (= index) order
-    double incl = mysum;
+// Inclusive scan of the threads' values in thread order (fp64): warp scans,
+// then the warps' totals in warp order.  `total` is the last thread's value,
+// bit for bit.  Block-wide (two barriers).
+__device__ __forceinline__ double block_incl_scan(double x, double* s_warp, double& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    double incl = x;
 #pragma unroll
     for (int k = 1; k < 32; k <<= 1) {
         const double o = __shfl_up_sync(FULL, incl, k);
@@ -656,70 +482,132 @@ __global__ void __launch_bounds__(NT, 3) verify_sample_draw_kernel(
     }
     if (lane == 31) s_warp[warp] = incl;
     __syncthreads();
-    double wbase = 0.0;
-    for (int w = 0; w < warp; ++w) wbase += s_warp[w];
-    incl += wbase;
-    s_scan[t] = incl;
-    if (s_base + incl > tt) atomicMin(&s_pick_thread, t);
+    double base = 0.0;
+    for (int w = 0; w < warp; ++w) base += s_warp[w];
+    double tot = 0.0;
+    for (int w = 0; w < DT / 32 - 1; ++w) tot += s_warp[w];
+    total = tot + s_warp[DT / 32 - 1];
     __syncthreads();
-    const int pt = s_pick_thread;
-    const bool with_q = I.mode == 0 && !use_p;
-    if (pt < NT && warp == 0) {
-        // warp 0 walks thread pt's 64 elements, two per lane, in index order
-        const int off = pt * EPT + 2 * lane;
-        const int64_t vb = v0 + off;
-        float w0 = 0.0f, w1 = 0.0f;
-        if (vb < vend)
-            w0 = draw_weight(smem_elem<BF16>(tbuf, off), with_q ? smem_elem<BF16>(qbuf, off) : 0.0f,
-                             vb, I, c2, inv_t, use_p);
-        if (vb + 1 < vend)
-            w1 = draw_weight(smem_elem<BF16>(tbuf, off + 1),
-                             with_q ? smem_elem<BF16>(qbuf, off + 1) : 0.0f, vb + 1, I, c2, inv_t,
-                             use_p);
-        double incl2 = (double)w0 + (double)w1;
-#pragma unroll
-        for (int kk = 1; kk < 32; kk <<= 1) {
-            const double o = __shfl_up_sync(FULL, incl2, kk);
-            if (lane >= kk) incl2 += o;
-        }
-        const double base = s_base + (pt > 0 ? s_scan[pt - 1] : 0.0);
-        const double before = base + incl2 - ((double)w0 + (double)w1);
-        const bool p0 = before + (double)w0 > tt;
-        const bool p1 = before + (double)w0 + (double)w1 > tt;
-        const unsigned m0 = __ballot_sync(FULL, p0), m1 = __ballot_sync(FULL, p1);
-        const unsigned has = __ballot_sync(FULL, w0 > 0.0f || w1 > 0.0f);
-        int pick = -1;
-        if (m0 | m1) {  // the first element whose inclusive prefix exceeds t
-            const int l0 = m0 ? __ffs(m0) - 1 : 32, l1 = m1 ? __ffs(m1) - 1 : 32;
-            pick = (l0 <= l1) ? 2 * l0 : 2 * l1 + 1;
-        } else if (has) {  // rounding: the last element with mass
-            const int ll = 31 - __clz(has);
-            const float lw1 = __shfl_sync(FULL, w1, ll);
-            pick = 2 * ll + (lw1 > 0.0f ? 1 : 0);
-        }
-        if (lane == 0 && pick >= 0) {
-            out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(v0 + pt * EPT + pick);
-            s_done = 1;
-        }
-    }
-    __syncthreads();
-    if (!s_done) {  // block-uniform: rounding left t above the chunk's scan
-        if (mysum > 0.0) {
-            int lastpos = -1;
-#pragma unroll 1
-            for (int e = 0; e < EPT; ++e) {
-                const int off = t * EPT + e;
-                const int64_t v = v0 + off;
-                if (v < vend &&
-                    draw_weight(smem_elem<BF16>(tbuf, off), with_q ? smem_elem<BF16>(qbuf, off) : 0.0f,
-                                v, I, c2, inv_t, use_p) > 0.0f)
-                    lastpos = e;
-            }
-            if (lastpos >= 0) atomicMax(&s_last, t * EPT + lastpos);
+    return base + incl;
+}
+
+// One mode of the draw (see verify_sample_draw_kernel).  first: every CTA
+// sums its own chunk and only the last of the sequence goes on; else (the
+// fallback to p_n) the calling CTA computes every chunk sum itself.
+template <bool BF16, bool VEC, int MODE>
+__device__ __forceinline__ void draw_body(const char* trow, const char* qrow, int64_t V, int D,
+                                          int c, int b, int G, float c2, float inv_t,
+                                          const SampleInfo& I, double* __restrict__ dsum,
+                                          unsigned* __restrict__ dcount,
+                                          int32_t* __restrict__ out_tok, double* s_sums, bool first) {
+    __shared__ double s_warp[DT / 32];
+    __shared__ double s_incl[DT];
+    __shared__ double s_base, s_t;
+    __shared__ int s_cstar, s_pick, s_last_mass, s_use_p;
+    __shared__ bool s_last;
+    const int t = threadIdx.x;
+    double total;
+    if (first) {  // this CTA's chunk sum; the last CTA of the sequence goes on
+        const double my = draw_thread_sum<BF16, VEC, MODE>(
+            trow, qrow, (int64_t)c * DLEN + (int64_t)DEPT * t, V, I, c2, inv_t);
+        block_incl_scan(my, s_warp, total);
+        if (t == 0) {
+            dsum[(int64_t)b * D + c] = total;
+            s_last = publish(&dcount[b], 1u, (unsigned)D);
         }
         __syncthreads();
-        if (t == 0 && s_last >= 0) out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(v0 + s_last);
+        if (!s_last) return;
+        for (int cc = t; cc < D; cc += DT) s_sums[cc] = __ldcg(&dsum[(int64_t)b * D + cc]);
+    } else {  // the chunk sums of p_n (the residual was empty by rounding)
+        for (int cc = 0; cc < D; ++cc) {
+            const double my = draw_thread_sum<BF16, VEC, MODE>(
+                trow, qrow, (int64_t)cc * DLEN + (int64_t)DEPT * t, V, I, c2, inv_t);
+            block_incl_scan(my, s_warp, total);
+            if (t == 0) s_sums[cc] = total;
+        }
     }
+    __syncthreads();
+    if (t == 0) {
+        double R = 0.0;
+        for (int cc = 0; cc < D; ++cc) R += s_sums[cc];
+        s_use_p = first && MODE != 2 && !(R > 0.0);
+        const double tt = (double)I.u_res * R;
+        double pre = 0.0;
+        int cstar = -1;
+        for (int cc = 0; cc < D; ++cc) {
+            if (pre + s_sums[cc] > tt) {
+                cstar = cc;
+                break;
+            }
+            pre += s_sums[cc];
+        }
+        if (cstar < 0) {  // unreachable while R > 0 (t < R): the last chunk with mass
+            pre = 0.0;
+            cstar = 0;
+            for (int cc = 0; cc < D; ++cc)
+                if (s_sums[cc] > 0.0) cstar = cc;
+            for (int cc = 0; cc < cstar; ++cc) pre += s_sums[cc];
+        }
+        s_cstar = cstar;
+        s_base = pre;
+        s_t = tt;
+        s_pick = DT;
+        s_last_mass = -1;
+    }
+    __syncthreads();
+    if constexpr (MODE != 2) {
+        if (s_use_p) {  // block-uniform
+            draw_body<BF16, VEC, 2>(trow, qrow, V, D, c, b, G, c2, inv_t, I, dsum, dcount,
+                                    out_tok, s_sums, false);
+            return;
+        }
+    }
+    const int cstar = s_cstar;
+    const int64_t vb = (int64_t)cstar * DLEN + (int64_t)DEPT * t;
+    const double my = draw_thread_sum<BF16, VEC, MODE>(trow, qrow, vb, V, I, c2, inv_t);
+    const double incl = block_incl_scan(my, s_warp, total);
+    s_incl[t] = incl;
+    const double tt = s_t, base = s_base;
+    if (base + incl > tt) atomicMin(&s_pick, t);
+    if (my > 0.0) atomicMax(&s_last_mass, t);
+    __syncthreads();
+    int pt = s_pick;
+    if (pt == DT) pt = s_last_mass;  // rounding left t above the chunk's scan
+    if (t == pt) {
+        const int e = draw_walk<BF16, VEC, MODE>(trow, qrow, vb, V, I, c2, inv_t,
+                                                 base + (t > 0 ? s_incl[t - 1] : 0.0), tt);
+        if (e >= 0) out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(vb + e);
+    }
+}
+
+// Grid (chunks of the drawn row, sequences).  Every CTA stores its chunk's
+// weight sum and counts itself in; the last CTA of a sequence takes
+// R = sum of the chunk sums in chunk order and t = u' R, finds the first chunk
+// whose inclusive prefix exceeds t, and scans it: the first thread whose
+// inclusive prefix exceeds t, then the first element of that thread.  If the
+// residual is empty by rounding (R = 0) the last CTA draws from p_n instead,
+// recomputing every chunk sum itself (rare).
+template <bool BF16, bool VEC>
+__global__ void __launch_bounds__(DT, 4) verify_sample_draw_kernel(
+    const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int D,
+    float c2, float inv_t, const SampleInfo* __restrict__ info, double* __restrict__ dsum,
+    unsigned* __restrict__ dcount, int32_t* __restrict__ out_tok) {
+    constexpr int ES = BF16 ? 2 : 4;
+    extern __shared__ double s_sums[];  // [D], the last CTA's copy of the chunk sums
+    const int c = blockIdx.x, b = blockIdx.y;
+    pdl_wait();  // the scan's SampleInfo, and every earlier write, are visible
+    const SampleInfo I = info[b];
+    const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
+    const char* qrow = (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
+    if (I.mode == 0)
+        draw_body<BF16, VEC, 0>(trow, qrow, V, D, c, b, G, c2, inv_t, I, dsum, dcount, out_tok,
+                                s_sums, true);
+    else if (I.mode == 1)
+        draw_body<BF16, VEC, 1>(trow, qrow, V, D, c, b, G, c2, inv_t, I, dsum, dcount, out_tok,
+                                s_sums, true);
+    else
+        draw_body<BF16, VEC, 2>(trow, qrow, V, D, c, b, G, c2, inv_t, I, dsum, dcount, out_tok,
+                                s_sums, true);
 }
 
 }  // namespace dfl
@@ -737,66 +625,27 @@ unsigned dfl_errors_verify(int clear) {
     return v;
 }
 
-template <class Kern>
-static int prep_stream_kernel(Kern kern, size_t dyn) {
-    if (dyn > 48 * 1024 &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess)
-        return DFLASH2_ECUDA;
-    return DFLASH2_OK;
-}
-
-// Cluster size of the draw: one CTA per chunk up to 16 (the non-portable
-// maximum), fewer if the device cannot co-schedule that many CTAs of this
-// shared-memory size.  The kernel's shared-memory ceiling is set once per
-// device to the largest size any vocabulary needs (the ceiling is a property
-// of the kernel, so a smaller call must not lower it); the cluster limit is
-// looked up once per device, kernel and size.
-template <class Kern>
-static int draw_cluster(Kern kern, size_t dyn, size_t dyn_max, int S) {
-    static std::mutex mu;
-    static std::map<std::tuple<int, const void*, size_t>, int> limit;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    std::lock_guard<std::mutex> g(mu);
-    const auto kkey = std::make_tuple(dev, (const void*)kern, (size_t)0);
-    if (limit.find(kkey) == limit.end()) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_max) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-                cudaSuccess)
-            return 0;
-        limit.emplace(kkey, 1);
-    }
-    const auto key = std::make_tuple(dev, (const void*)kern, dyn);
-    auto it = limit.find(key);
-    if (it == limit.end()) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(16);
-        cfg.blockDim = dim3(NT);
-        cfg.dynamicSmemBytes = dyn;
-        int n = 0;
-        if (cudaOccupancyMaxPotentialClusterSize(&n, (const void*)kern, &cfg) != cudaSuccess) return 0;
-        it = limit.emplace(key, n).first;
-    }
-    return std::min(std::min(S, 16), it->second);
-}
-
+// Launch as a programmatic dependent of the previous kernel on the stream:
+// the grid may start while that kernel finishes, and waits (griddepcontrol)
+// for its results before reading them.
 template <class Kern, class... Args>
-static int launch_cluster(Kern kern, int grid, int cl, size_t dyn, cudaStream_t s, Args... args) {
+static cudaError_t launch_dependent(Kern kern, dim3 grid, dim3 block, size_t dyn, cudaStream_t s,
+                                    Args... args) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(NT);
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
     cfg.dynamicSmemBytes = dyn;
     cfg.stream = s;
     cudaLaunchAttribute a[1];
-    a[0].id = cudaLaunchAttributeClusterDimension;
-    a[0].val.clusterDim.x = (unsigned)cl;
-    a[0].val.clusterDim.y = 1;
-    a[0].val.clusterDim.z = 1;
+    a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = a;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? DFLASH2_OK : DFLASH2_ECUDA;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
 }
+
+// Draw grid size per sequence: DLEN-element chunks of the drawn row.
+static inline int64_t draw_chunks(int64_t V) { return (V + DLEN - 1) / DLEN; }
 
 extern "C" int dflash2_verify_greedy(const void* target, int dtype, int B, int G, int64_t V,
                                      const int32_t* draft_tok, int32_t* n_accept, int32_t* out_tok,
@@ -809,10 +658,10 @@ extern "C" int dflash2_verify_greedy(const void* target, int dtype, int B, int G
     if (!aligned(target, es) || !aligned(draft_tok, 4) || !aligned(n_accept, 4) ||
         !aligned(out_tok, 4))
         return DFLASH2_EALIGN;
-    const int64_t S = n_chunks(V);
+    const int64_t S = row_chunks(V, es);
     const int64_t units = (int64_t)B * (G + 1) * S;
     if (units > (int64_t)INT32_MAX) return DFLASH2_ESHAPE;
-    const Layout L = greedy_layout(B, G, V);
+    const Layout L = greedy_layout(B, G, V, es);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return DFLASH2_EWORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     unsigned* counters = (unsigned*)((char*)ws + L.counters_off);
@@ -820,14 +669,13 @@ extern "C" int dflash2_verify_greedy(const void* target, int dtype, int B, int G
     if (cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
     // TMA bulk copies need 16-byte aligned chunk starts and 16-byte multiples
     const bool tma = aligned(target, 16) && (V * es) % 16 == 0;
-#define DFL_GREEDY(BF, TM)                                                                      \
-    do {                                                                                        \
-        auto kern = verify_greedy_kernel<BF, TM>;                                               \
-        const size_t dyn = TM ? 2 * (size_t)CHUNK * (BF ? 2 : 4) : 0;                           \
-        if (prep_stream_kernel(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;                  \
-        kern<<<persistent_grid(kern, NT, dyn, units), NT, dyn, s>>>(target, G, V, (int)S, units, \
-                                                                  draft_tok, n_accept, out_tok, \
-                                                                  part, counters);              \
+#define DFL_GREEDY(BF, TM)                                                                       \
+    do {                                                                                         \
+        auto kern = verify_greedy_kernel<BF, TM>;                                                \
+        const size_t dyn = TM ? (size_t)RING_BYTES : 0;                                          \
+        if (ring_prepare(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;                         \
+        kern<<<ring_grid(units), RING_THREADS, dyn, s>>>(target, G, V, (int)S, units, draft_tok, \
+                                                         n_accept, out_tok, part, counters);     \
     } while (0)
     if (dtype == DFLASH2_BF16) {
         if (tma) DFL_GREEDY(true, true);
@@ -858,35 +706,38 @@ extern "C" int dflash2_verify_sample(const void* target, const void* draft, int 
         !aligned(n_accept, 4) || !aligned(out_tok, 4) || (seq_id && !aligned(seq_id, 4)) ||
         (ratio_dbg && !aligned(ratio_dbg, 4)) || (u_dbg && !aligned(u_dbg, 4)))
         return DFLASH2_EALIGN;
-    const int64_t S = n_chunks(V);
-    if (S > DRAW_MAX_CHUNKS) return DFLASH2_ESHAPE;
+    const int64_t S = row_chunks(V, es);
+    const int64_t D = draw_chunks(V);
+    if (D > DRAW_MAX_CHUNKS) return DFLASH2_ESHAPE;
     const int rows_per_seq = (q_mode == DFLASH2_Q_SOFTMAX) ? 2 * G + 1 : G + 1;
     const int64_t units = (int64_t)B * rows_per_seq * S;
-    if (units > (int64_t)INT32_MAX) return DFLASH2_ESHAPE;
-    const Layout L = sample_layout(B, G, V);
+    if (units > (int64_t)INT32_MAX || B > 65535) return DFLASH2_ESHAPE;
+    const Layout L = sample_layout(B, G, V, es);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return DFLASH2_EWORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
-    unsigned* counters = (unsigned*)((char*)ws + L.counters_off);
+    unsigned* counters = (unsigned*)((char*)ws + L.counters_off);  // [B] scan, [B] draw
     LseD* part = (LseD*)((char*)ws + L.part_off);
+    double* dsum = (double*)((char*)ws + L.part2_off);
     SampleInfo* info = (SampleInfo*)((char*)ws + L.info_off);
-    if (cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
+    if (cudaMemsetAsync(counters, 0, (size_t)B * 8, s) != cudaSuccess) return DFLASH2_ECUDA;
     const void* q = (q_mode == DFLASH2_Q_SOFTMAX) ? draft : nullptr;
     const bool tma = aligned(target, 16) && (!q || aligned(q, 16)) && (V * es) % 16 == 0;
     const float c2 = (float)((double)inv_temperature * LOG2E);
-    const size_t dyn2 = draw_smem(es, S);
+    const size_t dyn2 = (size_t)D * sizeof(double);
 #define DFL_SAMPLE(BF, TM)                                                                        \
     do {                                                                                          \
         auto kern = verify_sample_scan_kernel<BF, TM>;                                            \
-        const size_t dyn = TM ? 2 * (size_t)CHUNK * (BF ? 2 : 4) : 0;                             \
-        if (prep_stream_kernel(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;                    \
-        kern<<<persistent_grid(kern, NT, dyn, units), NT, dyn, s>>>(                              \
+        const size_t dyn = TM ? (size_t)RING_BYTES : 0;                                           \
+        if (ring_prepare(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;                          \
+        kern<<<ring_grid(units), RING_THREADS, dyn, s>>>(                                         \
             target, q, G, V, (int)S, rows_per_seq, units, inv_temperature, c2, draft_tok, seed,   \
             step, seq_id, q_mode, n_accept, out_tok, ratio_dbg, u_dbg, part, info, counters);     \
         auto kern2 = verify_sample_draw_kernel<BF, TM>;                                           \
-        const int cl = draw_cluster(kern2, dyn2, draw_smem((BF ? 2 : 4), DRAW_MAX_CHUNKS), (int)S); \
-        if (cl < 1) return DFLASH2_ECUDA;                                                         \
-        if (launch_cluster(kern2, B * cl, cl, dyn2, s, target, q, G, V, (int)S, c2,               \
-                           inv_temperature, (const SampleInfo*)info, out_tok) != DFLASH2_OK)      \
+        if (ring_prepare(kern2, (size_t)DRAW_MAX_CHUNKS * sizeof(double)) != DFLASH2_OK)          \
+            return DFLASH2_ECUDA;                                                                 \
+        if (launch_dependent(kern2, dim3((unsigned)D, (unsigned)B), dim3(DT), dyn2, s, target, q, \
+                             G, V, (int)D, c2, inv_temperature, (const SampleInfo*)info, dsum,    \
+                             counters + B, out_tok) != cudaSuccess)                               \
             return DFLASH2_ECUDA;                                                                 \
     } while (0)
     if (dtype == DFLASH2_BF16) {

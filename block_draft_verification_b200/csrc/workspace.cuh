@@ -9,14 +9,16 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "ring.cuh"
 
 namespace dfl {
 
-// Partial result of one (row, chunk) unit of dflash2_topk_softmax.
-struct TopkPartial {
+// Partial result of one (row, chunk) unit of dflash2_topk_softmax: the
+// chunk maximum, the chunk's sum of exp2((x - m) c) and its top-16 keys.
+struct TopkPart {
     float m;
-    float s;
-    uint32_t pad[2];
+    float pad;
+    double s;
     uint64_t key[K];
 };
 
@@ -58,18 +60,24 @@ inline Layout make_layout(size_t counters, size_t part, size_t part2 = 0, size_t
     return L;
 }
 
-inline Layout topk_layout(int64_t rows, int64_t V) {
-    int64_t S = n_chunks(V);
-    return make_layout((size_t)rows * 4, (size_t)(rows * S) * sizeof(TopkPartial));
+// Layouts for an element size es (2 for bf16, 4 for fp32; a workspace sized
+// with es = 4 serves both, its chunks being the shorter).
+inline Layout topk_layout(int64_t rows, int64_t V, int es) {
+    const int64_t S = row_chunks(V, es);
+    return make_layout((size_t)rows * 4, (size_t)(rows * S) * sizeof(TopkPart));
 }
-inline Layout greedy_layout(int B, int G, int64_t V) {
-    int64_t S = n_chunks(V);
+inline Layout greedy_layout(int B, int G, int64_t V, int es) {
+    const int64_t S = row_chunks(V, es);
     return make_layout((size_t)B * 4, (size_t)((int64_t)B * (G + 1) * S) * sizeof(uint64_t));
 }
-inline Layout sample_layout(int B, int G, int64_t V) {
-    int64_t S = n_chunks(V);
-    return make_layout((size_t)B * 4, (size_t)((int64_t)B * (2 * G + 1) * S) * sizeof(LseD), 0,
-                       (size_t)B * sizeof(SampleInfo));
+// Sampling: counters of the scan and of the draw ([B] each), the scan's
+// per-unit partials, the draw's per-chunk weight sums (8192 elements per
+// chunk) and the per-sequence hand-over to the draw.
+inline Layout sample_layout(int B, int G, int64_t V, int es) {
+    const int64_t S = row_chunks(V, es);
+    const int64_t D = (V + 8191) / 8192;
+    return make_layout((size_t)B * 8, (size_t)((int64_t)B * (2 * G + 1) * S) * sizeof(LseD),
+                       (size_t)(B * D) * sizeof(double), (size_t)B * sizeof(SampleInfo));
 }
 inline Layout select_layout(int B, int G) {
     return make_layout((size_t)B * 4, (size_t)B * (K + (size_t)K * K * (G - 1)) * sizeof(float));
