@@ -134,31 +134,53 @@ __device__ __forceinline__ void topk_row_merge(const TopkPart* P, int S, int64_t
                                                float* __restrict__ logz) {
     const int lane = threadIdx.x & 31;
     auto ldkey = [](const uint64_t* p) { return (uint64_t)__ldcg((const unsigned long long*)p); };
-    // only a row segment's last chunk carries a list (key[0] != 0)
-    uint64_t acc = 0ull;
-    bool first = true;
-    for (int c0 = 0; c0 < S; c0 += 32) {
-        const int c = c0 + lane;
-        unsigned has = __ballot_sync(FULL, c < S && ldkey(&P[c].key[0]) != 0ull);
-        while (has) {
-            const int cc = c0 + __ffs(has) - 1;
-            has &= has - 1;
-            if (first) {
-                acc = (lane < K) ? ldkey(&P[cc].key[lane]) : 0ull;
-                first = false;
-            } else {
-                acc = warp_merge_desc(lane < K ? acc : ldkey(&P[cc].key[31 - lane]));
-            }
-        }
-    }
+    // round 1: every chunk's (max, sum) and whether it carries a list
     float M = -INFINITY;
     for (int c = lane; c < S; c += 32) M = fmaxf(M, __ldcg(&P[c].m));
     M = warp_max(M);
     double ssum = 0.0;
-    for (int c = lane; c < S; c += 32) {
-        const float mc = __ldcg(&P[c].m);
-        const double sc = __ldcg(&P[c].s);
+    uint64_t acc = 0ull;
+    bool first = true;
+    for (int c0 = 0; c0 < S; c0 += 32) {
+        const int c = c0 + lane;
+        float mc = -INFINITY;
+        double sc = 0.0;
+        uint64_t k0 = 0ull;
+        if (c < S) {
+            mc = __ldcg(&P[c].m);
+            sc = __ldcg(&P[c].s);
+            k0 = ldkey(&P[c].key[0]);
+        }
         if (mc != -INFINITY) ssum += sc * exp2(((double)mc - (double)M) * (double)c2);
+        // round 2: the lists of this group of chunks, loaded together, merged in chunk order
+        unsigned has = __ballot_sync(FULL, k0 != 0ull);
+        while (has) {
+            constexpr int PF = 8;
+            uint64_t kv[PF];
+            int nl = 0;
+            unsigned hh = has;
+#pragma unroll
+            for (int j = 0; j < PF; ++j) {
+                kv[j] = 0ull;
+                if (hh) {
+                    const int cc = c0 + __ffs(hh) - 1;
+                    hh &= hh - 1u;
+                    kv[j] = ldkey(&P[cc].key[lane < K ? lane : 31 - lane]);
+                    ++nl;
+                }
+            }
+            has = hh;
+#pragma unroll
+            for (int j = 0; j < PF; ++j)
+                if (j < nl) {
+                    if (first) {
+                        acc = (lane < K) ? kv[j] : 0ull;
+                        first = false;
+                    } else {
+                        acc = warp_merge_desc(lane < K ? acc : kv[j]);
+                    }
+                }
+        }
     }
     ssum = warp_sum(ssum);
     const double lns = log(ssum);

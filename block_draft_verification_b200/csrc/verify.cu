@@ -104,11 +104,11 @@ __device__ __forceinline__ void greedy_finish(const uint64_t* P, int S, int G, i
                                               int32_t* __restrict__ out_tok) {
     const int lane = threadIdx.x & 31;
     int32_t tj = -1;  // lane j: argmax of target row j (G + 1 <= 32)
-    for (int r0 = 0; r0 <= G; r0 += 4) {
-        uint64_t best[4];
-        rows_max_key<4>(P, S, r0, min(4, G + 1 - r0), best);
+    for (int r0 = 0; r0 <= G; r0 += 8) {
+        uint64_t best[8];
+        rows_max_key<8>(P, S, r0, min(8, G + 1 - r0), best);
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 8; ++j)
             if (lane == r0 + j) tj = (int32_t)key_index(best[j]);
     }
     const int32_t dj = (lane < G) ? draft_tok[(int64_t)b * G + lane] : -1;
@@ -178,12 +178,41 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_kernel(
 // ------------------------------------------------------------------ sampling, pass 1
 // (maximum, fp64 sum of exp2((x - maximum) c)) of rows r0 .. r0+NB-1 from
 // their S chunk partials, warp-collective: lane c takes chunks c, c + 32, ...
-// (the loads of all NB rows issued together), then fixed butterflies.  Every
-// lane returns the same values.
+// then fixed butterflies.  With S <= 64 every partial of the NB rows is
+// loaded in one round (kept in registers); longer rows take two passes.
+// Every lane returns the same values.
 template <int NB>
 __device__ __forceinline__ void rows_lse(const LseD* P, int S, int r0, int nrows, float c2,
                                          float (&Mo)[NB], double (&So)[NB]) {
     const int lane = threadIdx.x & 31;
+    if (S <= 64) {
+        float m[NB][2];
+        double sv[NB][2];
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int c = lane + 32 * h;
+                m[j][h] = -INFINITY;
+                sv[j][h] = 0.0;
+                if (j < nrows && c < S) {
+                    const LseD* p = &P[(int64_t)(r0 + j) * S + c];
+                    m[j][h] = __ldcg(&p->m);
+                    sv[j][h] = __ldcg(&p->s);
+                }
+            }
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+            const float M = warp_max(fmaxf(m[j][0], m[j][1]));
+            double t = 0.0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                if (m[j][h] != -INFINITY) t += sv[j][h] * exp2(((double)m[j][h] - (double)M) * (double)c2);
+            Mo[j] = M;
+            So[j] = warp_sum(t);
+        }
+        return;
+    }
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
         Mo[j] = -INFINITY;
@@ -224,15 +253,22 @@ __device__ __forceinline__ void sample_finish(
             return (double)__uint_as_float((uint32_t)((const uint16_t*)base)[row * V + v] << 16);
         return (double)((const float*)base)[row * V + v];
     };
+    // the drafted tokens and their logits first (independent of the partials)
+    const int32_t dn = (lane < G) ? draft_tok[(int64_t)b * G + lane] : -1;
+    double xt_d = 0.0, xq_d = 0.0;
+    if (lane < G) {
+        xt_d = elem(target, (int64_t)b * (G + 1) + lane, dn);
+        if (q_mode == DFLASH2_Q_SOFTMAX) xq_d = elem(draft, (int64_t)b * G + lane, dn);
+    }
     // lane j: (max, sum-exp) of target row j and draft row j
     LseD lt{-INFINITY, 0.0f, 0.0}, lq{-INFINITY, 0.0f, 0.0};
     const int nrows = (q_mode == DFLASH2_Q_SOFTMAX) ? 2 * G + 1 : G + 1;
-    for (int r0 = 0; r0 < nrows; r0 += 4) {
-        float Mr[4];
-        double Sr[4];
-        rows_lse<4>(P, S, r0, min(4, nrows - r0), c2, Mr, Sr);
+    for (int r0 = 0; r0 < nrows; r0 += 8) {
+        float Mr[8];
+        double Sr[8];
+        rows_lse<8>(P, S, r0, min(8, nrows - r0), c2, Mr, Sr);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 8; ++j) {
             const int rr = r0 + j;
             if (rr <= G && lane == rr) lt = LseD{Mr[j], 0.0f, Sr[j]};
             if (rr > G && rr < nrows && lane == rr - G - 1) lq = LseD{Mr[j], 0.0f, Sr[j]};
@@ -240,12 +276,9 @@ __device__ __forceinline__ void sample_finish(
     }
     bool reject = false;
     if (lane < G) {
-        const int32_t d = draft_tok[(int64_t)b * G + lane];
         // lp = z_t[d] - logZ_t = (x - m) * invT - ln(s); likewise lq
-        double lr = (elem(target, (int64_t)b * (G + 1) + lane, d) - (double)lt.m) * (double)inv_t -
-                    log(lt.s);
-        if (q_mode == DFLASH2_Q_SOFTMAX)
-            lr -= (elem(draft, (int64_t)b * G + lane, d) - (double)lq.m) * (double)inv_t - log(lq.s);
+        double lr = (xt_d - (double)lt.m) * (double)inv_t - log(lt.s);
+        if (q_mode == DFLASH2_Q_SOFTMAX) lr -= (xq_d - (double)lq.m) * (double)inv_t - log(lq.s);
         const double ratio = exp(lr);
         const float u = philox_uniform(seed, step, sid, (uint32_t)lane, 0u);
         reject = !((double)u < ratio);
@@ -254,7 +287,6 @@ __device__ __forceinline__ void sample_finish(
     }
     const unsigned rej = __ballot_sync(FULL, reject);
     const int n = rej ? (__ffs(rej) - 1) : G;
-    const int32_t dn = (lane < G) ? draft_tok[(int64_t)b * G + lane] : -1;
     if (lane <= G) out_tok[(int64_t)b * (G + 1) + lane] = (lane < n) ? dn : -1;  // draw fills n
     const float ltm = __shfl_sync(FULL, lt.m, n);
     const double lts = __shfl_sync(FULL, lt.s, n);
@@ -380,23 +412,25 @@ __device__ __forceinline__ float expm1_pos(float d) {
 // The draw of one sequence covers DLEN elements per CTA of the row it draws
 // from; thread t holds DEPT consecutive elements.  A thread's sum: fp32 over a
 // 16-byte vector (index order, pairwise), fp64 across vectors.
-constexpr int DLEN = 8192;
+constexpr int DLEN = DRAW_LEN;
 constexpr int DT = 256;
-constexpr int DEPT = DLEN / DT;
-// CTAs per row the draw handles (their sums sit in shared memory): V <= 4096 * 8192.
-constexpr int64_t DRAW_MAX_CHUNKS = 4096;
+constexpr int DEPT = DLEN / DT;  // 40: 5 bf16 / 10 fp32 vectors
+// CTAs per row the draw handles (their sums sit in shared memory): V <= 3072 * 10240.
+constexpr int64_t DRAW_MAX_CHUNKS = 3072;
 
-// The draw weight for a mode known at compile time (MODE 0: residual,
-// 1: p without d, 2: p; the residual-empty fallback draws with MODE 2).
-template <int MODE>
-__device__ __forceinline__ float draw_w(float xt, float xq, int64_t v, const SampleInfo& I, float c2,
-                                        float inv_t) {
-    if (MODE == 0) {
+// The draw weight of one element (mode 0: residual, 1: p without d, 2: p;
+// the residual-empty fallback draws with mode 2).  The mode is the same for
+// a whole CTA, so the branch is uniform.
+// off: the element's offset in the thread's run, d_off: the offset of d
+// there (anything outside [0, DEPT) when d is not in the run).
+__device__ __forceinline__ float draw_w(int mode, float xt, float xq, int off, int64_t d_off,
+                                        const SampleInfo& I, float c2, float inv_t) {
+    if (mode == 0) {
         const float dlog = (xt - xq) * inv_t - I.dl;
         if (!(dlog > 0.0f)) return 0.0f;
         return ex2((xq - I.mq) * c2 - I.l2q) * expm1_pos(dlog);
     }
-    if (MODE == 1 && v == I.d) return 0.0f;
+    if (mode == 1 && (int64_t)off == d_off) return 0.0f;
     return ex2((xt - I.mt) * c2 - I.l2t);
 }
 
@@ -411,30 +445,35 @@ __device__ __forceinline__ void draw_load(const char* row, int64_t vb, int64_t V
 #pragma unroll
         for (int g = 0; g < NV; ++g) x[g] = __ldg(p + g);
     } else {
-        const GlobalView<BF16> view{(const uint8_t*)row, vb, (int)max((int64_t)0, min((int64_t)DEPT, V - vb))};
+        const GlobalView<BF16> view{(const uint8_t*)row, vb,
+                                    (int)max((int64_t)0, min((int64_t)DEPT, V - vb))};
 #pragma unroll
         for (int g = 0; g < NV; ++g) x[g] = view.vec(g);
     }
 }
 
-// A thread's weight sum over its DEPT elements.
-template <bool BF16, bool VEC, int MODE>
-__device__ __forceinline__ double draw_thread_sum(const char* trow, const char* qrow, int64_t vb,
-                                                  int64_t V, const SampleInfo& I, float c2,
-                                                  float inv_t) {
+// A thread's weights over its DEPT elements and their sum (fp32 pairwise
+// within a 16-byte vector, fp64 across vectors); w may be null.
+template <bool BF16, bool VEC>
+__device__ __forceinline__ double draw_thread(const char* trow, const char* qrow, int64_t vb,
+                                              int64_t V, int mode, const SampleInfo& I, float c2,
+                                              float inv_t, float* w) {
     using C = ChunkT<BF16>;
     constexpr int NV = DEPT / C::VW;
     uint4 xt[NV], xq[NV];
     draw_load<BF16, VEC>(trow, vb, V, xt);
-    if (MODE == 0) draw_load<BF16, VEC>(qrow, vb, V, xq);
+    if (mode == 0) draw_load<BF16, VEC>(qrow, vb, V, xq);
+    const int64_t d_off = (int64_t)I.d - vb;
     double s = 0.0;
 #pragma unroll
     for (int g = 0; g < NV; ++g) {
         float sv[C::VW];
 #pragma unroll
-        for (int e = 0; e < C::VW; ++e)
-            sv[e] = draw_w<MODE>(C::elem(xt[g], e), MODE == 0 ? C::elem(xq[g], e) : 0.0f,
-                                 vb + g * C::VW + e, I, c2, inv_t);
+        for (int e = 0; e < C::VW; ++e) {
+            sv[e] = draw_w(mode, C::elem(xt[g], e), mode == 0 ? C::elem(xq[g], e) : 0.0f,
+                           g * C::VW + e, d_off, I, c2, inv_t);
+            if (w) w[g * C::VW + e] = sv[e];
+        }
 #pragma unroll
         for (int h = C::VW / 2; h > 0; h >>= 1)
 #pragma unroll
@@ -442,31 +481,6 @@ __device__ __forceinline__ double draw_thread_sum(const char* trow, const char* 
         s += (double)sv[0];
     }
     return s;
-}
-
-// The first element of [vb, vb + DEPT) whose running prefix (from `run`)
-// exceeds t, else the last element with mass, else -1.
-template <bool BF16, bool VEC, int MODE>
-__device__ __forceinline__ int draw_walk(const char* trow, const char* qrow, int64_t vb, int64_t V,
-                                         const SampleInfo& I, float c2, float inv_t, double run,
-                                         double tt) {
-    using C = ChunkT<BF16>;
-    constexpr int NV = DEPT / C::VW;
-    uint4 xt[NV], xq[NV];
-    draw_load<BF16, VEC>(trow, vb, V, xt);
-    if (MODE == 0) draw_load<BF16, VEC>(qrow, vb, V, xq);
-    int pick = -1, lastm = -1;
-#pragma unroll
-    for (int g = 0; g < NV; ++g)
-#pragma unroll
-        for (int e = 0; e < C::VW; ++e) {
-            const float w = draw_w<MODE>(C::elem(xt[g], e), MODE == 0 ? C::elem(xq[g], e) : 0.0f,
-                                         vb + g * C::VW + e, I, c2, inv_t);
-            if (w > 0.0f) lastm = g * C::VW + e;
-            run += (double)w;
-            if (pick < 0 && run > tt) pick = g * C::VW + e;
-        }
-    return pick >= 0 ? pick : lastm;
 }
 
 // Inclusive scan of the threads' values in thread order (fp64): warp scans,
@@ -491,123 +505,169 @@ __device__ __forceinline__ double block_incl_scan(double x, double* s_warp, doub
     return base + incl;
 }
 
-// One mode of the draw (see verify_sample_draw_kernel).  first: every CTA
-// sums its own chunk and only the last of the sequence goes on; else (the
-// fallback to p_n) the calling CTA computes every chunk sum itself.
-template <bool BF16, bool VEC, int MODE>
-__device__ __forceinline__ void draw_body(const char* trow, const char* qrow, int64_t V, int D,
-                                          int c, int b, int G, float c2, float inv_t,
-                                          const SampleInfo& I, double* __restrict__ dsum,
-                                          unsigned* __restrict__ dcount,
-                                          int32_t* __restrict__ out_tok, double* s_sums, bool first) {
-    __shared__ double s_warp[DT / 32];
-    __shared__ double s_incl[DT];
-    __shared__ double s_base, s_t;
-    __shared__ int s_cstar, s_pick, s_last_mass, s_use_p;
-    __shared__ bool s_last;
-    const int t = threadIdx.x;
-    double total;
-    if (first) {  // this CTA's chunk sum; the last CTA of the sequence goes on
-        const double my = draw_thread_sum<BF16, VEC, MODE>(
-            trow, qrow, (int64_t)c * DLEN + (int64_t)DEPT * t, V, I, c2, inv_t);
-        block_incl_scan(my, s_warp, total);
-        if (t == 0) {
-            dsum[(int64_t)b * D + c] = total;
-            s_last = publish(&dcount[b], 1u, (unsigned)D);
-        }
-        __syncthreads();
-        if (!s_last) return;
-        for (int cc = t; cc < D; cc += DT) s_sums[cc] = __ldcg(&dsum[(int64_t)b * D + cc]);
-    } else {  // the chunk sums of p_n (the residual was empty by rounding)
-        for (int cc = 0; cc < D; ++cc) {
-            const double my = draw_thread_sum<BF16, VEC, MODE>(
-                trow, qrow, (int64_t)cc * DLEN + (int64_t)DEPT * t, V, I, c2, inv_t);
-            block_incl_scan(my, s_warp, total);
-            if (t == 0) s_sums[cc] = total;
-        }
-    }
-    __syncthreads();
-    if (t == 0) {
-        double R = 0.0;
-        for (int cc = 0; cc < D; ++cc) R += s_sums[cc];
-        s_use_p = first && MODE != 2 && !(R > 0.0);
-        const double tt = (double)I.u_res * R;
-        double pre = 0.0;
-        int cstar = -1;
-        for (int cc = 0; cc < D; ++cc) {
-            if (pre + s_sums[cc] > tt) {
-                cstar = cc;
-                break;
-            }
-            pre += s_sums[cc];
-        }
-        if (cstar < 0) {  // unreachable while R > 0 (t < R): the last chunk with mass
-            pre = 0.0;
-            cstar = 0;
-            for (int cc = 0; cc < D; ++cc)
-                if (s_sums[cc] > 0.0) cstar = cc;
-            for (int cc = 0; cc < cstar; ++cc) pre += s_sums[cc];
-        }
-        s_cstar = cstar;
-        s_base = pre;
-        s_t = tt;
-        s_pick = DT;
-        s_last_mass = -1;
-    }
-    __syncthreads();
-    if constexpr (MODE != 2) {
-        if (s_use_p) {  // block-uniform
-            draw_body<BF16, VEC, 2>(trow, qrow, V, D, c, b, G, c2, inv_t, I, dsum, dcount,
-                                    out_tok, s_sums, false);
-            return;
-        }
-    }
-    const int cstar = s_cstar;
-    const int64_t vb = (int64_t)cstar * DLEN + (int64_t)DEPT * t;
-    const double my = draw_thread_sum<BF16, VEC, MODE>(trow, qrow, vb, V, I, c2, inv_t);
-    const double incl = block_incl_scan(my, s_warp, total);
-    s_incl[t] = incl;
-    const double tt = s_t, base = s_base;
-    if (base + incl > tt) atomicMin(&s_pick, t);
-    if (my > 0.0) atomicMax(&s_last_mass, t);
-    __syncthreads();
-    int pt = s_pick;
-    if (pt == DT) pt = s_last_mass;  // rounding left t above the chunk's scan
-    if (t == pt) {
-        const int e = draw_walk<BF16, VEC, MODE>(trow, qrow, vb, V, I, c2, inv_t,
-                                                 base + (t > 0 ? s_incl[t - 1] : 0.0), tt);
-        if (e >= 0) out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(vb + e);
-    }
-}
-
-// Grid (chunks of the drawn row, sequences).  Every CTA stores its chunk's
-// weight sum and counts itself in; the last CTA of a sequence takes
-// R = sum of the chunk sums in chunk order and t = u' R, finds the first chunk
-// whose inclusive prefix exceeds t, and scans it: the first thread whose
-// inclusive prefix exceeds t, then the first element of that thread.  If the
-// residual is empty by rounding (R = 0) the last CTA draws from p_n instead,
-// recomputing every chunk sum itself (rare).
+// Draw, part 1: grid (chunks of the drawn row, sequences).  Every thread's
+// inclusive prefix within the chunk is stored (dsum[b][c][t]); the last one
+// is the chunk's sum.
 template <bool BF16, bool VEC>
-__global__ void __launch_bounds__(DT, 4) verify_sample_draw_kernel(
+__global__ void __launch_bounds__(DT) verify_sample_draw_kernel(
     const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int D,
-    float c2, float inv_t, const SampleInfo* __restrict__ info, double* __restrict__ dsum,
-    unsigned* __restrict__ dcount, int32_t* __restrict__ out_tok) {
+    float c2, float inv_t, const SampleInfo* __restrict__ info, double* __restrict__ dsum) {
     constexpr int ES = BF16 ? 2 : 4;
-    extern __shared__ double s_sums[];  // [D], the last CTA's copy of the chunk sums
+    __shared__ double s_warp[DT / 32];
     const int c = blockIdx.x, b = blockIdx.y;
     pdl_wait();  // the scan's SampleInfo, and every earlier write, are visible
+    pdl_launch_dependents();
     const SampleInfo I = info[b];
     const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
     const char* qrow = (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
-    if (I.mode == 0)
-        draw_body<BF16, VEC, 0>(trow, qrow, V, D, c, b, G, c2, inv_t, I, dsum, dcount, out_tok,
-                                s_sums, true);
-    else if (I.mode == 1)
-        draw_body<BF16, VEC, 1>(trow, qrow, V, D, c, b, G, c2, inv_t, I, dsum, dcount, out_tok,
-                                s_sums, true);
-    else
-        draw_body<BF16, VEC, 2>(trow, qrow, V, D, c, b, G, c2, inv_t, I, dsum, dcount, out_tok,
-                                s_sums, true);
+    const double my = draw_thread<BF16, VEC>(trow, qrow, (int64_t)c * DLEN + (int64_t)DEPT * threadIdx.x,
+                                             V, I.mode, I, c2, inv_t, nullptr);
+    double total;
+    const double incl = block_incl_scan(my, s_warp, total);
+    dsum[((int64_t)b * D + c) * DT + threadIdx.x] = incl;
+}
+
+// Draw, part 2: one warp per sequence.  R = the chunk sums in chunk order,
+// t = u' R; in the first chunk whose inclusive prefix exceeds t, the first
+// thread of part 1 whose inclusive prefix exceeds t (from the stored
+// prefixes) recomputes its weights and walks them to the first element whose
+// running prefix exceeds t (else, rounding, the last element with mass).  If
+// the residual is empty by rounding (R = 0) the draw is redone from p_n by
+// this warp (rare, slow).
+template <bool BF16, bool VEC>
+__global__ void __launch_bounds__(32) verify_sample_pick_kernel(
+    const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int D,
+    float c2, float inv_t, const SampleInfo* __restrict__ info, const double* __restrict__ dsum,
+    int32_t* __restrict__ out_tok) {
+    constexpr int ES = BF16 ? 2 : 4;
+    const int lane = threadIdx.x, b = blockIdx.x;
+    pdl_wait();  // part 1's prefixes
+    const SampleInfo I = info[b];
+    const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
+    const char* qrow = (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
+    const double* P = dsum + (int64_t)b * D * DT;
+    // The chunk sums, loaded together, in an inclusive warp scan (fixed
+    // order; R is its last value); carried across groups of 32 chunks.
+    double carry = 0.0, tt = 0.0, pre = 0.0;
+    int cstar = -1, lastc = -1;
+    double lastc_pre = 0.0;
+    int mode = I.mode;
+    {
+        double R = 0.0;
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            const int cc = c0 + lane;
+            const double cs = (cc < D) ? __ldcg(&P[(int64_t)cc * DT + DT - 1]) : 0.0;
+            double incl = cs;
+#pragma unroll
+            for (int k = 1; k < 32; k <<= 1) {
+                const double o = __shfl_up_sync(FULL, incl, k);
+                if (lane >= k) incl += o;
+            }
+            incl += carry;
+            carry = __shfl_sync(FULL, incl, 31);
+        }
+        R = carry;
+        if (!(R > 0.0)) mode = 2;  // residual empty by rounding: draw from p_n (rare)
+        tt = (double)I.u_res * R;
+        carry = 0.0;
+        for (int c0 = 0; c0 < D && cstar < 0; c0 += 32) {  // the same scan again, now against t
+            const int cc = c0 + lane;
+            const double cs = (cc < D) ? __ldcg(&P[(int64_t)cc * DT + DT - 1]) : 0.0;
+            double incl = cs;
+#pragma unroll
+            for (int k = 1; k < 32; k <<= 1) {
+                const double o = __shfl_up_sync(FULL, incl, k);
+                if (lane >= k) incl += o;
+            }
+            incl += carry;
+            const unsigned cross = __ballot_sync(FULL, cc < D && incl > tt);
+            const unsigned mass = __ballot_sync(FULL, cc < D && cs > 0.0);
+            if (mass) {
+                const int l = 31 - __clz(mass);
+                lastc = c0 + l;
+                lastc_pre = __shfl_sync(FULL, incl - cs, l);
+            }
+            if (cross) {
+                const int l = __ffs(cross) - 1;
+                cstar = c0 + l;
+                pre = __shfl_sync(FULL, incl - cs, l);
+            }
+            carry = __shfl_sync(FULL, incl, 31);
+        }
+        if (cstar < 0) {  // unreachable while R > 0: the last chunk with mass
+            cstar = max(lastc, 0);
+            pre = lastc >= 0 ? lastc_pre : 0.0;
+        }
+    }
+    int pick = -1;
+    int64_t vb = 0;
+    if (mode == I.mode) {
+        // the first thread of chunk cstar whose inclusive prefix exceeds t;
+        // all 256 prefixes loaded in one round
+        const double* Q = P + (int64_t)cstar * DT;
+        double incl[DT / 32], prev[DT / 32];
+#pragma unroll
+        for (int j = 0; j < DT / 32; ++j) {
+            const int t = 32 * j + lane;
+            incl[j] = __ldcg(&Q[t]);
+            prev[j] = (t > 0) ? __ldcg(&Q[t - 1]) : 0.0;
+        }
+        int pt = DT, lastm = -1;
+#pragma unroll
+        for (int j = DT / 32 - 1; j >= 0; --j) {
+            const unsigned cross = __ballot_sync(FULL, pre + incl[j] > tt);
+            const unsigned mass = __ballot_sync(FULL, incl[j] > prev[j]);
+            if (cross) pt = 32 * j + __ffs(cross) - 1;
+            if (mass && lastm < 0) lastm = 32 * j + 31 - __clz(mass);
+        }
+        if (pt == DT) pt = lastm;  // rounding left t above the chunk's scan
+        if (pt >= 0) {
+            vb = (int64_t)cstar * DLEN + (int64_t)DEPT * pt;
+            const double base = pre + (pt > 0 ? __ldcg(&Q[pt - 1]) : 0.0);
+            if (lane == 0) {
+                float w[DEPT];
+                draw_thread<BF16, VEC>(trow, qrow, vb, V, mode, I, c2, inv_t, w);
+                double run = base;
+                int lm = -1;
+                for (int e = 0; e < DEPT; ++e) {
+                    if (w[e] > 0.0f) lm = e;
+                    run += (double)w[e];
+                    if (pick < 0 && run > tt) pick = e;
+                }
+                if (pick < 0) pick = lm;
+            }
+        }
+    } else if (lane == 0) {
+        // fallback: R and the walk over the whole row from p_n in thread order
+        double R = 0.0;
+        for (int cc = 0; cc < D; ++cc)
+            for (int t = 0; t < DT; ++t)
+                R += draw_thread<BF16, VEC>(trow, qrow, (int64_t)cc * DLEN + (int64_t)DEPT * t, V,
+                                            mode, I, c2, inv_t, nullptr);
+        tt = (double)I.u_res * R;
+        double run = 0.0;
+        int lm = -1;
+        for (int cc = 0; cc < D && pick < 0; ++cc)
+            for (int t = 0; t < DT && pick < 0; ++t) {
+                float w[DEPT];
+                const int64_t v0 = (int64_t)cc * DLEN + (int64_t)DEPT * t;
+                draw_thread<BF16, VEC>(trow, qrow, v0, V, mode, I, c2, inv_t, w);
+                for (int e = 0; e < DEPT; ++e) {
+                    if (w[e] > 0.0f) lm = (int)(v0 + e);
+                    run += (double)w[e];
+                    if (run > tt) {
+                        pick = e;
+                        vb = v0;
+                        break;
+                    }
+                }
+            }
+        if (pick < 0 && lm >= 0) {
+            pick = 0;
+            vb = lm;
+        }
+    }
+    if (lane == 0 && pick >= 0) out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(vb + pick);
 }
 
 }  // namespace dfl
@@ -715,15 +775,14 @@ extern "C" int dflash2_verify_sample(const void* target, const void* draft, int 
     const Layout L = sample_layout(B, G, V, es);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return DFLASH2_EWORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
-    unsigned* counters = (unsigned*)((char*)ws + L.counters_off);  // [B] scan, [B] draw
+    unsigned* counters = (unsigned*)((char*)ws + L.counters_off);  // [B] scan
     LseD* part = (LseD*)((char*)ws + L.part_off);
     double* dsum = (double*)((char*)ws + L.part2_off);
     SampleInfo* info = (SampleInfo*)((char*)ws + L.info_off);
-    if (cudaMemsetAsync(counters, 0, (size_t)B * 8, s) != cudaSuccess) return DFLASH2_ECUDA;
+    if (cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
     const void* q = (q_mode == DFLASH2_Q_SOFTMAX) ? draft : nullptr;
     const bool tma = aligned(target, 16) && (!q || aligned(q, 16)) && (V * es) % 16 == 0;
     const float c2 = (float)((double)inv_temperature * LOG2E);
-    const size_t dyn2 = (size_t)D * sizeof(double);
 #define DFL_SAMPLE(BF, TM)                                                                        \
     do {                                                                                          \
         auto kern = verify_sample_scan_kernel<BF, TM>;                                            \
@@ -733,11 +792,14 @@ extern "C" int dflash2_verify_sample(const void* target, const void* draft, int 
             target, q, G, V, (int)S, rows_per_seq, units, inv_temperature, c2, draft_tok, seed,   \
             step, seq_id, q_mode, n_accept, out_tok, ratio_dbg, u_dbg, part, info, counters);     \
         auto kern2 = verify_sample_draw_kernel<BF, TM>;                                           \
-        if (ring_prepare(kern2, (size_t)DRAW_MAX_CHUNKS * sizeof(double)) != DFLASH2_OK)          \
+        if (launch_dependent(kern2, dim3((unsigned)D, (unsigned)B), dim3(DT), 0, s, target, q, G, \
+                             V, (int)D, c2, inv_temperature, (const SampleInfo*)info, dsum) !=    \
+            cudaSuccess)                                                                          \
             return DFLASH2_ECUDA;                                                                 \
-        if (launch_dependent(kern2, dim3((unsigned)D, (unsigned)B), dim3(DT), dyn2, s, target, q, \
-                             G, V, (int)D, c2, inv_temperature, (const SampleInfo*)info, dsum,    \
-                             counters + B, out_tok) != cudaSuccess)                               \
+        auto kern3 = verify_sample_pick_kernel<BF, TM>;                                           \
+        if (launch_dependent(kern3, dim3((unsigned)B), dim3(32), 0, s, target, q, G, V, (int)D,    \
+                             c2, inv_temperature, (const SampleInfo*)info, (const double*)dsum,   \
+                             out_tok) != cudaSuccess)                                             \
             return DFLASH2_ECUDA;                                                                 \
     } while (0)
     if (dtype == DFLASH2_BF16) {

@@ -36,6 +36,10 @@ struct SampleInfo {
     int32_t pad;
 };
 
+// Elements of the drawn row per CTA of the sampling draw (40 per thread of
+// 256): its chunk sums sit in the sampling workspace.
+constexpr int DRAW_LEN = 10240;
+
 struct Layout {
     size_t counters_off, counters_bytes;
     size_t part_off, part_bytes;
@@ -70,14 +74,14 @@ inline Layout greedy_layout(int B, int G, int64_t V, int es) {
     const int64_t S = row_chunks(V, es);
     return make_layout((size_t)B * 4, (size_t)((int64_t)B * (G + 1) * S) * sizeof(uint64_t));
 }
-// Sampling: counters of the scan and of the draw ([B] each), the scan's
-// per-unit partials, the draw's per-chunk weight sums (8192 elements per
-// chunk) and the per-sequence hand-over to the draw.
+// Sampling: the scan's counters ([B]), its
+// per-unit partials, the draw's per-thread prefix sums (256 threads of
+// DRAW_LEN / 256 elements per chunk) and the per-sequence hand-over to the draw.
 inline Layout sample_layout(int B, int G, int64_t V, int es) {
     const int64_t S = row_chunks(V, es);
-    const int64_t D = (V + 8191) / 8192;
-    return make_layout((size_t)B * 8, (size_t)((int64_t)B * (2 * G + 1) * S) * sizeof(LseD),
-                       (size_t)(B * D) * sizeof(double), (size_t)B * sizeof(SampleInfo));
+    const int64_t D = (V + DRAW_LEN - 1) / DRAW_LEN;
+    return make_layout((size_t)B * 4, (size_t)((int64_t)B * (2 * G + 1) * S) * sizeof(LseD),
+                       (size_t)(B * D) * 256 * sizeof(double), (size_t)B * sizeof(SampleInfo));
 }
 inline Layout select_layout(int B, int G) {
     return make_layout((size_t)B * 4, (size_t)B * (K + (size_t)K * K * (G - 1)) * sizeof(float));
