@@ -124,7 +124,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 constexpr int TC_MAXCTA = 256;  // stream-K CTAs at most (one per SM)
 
 struct TcShape {
-    int H, T, ntok, BN, stages, nkb, nh;  // nh: channel tiles per token chunk
+    int H, T, ntok, BN, sw, sx, nkb, nh;  // W / X ring stages; nh: channel tiles per token chunk
     int bufcols;                           // TMEM columns per accumulator (power of 2, >= BN)
     int ngroups;                           // 32-column groups per accumulator
     int nctas;                             // stream-K CTAs
@@ -170,35 +170,42 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     __nv_bfloat16* __restrict__ out, TcShape sh, float4* __restrict__ partial,
     unsigned* __restrict__ flags) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // stage ring, 1024-byte aligned for the 128-byte swizzle
-    uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const int stage_bytes = TC_A_BYTES + sh.BN * TC_BK * 2;
-    uint8_t* tail = base + sh.stages * stage_bytes;
+    // two rings, 1024-byte aligned for the 128-byte swizzle: W tiles (HBM,
+    // deeper) and X tiles (L2), each with its own full / empty barriers
+    uint8_t* wring = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int xstage = sh.BN * TC_BK * 2;
+    uint8_t* xring = wring + sh.sw * TC_A_BYTES;
+    uint8_t* tail = xring + sh.sx * xstage;
     // an owned tile's inputs, row-major 128-byte rows (64 channels):
     // x of its BN tokens, x_prev of the R batches it touches, x of token tok0-1
     uint8_t* s_x = tail;
     uint8_t* s_xp = s_x + sh.BN * 128;
     uint8_t* s_x0 = s_xp + sh.R * 128;
     uint8_t* s_out = s_x0 + 128;  // [2][32 tokens][64 channels] bf16 outputs
-    // full[S], empty[S], tmem_full[2], tmem_empty[2], mma_done, x tile
+    // wfull[SW], wempty[SW], xfull[SX], xempty[SX], tmem_full[2], tmem_empty[2], mma_done, x tile
     uint64_t* bars = (uint64_t*)(s_out + 8192);
-    uint32_t* s_tmem = (uint32_t*)(bars + 2 * sh.stages + 6);
+    uint32_t* s_tmem = (uint32_t*)(bars + 2 * sh.sw + 2 * sh.sx + 6);
     int* s_fail = (int*)(s_tmem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int p = blockIdx.x;
     const int64_t s0 = run_start(sh, p), s1 = run_start(sh, p + 1);
-    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + sh.stages);
-    const uint32_t tfull0 = smem_u32(bars + 2 * sh.stages);
+    const uint32_t wfull0 = smem_u32(bars), wempty0 = wfull0 + 8 * sh.sw;
+    const uint32_t xfull0 = wempty0 + 8 * sh.sw, xempty0 = xfull0 + 8 * sh.sx;
+    const uint32_t tfull0 = xempty0 + 8 * sh.sx;
     const uint32_t tempty0 = tfull0 + 16;
     const uint32_t mdone = tfull0 + 32;
     const uint32_t xbar = tfull0 + 40;
     const uint32_t ncols = 2 * (uint32_t)sh.bufcols;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < sh.stages; ++i) {
-            mbar_init(full0 + 8 * i, 1);
-            mbar_init(empty0 + 8 * i, 1);
+        for (int i = 0; i < sh.sw; ++i) {
+            mbar_init(wfull0 + 8 * i, 1);
+            mbar_init(wempty0 + 8 * i, 1);
+        }
+        for (int i = 0; i < sh.sx; ++i) {
+            mbar_init(xfull0 + 8 * i, 1);
+            mbar_init(xempty0 + 8 * i, 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(tfull0 + 8 * i, 1);
@@ -220,13 +227,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    if (warp == 0 && lane == 0) {
-        // ---------------- TMA producer: the run's steps in order
-        const uint32_t tx = TC_A_BYTES + sh.BN * TC_BK * 2;
+    if ((warp == 0 || warp == 3) && lane == 0) {
+        // ---------------- TMA producers, the run's steps in order: warp 0
+        // the W tiles (HBM), warp 3 the X tiles (L2), each on its own ring
+        const bool is_w = warp == 0;
+        const int S = is_w ? sh.sw : sh.sx;
+        const uint32_t full0 = is_w ? wfull0 : xfull0, empty0 = is_w ? wempty0 : xempty0;
+        const uint32_t tx = is_w ? (uint32_t)TC_A_BYTES : (uint32_t)xstage;
         int i = 0;
         const int n = (int)(s1 - s0);
         for (; i < n; ++i) {
-            const int st = i % sh.stages, r = i / sh.stages;
+            const int st = i % S, r = i / S;
             if (r > 0 && !mbar_wait(empty0 + 8 * st, (r - 1) & 1)) {
                 atomicOr(&g_dev_err, ERR_PRODUCER);
                 break;
@@ -234,20 +245,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
             const int64_t step = s0 + i;
             const int tile = (int)(step / sh.nkb), kb = (int)(step - (int64_t)tile * sh.nkb);
             const int ct = tile / sh.nh, hb = tile - ct * sh.nh;
-            const int h0 = hb * TC_CH, tok0 = ct * TC_MAXN;
-            const uint32_t a = smem_u32(base + st * stage_bytes);
-            const uint32_t b = a + TC_A_BYTES;
             mbar_expect_tx(full0 + 8 * st, tx);
-            // one box of the 4-D view (k, 16 channels, a|b, 16-channel block):
-            // accumulator rows 32q .. 32q+15 are a of channels h0+16q ..
-            // h0+16q+15, rows 32q+16 .. 32q+31 are b of the same channels
-            tma_load_4d(a, &map_w, kb * TC_BK, 0, 0, h0 / 16, full0 + 8 * st);
-            tma_load_2d(b, &map_x, kb * TC_BK, tok0, full0 + 8 * st);
+            if (is_w) {
+                // one box of the 4-D view (k, 16 channels, a|b, 16-channel block):
+                // accumulator rows 32q .. 32q+15 are a of channels h0+16q ..
+                // h0+16q+15, rows 32q+16 .. 32q+31 are b of the same channels
+                tma_load_4d(smem_u32(wring + st * TC_A_BYTES), &map_w, kb * TC_BK, 0, 0,
+                            hb * TC_CH / 16, full0 + 8 * st);
+            } else {
+                tma_load_2d(smem_u32(xring + st * xstage), &map_x, kb * TC_BK, ct * TC_MAXN,
+                            full0 + 8 * st);
+            }
         }
         // drain: the last loads in flight have landed once their stages are
         // consumed (bounded; only a failed MMA thread leaves them pending)
-        for (int k = (i > sh.stages ? i - sh.stages : 0); k < i; ++k) {
-            const int st = k % sh.stages, r = k / sh.stages;
+        for (int k = (i > S ? i - S : 0); k < i; ++k) {
+            const int st = k % S, r = k / S;
             if (!mbar_wait(empty0 + 8 * st, r & 1)) {
                 atomicOr(&g_dev_err, ERR_DRAIN);
                 break;
@@ -270,20 +283,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
             tc_fence_after();
             const uint32_t d = tmem + (uint32_t)(buf * sh.bufcols);
             for (int kb = klo; kb < khi; ++kb, ++i) {
-                const int st = i % sh.stages, r = i / sh.stages;
-                if (!mbar_wait(full0 + 8 * st, r & 1)) {
+                const int sw = i % sh.sw, sx = i % sh.sx;
+                if (!mbar_wait(wfull0 + 8 * sw, (i / sh.sw) & 1) ||
+                    !mbar_wait(xfull0 + 8 * sx, (i / sh.sx) & 1)) {
                     atomicOr(&g_dev_err, ERR_MMA);
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a = smem_u32(base + st * stage_bytes);
-                const uint32_t b = a + TC_A_BYTES;
+                const uint32_t a = smem_u32(wring + sw * TC_A_BYTES);
+                const uint32_t b = smem_u32(xring + sx * xstage);
 #pragma unroll
                 for (int kk = 0; kk < TC_BK / 16; ++kk)
                     mma_bf16(d, smem_desc(a + kk * 32), smem_desc(b + kk * 32), idesc,
                              (kb > klo || kk > 0) ? 1u : 0u);
-                mma_commit(empty0 + 8 * st);
+                mma_commit(wempty0 + 8 * sw);
+                mma_commit(xempty0 + 8 * sx);
             }
             if (ok) mma_commit(tfull0 + 8 * buf);
             sg = (int64_t)tile * sh.nkb + khi;
@@ -582,12 +597,15 @@ int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_
     if (!make_map(&mxe, x, (uint64_t)H, (uint64_t)ntok, TC_CH, (uint32_t)P.BN, false) ||
         !make_map(&mpe, x_prev, (uint64_t)H, (uint64_t)B, TC_CH, (uint32_t)R, false))
         return DFLASH2_ECUDA;
-    const int stage_bytes = TC_A_BYTES + P.BN * TC_BK * 2;
-    const int fixed = 1024 + (P.BN + R + 1) * 128 + 8192 + 64 * 8 + 16;
-    int stages = (227 * 1024 - fixed) / stage_bytes;
-    stages = stages > 8 ? 8 : stages;
-    if (stages < 2) return DFLASH2_ESHAPE;
-    const int smem = fixed + stages * stage_bytes;
+    // W ring (HBM, ~2 us loaded latency) deeper than the X ring (L2): three X
+    // stages (four when they are small), the rest of 227 KB for W, at most 8
+    const int xstage = P.BN * TC_BK * 2;
+    const int fixed = 1024 + (P.BN + R + 1) * 128 + 8192 + 96 * 8 + 16;
+    const int sx = xstage <= 16384 ? 4 : 3;
+    int sw = (227 * 1024 - fixed - sx * xstage) / TC_A_BYTES;
+    sw = sw > 8 ? 8 : sw;
+    if (sw < 2) return DFLASH2_ESHAPE;
+    const int smem = fixed + sw * TC_A_BYTES + sx * xstage;
     {
         static std::mutex mu;
         static bool attr_set[64] = {};
@@ -602,7 +620,7 @@ int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_
     unsigned* flags = (unsigned*)ws;
     float4* part = (float4*)((char*)ws + P.flags_bytes);
     if (cudaMemsetAsync(flags, 0, (size_t)P.nctas * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
-    TcShape sh{H, T, ntok, P.BN, stages, P.nkb, P.nh, P.bufcols, P.ngroups, P.nctas, R, P.steps};
+    TcShape sh{H, T, ntok, P.BN, sw, sx, P.nkb, P.nh, P.bufcols, P.ngroups, P.nctas, R, P.steps};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)P.nctas);
     cfg.blockDim = dim3(TC_THREADS);

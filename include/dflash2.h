@@ -132,9 +132,10 @@ DFLASH2_API int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows
  * library until the process exits.  The call allocates nothing (no
  * cudaMalloc, no cudaFree, no allocating library routine); it clears the part
  * of the array it uses with cudaMemsetAsync on `stream`.
- *   - Limit: rows * ceil(V / 16384) * 144 + rows * 4 bytes (each rounded up
+ *   - Limit: rows * ceil(V / L) * 144 + rows * 4 bytes (L = 4096 for bf16,
+ *     2048 for fp32: the rows are reduced in chunks of 8 KB; each term rounded up
  *     to 256) must fit in the array; larger shapes return DFLASH2_EWORKSPACE
- *     and enqueue nothing.  At V = 151,936 that is up to 2,900 rows.
+ *     and enqueue nothing.  At V = 151,936 in bf16 that is up to 765 rows.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind: two calls that can overlap on the GPU (different streams without
  *     an ordering between them) race and give wrong results.
@@ -210,7 +211,7 @@ DFLASH2_API int dflash2_verify_greedy(const void* target, int dtype, int B, int 
  * for u_j, 1 for u' (position = n).
  *
  * target [B, G+1, V], draft [B, G, V] of `dtype`, rows 16-byte aligned for
- * the fast path; V <= 67,108,864 (4096 chunks of 16384; DFLASH2_ESHAPE
+ * the fast path; V <= 31,457,280 (3072 draw chunks of 10240; DFLASH2_ESHAPE
  * above); draft_tok [B, G] int32; seq_id [B] uint32 or NULL (= b).
  * n_accept [B], out_tok [B, G+1] as in dflash2_verify_greedy.
  * ratio_dbg [B, G] float r_j for every j, u_dbg [B, G] float u_j; both
