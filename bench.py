@@ -9,9 +9,10 @@ embeddings 151,936 x 128 bf16 and W 128 x 128 fp32, dynconv hidden 5,120 over
 32 x 8 tokens; seeded synthetic inputs of that shape (synth "b32").
 
 One step = the whole path over one batch, each call through the C ABI:
-  dflash2_topk_softmax (224 draft rows) -> dflash2_pair_select ->
-  dflash2_verify_sample (Philox, softmax q) -> dflash2_verify_greedy ->
-  dflash2_dynconv2.
+  dflash2_topk_softmax_ex (224 draft rows, with their normalisers) ->
+  dflash2_pair_select -> dflash2_verify_sample_ex (Philox, softmax q from the
+  drafter normalisers: the fused cycle, draft rows not streamed again) ->
+  dflash2_verify_greedy -> dflash2_dynconv2.
 value = steps per second over all ranks (each rank runs its own batch:
 weak scaling, no collective on the data path).  L2 (126 MB) is flushed by a
 256 MB write followed by a read of the same buffer (no dirty lines left)
@@ -69,9 +70,11 @@ def algorithmic_bytes(w, B):
     """Bytes each call must move at least once (inputs read once, outputs written once)."""
     G, V, d, H, T = w.G, w.V, w.d, w.H, w.T
     return {
-        "topk_softmax": 2 * B * G * V + B * G * (16 * 12 + 4),
+        "topk_softmax": 2 * B * G * V + B * G * (16 * 12 + 12),
         "pair_select": 2 * B * (1 + 16 * G) * d + 4 * d * d + B * G * (16 * 8) + B * G * 8 + B * 4,
-        "verify_sample": 2 * B * (2 * G + 1) * V + B * G * 4 + B * (G + 2) * 4,
+        # fused cycle: the target rows once, and the one draft row a residual
+        # draw reads per sequence (drafter normalisers come from topk)
+        "verify_sample": 2 * B * (G + 1) * V + 2 * B * V + B * G * 12 + B * (G + 2) * 4,
         "verify_greedy": 2 * B * (G + 1) * V + B * G * 4 + B * (G + 2) * 4,
         "dynconv2": 2 * (2 * H * H) + 2 * 2 * B * T * H + 2 * B * H,
     }
@@ -226,11 +229,17 @@ def run_ours(args, rank, world, local_rank):
         inputs.append(dict(T=dev_t(b.target), Q=dev_t(b.draft), anchor=dev_t(b.anchor),
                            sid=dev_t(b.seq_id.view(np.int32)), x=dev_t(c.x), xp=dev_t(c.x_prev)))
     ws = dfl.Workspace(dev, dfl.workspace_bytes(B, G, V) + dfl.workspace_bytes(B * G, 1, V))
+    def topk_out():
+        return (torch.empty((B * G, 16), dtype=torch.int32, device=dev),
+                torch.empty((B * G, 16), dtype=torch.float32, device=dev),
+                torch.empty((B * G, 16), dtype=torch.float32, device=dev),
+                torch.empty((B * G,), dtype=torch.float32, device=dev),
+                torch.empty((B * G,), dtype=torch.float32, device=dev),
+                torch.empty((B * G,), dtype=torch.float32, device=dev))
+
+    for k, inp in enumerate(inputs):
+        inp["topk"] = topk_out()  # per input set: the normalisers stay with their rows
     outs = dict(
-        topk=(torch.empty((B * G, 16), dtype=torch.int32, device=dev),
-              torch.empty((B * G, 16), dtype=torch.float32, device=dev),
-              torch.empty((B * G, 16), dtype=torch.float32, device=dev),
-              torch.empty((B * G,), dtype=torch.float32, device=dev)),
         sel=(torch.empty((B, G), dtype=torch.int32, device=dev),
              torch.empty((B, G), dtype=torch.int32, device=dev),
              torch.empty((B,), dtype=torch.float32, device=dev)),
@@ -243,17 +252,19 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_sink = torch.zeros((), dtype=torch.int64, device=dev)
     names = ["topk_softmax", "pair_select", "verify_sample", "verify_greedy", "dynconv2"]
-    kernels_per_step = {"topk_softmax": 1, "pair_select": 1, "verify_sample": 2,
+    kernels_per_step = {"topk_softmax": 1, "pair_select": 1, "verify_sample": 3,
                         "verify_greedy": 1, "dynconv2": 1}
 
     def calls(inp, step):
-        tk = outs["topk"]
+        tk = inp["topk"]
         return [
-            lambda: dfl.topk_softmax(inp["Q"].view(B * G, V), w.inv_temperature, out=tk, ws=ws),
+            lambda: dfl.topk_softmax(inp["Q"].view(B * G, V), w.inv_temperature, out=tk, ws=ws,
+                                     stats=True),
             lambda: dfl.pair_select(tk[0].view(B, G, 16), tk[2].view(B, G, 16), inp["anchor"], E,
                                     Wsel, out=outs["sel"], ws=ws),
             lambda: dfl.verify_sample(inp["T"], inp["Q"], outs["sel"][0], w.seed, step, inp["sid"],
-                                      w.inv_temperature, out=outs["samp"], ws=ws),
+                                      w.inv_temperature, out=outs["samp"], ws=ws,
+                                      draft_stats=(tk[4].view(B, G), tk[5].view(B, G))),
             lambda: dfl.verify_greedy(inp["T"], outs["sel"][0], out=outs["greedy"], ws=ws),
             lambda: dfl.dynconv2(inp["x"], inp["xp"], Wtap, out=outs["conv"]),
         ]
@@ -399,8 +410,9 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": "concurrency-32: B=32, block 8 (7 drafted + 1 bonus), V=151936, "
                                "bf16 logits, selector d=128 (emb 151936x128 bf16, W fp32), "
-                               "sampling at T=1.0 and greedy verify, dynconv H=5120 over 32x8 "
-                               "tokens; one step = all five calls",
+                               "sampling at T=1.0 (fused cycle: drafter normalisers from topk) "
+                               "and greedy verify, dynconv H=5120 over 32x8 tokens; one step = "
+                               "all five calls",
                    "global_batch": B * world, "parallelism": "dp%d (independent batches)" % world,
                    "l2": "256 MB write + read flush before every call, outside the timed intervals",
                    "step_hbm_GBps": round(step_gbs, 1),

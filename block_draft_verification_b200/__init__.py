@@ -45,18 +45,23 @@ def lib():
         L.dflash2_workspace_bytes.argtypes = [i32, i32, i64]
         L.dflash2_workspace_bytes.restype = sz
         L.dflash2_topk_softmax.argtypes = [vp, i32, i64, i64, i64, f32, vp, vp, vp, vp, vp, sz, vp]
+        L.dflash2_topk_softmax_ex.argtypes = [vp, i32, i64, i64, i64, f32, vp, vp, vp, vp, vp, vp,
+                                              vp, sz, vp]
         L.dflash2_pair_select.argtypes = [vp, vp, vp, vp, i32, i64, i32, vp, i32, i32, vp, vp, vp,
                                           vp, sz, vp]
         L.dflash2_verify_greedy.argtypes = [vp, i32, i32, i32, i64, vp, vp, vp, vp, sz, vp]
         L.dflash2_verify_sample.argtypes = [vp, vp, i32, i32, i32, i64, vp, f32, u64, u32, vp, i32,
                                             vp, vp, vp, vp, vp, sz, vp]
+        L.dflash2_verify_sample_ex.argtypes = [vp, vp, i32, i32, i32, i64, vp, vp, vp, f32, u64,
+                                               u32, vp, i32, vp, vp, vp, vp, vp, sz, vp]
         L.dflash2_dynconv2.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]
         L.dflash2_dynconv2_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.dflash2_dynconv2_workspace_bytes.restype = sz
         L.dflash2_device_errors.argtypes = [i32]
         L.dflash2_device_errors.restype = C.c_uint32
-        for f in ("dflash2_topk_softmax", "dflash2_pair_select", "dflash2_verify_greedy",
-                  "dflash2_verify_sample", "dflash2_dynconv2"):
+        for f in ("dflash2_topk_softmax", "dflash2_topk_softmax_ex", "dflash2_pair_select",
+                  "dflash2_verify_greedy", "dflash2_verify_sample", "dflash2_verify_sample_ex",
+                  "dflash2_dynconv2"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -140,9 +145,11 @@ def _ws(ws, dev, B, G, V):
     return ws.args(B, G, V)
 
 
-def topk_softmax(logits, inv_temperature=1.0, out=None, ws=None):
+def topk_softmax(logits, inv_temperature=1.0, out=None, ws=None, stats=False):
     """logits [..., V] (rows may be strided) -> idx [..., 16] int32, prob, logp
-    [..., 16] float32, logz [...] float32."""
+    [..., 16] float32, logz [...] float32; with stats=True also row_max and
+    row_lse [...] float32 (dflash2_topk_softmax_ex), the normalisers
+    verify_sample(draft_stats=...) reuses."""
     _cuda(logits)
     V = logits.shape[-1]
     x = logits.reshape(-1, V) if logits.dim() != 2 else logits
@@ -156,12 +163,23 @@ def topk_softmax(logits, inv_temperature=1.0, out=None, ws=None):
                torch.empty(lead + (K,), dtype=torch.float32, device=dev),
                torch.empty(lead + (K,), dtype=torch.float32, device=dev),
                torch.empty(lead, dtype=torch.float32, device=dev))
-    idx, prob, logp, logz = out
+    if stats and len(out) == 4:
+        out = tuple(out) + (torch.empty(lead, dtype=torch.float32, device=dev),
+                            torch.empty(lead, dtype=torch.float32, device=dev))
+    idx, prob, logp, logz = out[:4]
+    rmax = out[4] if len(out) > 4 else None
+    rlse = out[5] if len(out) > 5 else None
     wp, wb = _ws(ws, dev, rows, 1, V)
-    _check("dflash2_topk_softmax", lib().dflash2_topk_softmax(
-        _p(x), _dtype(x), rows, V, x.stride(0) if rows > 1 else V, float(inv_temperature),
-        _p(idx), _p(prob), _p(logp), _p(logz), wp, wb, _stream(dev)))
-    return idx, prob, logp, logz
+    stride = x.stride(0) if rows > 1 else V
+    if rmax is None and rlse is None:
+        _check("dflash2_topk_softmax", lib().dflash2_topk_softmax(
+            _p(x), _dtype(x), rows, V, stride, float(inv_temperature), _p(idx), _p(prob),
+            _p(logp), _p(logz), wp, wb, _stream(dev)))
+    else:
+        _check("dflash2_topk_softmax_ex", lib().dflash2_topk_softmax_ex(
+            _p(x), _dtype(x), rows, V, stride, float(inv_temperature), _p(idx), _p(prob),
+            _p(logp), _p(logz), _p(rmax), _p(rlse), wp, wb, _stream(dev)))
+    return tuple(out)
 
 
 def pair_select(idx, logp, anchor, emb, W, out=None, ws=None):
@@ -200,9 +218,12 @@ def verify_greedy(target, draft_tok, out=None, ws=None):
 
 
 def verify_sample(target, draft, draft_tok, seed, step, seq_id=None, inv_temperature=1.0,
-                  q_mode=Q_SOFTMAX, debug=False, out=None, ws=None):
+                  q_mode=Q_SOFTMAX, debug=False, out=None, ws=None, draft_stats=None):
     """target [B, G+1, V], draft [B, G, V] (None in one-hot mode), draft_tok [B, G]
-    -> n_accept [B], out_tok [B, G+1] (+ ratio [B, G], u [B, G] if debug)."""
+    -> n_accept [B], out_tok [B, G+1] (+ ratio [B, G], u [B, G] if debug).
+    draft_stats = (row_max, row_lse) [B, G] from topk_softmax(stats=True) on the
+    draft rows: the fused cycle (dflash2_verify_sample_ex), no second pass over
+    the draft rows."""
     _cuda(target, draft, draft_tok, seq_id)
     B, G1, V = target.shape
     G = G1 - 1
@@ -219,10 +240,21 @@ def verify_sample(target, draft, draft_tok, seed, step, seq_id=None, inv_tempera
     wp, wb = _ws(ws, dev, B, G, V)
     q = None if draft is None else draft.contiguous()
     sid = None if seq_id is None else seq_id.to(torch.int32).contiguous()
-    _check("dflash2_verify_sample", lib().dflash2_verify_sample(
-        _p(target.contiguous()), _p(q), _dtype(target), B, G, V, _p(draft_tok.contiguous()),
-        float(inv_temperature), int(seed) & (2 ** 64 - 1), int(step) & 0xFFFFFFFF, _p(sid),
-        int(q_mode), _p(n), _p(toks), _p(ratio), _p(u), wp, wb, _stream(dev)))
+    qmax = qlse = None
+    if draft_stats is not None:
+        qmax, qlse = (t.contiguous() for t in draft_stats)
+        _cuda(qmax, qlse)
+    seed, step = int(seed) & (2 ** 64 - 1), int(step) & 0xFFFFFFFF
+    if qmax is None:
+        _check("dflash2_verify_sample", lib().dflash2_verify_sample(
+            _p(target.contiguous()), _p(q), _dtype(target), B, G, V, _p(draft_tok.contiguous()),
+            float(inv_temperature), seed, step, _p(sid), int(q_mode), _p(n), _p(toks), _p(ratio),
+            _p(u), wp, wb, _stream(dev)))
+    else:
+        _check("dflash2_verify_sample_ex", lib().dflash2_verify_sample_ex(
+            _p(target.contiguous()), _p(q), _dtype(target), B, G, V, _p(draft_tok.contiguous()),
+            _p(qmax), _p(qlse), float(inv_temperature), seed, step, _p(sid), int(q_mode), _p(n),
+            _p(toks), _p(ratio), _p(u), wp, wb, _stream(dev)))
     return out
 
 

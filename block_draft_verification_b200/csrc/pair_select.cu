@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(NT, 2) pair_select_kernel(
     constexpr int IPT = (2 * K * RV + NT - 1) / NT;
     // W [D][D] in phase 1; the sequence's pair scores in phase 2
     extern __shared__ __align__(128) float s_dyn[];
-    __shared__ __align__(16) float s_left[K][LD];
+    __shared__ __align__(16) float s_leftT[D][K + 4];  // left rows transposed: [column][row]
     __shared__ __align__(16) float s_right[K][LD];
     __shared__ __align__(16) float s_f[K][LD];
     __shared__ int32_t s_tok[2 * K];           // right rows 0..15, left rows 16..
@@ -84,17 +84,21 @@ __global__ void __launch_bounds__(NT, 2) pair_select_kernel(
         for (int q = 0; q < IPT; ++q) {
             const int e = t + q * NT, r = e / RV, c = e - r * RV;
             if (r < K + nl) {
-                float4* dst = reinterpret_cast<float4*>((r < K) ? &s_right[r][c * VE]
-                                                                : &s_left[r - K][c * VE]);
                 const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-                if (EMB_BF16) {
-                    dst[0] = make_float4(__uint_as_float(w[0] << 16), __uint_as_float(w[0] & 0xFFFF0000u),
-                                         __uint_as_float(w[1] << 16), __uint_as_float(w[1] & 0xFFFF0000u));
-                    dst[1] = make_float4(__uint_as_float(w[2] << 16), __uint_as_float(w[2] & 0xFFFF0000u),
-                                         __uint_as_float(w[3] << 16), __uint_as_float(w[3] & 0xFFFF0000u));
+                float f[VE];
+#pragma unroll
+                for (int u = 0; u < VE; ++u)
+                    f[u] = EMB_BF16 ? __uint_as_float((u & 1) ? (w[u >> 1] & 0xFFFF0000u)
+                                                              : (w[u >> 1] << 16))
+                                    : __uint_as_float(w[u]);
+                if (r < K) {
+                    float4* dst = reinterpret_cast<float4*>(&s_right[r][c * VE]);
+#pragma unroll
+                    for (int u = 0; u < VE / 4; ++u)
+                        dst[u] = make_float4(f[4 * u], f[4 * u + 1], f[4 * u + 2], f[4 * u + 3]);
                 } else {
-                    dst[0] = make_float4(__uint_as_float(w[0]), __uint_as_float(w[1]),
-                                         __uint_as_float(w[2]), __uint_as_float(w[3]));
+#pragma unroll
+                    for (int u = 0; u < VE; ++u) s_leftT[c * VE + u][r - K] = f[u];
                 }
             }
         }
@@ -102,38 +106,55 @@ __global__ void __launch_bounds__(NT, 2) pair_select_kernel(
         if (!ok) {  // W never arrived: flag it, leave this position's scores unset
             if (t == 0) atomicOr(&g_dev_err, ERR_STREAM);
         } else {
-            // F = E_left W: thread -> 4 columns (a quad) of 16 / (NT / (D / 4)) left
-            // rows; each step of 4 along j reads 4 W rows and the rows' 4
-            // embedding values as 16-byte words (j ascending, one FMA chain
-            // per output)
-            constexpr int QUADS = D / 4;               // 32 for d = 128, 16 for d = 64
-            constexpr int RPT = K / (NT / QUADS);      // rows per thread: 2 or 1
-            const int cq = t % QUADS, r0 = (t / QUADS) * RPT;
+            // F = E_left W with K split over the eight warps (warp w: rows
+            // j of W in [w D/8, (w+1) D/8)); lane = a quad of 4 columns and
+            // RL left rows, so every W element is read from shared memory
+            // once.  Each warp's partial F goes to shared memory (over W once
+            // every warp is done with it) and the partials are added in warp
+            // order.
+            constexpr int QUADS = D / 4;             // 32 for d = 128, 16 for d = 64
+            constexpr int RL = K * QUADS / 32;       // left rows per lane: 16 or 8
+            constexpr int KW = D / (NT / 32);        // rows of W per warp: 16 or 8
+            const int cq = lane % QUADS, rg = (lane / QUADS) * RL;
             const float4* w4 = reinterpret_cast<const float4*>(s_dyn);
-            if (r0 < nl) {
-                float4 acc[RPT];
+            float4 acc[RL];
 #pragma unroll
-                for (int q = 0; q < RPT; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int r = 0; r < RL; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
-                for (int j = 0; j < D; j += 4) {
-                    const float4 wj[4] = {w4[(j + 0) * QUADS + cq], w4[(j + 1) * QUADS + cq],
-                                          w4[(j + 2) * QUADS + cq], w4[(j + 3) * QUADS + cq]};
+            for (int jj = 0; jj < KW; ++jj) {
+                const int j = warp * KW + jj;
+                const float4 wj = w4[j * QUADS + cq];
 #pragma unroll
-                    for (int q = 0; q < RPT; ++q) {
-                        const float4 el = *reinterpret_cast<const float4*>(&s_left[r0 + q][j]);
-                        const float ev[4] = {el.x, el.y, el.z, el.w};
+                for (int r4 = 0; r4 < RL / 4; ++r4) {
+                    const float4 e4 = *reinterpret_cast<const float4*>(&s_leftT[j][rg + 4 * r4]);
+                    const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            acc[q].x = fmaf(ev[u], wj[u].x, acc[q].x);
-                            acc[q].y = fmaf(ev[u], wj[u].y, acc[q].y);
-                            acc[q].z = fmaf(ev[u], wj[u].z, acc[q].z);
-                            acc[q].w = fmaf(ev[u], wj[u].w, acc[q].w);
-                        }
+                    for (int u = 0; u < 4; ++u) {
+                        float4& a = acc[4 * r4 + u];
+                        a.x = fmaf(ev[u], wj.x, a.x);
+                        a.y = fmaf(ev[u], wj.y, a.y);
+                        a.z = fmaf(ev[u], wj.z, a.z);
+                        a.w = fmaf(ev[u], wj.w, a.w);
                     }
                 }
+            }
+            __syncthreads();  // every warp is done with W
+            float4* part = reinterpret_cast<float4*>(s_dyn);  // [warp][row][quad]
 #pragma unroll
-                for (int q = 0; q < RPT; ++q)
-                    if (r0 + q < nl) *reinterpret_cast<float4*>(&s_f[r0 + q][4 * cq]) = acc[q];
+            for (int r = 0; r < RL; ++r) part[(warp * K + rg + r) * QUADS + cq] = acc[r];
+            __syncthreads();
+            for (int o = t; o < K * QUADS; o += NT) {  // (row, quad) outputs
+                const int r = o / QUADS, qd = o - r * QUADS;
+                float4 f = part[r * QUADS + qd];
+#pragma unroll
+                for (int w = 1; w < NT / 32; ++w) {
+                    const float4 g = part[(w * K + r) * QUADS + qd];
+                    f.x += g.x;
+                    f.y += g.y;
+                    f.z += g.z;
+                    f.w += g.w;
+                }
+                *reinterpret_cast<float4*>(&s_f[r][4 * qd]) = f;
             }
             __syncthreads();
             // S[k][k'] = F[k] . E_right[k'] (l ascending)
@@ -265,10 +286,11 @@ extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const 
 #define DFL_SEL(BF, DD)                                                                          \
     do {                                                                                         \
         auto kern = pair_select_kernel<BF, DD>;                                                  \
-        const int dyn = (int)(4 * std::max<int64_t>((int64_t)DD * DD, K + (int64_t)K * K * (G - 1))); \
-        if (dyn > 48 * 1024 &&                                                                   \
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) !=      \
-                cudaSuccess)                                                                     \
+        const int dyn = (int)(4 * std::max<int64_t>(std::max<int64_t>((int64_t)DD * DD, 8LL * K * DD),    \
+                                                    K + (int64_t)K * K * (G - 1)));              \
+        /* static + dynamic may pass 48 KB: raise the ceiling to what this call uses */          \
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) !=      \
+            cudaSuccess)                                                                         \
             return DFLASH2_ECUDA;                                                                \
         kern<<<grid, block, dyn, s>>>(idx, logp, anchor, emb, W, G, path_tok, path_rank,         \
                                       path_score, scores, counters);                             \

@@ -131,7 +131,9 @@ __device__ __forceinline__ void topk_chunk(const View& v, float c2, CandBuf& cb,
 __device__ __forceinline__ void topk_row_merge(const TopkPart* P, int S, int64_t row, float inv_t,
                                                float c2, int32_t* __restrict__ idx,
                                                float* __restrict__ prob, float* __restrict__ logp,
-                                               float* __restrict__ logz) {
+                                               float* __restrict__ logz,
+                                               float* __restrict__ row_max,
+                                               float* __restrict__ row_lse) {
     const int lane = threadIdx.x & 31;
     auto ldkey = [](const uint64_t* p) { return (uint64_t)__ldcg((const unsigned long long*)p); };
     // round 1: every chunk's (max, sum) and whether it carries a list
@@ -190,7 +192,11 @@ __device__ __forceinline__ void topk_row_merge(const TopkPart* P, int S, int64_t
         idx[o] = (int32_t)key_index(acc);
         prob[o] = (float)(exp2((x - (double)M) * (double)c2) / ssum);
         logp[o] = (float)((x - (double)M) * (double)inv_t - lns);
-        if (lane == 0) logz[row] = (float)((double)M * (double)inv_t + lns);
+        if (lane == 0) {
+            logz[row] = (float)((double)M * (double)inv_t + lns);
+            if (row_max) row_max[row] = M;
+            if (row_lse) row_lse[row] = (float)lns;
+        }
     }
 }
 
@@ -205,8 +211,8 @@ template <bool BF16, bool TMA>
 __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
     const void* __restrict__ logits, int64_t V, int64_t row_stride, int S, int64_t units,
     float inv_t, float c2, int32_t* __restrict__ idx, float* __restrict__ prob,
-    float* __restrict__ logp, float* __restrict__ logz, TopkPart* __restrict__ part,
-    unsigned* __restrict__ counters) {
+    float* __restrict__ logp, float* __restrict__ logz, float* __restrict__ row_max,
+    float* __restrict__ row_lse, TopkPart* __restrict__ part, unsigned* __restrict__ counters) {
     constexpr int ES = BF16 ? 2 : 4;
     constexpr int LEN = chunk_len(ES);
     extern __shared__ __align__(128) uint8_t ring[];
@@ -266,7 +272,8 @@ __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
             if (lane == 0) last = publish(&counters[row], seg, (unsigned)S);
             if (__shfl_sync(FULL, last, 0)) {
                 __syncwarp();  // lane 0's acquire covers the whole warp's reads
-                topk_row_merge(part + row * S, S, row, inv_t, c2, idx, prob, logp, logz);
+                topk_row_merge(part + row * S, S, row, inv_t, c2, idx, prob, logp, logz, row_max,
+                               row_lse);
             }
             run = 0ull;
             seg = 0;
@@ -289,10 +296,11 @@ unsigned dfl_errors_topk(int clear) {
     return v;
 }
 
-extern "C" int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows, int64_t V,
-                                    int64_t row_stride, float inv_temperature, int32_t* idx,
-                                    float* prob, float* logp, float* logz, void* ws,
-                                    size_t ws_bytes, dflash2_stream_t stream) {
+extern "C" int dflash2_topk_softmax_ex(const void* logits, int dtype, int64_t rows, int64_t V,
+                                       int64_t row_stride, float inv_temperature, int32_t* idx,
+                                       float* prob, float* logp, float* logz, float* row_max,
+                                       float* row_lse, void* ws, size_t ws_bytes,
+                                       dflash2_stream_t stream) {
     if (!dtype_ok(dtype)) return DFLASH2_EDTYPE;
     if (rows < 0 || V < K || V > INT32_MAX || row_stride < V) return DFLASH2_ESHAPE;
     if (!finite_pos(inv_temperature)) return DFLASH2_EINVAL;
@@ -300,7 +308,7 @@ extern "C" int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows,
     if (!logits || !idx || !prob || !logp || !logz) return DFLASH2_EINVAL;
     const int es = elem_size(dtype);
     if (!aligned(logits, es) || !aligned(idx, 4) || !aligned(prob, 4) || !aligned(logp, 4) ||
-        !aligned(logz, 4))
+        !aligned(logz, 4) || (row_max && !aligned(row_max, 4)) || (row_lse && !aligned(row_lse, 4)))
         return DFLASH2_EALIGN;
     const int64_t S = row_chunks(V, es);
     const int64_t units = rows * S;
@@ -323,7 +331,7 @@ extern "C" int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows,
         if (ring_prepare(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;                          \
         kern<<<ring_grid(units), RING_THREADS, dyn, s>>>(logits, V, row_stride, (int)S, units,    \
                                                          inv_temperature, c2, idx, prob, logp,    \
-                                                         logz, part, counters);                   \
+                                                         logz, row_max, row_lse, part, counters); \
     } while (0)
     if (dtype == DFLASH2_BF16) {
         if (tma) DFL_TOPK(true, true);
@@ -334,6 +342,14 @@ extern "C" int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows,
     }
 #undef DFL_TOPK
     return launch_status();
+}
+
+extern "C" int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows, int64_t V,
+                                    int64_t row_stride, float inv_temperature, int32_t* idx,
+                                    float* prob, float* logp, float* logz, void* ws,
+                                    size_t ws_bytes, dflash2_stream_t stream) {
+    return dflash2_topk_softmax_ex(logits, dtype, rows, V, row_stride, inv_temperature, idx, prob,
+                                   logp, logz, nullptr, nullptr, ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -246,7 +246,7 @@ __device__ __forceinline__ void sample_finish(
     int64_t V, int S, int es, float inv_t, float c2, const int32_t* __restrict__ draft_tok,
     uint64_t seed, uint32_t step, uint32_t sid, int q_mode, int b, int32_t* __restrict__ n_accept,
     int32_t* __restrict__ out_tok, float* __restrict__ ratio_dbg, float* __restrict__ u_dbg,
-    SampleInfo* __restrict__ info) {
+    SampleInfo* __restrict__ info, const float* __restrict__ q_max, const float* __restrict__ q_lse) {
     const int lane = threadIdx.x & 31;
     auto elem = [&](const void* base, int64_t row, int32_t v) -> double {
         if (es == 2)
@@ -260,9 +260,16 @@ __device__ __forceinline__ void sample_finish(
         xt_d = elem(target, (int64_t)b * (G + 1) + lane, dn);
         if (q_mode == DFLASH2_Q_SOFTMAX) xq_d = elem(draft, (int64_t)b * G + lane, dn);
     }
-    // lane j: (max, sum-exp) of target row j and draft row j
+    // lane j: (max, sum-exp) of target row j, and the draft row's max and
+    // ln sum-exp: from its partials, or as given (rows scanned: target only)
     LseD lt{-INFINITY, 0.0f, 0.0}, lq{-INFINITY, 0.0f, 0.0};
-    const int nrows = (q_mode == DFLASH2_Q_SOFTMAX) ? 2 * G + 1 : G + 1;
+    double lnq = 0.0;
+    const bool given = q_mode == DFLASH2_Q_SOFTMAX && q_max != nullptr;
+    if (given && lane < G) {
+        lq.m = q_max[(int64_t)b * G + lane];
+        lnq = (double)q_lse[(int64_t)b * G + lane];
+    }
+    const int nrows = (q_mode == DFLASH2_Q_SOFTMAX && !given) ? 2 * G + 1 : G + 1;
     for (int r0 = 0; r0 < nrows; r0 += 8) {
         float Mr[8];
         double Sr[8];
@@ -274,11 +281,12 @@ __device__ __forceinline__ void sample_finish(
             if (rr > G && rr < nrows && lane == rr - G - 1) lq = LseD{Mr[j], 0.0f, Sr[j]};
         }
     }
+    if (q_mode == DFLASH2_Q_SOFTMAX && !given && lane < G) lnq = log(lq.s);
     bool reject = false;
     if (lane < G) {
         // lp = z_t[d] - logZ_t = (x - m) * invT - ln(s); likewise lq
         double lr = (xt_d - (double)lt.m) * (double)inv_t - log(lt.s);
-        if (q_mode == DFLASH2_Q_SOFTMAX) lr -= (xq_d - (double)lq.m) * (double)inv_t - log(lq.s);
+        if (q_mode == DFLASH2_Q_SOFTMAX) lr -= (xq_d - (double)lq.m) * (double)inv_t - lnq;
         const double ratio = exp(lr);
         const float u = philox_uniform(seed, step, sid, (uint32_t)lane, 0u);
         reject = !((double)u < ratio);
@@ -291,7 +299,7 @@ __device__ __forceinline__ void sample_finish(
     const float ltm = __shfl_sync(FULL, lt.m, n);
     const double lts = __shfl_sync(FULL, lt.s, n);
     const float lqm = __shfl_sync(FULL, lq.m, n);
-    const double lqs = __shfl_sync(FULL, lq.s, n);
+    const double lqn = __shfl_sync(FULL, lnq, n);
     const int32_t d_n = __shfl_sync(FULL, dn, n);
     if (lane == 0) {
         SampleInfo I;
@@ -299,9 +307,8 @@ __device__ __forceinline__ void sample_finish(
         I.mt = ltm;
         I.l2t = (float)log2(lts);
         I.mq = lqm;
-        I.l2q = resid ? (float)log2(lqs) : 0.0f;
-        I.dl = resid ? (float)(((double)ltm - (double)lqm) * (double)inv_t + log(lts) - log(lqs))
-                     : 0.0f;
+        I.l2q = resid ? (float)(lqn * 1.4426950408889634) : 0.0f;
+        I.dl = resid ? (float)(((double)ltm - (double)lqm) * (double)inv_t + log(lts) - lqn) : 0.0f;
         I.u_res = philox_uniform(seed, step, sid, (uint32_t)n, 1u);
         I.n = n;
         I.mode = (n == G) ? 2 : (q_mode == DFLASH2_Q_SOFTMAX ? 0 : 1);
@@ -323,7 +330,8 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_scan_kernel(
     uint64_t seed, uint32_t step, const uint32_t* __restrict__ seq_id, int q_mode,
     int32_t* __restrict__ n_accept, int32_t* __restrict__ out_tok, float* __restrict__ ratio_dbg,
     float* __restrict__ u_dbg, LseD* __restrict__ part, SampleInfo* __restrict__ info,
-    unsigned* __restrict__ counters) {
+    unsigned* __restrict__ counters, const float* __restrict__ q_max,
+    const float* __restrict__ q_lse) {
     constexpr int ES = BF16 ? 2 : 4;
     constexpr int LEN = chunk_len(ES);
     extern __shared__ __align__(128) uint8_t ring[];
@@ -378,7 +386,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_scan_kernel(
                 __syncwarp();  // lane 0's acquire covers the whole warp's reads
                 sample_finish(target, draft, part + b * rows_per_seq * S, G, V, S, ES, inv_t, c2,
                               draft_tok, seed, step, seq_id ? seq_id[b] : (uint32_t)b, q_mode,
-                              (int)b, n_accept, out_tok, ratio_dbg, u_dbg, info);
+                              (int)b, n_accept, out_tok, ratio_dbg, u_dbg, info, q_max, q_lse);
             }
             seg = 0;
         }
@@ -527,6 +535,69 @@ __global__ void __launch_bounds__(DT) verify_sample_draw_kernel(
     dsum[((int64_t)b * D + c) * DT + threadIdx.x] = incl;
 }
 
+// The draw when the residual is empty by rounding: from p_n.  Two passes
+// over the row, chunk by chunk, the lanes taking part-1 threads 32 j + lane:
+// the thread sums in one inclusive scan (lane order within a group of 32,
+// groups and chunks in order), whose last value is R; then the same scan
+// against t = u' R, and the crossing thread walks its own elements.  Rare,
+// so kept out of line (the pick's common path stays small).  Returns the
+// element offset within the run starting at vb (lane 0; -1 if none).
+template <bool BF16, bool VEC>
+__device__ __noinline__ int draw_fallback(const char* trow, const char* qrow, int64_t V, int D,
+                                          const SampleInfo& I, float c2, float inv_t, int64_t& vb) {
+    const int lane = threadIdx.x & 31;
+    const int mode = 2;
+    int pick = -1;
+    auto scan_pass = [&](bool find, double tcut, int& cc_hit, int& t_hit, double& base) {
+        double acc = 0.0;
+        for (int cc = 0; cc < D; ++cc)
+            for (int j = 0; j < DT / 32; ++j) {
+                const int t = 32 * j + lane;
+                const double ts = draw_thread<BF16, VEC>(
+                    trow, qrow, (int64_t)cc * DLEN + (int64_t)DEPT * t, V, mode, I, c2, inv_t,
+                    nullptr);
+                double incl = ts;
+#pragma unroll
+                for (int k = 1; k < 32; k <<= 1) {
+                    const double o = __shfl_up_sync(FULL, incl, k);
+                    if (lane >= k) incl += o;
+                }
+                incl += acc;
+                if (find) {
+                    const unsigned cross = __ballot_sync(FULL, incl > tcut);
+                    if (cross) {
+                        const int l = __ffs(cross) - 1;
+                        cc_hit = cc;
+                        t_hit = 32 * j + l;
+                        base = __shfl_sync(FULL, incl - ts, l);
+                        return acc;
+                    }
+                }
+                acc = __shfl_sync(FULL, incl, 31);
+            }
+        return acc;
+    };
+    int cc_hit = -1, t_hit = -1;
+    double base = 0.0;
+    const double R = scan_pass(false, 0.0, cc_hit, t_hit, base);
+    const double tt = (double)I.u_res * R;
+    scan_pass(true, tt, cc_hit, t_hit, base);
+    if (cc_hit >= 0 && lane == 0) {
+        float w[DEPT];
+        vb = (int64_t)cc_hit * DLEN + (int64_t)DEPT * t_hit;
+        draw_thread<BF16, VEC>(trow, qrow, vb, V, mode, I, c2, inv_t, w);
+        double run = base;
+        int lm = -1;
+        for (int e = 0; e < DEPT; ++e) {
+            if (w[e] > 0.0f) lm = e;
+            run += (double)w[e];
+            if (pick < 0 && run > tt) pick = e;
+        }
+        if (pick < 0) pick = lm;
+    }
+    return pick;
+}
+
 // Draw, part 2: one warp per sequence.  R = the chunk sums in chunk order,
 // t = u' R; in the first chunk whose inclusive prefix exceeds t, the first
 // thread of part 1 whose inclusive prefix exceeds t (from the stored
@@ -637,35 +708,8 @@ __global__ void __launch_bounds__(32) verify_sample_pick_kernel(
                 if (pick < 0) pick = lm;
             }
         }
-    } else if (lane == 0) {
-        // fallback: R and the walk over the whole row from p_n in thread order
-        double R = 0.0;
-        for (int cc = 0; cc < D; ++cc)
-            for (int t = 0; t < DT; ++t)
-                R += draw_thread<BF16, VEC>(trow, qrow, (int64_t)cc * DLEN + (int64_t)DEPT * t, V,
-                                            mode, I, c2, inv_t, nullptr);
-        tt = (double)I.u_res * R;
-        double run = 0.0;
-        int lm = -1;
-        for (int cc = 0; cc < D && pick < 0; ++cc)
-            for (int t = 0; t < DT && pick < 0; ++t) {
-                float w[DEPT];
-                const int64_t v0 = (int64_t)cc * DLEN + (int64_t)DEPT * t;
-                draw_thread<BF16, VEC>(trow, qrow, v0, V, mode, I, c2, inv_t, w);
-                for (int e = 0; e < DEPT; ++e) {
-                    if (w[e] > 0.0f) lm = (int)(v0 + e);
-                    run += (double)w[e];
-                    if (run > tt) {
-                        pick = e;
-                        vb = v0;
-                        break;
-                    }
-                }
-            }
-        if (pick < 0 && lm >= 0) {
-            pick = 0;
-            vb = lm;
-        }
+    } else {
+        pick = draw_fallback<BF16, VEC>(trow, qrow, V, D, I, c2, inv_t, vb);
     }
     if (lane == 0 && pick >= 0) out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(vb + pick);
 }
@@ -748,12 +792,12 @@ extern "C" int dflash2_verify_greedy(const void* target, int dtype, int B, int G
     return launch_status();
 }
 
-extern "C" int dflash2_verify_sample(const void* target, const void* draft, int dtype, int B, int G,
-                                     int64_t V, const int32_t* draft_tok, float inv_temperature,
-                                     uint64_t seed, uint32_t step, const uint32_t* seq_id,
-                                     int q_mode, int32_t* n_accept, int32_t* out_tok,
-                                     float* ratio_dbg, float* u_dbg, void* ws, size_t ws_bytes,
-                                     dflash2_stream_t stream) {
+static int verify_sample_impl(const void* target, const void* draft, int dtype, int B, int G,
+                              int64_t V, const int32_t* draft_tok, const float* q_max,
+                              const float* q_lse, float inv_temperature, uint64_t seed,
+                              uint32_t step, const uint32_t* seq_id, int q_mode, int32_t* n_accept,
+                              int32_t* out_tok, float* ratio_dbg, float* u_dbg, void* ws,
+                              size_t ws_bytes, dflash2_stream_t stream) {
     if (!dtype_ok(dtype)) return DFLASH2_EDTYPE;
     if (B < 0 || G < 1 || G >= DFLASH2_MAX_BLOCK || V < 1 || V > INT32_MAX) return DFLASH2_ESHAPE;
     if (!finite_pos(inv_temperature)) return DFLASH2_EINVAL;
@@ -762,6 +806,9 @@ extern "C" int dflash2_verify_sample(const void* target, const void* draft, int 
     if (!target || !draft_tok || !n_accept || !out_tok) return DFLASH2_EINVAL;
     if (q_mode == DFLASH2_Q_SOFTMAX && !draft) return DFLASH2_EINVAL;
     const int es = elem_size(dtype);
+    if ((q_max == nullptr) != (q_lse == nullptr)) return DFLASH2_EINVAL;
+    if (q_mode != DFLASH2_Q_SOFTMAX) q_max = q_lse = nullptr;  // one-hot q needs no normaliser
+    if ((q_max && !aligned(q_max, 4)) || (q_lse && !aligned(q_lse, 4))) return DFLASH2_EALIGN;
     if (!aligned(target, es) || (draft && !aligned(draft, es)) || !aligned(draft_tok, 4) ||
         !aligned(n_accept, 4) || !aligned(out_tok, 4) || (seq_id && !aligned(seq_id, 4)) ||
         (ratio_dbg && !aligned(ratio_dbg, 4)) || (u_dbg && !aligned(u_dbg, 4)))
@@ -769,7 +816,8 @@ extern "C" int dflash2_verify_sample(const void* target, const void* draft, int 
     const int64_t S = row_chunks(V, es);
     const int64_t D = draw_chunks(V);
     if (D > DRAW_MAX_CHUNKS) return DFLASH2_ESHAPE;
-    const int rows_per_seq = (q_mode == DFLASH2_Q_SOFTMAX) ? 2 * G + 1 : G + 1;
+    // draft rows are scanned only when their normalisers are not given
+    const int rows_per_seq = (q_mode == DFLASH2_Q_SOFTMAX && !q_max) ? 2 * G + 1 : G + 1;
     const int64_t units = (int64_t)B * rows_per_seq * S;
     if (units > (int64_t)INT32_MAX || B > 65535) return DFLASH2_ESHAPE;
     const Layout L = sample_layout(B, G, V, es);
@@ -790,7 +838,8 @@ extern "C" int dflash2_verify_sample(const void* target, const void* draft, int 
         if (ring_prepare(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;                          \
         kern<<<ring_grid(units), RING_THREADS, dyn, s>>>(                                         \
             target, q, G, V, (int)S, rows_per_seq, units, inv_temperature, c2, draft_tok, seed,   \
-            step, seq_id, q_mode, n_accept, out_tok, ratio_dbg, u_dbg, part, info, counters);     \
+            step, seq_id, q_mode, n_accept, out_tok, ratio_dbg, u_dbg, part, info, counters,      \
+            q_max, q_lse);                                                                        \
         auto kern2 = verify_sample_draw_kernel<BF, TM>;                                           \
         if (launch_dependent(kern2, dim3((unsigned)D, (unsigned)B), dim3(DT), 0, s, target, q, G, \
                              V, (int)D, c2, inv_temperature, (const SampleInfo*)info, dsum) !=    \
@@ -811,4 +860,27 @@ extern "C" int dflash2_verify_sample(const void* target, const void* draft, int 
     }
 #undef DFL_SAMPLE
     return launch_status();
+}
+
+extern "C" int dflash2_verify_sample(const void* target, const void* draft, int dtype, int B, int G,
+                                     int64_t V, const int32_t* draft_tok, float inv_temperature,
+                                     uint64_t seed, uint32_t step, const uint32_t* seq_id,
+                                     int q_mode, int32_t* n_accept, int32_t* out_tok,
+                                     float* ratio_dbg, float* u_dbg, void* ws, size_t ws_bytes,
+                                     dflash2_stream_t stream) {
+    return verify_sample_impl(target, draft, dtype, B, G, V, draft_tok, nullptr, nullptr,
+                              inv_temperature, seed, step, seq_id, q_mode, n_accept, out_tok,
+                              ratio_dbg, u_dbg, ws, ws_bytes, stream);
+}
+
+extern "C" int dflash2_verify_sample_ex(const void* target, const void* draft, int dtype, int B,
+                                        int G, int64_t V, const int32_t* draft_tok,
+                                        const float* draft_max, const float* draft_lse,
+                                        float inv_temperature, uint64_t seed, uint32_t step,
+                                        const uint32_t* seq_id, int q_mode, int32_t* n_accept,
+                                        int32_t* out_tok, float* ratio_dbg, float* u_dbg, void* ws,
+                                        size_t ws_bytes, dflash2_stream_t stream) {
+    return verify_sample_impl(target, draft, dtype, B, G, V, draft_tok, draft_max, draft_lse,
+                              inv_temperature, seed, step, seq_id, q_mode, n_accept, out_tok,
+                              ratio_dbg, u_dbg, ws, ws_bytes, stream);
 }

@@ -120,6 +120,22 @@ DFLASH2_API int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows
                          dflash2_stream_t stream);
 
 /*
+ * dflash2_topk_softmax plus each row's normaliser in a form the sampling
+ * verify can reuse (the fused cycle: [tamsi] "L’idée, sans le papier" runs the
+ * drafter softmax once; dflash2_verify_sample_ex then needs no second pass
+ * over the draft rows).  Same arguments and results as
+ * dflash2_topk_softmax, and:
+ * row_max     [rows] float or NULL: max_v x_v (an element's value, exact);
+ * row_lse     [rows] float or NULL: ln sum_v exp((x_v - row_max) * inv_temperature),
+ *             so that logz = row_max * inv_temperature + row_lse.
+ */
+DFLASH2_API int dflash2_topk_softmax_ex(const void* logits, int dtype, int64_t rows, int64_t V,
+                                        int64_t row_stride, float inv_temperature, int32_t* idx,
+                                        float* prob, float* logp, float* logz, float* row_max,
+                                        float* row_lse, void* ws, size_t ws_bytes,
+                                        dflash2_stream_t stream);
+
+/*
  * Allocation-free dflash2_topk_softmax.  The paper has no counterpart: this
  * entry exists for callers that cannot give the library device memory -- an
  * inference engine that reserved nearly all of the GPU for its own pools at
@@ -222,6 +238,27 @@ DFLASH2_API int dflash2_verify_sample(const void* target, const void* draft, int
                           uint64_t seed, uint32_t step, const uint32_t* seq_id, int q_mode,
                           int32_t* n_accept, int32_t* out_tok, float* ratio_dbg, float* u_dbg,
                           void* ws, size_t ws_bytes, dflash2_stream_t stream);
+
+/*
+ * dflash2_verify_sample with the drafter's normalisers given (the fused
+ * cycle): draft_max, draft_lse [B, G] float as written by
+ * dflash2_topk_softmax_ex (row_max, row_lse) for the draft rows of the same
+ * inv_temperature.  Then q_j(d_j) = exp((x - draft_max) * inv_temperature
+ * - draft_lse) and the draft rows are not streamed: `draft` is read only at
+ * the drafted tokens and in the one row a residual draw uses.  Results as
+ * dflash2_verify_sample up to the float rounding of draft_lse (its ulp, at
+ * most 1e-6 for rows up to e^16 effective tokens, enters the ratios).
+ * draft_max and draft_lse are both given or both NULL (DFLASH2_EINVAL
+ * otherwise); both NULL, or q_mode DFLASH2_Q_ONEHOT, is
+ * dflash2_verify_sample exactly.
+ */
+DFLASH2_API int dflash2_verify_sample_ex(const void* target, const void* draft, int dtype, int B,
+                                         int G, int64_t V, const int32_t* draft_tok,
+                                         const float* draft_max, const float* draft_lse,
+                                         float inv_temperature, uint64_t seed, uint32_t step,
+                                         const uint32_t* seq_id, int q_mode, int32_t* n_accept,
+                                         int32_t* out_tok, float* ratio_dbg, float* u_dbg, void* ws,
+                                         size_t ws_bytes, dflash2_stream_t stream);
 
 /*
  * Two-tap dynamic depthwise conv fused with its tap projection and the

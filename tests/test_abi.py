@@ -138,6 +138,24 @@ def test_verify_validation(L):
     assert sample(t=ODD) == EALIGN
     assert sample(wsb=0) == EWORKSPACE
 
+    def sample_ex(qmax=P, qlse=P, qm=0, B=2, ws=P2, wsb=1 << 30):
+        return L.dflash2_verify_sample_ex(P, P, 1, B, 7, 151936, P, qmax, qlse, 1.0, 0, 0, None,
+                                          qm, P, P, None, None, ws, wsb, S0)
+    assert sample_ex(qlse=None) == EINVAL      # normalisers: both or neither
+    assert sample_ex(qmax=None) == EINVAL
+    assert sample_ex(qmax=ODD) == EALIGN
+    assert sample_ex(wsb=0) == EWORKSPACE
+    assert sample_ex(B=0) == OK
+
+
+def test_topk_ex_validation(L):
+    def topk_ex(rmax=P, rlse=P, V=151936):
+        return L.dflash2_topk_softmax_ex(P, 1, 4, V, V, 1.0, P, P, P, P, rmax, rlse, P2, 1 << 30,
+                                         S0)
+    assert topk_ex(V=15) == ESHAPE
+    assert topk_ex(rmax=ODD) == EALIGN
+    assert topk_ex(rlse=ODD) == EALIGN
+
 
 def test_dynconv_validation(L):
     def conv(x=P, xp=P, w=P, dt=1, B=2, T=8, H=5120, out=P2, ws=P2, wsb=1 << 30):

@@ -164,3 +164,24 @@ def test_large_magnitude_logits(orc, dt, invT):
     if dt == "bf16":
         x = synth.to_bf16_bits(x)
     check_rows(orc, x, invT)
+
+
+@pytest.mark.parametrize("name", ["tiny", "b8"])
+def test_row_stats(orc, name):
+    """dflash2_topk_softmax_ex: row_max is the row maximum exactly, row_lse =
+    logz - row_max * invT, the other outputs equal the plain call's bit for bit."""
+    need_cuda()
+    w = synth.WORKLOADS[name]
+    b = synth.gen_batch(w)
+    x = b.draft.reshape(-1, w.V)
+    for invT in (w.inv_temperature, 0.7):
+        X = to_dev(x)
+        plain = [to_host(t) for t in dfl.topk_softmax(X, invT)]
+        got = [to_host(t) for t in dfl.topk_softmax(X, invT, stats=True)]
+        torch.cuda.synchronize()
+        for a, g in zip(plain, got[:4]):
+            np.testing.assert_array_equal(a, g)
+        xf = synth.bf16_bits_to_f32(x) if x.dtype == np.uint16 else x
+        np.testing.assert_array_equal(got[4], xf.max(axis=1))
+        _, _, _, ologz = orc.topk_softmax(x, invT)
+        assert_close(got[5], ologz - xf.max(axis=1).astype(np.float64) * invT, RTOL_F32, "row_lse")

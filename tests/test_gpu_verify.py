@@ -101,14 +101,34 @@ def test_greedy_max_block(orc):
 
 
 # ------------------------------------------------------------------ sampling
+def draft_stats(orc, draft, invT):
+    """The drafter normalisers the fused cycle reuses: the row maximum (exact)
+    and ln sum exp((x - max) invT) in fp64 (scipy's logsumexp; any V, also
+    below the 16 candidates the top-16 needs), each rounded to float as
+    dflash2_topk_softmax_ex writes them."""
+    from scipy.special import logsumexp
+    B, G, V = draft.shape
+    rows = draft.reshape(-1, V)
+    x = (synth.bf16_bits_to_f32(rows) if rows.dtype == np.uint16 else rows).astype(np.float64)
+    mx = x.max(axis=1)
+    lse = logsumexp((x - mx[:, None]) * invT, axis=1)
+    return mx.astype(np.float32).reshape(B, G), lse.astype(np.float32).reshape(B, G)
+
+
 def check_sample(orc, target, draft, draft_tok, seed, step, seq_id=None, invT=1.0, q_mode=0,
-                 ties=None):
+                 ties=None, fused=False):
+    """fused: the drafter normalisers are given (dflash2_verify_sample_ex) and
+    the draft rows are read only at the drafted tokens and the drawn row; the
+    oracle is the same."""
     need_cuda()
     ties = ties if ties is not None else NearTies()
+    stats = None
+    if fused and draft is not None:
+        stats = tuple(to_dev(a) for a in draft_stats(orc, draft, invT))
     n, out, ratio, u = dfl.verify_sample(to_dev(target), None if draft is None else to_dev(draft),
                                          to_dev(draft_tok), seed, step,
                                          None if seq_id is None else to_dev(seq_id.view(np.int32)),
-                                         invT, q_mode, debug=True)
+                                         invT, q_mode, debug=True, draft_stats=stats)
     torch.cuda.synchronize()
     n, out, ratio, u = to_host(n), to_host(out), to_host(ratio), to_host(u)
     on, oout, oratio, ou, macc, mres = orc.verify_sample(target, draft, draft_tok, seed, step,
@@ -127,8 +147,8 @@ def check_sample(orc, target, draft, draft_tok, seed, step, seq_id=None, invT=1.
 
 
 @pytest.mark.parametrize("name", ["tiny", "b8", "b32", "ctx16"])
-@pytest.mark.parametrize("q_mode", [0, 1])
-def test_sample_workloads(orc, name, q_mode):
+@pytest.mark.parametrize("q_mode,fused", [(0, False), (1, False), (0, True)])
+def test_sample_workloads(orc, name, q_mode, fused):
     w = synth.WORKLOADS[name]
     B = min(w.B, 8) if name == "b32" else w.B
     b = synth.gen_batch(w, B=B)
@@ -136,16 +156,17 @@ def test_sample_workloads(orc, name, q_mode):
     ties = NearTies()
     for step in range(3):
         check_sample(orc, b.target, b.draft if q_mode == 0 else None, d, w.seed, step, b.seq_id,
-                     w.inv_temperature, q_mode, ties)
+                     w.inv_temperature, q_mode, ties, fused)
     print("near-ties:", ties.report())
 
 
-def test_sample_b32_full_batch_sampled(orc):
+@pytest.mark.parametrize("fused", [False, True])
+def test_sample_b32_full_batch_sampled(orc, fused):
     """The bench's launch (B=32); the oracle checks all 32 sequences once."""
     w = synth.WORKLOADS["b32"]
     b = synth.gen_batch(w)
     d = drafted_tokens(orc, w, b, np.random.default_rng(4), "cut")
-    check_sample(orc, b.target, b.draft, d, 7, 11, b.seq_id)
+    check_sample(orc, b.target, b.draft, d, 7, 11, b.seq_id, fused=fused)
 
 
 @pytest.mark.parametrize("V", [2, 8, 100, 16385, 33000])
@@ -163,6 +184,9 @@ def test_sample_small_vocab_many_sequences(orc, V, invT):
     on, _ = check_sample(orc, t, q, d, 99, 5, sid, invT, 0, ties)
     check_sample(orc, t, None, d, 99, 5, sid, invT, 1, ties)
     check_sample(orc, synth.to_bf16_bits(t), synth.to_bf16_bits(q), d, 99, 6, sid, invT, 0, ties)
+    check_sample(orc, t, q, d, 99, 7, sid, invT, 0, ties, fused=True)
+    check_sample(orc, synth.to_bf16_bits(t), synth.to_bf16_bits(q), d, 99, 8, sid, invT, 0, ties,
+                 fused=True)
     print("near-ties:", ties.report())
 
 
@@ -171,12 +195,13 @@ def test_sample_special_cases(orc):
     B, G, V = 32, 4, 300
     t = rng.standard_normal((B, G + 1, V)).astype(np.float32)
     d = rng.integers(0, V, (B, G)).astype(np.int32)
-    on, _ = check_sample(orc, t, t[:, :G].copy(), d, 1, 1)     # p = q: accept everything
-    assert np.all(on == G)
-    t2 = t.copy()
-    t2[np.arange(B), 0, d[:, 0]] = -1000.0                       # p(d_0) = 0: reject at 0
-    on, _ = check_sample(orc, t2, t[:, :G].copy(), d, 1, 2)
-    assert np.all(on == 0)
+    for fused in (False, True):
+        on, _ = check_sample(orc, t, t[:, :G].copy(), d, 1, 1, fused=fused)  # p = q: accept all
+        assert np.all(on == G)
+        t2 = t.copy()
+        t2[np.arange(B), 0, d[:, 0]] = -1000.0                   # p(d_0) = 0: reject at 0
+        on, _ = check_sample(orc, t2, t[:, :G].copy(), d, 1, 2, fused=fused)
+        assert np.all(on == 0)
     t3 = np.zeros((B, G + 1, V), np.float32)
     for j in range(G):
         t3[np.arange(B), j, d[:, j]] = 1000.0                    # one-hot, p(d) = 1: accept
@@ -196,6 +221,7 @@ def test_sample_large_magnitude_logits(orc):
     ties = NearTies()
     check_sample(orc, t, q, d, 3, 1, None, 1.0, 0, ties)
     check_sample(orc, t, None, d, 3, 2, None, 1.0, 1, ties)
+    check_sample(orc, t, q, d, 3, 1, None, 1.0, 0, ties, fused=True)
     print("near-ties:", ties.report())
 
 
@@ -212,3 +238,78 @@ def test_sample_batch_invariance(orc):
                                                  debug=True)]
     for a, o in zip(full, one):
         np.testing.assert_array_equal(a[2:3], o)
+
+
+def test_sample_fused_batch_invariance(orc):
+    """The fused cycle: a sequence's outputs do not depend on its batch."""
+    need_cuda()
+    w = synth.WORKLOADS["b8"]
+    b = synth.gen_batch(w)
+    d = drafted_tokens(orc, w, b, np.random.default_rng(6), "cut")
+    T, Q, D = to_dev(b.target), to_dev(b.draft), to_dev(d)
+    sid = to_dev(b.seq_id.view(np.int32))
+    mx, lse = (to_dev(a) for a in draft_stats(orc, b.draft, w.inv_temperature))
+    full = [to_host(x) for x in dfl.verify_sample(T, Q, D, 3, 4, sid, debug=True,
+                                                 draft_stats=(mx, lse))]
+    one = [to_host(x) for x in dfl.verify_sample(T[2:3].contiguous(), Q[2:3].contiguous(),
+                                                 D[2:3].contiguous(), 3, 4, sid[2:3].contiguous(),
+                                                 debug=True,
+                                                 draft_stats=(mx[2:3].contiguous(),
+                                                              lse[2:3].contiguous()))]
+    for a, o in zip(full, one):
+        np.testing.assert_array_equal(a[2:3], o)
+
+
+def test_fused_cycle_matches_topk_stats(orc):
+    """End to end: the statistics come from dflash2_topk_softmax_ex on the
+    GPU (not the oracle) and feed dflash2_verify_sample_ex; the oracle's
+    unfused verify decides."""
+    need_cuda()
+    w = synth.WORKLOADS["b8"]
+    b = synth.gen_batch(w)
+    d = drafted_tokens(orc, w, b, np.random.default_rng(8), "cut")
+    B, G, V = b.draft.shape
+    Q = to_dev(b.draft)
+    _, _, _, _, mx, lse = dfl.topk_softmax(Q.view(B * G, V), w.inv_temperature, stats=True)
+    n, out, ratio, u = dfl.verify_sample(to_dev(b.target), Q, to_dev(d), w.seed, 9,
+                                         to_dev(b.seq_id.view(np.int32)), w.inv_temperature,
+                                         debug=True, draft_stats=(mx.view(B, G), lse.view(B, G)))
+    torch.cuda.synchronize()
+    on, oout, oratio, ou, macc, mres = orc.verify_sample(b.target, b.draft, d, w.seed, 9, b.seq_id,
+                                                         w.inv_temperature, 0)
+    assert_close(to_host(ratio), oratio, RTOL_F32, "ratio")
+    n, out = to_host(n), to_host(out)
+    for s in range(B):
+        if n[s] != on[s]:
+            assert macc[s] < ACCEPT_BAND
+        elif not np.array_equal(out[s], oout[s]):
+            assert mres[s] < DRAW_BAND
+
+
+def test_sample_fallback_when_residual_empty(orc):
+    """A rejected row whose residual max(0, p - q) is empty makes the draw use
+    p_n (the reading for an empty residual).  Made here on purpose through the
+    fused entry: p_0 is a spike; the draft row equals the target row except a
+    large logit at the drafted token d_0 (q(d_0) ~ 5e-5, p(d_0) ~ 0: row 0
+    rejects), and the given normaliser is 1 too small, so q = e q_true covers
+    p everywhere (q(spike) ~ e > p(spike) = 1): the residual is empty and the
+    draw must return the spike's token."""
+    need_cuda()
+    rng = np.random.default_rng(17)
+    B, G, V = 6, 2, 25000                       # three draw chunks per row
+    t = rng.standard_normal((B, G + 1, V)).astype(np.float32)
+    spike = rng.integers(0, V, B)
+    t[np.arange(B), 0, spike] = 1000.0          # p_0 is one-hot at the spike
+    d = np.zeros((B, G), np.int32)
+    d[:, 0] = (spike + 1) % V                   # p_0(d_0) ~ exp(-1000): reject at 0
+    d[:, 1] = spike
+    q = t[:, :G].copy()
+    q[np.arange(B), 0, d[:, 0]] = 990.0
+    mx, lse = draft_stats(orc, q, 1.0)
+    n, out = dfl.verify_sample(to_dev(t), to_dev(q), to_dev(d), 5, 1,
+                               draft_stats=(to_dev(mx), to_dev(lse - 1.0)))[:2]
+    torch.cuda.synchronize()
+    n, out = to_host(n), to_host(out)
+    np.testing.assert_array_equal(n, np.zeros(B, np.int32))
+    np.testing.assert_array_equal(out[:, 0], spike.astype(np.int32))
+    assert np.all(out[:, 1:] == -1)
