@@ -182,9 +182,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     uint8_t* s_xp = s_x + sh.BN * 128;
     uint8_t* s_x0 = s_xp + sh.R * 128;
     uint8_t* s_out = s_x0 + 128;  // [2][32 tokens][64 channels] bf16 outputs
-    // wfull[SW], wempty[SW], xfull[SX], xempty[SX], tmem_full[2], tmem_empty[2], mma_done, x tile
+    // wfull[SW], wempty[SW], xfull[SX], xempty[SX], tmem_full[2], tmem_empty[2], mma_done,
+    // x tile, staged partial
     uint64_t* bars = (uint64_t*)(s_out + 8192);
-    uint32_t* s_tmem = (uint32_t*)(bars + 2 * sh.sw + 2 * sh.sx + 6);
+    uint32_t* s_tmem = (uint32_t*)(bars + 2 * sh.sw + 2 * sh.sx + 7);
     int* s_fail = (int*)(s_tmem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -196,6 +197,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     const uint32_t tempty0 = tfull0 + 16;
     const uint32_t mdone = tfull0 + 32;
     const uint32_t xbar = tfull0 + 40;
+    const uint32_t pbar = tfull0 + 48;  // a partial staged in the idle rings
     const uint32_t ncols = 2 * (uint32_t)sh.bufcols;
 
     if (threadIdx.x == 0) {
@@ -213,6 +215,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
         }
         mbar_init(mdone, 1);
         mbar_init(xbar, 1);
+        mbar_init(pbar, 1);
         mbar_fence_init();
         *s_fail = 0;
     }
@@ -309,7 +312,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
         const int q = warp - 4;  // TMEM lanes 32q .. 32q + 31
         const int e = threadIdx.x - 128;
         const int row = 32 * q + lane;
-        int j = 0, nown = 0;  // segments, owned segments (x tile barrier phases)
+        int j = 0, nown = 0, nstaged = 0;  // segments, owned segments, staged partials
+        const uint32_t part_bytes = (uint32_t)sh.ngroups * 8 * TC_BM * 16;
+        const uint32_t ring_bytes = (uint32_t)sh.sw * TC_A_BYTES + (uint32_t)sh.sx * xstage;
         float4 pp0[8], pp1[8];  // the first partial, two groups ahead of its use
         for (int64_t sg = s0; sg < s1; ++j) {
             const int tile = (int)(sg / sh.nkb);
@@ -322,9 +327,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
             // runs that start inside an owned tile hand it partials (CTA order = K order)
             int q_end = p + 1;
             const float4* part1 = partial + (int64_t)(p + 1) * sh.ngroups * 8 * TC_BM;
+            // the run's last segment: every load and MMA of this CTA is done by
+            // the time its accumulator is, so the first partial can come into
+            // the idle rings in one go; the next one is prefetched through
+            // registers two groups ahead, any further ones read in place
+            const bool will_stage = sg == s1 && part_bytes <= ring_bytes;
+            const int q_reg = p + 1 + (will_stage ? 1 : 0);
+            const float4* partr = partial + (int64_t)q_reg * sh.ngroups * 8 * TC_BM;
             auto load_part = [&](int g, float4 (&po)[8]) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) po[c] = __ldcg(&part1[((int64_t)g * 8 + c) * TC_BM + row]);
+                for (int c = 0; c < 8; ++c) po[c] = __ldcg(&partr[((int64_t)g * 8 + c) * TC_BM + row]);
             };
             if (klo == 0) {
                 // owned tile, while its MMAs run: stage its x rows, the x_prev
@@ -354,7 +366,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
                     __threadfence();
                 }
                 epi_sync();
-                if (!*s_fail && q_end > p + 1) {
+                if (!*s_fail && q_end > q_reg) {
                     load_part(0, pp0);
                     if (sh.ngroups > 1) load_part(1, pp1);
                 }
@@ -392,8 +404,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
                 *s_fail = 1;
             }
             ++nown;
-            epi_sync();
             const bool first_part = *s_fail == 0 && q_end > p + 1;
+            const bool staged = first_part && will_stage;
+            const bool reg_part = *s_fail == 0 && q_end > q_reg;
+            if (staged) {
+                if (e == 0) {  // 32 KB pieces into the rings (free: all MMAs are done)
+                    mbar_expect_tx(pbar, part_bytes);
+                    for (uint32_t off = 0; off < part_bytes; off += 32768u)
+                        bulk_g2s_nx(smem_u32(wring) + off, (const char*)part1 + off,
+                                    min(32768u, part_bytes - off), pbar);
+                }
+                if (!mbar_wait(pbar, (uint32_t)(nstaged & 1))) {
+                    atomicOr(&g_dev_err, ERR_EPILOGUE);
+                    *s_fail = 1;
+                }
+                ++nstaged;
+            }
+            epi_sync();
+            if (*s_fail) break;  // uniform over the four warps
+            const float4* sp = (const float4*)wring;
             // lane l of epilogue warp q: channel cl = 16q + (l & 15) of the tile,
             // tokens 16 (l >> 4) .. +15 of each 32-token group; a and b of the
             // channel meet by one exchange between lanes l and l ^ 16
@@ -401,7 +430,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
             for (int g = 0; g < sh.ngroups; ++g) {
                 float v[32];
                 tmem_ld32(tacc + 32 * g, v);
-                if (first_part) {
+                if (staged) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 w = sp[(g * 8 + c) * TC_BM + row];
+                        v[4 * c] += w.x;
+                        v[4 * c + 1] += w.y;
+                        v[4 * c + 2] += w.z;
+                        v[4 * c + 3] += w.w;
+                    }
+                }
+                if (reg_part) {
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         v[4 * c] += pp0[c].x;
@@ -411,7 +450,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
                         pp0[c] = pp1[c];
                     }
                     if (g + 2 < sh.ngroups) load_part(g + 2, pp1);
-                    for (int q2 = p + 2; q2 < q_end; ++q2) {  // further partials, in K order
+                }
+                if (first_part) {
+                    for (int q2 = q_reg + 1; q2 < q_end; ++q2) {  // further partials, in K order
                         const float4* src = partial + (int64_t)q2 * sh.ngroups * 8 * TC_BM;
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
