@@ -140,15 +140,18 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- traffic
 def recorded_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel's
-    source has not changed since it was captured; else None."""
+    """DRAM bytes per call from the committed ncu summary (profiles/traffic.json),
+    if none of the call's source files has changed since it was captured; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[kernel]
-        src = os.path.join(ROOT, "block_draft_verification_b200", "csrc", rec["source"])
-        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        return float(rec["dram_bytes_per_launch"]) if digest == rec["source_sha256_16"] else None
+        h = hashlib.sha256()
+        for name in rec["sources"]:
+            h.update(open(os.path.join(ROOT, "block_draft_verification_b200", "csrc", name), "rb").read())
+        if h.hexdigest()[:16] != rec["sources_sha256_16"]:
+            return None
+        return float(rec["dram_bytes_per_call"])
     except Exception:
         return None
 
