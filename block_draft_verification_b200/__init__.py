@@ -114,7 +114,9 @@ def _cuda(*ts):
 
 class Workspace:
     """A device scratch buffer for the calls that take one.  Calls on one
-    stream run in order, so one Workspace serves every call on that stream."""
+    stream run in order, so one Workspace serves every call on that stream.
+    It is zero-filled when (re)allocated: the calls expect their counters
+    (the first 64 KB) zero and leave them zero when they complete."""
 
     def __init__(self, device=None, nbytes=0):
         self.device = torch.device(device if device is not None else "cuda")
@@ -123,7 +125,7 @@ class Workspace:
 
     def reserve(self, nbytes):
         if nbytes > self.buf.numel():
-            self.buf = torch.empty(int(nbytes), dtype=torch.uint8, device=self.device)
+            self.buf = torch.zeros(int(nbytes), dtype=torch.uint8, device=self.device)
         return self
 
     def args(self, B, G, V):

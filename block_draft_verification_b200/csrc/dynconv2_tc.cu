@@ -46,6 +46,7 @@
 
 #include "common.cuh"
 #include "stream.cuh"
+#include "workspace.cuh"
 
 namespace dfl {
 
@@ -362,6 +363,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
                                 break;
                             }
                         }
+                        if (!*s_fail) flags[q2] = 0u;  // consumed: leave the flag zero
                     }
                     __threadfence();
                 }
@@ -604,7 +606,9 @@ static TcPlan tc_plan(int64_t ntok, int H, int sms) {
     P.nkb = H / TC_BK;
     P.steps = nt * P.nh * P.nkb;
     P.nctas = (int)std::min<int64_t>(std::min(sms, TC_MAXCTA), P.steps);
-    P.flags_bytes = (size_t)TC_MAXCTA * 4;
+    // flags in the workspace's control area (zero between calls: each owner
+    // resets the flags it consumed), partials after it
+    P.flags_bytes = dfl::CONTROL_BYTES;
     P.part_bytes = (size_t)P.nctas * P.ngroups * 8 * TC_BM * sizeof(float4);
     return P;
 }
@@ -660,7 +664,6 @@ int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_
     }
     unsigned* flags = (unsigned*)ws;
     float4* part = (float4*)((char*)ws + P.flags_bytes);
-    if (cudaMemsetAsync(flags, 0, (size_t)P.nctas * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
     TcShape sh{H, T, ntok, P.BN, sw, sx, P.nkb, P.nh, P.bufcols, P.ngroups, P.nctas, R, P.steps};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)P.nctas);

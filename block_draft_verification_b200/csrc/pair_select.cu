@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(NT, 2) pair_select_kernel(
     if (t == 0) __threadfence();
 
     if (!arrive_last(&counters[b], (unsigned)G)) return;
+    if (t == 0) counters[b] = 0u;  // every CTA of the sequence has arrived: leave it zero
     if (s_bad) return;  // this CTA's W copy may still be in flight: leave its smem alone
 
     // ---- last CTA of the sequence: everything the recursion reads, in one pass
@@ -281,7 +282,8 @@ extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const 
     cudaStream_t s = (cudaStream_t)stream;
     unsigned* counters = (unsigned*)((char*)ws + L.counters_off);
     float* scores = (float*)((char*)ws + L.part_off);
-    if (cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
+    if (!L.self_clean && cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess)
+        return DFLASH2_ECUDA;
     const dim3 grid((unsigned)((int64_t)B * G)), block(NT);
 #define DFL_SEL(BF, DD)                                                                          \
     do {                                                                                         \

@@ -274,6 +274,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
                 __syncwarp();  // lane 0's acquire covers the whole warp's reads
                 topk_row_merge(part + row * S, S, row, inv_t, c2, idx, prob, logp, logz, row_max,
                                row_lse);
+                if (lane == 0) counters[row] = 0u;  // the row is done: leave its counter zero
             }
             run = 0ull;
             seg = 0;
@@ -319,7 +320,8 @@ extern "C" int dflash2_topk_softmax_ex(const void* logits, int dtype, int64_t ro
     cudaStream_t s = (cudaStream_t)stream;
     unsigned* counters = (unsigned*)((char*)ws + L.counters_off);
     TopkPart* part = (TopkPart*)((char*)ws + L.part_off);
-    if (cudaMemsetAsync(counters, 0, (size_t)rows * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
+    if (!L.self_clean && cudaMemsetAsync(counters, 0, (size_t)rows * 4, s) != cudaSuccess)
+        return DFLASH2_ECUDA;
 
     // TMA bulk copies need 16-byte aligned chunk starts and 16-byte multiples
     const bool tma = aligned(logits, 16) && (row_stride * es) % 16 == 0 && (V * es) % 16 == 0;
@@ -397,6 +399,9 @@ extern "C" int dflash2_topk_softmax_noalloc(const void* logits, int dtype, int64
     if (rows == 0) return DFLASH2_OK;
     void* scratch = noalloc_scratch_on_current_device();
     if (!scratch) return DFLASH2_ECUDA;
+    // the array's counters start at zero whatever an earlier (failed) call left
+    if (cudaMemsetAsync(scratch, 0, (size_t)rows * 4, (cudaStream_t)stream) != cudaSuccess)
+        return DFLASH2_ECUDA;
     return dflash2_topk_softmax(logits, dtype, rows, V, row_stride, inv_temperature, idx, prob, logp,
                                 logz, scratch, NOALLOC_SCRATCH_BYTES, stream);
 }

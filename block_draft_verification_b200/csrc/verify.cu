@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_kernel(
             if (__shfl_sync(FULL, last, 0)) {
                 __syncwarp();  // lane 0's acquire covers the whole warp's reads
                 greedy_finish(part + b * (G + 1) * S, S, G, (int)b, draft_tok, n_accept, out_tok);
+                if (lane == 0) counters[b] = 0u;  // the sequence is done: leave its counter zero
             }
             seg = 0;
         }
@@ -387,6 +388,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_scan_kernel(
                 sample_finish(target, draft, part + b * rows_per_seq * S, G, V, S, ES, inv_t, c2,
                               draft_tok, seed, step, seq_id ? seq_id[b] : (uint32_t)b, q_mode,
                               (int)b, n_accept, out_tok, ratio_dbg, u_dbg, info, q_max, q_lse);
+                if (lane == 0) counters[b] = 0u;  // the sequence is done: leave its counter zero
             }
             seg = 0;
         }
@@ -770,7 +772,8 @@ extern "C" int dflash2_verify_greedy(const void* target, int dtype, int B, int G
     cudaStream_t s = (cudaStream_t)stream;
     unsigned* counters = (unsigned*)((char*)ws + L.counters_off);
     uint64_t* part = (uint64_t*)((char*)ws + L.part_off);
-    if (cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
+    if (!L.self_clean && cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess)
+        return DFLASH2_ECUDA;
     // TMA bulk copies need 16-byte aligned chunk starts and 16-byte multiples
     const bool tma = aligned(target, 16) && (V * es) % 16 == 0;
 #define DFL_GREEDY(BF, TM)                                                                       \
@@ -827,7 +830,8 @@ static int verify_sample_impl(const void* target, const void* draft, int dtype, 
     LseD* part = (LseD*)((char*)ws + L.part_off);
     double* dsum = (double*)((char*)ws + L.part2_off);
     SampleInfo* info = (SampleInfo*)((char*)ws + L.info_off);
-    if (cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess) return DFLASH2_ECUDA;
+    if (!L.self_clean && cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess)
+        return DFLASH2_ECUDA;
     const void* q = (q_mode == DFLASH2_Q_SOFTMAX) ? draft : nullptr;
     const bool tma = aligned(target, 16) && (!q || aligned(q, 16)) && (V * es) % 16 == 0;
     const float c2 = (float)((double)inv_temperature * LOG2E);

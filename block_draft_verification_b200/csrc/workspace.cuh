@@ -1,7 +1,12 @@
 // workspace.cuh -- layout of the caller-provided workspace of each call.
 //
-// Every layout puts the arrival counters first (cleared by the call with one
-// cudaMemsetAsync) and the per-unit partial results after them; both regions
+// The first CONTROL_BYTES of every workspace hold the calls' arrival counters
+// (and dynconv's flags); partial results start after them, so no call's
+// partials ever land on another call's counters.  A call whose counters fit
+// the control area relies on them being zero and leaves them zero when it
+// completes (its finishers reset what they used): a workspace is zeroed once,
+// when it is allocated.  A call with more counters than fit (shapes far beyond
+// the bench's) clears its own with one cudaMemsetAsync instead.  All regions
 // start on 256-byte boundaries.
 #pragma once
 
@@ -41,6 +46,7 @@ struct SampleInfo {
 constexpr int DRAW_LEN = 10240;
 
 struct Layout {
+    bool self_clean;  // counters in the control area: zero on entry, reset by the call
     size_t counters_off, counters_bytes;
     size_t part_off, part_bytes;
     size_t part2_off, part2_bytes;
@@ -50,11 +56,17 @@ struct Layout {
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+constexpr size_t CONTROL_BYTES = 65536;
+
+// True when a call's counters fit the control area (self-cleaning, no memset).
+inline bool counters_in_control(size_t counters) { return counters <= CONTROL_BYTES; }
+
 inline Layout make_layout(size_t counters, size_t part, size_t part2 = 0, size_t info = 0) {
     Layout L;
+    L.self_clean = counters_in_control(counters);
     L.counters_off = 0;
     L.counters_bytes = align256(counters);
-    L.part_off = L.counters_bytes;
+    L.part_off = L.counters_bytes > CONTROL_BYTES ? L.counters_bytes : CONTROL_BYTES;
     L.part_bytes = align256(part);
     L.part2_off = L.part_off + L.part_bytes;
     L.part2_bytes = align256(part2);

@@ -41,9 +41,15 @@
  *     buffers do not overlap inputs.
  *   - Calls that take a workspace (`ws`, `ws_bytes`): a device buffer of at
  *     least dflash2_workspace_bytes(B, G, V) bytes, 256-byte aligned, used
- *     for per-chunk partial results and arrival counters.  The call clears
- *     the part it needs at its start, so its contents between calls do not
- *     matter; two calls that may run concurrently need separate workspaces.
+ *     for arrival counters and per-chunk partial results.  Its first 64 KB
+ *     hold the counters of every call and must be ZERO when the workspace is
+ *     first used (e.g. cudaMemset once after allocating it); every call that
+ *     completes leaves them zero again (its kernels reset what they used), so
+ *     one workspace serves any sequence of calls on a stream without further
+ *     clearing.  After dflash2_device_errors reports a failure, zero those
+ *     64 KB again before reusing the workspace.  The rest of the workspace
+ *     needs no initialisation.  Two calls that may run concurrently need
+ *     separate workspaces.
  *   - Results are deterministic: a sequence's outputs depend only on its own
  *     inputs (and seq_id), not on the batch it runs in or on B.
  */
@@ -146,12 +152,12 @@ DFLASH2_API int dflash2_topk_softmax_ex(const void* logits, int dtype, int64_t r
  * workspace: the scratch is a fixed array of DFLASH2_NOALLOC_SCRATCH_BYTES in
  * the library's own device memory, present on every GPU that loads the
  * library until the process exits.  The call allocates nothing (no
- * cudaMalloc, no cudaFree, no allocating library routine); it clears the part
- * of the array it uses with cudaMemsetAsync on `stream`.
- *   - Limit: rows * ceil(V / L) * 144 + rows * 4 bytes (L = 4096 for bf16,
- *     2048 for fp32: the rows are reduced in chunks of 8 KB; each term rounded up
- *     to 256) must fit in the array; larger shapes return DFLASH2_EWORKSPACE
- *     and enqueue nothing.  At V = 151,936 in bf16 that is up to 765 rows.
+ * cudaMalloc, no cudaFree, no allocating library routine); it clears the
+ * array's counters with cudaMemsetAsync on `stream` before every call.
+ *   - Limit: 64 KB + rows * ceil(V / L) * 144 bytes (L = 4096 for bf16, 2048
+ *     for fp32: the rows are reduced in chunks of 8 KB; rounded up to 256)
+ *     must fit in the array; larger shapes return DFLASH2_EWORKSPACE
+ *     and enqueue nothing.  At V = 151,936 in bf16 that is up to 754 rows.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind: two calls that can overlap on the GPU (different streams without
  *     an ordering between them) race and give wrong results.
@@ -274,8 +280,9 @@ DFLASH2_API int dflash2_verify_sample_ex(const void* target, const void* draft, 
  * possibly split between SMs; the split depends on B * T, H and the SM
  * count only, and the parts are added in K order, so a given shape on a
  * given device always rounds the same way.  It needs a workspace of
- * dflash2_dynconv2_workspace_bytes bytes (256-byte aligned; contents need
- * not be initialised; one call at a time per workspace); fp32 needs none
+ * dflash2_dynconv2_workspace_bytes bytes (256-byte aligned; the same
+ * contract as the other calls' workspaces: the first 64 KB zero on first use,
+ * left zero by every completed call; one call at a time per workspace); fp32 needs none
  * (ws may be NULL).
  */
 DFLASH2_API int dflash2_dynconv2(const void* x, const void* x_prev, const void* w_tap, int dtype, int B,
