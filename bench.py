@@ -255,7 +255,7 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_sink = torch.zeros((), dtype=torch.int64, device=dev)
     names = ["topk_softmax", "pair_select", "verify_sample", "verify_greedy", "dynconv2"]
-    kernels_per_step = {"topk_softmax": 1, "pair_select": 1, "verify_sample": 3,
+    kernels_per_step = {"topk_softmax": 1, "pair_select": 1, "verify_sample": 1,
                         "verify_greedy": 1, "dynconv2": 1}
 
     def calls(inp, step):

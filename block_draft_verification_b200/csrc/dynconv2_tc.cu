@@ -136,14 +136,6 @@ struct TcShape {
 __device__ __forceinline__ int64_t run_start(const TcShape& sh, int p) {
     return sh.steps * p / sh.nctas;
 }
-__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 // One bf16 from shared memory, widened to fp32 (exact).
 __device__ __forceinline__ float lds_bf16(uint32_t addr) {
     unsigned short v;

@@ -88,6 +88,10 @@ struct WarpRing {
     __device__ __forceinline__ bool wait(int k) const {
         return mbar_wait(bar + 8 * (k & 1), (uint32_t)((k >> 1) & 1));
     }
+    // the same for a unit issued just before (polled, never suspended)
+    __device__ __forceinline__ bool wait_fresh(int k) const {
+        return mbar_wait_poll(bar + 8 * (k & 1), (uint32_t)((k >> 1) & 1));
+    }
     // every lane is done reading unit k's slot: lane 0 may refill it
     __device__ __forceinline__ void done(int k) const {
         __syncwarp();
@@ -96,27 +100,32 @@ struct WarpRing {
     }
 };
 
-// Set up the calling warp's ring (barriers in `bars`, two per warp) and
-// issue its first two units.  `ic` is the issue cursor, at the warp's first
-// unit; src(ic, p, bytes) gives that unit's address and size; ic ends two
-// units on.
-// Bring unit k in (lane 0 issues the copy); a short chunk's slot is filled
-// past its end with `fill` words (-inf), so every chunk in shared memory is
-// a full slot and the reductions need no bounds checks.
+// Bring unit k in: `bytes` from p (lane 0 issues the copy); a short chunk's
+// slot is filled past its end with `fill` words (-inf), so every chunk in
+// shared memory is a full slot and the reductions need no bounds checks.
+__device__ __forceinline__ void warp_ring_load(const WarpRing& r, int k, const char* p,
+                                               uint32_t bytes, uint32_t fill) {
+    if (bytes < (uint32_t)SLOT_BYTES) {
+        uint4* t = (uint4*)r.slot(k);
+        for (int q = (int)(bytes / 16) + (threadIdx.x & 31); q < SLOT_BYTES / 16; q += 32)
+            t[q] = make_uint4(fill, fill, fill, fill);
+        __syncwarp();  // the fill is seen by every lane that later reads the slot
+    }
+    if ((threadIdx.x & 31) == 0) r.issue(k, p, bytes);
+}
 template <class Src>
 __device__ __forceinline__ void warp_ring_issue(const WarpRing& r, int k, const UnitCursor& ic,
                                                 uint32_t fill, Src src) {
     const char* p;
     uint32_t bytes;
     src(ic, p, bytes);
-    if (bytes < (uint32_t)SLOT_BYTES) {
-        uint4* t = (uint4*)r.slot(k);
-        for (int q = (int)(bytes / 16) + (threadIdx.x & 31); q < SLOT_BYTES / 16; q += 32)
-            t[q] = make_uint4(fill, fill, fill, fill);
-    }
-    if ((threadIdx.x & 31) == 0) r.issue(k, p, bytes);
+    warp_ring_load(r, k, p, bytes, fill);
 }
 
+// Set up the calling warp's ring (barriers in `bars`, two per warp) and
+// issue its first two units.  `ic` is the issue cursor, at the warp's first
+// unit; src(ic, p, bytes) gives that unit's address and size; ic ends two
+// units on.
 template <class Src>
 __device__ __forceinline__ WarpRing warp_ring_start(uint8_t* ring, uint64_t* bars, int n,
                                                     UnitCursor& ic, uint32_t fill, Src src) {

@@ -73,6 +73,30 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
         if (global_ns() - t0 > WAIT_NS) return false;
     }
 }
+// The same wait without the suspend hint: test_wait (which never suspends)
+// polled with a short sleep, for a copy issued just before the wait (there
+// the hint's suspension can outlast the copy by far); false after WAIT_NS.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+__device__ __forceinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity) {
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        __nanosleep(64);
+        if (mbar_test(bar, parity)) return true;
+        if (global_ns() - t0 > WAIT_NS) return false;
+    }
+}
+
 // Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
 // from global to shared memory, completing on `bar` (which expects them).
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
@@ -101,6 +125,32 @@ __device__ __forceinline__ void bulk_g2s_nx(uint32_t dst, const void* src, uint3
 __device__ __forceinline__ void cta_range(int64_t units, int64_t& lo, int64_t& hi) {
     lo = units * (int64_t)blockIdx.x / gridDim.x;
     hi = units * (int64_t)(blockIdx.x + 1) / gridDim.x;
+}
+
+// Acquire load / release store of a flag word (gpu scope).
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Wait until *p is non-zero (acquire) and return it; 0 after WAIT_NS.  The
+// poll backs off from 64 ns to 1 us, so many waiting warps stay a light load
+// on the line.
+__device__ __forceinline__ unsigned wait_nonzero(const unsigned* p) {
+    unsigned v = ld_acquire(p);
+    if (v) return v;
+    const uint64_t t0 = global_ns();
+    unsigned ns = 64;
+    while (true) {
+        __nanosleep(ns);
+        if (ns < 1024) ns <<= 1;
+        v = ld_acquire(p);
+        if (v) return v;
+        if (global_ns() - t0 > WAIT_NS) return 0u;
+    }
 }
 
 // Publish `count` units of group g whose partials this thread (thread 0) has

@@ -10,18 +10,17 @@
 // tablas del proveedor": acceptance length = tokens completed per verify step.
 // Uniforms: Philox4x32-10 (Salmon et al., SC'11, section 5).
 //
-// Both verifies stream every logit row once, in chunks of 16 KB: work unit =
-// (sequence, row, chunk), one CTA per SM over a contiguous range of units, a
-// producer warp keeping TMA bulk copies in flight and consumer warps each
-// reducing whole chunks (ring.cuh).  A unit's partial is published with one
-// acquire-release add on its sequence's counter; the warp whose add completes
-// the sequence (no warp waits) reduces the partials in chunk order and
-// decides.  The sampling draw needs the normalisers first, so it is a second
-// kernel over the one row each sequence draws from (launched as a dependent
-// of the scan, so its launch overlaps the scan's tail): one CTA per 4096
-// elements of that row sums its draw weights; the last CTA of the sequence
-// finds the chunk where the inverse CDF crosses t = u' * R and scans it.
-// No probability vector is ever written to memory.
+// Both verifies stream every logit row once, in chunks of 8 KB: work unit =
+// (sequence, row, chunk), one CTA per SM over a contiguous range of units,
+// each warp bringing its own chunks in with TMA bulk copies and reducing them
+// (ring.cuh).  A unit's partial is published with one acquire-release add on
+// its sequence's counter; the warp whose add completes the sequence (no warp
+// waits) reduces the partials in chunk order and decides.  The sampling draw
+// needs the normalisers first; it runs in the same launch: a warp done with
+// its scan units takes draw units of the sequences that have finished (a
+// queue in finishing order), one chunk of the row the sequence draws from
+// each, and the warp completing a sequence's draw units walks the inverse
+// CDF to t = u' * R.  No probability vector is ever written to memory.
 #include "common.cuh"
 #include "ring.cuh"
 #include "workspace.cuh"
@@ -32,13 +31,6 @@
 namespace dfl {
 
 constexpr double LOG2E = 1.4426950408889634;
-
-// Programmatic dependent launch (PTX griddepcontrol): the scan lets its
-// dependent grid launch early; the draw waits for the scan's results.
-__device__ __forceinline__ void pdl_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ------------------------------------------------------------------ greedy
 // One chunk, one warp: the chunk maximum M and the lowest index holding it,
@@ -176,68 +168,53 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_kernel(
     }
 }
 
-// ------------------------------------------------------------------ sampling, pass 1
-// (maximum, fp64 sum of exp2((x - maximum) c)) of rows r0 .. r0+NB-1 from
-// their S chunk partials, warp-collective: lane c takes chunks c, c + 32, ...
-// then fixed butterflies.  With S <= 64 every partial of the NB rows is
-// loaded in one round (kept in registers); longer rows take two passes.
-// Every lane returns the same values.
-template <int NB>
-__device__ __forceinline__ void rows_lse(const LseD* P, int S, int r0, int nrows, float c2,
-                                         float (&Mo)[NB], double (&So)[NB]) {
-    const int lane = threadIdx.x & 31;
-    if (S <= 64) {
-        float m[NB][2];
-        double sv[NB][2];
+// ------------------------------------------------------------------ sampling, the scan
+// (maximum, fp64 sum of exp2((x - maximum) c)) of rows r0 .. r0+7 (the first
+// nrows of them) from their S chunk partials, lane-parallel: lanes 4j .. 4j+3
+// take row r0 + j, lane 4j + s its chunks s, s + 4, ... (the first 4 RC of
+// them held in registers, so a row of up to 4 RC chunks is read once); the
+// maximum, then the fp64 sum against it in chunk order; two butterfly steps
+// within the four lanes.  Every lane of group j returns row r0 + j's pair.
+constexpr int RC = 12;
+__device__ __forceinline__ void rows_lse8(const LseD* P, int S, int r0, int nrows, float c2,
+                                          float& Mo, double& So) {
+    const int lane = threadIdx.x & 31, j = lane >> 2, sub = lane & 3;
+    const bool on = j < nrows;
+    const LseD* p = P + (int64_t)(r0 + (on ? j : 0)) * S;
+    float pm[RC];
+    double ps[RC];
 #pragma unroll
-        for (int j = 0; j < NB; ++j)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int c = lane + 32 * h;
-                m[j][h] = -INFINITY;
-                sv[j][h] = 0.0;
-                if (j < nrows && c < S) {
-                    const LseD* p = &P[(int64_t)(r0 + j) * S + c];
-                    m[j][h] = __ldcg(&p->m);
-                    sv[j][h] = __ldcg(&p->s);
-                }
-            }
-#pragma unroll
-        for (int j = 0; j < NB; ++j) {
-            const float M = warp_max(fmaxf(m[j][0], m[j][1]));
-            double t = 0.0;
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-                if (m[j][h] != -INFINITY) t += sv[j][h] * exp2(((double)m[j][h] - (double)M) * (double)c2);
-            Mo[j] = M;
-            So[j] = warp_sum(t);
+    for (int i = 0; i < RC; ++i) {
+        const int c = sub + 4 * i;
+        pm[i] = -INFINITY;
+        ps[i] = 0.0;
+        if (on && c < S) {
+            pm[i] = __ldcg(&p[c].m);
+            ps[i] = __ldcg(&p[c].s);
         }
-        return;
     }
+    float M = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < NB; ++j) {
-        Mo[j] = -INFINITY;
-        So[j] = 0.0;
-    }
-    for (int c = lane; c < S; c += 32) {
+    for (int i = 0; i < RC; ++i) M = fmaxf(M, pm[i]);
+    if (on)
+        for (int c = sub + 4 * RC; c < S; c += 4) M = fmaxf(M, __ldcg(&p[c].m));
+    M = fmaxf(M, __shfl_xor_sync(FULL, M, 1));
+    M = fmaxf(M, __shfl_xor_sync(FULL, M, 2));
+    double t = 0.0;
+    if (M != -INFINITY) {
 #pragma unroll
-        for (int j = 0; j < NB; ++j)
-            if (j < nrows) Mo[j] = fmaxf(Mo[j], __ldcg(&P[(int64_t)(r0 + j) * S + c].m));
-    }
-#pragma unroll
-    for (int j = 0; j < NB; ++j) Mo[j] = warp_max(Mo[j]);
-    for (int c = lane; c < S; c += 32) {
-#pragma unroll
-        for (int j = 0; j < NB; ++j)
-            if (j < nrows) {
-                const LseD* p = &P[(int64_t)(r0 + j) * S + c];
-                const float pm = __ldcg(&p->m);
-                const double ps = __ldcg(&p->s);
-                if (pm != -INFINITY) So[j] += ps * exp2(((double)pm - (double)Mo[j]) * (double)c2);
+        for (int i = 0; i < RC; ++i)
+            if (pm[i] != -INFINITY) t += ps[i] * exp2(((double)pm[i] - (double)M) * (double)c2);
+        if (on)
+            for (int c = sub + 4 * RC; c < S; c += 4) {
+                const float m = __ldcg(&p[c].m);
+                if (m != -INFINITY) t += __ldcg(&p[c].s) * exp2(((double)m - (double)M) * (double)c2);
             }
     }
-#pragma unroll
-    for (int j = 0; j < NB; ++j) So[j] = warp_sum(So[j]);
+    t += __shfl_xor_sync(FULL, t, 1);
+    t += __shfl_xor_sync(FULL, t, 2);
+    Mo = M;
+    So = t;
 }
 
 // The accept tests of one sequence, by the warp whose unit completed it:
@@ -270,19 +247,24 @@ __device__ __forceinline__ void sample_finish(
         lq.m = q_max[(int64_t)b * G + lane];
         lnq = (double)q_lse[(int64_t)b * G + lane];
     }
-    const int nrows = (q_mode == DFLASH2_Q_SOFTMAX && !given) ? 2 * G + 1 : G + 1;
+    const bool scan_q = q_mode == DFLASH2_Q_SOFTMAX && !given;
+    const int nrows = scan_q ? 2 * G + 1 : G + 1;
     for (int r0 = 0; r0 < nrows; r0 += 8) {
-        float Mr[8];
-        double Sr[8];
-        rows_lse<8>(P, S, r0, min(8, nrows - r0), c2, Mr, Sr);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int rr = r0 + j;
-            if (rr <= G && lane == rr) lt = LseD{Mr[j], 0.0f, Sr[j]};
-            if (rr > G && rr < nrows && lane == rr - G - 1) lq = LseD{Mr[j], 0.0f, Sr[j]};
+        float Mr;
+        double Sr;
+        rows_lse8(P, S, r0, min(8, nrows - r0), c2, Mr, Sr);
+        // lane j takes target row j (and draft row j, row G + 1 + j) from group row - r0
+        const int jt = lane - r0, jq = lane + G + 1 - r0;
+        const float mt_ = __shfl_sync(FULL, Mr, 4 * (jt & 7));
+        const double st_ = __shfl_sync(FULL, Sr, 4 * (jt & 7));
+        if (lane <= G && jt >= 0 && jt < 8) lt = LseD{mt_, 0.0f, st_};
+        if (scan_q) {
+            const float mq_ = __shfl_sync(FULL, Mr, 4 * (jq & 7));
+            const double sq_ = __shfl_sync(FULL, Sr, 4 * (jq & 7));
+            if (lane < G && jq >= 0 && jq < 8) lq = LseD{mq_, 0.0f, sq_};
         }
     }
-    if (q_mode == DFLASH2_Q_SOFTMAX && !given && lane < G) lnq = log(lq.s);
+    if (scan_q && lane < G) lnq = log(lq.s);
     bool reject = false;
     if (lane < G) {
         // lp = z_t[d] - logZ_t = (x - m) * invT - ln(s); likewise lq
@@ -296,7 +278,7 @@ __device__ __forceinline__ void sample_finish(
     }
     const unsigned rej = __ballot_sync(FULL, reject);
     const int n = rej ? (__ffs(rej) - 1) : G;
-    if (lane <= G) out_tok[(int64_t)b * (G + 1) + lane] = (lane < n) ? dn : -1;  // draw fills n
+    if (lane <= G && lane != n) out_tok[(int64_t)b * (G + 1) + lane] = (lane < n) ? dn : -1;
     const float ltm = __shfl_sync(FULL, lt.m, n);
     const double lts = __shfl_sync(FULL, lt.s, n);
     const float lqm = __shfl_sync(FULL, lq.m, n);
@@ -320,29 +302,385 @@ __device__ __forceinline__ void sample_finish(
     }
 }
 
-// Units are (sequence b, row rr, chunk): rows 0..G of a sequence are its
-// target rows, G+1..2G its draft rows (softmax mode only).  A unit's partial
-// is the chunk maximum and the fp64 sum of exp2((x - m) c) against it; a
-// warp publishes its consecutive units of one sequence together.
+// ------------------------------------------------------------------ sampling, the draw
+// A sequence draws from one row (target row n, with draft row n for the
+// residual).  The row is cut into draw units of one chunk (the scan's chunk
+// length, so a unit fills one ring slot), and lane l of the warp that takes
+// a unit owns its vectors NVL l .. NVL l + NVL - 1: a contiguous run of the
+// row in index order.  Per unit the lanes' inclusive prefix sums of their
+// weights are stored (fp64, lane order); units in row order, lanes in unit
+// order and elements in run order give the inverse CDF the draw walks.
+//
+// Draw weight of one element:
+//   p_v = exp2((x_v - mt) * c - l2t),  q_v likewise,
+//   mode 0: w = max(0, p - q).  With d = ln p - ln q = (xt - xq) * invT -
+//           (logZ_t - logZ_q): w = 0 for d <= 0; for 0 < d <= 1/8,
+//           w = q * (e^d - 1) (the same value, without the cancellation of
+//           p - q when p and q agree); above, w = p - q directly (p > 1.13 q:
+//           the subtraction costs at most three bits; q = 0 gives p);
+//   mode 1: w = p, 0 at d;  mode 2: w = p (also the fallback when the
+//   residual is empty by rounding).
+// e^d - 1 for 0 < d <= 1/8: the Taylor series to d^5 (truncation below
+// 5e-8 relative there).
+constexpr float EXPM1_SPLIT = 0.125f;
+__device__ __forceinline__ float expm1_small(float d) {
+    float p = 1.0f / 120.0f;
+    p = fmaf(p, d, 1.0f / 24.0f);
+    p = fmaf(p, d, 1.0f / 6.0f);
+    p = fmaf(p, d, 0.5f);
+    p = fmaf(p, d, 1.0f);
+    return p * d;
+}
+
+// The weights of one 16-byte vector (first element index i0); -inf elements
+// (past the row) weigh 0 in every mode.  RESID: mode 0; else p, with the
+// element at index excl (mode 1's d; -1 for mode 2) weighing 0.
+template <bool BF16, bool RESID>
+__device__ __forceinline__ void draw_vec(const uint4& xt, const uint4& xq, int64_t i0,
+                                         const SampleInfo& I, int64_t excl, float c2, float inv_t,
+                                         float (&w)[ChunkT<BF16>::VW]) {
+    using C = ChunkT<BF16>;
+#pragma unroll
+    for (int e = 0; e < C::VW; ++e) {
+        const float t = C::elem(xt, e);
+        if (RESID) {  // both exponentials always, then selects: no branch per element
+            const float q = C::elem(xq, e);
+            const float dlog = (t - q) * inv_t - I.dl;
+            const float qv = ex2((q - I.mq) * c2 - I.l2q);
+            const float pv = ex2((t - I.mt) * c2 - I.l2t);
+            const float near = qv * expm1_small(fminf(dlog, EXPM1_SPLIT));
+            const float r = (dlog > EXPM1_SPLIT) ? pv - qv : near;
+            w[e] = (dlog > 0.0f) ? r : 0.0f;
+        } else {
+            const float pv = ex2((t - I.mt) * c2 - I.l2t);
+            w[e] = (i0 + e == excl) ? 0.0f : pv;
+        }
+    }
+}
+template <bool BF16>
+__device__ __forceinline__ void draw_vec(int mode, const uint4& xt, const uint4& xq, int64_t i0,
+                                         const SampleInfo& I, float c2, float inv_t,
+                                         float (&w)[ChunkT<BF16>::VW]) {
+    if (mode == 0) draw_vec<BF16, true>(xt, xq, i0, I, -1, c2, inv_t, w);
+    else draw_vec<BF16, false>(xt, xq, i0, I, mode == 1 ? (int64_t)I.d : -1, c2, inv_t, w);
+}
+
+// This lane's weight sum over its run of a unit: fp32 pairwise within a
+// vector, fp64 across the run's vectors.  The lanes of a warp read the run's
+// vectors in rotated order (lane l starts at its vector l mod NVL), so the
+// 16-byte reads of a quarter-warp fall in distinct banks; the order is fixed
+// per lane, so the sum is the same bits in any batch.
+template <bool BF16, bool RESID, class View>
+__device__ __forceinline__ double draw_lane_sum(const View& vt, const View& vq,
+                                                const SampleInfo& I, int64_t excl, float c2,
+                                                float inv_t) {
+    using C = ChunkT<BF16>;
+    const int lane = threadIdx.x & 31;
+    double s = 0.0;
+#pragma unroll 2
+    for (int g = 0; g < NVL; ++g) {
+        const int q = NVL * lane + ((g + lane) & (NVL - 1));
+        const uint4 xt = vt.vec(q);
+        const uint4 xq = RESID ? vq.vec(q) : make_uint4(0u, 0u, 0u, 0u);
+        float w[C::VW];
+        draw_vec<BF16, RESID>(xt, xq, vt.index(q, 0), I, excl, c2, inv_t, w);
+#pragma unroll
+        for (int h = C::VW / 2; h > 0; h >>= 1)
+#pragma unroll
+            for (int e = 0; e < h; ++e) w[e] += w[e + h];
+        s += (double)w[0];
+    }
+    return s;
+}
+template <bool BF16, class View>
+__device__ __forceinline__ double draw_lane_sum(const View& vt, const View& vq, int mode,
+                                                const SampleInfo& I, float c2, float inv_t) {
+    if (mode == 0) return draw_lane_sum<BF16, true>(vt, vq, I, -1, c2, inv_t);
+    return draw_lane_sum<BF16, false>(vt, vq, I, mode == 1 ? (int64_t)I.d : -1, c2, inv_t);
+}
+
+// Inclusive warp scan (fp64, lane order).
+__device__ __forceinline__ double warp_incl_scan(double x) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 1; k < 32; k <<= 1) {
+        const double o = __shfl_up_sync(FULL, x, k);
+        if (lane >= k) x += o;
+    }
+    return x;
+}
+
+// A row read straight from global memory as the vectors of a unit starting
+// at element v0: AL (16-byte aligned rows, V * es a multiple of 16) reads
+// whole vectors, else element by element; elements past V read as -inf.
+template <bool BF16, bool AL>
+struct RowView {
+    using C = ChunkT<BF16>;
+    const char* row;
+    int64_t v0, V;
+    __device__ __forceinline__ uint4 vec(int q) const {
+        const int64_t i0 = v0 + (int64_t)q * C::VW;
+        if (AL && i0 + C::VW <= V) return __ldg((const uint4*)(row + i0 * C::ES));
+        const GlobalView<BF16> g{(const uint8_t*)row, i0,
+                                 (int)max((int64_t)0, min((int64_t)C::VW, V - i0))};
+        return g.vec(0);
+    }
+    __device__ __forceinline__ int64_t index(int q, int e) const { return v0 + (int64_t)q * C::VW + e; }
+};
+
+// The walk inside the run holding t (first element rb, inverse CDF `base`
+// before it): lane j < NVL takes the run's vector j, the vector sums go
+// through an inclusive warp scan, and the first lane with mass whose prefix
+// exceeds t walks its elements to the first whose running prefix exceeds t
+// (else its last element with mass; if no lane crosses, the run's last
+// element with mass).  Returns the element index on every lane (-1: no mass).
+template <bool BF16, bool AL>
+__device__ __forceinline__ int64_t draw_walk(const char* trow, const char* qrow, int64_t V,
+                                             int mode, const SampleInfo& I, float c2, float inv_t,
+                                             int64_t rb, double base, double tt) {
+    using C = ChunkT<BF16>;
+    const int lane = threadIdx.x & 31;
+    float w[C::VW];
+    double sj = 0.0;
+    const int64_t i0 = rb + (int64_t)lane * C::VW;
+    if (lane < NVL) {
+        const RowView<BF16, AL> vt{trow, i0, V}, vq{qrow, i0, V};
+        const uint4 xt = vt.vec(0);
+        const uint4 xq = (mode == 0) ? vq.vec(0) : make_uint4(0u, 0u, 0u, 0u);
+        draw_vec<BF16>(mode, xt, xq, i0, I, c2, inv_t, w);
+#pragma unroll
+        for (int e = 0; e < C::VW; ++e) sj += (double)w[e];
+    } else {
+#pragma unroll
+        for (int e = 0; e < C::VW; ++e) w[e] = 0.0f;
+    }
+    const double incl = warp_incl_scan(sj);
+    const unsigned mass = __ballot_sync(FULL, sj > 0.0);
+    const unsigned cross = __ballot_sync(FULL, base + incl > tt) & mass;
+    if (!mass) return -1;
+    const int src = cross ? __ffs(cross) - 1 : 31 - __clz(mass);
+    int64_t pick = -1;
+    if (lane == src) {
+        double run = base + incl - sj;
+        int first = -1, last = -1;
+#pragma unroll
+        for (int e = 0; e < C::VW; ++e) {
+            if (w[e] > 0.0f) last = e;
+            run += (double)w[e];
+            if (first < 0 && run > tt && cross) first = e;
+        }
+        pick = i0 + (first >= 0 ? first : last);
+    }
+    return __shfl_sync(FULL, pick, src);
+}
+
+// The draw from p_n when the residual is empty by rounding (rare): the warp
+// sums the mode-2 weights of every unit's runs itself, twice (R, then the
+// crossing of t = u' R), and locates the run.  False if the row has no mass.
+template <bool BF16, bool AL>
+__device__ __noinline__ bool draw_locate_p(const char* trow, int64_t V, int ND,
+                                           const SampleInfo& I, float c2, float inv_t,
+                                           int& cstar, int& lstar, double& base, double& tt) {
+    using C = ChunkT<BF16>;
+    double R = 0.0;
+    for (int c = 0; c < ND; ++c) {
+        const RowView<BF16, AL> v{trow, (int64_t)c * C::LEN, V};
+        const double my = draw_lane_sum<BF16>(v, v, 2, I, c2, inv_t);
+        R = __shfl_sync(FULL, warp_incl_scan(my) + R, 31);
+    }
+    if (!(R > 0.0)) return false;
+    tt = (double)I.u_res * R;
+    double carry = 0.0;
+    int lastc = -1, lastl = -1;
+    double last_base = 0.0;
+    for (int c = 0; c < ND; ++c) {
+        const RowView<BF16, AL> v{trow, (int64_t)c * C::LEN, V};
+        const double my = draw_lane_sum<BF16>(v, v, 2, I, c2, inv_t);
+        const double incl = warp_incl_scan(my) + carry;
+        const unsigned mass = __ballot_sync(FULL, my > 0.0);
+        const unsigned cross = __ballot_sync(FULL, incl > tt) & mass;
+        if (cross) {
+            cstar = c;
+            lstar = __ffs(cross) - 1;
+            base = __shfl_sync(FULL, incl - my, lstar);
+            return true;
+        }
+        if (mass) {
+            lastc = c;
+            lastl = 31 - __clz(mass);
+            last_base = __shfl_sync(FULL, incl - my, lastl);
+        }
+        carry = __shfl_sync(FULL, incl, 31);
+    }
+    cstar = lastc;  // rounding left t at or above the total
+    lstar = lastl;
+    base = last_base;
+    return true;
+}
+
+// The pick of one sequence, by the warp whose draw unit completed it.
+// R = the unit totals in unit order (fp64 inclusive scan), t = u' R; the
+// first unit whose inclusive prefix exceeds t, in it the first lane with mass
+// whose prefix exceeds t (from the stored prefixes), then the walk in that
+// lane's run.  R = 0 (the residual empty by rounding) redraws from p_n.
+// Writes out_tok[n] (-1 if the row has no mass at all).
+template <bool BF16, bool AL>
+__device__ __noinline__ void draw_pick(const char* trow, const char* qrow, int64_t V, int ND,
+                                       SampleInfo I, float c2, float inv_t,
+                                       const double* __restrict__ P, int32_t* __restrict__ out) {
+    using C = ChunkT<BF16>;
+    const int lane = threadIdx.x & 31;
+    int mode = I.mode;
+    // the unit totals (each unit's last lane prefix): rows of up to 32 PT
+    // units are loaded once, into registers; longer ones are read per pass
+    constexpr int PT = 4;
+    double tot[PT], incl[PT];
+    double R = 0.0;
+    const bool held = ND <= 32 * PT;
+    if (held) {
+#pragma unroll
+        for (int k = 0; k < PT; ++k) {
+            const int c = 32 * k + lane;
+            tot[k] = (c < ND) ? __ldcg(&P[(int64_t)c * 32 + 31]) : 0.0;
+        }
+#pragma unroll
+        for (int k = 0; k < PT; ++k) {
+            incl[k] = warp_incl_scan(tot[k]) + R;
+            R = __shfl_sync(FULL, incl[k], 31);
+        }
+    } else {
+        for (int c0 = 0; c0 < ND; c0 += 32) {
+            const int c = c0 + lane;
+            const double cs = (c < ND) ? __ldcg(&P[(int64_t)c * 32 + 31]) : 0.0;
+            R = __shfl_sync(FULL, warp_incl_scan(cs) + R, 31);
+        }
+    }
+    int cstar = -1, lstar = -1;
+    double base = 0.0, tt = 0.0;
+    if (R > 0.0) {
+        tt = (double)I.u_res * R;
+        double pre = 0.0, lastc_pre = 0.0;
+        int lastc = -1;
+        // the first unit with mass whose inclusive prefix exceeds t, and the
+        // last unit with mass (for t at or above R by rounding)
+        auto look = [&](int c0, double cs, double in) {
+            const unsigned mass = __ballot_sync(FULL, cs > 0.0);
+            const unsigned cross = __ballot_sync(FULL, in > tt) & mass;
+            if (mass) {
+                const int l = 31 - __clz(mass);
+                lastc = c0 + l;
+                lastc_pre = __shfl_sync(FULL, in - cs, l);
+            }
+            if (cross && cstar < 0) {
+                const int l = __ffs(cross) - 1;
+                cstar = c0 + l;
+                pre = __shfl_sync(FULL, in - cs, l);
+            }
+        };
+        if (held) {
+#pragma unroll
+            for (int k = 0; k < PT; ++k) look(32 * k, tot[k], incl[k]);
+        } else {
+            double carry = 0.0;
+            for (int c0 = 0; c0 < ND && cstar < 0; c0 += 32) {
+                const int c = c0 + lane;
+                const double cs = (c < ND) ? __ldcg(&P[(int64_t)c * 32 + 31]) : 0.0;
+                const double in = warp_incl_scan(cs) + carry;
+                look(c0, cs, in);
+                carry = __shfl_sync(FULL, in, 31);
+            }
+        }
+        if (cstar < 0) {  // rounding left t at or above R: the last unit with mass
+            cstar = lastc;
+            pre = lastc_pre;
+        }
+        const double li = __ldcg(&P[(int64_t)cstar * 32 + lane]);
+        double lp = __shfl_up_sync(FULL, li, 1);
+        if (lane == 0) lp = 0.0;
+        const unsigned mass = __ballot_sync(FULL, li > lp);
+        const unsigned cross = __ballot_sync(FULL, pre + li > tt) & mass;
+        lstar = cross ? __ffs(cross) - 1 : (mass ? 31 - __clz(mass) : -1);
+        if (lstar >= 0) base = pre + __shfl_sync(FULL, lp, lstar);
+    } else {
+        mode = 2;
+        if (!draw_locate_p<BF16, AL>(trow, V, ND, I, c2, inv_t, cstar, lstar, base, tt)) lstar = -1;
+    }
+    int64_t pick = -1;
+    if (lstar >= 0)
+        pick = draw_walk<BF16, AL>(trow, qrow, V, mode, I, c2, inv_t,
+                                   (int64_t)cstar * C::LEN + (int64_t)lstar * NVL * C::VW, base, tt);
+    if (lane == 0) *out = (int32_t)pick;
+}
+
+// The per-sequence hand-over from the scan to the draw, read in L2 (written
+// by another SM in this launch).
+__device__ __forceinline__ SampleInfo load_info(const SampleInfo* p) {
+    SampleInfo I;
+    I.mt = __ldcg(&p->mt);
+    I.l2t = __ldcg(&p->l2t);
+    I.mq = __ldcg(&p->mq);
+    I.l2q = __ldcg(&p->l2q);
+    I.dl = __ldcg(&p->dl);
+    I.u_res = __ldcg(&p->u_res);
+    I.n = __ldcg(&p->n);
+    I.mode = __ldcg(&p->mode);
+    I.d = __ldcg(&p->d);
+    I.pad = 0;
+    return I;
+}
+
+// Sampling verify in one cooperative launch (every CTA resident).
+//
+// Scan: units are (sequence b, row rr, chunk): rows 0..G of a sequence are
+// its target rows, G+1..2G its draft rows (when their normalisers are not
+// given).  A unit's partial is the chunk maximum and the fp64 sum of
+// exp2((x - m) c) against it; a warp publishes its consecutive units of one
+// sequence together, and the warp whose add completes the sequence decides
+// its accept tests and appends it to the finish queue.
+//
+// Draw: draw unit i is (position i / ND in the finish queue, unit i % ND of
+// the row), and CTA c takes units c, c + grid, c + 2 grid, ... in that order
+// (a shared-memory counter hands them to its warps as they run out of scan
+// units), so every SM draws the same share.  A warp waits (bounded) until
+// the sequence at that position has finished, brings the unit of target row
+// n (and draft row n for the residual) into its ring slots, and stores its
+// lanes' prefix sums.  The warp whose unit completes a sequence picks the
+// token.  No warp waits on a warp that is itself waiting: a sequence
+// finishes within the scan, and a warp draws only after its own scan units.
+//
+// Control words (zero on entry, zero again on exit; sample_ctl_words): the
+// queue length and the count of warps done, each in a 128-byte line of its
+// own; scan units per sequence [B]; draw units per sequence [B]; then the
+// finish queue, one line per position (b + 1 of the sequence that finished
+// there), so the warps polling it spread over as many lines and never meet
+// the counters' adds.
 template <bool BF16, bool TMA>
-__global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_scan_kernel(
-    const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int S,
+__global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
+    const void* __restrict__ target, const void* __restrict__ draft, int B, int G, int64_t V, int S,
     int rows_per_seq, int64_t units, float inv_t, float c2, const int32_t* __restrict__ draft_tok,
     uint64_t seed, uint32_t step, const uint32_t* __restrict__ seq_id, int q_mode,
     int32_t* __restrict__ n_accept, int32_t* __restrict__ out_tok, float* __restrict__ ratio_dbg,
-    float* __restrict__ u_dbg, LseD* __restrict__ part, SampleInfo* __restrict__ info,
-    unsigned* __restrict__ counters, const float* __restrict__ q_max,
+    float* __restrict__ u_dbg, LseD* __restrict__ part, double* __restrict__ dsum,
+    SampleInfo* __restrict__ info, unsigned* __restrict__ ctl, const float* __restrict__ q_max,
     const float* __restrict__ q_lse) {
-    constexpr int ES = BF16 ? 2 : 4;
-    constexpr int LEN = chunk_len(ES);
+    using C = ChunkT<BF16>;
+    constexpr int ES = C::ES;
+    constexpr int LEN = C::LEN;
     extern __shared__ __align__(128) uint8_t ring[];
     __shared__ __align__(8) uint64_t bars[2 * NCW];
+    __shared__ unsigned s_next;  // this CTA's next draw unit (k: unit blockIdx.x + k grid)
     const int lane = threadIdx.x & 31;
+    unsigned* const fin_count = ctl;
+    unsigned* const retire = ctl + CTL_LINE;
+    unsigned* const counters = ctl + 2 * CTL_LINE;
+    unsigned* const dcount = counters + B;
+    unsigned* const fin = ctl + sample_fin_off(B);
     auto rowp = [&](int64_t b, int rr) {
         return (rr <= G) ? (const char*)target + (b * (G + 1) + rr) * V * ES
                          : (const char*)draft + (b * G + (rr - G - 1)) * V * ES;
     };
-    pdl_launch_dependents();
+    if (threadIdx.x == 0) s_next = 0u;
+    __syncthreads();
     int64_t lo, hi;
     warp_range(units, lo, hi);
     const int n = (int)(hi - lo);
@@ -355,7 +693,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_scan_kernel(
         bytes = (uint32_t)(min((int64_t)LEN, V - v0) * ES);
     };
     WarpRing r{nullptr, 0u};
-    if (TMA) r = warp_ring_start(ring, bars, n, ic, ChunkT<BF16>::NEG_INF_WORD, src);
+    if (TMA) r = warp_ring_start(ring, bars, n, ic, C::NEG_INF_WORD, src);
     unsigned seg = 0;
     for (int k = 0; k < n; ++k, uc.next()) {
         const int64_t b = uc.g, v0 = (int64_t)uc.c * LEN;
@@ -371,7 +709,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_scan_kernel(
             uint32_t vm[NVL];
             M = warp_max(chunk_pass1<BF16>(view, vm));
             Ssum = chunk_expsum<BF16>(view, M, c2);
-            warp_ring_next(r, k, n, ic, ChunkT<BF16>::NEG_INF_WORD, src);
+            warp_ring_next(r, k, n, ic, C::NEG_INF_WORD, src);
         } else {
             const GlobalView<BF16> view{(const uint8_t*)rowp(b, uc.r), v0, len};
             uint32_t vm[NVL];
@@ -388,332 +726,84 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_scan_kernel(
                 sample_finish(target, draft, part + b * rows_per_seq * S, G, V, S, ES, inv_t, c2,
                               draft_tok, seed, step, seq_id ? seq_id[b] : (uint32_t)b, q_mode,
                               (int)b, n_accept, out_tok, ratio_dbg, u_dbg, info, q_max, q_lse);
-                if (lane == 0) counters[b] = 0u;  // the sequence is done: leave its counter zero
+                if (lane == 0) {  // info[b] (lane 0's store) before the queue entry
+                    counters[b] = 0u;
+                    st_release(&fin[(size_t)atomicAdd(fin_count, 1u) * CTL_LINE], (unsigned)b + 1u);
+                }
             }
             seg = 0;
         }
     }
-}
 
-// ------------------------------------------------------------------ sampling, pass 2
-// Draw weight of one element of the row the sequence draws from (draw_w):
-//   p_v = exp2((x_v - mt) * c - l2t),  q_v likewise,
-//   mode 0: w = max(0, p - q), evaluated as q * expm1(ln p - ln q) with
-//           ln p - ln q = (xt - xq) * invT - (logZ_t - logZ_q): the same
-//           value, without the cancellation of p - q when p and q agree;
-//   mode 1: w = p, 0 at d;  mode 2: w = p (also the fallback when the
-//   residual is empty by rounding).
-// e^d - 1 for d > 0: the Taylor series to d^8 for d <= 1/2 (truncation below
-// 6e-9 relative there), e^d - 1 from exp2 above, where the subtraction costs
-// at most two bits.
-__device__ __forceinline__ float expm1_pos(float d) {
-    if (d > 0.5f) return ex2(d * 1.4426950408889634f) - 1.0f;
-    float p = 1.0f / 40320.0f;
-    p = fmaf(p, d, 1.0f / 5040.0f);
-    p = fmaf(p, d, 1.0f / 720.0f);
-    p = fmaf(p, d, 1.0f / 120.0f);
-    p = fmaf(p, d, 1.0f / 24.0f);
-    p = fmaf(p, d, 1.0f / 6.0f);
-    p = fmaf(p, d, 0.5f);
-    p = fmaf(p, d, 1.0f);
-    return p * d;
-}
-
-// The draw of one sequence covers DLEN elements per CTA of the row it draws
-// from; thread t holds DEPT consecutive elements.  A thread's sum: fp32 over a
-// 16-byte vector (index order, pairwise), fp64 across vectors.
-constexpr int DLEN = DRAW_LEN;
-constexpr int DT = 256;
-constexpr int DEPT = DLEN / DT;  // 40: 5 bf16 / 10 fp32 vectors
-// CTAs per row the draw handles (their sums sit in shared memory): V <= 3072 * 10240.
-constexpr int64_t DRAW_MAX_CHUNKS = 3072;
-
-// The draw weight of one element (mode 0: residual, 1: p without d, 2: p;
-// the residual-empty fallback draws with mode 2).  The mode is the same for
-// a whole CTA, so the branch is uniform.
-// off: the element's offset in the thread's run, d_off: the offset of d
-// there (anything outside [0, DEPT) when d is not in the run).
-__device__ __forceinline__ float draw_w(int mode, float xt, float xq, int off, int64_t d_off,
-                                        const SampleInfo& I, float c2, float inv_t) {
-    if (mode == 0) {
-        const float dlog = (xt - xq) * inv_t - I.dl;
-        if (!(dlog > 0.0f)) return 0.0f;
-        return ex2((xq - I.mq) * c2 - I.l2q) * expm1_pos(dlog);
-    }
-    if (mode == 1 && (int64_t)off == d_off) return 0.0f;
-    return ex2((xt - I.mt) * c2 - I.l2t);
-}
-
-// The DEPT elements [vb, vb + DEPT) of a row as 16-byte vectors (-inf past V).
-template <bool BF16, bool VEC>
-__device__ __forceinline__ void draw_load(const char* row, int64_t vb, int64_t V,
-                                          uint4 (&x)[DEPT / ChunkT<BF16>::VW]) {
-    using C = ChunkT<BF16>;
-    constexpr int NV = DEPT / C::VW;
-    if (VEC && vb + DEPT <= V) {
-        const uint4* p = (const uint4*)(row + vb * C::ES);
-#pragma unroll
-        for (int g = 0; g < NV; ++g) x[g] = __ldg(p + g);
-    } else {
-        const GlobalView<BF16> view{(const uint8_t*)row, vb,
-                                    (int)max((int64_t)0, min((int64_t)DEPT, V - vb))};
-#pragma unroll
-        for (int g = 0; g < NV; ++g) x[g] = view.vec(g);
-    }
-}
-
-// A thread's weights over its DEPT elements and their sum (fp32 pairwise
-// within a 16-byte vector, fp64 across vectors); w may be null.
-template <bool BF16, bool VEC>
-__device__ __forceinline__ double draw_thread(const char* trow, const char* qrow, int64_t vb,
-                                              int64_t V, int mode, const SampleInfo& I, float c2,
-                                              float inv_t, float* w) {
-    using C = ChunkT<BF16>;
-    constexpr int NV = DEPT / C::VW;
-    uint4 xt[NV], xq[NV];
-    draw_load<BF16, VEC>(trow, vb, V, xt);
-    if (mode == 0) draw_load<BF16, VEC>(qrow, vb, V, xq);
-    const int64_t d_off = (int64_t)I.d - vb;
-    double s = 0.0;
-#pragma unroll
-    for (int g = 0; g < NV; ++g) {
-        float sv[C::VW];
-#pragma unroll
-        for (int e = 0; e < C::VW; ++e) {
-            sv[e] = draw_w(mode, C::elem(xt[g], e), mode == 0 ? C::elem(xq[g], e) : 0.0f,
-                           g * C::VW + e, d_off, I, c2, inv_t);
-            if (w) w[g * C::VW + e] = sv[e];
+    // ---- the draw
+    const int ND = S;  // draw units per row
+    const unsigned total = (unsigned)B * (unsigned)ND;
+    int kk = n;  // this warp's next ring unit
+    while (true) {
+        unsigned k = 0;
+        if (lane == 0) k = atomicAdd(&s_next, 1u);
+        k = __shfl_sync(FULL, k, 0);
+        const uint64_t i64 = (uint64_t)blockIdx.x + (uint64_t)k * gridDim.x;
+        if (i64 >= total) break;
+        const unsigned i = (unsigned)i64;
+        const unsigned pos = i / (unsigned)ND, c = i - pos * (unsigned)ND;
+        unsigned b1 = 0;
+        if (lane == 0) b1 = wait_nonzero(&fin[(size_t)pos * CTL_LINE]);
+        b1 = __shfl_sync(FULL, b1, 0);
+        if (b1 == 0u) {  // the bound ran out
+            if (lane == 0) atomicOr(&g_dev_err, ERR_STREAM);
+            return;
         }
-#pragma unroll
-        for (int h = C::VW / 2; h > 0; h >>= 1)
-#pragma unroll
-            for (int e = 0; e < h; ++e) sv[e] += sv[e + h];
-        s += (double)sv[0];
-    }
-    return s;
-}
-
-// Inclusive scan of the threads' values in thread order (fp64): warp scans,
-// then the warps' totals in warp order.  `total` is the last thread's value,
-// bit for bit.  Block-wide (two barriers).
-__device__ __forceinline__ double block_incl_scan(double x, double* s_warp, double& total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    double incl = x;
-#pragma unroll
-    for (int k = 1; k < 32; k <<= 1) {
-        const double o = __shfl_up_sync(FULL, incl, k);
-        if (lane >= k) incl += o;
-    }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    double base = 0.0;
-    for (int w = 0; w < warp; ++w) base += s_warp[w];
-    double tot = 0.0;
-    for (int w = 0; w < DT / 32 - 1; ++w) tot += s_warp[w];
-    total = tot + s_warp[DT / 32 - 1];
-    __syncthreads();
-    return base + incl;
-}
-
-// Draw, part 1: grid (chunks of the drawn row, sequences).  Every thread's
-// inclusive prefix within the chunk is stored (dsum[b][c][t]); the last one
-// is the chunk's sum.
-template <bool BF16, bool VEC>
-__global__ void __launch_bounds__(DT) verify_sample_draw_kernel(
-    const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int D,
-    float c2, float inv_t, const SampleInfo* __restrict__ info, double* __restrict__ dsum) {
-    constexpr int ES = BF16 ? 2 : 4;
-    __shared__ double s_warp[DT / 32];
-    const int c = blockIdx.x, b = blockIdx.y;
-    pdl_wait();  // the scan's SampleInfo, and every earlier write, are visible
-    pdl_launch_dependents();
-    const SampleInfo I = info[b];
-    const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
-    const char* qrow = (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
-    const double my = draw_thread<BF16, VEC>(trow, qrow, (int64_t)c * DLEN + (int64_t)DEPT * threadIdx.x,
-                                             V, I.mode, I, c2, inv_t, nullptr);
-    double total;
-    const double incl = block_incl_scan(my, s_warp, total);
-    dsum[((int64_t)b * D + c) * DT + threadIdx.x] = incl;
-}
-
-// The draw when the residual is empty by rounding: from p_n.  Two passes
-// over the row, chunk by chunk, the lanes taking part-1 threads 32 j + lane:
-// the thread sums in one inclusive scan (lane order within a group of 32,
-// groups and chunks in order), whose last value is R; then the same scan
-// against t = u' R, and the crossing thread walks its own elements.  Rare,
-// so kept out of line (the pick's common path stays small).  Returns the
-// element offset within the run starting at vb (lane 0; -1 if none).
-template <bool BF16, bool VEC>
-__device__ __noinline__ int draw_fallback(const char* trow, const char* qrow, int64_t V, int D,
-                                          const SampleInfo& I, float c2, float inv_t, int64_t& vb) {
-    const int lane = threadIdx.x & 31;
-    const int mode = 2;
-    int pick = -1;
-    auto scan_pass = [&](bool find, double tcut, int& cc_hit, int& t_hit, double& base) {
-        double acc = 0.0;
-        for (int cc = 0; cc < D; ++cc)
-            for (int j = 0; j < DT / 32; ++j) {
-                const int t = 32 * j + lane;
-                const double ts = draw_thread<BF16, VEC>(
-                    trow, qrow, (int64_t)cc * DLEN + (int64_t)DEPT * t, V, mode, I, c2, inv_t,
-                    nullptr);
-                double incl = ts;
-#pragma unroll
-                for (int k = 1; k < 32; k <<= 1) {
-                    const double o = __shfl_up_sync(FULL, incl, k);
-                    if (lane >= k) incl += o;
-                }
-                incl += acc;
-                if (find) {
-                    const unsigned cross = __ballot_sync(FULL, incl > tcut);
-                    if (cross) {
-                        const int l = __ffs(cross) - 1;
-                        cc_hit = cc;
-                        t_hit = 32 * j + l;
-                        base = __shfl_sync(FULL, incl - ts, l);
-                        return acc;
-                    }
-                }
-                acc = __shfl_sync(FULL, incl, 31);
+        __syncwarp();  // lane 0's acquire covers the warp's reads of info[b]
+        const int b = (int)b1 - 1;
+        const SampleInfo I = load_info(&info[b]);
+        const int64_t v0 = (int64_t)c * LEN;
+        const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
+        const char* qrow =
+            (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
+        double my;
+        if (TMA) {
+            const int nu = (I.mode == 0) ? 2 : 1;
+            const uint32_t bytes = (uint32_t)(min((int64_t)LEN, V - v0) * ES);
+            warp_ring_load(r, kk, trow + v0 * ES, bytes, C::NEG_INF_WORD);
+            if (nu == 2) warp_ring_load(r, kk + 1, qrow + v0 * ES, bytes, C::NEG_INF_WORD);
+            __syncwarp();
+            bool ok = r.wait_fresh(kk);
+            if (nu == 2) ok = r.wait_fresh(kk + 1) && ok;
+            if (!ok) {
+                warp_ring_abort(r, kk, kk + nu);
+                return;
             }
-        return acc;
-    };
-    int cc_hit = -1, t_hit = -1;
-    double base = 0.0;
-    const double R = scan_pass(false, 0.0, cc_hit, t_hit, base);
-    const double tt = (double)I.u_res * R;
-    scan_pass(true, tt, cc_hit, t_hit, base);
-    if (cc_hit >= 0 && lane == 0) {
-        float w[DEPT];
-        vb = (int64_t)cc_hit * DLEN + (int64_t)DEPT * t_hit;
-        draw_thread<BF16, VEC>(trow, qrow, vb, V, mode, I, c2, inv_t, w);
-        double run = base;
-        int lm = -1;
-        for (int e = 0; e < DEPT; ++e) {
-            if (w[e] > 0.0f) lm = e;
-            run += (double)w[e];
-            if (pick < 0 && run > tt) pick = e;
+            const SmemView<BF16> vt{r.slot(kk), v0, LEN}, vq{r.slot(kk + 1), v0, LEN};
+            my = draw_lane_sum<BF16>(vt, vq, I.mode, I, c2, inv_t);
+            r.done(kk);  // both slots read: they may be refilled
+            kk += nu;
+        } else {
+            const RowView<BF16, false> vt{trow, v0, V}, vq{qrow, v0, V};
+            my = draw_lane_sum<BF16>(vt, vq, I.mode, I, c2, inv_t);
         }
-        if (pick < 0) pick = lm;
-    }
-    return pick;
-}
-
-// Draw, part 2: one warp per sequence.  R = the chunk sums in chunk order,
-// t = u' R; in the first chunk whose inclusive prefix exceeds t, the first
-// thread of part 1 whose inclusive prefix exceeds t (from the stored
-// prefixes) recomputes its weights and walks them to the first element whose
-// running prefix exceeds t (else, rounding, the last element with mass).  If
-// the residual is empty by rounding (R = 0) the draw is redone from p_n by
-// this warp (rare, slow).
-template <bool BF16, bool VEC>
-__global__ void __launch_bounds__(32) verify_sample_pick_kernel(
-    const void* __restrict__ target, const void* __restrict__ draft, int G, int64_t V, int D,
-    float c2, float inv_t, const SampleInfo* __restrict__ info, const double* __restrict__ dsum,
-    int32_t* __restrict__ out_tok) {
-    constexpr int ES = BF16 ? 2 : 4;
-    const int lane = threadIdx.x, b = blockIdx.x;
-    pdl_wait();  // part 1's prefixes
-    const SampleInfo I = info[b];
-    const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
-    const char* qrow = (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
-    const double* P = dsum + (int64_t)b * D * DT;
-    // The chunk sums, loaded together, in an inclusive warp scan (fixed
-    // order; R is its last value); carried across groups of 32 chunks.
-    double carry = 0.0, tt = 0.0, pre = 0.0;
-    int cstar = -1, lastc = -1;
-    double lastc_pre = 0.0;
-    int mode = I.mode;
-    {
-        double R = 0.0;
-        for (int c0 = 0; c0 < D; c0 += 32) {
-            const int cc = c0 + lane;
-            const double cs = (cc < D) ? __ldcg(&P[(int64_t)cc * DT + DT - 1]) : 0.0;
-            double incl = cs;
-#pragma unroll
-            for (int k = 1; k < 32; k <<= 1) {
-                const double o = __shfl_up_sync(FULL, incl, k);
-                if (lane >= k) incl += o;
-            }
-            incl += carry;
-            carry = __shfl_sync(FULL, incl, 31);
-        }
-        R = carry;
-        if (!(R > 0.0)) mode = 2;  // residual empty by rounding: draw from p_n (rare)
-        tt = (double)I.u_res * R;
-        carry = 0.0;
-        for (int c0 = 0; c0 < D && cstar < 0; c0 += 32) {  // the same scan again, now against t
-            const int cc = c0 + lane;
-            const double cs = (cc < D) ? __ldcg(&P[(int64_t)cc * DT + DT - 1]) : 0.0;
-            double incl = cs;
-#pragma unroll
-            for (int k = 1; k < 32; k <<= 1) {
-                const double o = __shfl_up_sync(FULL, incl, k);
-                if (lane >= k) incl += o;
-            }
-            incl += carry;
-            const unsigned cross = __ballot_sync(FULL, cc < D && incl > tt);
-            const unsigned mass = __ballot_sync(FULL, cc < D && cs > 0.0);
-            if (mass) {
-                const int l = 31 - __clz(mass);
-                lastc = c0 + l;
-                lastc_pre = __shfl_sync(FULL, incl - cs, l);
-            }
-            if (cross) {
-                const int l = __ffs(cross) - 1;
-                cstar = c0 + l;
-                pre = __shfl_sync(FULL, incl - cs, l);
-            }
-            carry = __shfl_sync(FULL, incl, 31);
-        }
-        if (cstar < 0) {  // unreachable while R > 0: the last chunk with mass
-            cstar = max(lastc, 0);
-            pre = lastc >= 0 ? lastc_pre : 0.0;
+        dsum[((int64_t)b * ND + c) * 32 + lane] = warp_incl_scan(my);
+        __syncwarp();  // every lane's prefix before lane 0's release
+        bool lastu = false;
+        if (lane == 0) lastu = publish(&dcount[b], 1u, (unsigned)ND);
+        if (__shfl_sync(FULL, lastu, 0)) {
+            __syncwarp();
+            draw_pick<BF16, TMA>(trow, qrow, V, ND, I, c2, inv_t, dsum + (int64_t)b * ND * 32,
+                                 &out_tok[(int64_t)b * (G + 1) + I.n]);
+            if (lane == 0) dcount[b] = 0u;
         }
     }
-    int pick = -1;
-    int64_t vb = 0;
-    if (mode == I.mode) {
-        // the first thread of chunk cstar whose inclusive prefix exceeds t;
-        // all 256 prefixes loaded in one round
-        const double* Q = P + (int64_t)cstar * DT;
-        double incl[DT / 32], prev[DT / 32];
-#pragma unroll
-        for (int j = 0; j < DT / 32; ++j) {
-            const int t = 32 * j + lane;
-            incl[j] = __ldcg(&Q[t]);
-            prev[j] = (t > 0) ? __ldcg(&Q[t - 1]) : 0.0;
+    // the last warp out leaves the queue words zero (every other warp is past
+    // its last access to them)
+    bool lastw = false;
+    if (lane == 0) lastw = publish(retire, 1u, gridDim.x * (unsigned)NCW);
+    if (__shfl_sync(FULL, lastw, 0)) {
+        for (int p = lane; p < B; p += 32) fin[(size_t)p * CTL_LINE] = 0u;
+        if (lane == 0) {
+            *fin_count = 0u;
+            *retire = 0u;
         }
-        int pt = DT, lastm = -1;
-#pragma unroll
-        for (int j = DT / 32 - 1; j >= 0; --j) {
-            const unsigned cross = __ballot_sync(FULL, pre + incl[j] > tt);
-            const unsigned mass = __ballot_sync(FULL, incl[j] > prev[j]);
-            if (cross) pt = 32 * j + __ffs(cross) - 1;
-            if (mass && lastm < 0) lastm = 32 * j + 31 - __clz(mass);
-        }
-        if (pt == DT) pt = lastm;  // rounding left t above the chunk's scan
-        if (pt >= 0) {
-            vb = (int64_t)cstar * DLEN + (int64_t)DEPT * pt;
-            const double base = pre + (pt > 0 ? __ldcg(&Q[pt - 1]) : 0.0);
-            if (lane == 0) {
-                float w[DEPT];
-                draw_thread<BF16, VEC>(trow, qrow, vb, V, mode, I, c2, inv_t, w);
-                double run = base;
-                int lm = -1;
-                for (int e = 0; e < DEPT; ++e) {
-                    if (w[e] > 0.0f) lm = e;
-                    run += (double)w[e];
-                    if (pick < 0 && run > tt) pick = e;
-                }
-                if (pick < 0) pick = lm;
-            }
-        }
-    } else {
-        pick = draw_fallback<BF16, VEC>(trow, qrow, V, D, I, c2, inv_t, vb);
     }
-    if (lane == 0 && pick >= 0) out_tok[(int64_t)b * (G + 1) + I.n] = (int32_t)(vb + pick);
 }
 
 }  // namespace dfl
@@ -730,28 +820,6 @@ unsigned dfl_errors_verify(int clear) {
     }
     return v;
 }
-
-// Launch as a programmatic dependent of the previous kernel on the stream:
-// the grid may start while that kernel finishes, and waits (griddepcontrol)
-// for its results before reading them.
-template <class Kern, class... Args>
-static cudaError_t launch_dependent(Kern kern, dim3 grid, dim3 block, size_t dyn, cudaStream_t s,
-                                    Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = dyn;
-    cfg.stream = s;
-    cudaLaunchAttribute a[1];
-    a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    a[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = a;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, args...);
-}
-
-// Draw grid size per sequence: DLEN-element chunks of the drawn row.
-static inline int64_t draw_chunks(int64_t V) { return (V + DLEN - 1) / DLEN; }
 
 extern "C" int dflash2_verify_greedy(const void* target, int dtype, int B, int G, int64_t V,
                                      const int32_t* draft_tok, int32_t* n_accept, int32_t* out_tok,
@@ -817,8 +885,6 @@ static int verify_sample_impl(const void* target, const void* draft, int dtype, 
         (ratio_dbg && !aligned(ratio_dbg, 4)) || (u_dbg && !aligned(u_dbg, 4)))
         return DFLASH2_EALIGN;
     const int64_t S = row_chunks(V, es);
-    const int64_t D = draw_chunks(V);
-    if (D > DRAW_MAX_CHUNKS) return DFLASH2_ESHAPE;
     // draft rows are scanned only when their normalisers are not given
     const int rows_per_seq = (q_mode == DFLASH2_Q_SOFTMAX && !q_max) ? 2 * G + 1 : G + 1;
     const int64_t units = (int64_t)B * rows_per_seq * S;
@@ -826,43 +892,44 @@ static int verify_sample_impl(const void* target, const void* draft, int dtype, 
     const Layout L = sample_layout(B, G, V, es);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return DFLASH2_EWORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
-    unsigned* counters = (unsigned*)((char*)ws + L.counters_off);  // [B] scan
+    unsigned* ctl = (unsigned*)((char*)ws + L.counters_off);  // sample_ctl_words(B)
     LseD* part = (LseD*)((char*)ws + L.part_off);
     double* dsum = (double*)((char*)ws + L.part2_off);
     SampleInfo* info = (SampleInfo*)((char*)ws + L.info_off);
-    if (!L.self_clean && cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess)
+    if (!L.self_clean && cudaMemsetAsync(ctl, 0, L.counters_bytes, s) != cudaSuccess)
         return DFLASH2_ECUDA;
     const void* q = (q_mode == DFLASH2_Q_SOFTMAX) ? draft : nullptr;
     const bool tma = aligned(target, 16) && (!q || aligned(q, 16)) && (V * es) % 16 == 0;
     const float c2 = (float)((double)inv_temperature * LOG2E);
-#define DFL_SAMPLE(BF, TM)                                                                        \
-    do {                                                                                          \
-        auto kern = verify_sample_scan_kernel<BF, TM>;                                            \
-        const size_t dyn = TM ? (size_t)RING_BYTES : 0;                                           \
-        if (ring_prepare(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;                          \
-        kern<<<ring_grid(units), RING_THREADS, dyn, s>>>(                                         \
-            target, q, G, V, (int)S, rows_per_seq, units, inv_temperature, c2, draft_tok, seed,   \
-            step, seq_id, q_mode, n_accept, out_tok, ratio_dbg, u_dbg, part, info, counters,      \
-            q_max, q_lse);                                                                        \
-        auto kern2 = verify_sample_draw_kernel<BF, TM>;                                           \
-        if (launch_dependent(kern2, dim3((unsigned)D, (unsigned)B), dim3(DT), 0, s, target, q, G, \
-                             V, (int)D, c2, inv_temperature, (const SampleInfo*)info, dsum) !=    \
-            cudaSuccess)                                                                          \
-            return DFLASH2_ECUDA;                                                                 \
-        auto kern3 = verify_sample_pick_kernel<BF, TM>;                                           \
-        if (launch_dependent(kern3, dim3((unsigned)B), dim3(32), 0, s, target, q, G, V, (int)D,    \
-                             c2, inv_temperature, (const SampleInfo*)info, (const double*)dsum,   \
-                             out_tok) != cudaSuccess)                                             \
-            return DFLASH2_ECUDA;                                                                 \
-    } while (0)
-    if (dtype == DFLASH2_BF16) {
-        if (tma) DFL_SAMPLE(true, true);
-        else DFL_SAMPLE(true, false);
-    } else {
-        if (tma) DFL_SAMPLE(false, true);
-        else DFL_SAMPLE(false, false);
-    }
-#undef DFL_SAMPLE
+    // cooperative: every CTA is resident, so a warp's bounded wait for a
+    // sequence to finish waits on warps that are running
+    auto launch = [&](auto kern, size_t dyn) -> int {
+        if (ring_prepare(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)ring_grid(units));
+        cfg.blockDim = dim3(RING_THREADS);
+        cfg.dynamicSmemBytes = dyn;
+        cfg.stream = s;
+        cudaLaunchAttribute a[1];
+        a[0].id = cudaLaunchAttributeCooperative;
+        a[0].val.cooperative = 1;
+        cfg.attrs = a;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, target, q, B, G, V, (int)S, rows_per_seq, units,
+                               inv_temperature, c2, draft_tok, seed, step, seq_id, q_mode,
+                               n_accept, out_tok, ratio_dbg, u_dbg, part, dsum, info, ctl, q_max,
+                               q_lse) != cudaSuccess)
+            return DFLASH2_ECUDA;
+        return DFLASH2_OK;
+    };
+    int rc;
+    if (dtype == DFLASH2_BF16)
+        rc = tma ? launch(verify_sample_kernel<true, true>, RING_BYTES)
+                 : launch(verify_sample_kernel<true, false>, 0);
+    else
+        rc = tma ? launch(verify_sample_kernel<false, true>, RING_BYTES)
+                 : launch(verify_sample_kernel<false, false>, 0);
+    if (rc != DFLASH2_OK) return rc;
     return launch_status();
 }
 

@@ -233,8 +233,10 @@ DFLASH2_API int dflash2_verify_greedy(const void* target, int dtype, int B, int 
  * for u_j, 1 for u' (position = n).
  *
  * target [B, G+1, V], draft [B, G, V] of `dtype`, rows 16-byte aligned for
- * the fast path; V <= 31,457,280 (3072 draw chunks of 10240; DFLASH2_ESHAPE
- * above); draft_tok [B, G] int32; seq_id [B] uint32 or NULL (= b).
+ * the fast path; B <= 65535 and B * (2G+1) * ceil(V / L) < 2^31 (L = 4096
+ * for bf16, 2048 for fp32; DFLASH2_ESHAPE otherwise); draft_tok [B, G]
+ * int32; seq_id [B] uint32 or NULL (= b).  One cooperative launch (every
+ * CTA resident; DFLASH2_ECUDA if the device cannot hold the grid).
  * n_accept [B], out_tok [B, G+1] as in dflash2_verify_greedy.
  * ratio_dbg [B, G] float r_j for every j, u_dbg [B, G] float u_j; both
  * optional (NULL).
