@@ -127,6 +127,11 @@ __device__ __forceinline__ void cta_range(int64_t units, int64_t& lo, int64_t& h
     hi = units * (int64_t)(blockIdx.x + 1) / gridDim.x;
 }
 
+// Prefetch the line holding p into L2, to be kept over streamed data.
+__device__ __forceinline__ void prefetch_l2_last(const void* p) {
+    asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
+}
+
 // Acquire load / release store of a flag word (gpu scope).
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
     unsigned v;

@@ -523,7 +523,8 @@ __device__ __noinline__ bool draw_locate_p(const char* trow, int64_t V, int ND,
 // first unit whose inclusive prefix exceeds t, in it the first lane with mass
 // whose prefix exceeds t (from the stored prefixes), then the walk in that
 // lane's run.  R = 0 (the residual empty by rounding) redraws from p_n.
-// Writes out_tok[n] (-1 if the row has no mass at all).
+// Writes out_tok[n] (-1 if the row has no mass at all; nothing if out is
+// null).
 template <bool BF16, bool AL>
 __device__ __noinline__ void draw_pick(const char* trow, const char* qrow, int64_t V, int ND,
                                        SampleInfo I, float c2, float inv_t,
@@ -609,7 +610,31 @@ __device__ __noinline__ void draw_pick(const char* trow, const char* qrow, int64
     if (lstar >= 0)
         pick = draw_walk<BF16, AL>(trow, qrow, V, mode, I, c2, inv_t,
                                    (int64_t)cstar * C::LEN + (int64_t)lstar * NVL * C::VW, base, tt);
-    if (lane == 0) *out = (int32_t)pick;
+    if (lane == 0 && out) *out = (int32_t)pick;
+}
+
+// One pick on a scratch table of 32 lane prefixes 1 .. 32 (one unit, target
+// row 0 for both rows, a residual of zero mass), and with rings one draw sum
+// over the warp's slots: the same code as the real ones, run early by an
+// idle warp so it is fetched into L2 while no pick waits on it.  Writes only
+// the scratch table; reads only row 0 and the warp's own slots.
+template <bool BF16, bool TMA>
+__device__ __noinline__ void warm_draw_code(const void* target, int64_t V, float c2, float inv_t,
+                                            double* scratch, WarpRing r) {
+    const int lane = threadIdx.x & 31;
+    SampleInfo I;
+    I.mt = I.l2t = I.mq = I.l2q = I.dl = 0.0f;
+    I.u_res = 0.5f;
+    I.n = I.mode = I.d = I.pad = 0;
+    double my = 0.0;
+    if (TMA) {
+        const SmemView<BF16> v{r.slot(0), 0, ChunkT<BF16>::LEN};
+        my = draw_lane_sum<BF16, true>(v, v, I, -1, c2, inv_t);
+    }
+    scratch[lane] = (double)(lane + 1) + 0.0 * my;
+    __syncwarp();
+    draw_pick<BF16, TMA>((const char*)target, (const char*)target, V, 1, I, c2, inv_t, scratch,
+                         nullptr);
 }
 
 // The per-sequence hand-over from the scan to the draw, read in L2 (written
@@ -680,6 +705,18 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
                          : (const char*)draft + (b * G + (rr - G - 1)) * V * ES;
     };
     if (threadIdx.x == 0) s_next = 0u;
+    {  // the accept tests' scattered reads (drafted tokens, their logits) into L2 now
+        const int64_t t = (int64_t)blockIdx.x * RING_THREADS + threadIdx.x;
+        if (t < (int64_t)B * G) {
+            const int64_t b = t / G, j = t - b * G;
+            const int32_t d = draft_tok[t];
+            if (d >= 0 && d < V) {
+                prefetch_l2_last((const char*)target + ((b * (G + 1) + j) * V + d) * ES);
+                if (q_mode == DFLASH2_Q_SOFTMAX)
+                    prefetch_l2_last((const char*)draft + ((b * G + j) * V + d) * ES);
+            }
+        }
+    }
     __syncthreads();
     int64_t lo, hi;
     warp_range(units, lo, hi);
@@ -738,13 +775,21 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
     // ---- the draw
     const int ND = S;  // draw units per row
     const unsigned total = (unsigned)B * (unsigned)ND;
+    double* const dsum_scratch = dsum + (int64_t)B * ND * 32;  // 32 doubles
     int kk = n;  // this warp's next ring unit
     while (true) {
         unsigned k = 0;
         if (lane == 0) k = atomicAdd(&s_next, 1u);
         k = __shfl_sync(FULL, k, 0);
         const uint64_t i64 = (uint64_t)blockIdx.x + (uint64_t)k * gridDim.x;
-        if (i64 >= total) break;
+        if (i64 >= total) {
+            // the first warp of CTA 0 with no unit left runs the pick (and,
+            // with rings, the draw sum) once on scratch, writing nothing, so
+            // their code is in L2 before the real picks need it
+            if (blockIdx.x == 0 && k == (total + gridDim.x - 1) / gridDim.x)
+                warm_draw_code<BF16, TMA>(target, V, c2, inv_t, dsum_scratch, r);
+            break;
+        }
         const unsigned i = (unsigned)i64;
         const unsigned pos = i / (unsigned)ND, c = i - pos * (unsigned)ND;
         unsigned b1 = 0;

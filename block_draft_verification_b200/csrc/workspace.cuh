@@ -85,7 +85,7 @@ inline Layout greedy_layout(int B, int G, int64_t V, int es) {
 // Sampling: the control words (two queue words, a line each; scan and draw
 // counters [B] each; the finish queue, a line per position), the scan's
 // per-unit partials, the draw's per-unit lane prefixes (32 per chunk of the
-// drawn row) and the per-sequence hand-over to the draw.
+// drawn row, and 32 of scratch) and the per-sequence hand-over to the draw.
 constexpr int CTL_LINE = 32;  // words in a 128-byte line
 __host__ __device__ inline size_t sample_fin_off(int B) {
     return (2 * (size_t)CTL_LINE + 2 * (size_t)B + CTL_LINE - 1) / CTL_LINE * CTL_LINE;
@@ -94,7 +94,7 @@ inline size_t sample_ctl_words(int B) { return sample_fin_off(B) + (size_t)B * C
 inline Layout sample_layout(int B, int G, int64_t V, int es) {
     const int64_t S = row_chunks(V, es);
     return make_layout(sample_ctl_words(B) * 4, (size_t)((int64_t)B * (2 * G + 1) * S) * sizeof(LseD),
-                       (size_t)((int64_t)B * S) * 32 * sizeof(double), (size_t)B * sizeof(SampleInfo));
+                       (size_t)((int64_t)B * S + 1) * 32 * sizeof(double), (size_t)B * sizeof(SampleInfo));
 }
 inline Layout select_layout(int B, int G) {
     return make_layout((size_t)B * 4, (size_t)B * (K + (size_t)K * K * (G - 1)) * sizeof(float));
