@@ -36,9 +36,11 @@ struct CandBuf {
 
 // Merge the buffered candidates into the running list (lanes 0..15 hold it,
 // descending; 0 = empty) sixteen at a time, and raise the threshold to the
-// list's 16th key once the list is full.  Warp-uniform.
+// list's 16th key once the list is full; a raised value also raises the
+// row's shared bound (thr: ord32 of a value at least 16 of the row's
+// elements reach; pub: what this warp last put there).  Warp-uniform.
 __device__ __forceinline__ void flush_candidates(CandBuf& cb, uint64_t& run, uint64_t& tkey,
-                                                 float& tv) {
+                                                 float& tv, unsigned* thr, uint32_t& pub) {
     const int lane = threadIdx.x & 31;
     __syncwarp();
     const unsigned n = *(volatile unsigned*)&cb.n;
@@ -59,6 +61,11 @@ __device__ __forceinline__ void flush_candidates(CandBuf& cb, uint64_t& run, uin
         tkey = k16;
         tv = key_value(k16);
     }
+    const uint32_t o16 = (uint32_t)(k16 >> 32);
+    if (o16 > pub) {  // the list is full: its 16th value bounds the row
+        pub = o16;
+        if (lane == 0) atomicMax(thr, o16);
+    }
 }
 
 // One chunk, one warp: the chunk maximum M, the sum of exp2((x - M) c) and
@@ -67,7 +74,11 @@ __device__ __forceinline__ void flush_candidates(CandBuf& cb, uint64_t& run, uin
 //   Pass 1: the packed maximum of every vector of the lane, kept in
 //   registers, and the lane maxima.  While the list is not full, T = the 16th
 //   largest lane maximum bounds the chunk's own top 16 (at least 16 elements
-//   are >= T); once it is full its 16th key is the bound.
+//   are >= T); once it is full its 16th key is the bound.  The row's shared
+//   bound (a value at least 16 of the row's elements reach, raised by every
+//   warp whose list fills) replaces either when higher: no element below it
+//   can be in the row's top 16, so the merged result is the same exact set,
+//   while a segment's own list may hold fewer than 16 keys.
 //   Candidates: only the vectors whose maximum reaches the bound's value are
 //   looked at element by element (one per lane per round); keys beating the
 //   bound are pushed and merged whenever more than CAND_FLUSH wait, and the
@@ -75,9 +86,11 @@ __device__ __forceinline__ void flush_candidates(CandBuf& cb, uint64_t& run, uin
 //   Pass 2: the exponentials (chunk_expsum).
 template <bool BF16, class View>
 __device__ __forceinline__ void topk_chunk(const View& v, float c2, CandBuf& cb, float& M_out,
-                                           double& S_out, uint64_t& run) {
+                                           double& S_out, uint64_t& run, unsigned* thr,
+                                           uint32_t& pub) {
     using C = ChunkT<BF16>;
     const int lane = threadIdx.x & 31, nv = v.nvec();
+    const uint32_t shared = *(volatile unsigned*)thr;  // used after pass 1
     uint32_t vm[NVL];
     const float m = chunk_pass1<BF16>(v, vm);
     const float M = warp_max(m);
@@ -93,6 +106,10 @@ __device__ __forceinline__ void topk_chunk(const View& v, float c2, CandBuf& cb,
             tkey = ((uint64_t)t16 << 32) - 1ull;  // below every key of value tv
         }
     }
+    if (shared != 0u && (((uint64_t)shared << 32) - 1ull) > tkey) {
+        tkey = ((uint64_t)shared << 32) - 1ull;
+        tv = unord32(shared);
+    }
     const uint32_t t2 = (tv == -INFINITY) ? C::NEG_INF_WORD : pack_value<BF16>(tv);
     uint32_t hits = 0;
 #pragma unroll
@@ -100,6 +117,8 @@ __device__ __forceinline__ void topk_chunk(const View& v, float c2, CandBuf& cb,
         if (32 * i + lane < nv && any_ge<BF16>(vm[i], t2)) hits |= 1u << i;
     if (__any_sync(FULL, hits != 0u)) {
         while (__any_sync(FULL, hits != 0u)) {  // one vector per lane per round
+            uint64_t kk[C::VW];
+            unsigned msk = 0;
             if (hits) {
                 const int i = __ffs(hits) - 1;
                 hits &= hits - 1u;
@@ -108,17 +127,31 @@ __device__ __forceinline__ void topk_chunk(const View& v, float c2, CandBuf& cb,
 #pragma unroll
                 for (int e = 0; e < C::VW; ++e) {
                     const float x = C::elem(w, e);
-                    if (x >= tv && q * C::VW + e < v.n) {
-                        const uint64_t key = make_key(x, (uint32_t)v.index(q, e));
-                        if (key > tkey) cb.key[atomicAdd(&cb.n, 1u)] = key;
-                    }
+                    kk[e] = make_key(x, (uint32_t)v.index(q, e));
+                    if (x >= tv && q * C::VW + e < v.n && kk[e] > tkey) msk |= 1u << e;
                 }
             }
+            // this round's keys appended in lane order: one prefix sum, no atomics
+            const unsigned cnt = __popc(msk);
+            unsigned incl = cnt;
+#pragma unroll
+            for (int k = 1; k < 32; k <<= 1) {
+                const unsigned o = __shfl_up_sync(FULL, incl, k);
+                if (lane >= k) incl += o;
+            }
+            const unsigned base = *(volatile unsigned*)&cb.n;
+            unsigned pos = base + incl - cnt;
+#pragma unroll
+            for (int e = 0; e < C::VW; ++e)
+                if (msk & (1u << e)) cb.key[pos++] = kk[e];
+            const unsigned nn = base + __shfl_sync(FULL, incl, 31);
             __syncwarp();
-            if (*(volatile unsigned*)&cb.n > CAND_FLUSH) flush_candidates(cb, run, tkey, tv);
+            if (lane == 0) cb.n = nn;
+            __syncwarp();
+            if (nn > CAND_FLUSH) flush_candidates(cb, run, tkey, tv, thr, pub);
         }
         __syncwarp();
-        if (*(volatile unsigned*)&cb.n > 0u) flush_candidates(cb, run, tkey, tv);
+        if (*(volatile unsigned*)&cb.n > 0u) flush_candidates(cb, run, tkey, tv, thr, pub);
     }
     M_out = M;
     S_out = chunk_expsum<BF16>(v, M, c2);
@@ -212,7 +245,8 @@ __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
     const void* __restrict__ logits, int64_t V, int64_t row_stride, int S, int64_t units,
     float inv_t, float c2, int32_t* __restrict__ idx, float* __restrict__ prob,
     float* __restrict__ logp, float* __restrict__ logz, float* __restrict__ row_max,
-    float* __restrict__ row_lse, TopkPart* __restrict__ part, unsigned* __restrict__ counters) {
+    float* __restrict__ row_lse, TopkPart* __restrict__ part, unsigned* __restrict__ counters,
+    unsigned* __restrict__ thr) {
     constexpr int ES = BF16 ? 2 : 4;
     constexpr int LEN = chunk_len(ES);
     extern __shared__ __align__(128) uint8_t ring[];
@@ -237,6 +271,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
     __syncwarp();
     uint64_t run = 0ull;  // the segment's running top-16
     unsigned seg = 0;     // chunks in the segment so far
+    uint32_t pub = 0u;    // the row bound this segment last raised thr to
     for (int k = 0; k < n; ++k, uc.next()) {
         const int64_t row = uc.g, v0 = (int64_t)uc.c * LEN;
         const int len = (int)min((int64_t)LEN, V - v0);
@@ -247,12 +282,13 @@ __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
                 warp_ring_abort(r, k, n);
                 return;
             }
-            topk_chunk<BF16>(SmemView<BF16>{r.slot(k), v0, len}, c2, cb, M, Ssum, run);
+            topk_chunk<BF16>(SmemView<BF16>{r.slot(k), v0, len}, c2, cb, M, Ssum, run, &thr[row],
+                             pub);
             warp_ring_next(r, k, n, ic, ChunkT<BF16>::NEG_INF_WORD, src);
         } else {
             topk_chunk<BF16>(
                 GlobalView<BF16>{(const uint8_t*)logits + row * row_stride * ES, v0, len}, c2, cb,
-                M, Ssum, run);
+                M, Ssum, run, &thr[row], pub);
         }
         ++seg;
         const bool seg_end = (k + 1 == n) || uc.last_of_row();
@@ -274,10 +310,14 @@ __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
                 __syncwarp();  // lane 0's acquire covers the whole warp's reads
                 topk_row_merge(part + row * S, S, row, inv_t, c2, idx, prob, logp, logz, row_max,
                                row_lse);
-                if (lane == 0) counters[row] = 0u;  // the row is done: leave its counter zero
+                if (lane == 0) {  // the row is done: leave its words zero
+                    counters[row] = 0u;
+                    thr[row] = 0u;
+                }
             }
             run = 0ull;
             seg = 0;
+            pub = 0u;
         }
     }
 }
@@ -320,7 +360,8 @@ extern "C" int dflash2_topk_softmax_ex(const void* logits, int dtype, int64_t ro
     cudaStream_t s = (cudaStream_t)stream;
     unsigned* counters = (unsigned*)((char*)ws + L.counters_off);
     TopkPart* part = (TopkPart*)((char*)ws + L.part_off);
-    if (!L.self_clean && cudaMemsetAsync(counters, 0, (size_t)rows * 4, s) != cudaSuccess)
+    unsigned* thr = counters + rows;  // the rows' shared top-16 bounds
+    if (!L.self_clean && cudaMemsetAsync(counters, 0, (size_t)rows * 8, s) != cudaSuccess)
         return DFLASH2_ECUDA;
 
     // TMA bulk copies need 16-byte aligned chunk starts and 16-byte multiples
@@ -333,7 +374,7 @@ extern "C" int dflash2_topk_softmax_ex(const void* logits, int dtype, int64_t ro
         if (ring_prepare(kern, dyn) != DFLASH2_OK) return DFLASH2_ECUDA;                          \
         kern<<<ring_grid(units), RING_THREADS, dyn, s>>>(logits, V, row_stride, (int)S, units,    \
                                                          inv_temperature, c2, idx, prob, logp,    \
-                                                         logz, row_max, row_lse, part, counters); \
+                                                         logz, row_max, row_lse, part, counters, thr); \
     } while (0)
     if (dtype == DFLASH2_BF16) {
         if (tma) DFL_TOPK(true, true);
@@ -400,7 +441,7 @@ extern "C" int dflash2_topk_softmax_noalloc(const void* logits, int dtype, int64
     void* scratch = noalloc_scratch_on_current_device();
     if (!scratch) return DFLASH2_ECUDA;
     // the array's counters start at zero whatever an earlier (failed) call left
-    if (cudaMemsetAsync(scratch, 0, (size_t)rows * 4, (cudaStream_t)stream) != cudaSuccess)
+    if (cudaMemsetAsync(scratch, 0, (size_t)rows * 8, (cudaStream_t)stream) != cudaSuccess)
         return DFLASH2_ECUDA;
     return dflash2_topk_softmax(logits, dtype, rows, V, row_stride, inv_temperature, idx, prob, logp,
                                 logz, scratch, NOALLOC_SCRATCH_BYTES, stream);

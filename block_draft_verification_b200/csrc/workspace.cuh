@@ -75,8 +75,8 @@ inline Layout make_layout(size_t counters, size_t part, size_t part2 = 0, size_t
 // Layouts for an element size es (2 for bf16, 4 for fp32; a workspace sized
 // with es = 4 serves both, its chunks being the shorter).
 inline Layout topk_layout(int64_t rows, int64_t V, int es) {
-    const int64_t S = row_chunks(V, es);
-    return make_layout((size_t)rows * 4, (size_t)(rows * S) * sizeof(TopkPart));
+    const int64_t S = row_chunks(V, es);  // counters [rows], then the rows' top-16 bounds [rows]
+    return make_layout((size_t)rows * 8, (size_t)(rows * S) * sizeof(TopkPart));
 }
 inline Layout greedy_layout(int B, int G, int64_t V, int es) {
     const int64_t S = row_chunks(V, es);
