@@ -57,6 +57,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time the step with eager launches instead of CUDA graph replays")
+    ap.add_argument("--acceptance", action="store_true",
+                    help="print the acceptance study (mean accepted tokens per verify step for "
+                         "the top-1 path, the pair selector and the top-16 oracle path) instead "
+                         "of a bench line")
     ap.add_argument("--only", choices=["topk_softmax", "pair_select", "verify_sample",
                                        "verify_greedy", "dynconv2"], default=None,
                     help="run and time one call of the step only (for profiling); prints a "
@@ -206,6 +210,67 @@ def run_reference(args, rank, world):
             "e2e": {"value": value, "unit": "cycles/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- acceptance study
+def acceptance_paths(dfl, torch, T, Q, anchor, E, Wsel, inv_t):
+    """The three drafted paths of a batch, every step in the library's kernels
+    (the path choice is a compare and a select on their outputs): the drafter's
+    top-1 per position, the pair selector's path, and the top-16 oracle path
+    (the target's own token wherever it is among the drafter's 16 candidates,
+    else the top-1).  Returns the paths and the per-position hit masks."""
+    B, G1, V = T.shape
+    G = G1 - 1
+    idx, _, logp, _ = dfl.topk_softmax(Q.reshape(-1, V), inv_t)
+    cand = idx.view(B, G, 16)
+    t = dfl.topk_softmax(T[:, :G].reshape(-1, V), inv_t)[0].view(B, G, 16)[:, :, 0]
+    hit16 = (cand == t[:, :, None]).any(-1)
+    top1 = cand[:, :, 0].contiguous()
+    oracle_path = torch.where(hit16, t, top1).contiguous()
+    sel = dfl.pair_select(cand, logp.view(B, G, 16), anchor, E, Wsel)[0]
+    return {"top1": top1, "selector": sel, "top16_oracle": oracle_path}, hit16, top1 == t
+
+
+def run_acceptance(args):
+    """Synthetic analog of the pages' top-16 oracle figure (a trained drafter:
+    4.27 accepted tokens per step on its top-1 path, 6.79 when told the target
+    token whenever it is in the top 16): mean (n + 1) under greedy verification
+    for the three paths, on the calibrated synthetic workloads."""
+    import torch
+
+    import block_draft_verification_b200 as dfl
+    import synth
+
+    dev = torch.device("cuda", 0)
+
+    def dev_t(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    out = {}
+    for name, ncyc in (("b1", 128), ("b8", 128), ("b32", 128)):
+        w = synth.WORKLOADS[name]
+        sel = synth.gen_selector(w)
+        E, Wsel = dev_t(sel.emb), dev_t(sel.W)
+        acc = {"top1": [], "selector": [], "top16_oracle": []}
+        h16, h1 = [], []
+        for first in range(0, ncyc, 32):
+            b = synth.gen_batch(w, B=min(32, ncyc - first), first=first)
+            T = dev_t(b.target)
+            paths, hit16, hit1 = acceptance_paths(dfl, torch, T, dev_t(b.draft), dev_t(b.anchor),
+                                                  E, Wsel, w.inv_temperature)
+            for k, p in paths.items():
+                acc[k] += (dfl.verify_greedy(T, p)[0] + 1).cpu().tolist()
+            h16.append(hit16.float().mean().item())
+            h1.append(hit1.float().mean().item())
+        out[name] = {k: round(float(np.mean(v)), 3) for k, v in acc.items()}
+        out[name].update(cycles=ncyc, target_in_top16=round(float(np.mean(h16)), 4),
+                         target_is_top1=round(float(np.mean(h1)), 4))
+    print(json.dumps({"acceptance_study": out, "block": 8,
+                      "pages": "trained drafter, top-1 path 4.27 -> top-16 oracle 6.79"}),
+          flush=True)
 
 
 # --------------------------------------------------------------------------- GPU
@@ -513,7 +578,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        if args.impl == "reference":
+        if args.acceptance:
+            if rank == 0:
+                run_acceptance(args)
+        elif args.impl == "reference":
             run_reference(args, rank, world)
         else:
             run_ours(args, rank, world, local_rank)

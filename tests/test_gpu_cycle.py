@@ -60,3 +60,37 @@ def test_chained_cycle(orc, name, sampling):
             ties.add("draw")
     print(name, "sampling" if sampling else "greedy", "mean acceptance %.2f" % (on + 1).mean(),
           "near-ties:", ties.report())
+
+
+def test_top16_oracle_paths(orc):
+    """The acceptance study's three paths (bench.py --acceptance): the top-1
+    and top-16 oracle paths and their greedy verification equal the oracle's
+    chain exactly; per sequence the oracle path is accepted at least as far as
+    any path drawn from the same 16 candidates (at the first position whose
+    target token is not among them every such path mismatches)."""
+    need_cuda()
+    import bench
+    w = synth.WORKLOADS["b1"]
+    b = synth.gen_batch(w, B=8)
+    sel = synth.gen_selector(w)
+    B, G, V = b.target.shape[0], w.G, w.V
+    T = to_dev(b.target)
+    paths, hit16, hit1 = bench.acceptance_paths(dfl, torch, T, to_dev(b.draft), to_dev(b.anchor),
+                                                to_dev(sel.emb), to_dev(sel.W), w.inv_temperature)
+    n = {k: to_host(dfl.verify_greedy(T, p)[0]) for k, p in paths.items()}
+    torch.cuda.synchronize()
+
+    oidx = orc.topk_softmax(b.draft.reshape(-1, V), w.inv_temperature)[0].reshape(B, G, 16)
+    tidx = orc.topk_softmax(b.target[:, :G].reshape(-1, V), w.inv_temperature)[0].reshape(B, G, 16)
+    t = tidx[:, :, 0]
+    ohit = (oidx == t[:, :, None]).any(-1)
+    otop1 = oidx[:, :, 0].astype(np.int32)
+    opath = np.where(ohit, t, otop1).astype(np.int32)
+    np.testing.assert_array_equal(to_host(paths["top1"]), otop1)
+    np.testing.assert_array_equal(to_host(paths["top16_oracle"]), opath)
+    np.testing.assert_array_equal(to_host(hit16), ohit)
+    np.testing.assert_array_equal(n["top1"], orc.verify_greedy(b.target, otop1)[0])
+    np.testing.assert_array_equal(n["top16_oracle"], orc.verify_greedy(b.target, opath)[0])
+    assert np.all(n["top16_oracle"] >= n["top1"]) and np.all(n["top16_oracle"] >= n["selector"])
+    first_miss = np.where((~ohit).any(1), (~ohit).argmax(1), G)
+    np.testing.assert_array_equal(n["top16_oracle"], first_miss)
