@@ -185,3 +185,25 @@ def test_row_stats(orc, name):
         np.testing.assert_array_equal(got[4], xf.max(axis=1))
         _, _, _, ologz = orc.topk_softmax(x, invT)
         assert_close(got[5], ologz - xf.max(axis=1).astype(np.float64) * invT, RTOL_F32, "row_lse")
+
+
+def test_many_rows_memset_control(orc):
+    """More rows than the 64 KB control area holds (10,000 rows: a counter and a
+    shared top-16 bound each), so the call clears its control words with a
+    memset; rows of one chunk and of two (V = 4,100 fp32: 2,048 + 2,048 + 4).
+    Two calls on one workspace: the second must not inherit the first's
+    bounds."""
+    need_cuda()
+    rng = np.random.default_rng(10000)
+    ws = dfl.Workspace(torch.device("cuda"))
+    for V in (64, 4100):
+        rows = 10000 if V == 64 else 2000
+        for rep in range(2):
+            x = (rng.standard_normal((rows, V)) * (1.0 + rep)).astype(np.float32)
+            idx, prob, logp, logz = (to_host(a) for a in
+                                     dfl.topk_softmax(to_dev(x), 1.0, ws=ws))
+            oi, op, ol, oz = orc.topk_softmax(x, 1.0)
+            np.testing.assert_array_equal(idx, oi)
+            assert_close(prob, op, RTOL_F32, "prob")
+            assert_close(logz, oz, RTOL_F32, "logz")
+    assert dfl.device_errors() == 0

@@ -313,3 +313,35 @@ def test_sample_fallback_when_residual_empty(orc):
     np.testing.assert_array_equal(n, np.zeros(B, np.int32))
     np.testing.assert_array_equal(out[:, 0], spike.astype(np.int32))
     assert np.all(out[:, 1:] == -1)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_sample_many_sequences_memset_control(orc, fused):
+    """More sequences than the 64 KB control area holds (B = 2,048: the finish
+    queue alone needs 256 KB), so the call clears its control words with a
+    memset; every V is one draw unit.  Two calls on one workspace: the second
+    must not see the first's queue."""
+    need_cuda()
+    rng = np.random.default_rng(2048)
+    B, G, V = 2048, 3, 64
+    t = (rng.standard_normal((B, G + 1, V)) * 2.0).astype(np.float32)
+    q = (t[:, :G] + rng.standard_normal((B, G, V)) * 0.5).astype(np.float32)
+    d = np.argmax(q, axis=2).astype(np.int32)
+    ws = dfl.Workspace(torch.device("cuda"))
+    stats = tuple(to_dev(a) for a in draft_stats(orc, q, 1.0)) if fused else None
+    ties = NearTies()
+    for step in (0, 1):
+        n, out = dfl.verify_sample(to_dev(t), to_dev(q), to_dev(d), 77, step, None, 1.0,
+                                   ws=ws, draft_stats=stats)[:2]
+        torch.cuda.synchronize()
+        n, out = to_host(n), to_host(out)
+        on, oout, _, _, macc, mres = orc.verify_sample(t, q, d, 77, step, None, 1.0, 0)
+        for s in range(B):
+            if n[s] != on[s]:
+                assert macc[s] < ACCEPT_BAND, (s, n[s], on[s])
+                ties.add("accept")
+            elif not np.array_equal(out[s], oout[s]):
+                assert mres[s] < DRAW_BAND, (s, out[s], oout[s])
+                ties.add("draw")
+    assert dfl.device_errors() == 0
+    print("near-ties:", ties.report())
