@@ -157,11 +157,11 @@ __device__ __forceinline__ void topk_chunk(const View& v, float c2, CandBuf& cb,
     S_out = chunk_expsum<BF16>(v, M, c2);
 }
 
-// The row's final merge, list by list: the segment lists (bitonic merges in
-// chunk order), the maximum, and the fp64 sum of the chunk sums rescaled to it
-// (lane c takes chunks c, c + 32, ...; then a fixed butterfly).  The fallback
-// of topk_row_merge for rows whose candidates do not fit its buffer.
-__device__ __noinline__ void topk_row_merge_lists(const TopkPart* P, int S, int64_t row, float inv_t,
+// The row's final merge by one warp, after its last chunk was published:
+// the segment lists (bitonic merges in chunk order), the maximum, and the
+// fp64 sum of the chunk sums rescaled to it (lane c takes chunks c, c + 32,
+// ...; then a fixed butterfly).
+__device__ __forceinline__ void topk_row_merge(const TopkPart* P, int S, int64_t row, float inv_t,
                                                float c2, int32_t* __restrict__ idx,
                                                float* __restrict__ prob, float* __restrict__ logp,
                                                float* __restrict__ logz,
@@ -231,131 +231,6 @@ __device__ __noinline__ void topk_row_merge_lists(const TopkPart* P, int S, int6
             if (row_lse) row_lse[row] = (float)lns;
         }
     }
-}
-
-// The row's final merge by one warp, after its last chunk was published.
-// Softmax: the maximum and the fp64 sum of the chunk sums rescaled to it (lane
-// c takes chunks c, c + 32, ...; then a fixed butterfly).  Top 16 of the
-// union of the segment lists (each descending, 0 = empty): T0 = the largest
-// 16th key of a full list (that list alone holds 16 keys >= T0, so no key
-// below T0 is in the row's top 16); every list's keys >= T0 (a prefix) are
-// gathered in the warp's candidate buffer at offsets from one warp prefix
-// sum, and a candidate's rank is the number of candidates above it (keys are
-// distinct): ranks below 16 are the output slots.  Rows with more than
-// MERGE_CAP candidates (or more than 64 chunks) take the list-by-list merge.
-constexpr int MERGE_CAP = 128;
-__device__ __forceinline__ void topk_row_merge(const TopkPart* P, int S, int64_t row, float inv_t,
-                                               float c2, CandBuf& cb, int32_t* __restrict__ idx,
-                                               float* __restrict__ prob, float* __restrict__ logp,
-                                               float* __restrict__ logz,
-                                               float* __restrict__ row_max,
-                                               float* __restrict__ row_lse) {
-    const int lane = threadIdx.x & 31;
-    if (S > 64) {
-        topk_row_merge_lists(P, S, row, inv_t, c2, idx, prob, logp, logz, row_max, row_lse);
-        return;
-    }
-    auto ldkey = [](const uint64_t* p) { return (uint64_t)__ldcg((const unsigned long long*)p); };
-    // one round: every chunk's (max, sum, first and 16th key); lane c holds c and c + 32
-    float mc[2];
-    double sc[2];
-    uint64_t k0[2], k15[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int c = lane + 32 * h;
-        mc[h] = -INFINITY;
-        sc[h] = 0.0;
-        k0[h] = k15[h] = 0ull;
-        if (c < S) {
-            mc[h] = __ldcg(&P[c].m);
-            sc[h] = __ldcg(&P[c].s);
-            k0[h] = ldkey(&P[c].key[0]);
-            k15[h] = ldkey(&P[c].key[K - 1]);
-        }
-    }
-    const float M = warp_max(fmaxf(mc[0], mc[1]));
-    double ssum = 0.0;
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-        if (mc[h] != -INFINITY) ssum += sc[h] * exp2(((double)mc[h] - (double)M) * (double)c2);
-    ssum = warp_sum(ssum);
-    // T0: the largest 16th key of a full list (0 if no list is full)
-    uint64_t t0 = 0ull;
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-        if (k0[h] != 0ull && k15[h] > t0) t0 = k15[h];
-#pragma unroll
-    for (int j = 16; j > 0; j >>= 1) {
-        const uint64_t o = shfl_xor(t0, j);
-        t0 = o > t0 ? o : t0;
-    }
-    // each list's keys >= T0, gathered in chunk order
-    uint64_t kl[2][K];
-    unsigned cnt[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        cnt[h] = 0;
-#pragma unroll
-        for (int k = 0; k < K; ++k) {
-            kl[h][k] = (k0[h] != 0ull) ? ldkey(&P[lane + 32 * h].key[k]) : 0ull;
-            cnt[h] += (kl[h][k] != 0ull && kl[h][k] >= t0) ? 1u : 0u;
-        }
-    }
-    unsigned incl0 = cnt[0], incl1 = cnt[1];
-#pragma unroll
-    for (int k = 1; k < 32; k <<= 1) {
-        const unsigned o0 = __shfl_up_sync(FULL, incl0, k), o1 = __shfl_up_sync(FULL, incl1, k);
-        if (lane >= k) {
-            incl0 += o0;
-            incl1 += o1;
-        }
-    }
-    const unsigned tot0 = __shfl_sync(FULL, incl0, 31);
-    const unsigned total = tot0 + __shfl_sync(FULL, incl1, 31);
-    if (total > (unsigned)MERGE_CAP) {
-        topk_row_merge_lists(P, S, row, inv_t, c2, idx, prob, logp, logz, row_max, row_lse);
-        return;
-    }
-    const unsigned off0 = incl0 - cnt[0], off1 = tot0 + incl1 - cnt[1];
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-        if ((unsigned)k < cnt[0]) cb.key[off0 + k] = kl[0][k];
-        if ((unsigned)k < cnt[1]) cb.key[off1 + k] = kl[1][k];
-    }
-    __syncwarp();
-    // ranks: every candidate against every candidate (broadcast reads)
-    constexpr int CPL = MERGE_CAP / 32;  // candidates per lane
-    uint64_t x[CPL];
-    unsigned rk[CPL];
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-        const unsigned t = (unsigned)lane + 32u * i;
-        x[i] = (t < total) ? cb.key[t] : 0ull;
-        rk[i] = 0;
-    }
-    for (unsigned u = 0; u < total; ++u) {
-        const uint64_t y = cb.key[u];
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) rk[i] += (y > x[i]) ? 1u : 0u;
-    }
-    const double lns = log(ssum);
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-        const unsigned t = (unsigned)lane + 32u * i;
-        if (t < total && rk[i] < (unsigned)K) {
-            const double v = (double)key_value(x[i]);
-            const int64_t o = row * K + rk[i];
-            idx[o] = (int32_t)key_index(x[i]);
-            prob[o] = (float)(exp2((v - (double)M) * (double)c2) / ssum);
-            logp[o] = (float)((v - (double)M) * (double)inv_t - lns);
-        }
-    }
-    if (lane == 0) {
-        logz[row] = (float)((double)M * (double)inv_t + lns);
-        if (row_max) row_max[row] = M;
-        if (row_lse) row_lse[row] = (float)lns;
-    }
-    __syncwarp();  // the buffer is the warp's candidate buffer again
 }
 
 // Units (row, chunk): one CTA per SM over a contiguous range, each warp a
@@ -433,8 +308,8 @@ __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
             if (lane == 0) last = publish(&counters[row], seg, (unsigned)S);
             if (__shfl_sync(FULL, last, 0)) {
                 __syncwarp();  // lane 0's acquire covers the whole warp's reads
-                topk_row_merge(part + row * S, S, row, inv_t, c2, cb, idx, prob, logp, logz,
-                               row_max, row_lse);
+                topk_row_merge(part + row * S, S, row, inv_t, c2, idx, prob, logp, logz, row_max,
+                               row_lse);
                 if (lane == 0) {  // the row is done: leave its words zero
                     counters[row] = 0u;
                     thr[row] = 0u;
