@@ -53,6 +53,10 @@ def _sig():
                                       vp, vp, vp, vp, vp]
     L.orc_verify_sample.argtypes = [vp, vp, i32, i32, i32, i64, vp, dbl, u64, u32, vp, i32,
                                     vp, vp, vp, vp, vp, vp]
+    L.orc_verify_sample_trunc_u.argtypes = [vp, vp, i32, i32, i32, i64, vp, dbl, i32, dbl, i32,
+                                            vp, vp, vp, vp, vp, vp, vp, vp]
+    L.orc_verify_sample_trunc.argtypes = [vp, vp, i32, i32, i32, i64, vp, dbl, i32, dbl, u64,
+                                          u32, vp, i32, vp, vp, vp, vp, vp, vp, vp]
     L.orc_dynconv2.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
 
 
@@ -203,6 +207,52 @@ def verify_sample(target, draft, draft_tok, seed, step, seq_id=None, inv_tempera
                                    _p(n), _p(out), _p(ratio), _p(u), _p(ma), _p(mr)),
            "verify_sample")
     return n, out, ratio, u, ma, mr
+
+
+def verify_sample_trunc_u(target, draft, draft_tok, u_acc, u_res, inv_temperature=1.0,
+                          top_k=20, top_p=0.95, q_mode=Q_SOFTMAX):
+    """Verification of top-k / top-p truncated distributions with explicit
+    uniforms u_acc [B,G], u_res [B,G+1].  Returns n, out, ratio, margin_acc,
+    margin_res, margin_trunc."""
+    t = np.ascontiguousarray(target)
+    B, G1, V = t.shape
+    G = G1 - 1
+    q = None if draft is None else np.ascontiguousarray(draft)
+    d = _c(draft_tok, np.int32)
+    ua = _c(u_acc, np.float64)
+    ur = _c(u_res, np.float64)
+    n = np.zeros(B, np.int32)
+    out = np.zeros((B, G1), np.int32)
+    ratio = np.zeros((B, G), np.float64)
+    ma, mr, mt = (np.zeros(B, np.float64) for _ in range(3))
+    _check(lib().orc_verify_sample_trunc_u(_p(t), _p(q), _dtype_of(t), B, G, V, _p(d),
+                                           float(inv_temperature), int(top_k), float(top_p),
+                                           q_mode, _p(ua), _p(ur), _p(n), _p(out), _p(ratio),
+                                           _p(ma), _p(mr), _p(mt)), "verify_sample_trunc_u")
+    return n, out, ratio, ma, mr, mt
+
+
+def verify_sample_trunc(target, draft, draft_tok, seed, step, seq_id=None, inv_temperature=1.0,
+                        top_k=20, top_p=0.95, q_mode=Q_SOFTMAX):
+    """Philox uniforms.  Returns n, out, ratio, u, margin_acc, margin_res,
+    margin_trunc."""
+    t = np.ascontiguousarray(target)
+    B, G1, V = t.shape
+    G = G1 - 1
+    q = None if draft is None else np.ascontiguousarray(draft)
+    d = _c(draft_tok, np.int32)
+    sid = None if seq_id is None else _c(seq_id, np.uint32)
+    n = np.zeros(B, np.int32)
+    out = np.zeros((B, G1), np.int32)
+    ratio = np.zeros((B, G), np.float64)
+    u = np.zeros((B, G), np.float64)
+    ma, mr, mt = (np.zeros(B, np.float64) for _ in range(3))
+    _check(lib().orc_verify_sample_trunc(_p(t), _p(q), _dtype_of(t), B, G, V, _p(d),
+                                         float(inv_temperature), int(top_k), float(top_p),
+                                         int(seed), int(step), _p(sid), q_mode, _p(n), _p(out),
+                                         _p(ratio), _p(u), _p(ma), _p(mr), _p(mt)),
+           "verify_sample_trunc")
+    return n, out, ratio, u, ma, mr, mt
 
 
 # ---------------------------------------------------------------- dynconv

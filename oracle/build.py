@@ -9,7 +9,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SOURCES = ["philox.cpp", "topk_softmax.cpp", "pair_select.cpp", "verify_greedy.cpp",
-           "verify_sample.cpp", "dynconv2.cpp"]
+           "verify_sample.cpp", "verify_sample_trunc.cpp", "dynconv2.cpp"]
 HEADERS = ["oracle.h", "oracle_util.h"]
 LIB = os.path.join(HERE, "liboracle.so")
 

@@ -86,6 +86,24 @@ int orc_verify_sample(const void* target, const void* draft, int dtype, int B, i
                       int32_t* n_accept, int32_t* out_tok, double* ratio, double* u,
                       double* margin_acc, double* margin_res);
 
+/* ---- the same verification of distributions truncated by top-k and top-p
+ *      ([latenode] "Preguntas frecuentes": temperature 1.0, top-p 0.95,
+ *      top-k 20 for the Qwen targets); top_k <= 0 and top_p >= 1 switch
+ *      either off.  margin_trunc[b] = the smallest top-p cut margin of the
+ *      rows the sequence's decisions and draw used ---- */
+int orc_verify_sample_trunc_u(const void* target, const void* draft, int dtype, int B, int G,
+                              int64_t V, const int32_t* draft_tok, double inv_temperature,
+                              int top_k, double top_p, int q_mode, const double* u_acc,
+                              const double* u_res, int32_t* n_accept, int32_t* out_tok,
+                              double* ratio, double* margin_acc, double* margin_res,
+                              double* margin_trunc);
+int orc_verify_sample_trunc(const void* target, const void* draft, int dtype, int B, int G,
+                            int64_t V, const int32_t* draft_tok, double inv_temperature,
+                            int top_k, double top_p, uint64_t seed, uint32_t step,
+                            const uint32_t* seq_id, int q_mode, int32_t* n_accept,
+                            int32_t* out_tok, double* ratio, double* u, double* margin_acc,
+                            double* margin_res, double* margin_trunc);
+
 /* ---- two-tap dynamic depthwise conv with its tap projection and residual
  *      ([tamsi] "L’idée, sans le papier": two-tap conv before/after each
  *      attention and MLP; [myaiexp] features: 2-tap dynamic convolution) ---- */
