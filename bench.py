@@ -273,6 +273,25 @@ def run_acceptance(args):
           flush=True)
 
 
+# --------------------------------------------------------------------------- ranks
+def rank_first_sequence(rank, k, B):
+    """First sequence of input set k (0 or 1) on a rank: every (rank, set)
+    pair takes its own block of B sequences, so the ranks' batches are
+    disjoint (weak scaling, no data-path collective)."""
+    return (rank * 2 + k) * B
+
+
+def max_over_ranks(values, world, device):
+    """Elementwise maximum of per-rank float values (the slowest rank's time),
+    as float64 on `device`; one all-reduce when world > 1."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t
+
+
 # --------------------------------------------------------------------------- GPU
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -287,7 +306,8 @@ def run_ours(args, rank, world, local_rank):
     B, G, V = w.B, w.G, w.V
 
     # inputs: two input sets per rank (alternated between steps), weights once
-    sets = [(synth.gen_batch(w, first=(rank * 2 + k) * B), synth.gen_conv(w, first=(rank * 2 + k) * B))
+    sets = [(synth.gen_batch(w, first=rank_first_sequence(rank, k, B)),
+             synth.gen_conv(w, first=rank_first_sequence(rank, k, B)))
             for k in range(2)]
     sel = synth.gen_selector(w)
     wtap = sets[0][1].w_tap
@@ -442,10 +462,8 @@ def run_ours(args, rank, world, local_rank):
                               "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1),
                               "steps": args.steps}), flush=True)
         return
-    local = torch.tensor([s0.elapsed_time(s1), float(per_call.sum(axis=1).mean())] +
-                         per_call.mean(axis=0).tolist(), dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(local, op=dist.ReduceOp.MAX)
+    local = max_over_ranks([s0.elapsed_time(s1), float(per_call.sum(axis=1).mean())] +
+                           per_call.mean(axis=0).tolist(), world, dev)
     ms_per_step = float(local[0]) / args.steps
     calls_sum_ms = float(local[1])
     mean_call_ms = local[2:].cpu().numpy()
@@ -493,10 +511,8 @@ def run_ours(args, rank, world, local_rank):
             e2e_step(s)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        t = torch.tensor([e0.elapsed_time(e1) / ne], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * 1000.0 / float(t), "unit": "cycles/s",
+        t = max_over_ranks([e0.elapsed_time(e1) / ne], world, dev)
+        e2e = {"value": world * 1000.0 / float(t[0]), "unit": "cycles/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     if rank != 0:
