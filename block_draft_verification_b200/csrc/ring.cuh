@@ -1,6 +1,6 @@
-// ring.cuh -- persistent streaming of vocabulary rows: one producer warp
-// keeps a ring of TMA bulk copies in flight, consumer warps each reduce whole
-// chunks on their own.
+// ring.cuh -- persistent streaming of vocabulary rows: every warp keeps its
+// own two-slot ring of TMA bulk copies in flight and reduces whole chunks on
+// its own.
 //
 // A unit is one chunk of a row: SLOT_BYTES of logits (4096 bf16 or 2048 fp32
 // elements; the last chunk of a row is shorter).  The chunk length depends on
