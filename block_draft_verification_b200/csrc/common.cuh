@@ -17,17 +17,7 @@ namespace dfl {
 constexpr unsigned FULL = 0xFFFFFFFFu;
 constexpr int K = DFLASH2_K;
 
-// ---------------------------------------------------------------------------
-// Work decomposition of a vocabulary row.  A row is cut into CHUNK-element
-// units; each unit is one CTA of NT threads, EPT elements per thread.  CHUNK
-// is fixed (it does not depend on B, the grid or the device), so every
-// floating-point reduction runs in the same order for a given V whatever
-// batch a row sits in: results are batch-invariant bit for bit.
-constexpr int NT = 256;
-constexpr int CHUNK = 16384;
-constexpr int EPT = CHUNK / NT;  // 64
-
-__host__ __device__ inline int64_t n_chunks(int64_t V) { return (V + CHUNK - 1) / CHUNK; }
+constexpr int NT = 256;  // threads per CTA of the select and fp32 conv kernels
 
 // ---------------------------------------------------------------------------
 // Orderable keys.  ord32 maps a float to a uint32 whose unsigned order is the
@@ -56,11 +46,6 @@ __device__ __forceinline__ uint64_t shfl_xor(uint64_t v, int m) {
 }
 __device__ __forceinline__ uint32_t shfl_xor(uint32_t v, int m) {
     return __shfl_xor_sync(FULL, v, m);
-}
-__device__ __forceinline__ uint64_t shfl_up64(uint64_t v) {
-    uint32_t lo = __shfl_up_sync(FULL, (uint32_t)v, 1);
-    uint32_t hi = __shfl_up_sync(FULL, (uint32_t)(v >> 32), 1);
-    return ((uint64_t)hi << 32) | lo;
 }
 __device__ __forceinline__ uint64_t shfl64(uint64_t v, int src) {
     uint32_t lo = __shfl_sync(FULL, (uint32_t)v, src);
@@ -154,27 +139,15 @@ __device__ __forceinline__ LseD warp_lse(LseD v, float c) {
 }
 
 // ---------------------------------------------------------------------------
-// Streaming loads of a vocabulary chunk.  A thread owns EPT elements of the
-// chunk as NV vectors of VW elements; vector i of thread t starts at element
-// v0 + (i * NT + t) * VW, so one warp instruction reads 512 contiguous bytes
-// and a thread's elements are in ascending index order (i, then e).
+// Elements of a 16-byte vector of bf16 (8) or fp32 (4) values, widened to
+// fp32 (exact).
 template <bool BF16>
 struct Row {
-    static constexpr int VW = BF16 ? 8 : 4;     // elements per 16-byte vector
-    static constexpr int NV = EPT / VW;         // vectors per thread
-    static constexpr uint32_t NEG_INF_WORD = BF16 ? 0xFF80FF80u : 0xFF800000u;
-
-    __device__ static __forceinline__ uint4 ld_stream(const void* p) {
-        uint4 r;
-        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                     : "l"(p));
-        return r;
-    }
+    static constexpr int VW = BF16 ? 8 : 4;  // elements per 16-byte vector
     __device__ static __forceinline__ uint32_t comp(const uint4& r, int i) {
         return i == 0 ? r.x : i == 1 ? r.y : i == 2 ? r.z : r.w;
     }
-    // Element e (0 <= e < VW) of a raw vector, widened to fp32 (exact).
+    // Element e (0 <= e < VW) of a raw vector.
     __device__ static __forceinline__ float elem(const uint4& r, int e) {
         if (BF16) {
             uint32_t w = comp(r, e >> 1);
@@ -182,59 +155,7 @@ struct Row {
         }
         return __uint_as_float(comp(r, e));
     }
-    __device__ static __forceinline__ uint32_t scalar_bits(const void* row, int64_t v) {
-        if (BF16) return (uint32_t)__ldg((const unsigned short*)row + v);
-        return __ldg((const unsigned int*)row + v);
-    }
-    // Load the thread's NV vectors of the chunk [v0, vend); elements at or
-    // beyond vend read as -inf.  VEC: the row start is 16-byte aligned.
-    template <bool VEC>
-    __device__ static __forceinline__ void load(const void* row, int64_t v0, int64_t vend,
-                                                uint4 (&r)[NV]) {
-        const int t = threadIdx.x;
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            int64_t vb = v0 + (int64_t)(i * NT + t) * VW;
-            if (VEC && vb + VW <= vend) {
-                r[i] = ld_stream((const char*)row + vb * (BF16 ? 2 : 4));
-            } else {
-                uint32_t w[4] = {NEG_INF_WORD, NEG_INF_WORD, NEG_INF_WORD, NEG_INF_WORD};
-#pragma unroll
-                for (int e = 0; e < VW; ++e) {
-                    if (vb + e < vend) {
-                        uint32_t bits = scalar_bits(row, vb + e);
-                        if (BF16) {
-                            uint32_t& word = w[e >> 1];
-                            word = (e & 1) ? ((word & 0x0000FFFFu) | (bits << 16))
-                                           : ((word & 0xFFFF0000u) | bits);
-                        } else {
-                            w[e] = bits;
-                        }
-                    }
-                }
-                r[i] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-        }
-    }
-    __device__ static __forceinline__ int64_t index_of(int64_t v0, int i, int e) {
-        return v0 + (int64_t)(i * NT + (int)threadIdx.x) * VW + e;
-    }
 };
-
-// Max of the 8 bf16 (or 4 fp32) elements of a 16-byte vector, widened to fp32.
-// bf16 uses packed two-lane max instructions (values are finite; -0 and +0
-// may come back either way, and every later compare treats them as equal).
-template <bool BF16>
-__device__ __forceinline__ float vec_max(const uint4& v) {
-    if (BF16) {
-        auto b2 = [](uint32_t w) { return *reinterpret_cast<const __nv_bfloat162*>(&w); };
-        const __nv_bfloat162 m = __hmax2(__hmax2(b2(v.x), b2(v.y)), __hmax2(b2(v.z), b2(v.w)));
-        const uint32_t mw = *reinterpret_cast<const uint32_t*>(&m);
-        return fmaxf(__uint_as_float(mw << 16), __uint_as_float(mw & 0xFFFF0000u));
-    }
-    return fmaxf(fmaxf(__uint_as_float(v.x), __uint_as_float(v.y)),
-                 fmaxf(__uint_as_float(v.z), __uint_as_float(v.w)));
-}
 
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon et al., SC'11, section 5): ten rounds of
