@@ -169,7 +169,7 @@ __device__ __forceinline__ void topk_row_merge(const TopkPart* P, int S, int64_t
                                                float* __restrict__ row_lse) {
     const int lane = threadIdx.x & 31;
     auto ldkey = [](const uint64_t* p) { return (uint64_t)__ldcg((const unsigned long long*)p); };
-    // round 1: every chunk's (max, sum) and whether it carries a list
+    // first load pass: every chunk's (max, sum) and whether it carries a list
     float M = -INFINITY;
     for (int c = lane; c < S; c += 32) M = fmaxf(M, __ldcg(&P[c].m));
     M = warp_max(M);
@@ -187,7 +187,7 @@ __device__ __forceinline__ void topk_row_merge(const TopkPart* P, int S, int64_t
             k0 = ldkey(&P[c].key[0]);
         }
         if (mc != -INFINITY) ssum += sc * exp2(((double)mc - (double)M) * (double)c2);
-        // round 2: the lists of this group of chunks, loaded together, merged in chunk order
+        // second load pass: the lists of this group of chunks, loaded together, merged in chunk order
         unsigned has = __ballot_sync(FULL, k0 != 0ull);
         while (has) {
             constexpr int PF = 8;
