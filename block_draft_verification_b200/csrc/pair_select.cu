@@ -34,7 +34,7 @@ template <bool EMB_BF16, int D>
 __global__ void __launch_bounds__(NT, 2) pair_select_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ logp,
     const int32_t* __restrict__ anchor, const void* __restrict__ emb, const float* __restrict__ W,
-    int G, int32_t* __restrict__ path_tok, int32_t* __restrict__ path_rank,
+    int64_t V, int G, int32_t* __restrict__ path_tok, int32_t* __restrict__ path_rank,
     float* __restrict__ path_score, float* __restrict__ scores, unsigned* __restrict__ counters) {
     constexpr int LD = D + 4;                  // padded rows, still 16-byte aligned
     constexpr int ES = EMB_BF16 ? 2 : 4;
@@ -73,11 +73,14 @@ __global__ void __launch_bounds__(NT, 2) pair_select_kernel(
         if (t < K) s_tok[t] = cand[i * K + t];
         else if (t < K + nl) s_tok[t] = (i == 0) ? anchor[b] : cand[(i - 1) * K + (t - K)];
         __syncthreads();
+        // a token id outside [0, V) gets a zero embedding (no load) and is flagged
+        if (t < K + nl && (uint32_t)s_tok[t] >= (uint64_t)V) atomicOr(&g_dev_err, ERR_INPUT);
         uint4 v[IPT];
 #pragma unroll
         for (int q = 0; q < IPT; ++q) {  // all loads first: one memory round trip
             const int e = t + q * NT, r = e / RV, c = e - r * RV;
-            if (r < K + nl)
+            v[q] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < K + nl && (uint32_t)s_tok[r] < (uint64_t)V)
                 v[q] = __ldg((const uint4*)((const char*)emb + (int64_t)s_tok[r] * (D * ES)) + c);
         }
 #pragma unroll
@@ -294,7 +297,7 @@ extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const 
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) !=      \
             cudaSuccess)                                                                         \
             return DFLASH2_ECUDA;                                                                \
-        kern<<<grid, block, dyn, s>>>(idx, logp, anchor, emb, W, G, path_tok, path_rank,         \
+        kern<<<grid, block, dyn, s>>>(idx, logp, anchor, emb, W, V, G, path_tok, path_rank,         \
                                       path_score, scores, counters);                             \
     } while (0)
     if (emb_dtype == DFLASH2_BF16) {

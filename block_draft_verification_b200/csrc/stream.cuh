@@ -22,7 +22,8 @@ enum : unsigned {
     ERR_MMA = 2u,
     ERR_EPILOGUE = 4u,
     ERR_DRAIN = 8u,
-    ERR_STREAM = 16u
+    ERR_STREAM = 16u,
+    ERR_INPUT = 32u  // a token id outside [0, V): treated as described at the call, no load
 };
 
 constexpr uint64_t WAIT_NS = 1000000000ull;  // bound on any single wait: 1 s

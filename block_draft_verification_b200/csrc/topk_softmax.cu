@@ -18,6 +18,8 @@
 // the chunk lists and softmax partials in chunk order and writes
 // idx / prob / logp / logz.  Keys compare (value, -index) exactly, so the
 // top-16 set does not depend on how the row was split.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "ring.cuh"
 #include "workspace.cuh"
@@ -337,11 +339,14 @@ unsigned dfl_errors_topk(int clear) {
     return v;
 }
 
-extern "C" int dflash2_topk_softmax_ex(const void* logits, int dtype, int64_t rows, int64_t V,
-                                       int64_t row_stride, float inv_temperature, int32_t* idx,
-                                       float* prob, float* logp, float* logz, float* row_max,
-                                       float* row_lse, void* ws, size_t ws_bytes,
-                                       dflash2_stream_t stream) {
+// The call behind every top-16 entry.  clear_first: zero the counters and
+// bounds with one memset after every check has passed (a scratch area whose
+// state a previous call may have left behind); otherwise they are zero on
+// entry (the workspace contract) unless they do not fit the control area.
+static int topk_softmax_impl(const void* logits, int dtype, int64_t rows, int64_t V,
+                             int64_t row_stride, float inv_temperature, int32_t* idx, float* prob,
+                             float* logp, float* logz, float* row_max, float* row_lse, void* ws,
+                             size_t ws_bytes, bool clear_first, dflash2_stream_t stream) {
     if (!dtype_ok(dtype)) return DFLASH2_EDTYPE;
     if (rows < 0 || V < K || V > INT32_MAX || row_stride < V) return DFLASH2_ESHAPE;
     if (!finite_pos(inv_temperature)) return DFLASH2_EINVAL;
@@ -361,7 +366,8 @@ extern "C" int dflash2_topk_softmax_ex(const void* logits, int dtype, int64_t ro
     unsigned* counters = (unsigned*)((char*)ws + L.counters_off);
     TopkPart* part = (TopkPart*)((char*)ws + L.part_off);
     unsigned* thr = counters + rows;  // the rows' shared top-16 bounds
-    if (!L.self_clean && cudaMemsetAsync(counters, 0, (size_t)rows * 8, s) != cudaSuccess)
+    if ((clear_first || !L.self_clean) &&
+        cudaMemsetAsync(counters, 0, (size_t)rows * 8, s) != cudaSuccess)
         return DFLASH2_ECUDA;
 
     // TMA bulk copies need 16-byte aligned chunk starts and 16-byte multiples
@@ -387,12 +393,21 @@ extern "C" int dflash2_topk_softmax_ex(const void* logits, int dtype, int64_t ro
     return launch_status();
 }
 
+extern "C" int dflash2_topk_softmax_ex(const void* logits, int dtype, int64_t rows, int64_t V,
+                                       int64_t row_stride, float inv_temperature, int32_t* idx,
+                                       float* prob, float* logp, float* logz, float* row_max,
+                                       float* row_lse, void* ws, size_t ws_bytes,
+                                       dflash2_stream_t stream) {
+    return topk_softmax_impl(logits, dtype, rows, V, row_stride, inv_temperature, idx, prob, logp,
+                             logz, row_max, row_lse, ws, ws_bytes, false, stream);
+}
+
 extern "C" int dflash2_topk_softmax(const void* logits, int dtype, int64_t rows, int64_t V,
                                     int64_t row_stride, float inv_temperature, int32_t* idx,
                                     float* prob, float* logp, float* logz, void* ws,
                                     size_t ws_bytes, dflash2_stream_t stream) {
-    return dflash2_topk_softmax_ex(logits, dtype, rows, V, row_stride, inv_temperature, idx, prob,
-                                   logp, logz, nullptr, nullptr, ws, ws_bytes, stream);
+    return topk_softmax_impl(logits, dtype, rows, V, row_stride, inv_temperature, idx, prob, logp,
+                             logz, nullptr, nullptr, ws, ws_bytes, false, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -408,23 +423,66 @@ namespace {
 constexpr size_t NOALLOC_SCRATCH_BYTES = DFLASH2_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 
-// Device address of the array on each device.  The host-side name of the
-// array is only a stand-in; the address a kernel can use is looked up once per
-// device, with that device current.
-constexpr int NOALLOC_MAX_DEVICES = 64;
-void* g_noalloc_addr[NOALLOC_MAX_DEVICES];
+// Device address of the array in each CUDA context.  The host-side name of
+// the array is only a stand-in; the address a kernel can use is looked up
+// (cudaGetSymbolAddress) with the context current, once per context.  The
+// cache is keyed by the context's unique id (cuCtxGetId), which no later
+// context reuses: after cudaDeviceReset, or in another context on the same
+// device, the library's module is loaded anew and the address looked up
+// again.
+constexpr int NOALLOC_MAX_CTX = 64;
+struct NoallocEntry {
+    unsigned long long ctx_id;
+    void* addr;
+};
+NoallocEntry g_noalloc_cache[NOALLOC_MAX_CTX];
+int g_noalloc_used;
 std::mutex g_noalloc_mu;
 
-void* noalloc_scratch_on_current_device() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES) return nullptr;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
+// The two driver calls, resolved through the runtime (the library does not
+// link the driver library itself).
+typedef CUresult (*PfnCtxGetCurrent)(CUcontext*);
+typedef CUresult (*PfnCtxGetId)(CUcontext, unsigned long long*);
+
+bool current_context_id(unsigned long long& id) {
+    static PfnCtxGetCurrent get_current = nullptr;
+    static PfnCtxGetId get_id = nullptr;
+    static std::once_flag resolved;
+    std::call_once(resolved, [] {
+        void* a = nullptr;
+        void* b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+            qa == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+            qb == cudaDriverEntryPointSuccess) {
+            get_current = (PfnCtxGetCurrent)a;
+            get_id = (PfnCtxGetId)b;
+        }
+    });
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, &id) == CUDA_SUCCESS;
+}
+
+void* noalloc_scratch_in_current_context() {
+    unsigned long long id = 0;
+    if (!current_context_id(id)) {
+        // no context current yet: the runtime's symbol lookup creates the
+        // device's primary context and makes it current
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-        g_noalloc_addr[dev] = p;
+        if (!current_context_id(id)) return nullptr;
     }
-    return g_noalloc_addr[dev];
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    for (int i = 0; i < g_noalloc_used; ++i)
+        if (g_noalloc_cache[i].ctx_id == id) return g_noalloc_cache[i].addr;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    const int slot = g_noalloc_used < NOALLOC_MAX_CTX ? g_noalloc_used++ : (int)(id % NOALLOC_MAX_CTX);
+    g_noalloc_cache[slot] = NoallocEntry{id, p};
+    return p;
 }
 
 }  // namespace
@@ -438,11 +496,10 @@ extern "C" int dflash2_topk_softmax_noalloc(const void* logits, int dtype, int64
     if (rows > 0 && topk_layout(rows, V, elem_size(dtype)).total > NOALLOC_SCRATCH_BYTES)
         return DFLASH2_EWORKSPACE;  // more rows than the built-in scratch holds
     if (rows == 0) return DFLASH2_OK;
-    void* scratch = noalloc_scratch_on_current_device();
+    void* scratch = noalloc_scratch_in_current_context();
     if (!scratch) return DFLASH2_ECUDA;
-    // the array's counters start at zero whatever an earlier (failed) call left
-    if (cudaMemsetAsync(scratch, 0, (size_t)rows * 8, (cudaStream_t)stream) != cudaSuccess)
-        return DFLASH2_ECUDA;
-    return dflash2_topk_softmax(logits, dtype, rows, V, row_stride, inv_temperature, idx, prob, logp,
-                                logz, scratch, NOALLOC_SCRATCH_BYTES, stream);
+    // every other argument is checked before anything is enqueued; then the
+    // array's counters are cleared (whatever an earlier, failed call left)
+    return topk_softmax_impl(logits, dtype, rows, V, row_stride, inv_temperature, idx, prob, logp,
+                             logz, nullptr, nullptr, scratch, NOALLOC_SCRATCH_BYTES, true, stream);
 }

@@ -90,7 +90,7 @@ __device__ __forceinline__ void rows_max_key(const uint64_t* P, int S, int r0, i
         }
 }
 
-__device__ __forceinline__ void greedy_finish(const uint64_t* P, int S, int G, int b,
+__device__ __forceinline__ void greedy_finish(const uint64_t* P, int S, int G, int64_t V, int b,
                                               const int32_t* __restrict__ draft_tok,
                                               int32_t* __restrict__ n_accept,
                                               int32_t* __restrict__ out_tok) {
@@ -104,6 +104,8 @@ __device__ __forceinline__ void greedy_finish(const uint64_t* P, int S, int G, i
             if (lane == r0 + j) tj = (int32_t)key_index(best[j]);
     }
     const int32_t dj = (lane < G) ? draft_tok[(int64_t)b * G + lane] : -1;
+    // a drafted token outside [0, V) never equals an argmax: a mismatch, flagged
+    if (lane < G && (uint32_t)dj >= (uint32_t)V) atomicOr(&g_dev_err, ERR_INPUT);
     const unsigned miss = __ballot_sync(FULL, lane < G && dj != tj);
     const int n = miss ? (__ffs(miss) - 1) : G;
     if (lane <= G) out_tok[(int64_t)b * (G + 1) + lane] = (lane < n) ? dj : (lane == n ? tj : -1);
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_kernel(
             if (lane == 0) last = publish(&counters[b], seg, (unsigned)((G + 1) * S));
             if (__shfl_sync(FULL, last, 0)) {
                 __syncwarp();  // lane 0's acquire covers the whole warp's reads
-                greedy_finish(part + b * (G + 1) * S, S, G, (int)b, draft_tok, n_accept, out_tok);
+                greedy_finish(part + b * (G + 1) * S, S, G, V, (int)b, draft_tok, n_accept, out_tok);
                 if (lane == 0) counters[b] = 0u;  // the sequence is done: leave its counter zero
             }
             seg = 0;
@@ -233,8 +235,11 @@ __device__ __forceinline__ void sample_finish(
     };
     // the drafted tokens and their logits first (independent of the partials)
     const int32_t dn = (lane < G) ? draft_tok[(int64_t)b * G + lane] : -1;
+    // a drafted token outside [0, V) is rejected (r = 0) without a load, and flagged
+    const bool dn_ok = lane < G && (uint32_t)dn < (uint32_t)V;
+    if (lane < G && !dn_ok) atomicOr(&g_dev_err, ERR_INPUT);
     double xt_d = 0.0, xq_d = 0.0;
-    if (lane < G) {
+    if (dn_ok) {
         xt_d = elem(target, (int64_t)b * (G + 1) + lane, dn);
         if (q_mode == DFLASH2_Q_SOFTMAX) xq_d = elem(draft, (int64_t)b * G + lane, dn);
     }
@@ -270,7 +275,7 @@ __device__ __forceinline__ void sample_finish(
         // lp = z_t[d] - logZ_t = (x - m) * invT - ln(s); likewise lq
         double lr = (xt_d - (double)lt.m) * (double)inv_t - log(lt.s);
         if (q_mode == DFLASH2_Q_SOFTMAX) lr -= (xq_d - (double)lq.m) * (double)inv_t - lnq;
-        const double ratio = exp(lr);
+        const double ratio = dn_ok ? exp(lr) : 0.0;
         const float u = philox_uniform(seed, step, sid, (uint32_t)lane, 0u);
         reject = !((double)u < ratio);
         if (ratio_dbg) ratio_dbg[(int64_t)b * G + lane] = (float)ratio;

@@ -37,8 +37,12 @@
  *     work was enqueued, except DFLASH2_ECUDA, which reports a failed launch
  *     or memset (read with cudaGetLastError, which also clears it).
  *   - Preconditions the library does not check on the device: logits,
- *     embeddings and weights are finite; token ids are in [0, V); output
- *     buffers do not overlap inputs.
+ *     embeddings and weights are finite; output buffers do not overlap
+ *     inputs.  Token ids (drafted tokens, candidate ids, the anchor) belong
+ *     in [0, V); one outside it is never used as an address: the verifies
+ *     treat it as not accepted (greedy: a mismatch; sampling: r = 0, so it
+ *     is rejected), the selector gives it a zero embedding, and the call
+ *     sets device error flag 32 (dflash2_device_errors).
  *   - Calls that take a workspace (`ws`, `ws_bytes`): a device buffer of at
  *     least dflash2_workspace_bytes(B, G, V) bytes, 256-byte aligned, used
  *     for arrival counters and per-chunk partial results.  Its first 64 KB
@@ -161,9 +165,14 @@ DFLASH2_API int dflash2_topk_softmax_ex(const void* logits, int dtype, int64_t r
  *   - Every call on a device shares the one array and leaves its contents
  *     behind: two calls that can overlap on the GPU (different streams without
  *     an ordering between them) race and give wrong results.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and keeps it; make that
- *     first call before any stream capture.
+ *   - The first call in each CUDA context looks up the array's device
+ *     address (cudaGetSymbolAddress, with that context current) and keeps it
+ *     under the context's unique id (cuCtxGetId), so a context created later
+ *     (after cudaDeviceReset, say) looks it up anew; make the first call in a
+ *     context before any stream capture.
+ *   - Every argument is checked before anything is enqueued; on DFLASH2_OK
+ *     the call enqueues one cudaMemsetAsync of the array's counters, then the
+ *     kernel.
  */
 #define DFLASH2_NOALLOC_SCRATCH_BYTES (4u << 20)
 DFLASH2_API int dflash2_topk_softmax_noalloc(const void* logits, int dtype, int64_t rows, int64_t V,
@@ -296,11 +305,14 @@ DFLASH2_API size_t dflash2_dynconv2_workspace_bytes(int dtype, int B, int T, int
 
 /*
  * Device-side error flags of the kernels on the current device (0 = none).
- * Every wait inside the kernels (on a TMA copy or a tensor-core MMA) is
- * bounded to one second; a wait that runs out sets a flag bit (1 producer,
- * 2 MMA issuer, 4 epilogue, 8 drain, 16 streamed copy), the kernel waits
- * (bounded) for its own copies in flight, releases its tensor memory and
- * returns, and the call's outputs are not valid.  Synchronous (reads device
+ * Every wait inside the kernels (on a TMA copy, a tensor-core MMA, or
+ * another CTA's result in the same launch) is bounded to one second; a wait
+ * that runs out sets a flag bit (1 producer, 2 MMA issuer, 4 epilogue,
+ * 8 drain, 16 streamed copy or cross-CTA wait), the kernel waits (bounded)
+ * for its own copies in flight, releases its tensor memory and returns, and
+ * the call's outputs are not valid; zero the workspace's first 64 KB before
+ * reusing it.  Bit 32: a token id was outside [0, V) (see the conventions
+ * above; the outputs follow the stated rule).  Synchronous (reads device
  * memory); clear != 0 resets the flags.  Returns 0xFFFFFFFF if the flags
  * cannot be read.
  */

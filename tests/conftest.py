@@ -18,3 +18,20 @@ def orc():
     import oracle
     oracle.lib()
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter):
+    """One line with every near-tie the parity tests excused (accept flips with
+    |u - r| < 1e-6, draw picks within 1e-6 R, Viterbi paths within the score
+    band), per kind, beside the number of decisions compared."""
+    try:
+        from parity import SESSION_COMPARED, SESSION_NEAR_TIES
+    except Exception:
+        return
+    if not SESSION_COMPARED and not SESSION_NEAR_TIES:
+        return
+    kinds = sorted(set(SESSION_COMPARED) | set(SESSION_NEAR_TIES))
+    terminalreporter.write_line(
+        "near-ties excused: " + ", ".join(
+            "%s %d of %d" % (k, SESSION_NEAR_TIES.get(k, 0), SESSION_COMPARED.get(k, 0))
+            for k in kinds))

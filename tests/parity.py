@@ -62,6 +62,17 @@ def assert_close(gpu_vals, oracle_vals, rtol, what=""):
                              % (what, bad.sum(), bad.size, rtol, i, g.ravel()[i], o.ravel()[i]))
 
 
+# Every near-tie excused in this test session, per kind (printed at the end of
+# the run by conftest.py, so the counts are part of the run's record).
+SESSION_NEAR_TIES = {}
+SESSION_COMPARED = {}
+
+
+def count_compared(kind, n):
+    """Record n integer decisions of `kind` compared with the oracle."""
+    SESSION_COMPARED[kind] = SESSION_COMPARED.get(kind, 0) + int(n)
+
+
 class NearTies:
     """Counts mismatches that the stated bands excuse; anything else fails."""
 
@@ -70,6 +81,7 @@ class NearTies:
 
     def add(self, kind, n=1):
         self.counts[kind] = self.counts.get(kind, 0) + n
+        SESSION_NEAR_TIES[kind] = SESSION_NEAR_TIES.get(kind, 0) + n
 
     def report(self):
         return ", ".join("%s=%d" % kv for kv in sorted(self.counts.items())) or "none"

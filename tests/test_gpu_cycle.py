@@ -9,7 +9,7 @@ import torch
 
 import block_draft_verification_b200 as dfl
 import synth
-from parity import ACCEPT_BAND, DRAW_BAND, PATH_BAND, NearTies, gpu, need_cuda, to_dev, to_host
+from parity import count_compared, ACCEPT_BAND, DRAW_BAND, PATH_BAND, NearTies, gpu, need_cuda, to_dev, to_host
 
 pytestmark = gpu
 
@@ -45,6 +45,10 @@ def test_chained_cycle(orc, name, sampling):
         on, oout = orc.verify_greedy(b.target, otok)
         macc = mres = np.zeros(B)
     ties = NearTies()
+    count_compared("path", B)
+    count_compared("accept" if sampling else "greedy", B)
+    if sampling:
+        count_compared("draw", B)
     for s in range(B):
         if not np.array_equal(rank[s], orank[s]):
             re = orc.path_rescore(oidx[s:s + 1], ologp[s:s + 1], b.anchor[s:s + 1], sel.emb, sel.W,

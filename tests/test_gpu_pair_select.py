@@ -13,7 +13,7 @@ import torch
 
 import block_draft_verification_b200 as dfl
 import synth
-from parity import PATH_BAND, RTOL_F32, NearTies, assert_close, gpu, need_cuda, to_dev, to_host
+from parity import count_compared, PATH_BAND, RTOL_F32, NearTies, assert_close, gpu, need_cuda, to_dev, to_host
 
 pytestmark = gpu
 
@@ -35,6 +35,7 @@ def run_and_check(orc, idx, logp, anchor, emb, W, ties=None):
     otok, orank, oscore = orc.pair_select(idx, logp, anchor, emb, W)
     assert_close(score, oscore, RTOL_F32, "path_score")
     ties = ties if ties is not None else NearTies()
+    count_compared("path", len(rank))
     diff = np.flatnonzero((rank != orank).any(axis=1))
     if diff.size:
         resc = orc.path_rescore(idx[diff], logp[diff], None if anchor is None else anchor[diff],

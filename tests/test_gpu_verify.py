@@ -15,7 +15,7 @@ import torch
 
 import block_draft_verification_b200 as dfl
 import synth
-from parity import (ACCEPT_BAND, DRAW_BAND, RTOL_F32, NearTies, assert_close, gpu, need_cuda,
+from parity import (ACCEPT_BAND, count_compared, DRAW_BAND, RTOL_F32, NearTies, assert_close, gpu, need_cuda,
                     to_dev, to_host)
 
 pytestmark = gpu
@@ -135,6 +135,8 @@ def check_sample(orc, target, draft, draft_tok, seed, step, seq_id=None, invT=1.
                                                          seq_id, invT, q_mode)
     np.testing.assert_array_equal(u.astype(np.float64), ou)       # Philox: bit-identical
     assert_close(ratio, oratio, RTOL_F32, "ratio")
+    count_compared("accept", len(n))
+    count_compared("draw", len(n))
     for b in range(len(n)):
         if n[b] != on[b]:
             assert macc[b] < ACCEPT_BAND, (b, n[b], on[b], macc[b])
@@ -336,6 +338,8 @@ def test_sample_many_sequences_memset_control(orc, fused):
         torch.cuda.synchronize()
         n, out = to_host(n), to_host(out)
         on, oout, _, _, macc, mres = orc.verify_sample(t, q, d, 77, step, None, 1.0, 0)
+        count_compared("accept", B)
+        count_compared("draw", B)
         for s in range(B):
             if n[s] != on[s]:
                 assert macc[s] < ACCEPT_BAND, (s, n[s], on[s])

@@ -1,6 +1,7 @@
 """dflash2_topk_softmax_noalloc, the allocation-free top-16 entry point, called
 through the C ABI and checked against dflash2_topk_softmax (the entry point
-that takes a caller workspace) on the same inputs.
+that takes a caller workspace) on the same inputs, and against the CPU oracle
+directly (indices bit-exact, probabilities within 1e-5 relative).
 
 It exists for callers that cannot give this library device memory: an
 inference engine that reserved nearly all of the GPU for its own pools and
@@ -56,18 +57,28 @@ def _same(got, ref):
     assert_close(gz, rz, RTOL_F32, "logz")
 
 
+def _matches_oracle(got, host_rows, inv_t, orc):
+    gi, gp, gl, gz = (to_host(t) for t in got)
+    oi, op, ol, oz = orc.topk_softmax(host_rows, inv_t)
+    np.testing.assert_array_equal(gi, oi)
+    assert_close(gp, op, RTOL_F32, "prob vs oracle")
+    assert_close(gl, ol, RTOL_F32, "logp vs oracle")
+    assert_close(gz, oz, RTOL_F32, "logz vs oracle")
+
+
 @pytest.mark.parametrize("name,B", [("tiny", 1), ("b32", 4)])
-def test_noalloc_matches_workspace_entry_on_two_calls(name, B):
+def test_noalloc_matches_workspace_entry_on_two_calls(name, B, orc):
     need_cuda()
     w = synth.WORKLOADS[name]
-    first = to_dev(synth.gen_batch(w, B=B).draft.reshape(-1, w.V))
-    second = to_dev(synth.gen_batch(w, B=B, first=B).draft.reshape(-1, w.V))
-    for x in (first, second):
+    hosts = [synth.gen_batch(w, B=B, first=f).draft.reshape(-1, w.V) for f in (0, B)]
+    for host_rows in hosts:
+        x = to_dev(host_rows)
         ref = dfl.topk_softmax(x, w.inv_temperature)
         got = _noalloc(x, w.inv_temperature)
         torch.cuda.synchronize()
         assert dfl.device_errors() == 0
         _same(got, ref)
+        _matches_oracle(got, host_rows, w.inv_temperature, orc)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
@@ -80,3 +91,27 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
                   C.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert rc == EWORKSPACE
     torch.cuda.synchronize()
+
+
+def test_noalloc_refuses_bad_arguments_then_works(orc):
+    """Bad scalars, pointers and alignment are refused with the same codes as
+    the workspace entry; a correct call right after is still correct."""
+    need_cuda()
+    w = synth.WORKLOADS["tiny"]
+    host_rows = synth.gen_batch(w, B=1, first=3).draft.reshape(-1, w.V)
+    x = to_dev(host_rows)
+    out = torch.empty(64, dtype=torch.float32, device="cuda")
+    p = C.c_void_p(out.data_ptr())
+    h = C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rows, V = x.shape
+    bad = [
+        (C.c_void_p(x.data_ptr()), 0, rows, V, V, float("nan"), p, p, p, p, h),  # EINVAL
+        (C.c_void_p(x.data_ptr()), 0, rows, V, V, 1.0, None, p, p, p, h),          # EINVAL
+        (C.c_void_p(x.data_ptr() + 2), 0, rows, V, V, 1.0, p, p, p, p, h),         # EALIGN
+        (C.c_void_p(x.data_ptr()), 7, rows, V, V, 1.0, p, p, p, p, h),             # EDTYPE
+    ]
+    assert [_entry()(*a) for a in bad] == [1, 1, 6, 2]
+    got = _noalloc(x, w.inv_temperature)
+    torch.cuda.synchronize()
+    assert dfl.device_errors() == 0
+    _matches_oracle(got, host_rows, w.inv_temperature, orc)
