@@ -3,30 +3,36 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     (N > 1: launched one rank per GPU by torch.distributed.run)
 
-Workload: the concurrency-32 case -- 32 sequences, block 8 (7 drafted
+Headline workload: the concurrency-32 case -- 32 sequences, block 8 (7 drafted
 positions + 1 bonus row), vocabulary 151,936, bf16 logits, selector
 embeddings 151,936 x 128 bf16 and W 128 x 128 fp32, dynconv hidden 5,120 over
-32 x 8 tokens; seeded synthetic inputs of that shape (synth "b32").
+32 x 8 tokens; seeded synthetic inputs of that shape (synth "b32").  The
+concurrency-1 and -8 cases and the block-16 context-reproduction case (b1, b8,
+ctx16) are measured the same way and reported under "workloads".
 
-One step = the whole path over one batch, each call through the C ABI:
-  dflash2_topk_softmax_ex (224 draft rows, with their normalisers) ->
+One cycle (the unit of `value`) = every call of the hot path once over one
+batch, each through the C ABI:
+  dflash2_topk_softmax_ex (the draft rows, with their normalisers) ->
   dflash2_pair_select -> dflash2_verify_sample_ex (Philox, softmax q from the
-  drafter normalisers: the fused cycle, draft rows not streamed again) ->
-  dflash2_verify_greedy -> dflash2_dynconv2.
-value = steps per second over all ranks (each rank runs its own batch:
-weak scaling, no collective on the data path), from K whole steps run back to
-back between two CUDA events (each step captured once in a CUDA graph).  A
-step reads ~344 MB of inputs, more than the 126 MB L2: two input sets
-alternate between steps and the greedy verify reads the other set's target
-rows, so no call finds its streamed rows in L2.  The per-call breakdown
-("calls", and the roofline of the dominant call) is a second pass: L2 is
-flushed by a 256 MB write followed by a read of the same buffer (no dirty
-lines left) before every call, each call timed alone with CUDA events, the
-flushes outside the timed intervals.
+  drafter normalisers: the fused cycle) -> dflash2_verify_greedy ->
+  dflash2_dynconv2.
+value = such cycles per second over all ranks (each rank runs its own batch:
+weak scaling, no collective on the data path), from K whole cycles captured
+back to back in one CUDA graph and replayed once between two CUDA events on
+the launching stream.  Every call in that graph is bracketed by event nodes,
+so each call's mean device time comes from the same timed region ("calls";
+the roofline of the call with the largest share).  A cycle reads ~344 MB of
+inputs at b32, more than the 126 MB L2: two input sets alternate between
+cycles and the greedy verify reads the other set's target rows, so no call
+finds its streamed rows in L2.  The draft-select-verify cycles the metric
+names (sampling: topk_ex -> pair_select -> verify_sample_ex; greedy: topk ->
+pair_select -> verify_greedy) and dynconv alone are timed the same way, each
+as a graph of K of its own cycles ("cycles").  A last pass times each call
+alone with L2 flushed before it ("calls_isolated").
 
 --impl reference times the CPU oracle (the plain fp64 restatement the tests
-check against) on the same workload, metric and unit, one sequence of the
-batch per step, on rank 0 only.
+check against) on whole cycles of the same workload, its sequences spread
+over the host's cores, on rank 0 only.
 """
 import argparse
 import hashlib
@@ -43,8 +49,26 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "draft-select-verify cycles/sec and HBM GB/s (% of peak) at B=1/8/32, V=151936"
-WORKLOAD = "b32"
+HEADLINE = "b32"
+OTHER_WORKLOADS = ("b1", "b8", "ctx16")
 FLUSH_BYTES = 256 << 20
+CALLS = ("topk_softmax", "pair_select", "verify_sample", "verify_greedy", "dynconv2")
+CYCLE_KINDS = ("sampling", "greedy", "greedy_early_exit", "sampling_truncated", "dynconv2")
+CYCLE_DEF = ("topk_softmax_ex -> pair_select -> verify_sample_ex -> verify_greedy -> dynconv2 "
+             "over one batch (every hot-path call once)")
+DESCRIBE = {
+    "b32": "concurrency-32: B=32, block 8 (7 drafted + 1 bonus), V=151936, bf16 logits, per-"
+           "sequence draft noise for mean acceptance 3.5-5.5, selector d=128 (emb 151936x128 "
+           "bf16, W fp32), sampling at T=1.0 (fused cycle) and greedy verify, dynconv H=5120 "
+           "over 32x8 tokens",
+    "b1": "concurrency-1: B=1, block 8, V=151936, bf16 logits, draft noise for mean acceptance "
+          "4.8, selector d=128, dynconv H=5120 over 8 tokens",
+    "b8": "concurrency-8: B=8, block 8, V=151936, bf16 logits, sampling at T=1.0 with per-"
+          "sequence Philox streams, selector d=128, dynconv H=5120 over 8x8 tokens",
+    "ctx16": "context reproduction: B=8, block 16 (15 drafted + 1), V=151936, bf16 logits, draft "
+             "noise 0.05, spike +20, selector d=128 (16x16 lattice), dynconv H=5120 over 8x16 "
+             "tokens",
+}
 
 
 def parse():
@@ -55,16 +79,23 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-graph", action="store_true",
-                    help="time the step with eager launches instead of CUDA graph replays")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="measure the headline workload only (no b1 / b8 / ctx16)")
     ap.add_argument("--acceptance", action="store_true",
                     help="print the acceptance study (mean accepted tokens per verify step for "
                          "the top-1 path, the pair selector and the top-16 oracle path) instead "
                          "of a bench line")
-    ap.add_argument("--only", choices=["topk_softmax", "pair_select", "verify_sample",
-                                       "verify_greedy", "dynconv2"], default=None,
-                    help="run and time one call of the step only (for profiling); prints a "
-                         "per-call line, not a bench line")
+    ap.add_argument("--drafter-layer", action="store_true",
+                    help="print the share of a random-weight drafter layer's time taken by the "
+                         "two-tap convs placed before and after its attention and MLP, instead "
+                         "of a bench line")
+    ap.add_argument("--select-sweep", action="store_true",
+                    help="print the pair selector's time for both implementations (CUDA cores, "
+                         "tensor cores) over a range of batch sizes, L2 flushed before every "
+                         "call, instead of a bench line")
+    ap.add_argument("--only", choices=list(CALLS), default=None,
+                    help="run and time one call of the headline workload only (for profiling); "
+                         "prints a per-call line, not a bench line")
     return ap.parse_args()
 
 
@@ -89,6 +120,13 @@ def algorithmic_bytes(w, B):
         "verify_greedy": 2 * B * (G + 1) * V + B * G * 4 + B * (G + 2) * 4,
         "dynconv2": 2 * (2 * H * H) + 2 * 2 * B * T * H + 2 * B * H,
     }
+
+
+def usable_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
 
 
 # --------------------------------------------------------------------------- clocks
@@ -168,44 +206,138 @@ def recorded_traffic(kernel):
 
 
 # --------------------------------------------------------------------------- CPU oracle
-def oracle_step_seconds(w, batch, sel, conv, seqs):
-    """The oracle's whole path for the given sequences of the batch (seconds)."""
+# Worker side (spawned processes, no CUDA).  The batch lives in shared memory
+# written once by the parent; the weights are regenerated once per worker from
+# their seeds.
+_WORKER = {}
+
+
+def _attach(desc):
+    from multiprocessing import shared_memory
+    out, keep = {}, []
+    for k, (shm_name, shape, dt) in desc.items():
+        shm = shared_memory.SharedMemory(name=shm_name)
+        keep.append(shm)
+        out[k] = np.ndarray(shape, dtype=np.dtype(dt), buffer=shm.buf)
+    return out, keep
+
+
+def _worker_init(name, desc):
+    import synth
+    w = _WORKER["w"] = synth.WORKLOADS[name]
+    _WORKER["arr"], _WORKER["keep"] = _attach(desc)
+    _WORKER["sel"] = synth.gen_selector(w)
+    _WORKER["wtap"] = synth.gen_conv_weights(w)
+
+
+class SharedBatch:
+    """Input set 0 of a workload (logits, anchors, seq ids, dynconv inputs) in
+    shared memory for the oracle's worker processes."""
+
+    def __init__(self, name):
+        from multiprocessing import shared_memory
+        import synth
+        w = synth.WORKLOADS[name]
+        b, c = synth.gen_batch(w), synth.gen_conv(w)
+        arrays = dict(target=b.target, draft=b.draft, anchor=b.anchor, seq_id=b.seq_id,
+                      x=c.x, x_prev=c.x_prev)
+        self.shm, self.desc = [], {}
+        for k, a in arrays.items():
+            a = np.ascontiguousarray(a)
+            shm = shared_memory.SharedMemory(create=True, size=max(1, a.nbytes))
+            np.ndarray(a.shape, a.dtype, buffer=shm.buf)[...] = a
+            self.shm.append(shm)
+            self.desc[k] = (shm.name, a.shape, a.dtype.str)
+
+    def close(self):
+        for shm in self.shm:
+            shm.close()
+            shm.unlink()
+        self.shm = []
+
+
+def oracle_sequence(s, step=0, collect=False):
+    """The oracle's whole path for sequence s of the shared batch: top-16 ->
+    selector -> sampling verify (Philox step `step`) -> greedy verify ->
+    dynconv of its tokens.  Returns (seconds, outputs or None)."""
     import oracle
+    w, a, sel, wtap = _WORKER["w"], _WORKER["arr"], _WORKER["sel"], _WORKER["wtap"]
+    tgt, drf = a["target"][s:s + 1], a["draft"][s:s + 1]
+    anchor, sid = a["anchor"][s:s + 1], a["seq_id"][s:s + 1]
     t0 = time.perf_counter()
-    for s in seqs:
-        idx, _, logp, _ = oracle.topk_softmax(batch.draft[s], w.inv_temperature)
-        tok, _, _ = oracle.pair_select(idx[None], logp.astype(np.float32)[None],
-                                       batch.anchor[s:s + 1], sel.emb, sel.W)
-        oracle.verify_sample(batch.target[s:s + 1], batch.draft[s:s + 1], tok, w.seed, 0,
-                             batch.seq_id[s:s + 1], w.inv_temperature)
-        oracle.verify_greedy(batch.target[s:s + 1], tok)
-        oracle.dynconv2(conv.x[s:s + 1], conv.x_prev[s:s + 1], conv.w_tap)
-    return time.perf_counter() - t0
+    idx, _, logp, _ = oracle.topk_softmax(drf[0], w.inv_temperature)
+    lp = logp.astype(np.float32)[None]
+    tok, rank, score = oracle.pair_select(idx[None], lp, anchor, sel.emb, sel.W)
+    sn, sout, _, _, macc, mres = oracle.verify_sample(tgt, drf, tok, w.seed, step, sid,
+                                                      w.inv_temperature)
+    gn, gout = oracle.verify_greedy(tgt, tok)
+    oracle.dynconv2(a["x"][s:s + 1], a["x_prev"][s:s + 1], wtap)
+    sec = time.perf_counter() - t0
+    if not collect:
+        return sec, None
+    return sec, dict(seq=s, idx=idx, logp=lp[0], anchor=int(anchor[0]), rank=rank[0],
+                     score=float(score[0]), sn=int(sn[0]), sout=sout[0], macc=float(macc[0]),
+                     mres=float(mres[0]), gn=int(gn[0]), gout=gout[0])
+
+
+def _oracle_task(args):
+    s, step, collect = args
+    return oracle_sequence(s, step, collect)
+
+
+class OraclePool:
+    """Spawned worker processes (no CUDA) that run the oracle on the shared
+    batch of a workload, one sequence per task."""
+
+    def __init__(self, name, procs):
+        import multiprocessing as mp
+        self.procs = procs
+        self.batch = SharedBatch(name)
+        self.pool = mp.get_context("spawn").Pool(processes=procs, initializer=_worker_init,
+                                                 initargs=(name, self.batch.desc))
+
+    def cycle(self, seqs, step=0, collect=False):
+        """Wall seconds of the oracle over `seqs` spread over the workers,
+        and the per-sequence (seconds, results)."""
+        t0 = time.perf_counter()
+        res = self.pool.map(_oracle_task, [(s, step, collect) for s in seqs], chunksize=1)
+        return time.perf_counter() - t0, res
+
+    def close(self):
+        self.pool.terminate()
+        self.pool.join()
+        self.batch.close()
 
 
 def run_reference(args, rank, world):
+    """The CPU oracle on whole cycles of the headline workload (all 32
+    sequences per cycle, spread over the host's cores), rank 0 only."""
     import synth
     if rank != 0:
         return
-    w = synth.WORKLOADS[WORKLOAD]
-    batch = synth.gen_batch(w)
-    sel = synth.gen_selector(w)
-    conv = synth.gen_conv(w)
-    for i in range(args.warmup):
-        oracle_step_seconds(w, batch, sel, conv, [i % w.B])
-    times = [oracle_step_seconds(w, batch, sel, conv, [i % w.B]) for i in range(args.steps)]
-    per_seq = float(np.mean(times))
-    value = 1.0 / (per_seq * w.B)                 # full 32-sequence steps per second
-    sample = "one of the 32 sequences per step (its 7 draft rows, 8 target rows, selector, " \
-             "both verifies and its 8 dynconv tokens), scaled by 32"
+    w = synth.WORKLOADS[HEADLINE]
+    procs = max(1, min(usable_cores(), w.B))
+    pool = OraclePool(HEADLINE, procs)
+    try:
+        seqs = list(range(w.B))
+        pool.cycle(list(range(procs)))  # every worker initialised
+        for _ in range(args.warmup):
+            pool.cycle(seqs)
+        times = [pool.cycle(seqs)[0] for _ in range(args.steps)]
+    finally:
+        pool.close()
+    per_cycle = float(np.mean(times))
+    value = 1.0 / per_cycle
+    sample = ("whole cycles: all 32 sequences of the batch per cycle (7 draft rows, 8 target "
+              "rows, selector, sampling and greedy verify, 8 dynconv tokens each), the "
+              "sequences spread over %d worker processes, timed by wall clock" % procs)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "cycles/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": per_seq * w.B * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": per_cycle * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "concurrency-32: B=32, block 8, V=151936, bf16 logits, "
-                                   "d=128 selector, dynconv H=5120 x 32x8 tokens",
-                       "parallelism": "rank 0 only (CPU)"},
-            "cpu_baseline": {"value": value, "unit": "cycles/s", "cores": 1, "kind": "oracle",
+            "config": {"workload": DESCRIBE[HEADLINE], "cycle": CYCLE_DEF,
+                       "parallelism": "rank 0 only (CPU, %d processes)" % procs},
+            "cpu_baseline": {"value": value, "unit": "cycles/s", "cores": procs, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "cycles/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -273,6 +405,140 @@ def run_acceptance(args):
           flush=True)
 
 
+# --------------------------------------------------------------------------- drafter layer
+def run_drafter_layer(args):
+    """The two-tap conv inside a drafter layer (tamsi page, "L'idée, sans le
+    papier": a conv before and after each attention and MLP, +0.7 % latency):
+    one random-weight bf16 decoder layer over the headline batch's tokens
+    (B = 32 sequences x 8 block tokens, hidden 5,120, 40 heads of 128,
+    attention within each block, gated MLP of width 3 x 5,120), timed as CUDA
+    graph replays with and without the four dflash2_dynconv2 calls (each with
+    its own tap weights [2H, H]).  The layer's projections and attention are
+    PyTorch (cuBLAS, SDPA): context for the share, not the product."""
+    import torch
+    import torch.nn.functional as F
+
+    import block_draft_verification_b200 as dfl
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev).manual_seed(20261202)
+    B, T, H, nh = 32, 8, 5120, 40
+    hd, I = H // nh, 3 * H
+    bf = torch.bfloat16
+
+    def w(*shape, scale):
+        return (torch.randn(*shape, device=dev, generator=g) * scale).to(bf)
+
+    x0 = w(B, T, H, scale=1.0)
+    wqkv, wo = w(3 * H, H, scale=H ** -0.5), w(H, H, scale=H ** -0.5)
+    wgu, wd = w(2 * I, H, scale=H ** -0.5), w(H, I, scale=I ** -0.5)
+    taps = [w(2 * H, H, scale=H ** -0.5) for _ in range(4)]
+    xprev = [w(B, H, scale=1.0) for _ in range(4)]
+    ln1, ln2 = torch.ones(H, device=dev, dtype=bf), torch.ones(H, device=dev, dtype=bf)
+    outs = [torch.empty(B, T, H, device=dev, dtype=bf) for _ in range(4)]
+    ws = dfl.Workspace(dev, dfl.lib().dflash2_dynconv2_workspace_bytes(1, B, T, H))
+
+    def conv(x, i, on):
+        return dfl.dynconv2(x, xprev[i], taps[i], out=outs[i], ws=ws) if on else x
+
+    def layer(x, on):
+        h = conv(x, 0, on)
+        a = F.rms_norm(h, (H,), ln1)
+        q, k, v = (a @ wqkv.t()).view(B, T, 3, nh, hd).permute(2, 0, 3, 1, 4)
+        o = F.scaled_dot_product_attention(q, k, v).transpose(1, 2).reshape(B, T, H) @ wo.t()
+        h = conv(h + o, 1, on)
+        h = conv(h, 2, on)
+        m = F.rms_norm(h, (H,), ln2) @ wgu.t()
+        gte, up = m.chunk(2, dim=-1)
+        h = h + (F.silu(gte) * up) @ wd.t()
+        return conv(h, 3, on)
+
+    K = max(args.steps, 20)
+    res = {}
+    for on in (False, True):
+        stream = torch.cuda.Stream(dev)
+        stream.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                layer(x0, on)
+        torch.cuda.synchronize(dev)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for _ in range(K):
+                y = layer(x0, on)
+        gr.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        gr.replay()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        res[on] = e0.elapsed_time(e1) / K * 1e3
+        del gr
+    conv_bytes = 4 * (2 * (2 * H * H) + 2 * 2 * B * T * H + 2 * B * H)
+    layer_w_bytes = 2 * (4 * H * H + 3 * H * I)
+    print(json.dumps({
+        "drafter_layer": {"tokens": B * T, "hidden": H, "heads": nh, "mlp": I,
+                          "us_without_convs": round(res[False], 2),
+                          "us_with_convs": round(res[True], 2),
+                          "conv_share": round((res[True] - res[False]) / res[True], 4),
+                          "conv_bytes": conv_bytes, "layer_weight_bytes": layer_w_bytes},
+        "pages": "+0.7 % of the cycle for the convs (a conv adding ~3 % params); here each conv "
+                 "has a dense [2H, H] tap (the tiny configuration's 256 -> 512 form), so the "
+                 "four convs stream ~%.0f MB against the layer's %.0f MB of weights"
+                 % (conv_bytes / 1e6, layer_w_bytes / 1e6)}), flush=True)
+
+
+# --------------------------------------------------------------------------- selector sweep
+def run_select_sweep(args):
+    """dflash2_pair_select_ex with each implementation over B = 1 .. 256
+    (block 8, V = 151,936, d = 128 bf16 table, fp32 W; random candidate lists
+    and log-probabilities: the cost does not depend on the values), each call
+    timed alone with CUDA events after a 256 MB L2 flush."""
+    import torch
+
+    import block_draft_verification_b200 as dfl
+    import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS["b32"]
+    sel = synth.gen_selector(w)
+    E = torch.from_numpy(sel.emb.view(np.int16)).to(dev).view(torch.bfloat16)
+    Wd = torch.from_numpy(sel.W).to(dev)
+    G, V = w.G, w.V
+    g = torch.Generator(device=dev).manual_seed(7)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    sink = torch.zeros((), dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for B in (1, 2, 4, 8, 16, 32, 64, 128, 256):
+        idx = torch.randint(0, V, (B, G, 16), device=dev, generator=g, dtype=torch.int32)
+        logp = -torch.rand((B, G, 16), device=dev, generator=g) * 8
+        anchor = torch.randint(0, V, (B,), device=dev, generator=g, dtype=torch.int32)
+        ws = dfl.Workspace(dev, dfl.workspace_bytes(B, G, V))
+        row = {}
+        for impl, label in ((dfl.SELECT_SIMT, "simt"), (dfl.SELECT_TENSOR, "tensor")):
+            for _ in range(3):
+                dfl.pair_select(idx, logp, anchor, E, Wd, ws=ws, impl=impl)
+            ts = []
+            for i in range(max(args.steps, 10)):
+                flush.fill_(i & 0xFF)
+                sink.add_(flush.view(torch.int64).sum())
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                dfl.pair_select(idx, logp, anchor, E, Wd, ws=ws, impl=impl)
+                e1.record(stream)
+                ts.append((e0, e1))
+            torch.cuda.synchronize(dev)
+            row[label] = round(float(np.median([a.elapsed_time(b) for a, b in ts])) * 1e3, 2)
+        out[B] = row
+    print(json.dumps({"pair_select_us_by_batch": out, "block": 8, "d": 128,
+                      "timing": "median CUDA-event time per call, L2 flushed before each"}),
+          flush=True)
+
+
 # --------------------------------------------------------------------------- ranks
 def rank_first_sequence(rank, k, B):
     """First sequence of input set k (0 or 1) on a rank: every (rank, set)
@@ -293,288 +559,504 @@ def max_over_ranks(values, world, device):
 
 
 # --------------------------------------------------------------------------- GPU
-def run_ours(args, rank, world, local_rank):
-    import torch
-    import torch.distributed as dist
+class Bench:
+    """One workload on one device: two input sets, the weights, the outputs,
+    one workspace, and the calls of a cycle as closures over them."""
 
-    import block_draft_verification_b200 as dfl
-    import synth
+    def __init__(self, name, rank, dev):
+        import torch
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w = synth.WORKLOADS[WORKLOAD]
-    B, G, V = w.B, w.G, w.V
+        import block_draft_verification_b200 as dfl
+        import synth
+        self.torch, self.dfl, self.synth = torch, dfl, synth
+        self.name, self.dev = name, dev
+        w = self.w = synth.WORKLOADS[name]
+        B, G, V = self.B, self.G, self.V = w.B, w.G, w.V
+        self.sets = [(synth.gen_batch(w, first=rank_first_sequence(rank, k, B)),
+                      synth.gen_conv(w, first=rank_first_sequence(rank, k, B)))
+                     for k in range(2)]
+        self.sel = synth.gen_selector(w)
+        self.E, self.Wsel, self.Wtap = (self.dev_t(self.sel.emb), self.dev_t(self.sel.W),
+                                        self.dev_t(self.sets[0][1].w_tap))
+        self.inputs = []
+        for b, c in self.sets:
+            self.inputs.append(dict(
+                T=self.dev_t(b.target), Q=self.dev_t(b.draft), anchor=self.dev_t(b.anchor),
+                sid=self.dev_t(b.seq_id.view(np.int32)), x=self.dev_t(c.x), xp=self.dev_t(c.x_prev),
+                topk=self.topk_out()))  # per input set: the normalisers stay with their rows
+        self.ws = dfl.Workspace(dev, dfl.workspace_bytes(B, G, V) + dfl.workspace_bytes(B * G, 1, V))
+        i32, f32 = torch.int32, torch.float32
+        self.outs = dict(
+            sel=(torch.empty((B, G), dtype=i32, device=dev), torch.empty((B, G), dtype=i32, device=dev),
+                 torch.empty((B,), dtype=f32, device=dev)),
+            samp=(torch.empty((B,), dtype=i32, device=dev),
+                  torch.empty((B, G + 1), dtype=i32, device=dev)),
+            greedy=(torch.empty((B,), dtype=i32, device=dev),
+                    torch.empty((B, G + 1), dtype=i32, device=dev)),
+            conv=torch.empty((B, w.T, w.H), dtype=torch.bfloat16, device=dev),
+        )
 
-    # inputs: two input sets per rank (alternated between steps), weights once
-    sets = [(synth.gen_batch(w, first=rank_first_sequence(rank, k, B)),
-             synth.gen_conv(w, first=rank_first_sequence(rank, k, B)))
-            for k in range(2)]
-    sel = synth.gen_selector(w)
-    wtap = sets[0][1].w_tap
-
-    def dev_t(a):
+    def dev_t(self, a):
+        torch = self.torch
         a = np.ascontiguousarray(a)
         if a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
-        return torch.from_numpy(a).to(dev)
+            return torch.from_numpy(a.view(np.int16)).to(self.dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(self.dev)
 
-    E, Wsel, Wtap = dev_t(sel.emb), dev_t(sel.W), dev_t(wtap)
-    inputs = []
-    for b, c in sets:
-        inputs.append(dict(T=dev_t(b.target), Q=dev_t(b.draft), anchor=dev_t(b.anchor),
-                           sid=dev_t(b.seq_id.view(np.int32)), x=dev_t(c.x), xp=dev_t(c.x_prev)))
-    ws = dfl.Workspace(dev, dfl.workspace_bytes(B, G, V) + dfl.workspace_bytes(B * G, 1, V))
-    def topk_out():
-        return (torch.empty((B * G, 16), dtype=torch.int32, device=dev),
-                torch.empty((B * G, 16), dtype=torch.float32, device=dev),
-                torch.empty((B * G, 16), dtype=torch.float32, device=dev),
-                torch.empty((B * G,), dtype=torch.float32, device=dev),
-                torch.empty((B * G,), dtype=torch.float32, device=dev),
-                torch.empty((B * G,), dtype=torch.float32, device=dev))
+    def topk_out(self):
+        torch, n = self.torch, self.B * self.G
+        return (torch.empty((n, 16), dtype=torch.int32, device=self.dev),
+                torch.empty((n, 16), dtype=torch.float32, device=self.dev),
+                torch.empty((n, 16), dtype=torch.float32, device=self.dev),
+                torch.empty((n,), dtype=torch.float32, device=self.dev),
+                torch.empty((n,), dtype=torch.float32, device=self.dev),
+                torch.empty((n,), dtype=torch.float32, device=self.dev))
 
-    for k, inp in enumerate(inputs):
-        inp["topk"] = topk_out()  # per input set: the normalisers stay with their rows
-    outs = dict(
-        sel=(torch.empty((B, G), dtype=torch.int32, device=dev),
-             torch.empty((B, G), dtype=torch.int32, device=dev),
-             torch.empty((B,), dtype=torch.float32, device=dev)),
-        samp=(torch.empty((B,), dtype=torch.int32, device=dev),
-              torch.empty((B, G + 1), dtype=torch.int32, device=dev)),
-        greedy=(torch.empty((B,), dtype=torch.int32, device=dev),
-                torch.empty((B, G + 1), dtype=torch.int32, device=dev)),
-        conv=torch.empty((B, w.T, w.H), dtype=torch.bfloat16, device=dev),
-    )
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    flush_sink = torch.zeros((), dtype=torch.int64, device=dev)
-    names = ["topk_softmax", "pair_select", "verify_sample", "verify_greedy", "dynconv2"]
-    kernels_per_step = {"topk_softmax": 1, "pair_select": 1, "verify_sample": 1,
-                        "verify_greedy": 1, "dynconv2": 1}
-
-    def calls(inp, step, t_greedy=None):
-        tk = inp["topk"]
-        tg = inp["T"] if t_greedy is None else t_greedy
+    def calls(self, k, step, greedy_other_set=True):
+        """The five calls of a cycle on input set k, as (name, fn)."""
+        dfl, w, B, G, V = self.dfl, self.w, self.B, self.G, self.V
+        inp, tk, outs, ws = self.inputs[k], self.inputs[k]["topk"], self.outs, self.ws
+        tg = self.inputs[1 - k]["T"] if greedy_other_set else inp["T"]
         return [
-            lambda: dfl.topk_softmax(inp["Q"].view(B * G, V), w.inv_temperature, out=tk, ws=ws,
-                                     stats=True),
-            lambda: dfl.pair_select(tk[0].view(B, G, 16), tk[2].view(B, G, 16), inp["anchor"], E,
-                                    Wsel, out=outs["sel"], ws=ws),
-            lambda: dfl.verify_sample(inp["T"], inp["Q"], outs["sel"][0], w.seed, step, inp["sid"],
-                                      w.inv_temperature, out=outs["samp"], ws=ws,
-                                      draft_stats=(tk[4].view(B, G), tk[5].view(B, G))),
-            lambda: dfl.verify_greedy(tg, outs["sel"][0], out=outs["greedy"], ws=ws),
-            lambda: dfl.dynconv2(inp["x"], inp["xp"], Wtap, out=outs["conv"]),
+            ("topk_softmax", lambda: dfl.topk_softmax(inp["Q"].view(B * G, V), w.inv_temperature,
+                                                      out=tk, ws=ws, stats=True)),
+            ("pair_select", lambda: dfl.pair_select(tk[0].view(B, G, 16), tk[2].view(B, G, 16),
+                                                    inp["anchor"], self.E, self.Wsel,
+                                                    out=outs["sel"], ws=ws)),
+            ("verify_sample", lambda: dfl.verify_sample(
+                inp["T"], inp["Q"], outs["sel"][0], w.seed, step, inp["sid"], w.inv_temperature,
+                out=outs["samp"], ws=ws, draft_stats=(tk[4].view(B, G), tk[5].view(B, G)))),
+            ("verify_greedy", lambda: dfl.verify_greedy(tg, outs["sel"][0], out=outs["greedy"],
+                                                        ws=ws)),
+            ("dynconv2", lambda: dfl.dynconv2(inp["x"], inp["xp"], self.Wtap, out=outs["conv"])),
         ]
 
-    stream = torch.cuda.current_stream(dev)
+    def extra_calls(self, k, step):
+        """The verify variants outside the five-call cycle: the greedy verify
+        with early exit, and the sampling verify of top-k 20 / top-p 0.95
+        truncated distributions (the pages' Qwen sampling settings)."""
+        dfl, w, outs, ws = self.dfl, self.w, self.outs, self.ws
+        inp = self.inputs[k]
+        return [
+            ("verify_greedy_early_exit", lambda: dfl.verify_greedy(
+                inp["T"], outs["sel"][0], out=outs["greedy"], ws=ws, early_exit=True)),
+            ("verify_sample_trunc", lambda: dfl.verify_sample_trunc(
+                inp["T"], inp["Q"], outs["sel"][0], w.seed, step, inp["sid"], w.inv_temperature,
+                20, 0.95, out=outs["samp"], ws=ws)),
+        ]
 
-    def run_calls(n, step0, record):
+    def cycle_calls(self, kind, k, step):
+        """The calls of one timed unit: 'step' (all five), the 'sampling',
+        'greedy', 'greedy_early_exit' and 'sampling_truncated'
+        draft-select-verify cycles, or 'dynconv2' alone."""
+        allc = dict(self.calls(k, step, greedy_other_set=(kind == "step")))
+        allc.update(dict(self.extra_calls(k, step)))
+        seq = {"step": list(CALLS),
+               "sampling": ["topk_softmax", "pair_select", "verify_sample"],
+               "greedy": ["topk_softmax", "pair_select", "verify_greedy"],
+               "greedy_early_exit": ["topk_softmax", "pair_select", "verify_greedy_early_exit"],
+               "sampling_truncated": ["topk_softmax", "pair_select", "verify_sample_trunc"],
+               "dynconv2": ["dynconv2"]}[kind]
+        return [(n, allc[n]) for n in seq]
+
+    def timed_graph(self, kind, K, W, step0=0, events=True):
+        """K units of `kind` (input sets alternating) captured back to back in
+        one CUDA graph, every call between two event nodes when `events`; W
+        eager units first.  Returns (ms per unit, {call: mean ms}, note)."""
+        torch, dev = self.torch, self.dev
+        stream = torch.cuda.current_stream(dev)
+        for s in range(W):
+            for _, fn in self.cycle_calls(kind, s % 2, step0 + s):
+                fn()
+        torch.cuda.synchronize(dev)
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
         evs = []
-        for s in range(n):
-            inp = inputs[(step0 + s) % 2]
-            row = []
-            for name, fn in zip(names, calls(inp, step0 + s)):
-                if record and args.only and name != args.only:
-                    continue
-                # L2 flush: write a buffer twice the size of L2, then read it,
-                # so the timed call starts with no data of its own in L2 and
-                # no dirty lines left to write back
+        try:
+            with torch.cuda.graph(g, stream=cap):
+                for s in range(K):
+                    row = []
+                    for name, fn in self.cycle_calls(kind, s % 2, step0 + W + s):
+                        if not events:
+                            fn()
+                            continue
+                        e0 = torch.cuda.Event(enable_timing=True, external=True)
+                        e1 = torch.cuda.Event(enable_timing=True, external=True)
+                        e0.record()
+                        fn()
+                        e1.record()
+                        row.append((name, e0, e1))
+                    evs.append(row)
+            note = ("one CUDA graph of K back-to-back units" +
+                    (", each call between event nodes" if events else ""))
+        except Exception as e:  # capture refused: eager launches with events
+            torch.cuda.synchronize(dev)
+            g, evs = None, []
+            note = "eager launches (graph capture failed: %s)" % str(e).splitlines()[0][:120]
+        torch.cuda.synchronize(dev)
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        if g is not None:
+            g.replay()
+        else:
+            for s in range(K):
+                row = []
+                for name, fn in self.cycle_calls(kind, s % 2, step0 + W + s):
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    fn()
+                    e1.record(stream)
+                    row.append((name, e0, e1))
+                evs.append(row)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        per = {}
+        for row in evs:
+            for name, e0, e1 in row:
+                per.setdefault(name, []).append(e0.elapsed_time(e1))
+        del g
+        return s0.elapsed_time(s1) / K, {n: float(np.mean(v)) for n, v in per.items()}, note
+
+    def time_select(self, impl, K):
+        """Mean ms of one pair_select with the given implementation, calls
+        back to back on input set 0 (its candidate lists from topk)."""
+        torch, dev, B, G = self.torch, self.dev, self.B, self.G
+        tk = self.inputs[0]["topk"]
+        dict(self.calls(0, 0))["topk_softmax"]()
+        fn = lambda: self.dfl.pair_select(tk[0].view(B, G, 16), tk[2].view(B, G, 16),
+                                          self.inputs[0]["anchor"], self.E, self.Wsel,
+                                          out=self.outs["sel"], ws=self.ws, impl=impl)
+        for _ in range(3):
+            fn()
+        stream = torch.cuda.current_stream(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / K
+
+    def isolated_calls(self, K, step0=0):
+        """Each call alone with L2 flushed before it (a 256 MB write then a
+        read of the same buffer, outside the timed intervals): {call: mean ms}."""
+        torch, dev = self.torch, self.dev
+        stream = torch.cuda.current_stream(dev)
+        flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        sink = torch.zeros((), dtype=torch.int64, device=dev)
+        evs = []
+        for s in range(K):
+            for name, fn in self.calls(s % 2, step0 + s):
                 flush.fill_(s & 0xFF)
-                flush_sink.add_(flush.view(torch.int64).sum())
+                sink.add_(flush.view(torch.int64).sum())
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 fn()
                 e1.record(stream)
-                row.append((e0, e1))
-            evs.append(row)
-        return evs
+                evs.append((name, e0, e1))
+        torch.cuda.synchronize(dev)
+        per = {}
+        for name, e0, e1 in evs:
+            per.setdefault(name, []).append(e0.elapsed_time(e1))
+        return {n: float(np.mean(v)) for n, v in per.items()}
+
+    def e2e(self, K, W, world, barrier):
+        """The cycle through the public API with the cycle's inputs copied
+        from pinned host memory and its results copied back, inside the timed
+        region.  Returns (ms per cycle, h2d bytes, d2h bytes)."""
+        torch, dev, B, G = self.torch, self.dev, self.B, self.G
+        stream = torch.cuda.current_stream(dev)
+        b0, c0 = self.sets[0]
+        host = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for k, v in
+                dict(T=b0.target.view(np.int16), Q=b0.draft.view(np.int16), anchor=b0.anchor,
+                     sid=b0.seq_id.view(np.int32), x=c0.x.view(np.int16),
+                     xp=c0.x_prev.view(np.int16)).items()}
+        res = dict(samp_n=torch.empty((B,), dtype=torch.int32).pin_memory(),
+                   samp_tok=torch.empty((B, G + 1), dtype=torch.int32).pin_memory(),
+                   greedy_tok=torch.empty((B, G + 1), dtype=torch.int32).pin_memory(),
+                   path=torch.empty((B, G), dtype=torch.int32).pin_memory(),
+                   conv=torch.empty((B, self.w.T, self.w.H), dtype=torch.int16).pin_memory())
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in res.values())
+        d = self.inputs[0]
+
+        def one(step):
+            d["T"].view(torch.int16).copy_(host["T"], non_blocking=True)
+            d["Q"].view(torch.int16).copy_(host["Q"], non_blocking=True)
+            d["anchor"].copy_(host["anchor"], non_blocking=True)
+            d["sid"].copy_(host["sid"], non_blocking=True)
+            d["x"].view(torch.int16).copy_(host["x"], non_blocking=True)
+            d["xp"].view(torch.int16).copy_(host["xp"], non_blocking=True)
+            for _, fn in self.calls(0, step, greedy_other_set=False):
+                fn()
+            res["samp_n"].copy_(self.outs["samp"][0], non_blocking=True)
+            res["samp_tok"].copy_(self.outs["samp"][1], non_blocking=True)
+            res["greedy_tok"].copy_(self.outs["greedy"][1], non_blocking=True)
+            res["path"].copy_(self.outs["sel"][0], non_blocking=True)
+            res["conv"].copy_(self.outs["conv"].view(torch.int16), non_blocking=True)
+
+        for s in range(max(1, W)):
+            one(s)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        ne = max(3, min(K, 20))
+        e0.record(stream)
+        for s in range(ne):
+            one(s)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / ne, h2d, d2h
+
+    def gpu_results(self, step=0):
+        """One eager cycle on input set 0 with Philox step `step`: the path,
+        the sampling and the greedy verdicts, on the host."""
+        torch = self.torch
+        for _, fn in self.calls(0, step, greedy_other_set=False):
+            fn()
+        torch.cuda.synchronize(self.dev)
+        o = self.outs
+        return dict(rank=o["sel"][1].cpu().numpy(), sn=o["samp"][0].cpu().numpy(),
+                    sout=o["samp"][1].cpu().numpy(), gn=o["greedy"][0].cpu().numpy(),
+                    gout=o["greedy"][1].cpu().numpy())
+
+
+def parity_sample(gpu, orc_results, bands=(1e-6, 1e-6, 1e-5)):
+    """The GPU's cycle against the oracle's on the sampled sequences: integer
+    outputs bit-exact, except near-ties inside the stated bands (accept
+    |u - r| < 1e-6, draw within 1e-6 R, path re-score within 1e-5 (1 + |best|)),
+    which are counted per kind; anything else is a failure."""
+    import oracle
+    acc_band, draw_band, path_band = bands
+    ties = {"accept": 0, "draw": 0, "path": 0}
+    fails, exact = [], 0
+    for r in orc_results:
+        s = r["seq"]
+        if not np.array_equal(gpu["rank"][s], r["rank"]):
+            re = oracle.path_rescore(r["idx"][None], r["logp"][None],
+                                     np.array([r["anchor"]], np.int32), _SEL["emb"], _SEL["W"],
+                                     gpu["rank"][s][None])[0]
+            if abs(re - r["score"]) / (1 + abs(r["score"])) < path_band:
+                ties["path"] += 1
+            else:
+                fails.append((s, "path"))
+            continue
+        ok = True
+        if gpu["gn"][s] != r["gn"] or not np.array_equal(gpu["gout"][s], r["gout"]):
+            fails.append((s, "greedy"))
+            ok = False
+        if gpu["sn"][s] != r["sn"]:
+            if r["macc"] < acc_band:
+                ties["accept"] += 1
+            else:
+                fails.append((s, "accept"))
+            ok = False
+        elif not np.array_equal(gpu["sout"][s], r["sout"]):
+            if r["mres"] < draw_band:
+                ties["draw"] += 1
+            else:
+                fails.append((s, "draw"))
+            ok = False
+        exact += ok
+    return {"sequences": len(orc_results), "exact": exact, "near_ties": ties,
+            "failures": len(fails), "failed": fails[:8]}
+
+
+_SEL = {}
+
+
+def summarize_calls(w, B, per_call_ms, peak):
+    alg = algorithmic_bytes(w, B)
+    out = {}
+    for n in CALLS:
+        if n not in per_call_ms:
+            continue
+        us = per_call_ms[n] * 1e3
+        gbs = alg[n] / (us * 1e-6) / 1e9
+        out[n] = {"us": round(us, 2), "algorithmic_bytes": alg[n], "GB/s": round(gbs, 1),
+                  "frac_of_hbm_peak": round(gbs / peak, 4)}
+    return out
+
+
+def measure_workload(name, args, rank, world, dev, barrier, peak, headline):
+    """Every figure of one workload; the headline also carries the clocks'
+    timed region (the caller's sampler)."""
+    import torch
+    bw = Bench(name, rank, dev)
+    w, B = bw.w, bw.B
+    K, W = args.steps, max(args.warmup, 3)
+    barrier()
+    ms_step, _, note = bw.timed_graph("step", K, W, events=False)
+    ms_ev, per_call, _ = bw.timed_graph("step", K, W, step0=500)
+    cyc, cyc_calls = {}, {}
+    for kind in CYCLE_KINDS:
+        ms, _, _ = bw.timed_graph(kind, K, W, step0=1000, events=False)
+        cyc[kind] = ms
+    for kind in ("greedy_early_exit", "sampling_truncated"):  # the variant call's own time
+        _, pc, _ = bw.timed_graph(kind, K, W, step0=2000)
+        cyc_calls[kind] = pc[bw.cycle_calls(kind, 0, 0)[-1][0]]
+    iso = bw.isolated_calls(max(3, min(K, 10)))
+    sel_impl = {}
+    if bw.w.dtype == 1:  # both selector implementations, the same inputs
+        for impl, label in ((1, "simt"), (2, "tensor")):
+            sel_impl[label] = bw.time_select(impl, K)
+    nc = len(CYCLE_KINDS)
+    vals = [ms_step] + [per_call[n] for n in CALLS] + [cyc[k] for k in CYCLE_KINDS] + \
+        [iso[n] for n in CALLS] + [ms_ev] + [cyc_calls[k] for k in sorted(cyc_calls)] + \
+        [sel_impl[k] for k in sorted(sel_impl)]
+    red = max_over_ranks(vals, world, dev).cpu().numpy()
+    ms_step = float(red[0])
+    per_call = dict(zip(CALLS, red[1:6].tolist()))
+    cyc = dict(zip(CYCLE_KINDS, red[6:6 + nc].tolist()))
+    o = 6 + nc
+    iso = dict(zip(CALLS, red[o:o + 5].tolist()))
+    ms_ev = float(red[o + 5])
+    cyc_calls = dict(zip(sorted(cyc_calls), red[o + 6:o + 6 + len(cyc_calls)].tolist()))
+    sel_impl = dict(zip(sorted(sel_impl), red[o + 6 + len(cyc_calls):].tolist()))
+    e2e = None
+    if not args.no_e2e:
+        ms, h2d, d2h = bw.e2e(K, W, world, barrier)
+        t = float(max_over_ranks([ms], world, dev)[0])
+        e2e = {"value": world * 1000.0 / t, "unit": "cycles/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+    alg = algorithmic_bytes(w, B)
+    calls = summarize_calls(w, B, per_call, peak)
+    dom = max(CALLS, key=lambda n: per_call[n])
+    step_bytes = sum(alg.values())
+    step_gbs = step_bytes / (ms_step * 1e-3) / 1e9
+    res = {
+        "value": world * 1000.0 / ms_step, "ms_per_step": ms_step,
+        "config": {"workload": DESCRIBE[name], "cycle": CYCLE_DEF,
+                   "global_batch": B * world, "timing": note,
+                   "us_per_cycle_with_call_events": round(ms_ev * 1e3, 2),
+                   "step_hbm_GBps": round(step_gbs, 1),
+                   "step_frac_of_hbm_peak": round(step_gbs / peak, 4)},
+        "cycles": {
+            "sampling": {"cycles_per_s": round(world * 1000.0 / cyc["sampling"], 1),
+                         "us": round(cyc["sampling"] * 1e3, 2),
+                         "calls": "topk_softmax_ex -> pair_select -> verify_sample_ex"},
+            "greedy": {"cycles_per_s": round(world * 1000.0 / cyc["greedy"], 1),
+                       "us": round(cyc["greedy"] * 1e3, 2),
+                       "calls": "topk_softmax -> pair_select -> verify_greedy"},
+            "greedy_early_exit": {
+                "cycles_per_s": round(world * 1000.0 / cyc["greedy_early_exit"], 1),
+                "us": round(cyc["greedy_early_exit"] * 1e3, 2),
+                "verify_us": round(cyc_calls["greedy_early_exit"] * 1e3, 2),
+                "calls": "topk_softmax -> pair_select -> verify_greedy_early_exit"},
+            "sampling_truncated": {
+                "cycles_per_s": round(world * 1000.0 / cyc["sampling_truncated"], 1),
+                "us": round(cyc["sampling_truncated"] * 1e3, 2),
+                "verify_us": round(cyc_calls["sampling_truncated"] * 1e3, 2),
+                "verify_GBps": round(2 * B * (2 * w.G + 1) * w.V /
+                                     (cyc_calls["sampling_truncated"] * 1e-3) / 1e9, 1),
+                "calls": "topk_softmax_ex -> pair_select -> verify_sample_trunc (top-k 20, "
+                         "top-p 0.95, T = 1; target and draft rows streamed once)"},
+            "dynconv2": {"calls_per_s": round(world * 1000.0 / cyc["dynconv2"], 1),
+                         "us": round(cyc["dynconv2"] * 1e3, 2)},
+        },
+        "calls": calls,
+        "calls_isolated": summarize_calls(w, B, iso, peak),
+        "pair_select_impls_us": {k: round(v * 1e3, 2) for k, v in sel_impl.items()},
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": calls[dom]["GB/s"], "peak": peak,
+                     "unit": "GB/s", "frac": round(calls[dom]["GB/s"] / peak, 4),
+                     "traffic": recorded_traffic(dom),
+                     "timing": "mean device time of the call inside the timed graph"},
+        "e2e": e2e,
+        "gpu_launches": int(K * len(CALLS)),
+    }
+    # accepted tokens per verify step on this workload's first input set
+    r = bw.gpu_results(step=0)
+    res["accepted_tokens_per_verify_step"] = {
+        "sampling": round(float((r["sn"] + 1).mean()), 3),
+        "greedy": round(float((r["gn"] + 1).mean()), 3)}
+    return bw, res
+
+
+def run_ours(args, rank, world, local_rank, pool):
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # The step as timed: the five calls back to back, no flush in between.
-    # Input sets alternate between steps and the greedy verify reads the
-    # other set's target rows, so no call finds the rows it streams in L2
-    # from an earlier call (a step reads ~344 MB of inputs, L2 is 126 MB);
-    # the sampling verify may find the draft rows topk just read (the fused
-    # cycle).  Each set's step is captured once in a CUDA graph (launch cost
-    # off the host); replays reuse the captured Philox step, which changes
-    # no cost.
-    def step_eager(k, step):
-        for fn in calls(inputs[k], step, t_greedy=inputs[1 - k]["T"]):
-            fn()
-
-    graphs, graph_note = None, "eager launches"
-    if not args.no_graph and not args.only:
-        try:
-            cap = torch.cuda.Stream(dev)
-            cap.wait_stream(stream)
-            with torch.cuda.stream(cap):
-                for k in range(2):
-                    step_eager(k, k)
-            cap.synchronize()
-            graphs = []
-            for k in range(2):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=cap):
-                    step_eager(k, k)
-                graphs.append(g)
-            torch.cuda.synchronize(dev)
-            graph_note = "CUDA graph replays (one graph per input set)"
-        except Exception as e:  # capture refused: time eager launches instead
-            graphs = None
-            graph_note = "eager launches (graph capture failed: %s)" % str(e).splitlines()[0][:120]
-            torch.cuda.synchronize(dev)
-
-    def run_step_pass(n, step0):
-        for s in range(n):
-            k = (step0 + s) % 2
-            if graphs is not None:
-                graphs[k].replay()
-            else:
-                step_eager(k, step0 + s)
-
-    run_calls(args.warmup, 0, False)
-    run_step_pass(max(args.warmup, 3), 0)
-    barrier()
-    sampler = ClockSampler(local_rank)
-    with sampler:
-        t_wall0 = time.perf_counter()
-        s0 = torch.cuda.Event(enable_timing=True)
-        s1 = torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        run_step_pass(args.steps, args.warmup)
-        s1.record(stream)
-        torch.cuda.synchronize(dev)
-        t_wall = time.perf_counter() - t_wall0
-        barrier()
-        evs = run_calls(args.steps, args.warmup, True)
-        torch.cuda.synchronize(dev)
-    barrier()
-    per_call = np.array([[e0.elapsed_time(e1) for (e0, e1) in row] for row in evs])  # ms
-    if args.only:  # one call alone: a per-call line for profiling, not a bench line
+    peak, peak_kind = peaks()
+    if args.only:
+        bw = Bench(HEADLINE, rank, dev)
+        for s in range(max(args.warmup, 3)):
+            dict(bw.calls(s % 2, s))[args.only]()
+        iso = bw.isolated_calls(args.steps)
         if rank == 0:
-            us = float(per_call.mean()) * 1e3
-            nbytes = algorithmic_bytes(w, B)[args.only]
+            us = iso[args.only] * 1e3
+            nbytes = algorithmic_bytes(bw.w, bw.B)[args.only]
             print(json.dumps({"only": args.only, "us": round(us, 2), "algorithmic_bytes": nbytes,
                               "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1),
                               "steps": args.steps}), flush=True)
         return
-    local = max_over_ranks([s0.elapsed_time(s1), float(per_call.sum(axis=1).mean())] +
-                           per_call.mean(axis=0).tolist(), world, dev)
-    ms_per_step = float(local[0]) / args.steps
-    calls_sum_ms = float(local[1])
-    mean_call_ms = local[2:].cpu().numpy()
 
-    # e2e: the public API with host buffers, copies inside the timed region
-    e2e = None
-    if not args.no_e2e:
-        b0, c0 = sets[0]
-        host = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for k, v in
-                dict(T=b0.target.view(np.int16), Q=b0.draft.view(np.int16), anchor=b0.anchor,
-                     sid=b0.seq_id.view(np.int32), x=c0.x.view(np.int16),
-                     xp=c0.x_prev.view(np.int16)).items()}
-        res_host = dict(samp_n=torch.empty((B,), dtype=torch.int32).pin_memory(),
-                        samp_tok=torch.empty((B, G + 1), dtype=torch.int32).pin_memory(),
-                        greedy_tok=torch.empty((B, G + 1), dtype=torch.int32).pin_memory(),
-                        path=torch.empty((B, G), dtype=torch.int32).pin_memory(),
-                        conv=torch.empty((B, w.T, w.H), dtype=torch.int16).pin_memory())
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
-        d2h = sum(t.numel() * t.element_size() for t in res_host.values())
-        dbuf = inputs[0]
+    sampler = ClockSampler(local_rank)
+    t_wall0 = time.perf_counter()
+    with sampler:
+        bw, head = measure_workload(HEADLINE, args, rank, world, dev, barrier, peak, True)
+    t_wall = time.perf_counter() - t_wall0
+    others = {}
+    if not args.headline_only:
+        for name in OTHER_WORKLOADS:
+            _, res = measure_workload(name, args, rank, world, dev, barrier, peak, False)
+            res.pop("gpu_launches", None)
+            others[name] = res
+            torch.cuda.empty_cache()
 
-        def e2e_step(step):
-            dbuf["T"].view(torch.int16).copy_(host["T"], non_blocking=True)
-            dbuf["Q"].view(torch.int16).copy_(host["Q"], non_blocking=True)
-            dbuf["anchor"].copy_(host["anchor"], non_blocking=True)
-            dbuf["sid"].copy_(host["sid"], non_blocking=True)
-            dbuf["x"].view(torch.int16).copy_(host["x"], non_blocking=True)
-            dbuf["xp"].view(torch.int16).copy_(host["xp"], non_blocking=True)
-            for fn in calls(dbuf, step):
-                fn()
-            res_host["samp_n"].copy_(outs["samp"][0], non_blocking=True)
-            res_host["samp_tok"].copy_(outs["samp"][1], non_blocking=True)
-            res_host["greedy_tok"].copy_(outs["greedy"][1], non_blocking=True)
-            res_host["path"].copy_(outs["sel"][0], non_blocking=True)
-            res_host["conv"].copy_(outs["conv"].view(torch.int16), non_blocking=True)
-
-        for s in range(max(1, args.warmup)):
-            e2e_step(s)
-        barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        ne = max(3, min(args.steps, 20))
-        e0.record(stream)
-        for s in range(ne):
-            e2e_step(s)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        t = max_over_ranks([e0.elapsed_time(e1) / ne], world, dev)
-        e2e = {"value": world * 1000.0 / float(t[0]), "unit": "cycles/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    cpu, cpu1, parity = None, None, None
+    if pool is not None and rank == 0:
+        procs = pool.procs
+        w = bw.w
+        seqs = list(range(w.B))
+        sec, orc = pool.cycle(seqs, step=0, collect=True)
+        cpu = {"value": 1.0 / sec, "unit": "cycles/s", "cores": procs, "kind": "oracle",
+               "sample": "one whole cycle of the headline batch (all %d sequences: top-16, "
+                         "selector, sampling and greedy verify, dynconv), the sequences spread "
+                         "over %d worker processes, wall clock" % (w.B, procs)}
+        one = [orc_r[0] for orc_r in orc[:2]]
+        cpu1 = {"value": 1.0 / (float(np.mean(one)) * w.B), "unit": "cycles/s", "cores": 1,
+                "kind": "oracle",
+                "sample": "2 of the %d sequences, each timed in one process, scaled by %d"
+                          % (w.B, w.B)}
+        _SEL["emb"], _SEL["W"] = bw.sel.emb, bw.sel.W
+        parity = parity_sample(bw.gpu_results(step=0), [r for _, r in orc])
 
     if rank != 0:
         return
-    peak, peak_kind = peaks()
-    alg = algorithmic_bytes(w, B)
-    calls_info = {}
-    for i, n in enumerate(names):
-        us = float(mean_call_ms[i]) * 1e3
-        gbs = alg[n] / (us * 1e-6) / 1e9
-        calls_info[n] = {"us": round(us, 2), "algorithmic_bytes": alg[n], "GB/s": round(gbs, 1),
-                         "frac_of_hbm_peak": round(gbs / peak, 4)}
-    dom = max(names, key=lambda n: calls_info[n]["us"])
-    kernel_of = {"topk_softmax": "topk_softmax", "pair_select": "pair_select",
-                 "verify_sample": "verify_sample", "verify_greedy": "verify_greedy",
-                 "dynconv2": "dynconv2"}
-    step_bytes = sum(alg.values())
-    step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
-    sample_cycle_us = sum(calls_info[n]["us"] for n in ("topk_softmax", "pair_select", "verify_sample"))
-    greedy_cycle_us = sum(calls_info[n]["us"] for n in ("topk_softmax", "pair_select", "verify_greedy"))
-
-    cpu = None
-    if not args.no_cpu_baseline and world == 1:
-        b0, c0 = sets[0]
-        seqs = list(range(8))
-        sec = oracle_step_seconds(w, b0, sel, synth.ConvInputs(c0.x, c0.x_prev, wtap), seqs)
-        cpu = {"value": 1.0 / (sec / len(seqs) * B), "unit": "cycles/s", "cores": 1,
-               "kind": "oracle",
-               "sample": "8 of the 32 sequences of one step (all five calls), scaled by 32/8; "
-                         "single-threaded fp64 oracle"}
-    value = world * 1000.0 / ms_per_step
     line = {
-        "metric": METRIC, "value": value, "unit": "cycles/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "metric": METRIC, "value": head["value"], "unit": "cycles/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "concurrency-32: B=32, block 8 (7 drafted + 1 bonus), V=151936, "
-                               "bf16 logits, selector d=128 (emb 151936x128 bf16, W fp32), "
-                               "sampling at T=1.0 (fused cycle: drafter normalisers from topk) "
-                               "and greedy verify, dynconv H=5120 over 32x8 tokens; one step = "
-                               "all five calls",
-                   "global_batch": B * world, "parallelism": "dp%d (independent batches)" % world,
-                   "timing": "K whole steps between two CUDA events on the launching "
-                             "stream, " + graph_note,
-                   "l2": "inputs larger than L2: a step reads ~344 MB of inputs (two input sets "
-                         "alternated, the greedy verify on the other set's target rows); the "
-                         "per-call breakdown ('calls', roofline) flushes L2 (256 MB write + "
-                         "read) before every call, outside its timed intervals",
-                   "calls_sum_us": round(calls_sum_ms * 1e3, 2),
-                   "step_hbm_GBps": round(step_gbs, 1),
-                   "step_frac_of_hbm_peak": round(step_gbs / peak, 4),
-                   "sampling_cycle_per_s": round(1e6 / sample_cycle_us, 1),
-                   "greedy_cycle_per_s": round(1e6 / greedy_cycle_us, 1),
-                   "wall_s_timed": round(t_wall, 3)},
-        "calls": calls_info,
-        "roofline": {"kernel": kernel_of[dom], "bound": "hbm",
-                     "achieved": calls_info[dom]["GB/s"], "peak": peak, "unit": "GB/s",
-                     "frac": round(calls_info[dom]["GB/s"] / peak, 4),
-                     "traffic": recorded_traffic(dom), "peak_kind": peak_kind},
+        "config": dict(head["config"], parallelism="dp%d (independent batches)" % world,
+                       l2="inputs larger than L2: a cycle reads ~344 MB of inputs (two input "
+                          "sets alternated, the greedy verify on the other set's target rows); "
+                          "'calls_isolated' flushes L2 (256 MB write + read) before every call",
+                       wall_s_timed=round(t_wall, 3)),
+        "cycles": head["cycles"],
+        "calls": head["calls"],
+        "calls_isolated": head["calls_isolated"],
+        "roofline": dict(head["roofline"], peak_kind=peak_kind),
+        "accepted_tokens_per_verify_step": head["accepted_tokens_per_verify_step"],
+        "workloads": others,
+        "parity_sample": parity,
         "cpu_baseline": cpu,
-        "e2e": e2e,
-        "gpu_launches": int(args.steps * sum(kernels_per_step.values())),
+        "cpu_baseline_single_thread": cpu1,
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
         "clocks": sampler.summary(),
     }
     print(json.dumps(line), flush=True)
@@ -585,6 +1067,12 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    pool = None
+    if (args.impl == "ours" and not args.acceptance and not args.only and world == 1
+            and not args.no_cpu_baseline and not args.drafter_layer and not args.select_sweep):
+        # spawned before the first CUDA call; its workers build the oracle's
+        # weights while the GPU runs
+        pool = OraclePool(HEADLINE, max(1, min(usable_cores(), 32)))
     if world > 1 and args.impl == "ours":
         import datetime
 
@@ -597,11 +1085,19 @@ def main():
         if args.acceptance:
             if rank == 0:
                 run_acceptance(args)
+        elif args.drafter_layer:
+            if rank == 0:
+                run_drafter_layer(args)
+        elif args.select_sweep:
+            if rank == 0:
+                run_select_sweep(args)
         elif args.impl == "reference":
             run_reference(args, rank, world)
         else:
-            run_ours(args, rank, world, local_rank)
+            run_ours(args, rank, world, local_rank, pool)
     finally:
+        if pool is not None:
+            pool.close()
         if world > 1 and args.impl == "ours":
             import torch.distributed as dist
             dist.destroy_process_group()

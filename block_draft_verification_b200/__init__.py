@@ -13,7 +13,7 @@ import torch
 
 __all__ = ["F32", "BF16", "Q_SOFTMAX", "Q_ONEHOT", "K", "DFlash2Error", "lib", "workspace_bytes",
            "Workspace", "topk_softmax", "pair_select", "verify_greedy", "verify_sample",
-           "dynconv2", "status_string", "version", "device_errors"]
+           "verify_sample_trunc", "dynconv2", "status_string", "version", "device_errors"]
 
 F32, BF16 = 0, 1
 Q_SOFTMAX, Q_ONEHOT = 0, 1
@@ -49,19 +49,26 @@ def lib():
                                               vp, sz, vp]
         L.dflash2_pair_select.argtypes = [vp, vp, vp, vp, i32, i64, i32, vp, i32, i32, vp, vp, vp,
                                           vp, sz, vp]
+        L.dflash2_pair_select_ex.argtypes = [vp, vp, vp, vp, i32, i64, i32, vp, i32, i32, vp, vp,
+                                             vp, i32, vp, sz, vp]
         L.dflash2_verify_greedy.argtypes = [vp, i32, i32, i32, i64, vp, vp, vp, vp, sz, vp]
+        L.dflash2_verify_greedy_early_exit.argtypes = [vp, i32, i32, i32, i64, vp, vp, vp, vp, sz,
+                                                       vp]
         L.dflash2_verify_sample.argtypes = [vp, vp, i32, i32, i32, i64, vp, f32, u64, u32, vp, i32,
                                             vp, vp, vp, vp, vp, sz, vp]
         L.dflash2_verify_sample_ex.argtypes = [vp, vp, i32, i32, i32, i64, vp, vp, vp, f32, u64,
                                                u32, vp, i32, vp, vp, vp, vp, vp, sz, vp]
+        L.dflash2_verify_sample_trunc.argtypes = [vp, vp, i32, i32, i32, i64, vp, f32, i32, f32,
+                                                  u64, u32, vp, i32, vp, vp, vp, vp, vp, sz, vp]
         L.dflash2_dynconv2.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]
         L.dflash2_dynconv2_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.dflash2_dynconv2_workspace_bytes.restype = sz
         L.dflash2_device_errors.argtypes = [i32]
         L.dflash2_device_errors.restype = C.c_uint32
         for f in ("dflash2_topk_softmax", "dflash2_topk_softmax_ex", "dflash2_pair_select",
+                  "dflash2_pair_select_ex", "dflash2_verify_greedy_early_exit",
                   "dflash2_verify_greedy", "dflash2_verify_sample", "dflash2_verify_sample_ex",
-                  "dflash2_dynconv2"):
+                  "dflash2_verify_sample_trunc", "dflash2_dynconv2"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -184,9 +191,14 @@ def topk_softmax(logits, inv_temperature=1.0, out=None, ws=None, stats=False):
     return tuple(out)
 
 
-def pair_select(idx, logp, anchor, emb, W, out=None, ws=None):
+SELECT_AUTO, SELECT_SIMT, SELECT_TENSOR = 0, 1, 2
+
+
+def pair_select(idx, logp, anchor, emb, W, out=None, ws=None, impl=SELECT_AUTO):
     """idx, logp [B, G, 16], anchor [B] int32 or None, emb [V, d], W [d, d] float32
-    -> path_tok [B, G] int32, path_rank [B, G] int32, path_score [B] float32."""
+    -> path_tok [B, G] int32, path_rank [B, G] int32, path_score [B] float32.
+    impl: SELECT_AUTO (tensor cores for bf16 tables, dflash2_pair_select),
+    SELECT_SIMT or SELECT_TENSOR (dflash2_pair_select_ex)."""
     _cuda(idx, logp, anchor, emb, W)
     B, G, _ = idx.shape
     V, d = emb.shape
@@ -197,14 +209,23 @@ def pair_select(idx, logp, anchor, emb, W, out=None, ws=None):
                torch.empty((B,), dtype=torch.float32, device=dev))
     tok, rank, score = out
     wp, wb = _ws(ws, dev, B, G, V)
-    _check("dflash2_pair_select", lib().dflash2_pair_select(
-        _p(idx.contiguous()), _p(logp.contiguous()), _p(anchor), _p(emb.contiguous()), _dtype(emb),
-        V, d, _p(W.contiguous()), B, G, _p(tok), _p(rank), _p(score), wp, wb, _stream(dev)))
+    if impl == SELECT_AUTO:
+        _check("dflash2_pair_select", lib().dflash2_pair_select(
+            _p(idx.contiguous()), _p(logp.contiguous()), _p(anchor), _p(emb.contiguous()),
+            _dtype(emb), V, d, _p(W.contiguous()), B, G, _p(tok), _p(rank), _p(score), wp, wb,
+            _stream(dev)))
+    else:
+        _check("dflash2_pair_select_ex", lib().dflash2_pair_select_ex(
+            _p(idx.contiguous()), _p(logp.contiguous()), _p(anchor), _p(emb.contiguous()),
+            _dtype(emb), V, d, _p(W.contiguous()), B, G, _p(tok), _p(rank), _p(score), int(impl),
+            wp, wb, _stream(dev)))
     return tok, rank, score
 
 
-def verify_greedy(target, draft_tok, out=None, ws=None):
-    """target [B, G+1, V], draft_tok [B, G] int32 -> n_accept [B], out_tok [B, G+1] int32."""
+def verify_greedy(target, draft_tok, out=None, ws=None, early_exit=False):
+    """target [B, G+1, V], draft_tok [B, G] int32 -> n_accept [B], out_tok [B, G+1] int32.
+    early_exit: dflash2_verify_greedy_early_exit (the same results; rows after
+    a sequence's first mismatch are not read)."""
     _cuda(target, draft_tok)
     B, G1, V = target.shape
     dev = target.device
@@ -213,7 +234,8 @@ def verify_greedy(target, draft_tok, out=None, ws=None):
                torch.empty((B, G1), dtype=torch.int32, device=dev))
     n, toks = out
     wp, wb = _ws(ws, dev, B, G1 - 1, V)
-    _check("dflash2_verify_greedy", lib().dflash2_verify_greedy(
+    name = "dflash2_verify_greedy_early_exit" if early_exit else "dflash2_verify_greedy"
+    _check(name, getattr(lib(), name)(
         _p(target.contiguous()), _dtype(target), B, G1 - 1, V, _p(draft_tok.contiguous()), _p(n),
         _p(toks), wp, wb, _stream(dev)))
     return n, toks
@@ -257,6 +279,36 @@ def verify_sample(target, draft, draft_tok, seed, step, seq_id=None, inv_tempera
             _p(target.contiguous()), _p(q), _dtype(target), B, G, V, _p(draft_tok.contiguous()),
             _p(qmax), _p(qlse), float(inv_temperature), seed, step, _p(sid), int(q_mode), _p(n),
             _p(toks), _p(ratio), _p(u), wp, wb, _stream(dev)))
+    return out
+
+
+def verify_sample_trunc(target, draft, draft_tok, seed, step, seq_id=None, inv_temperature=1.0,
+                        top_k=20, top_p=0.95, q_mode=Q_SOFTMAX, debug=False, out=None, ws=None):
+    """The sampling verify on top-k / top-p truncated distributions
+    (dflash2_verify_sample_trunc): target [B, G+1, V], draft [B, G, V] (None in
+    one-hot mode), draft_tok [B, G] -> n_accept [B], out_tok [B, G+1]
+    (+ ratio [B, G], u [B, G] if debug)."""
+    _cuda(target, draft, draft_tok, seq_id)
+    B, G1, V = target.shape
+    G = G1 - 1
+    dev = target.device
+    if out is None:
+        out = (torch.empty((B,), dtype=torch.int32, device=dev),
+               torch.empty((B, G1), dtype=torch.int32, device=dev))
+        if debug:
+            out = out + (torch.empty((B, G), dtype=torch.float32, device=dev),
+                         torch.empty((B, G), dtype=torch.float32, device=dev))
+    n, toks = out[0], out[1]
+    ratio = out[2] if len(out) > 2 else None
+    u = out[3] if len(out) > 3 else None
+    wp, wb = _ws(ws, dev, B, G, V)
+    q = None if draft is None else draft.contiguous()
+    sid = None if seq_id is None else seq_id.to(torch.int32).contiguous()
+    seed, step = int(seed) & (2 ** 64 - 1), int(step) & 0xFFFFFFFF
+    _check("dflash2_verify_sample_trunc", lib().dflash2_verify_sample_trunc(
+        _p(target.contiguous()), _p(q), _dtype(target), B, G, V, _p(draft_tok.contiguous()),
+        float(inv_temperature), int(top_k), float(top_p), seed, step, _p(sid), int(q_mode), _p(n),
+        _p(toks), _p(ratio), _p(u), wp, wb, _stream(dev)))
     return out
 
 

@@ -28,6 +28,8 @@ extern "C" size_t dflash2_workspace_bytes(int B, int G, int64_t V) {
     need = need > greedy_layout(B, G, V, 4).total ? need : greedy_layout(B, G, V, 4).total;
     need = need > sample_layout(B, G, V, 4).total ? need : sample_layout(B, G, V, 4).total;
     need = need > select_layout(B, G).total ? need : select_layout(B, G).total;
+    need = need > trunc_layout(B, G, V, 4).total ? need : trunc_layout(B, G, V, 4).total;
+    need = need > greedy_ee_layout(B, G, V, 4).total ? need : greedy_ee_layout(B, G, V, 4).total;
     return need;
 }
 
@@ -35,10 +37,15 @@ unsigned dfl_errors_topk(int clear);
 unsigned dfl_errors_verify(int clear);
 unsigned dfl_errors_dynconv(int clear);
 unsigned dfl_errors_select(int clear);
+unsigned dfl_errors_trunc(int clear);
+unsigned dfl_errors_select_tc(int clear);
+unsigned dfl_errors_greedy_ee(int clear);
 
 extern "C" unsigned dflash2_device_errors(int clear) {
-    const unsigned f[4] = {dfl_errors_topk(clear), dfl_errors_verify(clear),
-                           dfl_errors_dynconv(clear), dfl_errors_select(clear)};
+    const unsigned f[7] = {dfl_errors_topk(clear),      dfl_errors_verify(clear),
+                           dfl_errors_dynconv(clear),   dfl_errors_select(clear),
+                           dfl_errors_trunc(clear),     dfl_errors_select_tc(clear),
+                           dfl_errors_greedy_ee(clear)};
     unsigned v = 0;
     for (unsigned x : f) {
         if (x == 0xFFFFFFFFu) return 0xFFFFFFFFu;

@@ -47,6 +47,12 @@ __device__ __forceinline__ uint64_t shfl_xor(uint64_t v, int m) {
 __device__ __forceinline__ uint32_t shfl_xor(uint32_t v, int m) {
     return __shfl_xor_sync(FULL, v, m);
 }
+// Lane l gets lane l - 1's value (lane 0 keeps its own).
+__device__ __forceinline__ uint64_t shfl64_up1(uint64_t v) {
+    const uint32_t lo = __shfl_up_sync(FULL, (uint32_t)v, 1);
+    const uint32_t hi = __shfl_up_sync(FULL, (uint32_t)(v >> 32), 1);
+    return ((uint64_t)hi << 32) | lo;
+}
 __device__ __forceinline__ uint64_t shfl64(uint64_t v, int src) {
     uint32_t lo = __shfl_sync(FULL, (uint32_t)v, src);
     uint32_t hi = __shfl_sync(FULL, (uint32_t)(v >> 32), src);

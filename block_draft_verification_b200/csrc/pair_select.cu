@@ -264,12 +264,20 @@ unsigned dfl_errors_select(int clear) {
     return v;
 }
 
-extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const int32_t* anchor,
-                                   const void* emb, int emb_dtype, int64_t V, int d,
-                                   const float* W, int B, int G, int32_t* path_tok,
-                                   int32_t* path_rank, float* path_score, void* ws,
-                                   size_t ws_bytes, dflash2_stream_t stream) {
+int dfl_pair_select_tc(const int32_t* idx, const float* logp, const int32_t* anchor,
+                       const void* emb, int64_t V, int d, const float* W, int B, int G,
+                       int32_t* path_tok, int32_t* path_rank, float* path_score,
+                       cudaStream_t s);
+
+extern "C" int dflash2_pair_select_ex(const int32_t* idx, const float* logp,
+                                      const int32_t* anchor, const void* emb, int emb_dtype,
+                                      int64_t V, int d, const float* W, int B, int G,
+                                      int32_t* path_tok, int32_t* path_rank, float* path_score,
+                                      int impl, void* ws, size_t ws_bytes,
+                                      dflash2_stream_t stream) {
     if (!dtype_ok(emb_dtype)) return DFLASH2_EDTYPE;
+    if (impl < DFLASH2_SELECT_AUTO || impl > DFLASH2_SELECT_TENSOR) return DFLASH2_EINVAL;
+    if (impl == DFLASH2_SELECT_TENSOR && emb_dtype != DFLASH2_BF16) return DFLASH2_EDTYPE;
     if (B < 0 || G < 1 || G >= DFLASH2_MAX_BLOCK || V < K || (d != 64 && d != 128))
         return DFLASH2_ESHAPE;
     if (B == 0) return DFLASH2_OK;
@@ -283,6 +291,13 @@ extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const 
     const Layout L = select_layout(B, G);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return DFLASH2_EWORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
+    // the tensor cores take every bf16 table (the choice never depends on B,
+    // so a sequence's result does not depend on the batch it runs in)
+    const bool tensor = impl == DFLASH2_SELECT_TENSOR ||
+                        (impl == DFLASH2_SELECT_AUTO && emb_dtype == DFLASH2_BF16);
+    if (tensor)
+        return dfl_pair_select_tc(idx, logp, anchor, emb, V, d, W, B, G, path_tok, path_rank,
+                                  path_score, s);
     unsigned* counters = (unsigned*)((char*)ws + L.counters_off);
     float* scores = (float*)((char*)ws + L.part_off);
     if (!L.self_clean && cudaMemsetAsync(counters, 0, (size_t)B * 4, s) != cudaSuccess)
@@ -309,4 +324,14 @@ extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const 
     }
 #undef DFL_SEL
     return launch_status();
+}
+
+extern "C" int dflash2_pair_select(const int32_t* idx, const float* logp, const int32_t* anchor,
+                                   const void* emb, int emb_dtype, int64_t V, int d,
+                                   const float* W, int B, int G, int32_t* path_tok,
+                                   int32_t* path_rank, float* path_score, void* ws,
+                                   size_t ws_bytes, dflash2_stream_t stream) {
+    return dflash2_pair_select_ex(idx, logp, anchor, emb, emb_dtype, V, d, W, B, G, path_tok,
+                                  path_rank, path_score, DFLASH2_SELECT_AUTO, ws, ws_bytes,
+                                  stream);
 }

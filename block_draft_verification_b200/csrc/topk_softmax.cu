@@ -30,6 +30,7 @@ namespace dfl {
 // merged into the running list whenever more than CAND_FLUSH are waiting (at
 // most 32 lanes x 8 elements arrive between two checks).
 constexpr unsigned CAND_FLUSH = 64;
+constexpr unsigned SMALL_FLUSH = 4;  // up to this many keys are inserted one by one
 constexpr unsigned CAND_CAP = CAND_FLUSH + 32 * 8;
 struct CandBuf {
     uint64_t key[CAND_CAP];
@@ -46,14 +47,26 @@ __device__ __forceinline__ void flush_candidates(CandBuf& cb, uint64_t& run, uin
     const int lane = threadIdx.x & 31;
     __syncwarp();
     const unsigned n = *(volatile unsigned*)&cb.n;
-    for (unsigned base = 0; base < n; base += K) {
-        uint64_t v = run;
-        if (lane >= K) {
-            const unsigned j = base + (unsigned)(lane - K);
-            v = (j < n) ? cb.key[j] : 0ull;
+    if (n <= SMALL_FLUSH) {
+        // a few keys (the usual case once the list is full): insert each at
+        // its rank, found by one ballot, shifting the lower keys down a lane
+        for (unsigned i = 0; i < n; ++i) {
+            const uint64_t c = cb.key[i];
+            const unsigned above = __ballot_sync(FULL, lane < K && run > c);
+            const int pos = __popc(above);
+            const uint64_t up = shfl64_up1(run);
+            if (pos < K && lane < K && lane >= pos) run = (lane == pos) ? c : up;
         }
-        v = warp_sort_desc(v);
-        run = (lane < K) ? v : 0ull;
+    } else {
+        for (unsigned base = 0; base < n; base += K) {
+            uint64_t v = run;
+            if (lane >= K) {
+                const unsigned j = base + (unsigned)(lane - K);
+                v = (j < n) ? cb.key[j] : 0ull;
+            }
+            v = warp_sort_desc(v);
+            run = (lane < K) ? v : 0ull;
+        }
     }
     __syncwarp();
     if (lane == 0) cb.n = 0;
@@ -92,7 +105,6 @@ __device__ __forceinline__ void topk_chunk(const View& v, float c2, CandBuf& cb,
                                            uint32_t& pub) {
     using C = ChunkT<BF16>;
     const int lane = threadIdx.x & 31, nv = v.nvec();
-    const uint32_t shared = *(volatile unsigned*)thr;  // used after pass 1
     uint32_t vm[NVL];
     const float m = chunk_pass1<BF16>(v, vm);
     const float M = warp_max(m);
@@ -106,8 +118,15 @@ __device__ __forceinline__ void topk_chunk(const View& v, float c2, CandBuf& cb,
         if (t16 != 0u) {  // else fewer than 16 lanes hold elements: every element qualifies
             tv = unord32(t16);
             tkey = ((uint64_t)t16 << 32) - 1ull;  // below every key of value tv
+            // 16 lane maxima of this chunk reach t16: a bound for the whole
+            // row, shared at once with the warps on its other chunks
+            if (t16 > pub) {
+                pub = t16;
+                if (lane == 0) atomicMax(thr, t16);
+            }
         }
     }
+    const uint32_t shared = *(volatile unsigned*)thr;
     if (shared != 0u && (((uint64_t)shared << 32) - 1ull) > tkey) {
         tkey = ((uint64_t)shared << 32) - 1ull;
         tv = unord32(shared);

@@ -11,6 +11,8 @@
  *   dflash2_verify_greedy  greedy lossless verify (longest prefix match)
  *   dflash2_verify_sample  sampling lossless verify (rejection sampling with
  *                          residual resample and bonus draw)
+ *   dflash2_verify_sample_trunc  the same on top-k / top-p truncated
+ *                          distributions
  *   dflash2_dynconv2       two-tap dynamic depthwise conv fused with its tap
  *                          projection and the residual add
  *
@@ -21,7 +23,8 @@
  *   [myaiexp]  "DFlash 2" (myaiexp.com), section "主な機能" (features).
  *   [latenode] "DFlash 2: un drafter de 3.43× que cae a 1.45× bajo carga",
  *              sections "Un drafter que adivina el bloque entero de una vez",
- *              "El desacuerdo empieza en las propias tablas del proveedor".
+ *              "El desacuerdo empieza en las propias tablas del proveedor",
+ *              "Preguntas frecuentes".
  *   [psi]      "Qwen 3.8 27B + DFlash2: 140 Token/Sec?", section "Résumé".
  *   [philox]   Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3",
  *              SC'11, section 5.
@@ -206,6 +209,32 @@ DFLASH2_API int dflash2_pair_select(const int32_t* idx, const float* logp, const
                         void* ws, size_t ws_bytes, dflash2_stream_t stream);
 
 /*
+ * dflash2_pair_select with the implementation named.  Results of the two
+ * differ only in fp32 rounding (both accumulate in fp32; the path can differ
+ * only where two paths' scores are within that rounding).
+ * impl  DFLASH2_SELECT_AUTO: the tensor cores for bf16 tables, the CUDA cores
+ *       for fp32 ones -- a rule that depends on the dtype only, never on B,
+ *       so a sequence's result does not depend on its batch (what
+ *       dflash2_pair_select does);
+ *       DFLASH2_SELECT_SIMT: the CUDA cores, fp32 FMAs, one CTA per
+ *       (sequence, position) and a last-CTA recursion (any table);
+ *       DFLASH2_SELECT_TENSOR: one CTA per sequence, F = E W on tcgen05 with
+ *       W split into three bf16 planes (fp32 accuracy), the 16 x 16 blocks
+ *       from F on the CUDA cores, the recursion in shared memory (bf16
+ *       tables only: DFLASH2_EDTYPE otherwise); needs no workspace, though
+ *       ws is checked as for the other implementations.
+ * Other values: DFLASH2_EINVAL.
+ */
+#define DFLASH2_SELECT_AUTO 0
+#define DFLASH2_SELECT_SIMT 1
+#define DFLASH2_SELECT_TENSOR 2
+DFLASH2_API int dflash2_pair_select_ex(const int32_t* idx, const float* logp, const int32_t* anchor,
+                                       const void* emb, int emb_dtype, int64_t V, int d,
+                                       const float* W, int B, int G, int32_t* path_tok,
+                                       int32_t* path_rank, float* path_score, int impl, void* ws,
+                                       size_t ws_bytes, dflash2_stream_t stream);
+
+/*
  * Greedy lossless verify.  [tamsi] "Les chiffres qui comptent sur
  * Qwen3.8-27B" (greedy output is exactly the target's); [latenode] "El
  * desacuerdo..." (acceptance length = tokens completed per verify step).
@@ -221,6 +250,22 @@ DFLASH2_API int dflash2_pair_select(const int32_t* idx, const float* logp, const
 DFLASH2_API int dflash2_verify_greedy(const void* target, int dtype, int B, int G, int64_t V,
                           const int32_t* draft_tok, int32_t* n_accept, int32_t* out_tok,
                           void* ws, size_t ws_bytes, dflash2_stream_t stream);
+
+/*
+ * dflash2_verify_greedy with early exit: the same arguments and bit-identical
+ * results, but target rows after a sequence's first mismatch are not read.
+ * Row j mismatches exactly when one of its elements has a larger (value,
+ * -index) key than draft_tok[j]'s; the rows are streamed in step (all
+ * sequences' row 0 first, then row 1, ...), and a chunk of a row after a
+ * mismatch already found is skipped rather than read, so only rows 0..n are
+ * guaranteed to be read and the bytes saved depend on the acceptance.
+ * Workspace: dflash2_workspace_bytes(B, G, V).  Rows that are not 16-byte
+ * aligned, or V * element size not a multiple of 16, run dflash2_verify_greedy.
+ */
+DFLASH2_API int dflash2_verify_greedy_early_exit(const void* target, int dtype, int B, int G,
+                                                 int64_t V, const int32_t* draft_tok,
+                                                 int32_t* n_accept, int32_t* out_tok, void* ws,
+                                                 size_t ws_bytes, dflash2_stream_t stream);
 
 /*
  * Sampling lossless verify by rejection sampling.  [tamsi] "Les chiffres qui
@@ -276,6 +321,47 @@ DFLASH2_API int dflash2_verify_sample_ex(const void* target, const void* draft, 
                                          const uint32_t* seq_id, int q_mode, int32_t* n_accept,
                                          int32_t* out_tok, float* ratio_dbg, float* u_dbg, void* ws,
                                          size_t ws_bytes, dflash2_stream_t stream);
+
+/*
+ * Sampling verify of distributions truncated by top-k and top-p.
+ * [latenode] "Preguntas frecuentes" (the Qwen targets are sampled at
+ * temperature 1.0, top-p 0.95, top-k 20); rejection sampling as in
+ * dflash2_verify_sample.  The pages do not say how truncation meets the
+ * verification; this call reads it as: the truncated distribution is the one
+ * a token is drawn from, so the verify keeps the truncated target p~ exactly
+ * against the drafter's truncated q~.
+ *
+ * Truncation of a row (z = x * inv_temperature): order the tokens by
+ * (z descending, index ascending); keep the first min(top_k, V); renormalise
+ * over them; keep the shortest prefix whose cumulative sum reaches top_p
+ * (at least one token; top_p = 1 keeps all); renormalise again (fp64).
+ * r_j = p~_j(d_j) / q~_j(d_j) (q~(d) = 0 < p~(d): r = +inf; both 0: r = 0),
+ * or r_j = p~_j(d_j) for DFLASH2_Q_ONEHOT; accept iff u_j < r_j, stop at the
+ * first rejection; n < G: the last token is drawn from max(0, p~_n - q~_n)
+ * (one-hot: p~_n without d_n; p~_n if that is empty by rounding), n = G: the
+ * bonus from p~_G; the draw takes t = u' R and returns the smallest kept
+ * index whose inclusive prefix in index order exceeds t (the last index with
+ * mass if none).  Uniforms as in dflash2_verify_sample.
+ *
+ * Arguments as dflash2_verify_sample, and:
+ * top_k       1 <= top_k <= 32 (DFLASH2_ESHAPE otherwise); top_k > V keeps V.
+ * top_p       0 < top_p <= 1, finite (DFLASH2_EINVAL otherwise), compared in
+ *             fp64 after widening.
+ * Every row is streamed once for its exact 32 best (value, index) keys; the
+ * full-row normaliser cancels in the truncated distributions, so no
+ * exponential of the row is taken.  ratio_dbg holds every r_j as float (+inf
+ * where q~(d) = 0 < p~(d)).  Workspace: dflash2_workspace_bytes(B, G, V).
+ * The cut, sums and draw are fp64 in an order of their own: outputs can
+ * differ from an fp64 reference taking another order only where a top-p cut,
+ * an accept test or a draw sits within rounding of its boundary.
+ */
+DFLASH2_API int dflash2_verify_sample_trunc(const void* target, const void* draft, int dtype, int B,
+                                            int G, int64_t V, const int32_t* draft_tok,
+                                            float inv_temperature, int top_k, float top_p,
+                                            uint64_t seed, uint32_t step, const uint32_t* seq_id,
+                                            int q_mode, int32_t* n_accept, int32_t* out_tok,
+                                            float* ratio_dbg, float* u_dbg, void* ws,
+                                            size_t ws_bytes, dflash2_stream_t stream);
 
 /*
  * Two-tap dynamic depthwise conv fused with its tap projection and the

@@ -175,3 +175,49 @@ def test_dynconv_validation(L):
     need = L.dflash2_dynconv2_workspace_bytes(1, 32, 8, 5120)
     assert need > 0 and need == L.dflash2_dynconv2_workspace_bytes(1, 8, 32, 5120)
     assert L.dflash2_dynconv2_workspace_bytes(1, 2, 8, 100) == 0
+
+
+def test_greedy_early_exit_validation(L):
+    def ee(t=P, dt=1, B=2, G=7, V=151936, d=P, n=P, o=P, ws=P2, wsb=1 << 30):
+        return L.dflash2_verify_greedy_early_exit(t, dt, B, G, V, d, n, o, ws, wsb, S0)
+    assert ee(dt=2) == EDTYPE
+    assert ee(G=0) == ESHAPE
+    assert ee(G=32) == ESHAPE
+    assert ee(B=0) == OK
+    assert ee(n=None) == EINVAL
+    assert ee(o=ODD) == EALIGN
+    assert ee(ws=None) == EWORKSPACE
+    assert ee(wsb=64) == EWORKSPACE
+
+
+def test_select_ex_validation(L):
+    def sel(edt=1, impl=0, wsb=1 << 30, B=2):
+        return L.dflash2_pair_select_ex(P, P, None, P, edt, 151936, 128, P, B, 7, P, P, P, impl,
+                                        P2, wsb, S0)
+    assert sel(impl=3) == EINVAL
+    assert sel(impl=-1) == EINVAL
+    assert sel(edt=0, impl=2) == EDTYPE     # the tensor path takes bf16 tables only
+    assert sel(B=0) == OK
+    assert sel(wsb=16) == EWORKSPACE
+
+
+def test_verify_trunc_validation(L):
+    def trunc(t=P, q=P, dt=1, B=2, G=7, V=151936, d=P, invT=1.0, k=20, p=0.95, qm=0, n=P, o=P,
+              ws=P2, wsb=1 << 30):
+        return L.dflash2_verify_sample_trunc(t, q, dt, B, G, V, d, invT, k, p, 0, 0, None, qm, n,
+                                             o, None, None, ws, wsb, S0)
+    assert trunc(dt=3) == EDTYPE
+    assert trunc(G=0) == ESHAPE
+    assert trunc(k=0) == ESHAPE
+    assert trunc(k=33) == ESHAPE               # the kernel keeps 32 keys per row
+    assert trunc(p=0.0) == EINVAL
+    assert trunc(p=1.5) == EINVAL
+    assert trunc(p=float("nan")) == EINVAL
+    assert trunc(invT=0.0) == EINVAL
+    assert trunc(qm=3) == EINVAL
+    assert trunc(q=None) == EINVAL             # softmax q needs the draft logits
+    assert trunc(q=None, qm=1, B=0) == OK
+    assert trunc(B=0) == OK
+    assert trunc(o=ODD) == EALIGN
+    assert trunc(wsb=0) == EWORKSPACE
+    assert trunc(k=32, p=1.0, V=8, wsb=1 << 30) != ESHAPE   # top_k > V keeps V

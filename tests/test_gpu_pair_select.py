@@ -6,7 +6,9 @@ Both sides get identical inputs: the candidate lists and log-probabilities
 come from the oracle's top-16 (rounded to fp32), never from the GPU.  The
 path must equal the oracle's, except where the oracle's own rescore of the
 GPU path is within 1e-5 * (1 + |best|) of the best (a counted near-tie);
-path_score within 1e-5 relative."""
+path_score within 1e-5 relative.  bf16 tables run both implementations
+(dflash2_pair_select_ex): the CUDA-core one and the tensor-core one (F = E W on
+tcgen05 with W split into three bf16 planes)."""
 import numpy as np
 import pytest
 import torch
@@ -25,12 +27,13 @@ def oracle_inputs(orc, w, B, first=0):
     return idx.reshape(B, G, 16), logp.astype(np.float32).reshape(B, G, 16), b.anchor
 
 
-def run_and_check(orc, idx, logp, anchor, emb, W, ties=None):
+def run_and_check(orc, idx, logp, anchor, emb, W, ties=None, impl=dfl.SELECT_AUTO):
     need_cuda()
     tok, rank, score = dfl.pair_select(to_dev(idx), to_dev(logp),
                                        None if anchor is None else to_dev(anchor),
-                                       to_dev(emb), to_dev(W))
+                                       to_dev(emb), to_dev(W), impl=impl)
     torch.cuda.synchronize()
+    assert dfl.device_errors() == 0
     tok, rank, score = to_host(tok), to_host(rank), to_host(score)
     otok, orank, oscore = orc.pair_select(idx, logp, anchor, emb, W)
     assert_close(score, oscore, RTOL_F32, "path_score")
@@ -57,16 +60,20 @@ def test_tiny(orc):
     run_and_check(orc, idx, logp, None, sel.emb, sel.W)
 
 
+IMPLS = [dfl.SELECT_SIMT, dfl.SELECT_TENSOR]
+
+
 @pytest.mark.parametrize("name,B", [("b1", 1), ("b8", 8), ("b32", 32), ("ctx16", 8)])
-def test_full_vocab(orc, name, B):
+@pytest.mark.parametrize("impl", IMPLS)
+def test_full_vocab(orc, name, B, impl):
     w = synth.WORKLOADS[name]
     sel = synth.gen_selector(w)
     idx, logp, anchor = oracle_inputs(orc, w, B)
-    ties = run_and_check(orc, idx, logp, anchor, sel.emb, sel.W)
+    ties = run_and_check(orc, idx, logp, anchor, sel.emb, sel.W, impl=impl)
     print("near-ties:", ties.report())
 
 
-@pytest.mark.parametrize("G", [1, 2, 5, 31])
+@pytest.mark.parametrize("G", [1, 2, 5, 8, 9, 15, 16, 31])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 def test_shapes_and_pair_heavy_weights(orc, G, d, dt):
@@ -81,8 +88,20 @@ def test_shapes_and_pair_heavy_weights(orc, G, d, dt):
         emb = synth.to_bf16_bits(emb)
     W = (rng.standard_normal((d, d)) * 4 / np.sqrt(d)).astype(np.float32)
     anchor = rng.integers(0, V, B).astype(np.int32)
-    run_and_check(orc, idx, logp, anchor, emb, W)
-    run_and_check(orc, idx, logp, None, emb, W)
+    for impl in (IMPLS if dt == "bf16" else [dfl.SELECT_AUTO]):
+        run_and_check(orc, idx, logp, anchor, emb, W, impl=impl)
+        run_and_check(orc, idx, logp, None, emb, W, impl=impl)
+
+
+def test_tensor_path_needs_a_bf16_table():
+    need_cuda()
+    idx = torch.zeros((1, 2, 16), dtype=torch.int32, device="cuda")
+    logp = torch.zeros((1, 2, 16), dtype=torch.float32, device="cuda")
+    emb = torch.zeros((100, 64), dtype=torch.float32, device="cuda")
+    W = torch.zeros((64, 64), dtype=torch.float32, device="cuda")
+    with pytest.raises(dfl.DFlash2Error) as e:
+        dfl.pair_select(idx, logp, None, emb, W, impl=dfl.SELECT_TENSOR)
+    assert e.value.status == 2  # DFLASH2_EDTYPE
 
 
 def test_exact_ties_resolve_like_the_oracle(orc):
@@ -94,7 +113,34 @@ def test_exact_ties_resolve_like_the_oracle(orc):
     logp = np.full((B, G, 16), -2.0, np.float32)
     emb = (rng.standard_normal((V, d)) / 8).astype(np.float32)
     W = np.zeros((d, d), np.float32)
-    run_and_check(orc, idx, logp, rng.integers(0, V, B).astype(np.int32), emb, W)
+    anchor = rng.integers(0, V, B).astype(np.int32)
+    run_and_check(orc, idx, logp, anchor, emb, W)
+    embb = synth.to_bf16_bits(emb)
+    for impl in IMPLS:
+        run_and_check(orc, idx, logp, anchor, embb, W, impl=impl)
+
+
+def test_tensor_path_one_hot_embeddings_fix_the_orientation(orc):
+    """One-hot bf16 embeddings make pair(a, b) = W[a][b] exactly: the tensor
+    path must use W, not W^T, and split W's fp32 values into planes without
+    loss (W entries with more mantissa bits than bf16 holds)."""
+    need_cuda()
+    rng = np.random.default_rng(31)
+    d, V, B, G = 64, 64, 4, 3
+    emb = synth.to_bf16_bits(np.eye(V, d, dtype=np.float32))
+    W = (rng.standard_normal((d, d)) * (1 + 2 ** -20)).astype(np.float32)
+    idx = np.stack([np.stack([rng.choice(V, 16, replace=False) for _ in range(G)])
+                    for _ in range(B)]).astype(np.int32)
+    logp = np.zeros((B, G, 16), np.float32)
+    anchor = rng.integers(0, V, B).astype(np.int32)
+    for impl in IMPLS:
+        tok, rank, score = (to_host(t) for t in dfl.pair_select(
+            to_dev(idx), to_dev(logp), to_dev(anchor), to_dev(emb), to_dev(W), impl=impl))
+        for b in range(B):
+            expect = W[anchor[b], tok[b, 0]] + sum(W[tok[b, i - 1], tok[b, i]] for i in range(1, G))
+            assert abs(score[b] - expect) <= 1e-6 * (1 + abs(expect)), (impl, b)
+        otok, orank, oscore = orc.pair_select(idx, logp, anchor, emb, W)
+        np.testing.assert_array_equal(rank, orank)
 
 
 def test_batch_invariance(orc):

@@ -46,12 +46,15 @@ def drafted_tokens(orc, w, b, rng, mode):
 
 # ------------------------------------------------------------------ greedy
 def check_greedy(orc, target, draft_tok):
+    """Both greedy entries (the full verify and the early-exit one) against
+    the oracle: bit-exact n_accept and out_tok."""
     need_cuda()
-    n, out = dfl.verify_greedy(to_dev(target), to_dev(draft_tok))
-    torch.cuda.synchronize()
     on, oout = orc.verify_greedy(target, draft_tok)
-    np.testing.assert_array_equal(to_host(n), on)
-    np.testing.assert_array_equal(to_host(out), oout)
+    for early in (False, True):
+        n, out = dfl.verify_greedy(to_dev(target), to_dev(draft_tok), early_exit=early)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(to_host(n), on)
+        np.testing.assert_array_equal(to_host(out), oout)
     return on
 
 
@@ -88,6 +91,31 @@ def test_greedy_ragged(orc, V):
     d[::2, 2] = (d[::2, 2] + 1) % V
     check_greedy(orc, t, d)
     check_greedy(orc, synth.to_bf16_bits(t), d)
+
+
+def test_greedy_early_exit_every_mismatch_row(orc):
+    """The first mismatch at every row 0..G (and none), many sequences per
+    row, a workspace shared by consecutive calls: the early exit skips the
+    rows after it and still returns the full verify's results."""
+    rng = np.random.default_rng(12)
+    B, G, V = 64, 7, 20000
+    t = (rng.standard_normal((B, G + 1, V)) * 3).astype(np.float32)
+    d = t.argmax(axis=2)[:, :G].astype(np.int32)
+    cut = np.arange(B) % (G + 1)
+    for i in range(B):
+        if cut[i] < G:
+            d[i, cut[i]] = (d[i, cut[i]] + 1 + i) % V
+            d[i, cut[i] + 1:] = rng.integers(0, V, G - cut[i] - 1)
+    ws = dfl.Workspace(torch.device("cuda"))
+    on, oout = orc.verify_greedy(t, d)
+    np.testing.assert_array_equal(on, np.minimum(cut, G))
+    for arr in (t, synth.to_bf16_bits(t), t):
+        n, out = dfl.verify_greedy(to_dev(arr), to_dev(d), ws=ws, early_exit=True)
+        torch.cuda.synchronize()
+        o2 = orc.verify_greedy(arr, d)
+        np.testing.assert_array_equal(to_host(n), o2[0])
+        np.testing.assert_array_equal(to_host(out), o2[1])
+    assert dfl.device_errors() == 0
 
 
 def test_greedy_max_block(orc):
