@@ -53,7 +53,8 @@ HEADLINE = "b32"
 OTHER_WORKLOADS = ("b1", "b8", "ctx16")
 FLUSH_BYTES = 256 << 20
 CALLS = ("topk_softmax", "pair_select", "verify_sample", "verify_greedy", "dynconv2")
-CYCLE_KINDS = ("sampling", "greedy", "greedy_early_exit", "sampling_truncated", "dynconv2")
+CYCLE_KINDS = ("sampling", "greedy", "greedy_early_exit", "sampling_truncated", "dynconv2",
+               "dynconv2_packed")
 CYCLE_DEF = ("topk_softmax_ex -> pair_select -> verify_sample_ex -> verify_greedy -> dynconv2 "
              "over one batch (every hot-path call once)")
 DESCRIBE = {
@@ -93,9 +94,13 @@ def parse():
                     help="print the pair selector's time for both implementations (CUDA cores, "
                          "tensor cores) over a range of batch sizes, L2 flushed before every "
                          "call, instead of a bench line")
-    ap.add_argument("--only", choices=list(CALLS), default=None,
-                    help="run and time one call of the headline workload only (for profiling); "
-                         "prints a per-call line, not a bench line")
+    ap.add_argument("--only", choices=list(CALLS) + ["verify_greedy_early_exit",
+                                                     "verify_sample_trunc", "dynconv2_packed"],
+                    default=None,
+                    help="run and time one call only (for profiling); prints a per-call line, "
+                         "not a bench line")
+    ap.add_argument("--workload", choices=["b1", "b8", "b32", "ctx16"], default=HEADLINE,
+                    help="the workload --only runs (default the headline, b32)")
     return ap.parse_args()
 
 
@@ -484,9 +489,9 @@ def run_drafter_layer(args):
                           "us_with_convs": round(res[True], 2),
                           "conv_share": round((res[True] - res[False]) / res[True], 4),
                           "conv_bytes": conv_bytes, "layer_weight_bytes": layer_w_bytes},
-        "pages": "+0.7 % of the cycle for the convs (a conv adding ~3 % params); here each conv "
-                 "has a dense [2H, H] tap (the tiny configuration's 256 -> 512 form), so the "
-                 "four convs stream ~%.0f MB against the layer's %.0f MB of weights"
+        "pages": "+0.7 %% of the cycle for the convs (a conv adding ~3 %% params); here each "
+                 "conv has a dense [2H, H] tap (the tiny configuration's 256 -> 512 form), so "
+                 "the four convs stream ~%.0f MB against the layer's %.0f MB of weights"
                  % (conv_bytes / 1e6, layer_w_bytes / 1e6)}), flush=True)
 
 
@@ -578,6 +583,9 @@ class Bench:
         self.sel = synth.gen_selector(w)
         self.E, self.Wsel, self.Wtap = (self.dev_t(self.sel.emb), self.dev_t(self.sel.W),
                                         self.dev_t(self.sets[0][1].w_tap))
+        # the tap weights packed once for the tensor-core path (model parameters,
+        # packed at load time, outside every timed region)
+        self.Wpk = dfl.PackedTap(self.Wtap) if w.dtype == 1 else None
         self.inputs = []
         for b, c in self.sets:
             self.inputs.append(dict(
@@ -643,6 +651,8 @@ class Bench:
             ("verify_sample_trunc", lambda: dfl.verify_sample_trunc(
                 inp["T"], inp["Q"], outs["sel"][0], w.seed, step, inp["sid"], w.inv_temperature,
                 20, 0.95, out=outs["samp"], ws=ws)),
+            ("dynconv2_packed", lambda: dfl.dynconv2(inp["x"], inp["xp"], self.Wpk,
+                                                     out=outs["conv"])),
         ]
 
     def cycle_calls(self, kind, k, step):
@@ -656,7 +666,8 @@ class Bench:
                "greedy": ["topk_softmax", "pair_select", "verify_greedy"],
                "greedy_early_exit": ["topk_softmax", "pair_select", "verify_greedy_early_exit"],
                "sampling_truncated": ["topk_softmax", "pair_select", "verify_sample_trunc"],
-               "dynconv2": ["dynconv2"]}[kind]
+               "dynconv2": ["dynconv2"],
+               "dynconv2_packed": ["dynconv2_packed"]}[kind]
         return [(n, allc[n]) for n in seq]
 
     def timed_graph(self, kind, K, W, step0=0, events=True):
@@ -741,16 +752,22 @@ class Bench:
         torch.cuda.synchronize(dev)
         return e0.elapsed_time(e1) / K
 
-    def isolated_calls(self, K, step0=0):
+    def isolated_calls(self, K, step0=0, only=None):
         """Each call alone with L2 flushed before it (a 256 MB write then a
-        read of the same buffer, outside the timed intervals): {call: mean ms}."""
+        read of the same buffer, outside the timed intervals): {call: mean ms}.
+        only: that call alone (the five calls, or a verify variant)."""
         torch, dev = self.torch, self.dev
         stream = torch.cuda.current_stream(dev)
         flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
         sink = torch.zeros((), dtype=torch.int64, device=dev)
         evs = []
         for s in range(K):
-            for name, fn in self.calls(s % 2, step0 + s):
+            todo = self.calls(s % 2, step0 + s) + self.extra_calls(s % 2, step0 + s)
+            if only is not None:
+                todo = [(n, f) for n, f in todo if n == only]
+            else:
+                todo = todo[:len(CALLS)]
+            for name, fn in todo:
                 flush.fill_(s & 0xFF)
                 sink.add_(flush.view(torch.int64).sum())
                 e0 = torch.cuda.Event(enable_timing=True)
@@ -958,6 +975,11 @@ def measure_workload(name, args, rank, world, dev, barrier, peak, headline):
                          "top-p 0.95, T = 1; target and draft rows streamed once)"},
             "dynconv2": {"calls_per_s": round(world * 1000.0 / cyc["dynconv2"], 1),
                          "us": round(cyc["dynconv2"] * 1e3, 2)},
+            "dynconv2_packed": {
+                "calls_per_s": round(world * 1000.0 / cyc["dynconv2_packed"], 1),
+                "us": round(cyc["dynconv2_packed"] * 1e3, 2),
+                "GBps": round(alg["dynconv2"] / (cyc["dynconv2_packed"] * 1e-3) / 1e9, 1),
+                "calls": "dflash2_dynconv2_packed: the tap weights packed once at load time"},
         },
         "calls": calls,
         "calls_isolated": summarize_calls(w, B, iso, peak),
@@ -991,13 +1013,22 @@ def run_ours(args, rank, world, local_rank, pool):
 
     peak, peak_kind = peaks()
     if args.only:
-        bw = Bench(HEADLINE, rank, dev)
+        bw = Bench(args.workload, rank, dev)
         for s in range(max(args.warmup, 3)):
-            dict(bw.calls(s % 2, s))[args.only]()
-        iso = bw.isolated_calls(args.steps)
+            for name, fn in bw.calls(s % 2, s):
+                if name in ("topk_softmax", "pair_select") or name == args.only:
+                    fn()  # the path the verifies read comes from the selector
+            if args.only in ("verify_greedy_early_exit", "verify_sample_trunc",
+                             "dynconv2_packed"):
+                dict(bw.extra_calls(s % 2, s))[args.only]()
+        iso = bw.isolated_calls(args.steps, only=args.only)
         if rank == 0:
             us = iso[args.only] * 1e3
-            nbytes = algorithmic_bytes(bw.w, bw.B)[args.only]
+            alg = algorithmic_bytes(bw.w, bw.B)
+            alg["verify_greedy_early_exit"] = alg["verify_greedy"]
+            alg["verify_sample_trunc"] = 2 * bw.B * (2 * bw.w.G + 1) * bw.w.V
+            alg["dynconv2_packed"] = alg["dynconv2"]
+            nbytes = alg[args.only]
             print(json.dumps({"only": args.only, "us": round(us, 2), "algorithmic_bytes": nbytes,
                               "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1),
                               "steps": args.steps}), flush=True)

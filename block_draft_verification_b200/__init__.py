@@ -13,7 +13,8 @@ import torch
 
 __all__ = ["F32", "BF16", "Q_SOFTMAX", "Q_ONEHOT", "K", "DFlash2Error", "lib", "workspace_bytes",
            "Workspace", "topk_softmax", "pair_select", "verify_greedy", "verify_sample",
-           "verify_sample_trunc", "dynconv2", "status_string", "version", "device_errors"]
+           "verify_sample_trunc", "dynconv2", "PackedTap", "status_string", "version",
+           "device_errors"]
 
 F32, BF16 = 0, 1
 Q_SOFTMAX, Q_ONEHOT = 0, 1
@@ -61,6 +62,10 @@ def lib():
         L.dflash2_verify_sample_trunc.argtypes = [vp, vp, i32, i32, i32, i64, vp, f32, i32, f32,
                                                   u64, u32, vp, i32, vp, vp, vp, vp, vp, sz, vp]
         L.dflash2_dynconv2.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]
+        L.dflash2_dynconv2_packed.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]
+        L.dflash2_dynconv2_pack.argtypes = [vp, i32, i32, vp, vp]
+        L.dflash2_dynconv2_packed_bytes.argtypes = [i32, i32]
+        L.dflash2_dynconv2_packed_bytes.restype = sz
         L.dflash2_dynconv2_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.dflash2_dynconv2_workspace_bytes.restype = sz
         L.dflash2_device_errors.argtypes = [i32]
@@ -68,7 +73,8 @@ def lib():
         for f in ("dflash2_topk_softmax", "dflash2_topk_softmax_ex", "dflash2_pair_select",
                   "dflash2_pair_select_ex", "dflash2_verify_greedy_early_exit",
                   "dflash2_verify_greedy", "dflash2_verify_sample", "dflash2_verify_sample_ex",
-                  "dflash2_verify_sample_trunc", "dflash2_dynconv2"):
+                  "dflash2_verify_sample_trunc", "dflash2_dynconv2", "dflash2_dynconv2_pack",
+                  "dflash2_dynconv2_packed"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -312,8 +318,26 @@ def verify_sample_trunc(target, draft, draft_tok, seed, step, seq_id=None, inv_t
     return out
 
 
+class PackedTap:
+    """Tap weights [2H, H] bf16 packed once for the tensor-core path
+    (dflash2_dynconv2_pack); pass it to dynconv2 in place of w_tap."""
+
+    def __init__(self, w_tap):
+        _cuda(w_tap)
+        if w_tap.dtype != torch.bfloat16:
+            raise TypeError("packed tap weights are bf16")
+        self.H = w_tap.shape[1]
+        n = int(lib().dflash2_dynconv2_packed_bytes(BF16, self.H))
+        self.buf = torch.empty(n, dtype=torch.uint8, device=w_tap.device)
+        _check("dflash2_dynconv2_pack", lib().dflash2_dynconv2_pack(
+            _p(w_tap.contiguous()), BF16, self.H, _p(self.buf), _stream(w_tap.device)))
+
+
 def dynconv2(x, x_prev, w_tap, out=None, ws=None):
-    """x [B, T, H], x_prev [B, H], w_tap [2H, H] (one dtype) -> out [B, T, H]."""
+    """x [B, T, H], x_prev [B, H], w_tap [2H, H] (one dtype) or a PackedTap ->
+    out [B, T, H]."""
+    if isinstance(w_tap, PackedTap):
+        return _dynconv2_packed(x, x_prev, w_tap, out, ws)
     _cuda(x, x_prev, w_tap)
     B, T, H = x.shape
     if out is None:
@@ -326,4 +350,20 @@ def dynconv2(x, x_prev, w_tap, out=None, ws=None):
     _check("dflash2_dynconv2", lib().dflash2_dynconv2(
         _p(x.contiguous()), _p(x_prev.contiguous()), _p(w_tap.contiguous()), _dtype(x), B, T, H,
         _p(out), wp, wb, _stream(x.device)))
+    return out
+
+
+def _dynconv2_packed(x, x_prev, pk, out, ws):
+    _cuda(x, x_prev)
+    B, T, H = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    need = lib().dflash2_dynconv2_workspace_bytes(BF16, B, T, H)
+    if ws is None:
+        ws = _ws_cache.setdefault((x.device.index, torch.cuda.current_stream(x.device).cuda_stream),
+                                  Workspace(x.device))
+    wp, wb = ws.args_bytes(need)
+    _check("dflash2_dynconv2_packed", lib().dflash2_dynconv2_packed(
+        _p(x.contiguous()), _p(x_prev.contiguous()), _p(pk.buf), _dtype(x), B, T, H, _p(out), wp,
+        wb, _stream(x.device)))
     return out

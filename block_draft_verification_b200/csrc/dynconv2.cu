@@ -100,7 +100,8 @@ using namespace dfl;
 using namespace dfl_host;
 
 int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_tap, int B, int T,
-                               int H, void* out, void* ws, cudaStream_t s);
+                               int H, void* out, void* ws, cudaStream_t s, const void* w_packed);
+int dflash2_dynconv2_tc_pack(const void* w_tap, int H, void* packed, cudaStream_t s);
 size_t dflash2_dynconv2_tc_workspace(int64_t ntok, int H);
 
 static bool dynconv_shape_ok(int B, int T, int H) {
@@ -130,8 +131,37 @@ extern "C" int dflash2_dynconv2(const void* x, const void* x_prev, const void* w
     if (need > 0 && (!ws || !aligned(ws, 256) || ws_bytes < need)) return DFLASH2_EWORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     if (dtype == DFLASH2_BF16)  // tensor cores (tcgen05 + TMA), dynconv2_tc.cu
-        return dflash2_dynconv2_tc_launch(x, x_prev, w_tap, B, T, H, out, ws, s);
+        return dflash2_dynconv2_tc_launch(x, x_prev, w_tap, B, T, H, out, ws, s, nullptr);
     dynconv2_simt_kernel<false><<<(unsigned)blocks, NT, 0, s>>>(x, x_prev, w_tap, T, H, (int)ntok,
                                                                 out);
     return launch_status();
+}
+
+extern "C" size_t dflash2_dynconv2_packed_bytes(int dtype, int H) {
+    if (dtype != DFLASH2_BF16 || !dynconv_shape_ok(0, 0, H)) return 0;
+    return (size_t)4 * H * H;
+}
+
+extern "C" int dflash2_dynconv2_pack(const void* w_tap, int dtype, int H, void* w_packed,
+                                     dflash2_stream_t stream) {
+    if (dtype != DFLASH2_BF16) return DFLASH2_EDTYPE;  // the packed form feeds the tensor cores
+    if (!dynconv_shape_ok(0, 0, H)) return DFLASH2_ESHAPE;
+    if (!w_tap || !w_packed) return DFLASH2_EINVAL;
+    if (!aligned(w_tap, 16) || !aligned(w_packed, 256)) return DFLASH2_EALIGN;
+    return dflash2_dynconv2_tc_pack(w_tap, H, w_packed, (cudaStream_t)stream);
+}
+
+extern "C" int dflash2_dynconv2_packed(const void* x, const void* x_prev, const void* w_packed,
+                                       int dtype, int B, int T, int H, void* out, void* ws,
+                                       size_t ws_bytes, dflash2_stream_t stream) {
+    if (dtype != DFLASH2_BF16) return DFLASH2_EDTYPE;
+    if (!dynconv_shape_ok(B, T, H)) return DFLASH2_ESHAPE;
+    if ((int64_t)B * T == 0) return DFLASH2_OK;
+    if (!x || !x_prev || !w_packed || !out) return DFLASH2_EINVAL;
+    if (!aligned(x, 16) || !aligned(x_prev, 16) || !aligned(w_packed, 256) || !aligned(out, 16))
+        return DFLASH2_EALIGN;
+    const size_t need = dflash2_dynconv2_workspace_bytes(dtype, B, T, H);
+    if (!ws || !aligned(ws, 256) || ws_bytes < need) return DFLASH2_EWORKSPACE;
+    return dflash2_dynconv2_tc_launch(x, x_prev, nullptr, B, T, H, out, ws, (cudaStream_t)stream,
+                                      w_packed);
 }

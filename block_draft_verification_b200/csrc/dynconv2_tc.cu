@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     const __grid_constant__ CUtensorMap map_xe, const __grid_constant__ CUtensorMap map_pe,
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ x_prev,
     __nv_bfloat16* __restrict__ out, TcShape sh, float4* __restrict__ partial,
-    unsigned* __restrict__ flags) {
+    unsigned* __restrict__ flags, const uint8_t* __restrict__ wpk) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // two rings, 1024-byte aligned for the 128-byte swizzle: W tiles (HBM,
     // deeper) and X tiles (L2), each with its own full / empty barriers
@@ -194,7 +194,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
             const int tile = (int)(step / sh.nkb), kb = (int)(step - (int64_t)tile * sh.nkb);
             const int ct = tile / sh.nh, hb = tile - ct * sh.nh;
             mbar_expect_tx(full0 + 8 * st, tx);
-            if (is_w) {
+            if (is_w && wpk) {
+                // packed weights: the stage's 16 KB image, contiguous in memory
+                bulk_g2s_nx(smem_u32(wring + st * TC_A_BYTES),
+                            wpk + ((int64_t)hb * sh.nkb + kb) * TC_A_BYTES, (uint32_t)TC_A_BYTES,
+                            full0 + 8 * st);
+            } else if (is_w) {
                 // one box of the 4-D view (k, 16 channels, a|b, 16-channel block):
                 // accumulator rows 32q .. 32q+15 are a of channels h0+16q ..
                 // h0+16q+15, rows 32q+16 .. 32q+31 are b of the same channels
@@ -568,7 +573,7 @@ size_t dflash2_dynconv2_tc_workspace(int64_t ntok, int H) {
 // 16-byte aligned pointers and a large enough 256-byte aligned workspace,
 // checked by the caller).  Returns a dflash2 status.
 int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_tap, int B, int T,
-                               int H, void* out, void* ws, cudaStream_t s) {
+                               int H, void* out, void* ws, cudaStream_t s, const void* w_packed) {
     using namespace dfl;
     const int ntok = B * T;
     int dev = 0, sms = 0;
@@ -577,7 +582,9 @@ int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_
         return DFLASH2_ECUDA;
     const TcPlan P = tc_plan(ntok, H, sms);
     CUtensorMap mw, mx;
-    if (!make_wmap(&mw, w_tap, H)) return DFLASH2_ECUDA;
+    // (with packed weights the map is built over the packed buffer, which has
+    // the same size, and never used)
+    if (!make_wmap(&mw, w_packed ? w_packed : w_tap, H)) return DFLASH2_ECUDA;
     if (!make_map(&mx, x, (uint64_t)H, (uint64_t)ntok, TC_BK, (uint32_t)P.BN)) return DFLASH2_ECUDA;
     // epilogue staging: an owned tile's x rows and the x_prev rows of the
     // (at most R) batches its tokens belong to, 128 bytes per row, unswizzled
@@ -623,9 +630,39 @@ int dflash2_dynconv2_tc_launch(const void* x, const void* x_prev, const void* w_
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, dynconv2_tc_kernel, mw, mx, mxe, mpe, (const __nv_bfloat16*)x,
                            (const __nv_bfloat16*)x_prev, (__nv_bfloat16*)out, sh, part,
-                           flags) != cudaSuccess)
+                           flags, (const uint8_t*)w_packed) != cudaSuccess)
         return DFLASH2_ECUDA;
     return DFLASH2_OK;
+}
+
+namespace dfl {
+// W_tap [2H, H] bf16 (nn.Linear layout) rewritten as the W stages of the
+// tensor-core kernel: block (hb, kb), hb = 64-channel block, kb = 64-wide K
+// block, at byte (hb * H/64 + kb) * 16 KB holds the 128 x 64 tile the
+// producer's 4-D box brings in -- row 32 q + 16 ab + ch is channel
+// 64 hb + 16 q + ch of W_a (ab = 0) or W_b (ab = 1), its 64 K elements in
+// 16-byte chunks placed by the 128-byte swizzle (chunk c of row r at chunk
+// c ^ (r mod 8)).  One CTA per block, four 16-byte chunks per thread.
+__global__ void __launch_bounds__(256) dynconv2_pack_kernel(const uint4* __restrict__ w, int H,
+                                                            uint4* __restrict__ packed) {
+    const int nkb = H / TC_BK;
+    const int blk = blockIdx.x, hb = blk / nkb, kb = blk - hb * nkb;
+    const int rowv = H / 8;  // 16-byte vectors per W_tap row
+    for (int qi = threadIdx.x; qi < TC_A_BYTES / 16; qi += blockDim.x) {
+        const int r = qi >> 3, c = qi & 7;
+        const int q = r >> 5, ab = (r >> 4) & 1, ch = r & 15;
+        const int64_t g = (int64_t)ab * H + (int64_t)hb * TC_CH + q * 16 + ch;
+        packed[(int64_t)blk * (TC_A_BYTES / 16) + r * 8 + (c ^ (r & 7))] =
+            __ldg(&w[g * rowv + kb * (TC_BK / 8) + c]);
+    }
+}
+}  // namespace dfl
+
+int dflash2_dynconv2_tc_pack(const void* w_tap, int H, void* packed, cudaStream_t s) {
+    using namespace dfl;
+    const int blocks = (H / TC_CH) * (H / TC_BK);
+    dynconv2_pack_kernel<<<blocks, 256, 0, s>>>((const uint4*)w_tap, H, (uint4*)packed);
+    return cudaGetLastError() == cudaSuccess ? DFLASH2_OK : DFLASH2_ECUDA;
 }
 
 unsigned dfl_errors_dynconv(int clear) {

@@ -291,10 +291,12 @@ extern "C" int dflash2_pair_select_ex(const int32_t* idx, const float* logp,
     const Layout L = select_layout(B, G);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return DFLASH2_EWORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
-    // the tensor cores take every bf16 table (the choice never depends on B,
-    // so a sequence's result does not depend on the batch it runs in)
+    // automatic choice: the tensor cores for bf16 tables from DFLASH2_SELECT_TC_MIN_B
+    // sequences on (one CTA per sequence: its latency stays flat while the
+    // CUDA-core path's grid of B G CTAs grows past one wave), the CUDA cores below
     const bool tensor = impl == DFLASH2_SELECT_TENSOR ||
-                        (impl == DFLASH2_SELECT_AUTO && emb_dtype == DFLASH2_BF16);
+                        (impl == DFLASH2_SELECT_AUTO && emb_dtype == DFLASH2_BF16 &&
+                         B >= DFLASH2_SELECT_TC_MIN_B);
     if (tensor)
         return dfl_pair_select_tc(idx, logp, anchor, emb, V, d, W, B, G, path_tok, path_rank,
                                   path_score, s);

@@ -93,49 +93,59 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_kernel(
 }
 
 // ------------------------------------------------------------------ sampling, the scan
-// (maximum, fp64 sum of exp2((x - maximum) c)) of one row from its S chunk
-// partials, by one warp: lane l takes chunks l, l + 32, ... (the first four of
-// them held in registers), the maximum, then the fp64 sum against it in
-// chunk order per lane and a fixed butterfly across the lanes.  The order
-// depends on S alone, so a row's result does not depend on its batch.
-__device__ __forceinline__ LseD row_lse(const LseD* p, int S, float c2) {
-    const int lane = threadIdx.x & 31;
-    constexpr int RH = 4;
-    float pm[RH];
-    double ps[RH];
+// (maximum, fp64 sum of exp2((x - maximum) c)) of rows r0 .. r0+7 (the first
+// nrows of them) from their S chunk partials, lane-parallel: lanes 4j .. 4j+3
+// take row r0 + j, lane 4j + s its chunks s, s + 4, ... (the first 4 RC of
+// them held in registers, so a row of up to 4 RC chunks is read once); the
+// maximum, then the fp64 sum against it in chunk order; two butterfly steps
+// within the four lanes.  Every lane of group j returns row r0 + j's pair.
+constexpr int RC = 12;
+__device__ __forceinline__ void rows_lse8(const LseD* P, int S, int r0, int nrows, float c2,
+                                          float& Mo, double& So) {
+    const int lane = threadIdx.x & 31, j = lane >> 2, sub = lane & 3;
+    const bool on = j < nrows;
+    const LseD* p = P + (int64_t)(r0 + (on ? j : 0)) * S;
+    float pm[RC];
+    double ps[RC];
 #pragma unroll
-    for (int i = 0; i < RH; ++i) {
-        const int c = lane + 32 * i;
+    for (int i = 0; i < RC; ++i) {
+        const int c = sub + 4 * i;
         pm[i] = -INFINITY;
         ps[i] = 0.0;
-        if (c < S) {
+        if (on && c < S) {
             pm[i] = __ldcg(&p[c].m);
             ps[i] = __ldcg(&p[c].s);
         }
     }
     float M = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < RH; ++i) M = fmaxf(M, pm[i]);
-    for (int c = lane + 32 * RH; c < S; c += 32) M = fmaxf(M, __ldcg(&p[c].m));
-    M = warp_max(M);
+    for (int i = 0; i < RC; ++i) M = fmaxf(M, pm[i]);
+    if (on)
+        for (int c = sub + 4 * RC; c < S; c += 4) M = fmaxf(M, __ldcg(&p[c].m));
+    M = fmaxf(M, __shfl_xor_sync(FULL, M, 1));
+    M = fmaxf(M, __shfl_xor_sync(FULL, M, 2));
     double t = 0.0;
     if (M != -INFINITY) {
 #pragma unroll
-        for (int i = 0; i < RH; ++i)
+        for (int i = 0; i < RC; ++i)
             if (pm[i] != -INFINITY) t += ps[i] * exp2(((double)pm[i] - (double)M) * (double)c2);
-        for (int c = lane + 32 * RH; c < S; c += 32) {
-            const float m = __ldcg(&p[c].m);
-            if (m != -INFINITY) t += __ldcg(&p[c].s) * exp2(((double)m - (double)M) * (double)c2);
-        }
+        if (on)
+            for (int c = sub + 4 * RC; c < S; c += 4) {
+                const float m = __ldcg(&p[c].m);
+                if (m != -INFINITY) t += __ldcg(&p[c].s) * exp2(((double)m - (double)M) * (double)c2);
+            }
     }
-    return LseD{M, 0.0f, warp_sum(t)};
+    t += __shfl_xor_sync(FULL, t, 1);
+    t += __shfl_xor_sync(FULL, t, 2);
+    Mo = M;
+    So = t;
 }
 
-// The accept tests of one sequence, by the warp that completed its last row:
-// lane j takes target row j (and draft row j) from the row statistics.
+// The accept tests of one sequence, by the warp whose unit completed it:
+// lane j takes target row j (and draft row j) from the chunk partials.
 __device__ __forceinline__ void sample_finish(
-    const void* __restrict__ target, const void* __restrict__ draft, const LseD* RS, int G,
-    int64_t V, int es, float inv_t, const int32_t* __restrict__ draft_tok,
+    const void* __restrict__ target, const void* __restrict__ draft, const LseD* P, int G,
+    int64_t V, int S, int es, float inv_t, float c2, const int32_t* __restrict__ draft_tok,
     uint64_t seed, uint32_t step, uint32_t sid, int q_mode, int b, int32_t* __restrict__ n_accept,
     int32_t* __restrict__ out_tok, float* __restrict__ ratio_dbg, float* __restrict__ u_dbg,
     SampleInfo* __restrict__ info, const float* __restrict__ q_max, const float* __restrict__ q_lse) {
@@ -165,11 +175,23 @@ __device__ __forceinline__ void sample_finish(
         lnq = (double)q_lse[(int64_t)b * G + lane];
     }
     const bool scan_q = q_mode == DFLASH2_Q_SOFTMAX && !given;
-    if (lane <= G) lt = LseD{__ldcg(&RS[lane].m), 0.0f, __ldcg(&RS[lane].s)};
-    if (scan_q && lane < G) {
-        lq = LseD{__ldcg(&RS[G + 1 + lane].m), 0.0f, __ldcg(&RS[G + 1 + lane].s)};
-        lnq = log(lq.s);
+    const int nrows = scan_q ? 2 * G + 1 : G + 1;
+    for (int r0 = 0; r0 < nrows; r0 += 8) {
+        float Mr;
+        double Sr;
+        rows_lse8(P, S, r0, min(8, nrows - r0), c2, Mr, Sr);
+        // lane j takes target row j (and draft row j, row G + 1 + j) from group row - r0
+        const int jt = lane - r0, jq = lane + G + 1 - r0;
+        const float mt_ = __shfl_sync(FULL, Mr, 4 * (jt & 7));
+        const double st_ = __shfl_sync(FULL, Sr, 4 * (jt & 7));
+        if (lane <= G && jt >= 0 && jt < 8) lt = LseD{mt_, 0.0f, st_};
+        if (scan_q) {
+            const float mq_ = __shfl_sync(FULL, Mr, 4 * (jq & 7));
+            const double sq_ = __shfl_sync(FULL, Sr, 4 * (jq & 7));
+            if (lane < G && jq >= 0 && jq < 8) lq = LseD{mq_, 0.0f, sq_};
+        }
     }
+    if (scan_q && lane < G) lnq = log(lq.s);
     bool reject = false;
     if (lane < G) {
         // lp = z_t[d] - logZ_t = (x - m) * invT - ln(s); likewise lq
@@ -563,13 +585,10 @@ __device__ __forceinline__ SampleInfo load_info(const SampleInfo* p) {
 //
 // Scan: units are (sequence b, row rr, chunk): rows 0..G of a sequence are
 // its target rows, G+1..2G its draft rows (when their normalisers are not
-// given).  Warp w of the grid takes units w, w + W, w + 2 W, ... (W warps),
-// so all warps move through the sequences together and sequences finish one
-// after another during the scan.  A unit's partial is the chunk maximum and
-// the fp64 sum of exp2((x - m) c) against it; the warp whose publish
-// completes a row reduces the row's partials to its statistics, and the warp
-// whose row completes a sequence decides its accept tests from those and
-// appends it to the finish queue -- while the other warps still scan.
+// given).  A unit's partial is the chunk maximum and the fp64 sum of
+// exp2((x - m) c) against it; a warp publishes its consecutive units of one
+// sequence together, and the warp whose add completes the sequence decides
+// its accept tests and appends it to the finish queue.
 //
 // Draw: draw unit i is (position i / ND in the finish queue, unit i % ND of
 // the row), and CTA c takes units c, c + grid, c + 2 grid, ... in that order
@@ -583,10 +602,10 @@ __device__ __forceinline__ SampleInfo load_info(const SampleInfo* p) {
 //
 // Control words (zero on entry, zero again on exit; sample_ctl_words): the
 // queue length and the count of warps done, each in a 128-byte line of its
-// own; per sequence its finished rows [B] and its draw units [B]; per row
-// its scan units [B R]; then the finish queue, one line per position (b + 1
-// of the sequence that finished there), so the warps polling it spread over
-// as many lines and never meet the counters' adds.
+// own; scan units per sequence [B]; draw units per sequence [B]; then the
+// finish queue, one line per position (b + 1 of the sequence that finished
+// there), so the warps polling it spread over as many lines and never meet
+// the counters' adds.
 template <bool BF16, bool TMA>
 __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
     const void* __restrict__ target, const void* __restrict__ draft, int B, int G, int64_t V, int S,
@@ -594,21 +613,20 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
     uint64_t seed, uint32_t step, const uint32_t* __restrict__ seq_id, int q_mode,
     int32_t* __restrict__ n_accept, int32_t* __restrict__ out_tok, float* __restrict__ ratio_dbg,
     float* __restrict__ u_dbg, LseD* __restrict__ part, double* __restrict__ dsum,
-    SampleInfo* __restrict__ info, LseD* __restrict__ rowstat, unsigned* __restrict__ ctl,
-    const float* __restrict__ q_max, const float* __restrict__ q_lse) {
+    SampleInfo* __restrict__ info, unsigned* __restrict__ ctl, const float* __restrict__ q_max,
+    const float* __restrict__ q_lse) {
     using C = ChunkT<BF16>;
     constexpr int ES = C::ES;
     constexpr int LEN = C::LEN;
     extern __shared__ __align__(128) uint8_t ring[];
     __shared__ __align__(8) uint64_t bars[2 * NCW];
     __shared__ unsigned s_next;  // this CTA's next draw unit (k: unit blockIdx.x + k grid)
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31;
     unsigned* const fin_count = ctl;
     unsigned* const retire = ctl + CTL_LINE;
-    unsigned* const seqcnt = ctl + 2 * CTL_LINE;
-    unsigned* const dcount = seqcnt + B;
-    unsigned* const rowcnt = dcount + B;
-    unsigned* const fin = ctl + sample_fin_off(B, rows_per_seq);
+    unsigned* const counters = ctl + 2 * CTL_LINE;
+    unsigned* const dcount = counters + B;
+    unsigned* const fin = ctl + sample_fin_off(B);
     auto rowp = [&](int64_t b, int rr) {
         return (rr <= G) ? (const char*)target + (b * (G + 1) + rr) * V * ES
                          : (const char*)draft + (b * G + (rr - G - 1)) * V * ES;
@@ -626,40 +644,23 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
             }
         }
     }
-    WarpRing r{ring + 2 * warp * SLOT_BYTES, smem_u32(&bars[2 * warp])};
-    if (TMA && lane == 0) {
-        mbar_init(r.bar, 1);
-        mbar_init(r.bar + 8, 1);
-        mbar_fence_init();
-    }
     __syncthreads();
-    const int64_t gw = (int64_t)blockIdx.x * NCW + warp, nw = (int64_t)gridDim.x * NCW;
-    const int n = gw < units ? (int)((units - 1 - gw) / nw + 1) : 0;
-    const int64_t per_seq = (int64_t)rows_per_seq * S;
-    auto unit_of = [&](int k, int64_t& b, int& rr, int& c) {
-        const int64_t u = gw + (int64_t)k * nw;
-        b = u / per_seq;
-        const int64_t rem = u - b * per_seq;
-        rr = (int)(rem / S);
-        c = (int)(rem - (int64_t)rr * S);
+    int64_t lo, hi;
+    warp_range(units, lo, hi);
+    const int n = (int)(hi - lo);
+    UnitCursor uc, ic;  // (sequence, row, chunk) being reduced / to bring in
+    uc.init(lo, S, rows_per_seq);
+    ic = uc;
+    auto src = [&](const UnitCursor& cu, const char*& p, uint32_t& bytes) {
+        const int64_t v0 = (int64_t)cu.c * LEN;
+        p = rowp(cu.g, cu.r) + v0 * ES;
+        bytes = (uint32_t)(min((int64_t)LEN, V - v0) * ES);
     };
-    auto bring = [&](int k) {
-        int64_t b;
-        int rr, c;
-        unit_of(k, b, rr, c);
-        const int64_t v0 = (int64_t)c * LEN;
-        warp_ring_load(r, k, rowp(b, rr) + v0 * ES, (uint32_t)(min((int64_t)LEN, V - v0) * ES),
-                       C::NEG_INF_WORD);
-    };
-    if (TMA) {
-        for (int k = 0; k < 2 && k < n; ++k) bring(k);
-        __syncwarp();
-    }
-    for (int k = 0; k < n; ++k) {
-        int64_t b;
-        int rr, c;
-        unit_of(k, b, rr, c);
-        const int64_t v0 = (int64_t)c * LEN;
+    WarpRing r{nullptr, 0u};
+    if (TMA) r = warp_ring_start(ring, bars, n, ic, C::NEG_INF_WORD, src);
+    unsigned seg = 0;
+    for (int k = 0; k < n; ++k, uc.next()) {
+        const int64_t b = uc.g, v0 = (int64_t)uc.c * LEN;
         const int len = (int)min((int64_t)LEN, V - v0);
         float M;
         double Ssum;
@@ -672,39 +673,29 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
             uint32_t vm[NVL];
             M = warp_max(chunk_pass1<BF16>(view, vm));
             Ssum = chunk_expsum<BF16>(view, M, c2);
-            r.done(k);
-            if (k + 2 < n) bring(k + 2);
+            warp_ring_next(r, k, n, ic, C::NEG_INF_WORD, src);
         } else {
-            const GlobalView<BF16> view{(const uint8_t*)rowp(b, rr), v0, len};
+            const GlobalView<BF16> view{(const uint8_t*)rowp(b, uc.r), v0, len};
             uint32_t vm[NVL];
             M = warp_max(chunk_pass1<BF16>(view, vm));
             Ssum = chunk_expsum<BF16>(view, M, c2);
         }
-        const int64_t grow = b * rows_per_seq + rr;
-        bool last = false;
-        if (lane == 0) {
-            part[grow * S + c] = LseD{M, 0.0f, Ssum};
-            last = publish(&rowcnt[grow], 1u, (unsigned)S);
-        }
-        if (!__shfl_sync(FULL, last, 0)) continue;
-        __syncwarp();  // lane 0's acquire covers the whole warp's reads
-        // the row is complete: its statistics
-        const LseD st = row_lse(part + grow * S, S, c2);
-        bool lastrow = false;
-        if (lane == 0) {
-            rowstat[grow] = st;
-            rowcnt[grow] = 0u;
-            lastrow = publish(&seqcnt[b], 1u, (unsigned)rows_per_seq);
-        }
-        if (!__shfl_sync(FULL, lastrow, 0)) continue;
-        __syncwarp();
-        // the sequence is complete: its accept tests
-        sample_finish(target, draft, rowstat + b * rows_per_seq, G, V, ES, inv_t, draft_tok, seed,
-                      step, seq_id ? seq_id[b] : (uint32_t)b, q_mode, (int)b, n_accept, out_tok,
-                      ratio_dbg, u_dbg, info, q_max, q_lse);
-        if (lane == 0) {  // info[b] (lane 0's store) before the queue entry
-            seqcnt[b] = 0u;
-            st_release(&fin[(size_t)atomicAdd(fin_count, 1u) * CTL_LINE], (unsigned)b + 1u);
+        ++seg;
+        if (lane == 0) part[(b * rows_per_seq + uc.r) * S + uc.c] = LseD{M, 0.0f, Ssum};
+        if (k + 1 == n || uc.last_of_group()) {  // done with this sequence: publish
+            bool last = false;
+            if (lane == 0) last = publish(&counters[b], seg, (unsigned)(rows_per_seq * S));
+            if (__shfl_sync(FULL, last, 0)) {
+                __syncwarp();  // lane 0's acquire covers the whole warp's reads
+                sample_finish(target, draft, part + b * rows_per_seq * S, G, V, S, ES, inv_t, c2,
+                              draft_tok, seed, step, seq_id ? seq_id[b] : (uint32_t)b, q_mode,
+                              (int)b, n_accept, out_tok, ratio_dbg, u_dbg, info, q_max, q_lse);
+                if (lane == 0) {  // info[b] (lane 0's store) before the queue entry
+                    counters[b] = 0u;
+                    st_release(&fin[(size_t)atomicAdd(fin_count, 1u) * CTL_LINE], (unsigned)b + 1u);
+                }
+            }
+            seg = 0;
         }
     }
 
@@ -877,7 +868,6 @@ static int verify_sample_impl(const void* target, const void* draft, int dtype, 
     LseD* part = (LseD*)((char*)ws + L.part_off);
     double* dsum = (double*)((char*)ws + L.part2_off);
     SampleInfo* info = (SampleInfo*)((char*)ws + L.info_off);
-    LseD* rowstat = (LseD*)((char*)info + align256((size_t)B * sizeof(SampleInfo)));
     if (!L.self_clean && cudaMemsetAsync(ctl, 0, L.counters_bytes, s) != cudaSuccess)
         return DFLASH2_ECUDA;
     const void* q = (q_mode == DFLASH2_Q_SOFTMAX) ? draft : nullptr;
@@ -899,8 +889,8 @@ static int verify_sample_impl(const void* target, const void* draft, int dtype, 
         cfg.numAttrs = 1;
         if (cudaLaunchKernelEx(&cfg, kern, target, q, B, G, V, (int)S, rows_per_seq, units,
                                inv_temperature, c2, draft_tok, seed, step, seq_id, q_mode,
-                               n_accept, out_tok, ratio_dbg, u_dbg, part, dsum, info, rowstat,
-                               ctl, q_max, q_lse) != cudaSuccess)
+                               n_accept, out_tok, ratio_dbg, u_dbg, part, dsum, info, ctl, q_max,
+                               q_lse) != cudaSuccess)
             return DFLASH2_ECUDA;
         return DFLASH2_OK;
     };

@@ -33,6 +33,9 @@
 
 namespace dfl {
 
+constexpr int EE_MAX_TOK = 1024;  // drafted tokens (B G) the shared key table holds
+constexpr int EE_MAX_SEQ = 1024;  // sequences the shared skip words hold
+
 template <bool BF16>
 __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_ee_kernel(
     const void* __restrict__ target, int B, int G, int64_t V, int S, int64_t units,
@@ -44,7 +47,25 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_ee_kernel(
     constexpr int LEN = Ch::LEN;
     extern __shared__ __align__(128) uint8_t ring[];
     __shared__ __align__(8) uint64_t bars[2 * NCW];
+    __shared__ uint64_t s_dkey[EE_MAX_TOK];  // the drafted tokens' keys [B][G]
+    __shared__ unsigned s_skip[EE_MAX_SEQ];  // this CTA's view of the skip words [B]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // every drafted token's key in shared memory (one round of loads per CTA),
+    // so no unit waits on a dependent global load before its copy is issued
+    for (int i = threadIdx.x; i < B * G; i += blockDim.x) {
+        const int64_t b = i / G, j = i - b * G;
+        const int32_t d = draft_tok[i];
+        uint64_t dk = 0ull;  // a token outside [0, V): every chunk beats it (a mismatch)
+        if ((uint32_t)d < (uint64_t)V) {
+            const int64_t o = (b * (G + 1) + j) * V + d;
+            const float x = BF16 ? __uint_as_float((uint32_t)((const uint16_t*)target)[o] << 16)
+                                 : ((const float*)target)[o];
+            dk = make_key(x, (uint32_t)d);
+        }
+        s_dkey[i] = dk;
+    }
+    for (int i = threadIdx.x; i < B; i += blockDim.x) s_skip[i] = 0u;
+    __syncthreads();
     const int64_t gw = (int64_t)blockIdx.x * NCW + warp, nw = (int64_t)gridDim.x * NCW;
     const int n = gw < units ? (int)((units - 1 - gw) / nw + 1) : 0;
     const int64_t per_row = (int64_t)B * S;
@@ -62,35 +83,28 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_ee_kernel(
     bool skip[2] = {true, true};
     uint64_t dkey[2] = {0ull, 0ull};
     uint32_t issued[2] = {0u, 0u};
-    // bring unit k into slot S_ (= k & 1, a compile-time constant so the
-    // per-slot state stays in registers)
-    auto bring = [&](auto S_, int k) {
-        constexpr int s = decltype(S_)::value;
+    auto unit_of = [&](int k, int64_t& b, int& j, int& c) {
         const int64_t u = gw + (int64_t)k * nw;
-        const int j = (int)(u / per_row);
+        j = (int)(u / per_row);
         const int64_t rem = u - (int64_t)j * per_row;
-        const int64_t b = rem / S;
-        const int c = (int)(rem - b * S);
+        b = rem / S;
+        c = (int)(rem - b * S);
+    };
+    // bring unit k into slot S_ (= k & 1, a compile-time constant so the
+    // per-slot state stays in registers); seen: a value of the sequence's
+    // global skip word read earlier (or 0)
+    auto bring = [&](auto S_, int k, unsigned seen) {
+        constexpr int s = decltype(S_)::value;
+        int64_t b;
+        int j, c;
+        unit_of(k, b, j, c);
         sb[s] = b;
         sj[s] = j;
         sc[s] = c;
-        unsigned sk = 0u;
-        uint64_t dk = ~0ull;  // the row after the block has no drafted token
-        if (lane == 0) {
-            sk = (j + *(volatile unsigned*)&skipw[b] > (unsigned)(G + 1)) ? 1u : 0u;
-            if (!sk && j < G) {
-                const int32_t d = draft_tok[b * G + j];
-                dk = 0ull;  // a token outside [0, V): every chunk beats it (a mismatch)
-                if ((uint32_t)d < (uint64_t)V) {
-                    const int64_t o = (b * (G + 1) + j) * V + d;
-                    const float x = BF16 ? __uint_as_float((uint32_t)((const uint16_t*)target)[o] << 16)
-                                         : ((const float*)target)[o];
-                    dk = make_key(x, (uint32_t)d);
-                }
-            }
-        }
-        skip[s] = __shfl_sync(FULL, sk, 0) != 0u;
-        dkey[s] = shfl64(dk, 0);
+        // any lower bound of the skip word is safe: skipping less is never wrong
+        const unsigned w = max(seen, *(volatile unsigned*)&s_skip[b]);
+        skip[s] = j + w > (unsigned)(G + 1);
+        dkey[s] = (j < G) ? s_dkey[b * G + j] : ~0ull;  // row G has no drafted token
         if (!skip[s]) {
             const int64_t v0 = (int64_t)c * LEN;
             const char* p = (const char*)target + ((b * (G + 1) + j) * V + v0) * ES;
@@ -106,6 +120,15 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_ee_kernel(
         constexpr int s = decltype(S_)::value;
         const int64_t b = sb[s];
         const int j = sj[s], c = sc[s];
+        // the skip word of unit k + 2's sequence, read now and used after this
+        // unit's work, so its latency is hidden
+        unsigned seen = 0u;
+        if (k + 2 < n) {
+            int64_t b2;
+            int j2, c2;
+            unit_of(k + 2, b2, j2, c2);
+            seen = *(volatile unsigned*)&skipw[b2];
+        }
         if (!skip[s]) {
             if (!mbar_wait(r.bar + 8 * s, (issued[s] - 1u) & 1u)) {
                 if (lane == 0) {  // the copies still in flight land before the CTA may exit
@@ -121,10 +144,13 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_ee_kernel(
             r.done(k);
             if (lane == 0) {
                 part[(b * (G + 1) + j) * S + c] = key;
-                if (j < G && key > dkey[s]) atomicMax(&skipw[b], (unsigned)(G + 1 - j));
+                if (j < G && key > dkey[s]) {
+                    atomicMax(&skipw[b], (unsigned)(G + 1 - j));
+                    atomicMax(&s_skip[b], (unsigned)(G + 1 - j));
+                }
             }
         }
-        if (k + 2 < n) bring(S_, k + 2);
+        if (k + 2 < n) bring(S_, k + 2, seen);
         bool last = false;
         if (lane == 0) last = publish(&counters[b], 1u, (unsigned)((G + 1) * S));
         if (__shfl_sync(FULL, last, 0)) {
@@ -137,8 +163,8 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_ee_kernel(
         }
         return true;
     };
-    if (n > 0) bring(Slot0{}, 0);
-    if (n > 1) bring(Slot1{}, 1);
+    if (n > 0) bring(Slot0{}, 0, 0u);
+    if (n > 1) bring(Slot1{}, 1, 0u);
     for (int k = 0; k < n; k += 2) {
         if (!step(Slot0{}, k)) return;
         if (k + 1 < n && !step(Slot1{}, k + 1)) return;
@@ -166,8 +192,10 @@ extern "C" int dflash2_verify_greedy_early_exit(const void* target, int dtype, i
     if (!aligned(target, es) || !aligned(draft_tok, 4) || !aligned(n_accept, 4) ||
         !aligned(out_tok, 4))
         return DFLASH2_EALIGN;
-    // rows that TMA cannot copy in whole chunks: the full verify (same results)
-    if (!aligned(target, 16) || (V * es) % 16 != 0)
+    // rows that TMA cannot copy in whole chunks, or more drafted tokens than
+    // the kernel's shared tables hold: the full verify (same results)
+    if (!aligned(target, 16) || (V * es) % 16 != 0 || (int64_t)B * G > EE_MAX_TOK ||
+        B > EE_MAX_SEQ)
         return dflash2_verify_greedy(target, dtype, B, G, V, draft_tok, n_accept, out_tok, ws,
                                      ws_bytes, stream);
     const int64_t S = row_chunks(V, es);

@@ -87,24 +87,19 @@ inline Layout greedy_ee_layout(int B, int G, int64_t V, int es) {
     const int64_t S = row_chunks(V, es);
     return make_layout((size_t)B * 8, (size_t)((int64_t)B * (G + 1) * S) * sizeof(uint64_t));
 }
-// Sampling: the control words (two queue words, a line each; per sequence
-// its finished rows and its draw units [B] each; per row its scan units
-// [B R], R = rows per sequence; the finish queue, a line per position), the
-// scan's per-unit partials, the draw's per-unit lane prefixes (32 per chunk
-// of the drawn row, and 32 of scratch), and the per-sequence hand-over to the
-// draw followed by the rows' statistics.
+// Sampling: the control words (two queue words, a line each; scan and draw
+// counters [B] each; the finish queue, a line per position), the scan's
+// per-unit partials, the draw's per-unit lane prefixes (32 per chunk of the
+// drawn row, and 32 of scratch) and the per-sequence hand-over to the draw.
 constexpr int CTL_LINE = 32;  // words in a 128-byte line
-__host__ __device__ inline size_t sample_fin_off(int B, int R) {
-    return (2 * (size_t)CTL_LINE + 2 * (size_t)B + (size_t)B * R + CTL_LINE - 1) / CTL_LINE *
-           CTL_LINE;
+__host__ __device__ inline size_t sample_fin_off(int B) {
+    return (2 * (size_t)CTL_LINE + 2 * (size_t)B + CTL_LINE - 1) / CTL_LINE * CTL_LINE;
 }
-inline size_t sample_ctl_words(int B, int R) { return sample_fin_off(B, R) + (size_t)B * CTL_LINE; }
+inline size_t sample_ctl_words(int B) { return sample_fin_off(B) + (size_t)B * CTL_LINE; }
 inline Layout sample_layout(int B, int G, int64_t V, int es) {
     const int64_t S = row_chunks(V, es);
-    const int R = 2 * G + 1;
-    return make_layout(sample_ctl_words(B, R) * 4, (size_t)((int64_t)B * R * S) * sizeof(LseD),
-                       (size_t)((int64_t)B * S + 1) * 32 * sizeof(double),
-                       align256((size_t)B * sizeof(SampleInfo)) + (size_t)B * R * sizeof(LseD));
+    return make_layout(sample_ctl_words(B) * 4, (size_t)((int64_t)B * (2 * G + 1) * S) * sizeof(LseD),
+                       (size_t)((int64_t)B * S + 1) * 32 * sizeof(double), (size_t)B * sizeof(SampleInfo));
 }
 // Truncated sampling verify: control words (per row a counter and a shared
 // top-32 bound, per sequence a counter of finished rows; rows = B (2G+1), the

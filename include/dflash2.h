@@ -58,7 +58,9 @@
  *     needs no initialisation.  Two calls that may run concurrently need
  *     separate workspaces.
  *   - Results are deterministic: a sequence's outputs depend only on its own
- *     inputs (and seq_id), not on the batch it runs in or on B.
+ *     inputs (and seq_id), not on the batch it runs in or on B -- except that
+ *     dflash2_pair_select picks its implementation by B (see
+ *     dflash2_pair_select_ex, which fixes it).
  */
 #ifndef DFLASH2_H
 #define DFLASH2_H
@@ -212,10 +214,15 @@ DFLASH2_API int dflash2_pair_select(const int32_t* idx, const float* logp, const
  * dflash2_pair_select with the implementation named.  Results of the two
  * differ only in fp32 rounding (both accumulate in fp32; the path can differ
  * only where two paths' scores are within that rounding).
- * impl  DFLASH2_SELECT_AUTO: the tensor cores for bf16 tables, the CUDA cores
- *       for fp32 ones -- a rule that depends on the dtype only, never on B,
- *       so a sequence's result does not depend on its batch (what
- *       dflash2_pair_select does);
+ * impl  DFLASH2_SELECT_AUTO: the tensor cores for bf16 tables when
+ *       B >= DFLASH2_SELECT_TC_MIN_B, else the CUDA cores (what
+ *       dflash2_pair_select does).  The threshold is where the tensor path
+ *       became the faster one in measurements on B200 (block 8, d = 128, L2
+ *       cold): 18.4 us at every B up to 128 against the CUDA cores' 16.4 us
+ *       up to B = 16, 20.5 us at 32 and 45 us at 128.  A sequence's path_score
+ *       can therefore differ in its last bits between batches on either side
+ *       of the threshold; a caller that needs the same bits at every B names
+ *       the implementation;
  *       DFLASH2_SELECT_SIMT: the CUDA cores, fp32 FMAs, one CTA per
  *       (sequence, position) and a last-CTA recursion (any table);
  *       DFLASH2_SELECT_TENSOR: one CTA per sequence, F = E W on tcgen05 with
@@ -228,6 +235,7 @@ DFLASH2_API int dflash2_pair_select(const int32_t* idx, const float* logp, const
 #define DFLASH2_SELECT_AUTO 0
 #define DFLASH2_SELECT_SIMT 1
 #define DFLASH2_SELECT_TENSOR 2
+#define DFLASH2_SELECT_TC_MIN_B 32
 DFLASH2_API int dflash2_pair_select_ex(const int32_t* idx, const float* logp, const int32_t* anchor,
                                        const void* emb, int emb_dtype, int64_t V, int d,
                                        const float* W, int B, int G, int32_t* path_tok,
@@ -388,6 +396,32 @@ DFLASH2_API int dflash2_dynconv2(const void* x, const void* x_prev, const void* 
 /* Workspace bytes dflash2_dynconv2 needs for these arguments (0 when it
  * needs none or the arguments are invalid). */
 DFLASH2_API size_t dflash2_dynconv2_workspace_bytes(int dtype, int B, int T, int H);
+
+/*
+ * The tap weights in the tensor-core path's own layout, for a caller that
+ * keeps the weights across calls (they are model parameters).  The pages
+ * have no counterpart: this is a storage format.  In nn.Linear layout every
+ * 16 KB stage the kernel streams is 128 row pieces of 128 bytes, H * 2 bytes
+ * apart; packed, each stage is one contiguous 16 KB block, read with one bulk
+ * copy.  The arithmetic, and so every output bit, is that of dflash2_dynconv2.
+ *
+ * dflash2_dynconv2_packed_bytes  bytes of the packed form (4 H^2 for bf16;
+ *   0 for fp32, which has no tensor-core path, or an invalid H).
+ * dflash2_dynconv2_pack  w_tap [2H, H] bf16 (16-byte aligned) -> w_packed
+ *   (256-byte aligned, dflash2_dynconv2_packed_bytes bytes), one launch on
+ *   `stream`; bf16 only (DFLASH2_EDTYPE otherwise).  The layout is internal:
+ *   block (hb, kb) at (hb * H/64 + kb) * 16 KB holds channels 64 hb ..
+ *   64 hb + 63 of W_a and W_b (interleaved by 16) over K elements 64 kb ..
+ *   64 kb + 63, 128-byte swizzled.
+ * dflash2_dynconv2_packed  dflash2_dynconv2 with the packed weights; the
+ *   same arguments otherwise, the same workspace, the same results.
+ */
+DFLASH2_API size_t dflash2_dynconv2_packed_bytes(int dtype, int H);
+DFLASH2_API int dflash2_dynconv2_pack(const void* w_tap, int dtype, int H, void* w_packed,
+                                      dflash2_stream_t stream);
+DFLASH2_API int dflash2_dynconv2_packed(const void* x, const void* x_prev, const void* w_packed,
+                                        int dtype, int B, int T, int H, void* out, void* ws,
+                                        size_t ws_bytes, dflash2_stream_t stream);
 
 /*
  * Device-side error flags of the kernels on the current device (0 = none).

@@ -221,3 +221,23 @@ def test_verify_trunc_validation(L):
     assert trunc(o=ODD) == EALIGN
     assert trunc(wsb=0) == EWORKSPACE
     assert trunc(k=32, p=1.0, V=8, wsb=1 << 30) != ESHAPE   # top_k > V keeps V
+
+
+def test_dynconv_packed_validation(L):
+    assert L.dflash2_dynconv2_packed_bytes(1, 5120) == 4 * 5120 * 5120
+    assert L.dflash2_dynconv2_packed_bytes(0, 5120) == 0     # fp32 has no packed form
+    assert L.dflash2_dynconv2_packed_bytes(1, 100) == 0
+    assert L.dflash2_dynconv2_pack(P, 0, 128, P2, S0) == EDTYPE
+    assert L.dflash2_dynconv2_pack(P, 1, 100, P2, S0) == ESHAPE
+    assert L.dflash2_dynconv2_pack(None, 1, 128, P2, S0) == EINVAL
+    assert L.dflash2_dynconv2_pack(P, 1, 128, C.c_void_p(0x20010), S0) == EALIGN
+
+    def packed(x=P, xp=P, w=P2, dt=1, B=2, T=8, H=5120, out=P2, ws=P2, wsb=1 << 30):
+        return L.dflash2_dynconv2_packed(x, xp, w, dt, B, T, H, out, ws, wsb, S0)
+    assert packed(dt=0) == EDTYPE
+    assert packed(H=100) == ESHAPE
+    assert packed(T=0) == OK
+    assert packed(w=None) == EINVAL
+    assert packed(w=C.c_void_p(0x20010)) == EALIGN
+    assert packed(ws=None) == EWORKSPACE
+    assert packed(wsb=1000) == EWORKSPACE

@@ -75,3 +75,37 @@ def test_special_weights_exact(orc):
     for wt in (np.concatenate([eye, zero]), np.concatenate([zero, eye])):
         out = run(x, xp, wt)
         np.testing.assert_array_equal(out.astype(np.float64), orc.dynconv2(x, xp, wt))
+
+
+@pytest.mark.parametrize("name,B", [("b1", 1), ("b8", 8), ("b32", 32)])
+def test_packed_weights_give_the_same_bits(orc, name, B):
+    """dflash2_dynconv2_packed (the tap weights packed once, dflash2_dynconv2_pack)
+    reads the same bytes into the same shared-memory stages as dflash2_dynconv2:
+    every output bit is equal; and it matches the oracle on sampled sequences."""
+    need_cuda()
+    w = synth.WORKLOADS[name]
+    c = synth.gen_conv(w, B=B)
+    x, xp, wt = to_dev(c.x), to_dev(c.x_prev), to_dev(c.w_tap)
+    pk = dfl.PackedTap(wt)
+    a = dfl.dynconv2(x, xp, wt)
+    b = dfl.dynconv2(x, xp, pk)
+    torch.cuda.synchronize()
+    assert dfl.device_errors() == 0
+    np.testing.assert_array_equal(to_host(a), to_host(b))
+    s = [0, B - 1]
+    assert_close(as_f64(to_host(b)[s]), orc.dynconv2(c.x[s], c.x_prev[s], c.w_tap), RTOL_BF16,
+                 "packed")
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 1, 64), (3, 5, 192), (2, 40, 320)])
+def test_packed_weights_ragged_shapes(orc, B, T, H):
+    need_cuda()
+    rng = np.random.default_rng(B * 1000 + T * 10 + H)
+    x = synth.to_bf16_bits(rng.standard_normal((B, T, H)).astype(np.float32))
+    xp = synth.to_bf16_bits(rng.standard_normal((B, H)).astype(np.float32))
+    wt = synth.to_bf16_bits((rng.standard_normal((2 * H, H)) / np.sqrt(H)).astype(np.float32))
+    out = dfl.dynconv2(to_dev(x), to_dev(xp), dfl.PackedTap(to_dev(wt)))
+    torch.cuda.synchronize()
+    assert dfl.device_errors() == 0
+    np.testing.assert_array_equal(to_host(out), run(x, xp, wt))
+    assert_close(as_f64(to_host(out)), orc.dynconv2(x, xp, wt), RTOL_BF16, "packed ragged")

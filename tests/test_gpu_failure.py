@@ -3,10 +3,10 @@
 1. A bounded wait that runs out.  The sampling verify's draw warps wait
    (bounded, one second) for a sequence to be decided.  The test makes that
    wait run out by corrupting one word on the host, before the call: the
-   finished-row counter of the last sequence starts at 2^30 instead of 0, so
-   no publish of its rows ever brings it to the expected count (a small offset
-   could: a partial sum may land on it), the sequence is never decided and
-   never queued.  Its draw warps then give up
+   scan-unit counter of the last sequence starts at 2^30 instead of 0, so no
+   publish of its scan units ever brings it to the expected count (a small
+   offset could: a partial sum may land on it), the sequence is never decided
+   and never queued.  Its draw warps then give up
    after the bound, set error flag 16 and return; the call returns, the host
    reads the flag, re-zeroes the workspace's 64 KB control area as the
    header asks, and the next call is correct (checked against the oracle).
@@ -27,7 +27,7 @@ ERR_STREAM, ERR_INPUT = 16, 32
 CONTROL_BYTES = 65536
 # Sampling verify control words (workspace.cuh, sample layout): word 0 the
 # finish-queue length, word 32 the count of warps done (one 128-byte line
-# each), then one finished-row counter per sequence from word 64.
+# each), then one scan-unit counter per sequence from word 64.
 SCAN_COUNTER_WORD0 = 64
 
 
@@ -60,7 +60,7 @@ def test_draw_wait_runs_out_then_workspace_recovers(orc):
     np.testing.assert_array_equal(n0, on)
     np.testing.assert_array_equal(out0, oout)
     assert dfl.device_errors() == 0
-    # the last sequence's finished-row counter starts at 2^30: it is never decided
+    # the last sequence's scan-unit counter starts at 2^30: it is never decided
     ctl = ws.buf[:CONTROL_BYTES].view(torch.int32)
     ctl[SCAN_COUNTER_WORD0 + B - 1] = 1 << 30
     torch.cuda.synchronize()

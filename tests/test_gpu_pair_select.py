@@ -154,3 +154,21 @@ def test_batch_invariance(orc):
                                                to_dev(anchor[3:4]), E, Wd)]
     for a, o in zip(full, one):
         np.testing.assert_array_equal(a[3:4], o)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_named_implementation_is_batch_invariant(orc, impl):
+    """With the implementation named, a sequence's path and score are the same
+    bits in a batch of 40 (above the automatic threshold) and alone."""
+    need_cuda()
+    w = synth.WORKLOADS["b32"]
+    sel = synth.gen_selector(w)
+    idx, logp, anchor = oracle_inputs(orc, w, 40)
+    E, Wd = to_dev(sel.emb), to_dev(sel.W)
+    full = [to_host(t) for t in dfl.pair_select(to_dev(idx), to_dev(logp), to_dev(anchor), E, Wd,
+                                                impl=impl)]
+    for s in (0, 17, 39):
+        one = [to_host(t) for t in dfl.pair_select(to_dev(idx[s:s + 1]), to_dev(logp[s:s + 1]),
+                                                   to_dev(anchor[s:s + 1]), E, Wd, impl=impl)]
+        for a, o in zip(full, one):
+            np.testing.assert_array_equal(a[s:s + 1], o)
