@@ -82,6 +82,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--headline-only", action="store_true",
                     help="measure the headline workload only (no b1 / b8 / ctx16)")
+    ap.add_argument("--step-only", action="store_true",
+                    help="time only the headline cycle (the graph of K cycles and its per-call "
+                         "events): the launch list of exactly what `value` times, for profiling")
     ap.add_argument("--acceptance", action="store_true",
                     help="print the acceptance study (mean accepted tokens per verify step for "
                          "the top-1 path, the pair selector and the top-16 oracle path) instead "
@@ -910,6 +913,12 @@ def measure_workload(name, args, rank, world, dev, barrier, peak, headline):
     barrier()
     ms_step, _, note = bw.timed_graph("step", K, W, events=False)
     ms_ev, per_call, _ = bw.timed_graph("step", K, W, step0=500)
+    if args.step_only:
+        if rank == 0:
+            print(json.dumps({"step_only": name, "us_per_cycle": round(ms_step * 1e3, 2),
+                              "calls_us": {n: round(v * 1e3, 2) for n, v in per_call.items()}}),
+                  flush=True)
+        return bw, None
     cyc, cyc_calls = {}, {}
     for kind in CYCLE_KINDS:
         ms, _, _ = bw.timed_graph(kind, K, W, step0=1000, events=False)
@@ -1039,6 +1048,8 @@ def run_ours(args, rank, world, local_rank, pool):
     with sampler:
         bw, head = measure_workload(HEADLINE, args, rank, world, dev, barrier, peak, True)
     t_wall = time.perf_counter() - t_wall0
+    if head is None:  # --step-only
+        return
     others = {}
     if not args.headline_only:
         for name in OTHER_WORKLOADS:
@@ -1100,7 +1111,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     pool = None
     if (args.impl == "ours" and not args.acceptance and not args.only and world == 1
-            and not args.no_cpu_baseline and not args.drafter_layer and not args.select_sweep):
+            and not args.no_cpu_baseline and not args.drafter_layer and not args.select_sweep
+            and not args.step_only):
         # spawned before the first CUDA call; its workers build the oracle's
         # weights while the GPU runs
         pool = OraclePool(HEADLINE, max(1, min(usable_cores(), 32)))

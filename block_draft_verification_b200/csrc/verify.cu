@@ -231,9 +231,9 @@ __device__ __forceinline__ void sample_finish(
 
 // ------------------------------------------------------------------ sampling, the draw
 // A sequence draws from one row (target row n, with draft row n for the
-// residual).  The row is cut into draw units of one chunk (the scan's chunk
-// length, so a unit fills one ring slot), and lane l of the warp that takes
-// a unit owns its vectors NVL l .. NVL l + NVL - 1: a contiguous run of the
+// residual).  The row is cut into draw units of half a scan chunk (a unit
+// fills half a ring slot), and lane l of the warp that takes a unit owns its
+// vectors DRAW_NVL l .. DRAW_NVL l + DRAW_NVL - 1: a contiguous run of the
 // row in index order.  Per unit the lanes' inclusive prefix sums of their
 // weights are stored (fp64, lane order); units in row order, lanes in unit
 // order and elements in run order give the inverse CDF the draw walks.
@@ -249,6 +249,16 @@ __device__ __forceinline__ void sample_finish(
 //   residual is empty by rounding).
 // e^d - 1 for 0 < d <= 1/8: the Taylor series to d^5 (truncation below
 // 5e-8 relative there).
+// A draw unit is half a scan chunk: DRAW_NVL 16-byte vectors per lane, so a
+// row's draw work spreads over twice as many warps (most warps are idle by
+// the time the last sequences are decided).
+constexpr int DRAW_NVL = NVL / 2;
+template <bool BF16>
+__host__ __device__ constexpr int draw_len() { return 32 * DRAW_NVL * ChunkT<BF16>::VW; }
+__host__ __device__ inline int64_t draw_units(int64_t V, int es) {
+    const int64_t len = (int64_t)32 * DRAW_NVL * (16 / es);
+    return (V + len - 1) / len;
+}
 constexpr float EXPM1_SPLIT = 0.125f;
 __device__ __forceinline__ float expm1_small(float d) {
     float p = 1.0f / 120.0f;
@@ -294,7 +304,7 @@ __device__ __forceinline__ void draw_vec(int mode, const uint4& xt, const uint4&
 
 // This lane's weight sum over its run of a unit: fp32 pairwise within a
 // vector, fp64 across the run's vectors.  The lanes of a warp read the run's
-// vectors in rotated order (lane l starts at its vector l mod NVL), so the
+// vectors in rotated order (lane l starts at its vector l mod DRAW_NVL), so the
 // 16-byte reads of a quarter-warp fall in distinct banks; the order is fixed
 // per lane, so the sum is the same bits in any batch.
 template <bool BF16, bool RESID, class View>
@@ -305,8 +315,8 @@ __device__ __forceinline__ double draw_lane_sum(const View& vt, const View& vq,
     const int lane = threadIdx.x & 31;
     double s = 0.0;
 #pragma unroll 2
-    for (int g = 0; g < NVL; ++g) {
-        const int q = NVL * lane + ((g + lane) & (NVL - 1));
+    for (int g = 0; g < DRAW_NVL; ++g) {
+        const int q = DRAW_NVL * lane + ((g + lane) & (DRAW_NVL - 1));
         const uint4 xt = vt.vec(q);
         const uint4 xq = RESID ? vq.vec(q) : make_uint4(0u, 0u, 0u, 0u);
         float w[C::VW];
@@ -356,7 +366,7 @@ struct RowView {
 };
 
 // The walk inside the run holding t (first element rb, inverse CDF `base`
-// before it): lane j < NVL takes the run's vector j, the vector sums go
+// before it): lane j < DRAW_NVL takes the run's vector j, the vector sums go
 // through an inclusive warp scan, and the first lane with mass whose prefix
 // exceeds t walks its elements to the first whose running prefix exceeds t
 // (else its last element with mass; if no lane crosses, the run's last
@@ -370,7 +380,7 @@ __device__ __forceinline__ int64_t draw_walk(const char* trow, const char* qrow,
     float w[C::VW];
     double sj = 0.0;
     const int64_t i0 = rb + (int64_t)lane * C::VW;
-    if (lane < NVL) {
+    if (lane < DRAW_NVL) {
         const RowView<BF16, AL> vt{trow, i0, V}, vq{qrow, i0, V};
         const uint4 xt = vt.vec(0);
         const uint4 xq = (mode == 0) ? vq.vec(0) : make_uint4(0u, 0u, 0u, 0u);
@@ -411,7 +421,7 @@ __device__ __noinline__ bool draw_locate_p(const char* trow, int64_t V, int ND,
     using C = ChunkT<BF16>;
     double R = 0.0;
     for (int c = 0; c < ND; ++c) {
-        const RowView<BF16, AL> v{trow, (int64_t)c * C::LEN, V};
+        const RowView<BF16, AL> v{trow, (int64_t)c * draw_len<BF16>(), V};
         const double my = draw_lane_sum<BF16>(v, v, 2, I, c2, inv_t);
         R = __shfl_sync(FULL, warp_incl_scan(my) + R, 31);
     }
@@ -421,7 +431,7 @@ __device__ __noinline__ bool draw_locate_p(const char* trow, int64_t V, int ND,
     int lastc = -1, lastl = -1;
     double last_base = 0.0;
     for (int c = 0; c < ND; ++c) {
-        const RowView<BF16, AL> v{trow, (int64_t)c * C::LEN, V};
+        const RowView<BF16, AL> v{trow, (int64_t)c * draw_len<BF16>(), V};
         const double my = draw_lane_sum<BF16>(v, v, 2, I, c2, inv_t);
         const double incl = warp_incl_scan(my) + carry;
         const unsigned mass = __ballot_sync(FULL, my > 0.0);
@@ -536,7 +546,8 @@ __device__ __noinline__ void draw_pick(const char* trow, const char* qrow, int64
     int64_t pick = -1;
     if (lstar >= 0)
         pick = draw_walk<BF16, AL>(trow, qrow, V, mode, I, c2, inv_t,
-                                   (int64_t)cstar * C::LEN + (int64_t)lstar * NVL * C::VW, base, tt);
+                                   (int64_t)cstar * draw_len<BF16>() + (int64_t)lstar * DRAW_NVL * C::VW,
+                                   base, tt);
     if (lane == 0 && out) *out = (int32_t)pick;
 }
 
@@ -555,7 +566,7 @@ __device__ __noinline__ void warm_draw_code(const void* target, int64_t V, float
     I.n = I.mode = I.d = I.pad = 0;
     double my = 0.0;
     if (TMA) {
-        const SmemView<BF16> v{r.slot(0), 0, ChunkT<BF16>::LEN};
+        const SmemView<BF16> v{r.slot(0), 0, draw_len<BF16>()};
         my = draw_lane_sum<BF16, true>(v, v, I, -1, c2, inv_t);
     }
     scratch[lane] = (double)(lane + 1) + 0.0 * my;
@@ -700,7 +711,8 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
     }
 
     // ---- the draw
-    const int ND = S;  // draw units per row
+    const int ND = (int)draw_units(V, ES);  // draw units per row
+    constexpr int LEN_D = draw_len<BF16>();
     const unsigned total = (unsigned)B * (unsigned)ND;
     double* const dsum_scratch = dsum + (int64_t)B * ND * 32;  // 32 doubles
     int kk = n;  // this warp's next ring unit
@@ -729,14 +741,14 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
         __syncwarp();  // lane 0's acquire covers the warp's reads of info[b]
         const int b = (int)b1 - 1;
         const SampleInfo I = load_info(&info[b]);
-        const int64_t v0 = (int64_t)c * LEN;
+        const int64_t v0 = (int64_t)c * LEN_D;
         const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
         const char* qrow =
             (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
         double my;
         if (TMA) {
             const int nu = (I.mode == 0) ? 2 : 1;
-            const uint32_t bytes = (uint32_t)(min((int64_t)LEN, V - v0) * ES);
+            const uint32_t bytes = (uint32_t)(min((int64_t)LEN_D, V - v0) * ES);
             warp_ring_load(r, kk, trow + v0 * ES, bytes, C::NEG_INF_WORD);
             if (nu == 2) warp_ring_load(r, kk + 1, qrow + v0 * ES, bytes, C::NEG_INF_WORD);
             __syncwarp();
@@ -746,7 +758,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
                 warp_ring_abort(r, kk, kk + nu);
                 return;
             }
-            const SmemView<BF16> vt{r.slot(kk), v0, LEN}, vq{r.slot(kk + 1), v0, LEN};
+            const SmemView<BF16> vt{r.slot(kk), v0, LEN_D}, vq{r.slot(kk + 1), v0, LEN_D};
             my = draw_lane_sum<BF16>(vt, vq, I.mode, I, c2, inv_t);
             r.done(kk);  // both slots read: they may be refilled
             kk += nu;

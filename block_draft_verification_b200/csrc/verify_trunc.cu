@@ -109,6 +109,7 @@ __device__ __forceinline__ void top32_chunk(const View& v, CandBuf32& cb, uint64
                                             unsigned* thr, uint32_t& pub) {
     using C = ChunkT<BF16>;
     const int lane = threadIdx.x & 31, nv = v.nvec();
+    const uint32_t shared = *(volatile unsigned*)thr;  // used after pass 1 (its latency hidden)
     uint32_t vm[NVL];
     const float m = chunk_pass1<BF16>(v, vm);
     float tv = -INFINITY;
@@ -126,7 +127,6 @@ __device__ __forceinline__ void top32_chunk(const View& v, CandBuf32& cb, uint64
             if (lane == 0) atomicMax(thr, o);
         }
     }
-    const uint32_t shared = *(volatile unsigned*)thr;
     if (shared != 0u && (((uint64_t)shared << 32) - 1ull) > tkey) {
         tkey = ((uint64_t)shared << 32) - 1ull;
         tv = unord32(shared);

@@ -98,8 +98,10 @@ __host__ __device__ inline size_t sample_fin_off(int B) {
 inline size_t sample_ctl_words(int B) { return sample_fin_off(B) + (size_t)B * CTL_LINE; }
 inline Layout sample_layout(int B, int G, int64_t V, int es) {
     const int64_t S = row_chunks(V, es);
+    // the draw's units are half chunks: 2 S + 1 per row is enough
     return make_layout(sample_ctl_words(B) * 4, (size_t)((int64_t)B * (2 * G + 1) * S) * sizeof(LseD),
-                       (size_t)((int64_t)B * S + 1) * 32 * sizeof(double), (size_t)B * sizeof(SampleInfo));
+                       (size_t)((int64_t)B * (2 * S + 1) + 1) * 32 * sizeof(double),
+                       (size_t)B * sizeof(SampleInfo));
 }
 // Truncated sampling verify: control words (per row a counter and a shared
 // top-32 bound, per sequence a counter of finished rows; rows = B (2G+1), the
