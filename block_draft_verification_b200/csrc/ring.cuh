@@ -185,6 +185,13 @@ struct ChunkT {
         }
         return __uint_as_float(word(r, e));
     }
+    // The same for an index known only at run time (selects, no local memory).
+    __device__ static __forceinline__ float elem_at(const uint4& r, int e) {
+        const int wi = BF16 ? (e >> 1) : e;
+        const uint32_t wd = (wi & 2) ? ((wi & 1) ? r.w : r.z) : ((wi & 1) ? r.y : r.x);
+        if (BF16) return __uint_as_float((e & 1) ? (wd & 0xFFFF0000u) : (wd << 16));
+        return __uint_as_float(wd);
+    }
 };
 
 // The slot always holds SLOT_BYTES: past the chunk's n elements it is filled
@@ -305,31 +312,38 @@ __device__ __forceinline__ double warp_sum(double s) {
 }
 
 // sum over the vector's elements of exp2(x c2 - mc): fp32 pairwise within the
-// vector (index order), one FMA per exponent.
+// vector (index order), one FMA per exponent.  The FMAs and the first two
+// levels of the sum run on element pairs (fma / add .f32x2), each half
+// rounded as the scalar instruction rounds it.
 template <bool BF16>
 __device__ __forceinline__ float vec_expsum(const uint4& w, float c2, float nmc) {
     using C = ChunkT<BF16>;
-    float tt[C::VW];
+    const uint64_t cc = f2_pack(c2, c2), nn = f2_pack(nmc, nmc);
+    uint64_t p[C::VW / 2];  // exponentials of elements (2i, 2i + 1)
 #pragma unroll
-    for (int e = 0; e < C::VW; ++e) tt[e] = ex2(fmaf(C::elem(w, e), c2, nmc));
-#pragma unroll
-    for (int h = C::VW / 2; h > 0; h >>= 1)
-#pragma unroll
-        for (int e = 0; e < h; ++e) tt[e] += tt[e + h];
-    return tt[0];
+    for (int i = 0; i < C::VW / 2; ++i) {
+        const uint64_t a = f2_fma(f2_pack(C::elem(w, 2 * i), C::elem(w, 2 * i + 1)), cc, nn);
+        p[i] = f2_pack(ex2(f2_lo(a)), ex2(f2_hi(a)));
+    }
+    if (BF16) {
+        // a = (t0 + t4, t1 + t5), b = (t2 + t6, t3 + t7); then a + b, lo + hi
+        const uint64_t q = f2_add(f2_add(p[0], p[C::VW / 4]), f2_add(p[1], p[C::VW / 4 + 1]));
+        return f2_lo(q) + f2_hi(q);
+    }
+    // (t0 + t2, t1 + t3)
+    const uint64_t q = f2_add(p[0], p[1]);
+    return f2_lo(q) + f2_hi(q);
 }
 
-// Pass 2: the chunk's sum of exp2((x - M) c) against the warp maximum M (not
-// -inf).  Every exponent is one FMA x c2 - mc with mc = fl(M c2); the
-// product's rounding error M c2 - mc (exact in fp32 by the FMA) is taken out
-// once, in fp64.  Per lane: fp32 pairwise within a vector and over groups of
-// four vectors, fp64 across the groups; the warp's lanes in a fixed fp64
-// butterfly.  Every lane returns the same value.
+// Pass 2: the chunk's sum of exp2(x c2 - mc) with mc = fl(M c2), M the warp
+// maximum (not -inf): every exponent is one FMA.  Per lane: fp32 pairwise
+// within a vector and over groups of four vectors, fp64 across the groups;
+// the warp's lanes in a fixed fp64 butterfly.  Every lane returns the same
+// value.
 template <bool BF16, class View>
-__device__ __forceinline__ double chunk_expsum(const View& v, float M, float c2) {
+__device__ __forceinline__ double chunk_expsum_at_mc(const View& v, float M, float c2) {
     const int lane = threadIdx.x & 31;
-    const float mc = M * c2;
-    const float nmc = -mc;
+    const float nmc = -(M * c2);
     double s = 0.0;
 #pragma unroll
     for (int g = 0; g < NVL / 4; ++g) {
@@ -338,8 +352,14 @@ __device__ __forceinline__ double chunk_expsum(const View& v, float M, float c2)
         for (int j = 0; j < 4; ++j) e4[j] = vec_expsum<BF16>(v.vec_or(32 * (4 * g + j) + lane), c2, nmc);
         s += (double)((e4[0] + e4[1]) + (e4[2] + e4[3]));
     }
-    s = warp_sum(s);
-    return s * exp2(-(double)fmaf(M, c2, nmc));
+    return warp_sum(s);
+}
+// The same sum against M itself: the product's rounding error M c2 - mc
+// (exact in fp32 by the FMA) taken out once, in fp64.
+template <bool BF16, class View>
+__device__ __forceinline__ double chunk_expsum(const View& v, float M, float c2) {
+    const float mc = M * c2;
+    return chunk_expsum_at_mc<BF16>(v, M, c2) * exp2(-(double)fmaf(M, c2, -mc));
 }
 
 // ---------------------------------------------------------------------------

@@ -26,51 +26,56 @@
 
 namespace dfl {
 
-// Candidate buffer of one consumer warp: keys pushed during the exp pass,
-// merged into the running list whenever more than CAND_FLUSH are waiting (at
-// most 32 lanes x 8 elements arrive between two checks).
+// Candidate buffer of one consumer warp: keys pushed during the candidate
+// rounds, merged into the running list whenever more than CAND_FLUSH are
+// waiting (at most 32 lanes x 8 elements arrive between two checks) and at
+// the end of every chunk.  The count of waiting keys lives in a register of
+// the warp (the same value in every lane), not here.
 constexpr unsigned CAND_FLUSH = 64;
-constexpr unsigned SMALL_FLUSH = 4;  // up to this many keys are inserted one by one
 constexpr unsigned CAND_CAP = CAND_FLUSH + 32 * 8;
 struct CandBuf {
     uint64_t key[CAND_CAP];
-    unsigned n;
+    uint64_t out[K];  // the merged list, placed by rank
 };
 
-// Merge the buffered candidates into the running list (lanes 0..15 hold it,
-// descending; 0 = empty) sixteen at a time, and raise the threshold to the
-// list's 16th key once the list is full; a raised value also raises the
-// row's shared bound (thr: ord32 of a value at least 16 of the row's
-// elements reach; pub: what this warp last put there).  Warp-uniform.
-__device__ __forceinline__ void flush_candidates(CandBuf& cb, uint64_t& run, uint64_t& tkey,
-                                                 float& tv, unsigned* thr, uint32_t& pub) {
+// Merge the n buffered candidates into the running list (lanes 0..15 hold
+// it, descending; 0 = empty), up to 32 at a time, by rank: every key of the
+// union (keys are distinct) lands at its rank in it, so a batch costs one
+// broadcast read, two compares and a ballot per buffered key, and no sort.
+// Then the threshold rises to the list's 16th key once the list is full; a
+// raised value also raises the row's shared bound (thr: ord32 of a value at
+// least 16 of the row's elements reach; pub: what this warp last put there).
+// Warp-uniform; n is zero on return.
+__device__ __forceinline__ void flush_candidates(CandBuf& cb, unsigned& n, uint64_t& run,
+                                                 uint64_t& tkey, float& tv, unsigned* thr,
+                                                 uint32_t& pub) {
     const int lane = threadIdx.x & 31;
-    __syncwarp();
-    const unsigned n = *(volatile unsigned*)&cb.n;
-    if (n <= SMALL_FLUSH) {
-        // a few keys (the usual case once the list is full): insert each at
-        // its rank, found by one ballot, shifting the lower keys down a lane
-        for (unsigned i = 0; i < n; ++i) {
-            const uint64_t c = cb.key[i];
-            const unsigned above = __ballot_sync(FULL, lane < K && run > c);
-            const int pos = __popc(above);
-            const uint64_t up = shfl64_up1(run);
-            if (pos < K && lane < K && lane >= pos) run = (lane == pos) ? c : up;
+    __syncwarp();  // every lane's pushed keys are visible
+    for (unsigned base = 0; base < n; base += 32) {
+        const unsigned m = min(32u, n - base);
+        const uint64_t c = (unsigned)lane < m ? cb.key[base + lane] : 0ull;
+        unsigned rank_list = 0u;  // list keys above this lane's candidate
+        unsigned rank_new = 0u;   // batch keys above this lane's candidate
+        unsigned above_run = 0u;  // batch keys above this lane's list key
+#pragma unroll 4
+        for (unsigned j = 0; j < m; ++j) {
+            const uint64_t cj = cb.key[base + j];
+            const unsigned above = __ballot_sync(FULL, lane < K && run > cj);
+            if ((unsigned)lane == j) rank_list = __popc(above);
+            rank_new += cj > c;
+            above_run += cj > run;
         }
-    } else {
-        for (unsigned base = 0; base < n; base += K) {
-            uint64_t v = run;
-            if (lane >= K) {
-                const unsigned j = base + (unsigned)(lane - K);
-                v = (j < n) ? cb.key[j] : 0ull;
-            }
-            v = warp_sort_desc(v);
-            run = (lane < K) ? v : 0ull;
-        }
+        if (lane < K) cb.out[lane] = 0ull;
+        __syncwarp();
+        const unsigned pc = rank_list + rank_new;
+        if ((unsigned)lane < m && pc < K) cb.out[pc] = c;
+        const unsigned pr = (unsigned)lane + above_run;
+        if (lane < K && run != 0ull && pr < K) cb.out[pr] = run;
+        __syncwarp();
+        run = lane < K ? cb.out[lane] : 0ull;
+        __syncwarp();  // out is read before the next batch writes it
     }
-    __syncwarp();
-    if (lane == 0) cb.n = 0;
-    __syncwarp();
+    n = 0u;
     const uint64_t k16 = shfl64(run, K - 1);
     if (k16 > tkey) {
         tkey = k16;
@@ -91,21 +96,23 @@ __device__ __forceinline__ void flush_candidates(CandBuf& cb, uint64_t& run, uin
 //   largest lane maximum bounds the chunk's own top 16 (at least 16 elements
 //   are >= T); once it is full its 16th key is the bound.  The row's shared
 //   bound (a value at least 16 of the row's elements reach, raised by every
-//   warp whose list fills) replaces either when higher: no element below it
+//   warp whose list fills; `shared` is its value as read one chunk earlier,
+//   so the load's latency hides behind a whole chunk) replaces either when
+//   higher: no element below it
 //   can be in the row's top 16, so the merged result is the same exact set,
 //   while a segment's own list may hold fewer than 16 keys.
 //   Candidates: only the vectors whose maximum reaches the bound's value are
 //   looked at element by element (one per lane per round); keys beating the
 //   bound are pushed and merged whenever more than CAND_FLUSH wait, and the
 //   bound rises to the list's 16th key at every merge.
-//   Pass 2: the exponentials (chunk_expsum).
+//   Pass 2: the exponentials (chunk_expsum_at_mc: the sum against fl(M c),
+//   rescaled to the row maximum by the merge).
 template <bool BF16, class View>
 __device__ __forceinline__ void topk_chunk(const View& v, float c2, CandBuf& cb, float& M_out,
                                            double& S_out, uint64_t& run, unsigned* thr,
-                                           uint32_t& pub) {
+                                           uint32_t& pub, uint32_t shared) {
     using C = ChunkT<BF16>;
     const int lane = threadIdx.x & 31, nv = v.nvec();
-    const uint32_t shared = *(volatile unsigned*)thr;  // used after pass 1 (its latency hidden)
     uint32_t vm[NVL];
     const float m = chunk_pass1<BF16>(v, vm);
     const float M = warp_max(m);
@@ -137,51 +144,57 @@ __device__ __forceinline__ void topk_chunk(const View& v, float c2, CandBuf& cb,
     for (int i = 0; i < NVL; ++i)
         if (32 * i + lane < nv && any_ge<BF16>(vm[i], t2)) hits |= 1u << i;
     if (__any_sync(FULL, hits != 0u)) {
+        unsigned nbuf = 0u;  // keys waiting in cb (warp-uniform)
         while (__any_sync(FULL, hits != 0u)) {  // one vector per lane per round
-            uint64_t kk[C::VW];
-            unsigned msk = 0;
+            unsigned em = 0u;  // elements of the lane's vector that reach the bound
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            int q = 0;
             if (hits) {
                 const int i = __ffs(hits) - 1;
                 hits &= hits - 1u;
-                const int q = 32 * i + lane;
-                const uint4 w = v.vec(q);
+                q = 32 * i + lane;
+                w = v.vec(q);
 #pragma unroll
-                for (int e = 0; e < C::VW; ++e) {
-                    const float x = C::elem(w, e);
-                    kk[e] = make_key(x, (uint32_t)v.index(q, e));
-                    if (x >= tv && q * C::VW + e < v.n && kk[e] > tkey) msk |= 1u << e;
-                }
+                for (int e = 0; e < C::VW; ++e)
+                    if (C::elem(w, e) >= tv) em |= 1u << e;
+                // elements past the chunk's end read as -inf: they reach only a -inf bound
+                const int lim = v.n - q * C::VW;
+                if (lim < C::VW) em &= lim > 0 ? (1u << lim) - 1u : 0u;
             }
-            // this round's keys appended in lane order: one prefix sum, no atomics
-            const unsigned cnt = __popc(msk);
-            unsigned incl = cnt;
+            // Keys whose value equals the bound's but whose index part is below
+            // the list's 16th key are pushed too: the merge ranks them out.
+            const unsigned cnt = __popc(em);
+            // this round's keys appended in lane order: the exclusive prefix
+            // of the per-lane counts (at most 8: four bits) from four ballots
+            const unsigned below = (1u << lane) - 1u;
+            unsigned excl = 0u, total = 0u;
 #pragma unroll
-            for (int k = 1; k < 32; k <<= 1) {
-                const unsigned o = __shfl_up_sync(FULL, incl, k);
-                if (lane >= k) incl += o;
+            for (int bit = 0; bit < 4; ++bit) {
+                const unsigned b = __ballot_sync(FULL, (cnt >> bit) & 1u);
+                excl += (unsigned)__popc(b & below) << bit;
+                total += (unsigned)__popc(b) << bit;
             }
-            const unsigned base = *(volatile unsigned*)&cb.n;
-            unsigned pos = base + incl - cnt;
-#pragma unroll
-            for (int e = 0; e < C::VW; ++e)
-                if (msk & (1u << e)) cb.key[pos++] = kk[e];
-            const unsigned nn = base + __shfl_sync(FULL, incl, 31);
-            __syncwarp();
-            if (lane == 0) cb.n = nn;
-            __syncwarp();
-            if (nn > CAND_FLUSH) flush_candidates(cb, run, tkey, tv, thr, pub);
+            unsigned pos = nbuf + excl;
+            while (em) {
+                const int e = __ffs(em) - 1;
+                em &= em - 1u;
+                cb.key[pos++] = make_key(C::elem_at(w, e), (uint32_t)v.index(q, e));
+            }
+            nbuf += total;
+            if (nbuf > CAND_FLUSH) flush_candidates(cb, nbuf, run, tkey, tv, thr, pub);
         }
-        __syncwarp();
-        if (*(volatile unsigned*)&cb.n > 0u) flush_candidates(cb, run, tkey, tv, thr, pub);
+        if (nbuf > 0u) flush_candidates(cb, nbuf, run, tkey, tv, thr, pub);
     }
     M_out = M;
-    S_out = chunk_expsum<BF16>(v, M, c2);
+    S_out = chunk_expsum_at_mc<BF16>(v, M, c2);  // against fl(M c2); the merge rescales
 }
 
 // The row's final merge by one warp, after its last chunk was published:
 // the segment lists (bitonic merges in chunk order), the maximum, and the
 // fp64 sum of the chunk sums rescaled to it (lane c takes chunks c, c + 32,
-// ...; then a fixed butterfly).
+// ...; then a fixed butterfly).  Two dependent load rounds for rows of up to
+// 64 chunks: every chunk's (max, sum, first key), then the lists, up to
+// eight at once; longer rows add a round per further 32 chunks.
 __device__ __forceinline__ void topk_row_merge(const TopkPart* P, int S, int64_t row, float inv_t,
                                                float c2, int32_t* __restrict__ idx,
                                                float* __restrict__ prob, float* __restrict__ logp,
@@ -190,42 +203,48 @@ __device__ __forceinline__ void topk_row_merge(const TopkPart* P, int S, int64_t
                                                float* __restrict__ row_lse) {
     const int lane = threadIdx.x & 31;
     auto ldkey = [](const uint64_t* p) { return (uint64_t)__ldcg((const unsigned long long*)p); };
-    // first load pass: every chunk's (max, sum) and whether it carries a list
-    float M = -INFINITY;
-    for (int c = lane; c < S; c += 32) M = fmaxf(M, __ldcg(&P[c].m));
+    float m0 = -INFINITY, m1 = -INFINITY;  // chunks lane and lane + 32
+    double s0 = 0.0, s1 = 0.0;
+    uint64_t q0 = 0ull, q1 = 0ull;  // first key of the chunk's list (0: no list)
+    if (lane < S) {
+        m0 = __ldcg(&P[lane].m);
+        s0 = __ldcg(&P[lane].s);
+        q0 = ldkey(&P[lane].key[0]);
+    }
+    if (lane + 32 < S) {
+        m1 = __ldcg(&P[lane + 32].m);
+        s1 = __ldcg(&P[lane + 32].s);
+        q1 = ldkey(&P[lane + 32].key[0]);
+    }
+    float M = fmaxf(m0, m1);
+    for (int c = lane + 64; c < S; c += 32) M = fmaxf(M, __ldcg(&P[c].m));
     M = warp_max(M);
-    double ssum = 0.0;
+    // a chunk's sum is against fl(mc c2); M c2 is exact in fp64
+    const double Mc = (double)M * (double)c2;
+    auto rescaled = [&](float mc, double sc) {
+        return mc != -INFINITY ? sc * exp2((double)(mc * c2) - Mc) : 0.0;
+    };
+    double ssum = rescaled(m0, s0);
+    ssum += rescaled(m1, s1);
     uint64_t acc = 0ull;
     bool first = true;
-    for (int c0 = 0; c0 < S; c0 += 32) {
-        const int c = c0 + lane;
-        float mc = -INFINITY;
-        double sc = 0.0;
-        uint64_t k0 = 0ull;
-        if (c < S) {
-            mc = __ldcg(&P[c].m);
-            sc = __ldcg(&P[c].s);
-            k0 = ldkey(&P[c].key[0]);
-        }
-        if (mc != -INFINITY) ssum += sc * exp2(((double)mc - (double)M) * (double)c2);
-        // second load pass: the lists of this group of chunks, loaded together, merged in chunk order
-        unsigned has = __ballot_sync(FULL, k0 != 0ull);
-        while (has) {
-            constexpr int PF = 8;
+    // the lists of the chunks cbase + (set bits of hm), loaded up to eight at
+    // once, merged in chunk order
+    auto merge_lists = [&](uint64_t hm, int cbase) {
+        constexpr int PF = 8;
+        while (hm) {
             uint64_t kv[PF];
             int nl = 0;
-            unsigned hh = has;
 #pragma unroll
             for (int j = 0; j < PF; ++j) {
                 kv[j] = 0ull;
-                if (hh) {
-                    const int cc = c0 + __ffs(hh) - 1;
-                    hh &= hh - 1u;
+                if (hm) {
+                    const int cc = cbase + __ffsll((long long)hm) - 1;
+                    hm &= hm - 1ull;
                     kv[j] = ldkey(&P[cc].key[lane < K ? lane : 31 - lane]);
                     ++nl;
                 }
             }
-            has = hh;
 #pragma unroll
             for (int j = 0; j < PF; ++j)
                 if (j < nl) {
@@ -237,6 +256,21 @@ __device__ __forceinline__ void topk_row_merge(const TopkPart* P, int S, int64_t
                     }
                 }
         }
+    };
+    merge_lists(((uint64_t)__ballot_sync(FULL, q1 != 0ull) << 32) | __ballot_sync(FULL, q0 != 0ull),
+                0);
+    for (int c0 = 64; c0 < S; c0 += 32) {
+        const int c = c0 + lane;
+        float mc = -INFINITY;
+        double sc = 0.0;
+        uint64_t k0 = 0ull;
+        if (c < S) {
+            mc = __ldcg(&P[c].m);
+            sc = __ldcg(&P[c].s);
+            k0 = ldkey(&P[c].key[0]);
+        }
+        ssum += rescaled(mc, sc);
+        merge_lists(__ballot_sync(FULL, k0 != 0ull), c0);
     }
     ssum = warp_sum(ssum);
     const double lns = log(ssum);
@@ -275,7 +309,6 @@ __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
     __shared__ CandBuf cbuf[NCW];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     CandBuf& cb = cbuf[warp];
-    if (lane == 0) cb.n = 0;
     int64_t lo, hi;
     warp_range(units, lo, hi);
     const int n = (int)(hi - lo);
@@ -293,8 +326,14 @@ __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
     uint64_t run = 0ull;  // the segment's running top-16
     unsigned seg = 0;     // chunks in the segment so far
     uint32_t pub = 0u;    // the row bound this segment last raised thr to
+    // the row's shared bound, read one unit ahead: it only ever rises while
+    // the row is open (and its last unit is still to come), so an older value
+    // is a valid, slightly looser bound
+    uint32_t thr_now = n > 0 ? *(volatile unsigned*)&thr[uc.g] : 0u;
     for (int k = 0; k < n; ++k, uc.next()) {
         const int64_t row = uc.g, v0 = (int64_t)uc.c * LEN;
+        const uint32_t thr_ahead =
+            k + 1 < n ? *(volatile unsigned*)&thr[uc.last_of_row() ? row + 1 : row] : 0u;
         const int len = (int)min((int64_t)LEN, V - v0);
         float M;
         double Ssum;
@@ -304,12 +343,12 @@ __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
                 return;
             }
             topk_chunk<BF16>(SmemView<BF16>{r.slot(k), v0, len}, c2, cb, M, Ssum, run, &thr[row],
-                             pub);
+                             pub, thr_now);
             warp_ring_next(r, k, n, ic, ChunkT<BF16>::NEG_INF_WORD, src);
         } else {
             topk_chunk<BF16>(
                 GlobalView<BF16>{(const uint8_t*)logits + row * row_stride * ES, v0, len}, c2, cb,
-                M, Ssum, run, &thr[row], pub);
+                M, Ssum, run, &thr[row], pub, thr_now);
         }
         ++seg;
         const bool seg_end = (k + 1 == n) || uc.last_of_row();
@@ -340,6 +379,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) topk_softmax_kernel(
             seg = 0;
             pub = 0u;
         }
+        thr_now = thr_ahead;
     }
 }
 

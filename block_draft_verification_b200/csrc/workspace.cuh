@@ -19,7 +19,8 @@
 namespace dfl {
 
 // Partial result of one (row, chunk) unit of dflash2_topk_softmax: the
-// chunk maximum, the chunk's sum of exp2((x - m) c) and its top-16 keys.
+// chunk maximum m, the chunk's sum of exp2(x c - fl(m c)) and its top-16
+// keys.
 struct TopkPart {
     float m;
     float pad;
