@@ -142,9 +142,14 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
 __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-// Wait until *p is non-zero (acquire) and return it; 0 after WAIT_NS.  The
-// poll backs off from 64 ns to 1 us, so many waiting warps stay a light load
-// on the line.
+__device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// Wait until *p is non-zero and return it (read once more with acquire
+// semantics); 0 after WAIT_NS.  The poll is a relaxed load (cheap for the
+// SM's caches) that backs off from 64 to 256 ns.
 __device__ __forceinline__ unsigned wait_nonzero(const unsigned* p) {
     unsigned v = ld_acquire(p);
     if (v) return v;
@@ -152,9 +157,8 @@ __device__ __forceinline__ unsigned wait_nonzero(const unsigned* p) {
     unsigned ns = 64;
     while (true) {
         __nanosleep(ns);
-        if (ns < 1024) ns <<= 1;
-        v = ld_acquire(p);
-        if (v) return v;
+        if (ns < 256) ns <<= 1;
+        if (ld_relaxed(p)) return ld_acquire(p);
         if (global_ns() - t0 > WAIT_NS) return 0u;
     }
 }

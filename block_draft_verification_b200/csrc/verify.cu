@@ -94,7 +94,8 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_greedy_kernel(
 
 // ------------------------------------------------------------------ sampling, the scan
 // (maximum, fp64 sum of exp2((x - maximum) c)) of rows r0 .. r0+7 (the first
-// nrows of them) from their S chunk partials, lane-parallel: lanes 4j .. 4j+3
+// nrows of them) from their S chunk partials (chunk maximum m, sum of
+// exp2(x c - fl(m c))), lane-parallel: lanes 4j .. 4j+3
 // take row r0 + j, lane 4j + s its chunks s, s + 4, ... (the first 4 RC of
 // them held in registers, so a row of up to 4 RC chunks is read once); the
 // maximum, then the fp64 sum against it in chunk order; two butterfly steps
@@ -126,13 +127,15 @@ __device__ __forceinline__ void rows_lse8(const LseD* P, int S, int r0, int nrow
     M = fmaxf(M, __shfl_xor_sync(FULL, M, 2));
     double t = 0.0;
     if (M != -INFINITY) {
+        // a chunk's sum is against fl(m c2); M c2 is exact in fp64
+        const double Mc = (double)M * (double)c2;
 #pragma unroll
         for (int i = 0; i < RC; ++i)
-            if (pm[i] != -INFINITY) t += ps[i] * exp2(((double)pm[i] - (double)M) * (double)c2);
+            if (pm[i] != -INFINITY) t += ps[i] * exp2((double)(pm[i] * c2) - Mc);
         if (on)
             for (int c = sub + 4 * RC; c < S; c += 4) {
                 const float m = __ldcg(&p[c].m);
-                if (m != -INFINITY) t += __ldcg(&p[c].s) * exp2(((double)m - (double)M) * (double)c2);
+                if (m != -INFINITY) t += __ldcg(&p[c].s) * exp2((double)(m * c2) - Mc);
             }
     }
     t += __shfl_xor_sync(FULL, t, 1);
@@ -632,6 +635,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
     extern __shared__ __align__(128) uint8_t ring[];
     __shared__ __align__(8) uint64_t bars[2 * NCW];
     __shared__ unsigned s_next;  // this CTA's next draw unit (k: unit blockIdx.x + k grid)
+    __shared__ unsigned s_warm;  // warps of this CTA done with their scan
     const int lane = threadIdx.x & 31;
     unsigned* const fin_count = ctl;
     unsigned* const retire = ctl + CTL_LINE;
@@ -642,7 +646,10 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
         return (rr <= G) ? (const char*)target + (b * (G + 1) + rr) * V * ES
                          : (const char*)draft + (b * G + (rr - G - 1)) * V * ES;
     };
-    if (threadIdx.x == 0) s_next = 0u;
+    if (threadIdx.x == 0) {
+        s_next = 0u;
+        s_warm = 0u;
+    }
     {  // the accept tests' scattered reads (drafted tokens, their logits) into L2 now
         const int64_t t = (int64_t)blockIdx.x * RING_THREADS + threadIdx.x;
         if (t < (int64_t)B * G) {
@@ -683,13 +690,13 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
             const SmemView<BF16> view{r.slot(k), v0, len};
             uint32_t vm[NVL];
             M = warp_max(chunk_pass1<BF16>(view, vm));
-            Ssum = chunk_expsum<BF16>(view, M, c2);
+            Ssum = chunk_expsum_at_mc<BF16>(view, M, c2);
             warp_ring_next(r, k, n, ic, C::NEG_INF_WORD, src);
         } else {
             const GlobalView<BF16> view{(const uint8_t*)rowp(b, uc.r), v0, len};
             uint32_t vm[NVL];
             M = warp_max(chunk_pass1<BF16>(view, vm));
-            Ssum = chunk_expsum<BF16>(view, M, c2);
+            Ssum = chunk_expsum_at_mc<BF16>(view, M, c2);
         }
         ++seg;
         if (lane == 0) part[(b * rows_per_seq + uc.r) * S + uc.c] = LseD{M, 0.0f, Ssum};
@@ -715,66 +722,114 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_sample_kernel(
     constexpr int LEN_D = draw_len<BF16>();
     const unsigned total = (unsigned)B * (unsigned)ND;
     double* const dsum_scratch = dsum + (int64_t)B * ND * 32;  // 32 doubles
-    int kk = n;  // this warp's next ring unit
-    while (true) {
+    // The first warp of the CTA done with its scan runs the draw sum and the
+    // pick once on a scratch table (storing nothing else): their code is then
+    // in this SM's instruction cache before the real calls need it.
+    {
+        unsigned first = 0;
+        if (lane == 0) first = atomicAdd(&s_warm, 1u) == 0u;
+        if (__shfl_sync(FULL, first, 0))
+            warm_draw_code<BF16, TMA>(target, V, c2, inv_t, dsum_scratch, r);
+    }
+    // Units in queue order, per CTA: unit blockIdx.x + k grid, k from s_next
+    // (total: none left).
+    auto grab = [&]() -> unsigned {
         unsigned k = 0;
         if (lane == 0) k = atomicAdd(&s_next, 1u);
         k = __shfl_sync(FULL, k, 0);
         const uint64_t i64 = (uint64_t)blockIdx.x + (uint64_t)k * gridDim.x;
-        if (i64 >= total) {
-            // the first warp of CTA 0 with no unit left runs the pick (and,
-            // with rings, the draw sum) once on scratch, writing nothing, so
-            // their code is in L2 before the real picks need it
-            if (blockIdx.x == 0 && k == (total + gridDim.x - 1) / gridDim.x)
-                warm_draw_code<BF16, TMA>(target, V, c2, inv_t, dsum_scratch, r);
-            break;
-        }
-        const unsigned i = (unsigned)i64;
-        const unsigned pos = i / (unsigned)ND, c = i - pos * (unsigned)ND;
-        unsigned b1 = 0;
-        if (lane == 0) b1 = wait_nonzero(&fin[(size_t)pos * CTL_LINE]);
-        b1 = __shfl_sync(FULL, b1, 0);
-        if (b1 == 0u) {  // the bound ran out
-            if (lane == 0) atomicOr(&g_dev_err, ERR_STREAM);
-            return;
-        }
-        __syncwarp();  // lane 0's acquire covers the warp's reads of info[b]
-        const int b = (int)b1 - 1;
-        const SampleInfo I = load_info(&info[b]);
-        const int64_t v0 = (int64_t)c * LEN_D;
-        const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
-        const char* qrow =
-            (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
-        double my;
-        if (TMA) {
-            const int nu = (I.mode == 0) ? 2 : 1;
-            const uint32_t bytes = (uint32_t)(min((int64_t)LEN_D, V - v0) * ES);
-            warp_ring_load(r, kk, trow + v0 * ES, bytes, C::NEG_INF_WORD);
-            if (nu == 2) warp_ring_load(r, kk + 1, qrow + v0 * ES, bytes, C::NEG_INF_WORD);
-            __syncwarp();
-            bool ok = r.wait_fresh(kk);
-            if (nu == 2) ok = r.wait_fresh(kk + 1) && ok;
-            if (!ok) {
-                warp_ring_abort(r, kk, kk + nu);
-                return;
-            }
-            const SmemView<BF16> vt{r.slot(kk), v0, LEN_D}, vq{r.slot(kk + 1), v0, LEN_D};
-            my = draw_lane_sum<BF16>(vt, vq, I.mode, I, c2, inv_t);
-            r.done(kk);  // both slots read: they may be refilled
-            kk += nu;
-        } else {
-            const RowView<BF16, false> vt{trow, v0, V}, vq{qrow, v0, V};
-            my = draw_lane_sum<BF16>(vt, vq, I.mode, I, c2, inv_t);
-        }
+        return i64 < total ? (unsigned)i64 : total;
+    };
+    // A unit's lane prefixes out, and its sequence's pick by the warp whose
+    // unit completes the row.
+    auto publish_unit = [&](unsigned c, double my, int b, const SampleInfo& I) {
         dsum[((int64_t)b * ND + c) * 32 + lane] = warp_incl_scan(my);
         __syncwarp();  // every lane's prefix before lane 0's release
         bool lastu = false;
         if (lane == 0) lastu = publish(&dcount[b], 1u, (unsigned)ND);
         if (__shfl_sync(FULL, lastu, 0)) {
             __syncwarp();
+            const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
+            const char* qrow =
+                (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
             draw_pick<BF16, TMA>(trow, qrow, V, ND, I, c2, inv_t, dsum + (int64_t)b * ND * 32,
                                  &out_tok[(int64_t)b * (G + 1) + I.n]);
             if (lane == 0) dcount[b] = 0u;
+        }
+    };
+    if (TMA) {
+        // One unit per ring slot: its target run in the first half, its draft
+        // run (residual draws) in the second, both copies on the slot's barrier.
+        constexpr uint32_t HALF = (uint32_t)SLOT_BYTES / 2;
+        static_assert(LEN_D * ES == (int)HALF, "a draw unit fills half a ring slot");
+        int kk = n;  // this warp's next ring unit
+        while (true) {
+            const unsigned i = grab();
+            if (i >= total) break;
+            unsigned b1 = 0;
+            if (lane == 0) b1 = wait_nonzero(&fin[(size_t)(i / (unsigned)ND) * CTL_LINE]);
+            b1 = __shfl_sync(FULL, b1, 0);
+            if (b1 == 0u) {  // the bound ran out
+                if (lane == 0) atomicOr(&g_dev_err, ERR_STREAM);
+                return;
+            }
+            __syncwarp();  // lane 0's acquire covers the warp's reads of info[b]
+            const int b = (int)b1 - 1;
+            const SampleInfo I = load_info(&info[b]);
+            const unsigned c = i - (i / (unsigned)ND) * (unsigned)ND;
+            const int64_t v0 = (int64_t)c * LEN_D;
+            const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
+            const char* qrow = (const char*)draft + ((int64_t)b * G + I.n) * V * ES;
+            const bool two = I.mode == 0;
+            const uint32_t bytes = (uint32_t)(min((int64_t)LEN_D, V - v0) * ES);
+            uint8_t* sl = r.slot(kk);
+            if (bytes < HALF) {  // past the row: -inf, in both runs
+                const uint4 f = make_uint4(C::NEG_INF_WORD, C::NEG_INF_WORD, C::NEG_INF_WORD,
+                                           C::NEG_INF_WORD);
+                for (uint32_t q = bytes / 16 + lane; q < HALF / 16; q += 32) {
+                    ((uint4*)sl)[q] = f;
+                    if (two) ((uint4*)(sl + HALF))[q] = f;
+                }
+                __syncwarp();
+            }
+            if (lane == 0) {
+                const uint32_t bar = r.bar + 8 * (kk & 1);
+                mbar_expect_tx(bar, two ? 2 * bytes : bytes);
+                bulk_g2s_nx(smem_u32(sl), trow + v0 * ES, bytes, bar);
+                if (two) bulk_g2s_nx(smem_u32(sl + HALF), qrow + v0 * ES, bytes, bar);
+            }
+            __syncwarp();
+            if (!r.wait_fresh(kk)) {
+                warp_ring_abort(r, kk, kk + 1);
+                return;
+            }
+            const SmemView<BF16> vt{sl, v0, LEN_D}, vq{sl + HALF, v0, LEN_D};
+            const double my = draw_lane_sum<BF16>(vt, vq, I.mode, I, c2, inv_t);
+            r.done(kk);  // the slot is read: it may be refilled
+            ++kk;
+            publish_unit(c, my, b, I);
+        }
+    } else {
+        while (true) {
+            const unsigned i = grab();
+            if (i >= total) break;
+            unsigned b1 = 0;
+            if (lane == 0) b1 = wait_nonzero(&fin[(size_t)(i / (unsigned)ND) * CTL_LINE]);
+            b1 = __shfl_sync(FULL, b1, 0);
+            if (b1 == 0u) {  // the bound ran out
+                if (lane == 0) atomicOr(&g_dev_err, ERR_STREAM);
+                return;
+            }
+            __syncwarp();  // lane 0's acquire covers the warp's reads of info[b]
+            const int b = (int)b1 - 1;
+            const SampleInfo I = load_info(&info[b]);
+            const unsigned c = i - (i / (unsigned)ND) * (unsigned)ND;
+            const int64_t v0 = (int64_t)c * LEN_D;
+            const char* trow = (const char*)target + ((int64_t)b * (G + 1) + I.n) * V * ES;
+            const char* qrow =
+                (I.mode == 0) ? (const char*)draft + ((int64_t)b * G + I.n) * V * ES : nullptr;
+            const RowView<BF16, false> vt{trow, v0, V}, vq{qrow, v0, V};
+            publish_unit(c, draw_lane_sum<BF16>(vt, vq, I.mode, I, c2, inv_t), b, I);
         }
     }
     // the last warp out leaves the queue words zero (every other warp is past
