@@ -76,6 +76,14 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
 }
 constexpr int TC_MAXCTA = 256;  // stream-K CTAs at most (one per SM)
 
+// What the epilogue of an owned tile needs: its accumulator (TMEM column
+// base), channels, tokens, and which partials it adds.
+struct OwnTile {
+    uint32_t tacc;
+    int h0, tok0, bi0, q_reg, q_end;
+    bool staged, reg_part, first_part;
+};
+
 struct TcShape {
     int H, T, ntok, BN, sw, sx, nkb, nh;  // W / X ring stages; nh: channel tiles per token chunk
     int bufcols;                           // TMEM columns per accumulator (power of 2, >= BN)
@@ -128,10 +136,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     uint8_t* s_x0 = s_xp + sh.R * 128;
     uint8_t* s_out = s_x0 + 128;  // [2][32 tokens][64 channels] bf16 outputs
     // wfull[SW], wempty[SW], xfull[SX], xempty[SX], tmem_full[2], tmem_empty[2], mma_done,
-    // x tile, staged partial
+    // x tile, staged partial, helpers' go
     uint64_t* bars = (uint64_t*)(s_out + 8192);
-    uint32_t* s_tmem = (uint32_t*)(bars + 2 * sh.sw + 2 * sh.sx + 7);
+    uint32_t* s_tmem = (uint32_t*)(bars + 2 * sh.sw + 2 * sh.sx + 8);
     int* s_fail = (int*)(s_tmem + 1);
+    OwnTile& s_own = *(OwnTile*)(s_fail + 1);  // the last owned tile, for the helper warps
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int p = blockIdx.x;
@@ -143,6 +152,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     const uint32_t mdone = tfull0 + 32;
     const uint32_t xbar = tfull0 + 40;
     const uint32_t pbar = tfull0 + 48;  // a partial staged in the idle rings
+    const uint32_t hbar = tfull0 + 56;  // the last owned tile is ready for the helper warps
     const uint32_t ncols = 2 * (uint32_t)sh.bufcols;
 
     if (threadIdx.x == 0) {
@@ -161,6 +171,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
         mbar_init(mdone, 1);
         mbar_init(xbar, 1);
         mbar_init(pbar, 1);
+        mbar_init(hbar, 1);
         mbar_fence_init();
         *s_fail = 0;
     }
@@ -174,6 +185,123 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+
+    // An owned tile's 32-token groups g0 .. g1-1, by a set of four warps
+    // (warp w takes TMEM lanes 32 (w mod 4) ..; e: the thread's index in the
+    // set): accumulator + partials in K order, the conv and the residual, bf16
+    // rounding, 16-byte stores through the set's double-buffered output tile
+    // `so` (synchronised by named barrier `bid`).  pp0 / pp1 hold groups g0 and
+    // g0 + 1 of the register-prefetched partial, refilled two groups ahead.
+    const uint32_t part_bytes = (uint32_t)sh.ngroups * 8 * TC_BM * 16;
+    const uint32_t ring_bytes = (uint32_t)sh.sw * TC_A_BYTES + (uint32_t)sh.sx * xstage;
+    auto own_groups = [&](const OwnTile& o, int g0, int g1, uint32_t so, int bid,
+                          float4 (&pp0)[8], float4 (&pp1)[8]) {
+        const int q = warp & 3, e = threadIdx.x & 127, row = 32 * q + lane;
+        const uint32_t tacc = o.tacc + ((uint32_t)(32 * q) << 16);
+        const float4* sp = (const float4*)wring;
+        const float4* partr = partial + (int64_t)o.q_reg * sh.ngroups * 8 * TC_BM;
+        auto set_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(bid) : "memory"); };
+        // lane l of warp q: channel cl = 16q + (l & 15) of the tile, tokens
+        // 16 (l >> 4) .. +15 of each 32-token group; a and b of the channel
+        // meet by one exchange between lanes l and l ^ 16
+        const int cl = 16 * q + (lane & 15), half = lane >> 4;
+        for (int g = g0; g < g1; ++g) {
+            float v[32];
+            tmem_ld32(tacc + 32 * g, v);
+            if (o.staged) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float4 w = sp[(g * 8 + c) * TC_BM + row];
+                    v[4 * c] += w.x;
+                    v[4 * c + 1] += w.y;
+                    v[4 * c + 2] += w.z;
+                    v[4 * c + 3] += w.w;
+                }
+            }
+            if (o.reg_part) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    v[4 * c] += pp0[c].x;
+                    v[4 * c + 1] += pp0[c].y;
+                    v[4 * c + 2] += pp0[c].z;
+                    v[4 * c + 3] += pp0[c].w;
+                    pp0[c] = pp1[c];
+                }
+                if (g + 2 < g1)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        pp1[c] = __ldcg(&partr[((int64_t)(g + 2) * 8 + c) * TC_BM + row]);
+            }
+            if (o.first_part) {
+                for (int q2 = o.q_reg + 1; q2 < o.q_end; ++q2) {  // further partials, in K order
+                    const float4* src = partial + (int64_t)q2 * sh.ngroups * 8 * TC_BM;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 w = __ldcg(&src[((int64_t)g * 8 + c) * TC_BM + row]);
+                        v[4 * c] += w.x;
+                        v[4 * c + 1] += w.y;
+                        v[4 * c + 2] += w.z;
+                        v[4 * c + 3] += w.w;
+                    }
+                }
+            }
+            float av[16], bv[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                const float recv = __shfl_xor_sync(FULL, half ? v[t] : v[16 + t], 16);
+                av[t] = half ? recv : v[t];
+                bv[t] = half ? v[16 + t] : recv;
+            }
+            const int jt0 = 32 * g + 16 * half;
+            const int tokf = o.tok0 + jt0, bif = tokf / sh.T;
+            // every shared-memory read first (branch-free, so they overlap):
+            // x of tokens jt0-1 .. jt0+15, and x_prev of each token's batch
+            float xv[17], pv[16];
+            xv[0] = jt0 == 0 ? lds_bf16(smem_u32(s_x0) + 2 * cl)
+                             : lds_bf16(smem_u32(s_x) + (min(jt0, sh.BN) - 1) * 128 + 2 * cl);
+            bool bstart[16];
+            {
+                int ti = tokf - bif * sh.T, bl = bif - o.bi0;
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const int jt = min(jt0 + t, sh.BN - 1);
+                    xv[t + 1] = lds_bf16(smem_u32(s_x) + jt * 128 + 2 * cl);
+                    bstart[t] = ti == 0;
+                    pv[t] = lds_bf16(smem_u32(s_xp) + min(bl, sh.R - 1) * 128 + 2 * cl);
+                    if (++ti == sh.T) {
+                        ti = 0;
+                        ++bl;
+                    }
+                }
+            }
+            // the 16 outputs of this lane into the group's output tile
+            // [32 tokens][64 channels] bf16 (double-buffered by group)
+            const uint32_t ob = so + (g & 1) * 4096 + (16 * half) * 128 + 2 * cl;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                const float xc = xv[t + 1], xm = bstart[t] ? pv[t] : xv[t];
+                sts_bf16(ob + t * 128, fmaf(bv[t], xm, fmaf(av[t], xc, xc)));
+            }
+            set_sync();
+            // 16-byte rows out: item = (token, 8-channel group)
+#pragma unroll
+            for (int rep = 0; rep < 2; ++rep) {
+                const int it = e + 128 * rep, tl = it >> 3, gg = it & 7;
+                const int jt = 32 * g + tl, tok = o.tok0 + jt;
+                if (jt < sh.BN && tok < sh.ntok)
+                    *(uint4*)(out + (int64_t)tok * sh.H + o.h0 + 8 * gg) =
+                        lds_v4(so + (g & 1) * 4096 + tl * 128 + 16 * gg);
+            }
+        }
+    };
+    // The run's last segment, if it owns its tile, has nothing after it: the
+    // producer, MMA and allocation warps (0-3) then take the second half of
+    // its groups, their output tile in the rings behind the staged partial.
+    const int64_t last_tile = (s1 - 1) / sh.nkb;
+    const uint32_t hso = part_bytes <= ring_bytes ? part_bytes : 0u;
+    const bool helpers = s1 > s0 && s0 <= last_tile * sh.nkb && sh.ngroups >= 2 &&
+                         hso + 8192u <= ring_bytes;
+    const int gh = helpers ? (sh.ngroups + 1) / 2 : sh.ngroups;
 
     if ((warp == 0 || warp == 3) && lane == 0) {
         // ---------------- TMA producers, the run's steps in order: warp 0
@@ -263,8 +391,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
         const int e = threadIdx.x - 128;
         const int row = 32 * q + lane;
         int j = 0, nown = 0, nstaged = 0;  // segments, owned segments, staged partials
-        const uint32_t part_bytes = (uint32_t)sh.ngroups * 8 * TC_BM * 16;
-        const uint32_t ring_bytes = (uint32_t)sh.sw * TC_A_BYTES + (uint32_t)sh.sx * xstage;
         float4 pp0[8], pp1[8];  // the first partial, two groups ahead of its use
         for (int64_t sg = s0; sg < s1; ++j) {
             const int tile = (int)(sg / sh.nkb);
@@ -373,99 +499,47 @@ __global__ void __launch_bounds__(TC_THREADS, 1) dynconv2_tc_kernel(
             }
             epi_sync();
             if (*s_fail) break;  // uniform over the four warps
-            const float4* sp = (const float4*)wring;
-            // lane l of epilogue warp q: channel cl = 16q + (l & 15) of the tile,
-            // tokens 16 (l >> 4) .. +15 of each 32-token group; a and b of the
-            // channel meet by one exchange between lanes l and l ^ 16
-            const int cl = 16 * q + (lane & 15), half = lane >> 4;
-            for (int g = 0; g < sh.ngroups; ++g) {
-                float v[32];
-                tmem_ld32(tacc + 32 * g, v);
-                if (staged) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const float4 w = sp[(g * 8 + c) * TC_BM + row];
-                        v[4 * c] += w.x;
-                        v[4 * c + 1] += w.y;
-                        v[4 * c + 2] += w.z;
-                        v[4 * c + 3] += w.w;
-                    }
-                }
-                if (reg_part) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        v[4 * c] += pp0[c].x;
-                        v[4 * c + 1] += pp0[c].y;
-                        v[4 * c + 2] += pp0[c].z;
-                        v[4 * c + 3] += pp0[c].w;
-                        pp0[c] = pp1[c];
-                    }
-                    if (g + 2 < sh.ngroups) load_part(g + 2, pp1);
-                }
-                if (first_part) {
-                    for (int q2 = q_reg + 1; q2 < q_end; ++q2) {  // further partials, in K order
-                        const float4* src = partial + (int64_t)q2 * sh.ngroups * 8 * TC_BM;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const float4 w = __ldcg(&src[((int64_t)g * 8 + c) * TC_BM + row]);
-                            v[4 * c] += w.x;
-                            v[4 * c + 1] += w.y;
-                            v[4 * c + 2] += w.z;
-                            v[4 * c + 3] += w.w;
-                        }
-                    }
-                }
-                float av[16], bv[16];
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const float recv = __shfl_xor_sync(FULL, half ? v[t] : v[16 + t], 16);
-                    av[t] = half ? recv : v[t];
-                    bv[t] = half ? v[16 + t] : recv;
-                }
-                const int jt0 = 32 * g + 16 * half;
-                const int tokf = tok0 + jt0, bif = tokf / sh.T;
-                // every shared-memory read first (branch-free, so they overlap):
-                // x of tokens jt0-1 .. jt0+15, and x_prev of each token's batch
-                float xv[17], pv[16];
-                xv[0] = jt0 == 0 ? lds_bf16(smem_u32(s_x0) + 2 * cl)
-                                 : lds_bf16(smem_u32(s_x) + (min(jt0, sh.BN) - 1) * 128 + 2 * cl);
-                bool bstart[16];
-                {
-                    int ti = tokf - bif * sh.T, bl = bif - bi0;
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) {
-                        const int jt = min(jt0 + t, sh.BN - 1);
-                        xv[t + 1] = lds_bf16(smem_u32(s_x) + jt * 128 + 2 * cl);
-                        bstart[t] = ti == 0;
-                        pv[t] = lds_bf16(smem_u32(s_xp) + min(bl, sh.R - 1) * 128 + 2 * cl);
-                        if (++ti == sh.T) {
-                            ti = 0;
-                            ++bl;
-                        }
-                    }
-                }
-                // the 16 outputs of this lane into the group's output tile
-                // [32 tokens][64 channels] bf16 (double-buffered by group)
-                const uint32_t ob = smem_u32(s_out) + (g & 1) * 4096 + (16 * half) * 128 + 2 * cl;
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const float xc = xv[t + 1], xm = bstart[t] ? pv[t] : xv[t];
-                    sts_bf16(ob + t * 128, fmaf(bv[t], xm, fmaf(av[t], xc, xc)));
-                }
-                epi_sync();
-                // 16-byte rows out: item = (token, 8-channel group)
-#pragma unroll
-                for (int rep = 0; rep < 2; ++rep) {
-                    const int it = e + 128 * rep, tl = it >> 3, gg = it & 7;
-                    const int jt = 32 * g + tl, tok = tok0 + jt;
-                    if (jt < sh.BN && tok < sh.ntok)
-                        *(uint4*)(out + (int64_t)tok * sh.H + h0 + 8 * gg) =
-                            lds_v4(smem_u32(s_out) + (g & 1) * 4096 + tl * 128 + 16 * gg);
-                }
+            OwnTile o;
+            o.tacc = tmem + (uint32_t)(buf * sh.bufcols);
+            o.h0 = h0;
+            o.tok0 = tok0;
+            o.bi0 = bi0;
+            o.q_reg = q_reg;
+            o.q_end = q_end;
+            o.staged = staged;
+            o.reg_part = reg_part;
+            o.first_part = first_part;
+            const bool helped = helpers && sg == s1;
+            if (helped && e == 0) {  // hand the second half of the groups to warps 0-3
+                s_own = o;
+                mbar_arrive(hbar);
             }
+            own_groups(o, 0, helped ? gh : sh.ngroups, smem_u32(s_out), 1, pp0, pp1);
             tc_fence_before();
             epi_sync();
             if (e == 0) mbar_arrive(tempty0 + 8 * buf);
+        }
+    }
+    if (warp < 4 && helpers) {
+        __syncwarp();  // lane 0 of warps 0, 1 and 3 is back from its role
+        if (!mbar_wait(hbar, 0)) {
+            if (lane == 0) atomicOr(&g_dev_err, ERR_EPILOGUE);
+        } else {
+            tc_fence_after();
+            const OwnTile o = s_own;
+            float4 pp0[8], pp1[8];
+            if (o.reg_part) {
+                const float4* partr = partial + (int64_t)o.q_reg * sh.ngroups * 8 * TC_BM;
+                const int row = 32 * warp + lane;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    pp0[c] = __ldcg(&partr[((int64_t)gh * 8 + c) * TC_BM + row]);
+                    if (gh + 1 < sh.ngroups)
+                        pp1[c] = __ldcg(&partr[((int64_t)(gh + 1) * 8 + c) * TC_BM + row]);
+                }
+            }
+            own_groups(o, gh, sh.ngroups, smem_u32(wring) + hso, 2, pp0, pp1);
+            tc_fence_before();
         }
     }
     __syncthreads();
