@@ -48,16 +48,16 @@ __device__ __forceinline__ uint32_t swz_off(int r, int k, int rows) {
 }
 
 // Shared memory of one CTA (dynamic, 1024-byte aligned): the three W planes
-// (B operand, d x d each), the left rows (A operand, 128 x d), the right rows
-// (row-major, padded rows), the pair scores of the sequence.
+// (B operand of F, d x d each), the left rows (A operand of F, 128 x d; then,
+// one plane at a time, the bf16 planes of F as the A operand of S), the right
+// rows (B operand of S, 128 x d), the pair scores of the sequence.
 template <int D>
 struct PtLayout {
-    static constexpr int ROWB = D * 2 + 16;  // padded right row: 16-byte loads spread over banks
     static constexpr uint32_t W_OFF = 0;
     static constexpr uint32_t W_PLANE = D * D * 2;
     static constexpr uint32_t A_OFF = 3 * W_PLANE;
     static constexpr uint32_t R_OFF = A_OFF + PT_ROWS * D * 2;
-    static constexpr uint32_t S_OFF = R_OFF + PT_ROWS * ROWB;
+    static constexpr uint32_t S_OFF = R_OFF + PT_ROWS * D * 2;
     static size_t bytes(int G) {
         return 1024 + S_OFF + 4 * (size_t)(K + (size_t)K * K * (G > 1 ? G - 1 : 0));
     }
@@ -94,14 +94,17 @@ __global__ void __launch_bounds__(PT_THREADS, 1) pair_select_tc_kernel(
         mbar_init(wbar, 1);
         mbar_fence_init();
         s_fail = 0;
-        // W (fp32, d x d) in one bulk copy into the operand tiles' space,
-        // which the gathered rows overwrite only after the split
-        bulk_g2s(smem_u32(sm + L::A_OFF), W, (uint32_t)(D * D * 4), wbar);
+        // W (fp32, d x d) into the operand tiles' space (which the gathered
+        // rows overwrite only after the split), in 8 KB bulk copies that
+        // proceed side by side
+        mbar_expect_tx(wbar, (uint32_t)(D * D * 4));
+        for (uint32_t off = 0; off < (uint32_t)(D * D * 4); off += 8192u)
+            bulk_g2s_nx(smem_u32(sm + L::A_OFF) + off, (const char*)W + off, 8192u, wbar);
     }
-    if (warp == 2) {  // 128 TMEM columns: the F accumulator (d columns)
+    if (warp == 2) {  // 256 TMEM columns: F (d columns at 0), S (128 columns at 128)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&s_tmem)),
-                     "r"(128));
+                     "r"(256));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
         tc_fence_before();
     }
@@ -117,6 +120,7 @@ __global__ void __launch_bounds__(PT_THREADS, 1) pair_select_tc_kernel(
     constexpr int VPR = D / 8;                        // 16-byte vectors per embedding row
     constexpr int NV = 2 * PT_ROWS * VPR / PT_THREADS;  // vectors per thread (both tiles)
     const int nwin = (G + PT_SLOTS - 1) / PT_SLOTS;
+    int ncommit = 0;  // commits waited on so far (the barrier's phase)
     for (int wdw = 0; wdw < nwin; ++wdw) {
         // ---- gather: left rows (slot s: the anchor for s = 0, else the
         // candidates of position s - 1) and right rows (the candidates of
@@ -198,8 +202,7 @@ __global__ void __launch_bounds__(PT_THREADS, 1) pair_select_tc_kernel(
             const int tile = e / (PT_ROWS * VPR);
             const int rem = e - tile * PT_ROWS * VPR;
             const int r = rem / VPR, c = rem - r * VPR;
-            if (tile == 0) *(uint4*)(sm + L::A_OFF + swz_off(r, 8 * c, PT_ROWS)) = v[j];
-            else *(uint4*)(sm + L::R_OFF + r * L::ROWB + 16 * c) = v[j];
+            *(uint4*)(sm + (tile == 0 ? L::A_OFF : L::R_OFF) + swz_off(r, 8 * c, PT_ROWS)) = v[j];
         }
         // generic-proxy writes of the operands before the tensor core reads them
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -220,48 +223,93 @@ __global__ void __launch_bounds__(PT_THREADS, 1) pair_select_tc_kernel(
                 }
             mma_commit(bar);
         }
-        const bool ok = mbar_wait(bar, (uint32_t)(wdw & 1));
+        bool ok = mbar_wait(bar, (uint32_t)(ncommit++ & 1));
+        ok = __syncthreads_and(ok) != 0;  // one verdict for the CTA
+        tc_fence_after();
+        // ---- S blocks on the tensor cores: F (fp32, TMEM) is split into
+        // three bf16 planes F1 + F2 + F3 (24 bits in all: exact), each
+        // written over the left-row tile in turn and multiplied by the right
+        // rows into one fp32 accumulator, S_all = F E_right^T (128 x 128);
+        // its diagonal 16 x 16 blocks are the S_pos.  Thread (quadrant q,
+        // half h) splits columns [h d/2, h d/2 + d/2) of F row 32 q + lane.
+        const int q = warp & 3, h = warp >> 2;
+        const int r = 32 * q + lane;
+        constexpr int HC = D / 2;
+        float res[HC];
+#pragma unroll
+        for (int cc = 0; cc < HC / 32; ++cc) {
+            float f[32];
+            tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(h * HC + 32 * cc), f);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) res[32 * cc + j] = f[j];
+        }
+        const uint32_t idesc_s = instr_desc(PT_ROWS, PT_ROWS);
+        // With one window W is no longer needed: the three planes go into its
+        // space (and the left tile's, when d is small) and meet the right rows
+        // in one round; with more, each plane in turn over the left-row tile
+        // (W stays for the next window).
+        constexpr bool FIT3 = 3 * PT_ROWS * D * 2 <= (int)L::R_OFF;  // W's space and the left tile
+        const bool one_round = FIT3 && nwin == 1;
+        const int nround = one_round ? 1 : 3;
+#pragma unroll 1
+        for (int rd = 0; rd < nround && ok; ++rd) {
+#pragma unroll
+            for (int vv = 0; vv < HC / 8; ++vv) {
+#pragma unroll 1
+                for (int p = one_round ? 0 : rd; p < (one_round ? 3 : rd + 1); ++p) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const __nv_bfloat16 b0 = __float2bfloat16_rn(res[8 * vv + 2 * i]);
+                        const __nv_bfloat16 b1 = __float2bfloat16_rn(res[8 * vv + 2 * i + 1]);
+                        res[8 * vv + 2 * i] -= __bfloat162float(b0);
+                        res[8 * vv + 2 * i + 1] -= __bfloat162float(b1);
+                        w4[i] = (uint32_t)__bfloat16_as_ushort(b0) |
+                                ((uint32_t)__bfloat16_as_ushort(b1) << 16);
+                    }
+                    const uint32_t base = one_round ? L::W_OFF + p * (uint32_t)(PT_ROWS * D * 2) : L::A_OFF;
+                    *(uint4*)(sm + base + swz_off(r, h * HC + 8 * vv, PT_ROWS)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc_fence_before();
+            __syncthreads();
+            if (t == 0) {
+                tc_fence_after();
+                const uint32_t b0 = smem_u32(sm + L::R_OFF);
+                for (int p = 0; p < (one_round ? 3 : 1); ++p) {
+                    const uint32_t a0 = smem_u32(sm + (one_round ? L::W_OFF + p * (uint32_t)(PT_ROWS * D * 2) : L::A_OFF));
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t a = a0 + (ks >> 2) * (PT_ROWS * 128) + (ks & 3) * 32;
+                        const uint32_t bb = b0 + (ks >> 2) * (PT_ROWS * 128) + (ks & 3) * 32;
+                        mma_bf16(tmem + 128u, smem_desc(a), smem_desc(bb), idesc_s,
+                                 (rd | p | ks) ? 1u : 0u);
+                    }
+                }
+                mma_commit(bar);
+            }
+            ok = __syncthreads_and(mbar_wait(bar, (uint32_t)(ncommit++ & 1))) != 0;
+            tc_fence_after();
+        }
         if (!ok && lane == 0) {
             atomicOr(&g_dev_err, ERR_MMA);
             s_fail = 1;
         }
-        tc_fence_after();
-        // ---- S blocks: thread (quadrant q, half h) holds left row r = 32 q +
-        // lane (slot r / 16, rank r % 16) and the right ranks 8 h .. 8 h + 7
-        // of the same slot; F comes in 32 columns at a time
-        const int q = warp & 3, h = warp >> 2;
-        const int r = 32 * q + lane, slot = r >> 4, kr = r & 15;
-        const int pos = PT_SLOTS * wdw + slot;  // S_pos: left slot pos, right position pos
-        const bool valid = ok && pos < G && (pos > 0 || (anchor && kr == 0));
-        float acc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-            float f[32];
-            tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * cc), f);
+        // the diagonal blocks: warp q (h = 0) reads S columns 32 q .. 32 q + 31
+        // (rows 32 q .. 32 q + 15 need the first 16, the next 16 rows the rest)
+        if (h == 0) {
+            const int slot = r >> 4, kr = r & 15;
+            const int pos = PT_SLOTS * wdw + slot;  // S_pos: left slot pos, right position pos
+            const bool valid = ok && pos < G && (pos > 0 || (anchor && kr == 0));
+            float sv[32];
+            tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + 128u + (uint32_t)(32 * q), sv);
             if (valid) {
+                float* dst = (pos == 0) ? s_sc : s_sc + K + (size_t)K * K * (pos - 1) + kr * K;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint8_t* row = sm + L::R_OFF + (16 * slot + 8 * h + j) * L::ROWB + 64 * cc;
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const uint4 e8 = *(const uint4*)(row + 16 * g);
-                        const uint32_t ww[4] = {e8.x, e8.y, e8.z, e8.w};
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            acc[j] = fmaf(f[8 * g + 2 * u], __uint_as_float(ww[u] << 16), acc[j]);
-                            acc[j] = fmaf(f[8 * g + 2 * u + 1], __uint_as_float(ww[u] & 0xFFFF0000u),
-                                          acc[j]);
-                        }
-                    }
-                }
+                for (int j = 0; j < K; ++j) dst[j] = (lane < 16) ? sv[j] : sv[16 + j];
             }
-        }
-        if (valid) {
-            float* dst = (pos == 0) ? s_sc : s_sc + K + (size_t)K * K * (pos - 1) + kr * K;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) dst[8 * h + j] = acc[j];
         }
         tc_fence_before();
         __syncthreads();  // TMEM and both tiles free for the next window
@@ -277,14 +325,26 @@ __global__ void __launch_bounds__(PT_THREADS, 1) pair_select_tc_kernel(
             __syncwarp();
             const double* dprev = s_delta[(p - 1) & 1];
             const float* Sp = s_sc + K + K * K * (p - 1);
+            // lanes 0..15 take predecessors 0..7, lanes 16..31 predecessors
+            // 8..15; the halves meet by one exchange (ties: the smaller rank)
             double best = 0.0;
             int arg = -1;
+            const int k0 = (lane >> 4) * (K / 2);
 #pragma unroll
-            for (int kk = 0; kk < K; ++kk) {
+            for (int i = 0; i < K / 2; ++i) {
+                const int kk = k0 + i;
                 const double c_s = dprev[kk] + (double)Sp[kk * K + k];
                 if (arg < 0 || c_s > best) {
                     best = c_s;
                     arg = kk;
+                }
+            }
+            {
+                const double ob = __shfl_xor_sync(FULL, best, 16);
+                const int oa = __shfl_xor_sync(FULL, arg, 16);
+                if (ob > best || (ob == best && oa < arg)) {
+                    best = ob;
+                    arg = oa;
                 }
             }
             delta = (double)s_lp[p * K + k] + best;
@@ -320,7 +380,7 @@ __global__ void __launch_bounds__(PT_THREADS, 1) pair_select_tc_kernel(
     if (warp == 2) {
         __syncwarp();
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
     }
 }
 
