@@ -18,7 +18,7 @@
 // waits) reduces the partials in chunk order and decides.  The sampling draw
 // needs the normalisers first; it runs in the same launch: a warp done with
 // its scan units takes draw units of the sequences that have finished (a
-// queue in finishing order), one chunk of the row the sequence draws from
+// queue in finishing order), half a chunk of the row the sequence draws from
 // each, and the warp completing a sequence's draw units walks the inverse
 // CDF to t = u' * R.  No probability vector is ever written to memory.
 #include "common.cuh"
@@ -609,8 +609,8 @@ __device__ __forceinline__ SampleInfo load_info(const SampleInfo* p) {
 // (a shared-memory counter hands them to its warps as they run out of scan
 // units), so every SM draws the same share.  A warp waits (bounded) until
 // the sequence at that position has finished, brings the unit of target row
-// n (and draft row n for the residual) into its ring slots, and stores its
-// lanes' prefix sums.  The warp whose unit completes a sequence picks the
+// n (and draft row n for the residual) into the two halves of one ring slot,
+// and stores its lanes' prefix sums.  The warp whose unit completes a sequence picks the
 // token.  No warp waits on a warp that is itself waiting: a sequence
 // finishes within the scan, and a warp draws only after its own scan units.
 //
