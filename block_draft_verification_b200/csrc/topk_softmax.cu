@@ -7,13 +7,13 @@
 // those 16 per position; "DFlash 2" (myaiexp.com), section "主な機能": the
 // path selector keeps the top-16 candidates of each position.
 //
-// Work unit: (row, chunk of 16 KB of logits).  One CTA per SM streams a
-// contiguous range of units through a ring of TMA bulk copies kept in flight
-// by a producer warp (rows whose start is 16-byte aligned; others are read
-// element by element); each consumer warp reduces whole chunks on its own:
-// the chunk maximum, the sum of exp2((x - M) c) against it and the chunk's
-// exact top-16, all in a fixed order, so a chunk's partial does not depend
-// on the batch or the grid.  A unit's partial is published with one
+// Work unit: (row, chunk of 8 KB of logits).  One CTA per SM streams a
+// contiguous range of units, each warp a contiguous part of it brought in by
+// its own TMA bulk copies (rows whose start is 16-byte aligned; others are
+// read element by element), and each warp reduces whole chunks on its own:
+// the chunk maximum M, the sum of exp2(x c - fl(M c)) and the chunk's exact
+// top-16, all in a fixed order, so a chunk's partial does not depend on the
+// batch or the grid.  A unit's partial is published with one
 // acquire-release add; the warp that completes a row (no warp waits) merges
 // the chunk lists and softmax partials in chunk order and writes
 // idx / prob / logp / logz.  Keys compare (value, -index) exactly, so the
