@@ -33,7 +33,9 @@
 //   warps 4-7 epilogue: tcgen05.ld of their 32 TMEM lanes; a partial goes to
 //            the workspace, an owned tile adds the partials, stages the
 //            values in shared memory, then (token, 8-channel) items with
-//            16-byte loads of x_t and x_{t-1} and one 16-byte store
+//            16-byte loads of x_t and x_{t-1} and one 16-byte store; warps
+//            0-3, idle once the run's MMAs are issued, take half of the run's
+//            last owned tile
 // Every wait is bounded (one second, stream.cuh); on a timeout the kernel
 // records a flag (dflash2_device_errors), stops issuing work, waits (bounded)
 // for its tensor-core work in flight, releases TMEM and returns.  No TMA load

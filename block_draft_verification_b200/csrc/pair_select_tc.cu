@@ -20,10 +20,11 @@
 // fp32 and is split into three bf16 planes, W = W1 + W2 + W3 (each plane the
 // bf16 rounding of what the previous ones leave; 24 bits in all, W's fp32
 // mantissa), accumulated in the same fp32 accumulator: F keeps fp32 accuracy.
-// The 16 x 16 blocks S_i = F_i E_i^T, a few hundred thousand FMAs per
-// sequence, are taken on the CUDA cores from F in TMEM (tcgen05.ld) and the
-// right rows in shared memory, and the max-sum recursion runs in one warp
-// from shared memory.  Nothing but the path leaves the SM.
+// The 16 x 16 blocks S_i = F_i E_i^T run on the tensor cores too: F is split
+// the same way into three bf16 planes (exact), and S_all = F E_right^T
+// (M = N = 128) accumulates them in a second TMEM region, whose diagonal
+// blocks are the S_i; the max-sum recursion runs in one warp from shared
+// memory.  Nothing but the path leaves the SM.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
