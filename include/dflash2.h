@@ -227,9 +227,9 @@ DFLASH2_API int dflash2_pair_select(const int32_t* idx, const float* logp, const
  *       (sequence, position) and a last-CTA recursion (any table);
  *       DFLASH2_SELECT_TENSOR: one CTA per sequence, F = E W on tcgen05 with
  *       W split into three bf16 planes (fp32 accuracy), the 16 x 16 blocks
- *       from F on the CUDA cores, the recursion in shared memory (bf16
- *       tables only: DFLASH2_EDTYPE otherwise); needs no workspace, though
- *       ws is checked as for the other implementations.
+ *       F E^T on tcgen05 as well (F split the same way), the recursion in
+ *       shared memory (bf16 tables only: DFLASH2_EDTYPE otherwise); needs no
+ *       workspace, though ws is checked as for the other implementations.
  * Other values: DFLASH2_EINVAL.
  */
 #define DFLASH2_SELECT_AUTO 0
