@@ -39,12 +39,14 @@ constexpr int KT = TRUNC_K;  // keys kept per row: top_k <= 32
 
 // Candidate buffer of one warp: keys pushed by the filter, merged into the
 // running list whenever more than TC_FLUSH wait (at most 32 lanes x 8
-// elements arrive between two checks).
+// elements arrive between two checks) and at the end of every chunk.  The
+// count of waiting keys lives in a register of the warp (the same value in
+// every lane).
 constexpr unsigned TC_FLUSH = 64;
 constexpr unsigned TC_CAP = TC_FLUSH + 32 * 8;
 struct CandBuf32 {
     uint64_t key[TC_CAP];
-    unsigned n;
+    uint64_t out[KT];  // the merged list, placed by rank
 };
 
 // The 32 largest of a descending list (one key per lane, 0 = empty) and an
@@ -53,37 +55,45 @@ struct CandBuf32 {
 __device__ __forceinline__ uint64_t merge_desc_asc(uint64_t desc, uint64_t asc) {
     return warp_merge_desc(desc > asc ? desc : asc);
 }
-__device__ __forceinline__ uint64_t merge32(uint64_t run, uint64_t unsorted) {
-    const int lane = threadIdx.x & 31;
-    const uint64_t s = shfl64(warp_sort_desc(unsorted), 31 - lane);  // ascending
-    return merge_desc_asc(run, s);
-}
 
-// Merge the buffered candidates into the running list 32 at a time; raise the
-// bound to the list's 32nd key; once the list is full its 32nd value also
-// raises the row's shared bound (thr: ord32 of a value at least 32 of the
-// row's elements reach; pub: what this warp last put there).  Warp-uniform.
-__device__ __forceinline__ void flush32(CandBuf32& cb, uint64_t& run, uint64_t& tkey, float& tv,
-                                        unsigned* thr, uint32_t& pub) {
+// Merge the n buffered candidates into the running list (one key per lane,
+// descending; 0 = empty) up to 32 at a time, by rank: every key of the union
+// (keys are distinct) lands at its rank in it, so a batch costs one broadcast
+// read, a ballot and two compares per buffered key, and no sort.  Then the
+// bound rises to the list's 32nd key; once the list is full its 32nd value
+// also raises the row's shared bound (thr: ord32 of a value at least 32 of
+// the row's elements reach; pub: what this warp last put there).
+// Warp-uniform; n is zero on return.
+__device__ __forceinline__ void flush32(CandBuf32& cb, unsigned& n, uint64_t& run,
+                                        uint64_t& tkey, float& tv, unsigned* thr,
+                                        uint32_t& pub) {
     const int lane = threadIdx.x & 31;
-    __syncwarp();
-    const unsigned n = *(volatile unsigned*)&cb.n;
-    if (n <= 4) {  // a few keys: each inserted at its rank (one ballot, one shift)
-        for (unsigned i = 0; i < n; ++i) {
-            const uint64_t c = cb.key[i];
-            const int pos = __popc(__ballot_sync(FULL, run > c));
-            const uint64_t up = shfl64_up1(run);
-            if (pos < KT && lane >= pos) run = (lane == pos) ? c : up;
+    __syncwarp();  // every lane's pushed keys are visible
+    for (unsigned base = 0; base < n; base += 32) {
+        const unsigned m = min(32u, n - base);
+        const uint64_t c = (unsigned)lane < m ? cb.key[base + lane] : 0ull;
+        unsigned rank_list = 0u;  // list keys above this lane's candidate
+        unsigned rank_new = 0u;   // batch keys above this lane's candidate
+        unsigned above_run = 0u;  // batch keys above this lane's list key
+#pragma unroll 4
+        for (unsigned j = 0; j < m; ++j) {
+            const uint64_t cj = cb.key[base + j];
+            const unsigned above = __ballot_sync(FULL, run > cj);
+            if ((unsigned)lane == j) rank_list = __popc(above);
+            rank_new += cj > c;
+            above_run += cj > run;
         }
-    } else {
-        for (unsigned base = 0; base < n; base += KT) {
-            const unsigned j = base + (unsigned)lane;
-            run = merge32(run, j < n ? cb.key[j] : 0ull);
-        }
+        cb.out[lane] = 0ull;
+        __syncwarp();
+        const unsigned pc = rank_list + rank_new;
+        if ((unsigned)lane < m && pc < (unsigned)KT) cb.out[pc] = c;
+        const unsigned pr = (unsigned)lane + above_run;
+        if (run != 0ull && pr < (unsigned)KT) cb.out[pr] = run;
+        __syncwarp();
+        run = cb.out[lane];
+        __syncwarp();  // out is read before the next batch writes it
     }
-    __syncwarp();
-    if (lane == 0) cb.n = 0;
-    __syncwarp();
+    n = 0u;
     const uint64_t k32 = shfl64(run, KT - 1);
     if (k32 > tkey) {
         tkey = k32;
@@ -100,16 +110,17 @@ __device__ __forceinline__ void flush32(CandBuf32& cb, uint64_t& run, uint64_t& 
 // with the chunk's elements.  Pass 1 keeps every vector's packed maximum.
 // The bound: the list's 32nd key once it is full; before, the smallest lane
 // maximum when every lane holds an element (each lane maximum is an element,
-// so at least 32 elements reach it); the row's shared bound when higher.  No
+// so at least 32 elements reach it); the row's shared bound when higher
+// (`shared`: its value as read one chunk earlier, a valid, looser bound).  No
 // element below the bound can be in the row's top 32, so only vectors whose
-// maximum reaches it are looked at element by element, and the merged row
-// list is the exact top 32 whatever the timing.
+// maximum reaches it are looked at (one per lane per round: its elements are
+// compared with the bound's value and keys built only for those that reach
+// it), and the merged row list is the exact top 32 whatever the timing.
 template <bool BF16, class View>
 __device__ __forceinline__ void top32_chunk(const View& v, CandBuf32& cb, uint64_t& run,
-                                            unsigned* thr, uint32_t& pub) {
+                                            unsigned* thr, uint32_t& pub, uint32_t shared) {
     using C = ChunkT<BF16>;
     const int lane = threadIdx.x & 31, nv = v.nvec();
-    const uint32_t shared = *(volatile unsigned*)thr;  // used after pass 1 (its latency hidden)
     uint32_t vm[NVL];
     const float m = chunk_pass1<BF16>(v, vm);
     float tv = -INFINITY;
@@ -137,41 +148,46 @@ __device__ __forceinline__ void top32_chunk(const View& v, CandBuf32& cb, uint64
     for (int i = 0; i < NVL; ++i)
         if (32 * i + lane < nv && any_ge<BF16>(vm[i], t2)) hits |= 1u << i;
     if (!__any_sync(FULL, hits != 0u)) return;
+    unsigned nbuf = 0u;  // keys waiting in cb (warp-uniform)
     while (__any_sync(FULL, hits != 0u)) {  // one vector per lane per round
-        uint64_t kk[C::VW];
-        unsigned msk = 0;
+        unsigned em = 0u;  // elements of the lane's vector that reach the bound
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        int q = 0;
         if (hits) {
             const int i = __ffs(hits) - 1;
             hits &= hits - 1u;
-            const int q = 32 * i + lane;
-            const uint4 w = v.vec(q);
+            q = 32 * i + lane;
+            w = v.vec(q);
 #pragma unroll
-            for (int e = 0; e < C::VW; ++e) {
-                const float x = C::elem(w, e);
-                kk[e] = make_key(x, (uint32_t)v.index(q, e));
-                if (x >= tv && q * C::VW + e < v.n && kk[e] > tkey) msk |= 1u << e;
-            }
+            for (int e = 0; e < C::VW; ++e)
+                if (C::elem(w, e) >= tv) em |= 1u << e;
+            // elements past the chunk's end read as -inf: they reach only a -inf bound
+            const int lim = v.n - q * C::VW;
+            if (lim < C::VW) em &= lim > 0 ? (1u << lim) - 1u : 0u;
         }
-        const unsigned cnt = __popc(msk);
-        unsigned incl = cnt;
+        // Keys whose value equals the bound's but whose index part is below
+        // the list's 32nd key are pushed too: the merge ranks them out.
+        // This round's keys appended in lane order: the exclusive prefix of
+        // the per-lane counts (at most 8: four bits) from four ballots.
+        const unsigned cnt = __popc(em);
+        const unsigned below = (1u << lane) - 1u;
+        unsigned excl = 0u, total = 0u;
 #pragma unroll
-        for (int k = 1; k < 32; k <<= 1) {
-            const unsigned o = __shfl_up_sync(FULL, incl, k);
-            if (lane >= k) incl += o;
+        for (int bit = 0; bit < 4; ++bit) {
+            const unsigned bb = __ballot_sync(FULL, (cnt >> bit) & 1u);
+            excl += (unsigned)__popc(bb & below) << bit;
+            total += (unsigned)__popc(bb) << bit;
         }
-        const unsigned base = *(volatile unsigned*)&cb.n;
-        unsigned pos = base + incl - cnt;
-#pragma unroll
-        for (int e = 0; e < C::VW; ++e)
-            if (msk & (1u << e)) cb.key[pos++] = kk[e];
-        const unsigned nn = base + __shfl_sync(FULL, incl, 31);
-        __syncwarp();
-        if (lane == 0) cb.n = nn;
-        __syncwarp();
-        if (nn > TC_FLUSH) flush32(cb, run, tkey, tv, thr, pub);
+        unsigned pos = nbuf + excl;
+        while (em) {
+            const int e = __ffs(em) - 1;
+            em &= em - 1u;
+            cb.key[pos++] = make_key(C::elem_at(w, e), (uint32_t)v.index(q, e));
+        }
+        nbuf += total;
+        if (nbuf > TC_FLUSH) flush32(cb, nbuf, run, tkey, tv, thr, pub);
     }
-    __syncwarp();
-    if (*(volatile unsigned*)&cb.n > 0u) flush32(cb, run, tkey, tv, thr, pub);
+    if (nbuf > 0u) flush32(cb, nbuf, run, tkey, tv, thr, pub);
 }
 
 static_assert(sizeof(List32) == KT * sizeof(uint64_t), "one segment list per unit");
@@ -361,7 +377,6 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_trunc_kernel(
     unsigned* const thr = ctl + nrows;
     unsigned* const seqcnt = ctl + 2 * nrows;
     CandBuf32& cb = cbuf[warp];
-    if (lane == 0) cb.n = 0;
     auto rowp = [&](int64_t b, int rr) {
         return (rr <= G) ? (const char*)target + (b * (G + 1) + rr) * V * ES
                          : (const char*)draft + (b * G + (rr - G - 1)) * V * ES;
@@ -383,21 +398,29 @@ __global__ void __launch_bounds__(RING_THREADS, 1) verify_trunc_kernel(
     uint64_t run = 0ull;
     unsigned seg = 0;
     uint32_t pub = 0u;
+    // the row's shared bound, read one unit ahead: it only rises while the
+    // row is open (and its last unit is still to come), so an older value is
+    // a valid, slightly looser bound
+    uint32_t thr_now = n > 0 ? *(volatile unsigned*)&thr[uc.g * rows_per_seq + uc.r] : 0u;
     for (int k = 0; k < n; ++k, uc.next()) {
         const int64_t b = uc.g, v0 = (int64_t)uc.c * LEN;
         const int64_t grow = b * rows_per_seq + uc.r;
         const int len = (int)min((int64_t)LEN, V - v0);
+        const uint32_t thr_ahead =
+            k + 1 < n ? *(volatile unsigned*)&thr[uc.last_of_row() ? grow + 1 : grow] : 0u;
         if (TMA) {
             if (!r.wait(k)) {
                 warp_ring_abort(r, k, n);
                 return;
             }
-            top32_chunk<BF16>(SmemView<BF16>{r.slot(k), v0, len}, cb, run, &thr[grow], pub);
+            top32_chunk<BF16>(SmemView<BF16>{r.slot(k), v0, len}, cb, run, &thr[grow], pub,
+                              thr_now);
             warp_ring_next(r, k, n, ic, Ch::NEG_INF_WORD, src);
         } else {
             top32_chunk<BF16>(GlobalView<BF16>{(const uint8_t*)rowp(b, uc.r), v0, len}, cb, run,
-                              &thr[grow], pub);
+                              &thr[grow], pub, thr_now);
         }
+        thr_now = thr_ahead;
         ++seg;
         const bool seg_end = (k + 1 == n) || uc.last_of_row();
         if (!seg_end) {  // no list at this chunk (the entry may hold an earlier call's)
