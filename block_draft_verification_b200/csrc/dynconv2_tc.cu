@@ -38,8 +38,8 @@
 //            last owned tile
 // Every wait is bounded (one second, stream.cuh); on a timeout the kernel
 // records a flag (dflash2_device_errors), stops issuing work, waits (bounded)
-// for its tensor-core work in flight, releases TMEM and returns.  No TMA load
-// here uses cluster multicast.
+// for its tensor-core work in flight, releases TMEM and returns.  Every TMA
+// load here fills only the issuing CTA's own shared memory.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
